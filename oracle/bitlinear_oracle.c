@@ -1,0 +1,349 @@
+/*
+ * bitlinear_oracle.c -- plain, slow, single-threaded CPU oracle for the
+ * BitNet b1.58 BitLinear forward pass.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or
+ * load this file: only the test suite, the smoke check of the graft entry
+ * point and the CPU-baseline leg of bench.py use it.  It shares no code,
+ * header, table or constant with the CUDA library; it is built by gcc without
+ * fast-math (IEEE single/double, round-to-nearest-even, no FMA contraction).
+ *
+ * Sources (web pages; cited by title and section):
+ *   [P1] "QAT与BitNet：1-bit及1.58-bit量化训练解析" (kongchang.com)
+ *   [P3] "BitNet b1.58深度解析：三值权重如何重塑大模型推理" (0539edu.com)
+ *   [P5] "QAT and BitNet: A Deep Dive into 1-bit and 1.58-bit
+ *         Quantization-Aware Training" (kongchang.com/en)
+ *
+ * What the pages leave open is fixed here by the plainest reading; every such
+ * reading is listed next to the function that takes it.
+ *
+ * Parity pins: every function below is pinned by a CPU test against the
+ * pages' worked examples, closed forms, exact arithmetic or brute force; none
+ * is "parity unpinned".
+ */
+#include <float.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#if !defined(FLT_EVAL_METHOD) || FLT_EVAL_METHOD != 0
+#error "the oracle needs single-precision float evaluation (FLT_EVAL_METHOD == 0)"
+#endif
+
+#define ORC_F32 0
+#define ORC_BF16 1
+#define ORC_I8 2
+#define ORC_I32 3
+
+#define ORC_PACK_I2 0 /* 2 bits per weight, 4 weights per byte */
+#define ORC_PACK_T5 1 /* 5 trits per byte, base 3 */
+
+/* ------------------------------------------------------------------------ */
+/* dtype helpers                                                            */
+/* ------------------------------------------------------------------------ */
+
+float orc_bf16_to_f32(uint16_t h) {
+  uint32_t u = (uint32_t)h << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+/* fp32 -> bf16, round to nearest, ties to even (NaN -> quiet NaN). */
+uint16_t orc_f32_to_bf16(float f) {
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x0040u);
+  uint32_t lsb = (u >> 16) & 1u;
+  u += 0x7fffu + lsb;
+  return (uint16_t)(u >> 16);
+}
+
+static float load_f(const void *p, int dt, int64_t i) {
+  if (dt == ORC_F32) return ((const float *)p)[i];
+  return orc_bf16_to_f32(((const uint16_t *)p)[i]);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Step 1: absmean scale gamma = mean(|W|) over the whole weight matrix.     */
+/* [P1]/[P5] "The Ternary Weight Recipe" (gamma = w.abs().mean());           */
+/* [P3] §3.1 (gamma = mean(|W|), one per weight matrix).                     */
+/*                                                                          */
+/* Reading (pages silent on summation order): the sum of |w| is taken in     */
+/* fp64 in this fixed order, so that every implementation reaches the same  */
+/* bits:                                                                    */
+/*   - elements in row-major order e = n*K + k, T = N*K;                    */
+/*   - chunk c holds e in [c*8192, (c+1)*8192);                             */
+/*   - in chunk c, lane l (0..255) adds, in this order, the elements        */
+/*     c*8192 + 2048*i + 8*l + j for i = 0..3, j = 0..7 (those below T),    */
+/*     starting from 0.0;                                                   */
+/*   - lane sums combine by the stride-halving tree p[l] += p[l+s],          */
+/*     s = 128, 64, ..., 1; p[0] is the chunk sum;                          */
+/*   - chunk sums, padded with 0.0 up to the next power of two P, combine   */
+/*     by the same tree with s = P/2, ..., 1.                               */
+/* gamma64 = S / T, and gamma is gamma64 rounded to fp32.                    */
+/* ------------------------------------------------------------------------ */
+
+#define ORC_CHUNK 8192
+#define ORC_LANES 256
+
+static double chunk_sum(const void *W, int dt, int64_t T, int64_t c) {
+  double p[ORC_LANES];
+  for (int l = 0; l < ORC_LANES; ++l) {
+    double acc = 0.0;
+    for (int i = 0; i < 4; ++i)
+      for (int j = 0; j < 8; ++j) {
+        int64_t e = c * ORC_CHUNK + 2048 * (int64_t)i + 8 * (int64_t)l + j;
+        if (e < T) acc += (double)fabsf(load_f(W, dt, e));
+      }
+    p[l] = acc;
+  }
+  for (int s = ORC_LANES / 2; s >= 1; s /= 2)
+    for (int l = 0; l < s; ++l) p[l] += p[l + s];
+  return p[0];
+}
+
+double orc_absmean_sum(const void *W, int dt, int64_t N, int64_t K) {
+  int64_t T = N * K;
+  if (T <= 0) return 0.0;
+  int64_t C = (T + ORC_CHUNK - 1) / ORC_CHUNK;
+  int64_t P = 1;
+  while (P < C) P *= 2;
+  double *q = (double *)calloc((size_t)P, sizeof(double));
+  if (!q) return NAN;
+  for (int64_t c = 0; c < C; ++c) q[c] = chunk_sum(W, dt, T, c);
+  for (int64_t s = P / 2; s >= 1; s /= 2)
+    for (int64_t c = 0; c < s; ++c) q[c] += q[c + s];
+  double S = q[0];
+  free(q);
+  return S;
+}
+
+float orc_gamma(const void *W, int dt, int64_t N, int64_t K) {
+  double S = orc_absmean_sum(W, dt, N, K);
+  double g = S / (double)(N * K);
+  return (float)g;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Step 2: ternarize, W_q = clamp(round(W / (gamma + eps)), -1, 1).          */
+/* [P1]/[P5] "The Ternary Weight Recipe" (ternary_weights, eps = 1e-5);      */
+/* [P3] §3.1 (W_norm = W / gamma, round, clamp to [-1, 1]).                  */
+/* Readings: d = gamma + eps is one fp32 add; the division is one IEEE fp32  */
+/* division; round is half-to-even (torch.round), so a ratio of exactly 0.5 */
+/* goes to 0, which agrees with the page's "|w| <= gamma/2 -> 0".            */
+/* ------------------------------------------------------------------------ */
+
+void orc_ternarize(const void *W, int dt, int64_t N, int64_t K, float gamma,
+                   float eps, int8_t *codes) {
+  float d = gamma + eps;
+  for (int64_t e = 0; e < N * K; ++e) {
+    float r = load_f(W, dt, e) / d;
+    float q = nearbyintf(r);
+    if (q > 1.0f) q = 1.0f;
+    if (q < -1.0f) q = -1.0f;
+    codes[e] = (int8_t)q;
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Step 3: packing.                                                         */
+/* [P1]/[P5] "Why Is It Called 1.58 Bits?" (2 bits per weight; five trits   */
+/* per byte, 3^5 = 243 <= 256); [P3] §2.3 and §6.3 (codes "00, 01, 10",     */
+/* four weights per byte; five per byte by table lookup or bit operations). */
+/* Readings: code = q + 1 (-1 -> 00, 0 -> 01, +1 -> 10), first weight in    */
+/* the least significant bits; base 3 byte = sum (q_i + 1) * 3^i with the   */
+/* first weight least significant; each row is padded to a multiple of 16  */
+/* bytes with digits that encode weight 0 (a whole pad byte is 0x55 in the  */
+/* 2-bit format, 121 in base 3).                                            */
+/* ------------------------------------------------------------------------ */
+
+static int per_byte(int fmt) { return fmt == ORC_PACK_I2 ? 4 : 5; }
+
+int64_t orc_packed_row_bytes(int64_t K, int fmt) {
+  int64_t per = per_byte(fmt);
+  int64_t used = (K + per - 1) / per;
+  return (used + 15) / 16 * 16;
+}
+
+/* returns 0, or -1 if a code is outside {-1, 0, 1} */
+int orc_pack(const int8_t *codes, int64_t N, int64_t K, int fmt,
+             uint8_t *packed) {
+  int per = per_byte(fmt);
+  int64_t rb = orc_packed_row_bytes(K, fmt);
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t j = 0; j < rb; ++j) {
+      unsigned byte = 0, pow3 = 1;
+      for (int i = 0; i < per; ++i) {
+        int64_t k = j * per + i;
+        int q = 0;
+        if (k < K) {
+          q = codes[n * K + k];
+          if (q < -1 || q > 1) return -1;
+        }
+        unsigned digit = (unsigned)(q + 1);
+        if (fmt == ORC_PACK_I2)
+          byte |= digit << (2 * i);
+        else
+          byte += digit * pow3;
+        pow3 *= 3;
+      }
+      packed[n * rb + j] = (uint8_t)byte;
+    }
+  return 0;
+}
+
+/* Inverse of orc_pack.  Returns 0, -1 for an invalid code (2-bit code 11 or
+ * a base-3 byte >= 243), -2 for a padding digit that is not weight 0. */
+int orc_unpack(const uint8_t *packed, int64_t N, int64_t K, int fmt,
+               int8_t *codes) {
+  int per = per_byte(fmt);
+  int64_t rb = orc_packed_row_bytes(K, fmt);
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t j = 0; j < rb; ++j) {
+      unsigned byte = packed[n * rb + j];
+      if (fmt == ORC_PACK_T5 && byte >= 243) return -1;
+      for (int i = 0; i < per; ++i) {
+        unsigned digit;
+        if (fmt == ORC_PACK_I2) {
+          digit = (byte >> (2 * i)) & 3u;
+          if (digit == 3) return -1;
+        } else {
+          digit = byte % 3;
+          byte /= 3;
+        }
+        int64_t k = j * per + i;
+        if (k < K)
+          codes[n * K + k] = (int8_t)((int)digit - 1);
+        else if (digit != 1)
+          return -2;
+      }
+    }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Step 4: per-token absmax INT8 activation quantization.                   */
+/* [P3] §3.2 (scale = max|x| per token; x_q = clamp(round(x/scale*127),      */
+/* -127, 127)) and §5.2 (activation_quantize_int8 floors the scale at 1e-6). */
+/* Readings: a token is one row of x over K; s = max(max|x|, 1e-6); the     */
+/* quotient x/s is one fp32 division, then one fp32 multiply by 127, then  */
+/* round half-to-even; the range is symmetric, -128 never occurs.           */
+/* ------------------------------------------------------------------------ */
+
+void orc_act_quant(const void *x, int dt, int64_t M, int64_t K, int8_t *xq,
+                   float *scale) {
+  for (int64_t m = 0; m < M; ++m) {
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+      float a = fabsf(load_f(x, dt, m * K + k));
+      if (a > amax) amax = a;
+    }
+    float s = amax > 1e-6f ? amax : 1e-6f;
+    scale[m] = s;
+    for (int64_t k = 0; k < K; ++k) {
+      float t = load_f(x, dt, m * K + k) / s;
+      t = t * 127.0f;
+      float q = nearbyintf(t);
+      if (q > 127.0f) q = 127.0f;
+      if (q < -127.0f) q = -127.0f;
+      xq[m * K + k] = (int8_t)q;
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Step 5: ternary x INT8 matrix product with INT32 accumulation,            */
+/* acc[m][n] = sum_k W_q[n][k] * x_q[m][k]  (y = x W^T as in F.linear).      */
+/* [P3] §4.2 (y_i = sum_j w_ij x_j: add for +1, subtract for -1, skip 0);   */
+/* [P3] §3.3 (INT32 accumulator).                                           */
+/* ------------------------------------------------------------------------ */
+
+void orc_matmul_i32(const int8_t *codes, const int8_t *xq, int64_t M,
+                    int64_t N, int64_t K, int32_t *acc) {
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t n = 0; n < N; ++n) {
+      int32_t s = 0;
+      for (int64_t k = 0; k < K; ++k)
+        s += (int32_t)codes[n * K + k] * (int32_t)xq[m * K + k];
+      acc[m * N + n] = s;
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Step 6: dequantize, y = acc * gamma * s_m / 127.                          */
+/* [P1]/[P5] "The BitLinear Recipe" step 4 (rescale by both factors);        */
+/* [P3] §3.2 (x is x_q * scale / 127) and §5.3 (output multiplied by gamma). */
+/* Readings: the weight factor is gamma itself (not gamma + eps); the order */
+/* is c_m = (gamma * s_m) / 127 in fp32, then y = (float)acc * c_m; a bf16  */
+/* output is that fp32 value rounded to nearest even.                       */
+/* ------------------------------------------------------------------------ */
+
+void orc_dequant(const int32_t *acc, float gamma, const float *scale,
+                 int64_t M, int64_t N, void *y, int ydt) {
+  for (int64_t m = 0; m < M; ++m) {
+    float c = (gamma * scale[m]) / 127.0f;
+    for (int64_t n = 0; n < N; ++n) {
+      int64_t i = m * N + n;
+      float v = (float)acc[i] * c;
+      if (ydt == ORC_F32)
+        ((float *)y)[i] = v;
+      else if (ydt == ORC_BF16)
+        ((uint16_t *)y)[i] = orc_f32_to_bf16(v);
+      else
+        ((int32_t *)y)[i] = acc[i];
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Whole forward: unpack, quantize activations (or take x_q and its scales  */
+/* as given when xdt is ORC_I8), multiply, dequantize.  The same arguments  */
+/* as the library's forward entry point.  Returns 0, or the unpack status. */
+/* ------------------------------------------------------------------------ */
+
+int orc_forward(const uint8_t *packed, int fmt, float gamma, int64_t N,
+                int64_t K, const void *x, int xdt, float *scale, int64_t M,
+                void *y, int ydt) {
+  int8_t *codes = (int8_t *)malloc((size_t)(N * K));
+  int8_t *xq = (int8_t *)malloc((size_t)(M * K));
+  int32_t *acc = (int32_t *)malloc((size_t)(M * N) * sizeof(int32_t));
+  int rc = -3;
+  if (!codes || !xq || !acc) goto out;
+  rc = orc_unpack(packed, N, K, fmt, codes);
+  if (rc != 0) goto out;
+  if (xdt == ORC_I8)
+    memcpy(xq, x, (size_t)(M * K));
+  else
+    orc_act_quant(x, xdt, M, K, xq, scale);
+  orc_matmul_i32(codes, xq, M, N, K, acc);
+  orc_dequant(acc, gamma, scale, M, N, y, ydt);
+out:
+  free(codes);
+  free(xq);
+  free(acc);
+  return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* 1-bit BitNet weights, used to reproduce the pages' five-weight example.   */
+/* [P1]/[P5] "The BitLinear Recipe" step 2 (alpha = mean of the weights,    */
+/* above alpha -> +1, below -> -1) and step 4 (beta = mean |W|); "A         */
+/* Five-Weight Example".                                                    */
+/* Reading: a weight equal to alpha maps to -1 (the pages do not say);      */
+/* beta is the uncentred mean |w| (the example's 0.57 requires it).         */
+/* ------------------------------------------------------------------------ */
+
+void orc_onebit(const float *w, int64_t n, int8_t *b, float *alpha,
+                float *beta) {
+  double s = 0.0, sa = 0.0;
+  for (int64_t i = 0; i < n; ++i) {
+    s += (double)w[i];
+    sa += (double)fabsf(w[i]);
+  }
+  float a = (float)(s / (double)n);
+  *alpha = a;
+  *beta = (float)(sa / (double)n);
+  for (int64_t i = 0; i < n; ++i) b[i] = (int8_t)(w[i] > a ? 1 : -1);
+}
