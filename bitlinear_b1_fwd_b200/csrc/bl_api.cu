@@ -1,0 +1,164 @@
+// bl_api.cu -- the C ABI declared in include/bitlinear.h: argument checks on the
+// host, workspace carving, and kernel selection.  Nothing here computes.
+#include <cmath>
+#include <cstring>
+
+#include "bitlinear.h"
+#include "bl_common.cuh"
+#include "bl_kernels.h"
+
+namespace {
+
+constexpr int64_t kMaxK = int64_t{1} << 20;
+constexpr int64_t kMaxNK = int64_t{1} << 32;
+constexpr int kVersion = 100;  // 0.1.0
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+inline size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+inline bool float_dt(int dt) { return dt == BL_F32 || dt == BL_BF16; }
+inline bool fmt_ok(int fmt) { return fmt == BL_PACK_I2 || fmt == BL_PACK_T5; }
+
+inline bl_status cuda_status(cudaError_t e) { return e == cudaSuccess ? BL_OK : BL_ERR_CUDA; }
+
+bool nk_ok(int64_t N, int64_t K) {
+  if (N < 0 || K < 1 || K > kMaxK) return false;
+  return N <= kMaxNK / K;
+}
+
+}  // namespace
+
+extern "C" {
+
+int bitlinear_version(void) { return kVersion; }
+
+const char* bitlinear_status_string(int status) {
+  switch (status) {
+    case BL_OK: return "BL_OK: success";
+    case BL_ERR_INVALID_VALUE: return "BL_ERR_INVALID_VALUE: a size, dtype, format or pointer is invalid";
+    case BL_ERR_UNSUPPORTED: return "BL_ERR_UNSUPPORTED: valid arguments, but not supported on this device";
+    case BL_ERR_MISALIGNED: return "BL_ERR_MISALIGNED: an array pointer is not 16-byte aligned";
+    case BL_ERR_WORKSPACE_TOO_SMALL: return "BL_ERR_WORKSPACE_TOO_SMALL: workspace below the queried size";
+    case BL_ERR_CUDA: return "BL_ERR_CUDA: a CUDA runtime call failed";
+    case BL_ERR_DEVICE_TIMEOUT: return "BL_ERR_DEVICE_TIMEOUT: a bounded wait in a kernel ran out";
+    case BL_ERR_BAD_CODE: return "BL_ERR_BAD_CODE: a weight code outside {-1, 0, 1} was packed";
+    default: return "unknown bitlinear status";
+  }
+}
+
+int64_t bitlinear_packed_row_bytes(int64_t K, int fmt) {
+  if (K < 1 || K > kMaxK || !fmt_ok(fmt)) return -1;
+  const int64_t per = fmt == BL_PACK_I2 ? 4 : 5;
+  return ((K + per - 1) / per + 15) / 16 * 16;
+}
+
+size_t bitlinear_quantize_weights_workspace_bytes(int64_t N, int64_t K) {
+  if (N < 1 || !nk_ok(N, K)) return 0;
+  const int64_t chunks = (N * K + bl::kChunk - 1) / bl::kChunk;
+  return BL_WS_HEADER_BYTES + round256(static_cast<size_t>(chunks) * sizeof(double));
+}
+
+size_t bitlinear_forward_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int xdt) {
+  if (M < 0 || !nk_ok(N, K) || !fmt_ok(fmt)) return 0;
+  (void)xdt;
+  return BL_WS_HEADER_BYTES;
+}
+
+bl_status bitlinear_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (ws == nullptr || ws_bytes < BL_WS_HEADER_BYTES) return BL_ERR_INVALID_VALUE;
+  return cuda_status(cudaMemsetAsync(ws, 0, BL_WS_HEADER_BYTES, static_cast<cudaStream_t>(stream)));
+}
+
+bl_status bitlinear_quantize_weights(const void* W, int wdt, int64_t N, int64_t K, float eps, int fmt,
+                                     uint8_t* packed, int8_t* codes, float* gamma, void* ws,
+                                     size_t ws_bytes, void* stream) {
+  if (W == nullptr || gamma == nullptr || ws == nullptr || (packed == nullptr && codes == nullptr))
+    return BL_ERR_INVALID_VALUE;
+  if (!float_dt(wdt) || !fmt_ok(fmt) || N < 1 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
+  if (!(eps > 0.0f) || !std::isfinite(eps)) return BL_ERR_INVALID_VALUE;
+  if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(codes, 16) || !aligned(gamma, 4) ||
+      !aligned(ws, 16))
+    return BL_ERR_MISALIGNED;
+  if (ws_bytes < bitlinear_quantize_weights_workspace_bytes(N, K)) return BL_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = bl::launch_absmean(W, wdt, N, K, ws, gamma, st);
+  if (e != cudaSuccess) return BL_ERR_CUDA;
+  const int64_t rb = bitlinear_packed_row_bytes(K, fmt);
+  return cuda_status(bl::launch_ternarize_pack(W, wdt, N, K, gamma, eps, fmt, packed, codes, rb, st));
+}
+
+bl_status bitlinear_absmean(const void* W, int wdt, int64_t N, int64_t K, float* gamma, void* ws,
+                            size_t ws_bytes, void* stream) {
+  if (W == nullptr || gamma == nullptr || ws == nullptr) return BL_ERR_INVALID_VALUE;
+  if (!float_dt(wdt) || N < 1 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
+  if (!aligned(W, 16) || !aligned(gamma, 4) || !aligned(ws, 16)) return BL_ERR_MISALIGNED;
+  if (ws_bytes < bitlinear_quantize_weights_workspace_bytes(N, K)) return BL_ERR_WORKSPACE_TOO_SMALL;
+  return cuda_status(bl::launch_absmean(W, wdt, N, K, ws, gamma, static_cast<cudaStream_t>(stream)));
+}
+
+bl_status bitlinear_ternarize_pack(const void* W, int wdt, int64_t N, int64_t K, const float* gamma,
+                                   float eps, int fmt, uint8_t* packed, int8_t* codes, void* stream) {
+  if (W == nullptr || gamma == nullptr || (packed == nullptr && codes == nullptr)) return BL_ERR_INVALID_VALUE;
+  if (!float_dt(wdt) || !fmt_ok(fmt) || N < 1 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
+  if (!(eps > 0.0f) || !std::isfinite(eps)) return BL_ERR_INVALID_VALUE;
+  if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(codes, 16) || !aligned(gamma, 4))
+    return BL_ERR_MISALIGNED;
+  const int64_t rb = bitlinear_packed_row_bytes(K, fmt);
+  return cuda_status(bl::launch_ternarize_pack(W, wdt, N, K, gamma, eps, fmt, packed, codes, rb,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+bl_status bitlinear_pack(const int8_t* codes, int64_t N, int64_t K, int fmt, uint8_t* packed, void* ws,
+                         size_t ws_bytes, void* stream) {
+  if (!fmt_ok(fmt) || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
+  if (N == 0) return BL_OK;
+  if (codes == nullptr || packed == nullptr || ws == nullptr) return BL_ERR_INVALID_VALUE;
+  if (!aligned(codes, 16) || !aligned(packed, 16) || !aligned(ws, 16)) return BL_ERR_MISALIGNED;
+  if (ws_bytes < BL_WS_HEADER_BYTES) return BL_ERR_WORKSPACE_TOO_SMALL;
+  const int64_t rb = bitlinear_packed_row_bytes(K, fmt);
+  return cuda_status(bl::launch_pack(codes, N, K, fmt, packed, rb, ws, static_cast<cudaStream_t>(stream)));
+}
+
+bl_status bitlinear_quantize_acts(const void* x, int xdt, int64_t M, int64_t K, int8_t* xq, float* scale,
+                                  void* stream) {
+  if (!float_dt(xdt) || M < 0 || K < 1 || K > kMaxK) return BL_ERR_INVALID_VALUE;
+  if (M == 0) return BL_OK;
+  if (x == nullptr || xq == nullptr || scale == nullptr) return BL_ERR_INVALID_VALUE;
+  if (!aligned(x, 16) || !aligned(xq, 16) || !aligned(scale, 4)) return BL_ERR_MISALIGNED;
+  return cuda_status(bl::launch_act_quant(x, xdt, M, K, xq, scale, static_cast<cudaStream_t>(stream)));
+}
+
+bl_status bitlinear_forward(const uint8_t* packed, int fmt, const float* gamma, int64_t N, int64_t K,
+                            const void* x, int xdt, float* scale, int64_t M, void* y, int ydt, void* ws,
+                            size_t ws_bytes, void* stream) {
+  if (!fmt_ok(fmt) || !(float_dt(xdt) || xdt == BL_I8) || !(float_dt(ydt) || ydt == BL_I32))
+    return BL_ERR_INVALID_VALUE;
+  if (M < 0 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
+  if (M == 0 || N == 0) return BL_OK;  // empty output: nothing to read or write
+  if (packed == nullptr || gamma == nullptr || x == nullptr || scale == nullptr || y == nullptr ||
+      ws == nullptr)
+    return BL_ERR_INVALID_VALUE;
+  if (!aligned(packed, 16) || !aligned(x, 16) || !aligned(y, 16) || !aligned(scale, 4) ||
+      !aligned(gamma, 4) || !aligned(ws, 16))
+    return BL_ERR_MISALIGNED;
+  if (ws_bytes < bitlinear_forward_workspace_bytes(M, N, K, fmt, xdt)) return BL_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (bl::gemv_max_tokens(fmt, bitlinear_packed_row_bytes(K, fmt)) < 1) return BL_ERR_UNSUPPORTED;
+  return cuda_status(bl::launch_gemv(packed, fmt, gamma, N, K, x, xdt, scale, M, y, ydt, st));
+}
+
+bl_status bitlinear_device_status(void* ws, void* stream) {
+  if (ws == nullptr) return BL_ERR_INVALID_VALUE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t h[2] = {0, 0};
+  if (cudaMemcpyAsync(h, ws, sizeof h, cudaMemcpyDeviceToHost, st) != cudaSuccess) return BL_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return BL_ERR_CUDA;
+  if (h[0] != 0) {
+    if (cudaMemsetAsync(ws, 0, sizeof h, st) != cudaSuccess) return BL_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return BL_ERR_CUDA;
+  }
+  if (h[0] & bl::kFlagTimeout) return BL_ERR_DEVICE_TIMEOUT;
+  if (h[0] & bl::kFlagBadCode) return BL_ERR_BAD_CODE;
+  return BL_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,95 @@
+// bl_common.cuh -- helpers shared by the BitLinear kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "bitlinear.h"
+
+namespace bl {
+
+// Fixed reduction order of gamma: 8192-element chunks, 256 lanes, groups of 8.
+constexpr int kChunk = 8192;
+constexpr int kLanes = 256;
+
+// Device flags in the first word of a workspace header.
+constexpr uint32_t kFlagTimeout = 1u;
+constexpr uint32_t kFlagBadCode = 2u;
+
+struct WsHeader {
+  uint32_t flags;   // kFlag* bits, sticky until bitlinear_device_status
+  uint32_t site;    // where a bounded wait gave up (kernel-defined code)
+  uint32_t ticket;  // absmean: CTAs done so far (back to 0 when a call ends)
+  uint32_t reserved[61];
+};
+static_assert(sizeof(WsHeader) == BL_WS_HEADER_BYTES, "header size");
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) {
+  return __uint_as_float(static_cast<uint32_t>(h) << 16);
+}
+
+// Load element i of a float-valued array (fp32 or bf16 bit patterns).
+template <int DT>
+__device__ __forceinline__ float load_elem(const void* p, int64_t i) {
+  if constexpr (DT == BL_F32) {
+    return __ldg(static_cast<const float*>(p) + i);
+  } else {
+    return bf16_bits_to_f32(__ldg(static_cast<const uint16_t*>(p) + i));
+  }
+}
+
+// Load 8 consecutive elements starting at element e (e a multiple of 8 and
+// the array 16-byte aligned), widened to fp32.
+template <int DT>
+__device__ __forceinline__ void load8_aligned(const void* p, int64_t e, float v[8]) {
+  if constexpr (DT == BL_F32) {
+    const float4* q = reinterpret_cast<const float4*>(static_cast<const float*>(p) + e);
+    float4 a = __ldg(q), b = __ldg(q + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    uint4 a = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p) + e));
+    uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+}
+
+// Per-token INT8 code of x against scale s: rint(fl(fl(x / s) * 127)) clamped
+// to [-127, 127]; IEEE quotient, round half to even.
+__device__ __forceinline__ int quant_act(float x, float s) {
+  float t = __fmul_rn(__fdiv_rn(x, s), 127.0f);
+  t = fminf(fmaxf(rintf(t), -127.0f), 127.0f);
+  return __float2int_rn(t);
+}
+
+// Dequantization factor c = (gamma * s) / 127 and the dequantized value.
+__device__ __forceinline__ float dequant_factor(float gamma, float s) {
+  return __fdiv_rn(__fmul_rn(gamma, s), 127.0f);
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_max(T v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_maxf(float v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ void set_flag(void* ws, uint32_t bit, uint32_t site) {
+  if (ws == nullptr) return;
+  WsHeader* h = static_cast<WsHeader*>(ws);
+  atomicOr(&h->flags, bit);
+  atomicExch(&h->site, site);
+}
+
+}  // namespace bl

@@ -1,0 +1,36 @@
+// bl_kernels.h -- launchers of the BitLinear kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace bl {
+
+// absmean: the last CTA folds 2^lgR chunk sums per lane (lgR <= 11 allows
+// 2^19 chunks of 8192 elements, so N*K <= 2^32).
+constexpr int kFinishMaxLevels = 11;
+
+// Number of SMs of the current device (cached per device).
+constexpr int kMaxDevices = 64;
+int device_sms();
+
+// decode GEMV: shared memory for activations, tokens per launch.
+constexpr int64_t kGemvSmemBudget = 200 * 1024;
+constexpr int kGemvMaxTokens = 4;
+
+// ws: a workspace whose header ticket is zero; partial sums follow the header.
+cudaError_t launch_absmean(const void* W, int wdt, int64_t N, int64_t K, void* ws, float* gamma,
+                           cudaStream_t st);
+cudaError_t launch_ternarize_pack(const void* W, int wdt, int64_t N, int64_t K, const float* gamma,
+                                  float eps, int fmt, uint8_t* packed, int8_t* codes, int64_t rowbytes,
+                                  cudaStream_t st);
+cudaError_t launch_pack(const int8_t* codes, int64_t N, int64_t K, int fmt, uint8_t* packed,
+                        int64_t rowbytes, void* ws, cudaStream_t st);
+cudaError_t launch_act_quant(const void* x, int xdt, int64_t M, int64_t K, int8_t* xq, float* scale,
+                             cudaStream_t st);
+int gemv_max_tokens(int fmt, int64_t rowbytes);
+cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int64_t N, int64_t K,
+                        const void* x, int xdt, float* scale, int64_t M, void* y, int ydt,
+                        cudaStream_t st);
+
+}  // namespace bl

@@ -1,0 +1,126 @@
+"""The C ABI on the CPU: the library builds and loads, exports every function
+that include/bitlinear.h declares, and rejects bad arguments on the host
+before any CUDA call (no compute runs here)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "bitlinear.h")
+
+
+@pytest.fixture(scope="module")
+def bl():
+    from bitlinear_b1_fwd_b200 import build, binding
+    build.build()
+    return binding
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    names = re.findall(r"^(?:BL_API\s+)?(?:const\s+)?\w+\s*\*?\s*(bitlinear_\w+)\s*\(", text, flags=re.M)
+    unmarked = re.findall(r"^(?!BL_API)(?:const\s+)?\w+\s*\*?\s*(bitlinear_\w+)\s*\(", text, flags=re.M)
+    assert not unmarked, f"declared without BL_API (not exported): {unmarked}"
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("bitlinear_quantize_weights", "bitlinear_pack", "bitlinear_quantize_acts",
+                     "bitlinear_forward"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(bl):
+    L = bl.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    assert set(declared_functions()) <= set(bl.SIGNATURES)
+    assert bl.bitlinear_version() >= 100
+
+
+def test_row_bytes_match_oracle(bl, orc):
+    for K in (1, 4, 5, 63, 64, 65, 256, 3200, 8192, 8640, 28672, 1 << 20):
+        for fmt in (0, 1):
+            assert bl.bitlinear_packed_row_bytes(K, fmt) == orc.packed_row_bytes(K, fmt)
+    assert bl.bitlinear_packed_row_bytes(0, 0) == -1
+    assert bl.bitlinear_packed_row_bytes(5, 7) == -1
+    assert bl.bitlinear_packed_row_bytes((1 << 20) + 1, 0) == -1
+
+
+def test_workspace_sizes(bl):
+    assert bl.bitlinear_quantize_weights_workspace_bytes(512, 256) == 256 + 256   # 16 chunks
+    assert bl.bitlinear_quantize_weights_workspace_bytes(8640, 3200) == 256 + 3375 * 8 + (256 - 3375 * 8 % 256)
+    assert bl.bitlinear_quantize_weights_workspace_bytes(0, 5) == 0
+    assert bl.bitlinear_forward_workspace_bytes(1, 8640, 3200, 0, 1) >= bl.BL_WS_HEADER_BYTES
+    assert bl.bitlinear_forward_workspace_bytes(1, 8640, 0, 0, 1) == 0
+
+
+def test_status_strings(bl):
+    for s in range(8):
+        assert bl.status_string(s).startswith("BL_")
+    assert "unknown" in bl.status_string(99)
+
+
+def test_host_validation_without_gpu(bl):
+    """Each call returns its error code before launching anything."""
+    L = bl.lib()
+    p = C.c_void_p(1 << 20)            # an aligned, never-dereferenced address
+    odd = C.c_void_p((1 << 20) + 4)    # 4-byte aligned only
+    null = None
+    # quantize_weights
+    assert L.bitlinear_quantize_weights(null, 0, 4, 4, 1e-5, 0, p, null, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_quantize_weights(p, 2, 4, 4, 1e-5, 0, p, null, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_quantize_weights(p, 0, 4, 4, 0.0, 0, p, null, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_quantize_weights(p, 0, 4, 4, float("nan"), 0, p, null, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_quantize_weights(p, 0, 4, 4, 1e-5, 3, p, null, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_quantize_weights(p, 0, 4, 0, 1e-5, 0, p, null, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_quantize_weights(p, 0, 0, 4, 1e-5, 0, p, null, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_quantize_weights(p, 0, 4, (1 << 20) + 1, 1e-5, 0, p, null, p, p, 1 << 30, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_quantize_weights(p, 0, 1 << 13, 1 << 20, 1e-5, 0, p, null, p, p, 1 << 30, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_quantize_weights(p, 0, 4, 4, 1e-5, 0, null, null, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_quantize_weights(odd, 0, 4, 4, 1e-5, 0, p, null, p, p, 4096, null) == bl.BL_ERR_MISALIGNED
+    assert L.bitlinear_quantize_weights(p, 0, 4, 4, 1e-5, 0, p, null, p, p, 100, null) == bl.BL_ERR_WORKSPACE_TOO_SMALL
+    # ternarize_pack
+    assert L.bitlinear_ternarize_pack(p, 0, 4, 4, null, 1e-5, 0, p, null, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_ternarize_pack(p, 0, 4, 4, p, -1.0, 0, p, null, null) == bl.BL_ERR_INVALID_VALUE
+    # pack
+    assert L.bitlinear_pack(p, 4, 4, 0, p, p, 10, null) == bl.BL_ERR_WORKSPACE_TOO_SMALL
+    assert L.bitlinear_pack(null, 0, 4, 0, null, null, 0, null) == bl.BL_OK
+    assert L.bitlinear_pack(odd, 4, 4, 0, p, p, 4096, null) == bl.BL_ERR_MISALIGNED
+    assert L.bitlinear_pack(p, 4, 4, 2, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_pack(p, 0, 4, 0, p, p, 4096, null) == bl.BL_OK          # empty: nothing to do
+    # quantize_acts
+    assert L.bitlinear_quantize_acts(p, 2, 4, 4, p, p, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_quantize_acts(p, 1, 4, 0, p, p, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_quantize_acts(odd, 1, 4, 4, p, p, null) == bl.BL_ERR_MISALIGNED
+    assert L.bitlinear_quantize_acts(p, 1, 0, 4, p, p, null) == bl.BL_OK
+    # forward
+    args = lambda **kw: [kw.get(k, v) for k, v in dict(
+        packed=p, fmt=0, gamma=p, N=4, K=4, x=p, xdt=1, scale=p, M=1, y=p, ydt=1, ws=p,
+        ws_bytes=4096, stream=null).items()]
+    assert L.bitlinear_forward(*args(packed=null)) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_forward(*args(fmt=5)) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_forward(*args(xdt=3)) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_forward(*args(ydt=2)) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_forward(*args(M=-1)) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_forward(*args(K=0)) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_forward(*args(y=odd)) == bl.BL_ERR_MISALIGNED
+    assert L.bitlinear_forward(*args(ws_bytes=8)) == bl.BL_ERR_WORKSPACE_TOO_SMALL
+    assert L.bitlinear_forward(*args(M=0)) == bl.BL_OK
+    assert L.bitlinear_forward(*args(N=0)) == bl.BL_OK
+    assert L.bitlinear_forward(*args(M=0, x=null, y=null, scale=null, ws=null)) == bl.BL_OK
+    # workspace helpers
+    assert L.bitlinear_workspace_init(null, 4096, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_device_status(null, null) == bl.BL_ERR_INVALID_VALUE
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    from bitlinear_b1_fwd_b200 import binding
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        binding.lib()

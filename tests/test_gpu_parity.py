@@ -1,0 +1,284 @@
+"""GPU parity: the CUDA path through the C ABI against the oracle, element by
+element, on the seeded workloads and edge shapes.
+
+Integers (gamma's bits, codes, packed bytes, x_q, scales, INT32 accumulators)
+must be bit-exact; fp32 outputs within 1e-6 relative; bf16 outputs within 1 ulp.
+"""
+import numpy as np
+import pytest
+import torch
+
+from bitlinear_b1_fwd_b200 import binding as B
+from bitlinear_b1_fwd_b200 import synth
+from gpu_helpers import assert_bf16_ulp, assert_f32_rel, dev, forward, host, quantize_weights
+
+pytestmark = pytest.mark.gpu
+
+I2, T5 = B.BL_PACK_I2, B.BL_PACK_T5
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from bitlinear_b1_fwd_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+    torch.cuda.init()
+
+
+def check_weights(orc, W, fmt):
+    g, codes, packed = quantize_weights(W, fmt)
+    g_ref = orc.gamma(W)
+    assert g.view(np.uint32) == g_ref.view(np.uint32), (g, g_ref)
+    codes_ref = orc.ternarize(W, g_ref, 1e-5, parallel=True)
+    assert np.array_equal(codes, codes_ref)
+    assert np.array_equal(packed, orc.pack(codes_ref, fmt))
+    return g, packed
+
+
+def check_forward(orc, packed, fmt, g, N, K, x, scale=None, ydts=(B.BL_I32, B.BL_F32, B.BL_BF16)):
+    for ydt in ydts:
+        y, s = forward(packed, fmt, g, N, K, x, ydt, scale)
+        y_ref, s_ref = orc.forward(packed, fmt, g, N, K, x, ydt=ydt, scale=scale)
+        assert np.array_equal(s, s_ref)
+        if ydt == B.BL_I32:
+            assert np.array_equal(y, y_ref)
+        elif ydt == B.BL_F32:
+            assert_f32_rel(y, y_ref)
+        else:
+            assert_bf16_ulp(y, y_ref)
+
+
+# --- step 4: activation quantization ----------------------------------------------
+
+def _act_cases():
+    yield "tiny_f32_outliers", synth.tiny_inputs()[1]
+    yield "3b_decode_bf16", synth.decode_3b_inputs(0)[1]
+    yield "ragged_3x5_f32", synth.normal_f32(41, (3, 5))
+    yield "ragged_17x129_bf16", synth.to_bf16_bits(synth.normal_f32(42, (17, 129)))
+    yield "ragged_2x1000_f32", synth.normal_f32(43, (2, 1000))
+    yield "ragged_5x7_bf16", synth.to_bf16_bits(synth.normal_f32(44, (5, 7)))
+    z = synth.normal_f32(45, (4, 64))
+    z[1] = 0.0
+    z[2] = 1e-9
+    yield "zero_and_tiny_rows", z
+
+
+@pytest.mark.parametrize("name,x", list(_act_cases()), ids=lambda v: v if isinstance(v, str) else "")
+def test_quantize_acts(orc, name, x):
+    M, K = x.shape
+    xd = dev(x)
+    xq = torch.full((M, K), 99, dtype=torch.int8, device="cuda")
+    s = torch.empty(M, dtype=torch.float32, device="cuda")
+    B.bitlinear_quantize_acts(xd, xq, s)
+    torch.cuda.synchronize()
+    xq_ref, s_ref = orc.act_quant(x)
+    assert np.array_equal(host(xq), xq_ref)
+    assert np.array_equal(host(s), s_ref)
+
+
+def test_quantize_acts_prefill_full(orc):
+    """3B prefill activations: 4096 tokens x 3200 with 16 outlier channels."""
+    _, x = synth.prefill_3b_inputs()
+    xd = dev(x)
+    xq = torch.empty((4096, 3200), dtype=torch.int8, device="cuda")
+    s = torch.empty(4096, dtype=torch.float32, device="cuda")
+    B.bitlinear_quantize_acts(xd, xq, s)
+    torch.cuda.synchronize()
+    xq_ref, s_ref = orc.act_quant(x)
+    assert np.array_equal(host(xq), xq_ref)
+    assert np.array_equal(host(s), s_ref)
+
+
+def test_quantize_acts_round_half_even(orc):
+    """Entries that land exactly on k + 0.5 after the multiply by 127."""
+    xs = [np.float32(1.0)]
+    for t in (0.5, 1.5, 2.5, 3.5, 126.5):
+        v = np.float32(t / 127.0)
+        for _ in range(400):
+            r = np.float32(v * np.float32(127.0))
+            if r == np.float32(t):
+                break
+            v = np.nextafter(v, np.float32(1) if r < t else np.float32(0))
+        xs += [v, -v]
+    x = np.array([xs + [0.0] * (16 - len(xs))], np.float32)
+    xd = dev(x)
+    xq = torch.empty_like(xd, dtype=torch.int8)
+    s = torch.empty(1, dtype=torch.float32, device="cuda")
+    B.bitlinear_quantize_acts(xd, xq, s)
+    torch.cuda.synchronize()
+    assert host(xq)[0, :11].tolist() == [127, 0, 0, 2, -2, 2, -2, 4, -4, 126, -126]
+    assert np.array_equal(host(xq), orc.act_quant(x)[0])
+
+
+# --- steps 1-3: weights -------------------------------------------------------------
+
+def test_worked_examples(orc):
+    for W, codes in ((synth.EXAMPLE_A, [0, -1, 1, -1, 0]), (synth.EXAMPLE_B, [1, -1, 0, -1, 1])):
+        for fmt in (I2, T5):
+            g, c, p = quantize_weights(W, fmt)
+            assert c[0].tolist() == codes
+            assert g == orc.gamma(W)
+            assert np.array_equal(p, orc.pack(c, fmt))
+
+
+def _weight_cases():
+    yield "tiny", synth.tiny_inputs()[0]
+    yield "ragged_3x7", synth.normal_f32(51, (3, 7), 0.02)
+    yield "ragged_5x129", synth.normal_f32(52, (5, 129), 0.02)
+    yield "ragged_2x8193", synth.normal_f32(53, (2, 8193), 0.02)
+    yield "one", np.array([[0.3]], np.float32)
+    yield "ragged_7x81", synth.normal_f32(54, (7, 81), 1.0)
+    yield "bf16_300x1000", synth.to_bf16_bits(synth.normal_f32(55, (300, 1000), 0.02))
+    yield "bf16_ragged_9x77", synth.to_bf16_bits(synth.normal_f32(56, (9, 77), 0.02))
+    yield "zeros", np.zeros((4, 100), np.float32)
+    yield "many_chunks_40x100003", synth.normal_f32(57, (40, 100003), 0.01)
+
+
+@pytest.mark.parametrize("fmt", [I2, T5])
+@pytest.mark.parametrize("name,W", list(_weight_cases()), ids=lambda v: v if isinstance(v, str) else "")
+def test_quantize_weights(orc, name, W, fmt):
+    check_weights(orc, W, fmt)
+
+
+@pytest.mark.parametrize("layer", [0, 1])
+def test_quantize_weights_3b(orc, layer):
+    W, _ = synth.decode_3b_inputs(layer)
+    check_weights(orc, W, I2)
+    if layer == 0:
+        check_weights(orc, W, T5)
+
+
+def test_ternarize_threshold_boundary(orc):
+    """A fixed gamma and weights planted at and next to d/2 = (gamma + eps)/2,
+    including fp32 values whose quotient by d rounds to exactly 0.5."""
+    gamma = np.float32(0.0163)
+    d = np.float32(gamma + np.float32(1e-5))
+    half = np.float32(d / np.float32(2))
+    plant = [half, -half, np.float32(0), np.float32(-0.0), d, -d, np.float32(1.5) * d]
+    v = half
+    for _ in range(64):  # the fp32 values just above d/2
+        v = np.nextafter(v, np.float32(1))
+        plant += [v, -v]
+    v = half
+    for _ in range(16):
+        v = np.nextafter(v, np.float32(0))
+        plant += [v, -v]
+    W = synth.normal_f32(61, (3, 1000), 0.02)
+    W[0, :len(plant)] = plant
+    ratio_half = sum(1 for p in plant if np.float32(abs(p) / d) == np.float32(0.5))
+    assert ratio_half > 2   # some planted quotients round to exactly 0.5
+    for fmt in (I2, T5):
+        Wd = dev(W)
+        g = torch.tensor([float(gamma)], dtype=torch.float32, device="cuda")
+        packed = torch.empty((3, B.bitlinear_packed_row_bytes(1000, fmt)), dtype=torch.uint8, device="cuda")
+        codes = torch.empty((3, 1000), dtype=torch.int8, device="cuda")
+        B.bitlinear_ternarize_pack(Wd, g, 1e-5, fmt, packed, codes)
+        torch.cuda.synchronize()
+        ref = orc.ternarize(W, gamma, 1e-5)
+        assert np.array_equal(host(codes), ref)
+        assert np.array_equal(host(packed), orc.pack(ref, fmt))
+
+
+def test_pack_and_bad_codes(orc):
+    rng = np.random.default_rng(3)
+    for (N, K) in [(5, 3), (7, 129), (64, 3200), (3, 8193)]:
+        codes = rng.integers(-1, 2, (N, K), dtype=np.int8)
+        for fmt in (I2, T5):
+            packed = torch.empty((N, B.bitlinear_packed_row_bytes(K, fmt)), dtype=torch.uint8, device="cuda")
+            ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+            B.bitlinear_pack(dev(codes), fmt, packed, ws)
+            assert B.bitlinear_device_status(ws) == B.BL_OK
+            assert np.array_equal(host(packed), orc.pack(codes, fmt))
+    bad = rng.integers(-1, 2, (4, 40), dtype=np.int8)
+    bad[2, 17] = 3
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    packed = torch.empty((4, 16), dtype=torch.uint8, device="cuda")
+    B.bitlinear_pack(dev(bad), I2, packed, ws)
+    assert B.bitlinear_device_status(ws) == B.BL_ERR_BAD_CODE
+    assert B.bitlinear_device_status(ws) == B.BL_OK      # read clears the flag
+    fixed = bad.copy()
+    fixed[2, 17] = 0
+    assert np.array_equal(host(packed), orc.pack(fixed, I2))
+
+
+# --- steps 4-6: forward ------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt", [I2, T5])
+def test_forward_tiny(orc, fmt):
+    W, x = synth.tiny_inputs()
+    g, packed = check_weights(orc, W, fmt)
+    check_forward(orc, packed, fmt, g, 512, 256, x)
+
+
+def test_forward_worked_example(orc):
+    g, _, packed = quantize_weights(synth.EXAMPLE_A, I2)
+    y, s = forward(packed, I2, g, 1, 5, np.ones((1, 5), np.float32), B.BL_I32)
+    assert y.tolist() == [[-127]] and s.tolist() == [1.0]
+    y, _ = forward(packed, I2, g, 1, 5, np.ones((1, 5), np.float32), B.BL_F32)
+    assert abs(float(y[0, 0]) + 0.61) < 1e-6
+
+
+@pytest.mark.parametrize("layer", [0, 1])
+@pytest.mark.parametrize("fmt", [I2, T5])
+def test_forward_3b_decode(orc, layer, fmt):
+    W, x = synth.decode_3b_inputs(layer)
+    c = synth.DECODE_3B[layer]
+    g, _, packed = quantize_weights(W, fmt, codes=False)
+    check_forward(orc, packed, fmt, g, c["N"], c["K"], x)
+
+
+@pytest.mark.parametrize("fmt", [I2, T5])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 16, 17])
+def test_forward_token_counts(orc, fmt, M):
+    W = synth.normal_f32(71, (300, 1000), 0.02)
+    x = synth.to_bf16_bits(synth.normal_f32(72, (M, 1000)))
+    g, _, packed = quantize_weights(W, fmt, codes=False)
+    check_forward(orc, packed, fmt, g, 300, 1000, x)
+
+
+@pytest.mark.parametrize("fmt", [I2, T5])
+@pytest.mark.parametrize("N,K,M", [(1, 1, 1), (3, 5, 2), (33, 7, 3), (65, 129, 1), (17, 8193, 2),
+                                   (129, 4097, 4), (2, 20001, 1)])
+def test_forward_ragged(orc, fmt, N, K, M):
+    W = synth.normal_f32(N * 7 + K, (N, K), 0.02)
+    x = synth.normal_f32(K * 3 + M, (M, K))
+    g, _, packed = quantize_weights(W, fmt, codes=False)
+    check_forward(orc, packed, fmt, g, N, K, x)
+
+
+def test_forward_prequantized_and_degenerate(orc):
+    W, x = synth.tiny_inputs()
+    g, _, packed = quantize_weights(W, I2, codes=False)
+    xq, s = orc.act_quant(x)
+    check_forward(orc, packed, I2, g, 512, 256, xq, scale=s)
+    # zero tokens, and an all-zero weight matrix (gamma 0)
+    xz = x.copy()
+    xz[3] = 0.0
+    check_forward(orc, packed, I2, g, 512, 256, xz)
+    gz, _, pz = quantize_weights(np.zeros((64, 256), np.float32), T5, codes=False)
+    assert gz == 0.0
+    y, _ = forward(pz, T5, gz, 64, 256, x, B.BL_F32)
+    assert not y.any()
+    # M = 0 launches nothing and returns success
+    y, _ = forward(packed, I2, g, 512, 256, np.zeros((0, 256), np.float32), B.BL_F32)
+    assert y.shape == (0, 512)
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_forward_3b_block(orc, M):
+    """The six BitLinears of a 3B block (Q, K, V, O, up, down), each with its
+    own per-token quantization, at M = 1 and 16 tokens."""
+    for layer in range(6):
+        W, x = synth.block_3b_inputs(layer, M)
+        c = synth.BLOCK_3B[layer]
+        g, _, packed = quantize_weights(W, I2, codes=False)
+        check_forward(orc, packed, I2, g, c["N"], c["K"], x, ydts=(B.BL_I32, B.BL_BF16))
+
+
+def test_misaligned_pointer_rejected():
+    x = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
+    xq = torch.zeros(64, dtype=torch.int8, device="cuda")
+    s = torch.zeros(2, dtype=torch.float32, device="cuda")
+    with pytest.raises(B.BitLinearError) as e:
+        B.bitlinear_quantize_acts(x[1:33].view(1, 32), xq[:32].view(1, 32), s[:1])
+    assert e.value.status == B.BL_ERR_MISALIGNED
