@@ -1,0 +1,479 @@
+#!/usr/bin/env python3
+"""BitLinear forward throughput on B200: one JSON line on rank 0.
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+for every layer of the workload, the absmean scale (step 1), ternarize + pack
+(steps 2-3) and the forward (per-token INT8 quantization, ternary x INT8
+product, dequantization: steps 4-6), each through the C ABI of
+libbitlinear.so.  ``--phase forward`` times steps 4-6 alone on weights packed
+beforehand (an inference server's per-token work).
+
+Timing: W untimed warm-up steps; then exactly K steps captured into one CUDA
+graph with timing events between the library calls, replayed once between
+barrier + synchronize on both sides; the device time is the max over ranks.
+The weights are larger than L2 (phase all) or rotated over enough packed copies
+to exceed 4x L2 (phase forward).  Multi-GPU: one process per GPU (torchrun),
+every rank runs its own independent replica of the workload (weak scaling).
+
+``--impl reference`` times the CPU oracle instead (rank 0 only), each step a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "BitLinear GB/s (decode GEMV) & INT8 TOPS (prefill) vs roofline, 1×B200"
+FALLBACK_HBM_GBS = 6650.0
+
+# workload name -> layers (N, K), tokens M, packed format, activation dtype
+WORKLOADS = {
+    "3b_decode": dict(desc="3B-shaped decode GEMV: M=1, up K=3200->N=8640 and down K=8640->N=3200, "
+                           "fp32 latent W N(0,0.02), bf16 x N(0,1), 2-bit pack, bf16 y",
+                      layers=[(8640, 3200), (3200, 8640)], M=1, fmt=0, sigma=0.02, seed=2),
+    "3b_decode_t5": dict(desc="3B-shaped decode GEMV, base-3 (5 trits/byte) pack",
+                         layers=[(8640, 3200), (3200, 8640)], M=1, fmt=1, sigma=0.02, seed=2),
+    "70b_decode": dict(desc="70B-shaped layer decode: M=1, K=8192->N=28672 and K=28672->N=8192, "
+                            "fp32 latent W N(0,0.01), bf16 x, 2-bit pack",
+                       layers=[(28672, 8192), (8192, 28672)], M=1, fmt=0, sigma=0.01, seed=5),
+    "70b_decode_t5": dict(desc="70B-shaped layer decode, base-3 pack",
+                          layers=[(28672, 8192), (8192, 28672)], M=1, fmt=1, sigma=0.01, seed=5),
+}
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+
+def csrc_digest() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "bitlinear_b1_fwd_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    digest = csrc_digest()
+    for p in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        kv = {}
+        with open(p) as f:
+            for line in f:
+                if ":" in line and line.startswith("- "):
+                    k, v = line[2:].split(":", 1)
+                    kv[k.strip()] = v.strip().strip("`")
+        if kv.get("kernel") == kernel and kv.get("workload") == workload and kv.get("csrc_sha256") == digest:
+            try:
+                return int(kv["dram_bytes_per_launch"])
+            except (KeyError, ValueError):
+                return None
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self._stop, self._t = period_s, threading.Event(), None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------
+# algorithmic bytes per launch (the unit of work of each kernel)
+# ----------------------------------------------------------------------------
+
+def layer_bytes(N, K, M, rb, w_es=4, x_es=2, y_es=2):
+    absmean = N * K * w_es + 4
+    ternarize = N * K * w_es + N * rb + 4
+    forward = N * rb + M * K * x_es + M * N * y_es + 4 * M + 4
+    return dict(absmean=absmean, ternarize_pack=ternarize, forward=forward)
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (the baseline and the reference arm)
+# ----------------------------------------------------------------------------
+
+def oracle_layer_inputs(wl, rows_frac=1.0):
+    from bitlinear_b1_fwd_b200 import synth
+    out = []
+    for i, (N, K) in enumerate(wl["layers"]):
+        n = max(1, int(N * rows_frac))
+        W = synth.normal_f32(1000 + wl["seed"] + 100 * i, (N, K), wl["sigma"])[:n]
+        x = synth.to_bf16_bits(synth.normal_f32(2000 + wl["seed"] + 100 * i, (wl["M"], K)))
+        out.append((W, x))
+    return out
+
+
+def oracle_step(orc, wl, inputs, phase):
+    """One oracle pass over the inputs; returns algorithmic bytes processed."""
+    total = 0
+    for (W, x) in inputs:
+        n, K = W.shape
+        rb = orc.packed_row_bytes(K, wl["fmt"])
+        b = layer_bytes(n, K, wl["M"], rb)
+        g = orc.gamma(W)
+        packed = orc.pack(orc.ternarize(W, g), wl["fmt"])
+        orc.forward(packed, wl["fmt"], g, n, K, x, ydt=orc.BF16)
+        total += b["forward"] + (b["absmean"] + b["ternarize_pack"] if phase == "all" else 0)
+    return total
+
+
+def time_oracle(wl, phase, budget_s, min_steps=1, rows_frac=1.0):
+    import oracle
+    oracle.build()
+    inputs = oracle_layer_inputs(wl, rows_frac)
+    steps, nbytes, t0 = 0, 0, time.perf_counter()
+    while steps < min_steps or time.perf_counter() - t0 < budget_s:
+        nbytes += oracle_step(oracle, wl, inputs, phase)
+        steps += 1
+    dt = time.perf_counter() - t0
+    return nbytes / dt / 1e9, steps, dt
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+
+def run_gpu(args, wl, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    from bitlinear_b1_fwd_b200 import binding as B
+    from bitlinear_b1_fwd_b200 import build as libbuild
+    from bitlinear_b1_fwd_b200 import synth
+
+    if rank == 0:
+        libbuild.build()
+    if world > 1:
+        torch.distributed.barrier()
+    B.lib()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    fmt, M = wl["fmt"], wl["M"]
+    rank_seed = 10000 * rank
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+
+    layers = []
+    for i, (N, K) in enumerate(wl["layers"]):
+        Wh = synth.normal_f32(1000 + wl["seed"] + 100 * i + rank_seed, (N, K), wl["sigma"])
+        xh = synth.to_bf16_bits(synth.normal_f32(2000 + wl["seed"] + 100 * i + rank_seed, (M, K)))
+        rb = B.bitlinear_packed_row_bytes(K, fmt)
+        L = dict(N=N, K=K, rb=rb)
+        L["W"] = torch.from_numpy(Wh).to(dev)
+        L["x"] = torch.from_numpy(xh.view(np.int16)).to(dev).view(torch.bfloat16)
+        L["W_host"] = torch.from_numpy(Wh).pin_memory()
+        L["x_host"] = torch.from_numpy(xh.view(np.int16)).view(torch.bfloat16).pin_memory()
+        L["gamma"] = torch.empty(1, dtype=torch.float32, device=dev)
+        L["ws"] = torch.zeros(B.bitlinear_quantize_weights_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+        L["packed"] = torch.empty((N, rb), dtype=torch.uint8, device=dev)
+        L["scale"] = torch.empty(M, dtype=torch.float32, device=dev)
+        L["y"] = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        L["y_host"] = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        L["fws"] = torch.zeros(B.bitlinear_forward_workspace_bytes(M, N, K, fmt, B.BL_BF16),
+                               dtype=torch.uint8, device=dev)
+        L["bytes"] = layer_bytes(N, K, M, rb)
+        layers.append(L)
+        del Wh
+
+    stream = torch.cuda.Stream(device=dev)
+    eps = 1e-5
+
+    # phase forward: pack once, then rotate over copies of the packed weights
+    rot = 1
+    if args.phase == "forward":
+        with torch.cuda.stream(stream):
+            for L in layers:
+                B.bitlinear_quantize_weights(L["W"], eps, fmt, L["packed"], None, L["gamma"], L["ws"], stream)
+        stream.synchronize()
+        packed_bytes = sum(L["N"] * L["rb"] for L in layers)
+        rot = max(1, -(-4 * l2 // packed_bytes))
+        for L in layers:
+            L["copies"] = [L["packed"]] + [L["packed"].clone() for _ in range(rot - 1)]
+            del L["W"]
+
+    ops = ["absmean", "ternarize_pack", "forward"] if args.phase == "all" else ["forward"]
+
+    def step(i, evs=None):
+        for li, L in enumerate(layers):
+            def mark(op_i):
+                if evs is not None:
+                    evs[(li, op_i)].record(stream)
+            if args.phase == "all":
+                mark(0)
+                B.bitlinear_absmean(L["W"], L["gamma"], L["ws"], stream)
+                mark(1)
+                B.bitlinear_ternarize_pack(L["W"], L["gamma"], eps, fmt, L["packed"], None, stream)
+                mark(2)
+                packed = L["packed"]
+            else:
+                mark(0)
+                packed = L["copies"][i % rot]
+            B.bitlinear_forward(packed, fmt, L["gamma"], L["N"], L["K"], L["x"], L["scale"], L["y"],
+                                L["fws"], stream)
+            mark(len(ops))
+
+    def new_events():
+        d = {}
+        for li in range(len(layers)):
+            for oi in range(len(ops) + 1):
+                d[(li, oi)] = torch.cuda.Event(enable_timing=True, external=True)
+        return d
+
+    # warm-up (eager), then capture the K timed steps into one graph
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    stream.synchronize()
+
+    step_events = [new_events() for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True, external=True)
+    t_end = torch.cuda.Event(enable_timing=True, external=True)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream, capture_error_mode="relaxed"):
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(i, step_events[i])
+        t_end.record(stream)
+    graph.replay()              # one untimed replay (first-launch costs of the graph)
+    stream.synchronize()
+
+    sampler = ClockSampler(local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        graph.replay()
+        stream.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = t_start.elapsed_time(t_end)
+    for L in layers:
+        st = B.bitlinear_device_status(L["fws"], stream)
+        if st != B.BL_OK:
+            raise RuntimeError(f"device status {B.status_string(st)}")
+
+    # per-op device time (ms per launch) from the events inside the graph
+    per_op = {op: [] for op in ops}
+    for evs in step_events:
+        for li in range(len(layers)):
+            for oi, op in enumerate(ops):
+                per_op[op].append((li, evs[(li, oi)].elapsed_time(evs[(li, oi + 1)])))
+    step_bytes = sum(sum(L["bytes"][op] for op in ops) for L in layers)
+
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+
+    # ---- end to end through the public API from pinned host buffers ----
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    h2d = sum((L["W_host"].numel() * 4 if args.phase == "all" else 0) + L["x_host"].numel() * 2 for L in layers)
+    d2h = sum(L["y_host"].numel() * 2 for L in layers)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(e2e_steps):
+            for L in layers:
+                if args.phase == "all":
+                    L["W"].copy_(L["W_host"], non_blocking=True)
+                L["x"].copy_(L["x_host"], non_blocking=True)
+            step(i)
+            for L in layers:
+                L["y_host"].copy_(L["y"], non_blocking=True)
+        e1.record(stream)
+    stream.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
+    e2e_ms = float(e2e_t.item())
+
+    del graph
+    res = dict(ms_total=ms_max, per_op=per_op, step_bytes=step_bytes, layers=layers, ops=ops,
+               clocks=sampler.summary(), e2e_ms=e2e_ms, e2e_steps=e2e_steps, h2d=h2d, d2h=d2h,
+               rot=rot, l2=l2, launches_per_step=len(layers) * len(ops))
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="3b_decode")
+    ap.add_argument("--phase", choices=["all", "forward"], default="all")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-budget", type=float, default=10.0,
+                    help="seconds of oracle time for the cpu_baseline sample (0 = skip)")
+    args = ap.parse_args()
+    wl = WORKLOADS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    config = {"workload": args.workload, "desc": wl["desc"], "phase": args.phase, "M": wl["M"],
+              "layers_NK": wl["layers"], "pack": ["2-bit", "base-3"][wl["fmt"]],
+              "parallelism": f"replicas x{args.gpus}"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        # per-step sample of the oracle sized so the whole run stays within ~2 minutes
+        import oracle
+        oracle.build()
+        probe_frac = 0.02
+        v, s, dt = time_oracle(wl, args.phase, 0.0, min_steps=1, rows_frac=probe_frac)
+        per_step_full = dt / s / probe_frac
+        budget = 120.0 / max(1, args.steps + args.warmup)
+        frac = min(1.0, max(1e-4, budget / per_step_full))
+        inputs = oracle_layer_inputs(wl, frac)
+        for _ in range(args.warmup):
+            oracle_step(oracle, wl, inputs, args.phase)
+        t0 = time.perf_counter()
+        nbytes = sum(oracle_step(oracle, wl, inputs, args.phase) for _ in range(args.steps))
+        dt = time.perf_counter() - t0
+        val = nbytes / dt / 1e9
+        sample = f"first {frac:.4%} of each layer's weight rows per step, all steps of the path"
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64+i32",
+            "data": "synthetic", "config": config,
+            "cpu_baseline": {"value": val, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }))
+        return
+
+    import torch
+    if world > 1:
+        torch.distributed.init_process_group("nccl", device_id=torch.device("cuda", local_rank),
+                                             timeout=__import__("datetime").timedelta(seconds=120))
+    res = run_gpu(args, wl, rank, world, local_rank)
+
+    if rank == 0:
+        ms = res["ms_total"] / args.steps
+        value = res["step_bytes"] * world / (ms * 1e-3) / 1e9
+        peak, peak_kind = measured_peaks()
+        # per-op summary and the dominant kernel
+        stages = {}
+        for op in res["ops"]:
+            times = [t for (_, t) in res["per_op"][op]]
+            nb = sum(L["bytes"][op] for L in res["layers"])
+            tot = sum(times) / args.steps
+            stages[op] = {"ms_per_step": tot, "bytes_per_step": nb, "GB_s": nb / (tot * 1e-3) / 1e9,
+                          "frac_of_hbm": nb / (tot * 1e-3) / 1e9 / peak,
+                          "per_layer_us": [statistics.mean(t for (li, t) in res["per_op"][op] if li == j) * 1e3
+                                           for j in range(len(res["layers"]))]}
+        dom = max(stages, key=lambda o: stages[o]["ms_per_step"])
+        launches = len(res["layers"]) * args.steps
+        avg_launch_ms = stages[dom]["ms_per_step"] * args.steps / launches
+        bytes_per_launch = stages[dom]["bytes_per_step"] / len(res["layers"])
+        achieved = bytes_per_launch / (avg_launch_ms * 1e-3) / 1e9
+        kernel_name = {"absmean": "absmean_kernel", "ternarize_pack": "ternarize_pack_kernel",
+                       "forward": "gemv_kernel"}[dom]
+        traffic = profiled_traffic(kernel_name, args.workload)
+        cpu = None
+        if args.cpu_budget > 0 and world == 1:
+            v, s, dt = time_oracle(wl, args.phase, args.cpu_budget)
+            cpu = {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                   "sample": f"{s} full oracle steps of the same workload ({dt:.1f} s, 1 thread)"}
+        e2e_value = res["step_bytes"] * world / (res["e2e_ms"] * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "i8xternary->i32 (fp32 scales, fp64 gamma)",
+            "data": "synthetic (seeded N(0,sigma) latent weights, N(0,1) bf16 activations)",
+            "config": dict(config, l2=("inputs larger than L2 (fp32 latent weights "
+                                       f"{sum(L['N'] * L['K'] * 4 for L in res['layers']) / 1e6:.0f} MB per step)"
+                                       if args.phase == "all" else
+                                       f"packed weights rotated over {res['rot']} copies (>= 4x L2)"),
+                           kernels_per_step=res["launches_per_step"]),
+            "roofline": {"bound": "hbm", "kernel": kernel_name, "achieved": achieved, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": traffic, "bytes_per_launch": bytes_per_launch},
+            "stages": stages,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": res["h2d"],
+                    "d2h_bytes_per_step": res["d2h"], "steps": res["e2e_steps"]},
+            "gpu_launches": res["launches_per_step"] * args.steps,
+            "clocks": res["clocks"],
+        }
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -35,6 +35,7 @@ SIGNATURES = {
     "bitlinear_pack": (_I, [_P, _I64, _I64, _I, _P, _P, _SZ, _P]),
     "bitlinear_quantize_acts": (_I, [_P, _I, _I64, _I64, _P, _P, _P]),
     "bitlinear_forward": (_I, [_P, _I, _P, _I64, _I64, _P, _I, _P, _I64, _P, _I, _P, _SZ, _P]),
+    "bitlinear_selftest_wait_timeout": (_I, [_P, _SZ, _P]),
     "bitlinear_device_status": (_I, [_P, _P]),
     "bitlinear_status_string": (C.c_char_p, [_I]),
     "bitlinear_version": (_I, []),
@@ -173,6 +174,11 @@ def bitlinear_forward(packed, fmt, gamma, N, K, x, scale, y, ws, stream=None) ->
 def bitlinear_device_status(ws, stream=None) -> int:
     """Synchronize and return (and clear) the workspace's device status."""
     return int(lib().bitlinear_device_status(_ptr(ws), _stream(stream)))
+
+
+def bitlinear_selftest_wait_timeout(ws, stream=None) -> None:
+    _check(lib().bitlinear_selftest_wait_timeout(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "bitlinear_selftest_wait_timeout")
 
 
 def bitlinear_version() -> int:

@@ -57,10 +57,18 @@ size_t bitlinear_quantize_weights_workspace_bytes(int64_t N, int64_t K) {
   return BL_WS_HEADER_BYTES + round256(static_cast<size_t>(chunks) * sizeof(double));
 }
 
+// The tensor-core path serves more tokens than one GEMV launch holds, when the
+// x_q rows can be a TMA tensor (row stride a multiple of 16 bytes).
+bool uses_gemm(int64_t M, int64_t K) { return M > bl::kGemvMaxTokens && (K % 16) == 0; }
+
 size_t bitlinear_forward_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int xdt) {
   if (M < 0 || !nk_ok(N, K) || !fmt_ok(fmt)) return 0;
-  (void)xdt;
-  return BL_WS_HEADER_BYTES;
+  size_t bytes = BL_WS_HEADER_BYTES;
+  if (uses_gemm(M, K)) {
+    if (xdt != BL_I8) bytes += round256(static_cast<size_t>(M * K));
+    if (fmt == BL_PACK_T5) bytes += round256(static_cast<size_t>(N * bitlinear_packed_row_bytes(K, BL_PACK_I2)));
+  }
+  return bytes;
 }
 
 bl_status bitlinear_workspace_init(void* ws, size_t ws_bytes, void* stream) {
@@ -142,8 +150,36 @@ bl_status bitlinear_forward(const uint8_t* packed, int fmt, const float* gamma, 
     return BL_ERR_MISALIGNED;
   if (ws_bytes < bitlinear_forward_workspace_bytes(M, N, K, fmt, xdt)) return BL_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (bl::gemv_max_tokens(fmt, bitlinear_packed_row_bytes(K, fmt)) < 1) return BL_ERR_UNSUPPORTED;
-  return cuda_status(bl::launch_gemv(packed, fmt, gamma, N, K, x, xdt, scale, M, y, ydt, st));
+  if (!uses_gemm(M, K)) {
+    if (bl::gemv_max_tokens(fmt, bitlinear_packed_row_bytes(K, fmt)) < 1) return BL_ERR_UNSUPPORTED;
+    return cuda_status(bl::launch_gemv(packed, fmt, gamma, N, K, x, xdt, scale, M, y, ydt, st));
+  }
+  uint8_t* scratch = static_cast<uint8_t*>(ws) + BL_WS_HEADER_BYTES;
+  const int8_t* xq = static_cast<const int8_t*>(x);
+  if (xdt != BL_I8) {
+    if (bl::launch_act_quant(x, xdt, M, K, reinterpret_cast<int8_t*>(scratch), scale, st) != cudaSuccess)
+      return BL_ERR_CUDA;
+    xq = reinterpret_cast<const int8_t*>(scratch);
+    scratch += round256(static_cast<size_t>(M * K));
+  }
+  const int64_t rb2 = bitlinear_packed_row_bytes(K, BL_PACK_I2);
+  const uint8_t* w2 = packed;
+  if (fmt == BL_PACK_T5) {
+    if (bl::launch_t5_to_i2(packed, N, K, bitlinear_packed_row_bytes(K, fmt), scratch, rb2, st) != cudaSuccess)
+      return BL_ERR_CUDA;
+    w2 = scratch;
+  }
+  return cuda_status(bl::launch_gemm_i2(xq, w2, rb2, gamma, scale, y, ydt, M, N, K, ws, 0, 0, st));
+}
+
+bl_status bitlinear_selftest_wait_timeout(void* ws, size_t ws_bytes, void* stream) {
+  // 16 tokens x 128 rows x 128 K: the header plus 8 KB of operand space that is never touched
+  if (ws == nullptr || ws_bytes < BL_WS_HEADER_BYTES + 8192) return BL_ERR_INVALID_VALUE;
+  if (!aligned(ws, 16)) return BL_ERR_MISALIGNED;
+  uint8_t* op = static_cast<uint8_t*>(ws) + BL_WS_HEADER_BYTES;
+  const float* g = reinterpret_cast<const float*>(op);
+  return cuda_status(bl::launch_gemm_i2(reinterpret_cast<const int8_t*>(op), op, 32, g, g, op, BL_I32, 16, 128,
+                                        128, ws, int64_t{1} << 20, 1, static_cast<cudaStream_t>(stream)));
 }
 
 bl_status bitlinear_device_status(void* ws, void* stream) {

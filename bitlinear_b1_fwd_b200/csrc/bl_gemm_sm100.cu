@@ -1,0 +1,530 @@
+// bl_gemm_sm100.cu -- prefill GEMM on the 5th-generation tensor cores.
+//
+// acc[t, n] = sum_k W_q[n, k] x_q[t, k] with INT32 accumulation, then the
+// dequantization y = acc * gamma * s_t / 127 in the epilogue ("BitNet b1.58深度
+// 解析：三值权重如何重塑大模型推理" §4.2, §3.3, §5.3).  For many tokens the
+// product is a dense contraction, so it runs as int8 x int8 -> s32 MMAs:
+//
+//   - the MMA's M dimension is 128 weight rows and its N dimension is BT
+//     tokens (16..256), so one tile expands each packed weight once and reuses
+//     it for BT tokens;
+//   - per pipeline stage a TMA load brings the x_q tile [BT x 128 B] in the
+//     128-byte-swizzled K-major layout the MMA reads, and a second one the
+//     packed 2-bit tile [128 rows x 32 B];
+//   - four expansion warps turn 2-bit digits into signed int8 weights with a
+//     byte-permute lookup and write them in the same swizzled layout;
+//   - one thread issues tcgen05.mma.kind::i8 (K = 32 each) into an INT32
+//     accumulator in tensor memory, double-buffered across tiles;
+//   - four epilogue warps read the accumulator with tcgen05.ld, dequantize
+//     and store, overlapping the next tile's main loop.
+// The kernel is persistent (one CTA per SM, tiles strided by the grid).  Every
+// wait is bounded: on expiry the kernel sets the workspace timeout flag, drains
+// what it issued, frees its tensor memory and returns.
+#include <cuda.h>
+
+#include "bl_common.cuh"
+#include "bl_kernels.h"
+
+namespace bl {
+namespace {
+
+constexpr int kGemmThreads = 384;  // warp 0 TMA, 1 MMA, 4-7 expansion, 8-11 epilogue
+constexpr int kStages = 4;
+constexpr int kBN = 128;  // weight rows per tile = MMA M
+constexpr int kBK = 128;  // K per stage = 4 MMAs of K = 32
+constexpr uint32_t kPackedStage = kBN * kBK / 4;  // 4096 bytes
+constexpr uint32_t kExpStage = kBN * kBK;         // 16384 bytes
+constexpr long long kTimeoutCycles = 1ll << 32;   // ~2 s at 1.9 GHz
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---- mbarrier ----------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Single-thread bounded wait.  False if the limit ran out or another role aborted.
+__device__ __forceinline__ bool wait1(uint64_t* bar, uint32_t parity, long long limit,
+                                      volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > limit) return false;
+  }
+}
+
+// Bounded wait that ignores the abort flag (used to drain work already issued).
+__device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity, long long limit) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > limit) return false;
+  return true;
+}
+
+// Warp-uniform bounded wait: every lane returns the same answer.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, long long limit,
+                                          volatile int* abort_flag) {
+  const long long t0 = clock64();
+  for (;;) {
+    const bool done = mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, done)) return true;
+    const bool give_up = (*abort_flag != 0) || (clock64() - t0 > limit);
+    if (__any_sync(0xffffffffu, give_up)) return false;
+  }
+}
+
+// ---- TMA --------------------------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
+          "r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+// ---- tcgen05 ----------------------------------------------------------------------
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (the layout a 128-byte-swizzled TMA load writes).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3fffu);  // start address
+  d |= static_cast<uint64_t>(1) << 16;                 // leading offset (unused when swizzled K-major)
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;         // stride offset between 8-row groups
+  d |= static_cast<uint64_t>(1) << 46;                 // descriptor version
+  d |= static_cast<uint64_t>(2) << 61;                 // 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor of kind::i8: s32 accumulator, signed A and B, both
+// K-major, MMA shape M x N.
+__host__ __device__ constexpr uint32_t i8_idesc(int m, int n) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+template <int NCOL>
+__device__ __forceinline__ void tmem_load(uint32_t taddr, uint32_t (&r)[NCOL]);
+
+template <>
+__device__ __forceinline__ void tmem_load<32>(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+template <>
+__device__ __forceinline__ void tmem_load<16>(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// 16 two-bit digits (q + 1) -> 16 signed int8 weights q, in K order.  The
+// digits are spread into nibbles, which select bytes of 0x000100FF
+// (digit 0 -> 0xFF = -1, 1 -> 0, 2 -> +1, 3 -> 0).
+__device__ __forceinline__ uint32_t spread8(uint32_t h) {  // 8 digits in bits 0..15 -> 8 nibbles
+  uint32_t x = h & 0xffffu;
+  x = (x | (x << 8)) & 0x00ff00ffu;
+  x = (x | (x << 4)) & 0x0f0f0f0fu;
+  x = (x | (x << 2)) & 0x33333333u;
+  return x;
+}
+__device__ __forceinline__ uint4 expand16(uint32_t w) {
+  const uint32_t lo = spread8(w), hi = spread8(w >> 16);
+  uint4 o;
+  o.x = __byte_perm(0x000100ffu, 0u, lo & 0xffffu);
+  o.y = __byte_perm(0x000100ffu, 0u, lo >> 16);
+  o.z = __byte_perm(0x000100ffu, 0u, hi & 0xffffu);
+  o.w = __byte_perm(0x000100ffu, 0u, hi >> 16);
+  return o;
+}
+
+template <int BT>
+struct GemmCfg {
+  static constexpr uint32_t kXStage = BT * 128;
+  static constexpr uint32_t kTmemCols = (2 * BT < 32) ? 32 : 2 * BT;
+  static constexpr uint32_t kChunk = BT < 32 ? BT : 32;  // accumulator columns per tcgen05.ld
+  static constexpr size_t kSmem =
+      1024 + kStages * (kXStage + kExpStage + kPackedStage) + 8 * (3 * kStages + 5) + 16;
+};
+
+template <int BT>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_i2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                   const float* __restrict__ gamma, const float* __restrict__ scale, void* __restrict__ y,
+                   int ydt, int M, int N, int K, WsHeader* __restrict__ hdr, long long limit,
+                   int skip_producer) {
+  using Cfg = GemmCfg<BT>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* base = smem_raw + pad;
+  uint8_t* xs = base;                              // kStages x [BT x 128 B], swizzled
+  uint8_t* es = xs + kStages * Cfg::kXStage;       // kStages x [128 x 128 B], swizzled
+  uint8_t* ps = es + kStages * kExpStage;          // kStages x [128 x 32 B]
+  uint64_t* full = reinterpret_cast<uint64_t*>(ps + kStages * kPackedStage);
+  uint64_t* expd = full + kStages;
+  uint64_t* empty = expd + kStages;
+  uint64_t* accf = empty + kStages;  // 2
+  uint64_t* acce = accf + 2;         // 2
+  uint64_t* drain = acce + 2;        // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kblocks = (K + kBK - 1) / kBK;
+  const int n_tiles = (N + kBN - 1) / kBN;
+  const int t_tiles = (M + BT - 1) / BT;
+  const int tiles = n_tiles * t_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(expd + s, 4);
+      mbar_init(empty + s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(accf + a, 1);
+      mbar_init(acce + a, 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(Cfg::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto fail = [&](uint32_t site) {
+    set_flag(hdr, kFlagTimeout, site);
+    *abort_flag = 1;
+  };
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0 && !skip_producer) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+        const int n_t = tile % n_tiles, t_t = tile / n_tiles;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          if (!wait1(empty + s, ph ^ 1, limit, abort_flag)) {
+            fail(0x201);
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(full + s, Cfg::kXStage + kPackedStage);
+          tma_load_2d(xs + s * Cfg::kXStage, &tm_x, full + s, kb * kBK, t_t * BT);
+          tma_load_2d(ps + s * kPackedStage, &tm_w, full + s, kb * (kBK / 4), n_t * kBN);
+        }
+      }
+      // copies still in flight land before the CTA leaves (bounded)
+      for (int j = (it > kStages ? it - kStages : 0); j < it; ++j)
+        (void)wait_drain(full + (j % kStages), (j / kStages) & 1, limit);
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ---------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = i8_idesc(kBN, BT);
+      int it = 0, tc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tc) {
+        const int a = tc & 1;
+        if (!wait1(acce + a, ((tc >> 1) & 1) ^ 1, limit, abort_flag)) {
+          fail(0x301);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + static_cast<uint32_t>(a * BT);
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          if (!wait1(full + s, ph, limit, abort_flag) || !wait1(expd + s, ph, limit, abort_flag)) {
+            fail(0x302);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t xa = smem_u32(xs + s * Cfg::kXStage), ea = smem_u32(es + s * kExpStage);
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k)
+            mma_i8(d, sw128_desc(ea + 32 * k), sw128_desc(xa + 32 * k), idesc, (kb | k) != 0);
+          mma_commit(empty + s);
+        }
+        if (ok) mma_commit(accf + a);
+      }
+      // every MMA issued above completes before the accumulator memory is freed
+      mma_commit(drain);
+      (void)wait_drain(drain, 0, limit);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------ expansion ----------------------------------
+    const int r = threadIdx.x - 128;  // weight row of the tile, 0..127
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+      for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        if (!wait_warp(full + s, ph, limit, abort_flag)) {
+          if (lane == 0) fail(0x401);
+          ok = false;
+          break;
+        }
+        const uint4* src = reinterpret_cast<const uint4*>(ps + s * kPackedStage + r * 32);
+        const uint4 p0 = src[0], p1 = src[1];
+        const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+        uint8_t* row = es + s * kExpStage + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(row + ((j ^ (r & 7)) << 4)) = expand16(w[j]);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(expd + s);
+      }
+    }
+  } else if (warp >= 8) {
+    // ------------------------------ epilogue -----------------------------------
+    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    const float g = __ldg(gamma);
+    int tc = 0;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
+      const int a = tc & 1;
+      if (!wait_warp(accf + a, (tc >> 1) & 1, limit, abort_flag)) {
+        if (lane == 0) fail(0x501);
+        break;
+      }
+      tc_fence_after();
+      const int n_t = tile % n_tiles, t_t = tile / n_tiles;
+      const int n = n_t * kBN + 32 * q + lane;
+#pragma unroll 1
+      for (int j0 = 0; j0 < BT; j0 += Cfg::kChunk) {
+        uint32_t acc[Cfg::kChunk];
+        tmem_load<Cfg::kChunk>(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(a * BT + j0),
+                               acc);
+#pragma unroll
+        for (int j = 0; j < static_cast<int>(Cfg::kChunk); ++j) {
+          const int t = t_t * BT + j0 + j;
+          if (t < M && n < N) {
+            const int64_t o = static_cast<int64_t>(t) * N + n;
+            const int v = static_cast<int>(acc[j]);
+            if (ydt == BL_I32) {
+              static_cast<int32_t*>(y)[o] = v;
+            } else {
+              const float yv = __fmul_rn(__int2float_rn(v), dequant_factor(g, __ldg(scale + t)));
+              if (ydt == BL_F32)
+                static_cast<float*>(y)[o] = yv;
+              else
+                static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(yv);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce + a);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(Cfg::kTmemCols)
+                 : "memory");
+  }
+}
+
+// T5 -> 2-bit transcoding (for the tensor-core path on base-3 weights): one
+// thread writes one 16-byte segment (64 weights) of a 2-bit row.  The base-3
+// digit of a weight is its 2-bit code (both are q + 1); invalid bytes (>= 243)
+// read as weight 0, as in the decode kernel.
+__global__ void __launch_bounds__(256)
+    t5_to_i2_kernel(const uint8_t* __restrict__ t5, int64_t N, int64_t K, int64_t rb5, uint8_t* __restrict__ i2,
+                    int64_t rb2) {
+  __shared__ uint16_t lut[256];
+  for (int b = threadIdx.x; b < 256; b += blockDim.x) {
+    uint32_t v = b, d = 0;
+    if (b < 243) {
+      for (int i = 0; i < 5; ++i) {
+        d |= (v % 3) << (2 * i);
+        v /= 3;
+      }
+    } else {
+      d = 0x155;  // five weight-0 digits
+    }
+    lut[b] = static_cast<uint16_t>(d);
+  }
+  __syncthreads();
+  const int64_t segs = rb2 / 16;
+  for (int64_t gid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; gid < N * segs;
+       gid += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = gid / segs, sg = gid - n * segs;
+    const int64_t kb = 64 * sg;
+    uint32_t out[4] = {0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u};
+    const uint8_t* row = t5 + n * rb5;
+    for (int64_t b = kb / 5; b <= (kb + 63) / 5; ++b) {
+      const uint32_t digs = lut[b < rb5 ? row[b] : 121];
+#pragma unroll
+      for (int i = 0; i < 5; ++i) {
+        const int64_t k = 5 * b + i, kk = k - kb;
+        if (kk >= 0 && kk < 64) {
+          const uint32_t code = (k < K) ? ((digs >> (2 * i)) & 3u) : 1u;
+          const int wi = static_cast<int>(kk >> 4), sh = static_cast<int>(2 * (kk & 15));
+          out[wi] = (out[wi] & ~(3u << sh)) | (code << sh);
+        }
+      }
+    }
+    *reinterpret_cast<uint4*>(i2 + n * rb2 + sg * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
+// ---- host side --------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool encode_2d_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t stride,
+                  uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {stride};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BT>
+cudaError_t launch_gemm_bt(const int8_t* xq, const uint8_t* w, int64_t rb, const float* gamma, const float* scale,
+                           void* y, int ydt, int64_t M, int64_t N, int64_t K, void* ws, long long limit,
+                           int skip_producer, cudaStream_t st) {
+  CUtensorMap tx, tw;
+  if (!encode_2d_u8(&tx, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(K), 128, BT,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (!encode_2d_u8(&tw, w, static_cast<uint64_t>(rb), static_cast<uint64_t>(N), static_cast<uint64_t>(rb),
+                    kBK / 4, kBN, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  auto kern = gemm_i2_kernel<BT>;
+  const size_t smem = GemmCfg<BT>::kSmem;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = ((N + kBN - 1) / kBN) * ((M + BT - 1) / BT);
+  const int sms = device_sms();
+  const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
+  kern<<<grid, kGemmThreads, smem, st>>>(tx, tw, gamma, scale, y, ydt, static_cast<int>(M), static_cast<int>(N),
+                                         static_cast<int>(K), static_cast<WsHeader*>(ws), limit, skip_producer);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int gemm_token_tile(int64_t M) {
+  if (M > 128) return 256;
+  if (M > 64) return 128;
+  if (M > 32) return 64;
+  if (M > 16) return 32;
+  return 16;
+}
+
+cudaError_t launch_gemm_i2(const int8_t* xq, const uint8_t* w, int64_t rb, const float* gamma, const float* scale,
+                           void* y, int ydt, int64_t M, int64_t N, int64_t K, void* ws, long long limit_cycles,
+                           int skip_producer, cudaStream_t st) {
+  const long long limit = limit_cycles > 0 ? limit_cycles : kTimeoutCycles;
+  switch (gemm_token_tile(M)) {
+    case 16: return launch_gemm_bt<16>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ws, limit, skip_producer, st);
+    case 32: return launch_gemm_bt<32>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ws, limit, skip_producer, st);
+    case 64: return launch_gemm_bt<64>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ws, limit, skip_producer, st);
+    case 128: return launch_gemm_bt<128>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ws, limit, skip_producer, st);
+    default: return launch_gemm_bt<256>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ws, limit, skip_producer, st);
+  }
+}
+
+cudaError_t launch_t5_to_i2(const uint8_t* t5, int64_t N, int64_t K, int64_t rb5, uint8_t* i2, int64_t rb2,
+                            cudaStream_t st) {
+  const int64_t work = N * (rb2 / 16);
+  const int64_t cap = static_cast<int64_t>(device_sms()) * 8;
+  int64_t grid = (work + 255) / 256;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  t5_to_i2_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(t5, N, K, rb5, i2, rb2);
+  return cudaGetLastError();
+}
+
+}  // namespace bl

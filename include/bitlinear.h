@@ -165,6 +165,15 @@ BL_API bl_status bitlinear_forward(const uint8_t *packed, int fmt, const float *
                             int64_t K, const void *x, int xdt, float *scale, int64_t M, void *y,
                             int ydt, void *ws, size_t ws_bytes, void *stream);
 
+/* Failure-detection self test: launches the tensor-core kernel with its data
+ * producer switched off and a wait limit of about a millisecond, so that its
+ * bounded waits run out; the kernel then records BL_ERR_DEVICE_TIMEOUT in the
+ * workspace flag, frees what it holds and exits (no memory is read or written
+ * besides the flag).  Read the result with bitlinear_device_status.  The pages
+ * have no counterpart; this tests the error path of every wait.
+ *   ws  at least BL_WS_HEADER_BYTES + 8192 bytes. */
+BL_API bl_status bitlinear_selftest_wait_timeout(void *ws, size_t ws_bytes, void *stream);
+
 /* Synchronize `stream`, then read and clear the workspace's device flags.
  * Returns BL_OK, BL_ERR_DEVICE_TIMEOUT, BL_ERR_BAD_CODE or BL_ERR_CUDA. */
 BL_API bl_status bitlinear_device_status(void *ws, void *stream);

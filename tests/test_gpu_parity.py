@@ -149,8 +149,8 @@ def test_quantize_weights_3b(orc, layer):
 
 
 def test_ternarize_threshold_boundary(orc):
-    """A fixed gamma and weights planted at and next to d/2 = (gamma + eps)/2,
-    including fp32 values whose quotient by d rounds to exactly 0.5."""
+    """A fixed gamma and weights planted at and next to d/2 = (gamma + eps)/2:
+    the codes must equal the oracle's IEEE-division codes at the boundary."""
     gamma = np.float32(0.0163)
     d = np.float32(gamma + np.float32(1e-5))
     half = np.float32(d / np.float32(2))
@@ -165,8 +165,9 @@ def test_ternarize_threshold_boundary(orc):
         plant += [v, -v]
     W = synth.normal_f32(61, (3, 1000), 0.02)
     W[0, :len(plant)] = plant
-    ratio_half = sum(1 for p in plant if np.float32(abs(p) / d) == np.float32(0.5))
-    assert ratio_half > 2   # some planted quotients round to exactly 0.5
+    # exactly d/2 divides to 0.5 (-> 0); every fp32 above it divides to more than 0.5
+    assert np.float32(half / d) == np.float32(0.5)
+    assert all(np.float32(abs(p) / d) > np.float32(0.5) for p in plant[7:7 + 128])
     for fmt in (I2, T5):
         Wd = dev(W)
         g = torch.tensor([float(gamma)], dtype=torch.float32, device="cuda")
