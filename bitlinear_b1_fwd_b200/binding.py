@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(HERE, "libbitlinear.so")
 
 BL_OK, BL_ERR_INVALID_VALUE, BL_ERR_UNSUPPORTED, BL_ERR_MISALIGNED = 0, 1, 2, 3
 BL_ERR_WORKSPACE_TOO_SMALL, BL_ERR_CUDA, BL_ERR_DEVICE_TIMEOUT, BL_ERR_BAD_CODE = 4, 5, 6, 7
+BL_ERR_SCRATCH_LIMIT = 8
 BL_F32, BL_BF16, BL_I8, BL_I32 = 0, 1, 2, 3
 BL_PACK_I2, BL_PACK_T5 = 0, 1
 BL_WS_HEADER_BYTES = 256
@@ -31,6 +32,7 @@ SIGNATURES = {
     "bitlinear_workspace_init": (_I, [_P, _SZ, _P]),
     "bitlinear_quantize_weights": (_I, [_P, _I, _I64, _I64, _F, _I, _P, _P, _P, _P, _SZ, _P]),
     "bitlinear_absmean": (_I, [_P, _I, _I64, _I64, _P, _P, _SZ, _P]),
+    "bitlinear_absmean_noalloc": (_I, [_P, _I, _I64, _I64, _P, _P]),
     "bitlinear_ternarize_pack": (_I, [_P, _I, _I64, _I64, _P, _F, _I, _P, _P, _P]),
     "bitlinear_pack": (_I, [_P, _I64, _I64, _I, _P, _P, _SZ, _P]),
     "bitlinear_quantize_acts": (_I, [_P, _I, _I64, _I64, _P, _P, _P]),
@@ -138,6 +140,14 @@ def bitlinear_absmean(W, gamma, ws, stream=None) -> None:
     N, K = W.shape
     _check(lib().bitlinear_absmean(_ptr(W), dtype_code(W), N, K, _ptr(gamma), _ptr(ws),
                                    ws.numel() * ws.element_size(), _stream(stream)), "bitlinear_absmean")
+
+
+def bitlinear_absmean_noalloc(W, gamma, stream=None) -> None:
+    """gamma of W without a workspace (the library's fixed device scratch)."""
+    _contig(W, gamma)
+    N, K = W.shape
+    _check(lib().bitlinear_absmean_noalloc(_ptr(W), dtype_code(W), N, K, _ptr(gamma), _stream(stream)),
+           "bitlinear_absmean_noalloc")
 
 
 def bitlinear_ternarize_pack(W, gamma, eps, fmt, packed, codes, stream=None) -> None:

@@ -41,6 +41,8 @@ const char* bitlinear_status_string(int status) {
     case BL_ERR_CUDA: return "BL_ERR_CUDA: a CUDA runtime call failed";
     case BL_ERR_DEVICE_TIMEOUT: return "BL_ERR_DEVICE_TIMEOUT: a bounded wait in a kernel ran out";
     case BL_ERR_BAD_CODE: return "BL_ERR_BAD_CODE: a weight code outside {-1, 0, 1} was packed";
+    case BL_ERR_SCRATCH_LIMIT:
+      return "BL_ERR_SCRATCH_LIMIT: N*K exceeds the fixed scratch of bitlinear_absmean_noalloc (2^28 elements)";
     default: return "unknown bitlinear status";
   }
 }

@@ -77,7 +77,8 @@ typedef enum {
   BL_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes below the query function's size */
   BL_ERR_CUDA = 5,                /* a CUDA runtime call failed */
   BL_ERR_DEVICE_TIMEOUT = 6,      /* a kernel's bounded wait ran out (device flag) */
-  BL_ERR_BAD_CODE = 7             /* bitlinear_pack met a code outside {-1,0,1} */
+  BL_ERR_BAD_CODE = 7,            /* bitlinear_pack met a code outside {-1,0,1} */
+  BL_ERR_SCRATCH_LIMIT = 8        /* too large for bitlinear_absmean_noalloc's fixed scratch */
 } bl_status;
 
 typedef enum { BL_F32 = 0, BL_BF16 = 1, BL_I8 = 2, BL_I32 = 3 } bl_dtype;
@@ -132,6 +133,26 @@ BL_API bl_status bitlinear_quantize_weights(const void *W, int wdt, int64_t N, i
  *          that are done). */
 BL_API bl_status bitlinear_absmean(const void *W, int wdt, int64_t N, int64_t K, float *gamma,
                                    void *ws, size_t ws_bytes, void *stream);
+
+/* The absmean scale (step 1, the same result as bitlinear_absmean) for
+ * callers that cannot allocate device memory at the time they need it: for
+ * example code whose device memory belongs to another runtime or pool that
+ * hands out no raw buffers, or a service that reserves all its memory at
+ * start-up and may not call cudaMalloc / cudaFree (which can synchronize the
+ * device) afterwards.  The pages have no counterpart; this is a library
+ * convenience.
+ *   W      [N, K] fp32 or bf16, 16-byte aligned;  gamma [1] fp32 device output.
+ *   Limit  N * K <= 2^28 elements (32768 chunks of 8192); larger sizes return
+ *          BL_ERR_SCRATCH_LIMIT without launching anything.
+ * The partial sums live in a 256 KiB device array owned by the library (held
+ * on every GPU that loads it, until the process exits); nothing is allocated.
+ * The first call on a device looks up the array's device address (once per
+ * device), so make that first call before any stream capture.  Every call
+ * shares the one array and resets its counter: calls whose kernels overlap on
+ * the GPU (different streams, or different host threads) race and must be
+ * serialized by the caller. */
+BL_API bl_status bitlinear_absmean_noalloc(const void *W, int wdt, int64_t N, int64_t K, float *gamma,
+                                           void *stream);
 
 /* Ternarize and pack with a gamma that is already on the device (step 2-3 only;
  * for instance a gamma reduced across ranks).  Same arrays as above; `gamma`
