@@ -63,6 +63,10 @@ def csrc_digest() -> str:
     return h.hexdigest()[:16]
 
 
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_PER_BF16 = 2.0  # nominal dense ratio: 4.5 PFLOP/s int8 : 2.25 bf16
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -71,6 +75,17 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_int8_peak():
+    """int8 dense peak = the measured bf16 burst peak x the nominal int8 : bf16 ratio."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]) * INT8_PER_BF16, "measured bf16 burst x 2"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS * INT8_PER_BF16, "fallback bf16 x 2"
 
 
 def profiled_traffic(kernel: str, workload: str):
@@ -141,6 +156,29 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
                 "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------
+# multi-rank plumbing (one process per GPU; weak scaling over replicas)
+# ----------------------------------------------------------------------------
+
+def rank_seed_offset(rank: int) -> int:
+    """Each rank draws its own replica of the workload."""
+    return 10000 * rank
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The slowest rank's time (all ranks take part; identity for one rank)."""
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(step_bytes: int, world: int, ms_per_step: float) -> float:
+    """Aggregate GB/s: the bytes every rank processed in one step over the step time."""
+    return step_bytes * world / (ms_per_step * 1e-3) / 1e9
 
 
 # ----------------------------------------------------------------------------
@@ -215,7 +253,7 @@ def run_gpu(args, wl, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     fmt, M = wl["fmt"], wl["M"]
-    rank_seed = 10000 * rank
+    rank_seed = rank_seed_offset(rank)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
 
     layers = []
@@ -299,17 +337,18 @@ def run_gpu(args, wl, rank, world, local_rank):
         for i in range(args.steps):
             step(i, step_events[i])
         t_end.record(stream)
-    graph.replay()              # one untimed replay (first-launch costs of the graph)
-    stream.synchronize()
+    with torch.cuda.stream(stream):
+        graph.replay()          # one untimed replay (first-launch costs of the graph)
+    torch.cuda.synchronize()
 
     sampler = ClockSampler(local_rank)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     with sampler:
-        graph.replay()
-        stream.synchronize()
-    torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            graph.replay()
+        torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     ms = t_start.elapsed_time(t_end)
@@ -326,10 +365,7 @@ def run_gpu(args, wl, rank, world, local_rank):
                 per_op[op].append((li, evs[(li, oi)].elapsed_time(evs[(li, oi + 1)])))
     step_bytes = sum(sum(L["bytes"][op] for op in ops) for L in layers)
 
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms, world, dev)
 
     # ---- end to end through the public API from pinned host buffers ----
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
@@ -352,28 +388,118 @@ def run_gpu(args, wl, rank, world, local_rank):
                 L["y_host"].copy_(L["y"], non_blocking=True)
         e1.record(stream)
     stream.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
-    e2e_ms = float(e2e_t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
 
     del graph
-    res = dict(ms_total=ms_max, per_op=per_op, step_bytes=step_bytes, layers=layers, ops=ops,
+    prefill = run_prefill(args, dev, stream, rank_seed, l2) if args.prefill else None
+    res = dict(prefill=prefill, ms_total=ms_max, per_op=per_op, step_bytes=step_bytes, layers=layers, ops=ops,
                clocks=sampler.summary(), e2e_ms=e2e_ms, e2e_steps=e2e_steps, h2d=h2d, d2h=d2h,
                rot=rot, l2=l2, launches_per_step=len(layers) * len(ops))
     return res
 
 
+def run_prefill(args, dev, stream, rank_seed, l2):
+    """3B prefill layer (M=4096, K=3200 -> N=8640, 2-bit): per-token INT8
+    quantization and the tensor-core product timed separately (CUDA events in
+    one graph), inputs rotated over copies that together exceed L2."""
+    import numpy as np
+    import torch
+
+    from bitlinear_b1_fwd_b200 import binding as B
+    from bitlinear_b1_fwd_b200 import synth
+
+    M, K, N = 4096, 3200, 8640
+    Wh, xh = synth.prefill_3b_inputs()
+    if rank_seed:
+        Wh = synth.normal_f32(1003 + rank_seed, (N, K), 0.02)
+    rb = B.bitlinear_packed_row_bytes(K, 0)
+    W = torch.from_numpy(Wh).to(dev)
+    x0 = torch.from_numpy(xh.view(np.int16)).to(dev).view(torch.bfloat16)
+    gamma = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = torch.zeros(B.bitlinear_quantize_weights_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+    packed0 = torch.empty((N, rb), dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(stream):
+        B.bitlinear_quantize_weights(W, 1e-5, 0, packed0, None, gamma, ws, stream)
+    stream.synchronize()
+    del W
+    per_copy = M * K * 2 + M * K + N * rb + M * N * 2
+    rot = max(2, -(-2 * l2 // per_copy))
+    xs = [x0] + [x0.clone() for _ in range(rot - 1)]
+    pk = [packed0] + [packed0.clone() for _ in range(rot - 1)]
+    xq = [torch.empty((M, K), dtype=torch.int8, device=dev) for _ in range(rot)]
+    sc = [torch.empty(M, dtype=torch.float32, device=dev) for _ in range(rot)]
+    ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(rot)]
+    fws = torch.zeros(B.bitlinear_forward_workspace_bytes(M, N, K, 0, B.BL_I8), dtype=torch.uint8, device=dev)
+
+    def step(i, ev=None):
+        r = i % rot
+        if ev is not None:
+            ev[0].record(stream)
+        B.bitlinear_quantize_acts(xs[r], xq[r], sc[r], stream)
+        if ev is not None:
+            ev[1].record(stream)
+        B.bitlinear_forward(pk[r], 0, gamma, N, K, xq[r], sc[r], ys[r], fws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    steps = max(1, args.prefill_steps)
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            step(i)
+    stream.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(steps)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+        for i in range(steps):
+            step(i, evs[i])
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    st = B.bitlinear_device_status(fws, stream)
+    if st != B.BL_OK:
+        raise RuntimeError(f"prefill device status {B.status_string(st)}")
+    act_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    gemm_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    del g
+    ops = 2.0 * M * N * K
+    return dict(M=M, K=K, N=N, act_ms=act_ms, gemm_ms=gemm_ms, ops=ops, rot=rot, steps=steps,
+                act_bytes=M * K * 2 + M * K + 4 * M)
+
+
+def prefill_summary(p):
+    if p is None:
+        return None
+    peak, kind = measured_int8_peak()
+    tops = p["ops"] / (p["gemm_ms"] * 1e-3) / 1e12
+    fwd_tops = p["ops"] / ((p["gemm_ms"] + p["act_ms"]) * 1e-3) / 1e12
+    hbm, hkind = measured_peaks()
+    act_gbs = p["act_bytes"] / (p["act_ms"] * 1e-3) / 1e9
+    return {"workload": f"3B prefill: M={p['M']} tokens, K={p['K']} -> N={p['N']}, 2-bit, bf16 x with "
+                        "16 outlier channels x30, bf16 y",
+            "value": tops, "unit": "TOPS (int8)", "forward_TOPS_incl_act_quant": fwd_tops,
+            "gemm_us": p["gemm_ms"] * 1e3, "act_quant_us": p["act_ms"] * 1e3,
+            "act_quant_GB_s": act_gbs, "act_quant_frac_of_hbm": act_gbs / hbm,
+            "roofline": {"bound": "tensor", "kernel": "gemm_i2_kernel", "achieved": tops, "peak": peak,
+                         "peak_kind": kind, "unit": "TOPS", "frac": tops / peak,
+                         "traffic": profiled_traffic("gemm_i2_kernel", "3b_prefill")},
+            "steps": p["steps"], "l2": f"inputs rotated over {p['rot']} copies (> 2x L2)"}
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="3b_decode")
     ap.add_argument("--phase", choices=["all", "forward"], default="all")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--prefill", action=argparse.BooleanOptionalAction, default=True,
+                    help="also time the 3B prefill layer (INT8 TOPS of the tensor-core product)")
+    ap.add_argument("--prefill-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=10.0,
                     help="seconds of oracle time for the cpu_baseline sample (0 = skip)")
     args = ap.parse_args()
@@ -423,7 +549,7 @@ def main():
 
     if rank == 0:
         ms = res["ms_total"] / args.steps
-        value = res["step_bytes"] * world / (ms * 1e-3) / 1e9
+        value = whole_job_gbs(res["step_bytes"], world, ms)
         peak, peak_kind = measured_peaks()
         # per-op summary and the dominant kernel
         stages = {}
@@ -440,7 +566,9 @@ def main():
         avg_launch_ms = stages[dom]["ms_per_step"] * args.steps / launches
         bytes_per_launch = stages[dom]["bytes_per_step"] / len(res["layers"])
         achieved = bytes_per_launch / (avg_launch_ms * 1e-3) / 1e9
-        kernel_name = {"absmean": "absmean_kernel", "ternarize_pack": "ternarize_pack_kernel",
+        flat = wl["fmt"] == 0 and all(K % 64 == 0 for (_, K) in wl["layers"])
+        kernel_name = {"absmean": "absmean_bulk_kernel",
+                       "ternarize_pack": "ternarize_flat_kernel" if flat else "ternarize_pack_kernel",
                        "forward": "gemv_kernel"}[dom]
         traffic = profiled_traffic(kernel_name, args.workload)
         cpu = None
@@ -448,7 +576,7 @@ def main():
             v, s, dt = time_oracle(wl, args.phase, args.cpu_budget)
             cpu = {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
                    "sample": f"{s} full oracle steps of the same workload ({dt:.1f} s, 1 thread)"}
-        e2e_value = res["step_bytes"] * world / (res["e2e_ms"] * 1e-3) / 1e9
+        e2e_value = whole_job_gbs(res["step_bytes"], world, res["e2e_ms"])
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -466,6 +594,7 @@ def main():
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": res["h2d"],
                     "d2h_bytes_per_step": res["d2h"], "steps": res["e2e_steps"]},
+            "prefill": prefill_summary(res["prefill"]),
             "gpu_launches": res["launches_per_step"] * args.steps,
             "clocks": res["clocks"],
         }

@@ -38,6 +38,7 @@ __global__ void __launch_bounds__(kActThreads)
 #pragma unroll
     for (int w = 1; w < kActThreads / 32; ++w) a = fmaxf(a, red[w]);
     const float s = fmaxf(a, 1e-6f);
+    const float c127 = __fdiv_rn(127.0f, s);
     if (vec) {
       for (int64_t v = threadIdx.x; v < K / 8; v += blockDim.x) {
         float e[8];
@@ -45,14 +46,14 @@ __global__ void __launch_bounds__(kActThreads)
         uint32_t lo = 0, hi = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          lo |= static_cast<uint32_t>(quant_act(e[j], s) & 0xff) << (8 * j);
-          hi |= static_cast<uint32_t>(quant_act(e[j + 4], s) & 0xff) << (8 * j);
+          lo |= static_cast<uint32_t>(quant_act_fast(e[j], s, c127) & 0xff) << (8 * j);
+          hi |= static_cast<uint32_t>(quant_act_fast(e[j + 4], s, c127) & 0xff) << (8 * j);
         }
         *reinterpret_cast<uint2*>(xq + base + 8 * v) = make_uint2(lo, hi);
       }
     } else {
       for (int64_t k = threadIdx.x; k < K; k += blockDim.x)
-        xq[base + k] = static_cast<int8_t>(quant_act(load_elem<XDT>(x, base + k), s));
+        xq[base + k] = static_cast<int8_t>(quant_act_fast(load_elem<XDT>(x, base + k), s, c127));
     }
     if (threadIdx.x == 0) scale[m] = s;
     __syncthreads();  // red[] is reused by the next token

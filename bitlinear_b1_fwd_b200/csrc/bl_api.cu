@@ -93,7 +93,7 @@ bl_status bitlinear_quantize_weights(const void* W, int wdt, int64_t N, int64_t 
   cudaError_t e = bl::launch_absmean(W, wdt, N, K, ws, gamma, st);
   if (e != cudaSuccess) return BL_ERR_CUDA;
   const int64_t rb = bitlinear_packed_row_bytes(K, fmt);
-  return cuda_status(bl::launch_ternarize_pack(W, wdt, N, K, gamma, eps, fmt, packed, codes, rb, st));
+  return cuda_status(bl::launch_ternarize_pack(W, wdt, N, K, gamma, eps, fmt, packed, codes, rb, ws, st));
 }
 
 bl_status bitlinear_absmean(const void* W, int wdt, int64_t N, int64_t K, float* gamma, void* ws,
@@ -113,7 +113,7 @@ bl_status bitlinear_ternarize_pack(const void* W, int wdt, int64_t N, int64_t K,
   if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(codes, 16) || !aligned(gamma, 4))
     return BL_ERR_MISALIGNED;
   const int64_t rb = bitlinear_packed_row_bytes(K, fmt);
-  return cuda_status(bl::launch_ternarize_pack(W, wdt, N, K, gamma, eps, fmt, packed, codes, rb,
+  return cuda_status(bl::launch_ternarize_pack(W, wdt, N, K, gamma, eps, fmt, packed, codes, rb, nullptr,
                                                static_cast<cudaStream_t>(stream)));
 }
 

@@ -67,6 +67,20 @@ __device__ __forceinline__ int quant_act(float x, float s) {
   return __float2int_rn(t);
 }
 
+// The same code as quant_act without a division per element.  With
+// c127 = fl(127 / s), t_a = fl(x c127) differs from t = fl(fl(x / s) 127) by
+// less than 4.0001 * 2^-24 |t| (two roundings on each side), so when t_a is
+// farther than |t_a| 2^-21 from every half-integer both round to the same
+// integer and t is not a tie; otherwise (rare) the exact quotient decides.
+__device__ __forceinline__ int quant_act_fast(float x, float s, float c127) {
+  const float ta = __fmul_rn(x, c127);
+  const float qa = rintf(ta);
+  const float dist = __fsub_rn(0.5f, fabsf(__fsub_rn(ta, qa)));  // to the nearest half-integer
+  if (dist > __fmaf_rn(fabsf(ta), 0x1p-21f, 0x1p-126f))
+    return __float2int_rn(fminf(fmaxf(qa, -127.0f), 127.0f));
+  return quant_act(x, s);
+}
+
 // Dequantization factor c = (gamma * s) / 127 and the dequantized value.
 __device__ __forceinline__ float dequant_factor(float gamma, float s) {
   return __fdiv_rn(__fmul_rn(gamma, s), 127.0f);

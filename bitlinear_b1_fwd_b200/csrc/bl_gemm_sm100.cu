@@ -24,6 +24,7 @@
 
 #include "bl_common.cuh"
 #include "bl_kernels.h"
+#include "bl_sm100.cuh"
 
 namespace bl {
 namespace {
@@ -35,74 +36,6 @@ constexpr int kBK = 128;  // K per stage = 4 MMAs of K = 32
 constexpr uint32_t kPackedStage = kBN * kBK / 4;  // 4096 bytes
 constexpr uint32_t kExpStage = kBN * kBK;         // 16384 bytes
 constexpr long long kTimeoutCycles = 1ll << 32;   // ~2 s at 1.9 GHz
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// ---- mbarrier ----------------------------------------------------------------
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.b32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Single-thread bounded wait.  False if the limit ran out or another role aborted.
-__device__ __forceinline__ bool wait1(uint64_t* bar, uint32_t parity, long long limit,
-                                      volatile int* abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (clock64() - t0 > limit) return false;
-  }
-}
-
-// Bounded wait that ignores the abort flag (used to drain work already issued).
-__device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity, long long limit) {
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity))
-    if (clock64() - t0 > limit) return false;
-  return true;
-}
-
-// Warp-uniform bounded wait: every lane returns the same answer.
-__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, long long limit,
-                                          volatile int* abort_flag) {
-  const long long t0 = clock64();
-  for (;;) {
-    const bool done = mbar_try_wait(bar, parity);
-    if (__all_sync(0xffffffffu, done)) return true;
-    const bool give_up = (*abort_flag != 0) || (clock64() - t0 > limit);
-    if (__any_sync(0xffffffffu, give_up)) return false;
-  }
-}
-
-// ---- TMA --------------------------------------------------------------------------
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
-          "r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
-      : "memory");
-}
 
 // ---- tcgen05 ----------------------------------------------------------------------
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -198,7 +131,7 @@ struct GemmCfg {
   static constexpr uint32_t kTmemCols = (2 * BT < 32) ? 32 : 2 * BT;
   static constexpr uint32_t kChunk = BT < 32 ? BT : 32;  // accumulator columns per tcgen05.ld
   static constexpr size_t kSmem =
-      1024 + kStages * (kXStage + kExpStage + kPackedStage) + 8 * (3 * kStages + 5) + 16;
+      1024 + kStages * (kXStage + kExpStage + kPackedStage) + 8 * (3 * kStages + 5) + 16 + 2 * 4 * BT;
 };
 
 template <int BT>
@@ -222,6 +155,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain = acce + 2;        // 1
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* cfac = reinterpret_cast<float*>(tmem_slot + 4);  // [2][BT] dequant factors per accumulator buffer
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kblocks = (K + kBK - 1) / kBK;
@@ -351,13 +285,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int tc = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
       const int a = tc & 1;
-      if (!wait_warp(accf + a, (tc >> 1) & 1, limit, abort_flag)) {
-        if (lane == 0) fail(0x501);
+      const int n_t = tile % n_tiles, t_t = tile / n_tiles;
+      const int n = n_t * kBN + 32 * q + lane;
+      // dequant factor c_t = (gamma s_t) / 127 of each token of the tile, once
+      float* cf = cfac + a * BT;
+      for (int j = threadIdx.x - 256; j < BT; j += 128) {
+        const int t = t_t * BT + j;
+        cf[j] = (t < M && ydt != BL_I32) ? dequant_factor(g, __ldg(scale + t)) : 0.0f;
+      }
+      const uint32_t ok_w = wait_warp(accf + a, (tc >> 1) & 1, limit, abort_flag) ? 1u : 0u;
+      // the four epilogue warps agree (and see each other's factors) before going on
+      uint32_t ok_all;
+      asm volatile(
+          "{\n\t.reg .pred pi, po;\n\t"
+          "setp.ne.u32 pi, %1, 0;\n\t"
+          "bar.red.and.pred po, 1, 128, pi;\n\t"
+          "selp.u32 %0, 1, 0, po;\n\t}"
+          : "=r"(ok_all)
+          : "r"(ok_w)
+          : "memory");
+      if (!ok_all) {
+        if (!ok_w && lane == 0) fail(0x501);
         break;
       }
       tc_fence_after();
-      const int n_t = tile % n_tiles, t_t = tile / n_tiles;
-      const int n = n_t * kBN + 32 * q + lane;
 #pragma unroll 1
       for (int j0 = 0; j0 < BT; j0 += Cfg::kChunk) {
         uint32_t acc[Cfg::kChunk];
@@ -372,7 +323,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (ydt == BL_I32) {
               static_cast<int32_t*>(y)[o] = v;
             } else {
-              const float yv = __fmul_rn(__int2float_rn(v), dequant_factor(g, __ldg(scale + t)));
+              const float yv = __fmul_rn(__int2float_rn(v), cf[j0 + j]);
               if (ydt == BL_F32)
                 static_cast<float*>(y)[o] = yv;
               else

@@ -20,9 +20,9 @@
 
 namespace bl {
 
-constexpr int kGemvThreads = 512;
+constexpr int kGemvThreads = 256;
 constexpr int kGemvWarps = kGemvThreads / 32;
-constexpr int kGemvU = 4;  // 16-byte segments per lane per pass
+constexpr int kGemvDepth = 4;  // row-block items whose loads are in flight per warp
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   uint4 v;
@@ -46,37 +46,74 @@ __device__ __forceinline__ float load_x(const void* x, int64_t i) {
   }
 }
 
+// Shared activation layout (per token), chosen so that the 32 lanes of a warp,
+// which work on 32 consecutive 16-byte segments s of a row, read consecutive
+// shared words (no bank conflicts):
+//   2-bit:  segment s, packed word w (0..3): 16 bytes at ((w * segs) + s) * 16,
+//           byte 4j + b = x[64 s + 16 w + 4 b + j]  (the digit order of the word)
+//   base 3: segment s, packed byte wb = 4 w + b: 8 bytes at ((wb * segs) + s) * 8,
+//           {x[5 p], .., x[5 p + 3]} and {x[5 p + 4], 0, 0, 0}, p = 16 s + wb
+__device__ __forceinline__ uint32_t x_slot(int fmt, uint32_t k, uint32_t segs) {  // k < 2^20
+  if (fmt == BL_PACK_I2) {
+    const uint32_t g = k >> 4, r = k & 15;            // packed word g, digit r
+    const uint32_t s = g >> 2, w = g & 3, j = r & 3, b = r >> 2;
+    return ((w * segs) + s) * 16 + 4 * j + b;
+  } else {
+    const uint32_t p = k / 5, i = k - 5 * p;          // packed byte p, digit i
+    const uint32_t s = p >> 4, wb = p & 15;
+    return ((wb * segs) + s) * 8 + (i < 4 ? i : 4);
+  }
+}
+
 template <int FMT, int MT, int XDT>
-__global__ void __launch_bounds__(kGemvThreads, 1)
+__global__ void __launch_bounds__(kGemvThreads, 3)
     gemv_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
                 int64_t N, int64_t K, const void* __restrict__ x, float* __restrict__ scale,
                 void* __restrict__ y, int ydt, int write_scale) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int64_t xb = gemv_x_bytes(FMT, rowbytes);
-  uint8_t* xs = smem;                                           // [MT][xb]
-  uint2* lut = reinterpret_cast<uint2*>(smem + MT * xb);        // base 3 only
-  __shared__ float red_f[kGemvWarps][MT];
-  __shared__ int red_i[kGemvWarps][MT];
-  __shared__ float s_tok[MT];
-  __shared__ int sum_tok[MT];
+  uint8_t* xs = smem;                                     // [MT][xb]
+  uint2* lut = reinterpret_cast<uint2*>(smem + MT * xb);  // base 3 only
+  __shared__ float red_f[MT][kGemvWarps];
+  __shared__ int red_i[MT][kGemvWarps];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t segs = rowbytes >> 4;
+  const uint32_t segs = static_cast<uint32_t>(rowbytes >> 4);
+  const uint32_t nb = (segs + 31) >> 5;  // 32-segment blocks per row
   const int64_t TW = static_cast<int64_t>(gridDim.x) * kGemvWarps;
-  int64_t r = static_cast<int64_t>(blockIdx.x) * kGemvWarps + warp;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kGemvWarps + warp;
+  const int64_t nrows = r0 < N ? (N - 1 - r0) / TW + 1 : 0;
 
-  // 1. first packed loads of this warp's first row go out before the prologue.
-  uint4 pre[kGemvU];
-  if (r < N) {
-    const uint4* rp = reinterpret_cast<const uint4*>(packed + r * rowbytes);
-#pragma unroll
-    for (int u = 0; u < kGemvU; ++u) {
-      const int64_t s = lane + 32 * u;
-      if (s < segs) pre[u] = ld_stream(rp + s);
+  // The warp's items are (row r0 + ri TW, 32-segment block blk), in order;
+  // the lane's segment of an item is 32 blk + lane.  Two cursors walk them:
+  // one for the loads in flight, one for the item being reduced.
+  int64_t l_ri = 0;
+  uint32_t l_blk = 0;
+  const uint8_t* l_row = packed + r0 * rowbytes;
+  auto load_next = [&](uint4& dst) {
+    const uint32_t s = 32 * l_blk + lane;
+    if (s < segs) dst = ld_stream(reinterpret_cast<const uint4*>(l_row) + s);
+    if (++l_blk == nb) {
+      l_blk = 0;
+      ++l_ri;
+      l_row += TW * rowbytes;
     }
+  };
+
+  // 1. the first kGemvDepth items' loads go out before the prologue
+  uint4 buf[kGemvDepth];
+#pragma unroll
+  for (int d = 0; d < kGemvDepth; ++d) {
+    buf[d] = make_uint4(0, 0, 0, 0);
+    if (l_ri < nrows) load_next(buf[d]);
   }
 
-  // 2. prologue: quantize the MT tokens into shared memory.
+  // 2. prologue: zero the activation area, per-token absmax, then scatter the
+  //    INT8 codes into the layout above.
+  {
+    uint4* z = reinterpret_cast<uint4*>(xs);
+    for (int64_t i = threadIdx.x; i < MT * xb / 16; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
+  }
   if constexpr (FMT == BL_PACK_T5) {
     for (int b = threadIdx.x; b < 256; b += blockDim.x) {
       uint32_t lo = 0, hi = 0;
@@ -93,123 +130,102 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
       lut[b] = make_uint2(lo, hi);
     }
   }
-  // one "group" = the activations of one packed 32-bit word: 16 weights (2-bit)
-  // or 20 weights (base 3)
-  constexpr int GW = (FMT == BL_PACK_I2) ? 16 : 20;
-  const int64_t groups = rowbytes / 4;
+  const bool vec = (K % 8) == 0;
+  float s_tok[MT];
+  if constexpr (XDT != BL_I8) {
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      float amax = 0.0f;
+      if (vec) {
+        for (int64_t v = threadIdx.x; v < K / 8; v += blockDim.x) {
+          float e[8];
+          load8_aligned<XDT>(x, m * K + 8 * v, e);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(e[j]));
+        }
+      } else {
+        for (int64_t k = threadIdx.x; k < K; k += blockDim.x) amax = fmaxf(amax, fabsf(load_x<XDT>(x, m * K + k)));
+      }
+      amax = warp_maxf(amax);
+      if (lane == 0) red_f[m][warp] = amax;
+    }
+  }
+  __syncthreads();  // zeroed activations, table and per-warp maxima are visible
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
-    float s;
     if constexpr (XDT != BL_I8) {
-      float amax = 0.0f;
-      for (int64_t k = threadIdx.x; k < K; k += blockDim.x)
-        amax = fmaxf(amax, fabsf(load_x<XDT>(x, m * K + k)));
-      amax = warp_maxf(amax);
-      if (lane == 0) red_f[warp][m] = amax;
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        float a = red_f[0][m];
-        for (int w = 1; w < kGemvWarps; ++w) a = fmaxf(a, red_f[w][m]);
-        s_tok[m] = fmaxf(a, 1e-6f);
-      }
-      __syncthreads();
-      s = s_tok[m];
+      float a = red_f[m][0];
+#pragma unroll
+      for (int w = 1; w < kGemvWarps; ++w) a = fmaxf(a, red_f[m][w]);
+      s_tok[m] = fmaxf(a, 1e-6f);
     } else {
-      s = 0.0f;
+      s_tok[m] = __ldg(scale + m);
     }
+  }
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
     int part = 0;
-    for (int64_t g = threadIdx.x; g < groups; g += blockDim.x) {
-      int q[GW];
+    uint8_t* xm = xs + m * xb;
+    const float c127 = (XDT == BL_I8) ? 0.0f : __fdiv_rn(127.0f, s_tok[m]);
+    if (vec) {
+      for (int64_t v = threadIdx.x; v < K / 8; v += blockDim.x) {
+        int q[8];
+        if constexpr (XDT == BL_I8) {
+          const uint2 raw = __ldg(reinterpret_cast<const uint2*>(static_cast<const int8_t*>(x) + m * K + 8 * v));
 #pragma unroll
-      for (int i = 0; i < GW; ++i) {
-        const int64_t k = g * GW + i;
-        if (k < K) {
-          if constexpr (XDT == BL_I8)
-            q[i] = static_cast<const int8_t*>(x)[m * K + k];
-          else
-            q[i] = quant_act(load_x<XDT>(x, m * K + k), s);
+          for (int j = 0; j < 8; ++j) q[j] = static_cast<int8_t>((j < 4 ? raw.x : raw.y) >> (8 * (j & 3)));
         } else {
-          q[i] = 0;
+          float e[8];
+          load8_aligned<XDT>(x, m * K + 8 * v, e);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) q[j] = quant_act_fast(e[j], s_tok[m], c127);
         }
-        part += q[i];
-      }
-      if constexpr (FMT == BL_PACK_I2) {
-        // word j holds x[16g + j + 4b] in byte b
-        uint32_t w4[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          w4[j] = (static_cast<uint32_t>(q[j] & 0xff)) | (static_cast<uint32_t>(q[j + 4] & 0xff) << 8) |
-                  (static_cast<uint32_t>(q[j + 8] & 0xff) << 16) |
-                  (static_cast<uint32_t>(q[j + 12] & 0xff) << 24);
-        reinterpret_cast<uint4*>(xs + m * xb)[g] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-      } else {
-        // byte j of the word: {x[5j..5j+3]} and {x[5j+4], 0, 0, 0}
-        uint2* dst = reinterpret_cast<uint2*>(xs + m * xb) + 4 * g;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const int* qq = q + 5 * b;
-          const uint32_t lo = (static_cast<uint32_t>(qq[0] & 0xff)) | (static_cast<uint32_t>(qq[1] & 0xff) << 8) |
-                              (static_cast<uint32_t>(qq[2] & 0xff) << 16) |
-                              (static_cast<uint32_t>(qq[3] & 0xff) << 24);
-          dst[b] = make_uint2(lo, static_cast<uint32_t>(qq[4] & 0xff));
+        for (int j = 0; j < 8; ++j) {
+          xm[x_slot(FMT, static_cast<uint32_t>(8 * v + j), segs)] = static_cast<uint8_t>(q[j]);
+          part += q[j];
         }
       }
-    }
-    if constexpr (FMT == BL_PACK_I2) {
-      part = __reduce_add_sync(0xffffffffu, part);
-      if (lane == 0) red_i[warp][m] = part;
-    }
-    if constexpr (XDT == BL_I8) {
-      if (threadIdx.x == 0) s_tok[m] = scale[m];
-    }
-  }
-  __syncthreads();
-  if (threadIdx.x < MT) {
-    const int m = threadIdx.x;
-    if constexpr (FMT == BL_PACK_I2) {
-      int t = 0;
-      for (int w = 0; w < kGemvWarps; ++w) t += red_i[w][m];
-      sum_tok[m] = t;
     } else {
-      sum_tok[m] = 0;
+      for (int64_t k = threadIdx.x; k < K; k += blockDim.x) {
+        const int q = (XDT == BL_I8) ? static_cast<int>(static_cast<const int8_t*>(x)[m * K + k])
+                                     : quant_act_fast(load_x<XDT>(x, m * K + k), s_tok[m], c127);
+        xm[x_slot(FMT, static_cast<uint32_t>(k), segs)] = static_cast<uint8_t>(q);
+        part += q;
+      }
     }
-    if (XDT != BL_I8 && write_scale && blockIdx.x == 0) scale[m] = s_tok[m];
+    part = __reduce_add_sync(0xffffffffu, part);
+    if (lane == 0) red_i[m][warp] = part;
   }
-  __syncthreads();
-
+  __syncthreads();  // activations and per-warp sums are visible
   const float g = __ldg(gamma);
   float cfac[MT];
   int corr[MT];
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
+    int t = 0;
+#pragma unroll
+    for (int w = 0; w < kGemvWarps; ++w) t += red_i[m][w];
+    corr[m] = (FMT == BL_PACK_I2) ? t : 0;  // 2-bit digits are q + 1: subtract sum x once
     cfac[m] = dequant_factor(g, s_tok[m]);
-    corr[m] = sum_tok[m];
+    if (XDT != BL_I8 && write_scale && blockIdx.x == 0 && threadIdx.x == 0) scale[m] = s_tok[m];
   }
 
-  // 3. rows: warp-per-row, lanes stride over the row's 16-byte segments.
-  bool first = true;
-  for (; r < N; r += TW) {
-    const uint4* rp = reinterpret_cast<const uint4*>(packed + r * rowbytes);
-    int acc[MT];
+  // 3. stream the items, kGemvDepth loads always in flight.
+  int acc[MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m] = 0;
-    for (int64_t s0 = 0; s0 < segs; s0 += 32 * kGemvU) {
-      uint4 buf[kGemvU];
-      if (first && s0 == 0) {
+  for (int m = 0; m < MT; ++m) acc[m] = 0;
+  int64_t c_ri = 0;
+  uint32_t c_blk = 0;
+  while (c_ri < nrows) {
 #pragma unroll
-        for (int u = 0; u < kGemvU; ++u) buf[u] = pre[u];
-      } else {
-#pragma unroll
-        for (int u = 0; u < kGemvU; ++u) {
-          const int64_t s = s0 + lane + 32 * u;
-          if (s < segs) buf[u] = ld_stream(rp + s);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kGemvU; ++u) {
-        const int64_t s = s0 + lane + 32 * u;
-        if (s >= segs) break;
-        const uint32_t wd[4] = {buf[u].x, buf[u].y, buf[u].z, buf[u].w};
+    for (int d = 0; d < kGemvDepth; ++d) {
+      if (c_ri >= nrows) break;
+      const uint4 cur = buf[d];
+      if (l_ri < nrows) load_next(buf[d]);
+      const uint32_t s = 32 * c_blk + lane;
+      if (s < segs) {
+        const uint32_t wd[4] = {cur.x, cur.y, cur.z, cur.w};
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
           if constexpr (FMT == BL_PACK_I2) {
@@ -217,7 +233,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
             const uint32_t c2 = (wd[w] >> 4) & 0x03030303u, c3 = (wd[w] >> 6) & 0x03030303u;
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
-              const uint4 X = reinterpret_cast<const uint4*>(xs + m * xb)[4 * s + w];
+              const uint4 X = *reinterpret_cast<const uint4*>(xs + m * xb + ((w * segs) + s) * 16);
               acc[m] = __dp4a(static_cast<int>(c0), static_cast<int>(X.x), acc[m]);
               acc[m] = __dp4a(static_cast<int>(c1), static_cast<int>(X.y), acc[m]);
               acc[m] = __dp4a(static_cast<int>(c2), static_cast<int>(X.z), acc[m]);
@@ -226,32 +242,37 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
           } else {
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
-              const uint2 L = lut[(wd[w] >> (8 * b)) & 0xffu];
+              const uint2 Lw = lut[(wd[w] >> (8 * b)) & 0xffu];
 #pragma unroll
               for (int m = 0; m < MT; ++m) {
-                const uint2 X = reinterpret_cast<const uint2*>(xs + m * xb)[16 * s + 4 * w + b];
-                acc[m] = __dp4a(static_cast<int>(L.x), static_cast<int>(X.x), acc[m]);
-                acc[m] = __dp4a(static_cast<int>(L.y), static_cast<int>(X.y), acc[m]);
+                const uint2 X = *reinterpret_cast<const uint2*>(xs + m * xb + (((4 * w + b) * segs) + s) * 8);
+                acc[m] = __dp4a(static_cast<int>(Lw.x), static_cast<int>(X.x), acc[m]);
+                acc[m] = __dp4a(static_cast<int>(Lw.y), static_cast<int>(X.y), acc[m]);
               }
             }
           }
         }
       }
-    }
-    first = false;
+      if (c_blk == nb - 1) {  // the row is complete: reduce, dequantize, store
+        const int64_t r = r0 + c_ri * TW;
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m] = __reduce_add_sync(0xffffffffu, acc[m]);
-    if (lane == 0) {
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        const int a = acc[m] - corr[m];
-        const int64_t o = m * N + r;
-        if (ydt == BL_I32)
-          static_cast<int32_t*>(y)[o] = a;
-        else if (ydt == BL_F32)
-          static_cast<float*>(y)[o] = __fmul_rn(__int2float_rn(a), cfac[m]);
-        else
-          static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(a), cfac[m]));
+        for (int m = 0; m < MT; ++m) {
+          const int a = __reduce_add_sync(0xffffffffu, acc[m]) - corr[m];
+          acc[m] = 0;
+          if (lane == 0) {
+            const int64_t o = m * N + r;
+            if (ydt == BL_I32)
+              static_cast<int32_t*>(y)[o] = a;
+            else if (ydt == BL_F32)
+              static_cast<float*>(y)[o] = __fmul_rn(__int2float_rn(a), cfac[m]);
+            else
+              static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(a), cfac[m]));
+          }
+        }
+        c_blk = 0;
+        ++c_ri;
+      } else {
+        ++c_blk;
       }
     }
   }

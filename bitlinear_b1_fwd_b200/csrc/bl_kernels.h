@@ -21,8 +21,10 @@ constexpr int kGemvMaxTokens = 4;
 // ws: a workspace whose header ticket is zero; partial sums follow the header.
 cudaError_t launch_absmean(const void* W, int wdt, int64_t N, int64_t K, void* ws, float* gamma,
                            cudaStream_t st);
+// ws: a workspace header for device flags, or nullptr (then a bounded wait
+// that runs out goes unreported).
 cudaError_t launch_ternarize_pack(const void* W, int wdt, int64_t N, int64_t K, const float* gamma,
-                                  float eps, int fmt, uint8_t* packed, int8_t* codes, int64_t rowbytes,
+                                  float eps, int fmt, uint8_t* packed, int8_t* codes, int64_t rowbytes, void* ws,
                                   cudaStream_t st);
 cudaError_t launch_pack(const int8_t* codes, int64_t N, int64_t K, int fmt, uint8_t* packed,
                         int64_t rowbytes, void* ws, cudaStream_t st);

@@ -283,3 +283,44 @@ def test_misaligned_pointer_rejected():
     with pytest.raises(B.BitLinearError) as e:
         B.bitlinear_quantize_acts(x[1:33].view(1, 32), xq[:32].view(1, 32), s[:1])
     assert e.value.status == B.BL_ERR_MISALIGNED
+
+
+def test_quantize_acts_near_ties(orc):
+    """Entries whose quotient x / s * 127 lands within a few fp32 ulps of a
+    half-integer, at several token scales: the cases the kernel settles with
+    the exact quotient.  Both the standalone quantizer and the GEMV prologue."""
+    rows = []
+    for smax in (1.0, 3.7, 0.013, 250.0, 1e-6):
+        xs = [np.float32(smax)]
+        for t in (0.5, 1.5, 2.5, 63.5, 100.5, 126.5):
+            v0 = np.float32(t / 127.0 * smax)
+            up, dn = v0, v0
+            xs += [v0, -v0]
+            for _ in range(12):
+                up = np.nextafter(up, np.float32(np.inf))
+                dn = np.nextafter(dn, np.float32(0))
+                xs += [up, -up, dn, -dn]
+        rows.append(xs)
+    width = max(len(r) for r in rows)
+    width += (-width) % 16
+    x = np.zeros((len(rows), width), np.float32)
+    for i, r in enumerate(rows):
+        x[i, :len(r)] = r
+    xq_ref, s_ref = orc.act_quant(x)
+    xd = dev(x)
+    xq = torch.empty(x.shape, dtype=torch.int8, device="cuda")
+    s = torch.empty(x.shape[0], dtype=torch.float32, device="cuda")
+    B.bitlinear_quantize_acts(xd, xq, s)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(xq), xq_ref)
+    assert np.array_equal(host(s), s_ref)
+    # the decode path quantizes in its prologue: an identity-like weight matrix
+    # (row n has +1 at column n) makes y[:, n] = x_q[:, n] for n < K
+    K = x.shape[1]
+    codes = np.zeros((K, K), np.int8)
+    np.fill_diagonal(codes, 1)
+    packed = orc.pack(codes, I2)
+    for m in range(x.shape[0]):
+        y, sm = forward(packed, I2, np.float32(1.0), K, K, x[m:m + 1], B.BL_I32)
+        assert np.array_equal(y[0], xq_ref[m].astype(np.int32))
+        assert sm[0] == s_ref[m]
