@@ -347,6 +347,263 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Two-SM variant for many tokens.  A cluster of two CTAs computes a tile of
+// 256 weight rows x BT tokens with tcgen05.mma.cta_group::2 (M = 256): CTA r
+// stages its own 128 weight rows and tokens r BT/2 .. (r+1) BT/2 - 1, so per
+// SM the staged bytes per MAC fall to about 2/3 of the one-SM tile and six
+// stages fit.  Each CTA's accumulator in tensor memory holds its 128 rows x BT
+// tokens.  The leader (rank 0) issues the MMAs; the x loads of both CTAs count
+// on the leader's barrier, the packed loads on the local one (the expansion
+// warps of each CTA wait there), and the expansion and epilogue warps of both
+// CTAs report to the leader by remote arrives.  MMA completion is committed to
+// the barriers of both CTAs.  Every wait is bounded as in the one-SM kernel.
+// ---------------------------------------------------------------------------
+constexpr int kStages2 = 6;
+
+template <int BT>
+struct Gemm2Cfg {
+  static constexpr uint32_t kXHalf = (BT / 2) * 128;
+  static constexpr uint32_t kTmemCols = 2 * BT;  // BT >= 128: a power of two
+  static constexpr size_t kSmem =
+      1024 + kStages2 * (kXHalf + kExpStage + kPackedStage) + 8 * (4 * kStages2 + 5) + 16 + 2 * 4 * BT;
+};
+
+__device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// arrive on the barrier at this offset in each CTA of `mask` when the MMAs
+// issued so far complete
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
+template <int BT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_i2_2sm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                       const float* __restrict__ gamma, const float* __restrict__ scale, void* __restrict__ y,
+                       int ydt, int M, int N, int K, WsHeader* __restrict__ hdr, long long limit) {
+  using Cfg = Gemm2Cfg<BT>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* base = smem_raw + pad;
+  uint8_t* xs = base;                              // kStages2 x [BT/2 x 128 B], swizzled
+  uint8_t* es = xs + kStages2 * Cfg::kXHalf;       // kStages2 x [128 x 128 B], swizzled
+  uint8_t* ps = es + kStages2 * kExpStage;         // kStages2 x [128 x 32 B]
+  uint64_t* xfull = reinterpret_cast<uint64_t*>(ps + kStages2 * kPackedStage);  // leader: x of both CTAs
+  uint64_t* pfull = xfull + kStages2;              // local: packed tile
+  uint64_t* expd = pfull + kStages2;               // leader: expansion of both CTAs (8 warps)
+  uint64_t* empty = expd + kStages2;               // local: the MMAs read the stage
+  uint64_t* accf = empty + kStages2;               // local: accumulator ready (2)
+  uint64_t* acce = accf + 2;                       // leader: epilogues of both CTAs done (2)
+  uint64_t* drain = acce + 2;                      // leader
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* cfac = reinterpret_cast<float*>(tmem_slot + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int kblocks = (K + kBK - 1) / kBK;
+  const int n_tiles = (N + 2 * kBN - 1) / (2 * kBN);
+  const int t_tiles = (M + BT - 1) / BT;
+  const int tiles = n_tiles * t_tiles;
+  const int pair = blockIdx.x >> 1, pairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages2; ++s) {
+      mbar_init(xfull + s, 1);
+      mbar_init(pfull + s, 1);
+      mbar_init(expd + s, 8);
+      mbar_init(empty + s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(accf + a, 1);
+      mbar_init(acce + a, 8);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(Cfg::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers exist before any remote arrive or copy
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto fail = [&](uint32_t site) {
+    set_flag(hdr, kFlagTimeout, site);
+    *abort_flag = 1;
+  };
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer (both CTAs) ------------------
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = pair; tile < tiles && ok; tile += pairs) {
+        const int n_t = tile % n_tiles, t_t = tile / n_tiles;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % kStages2;
+          const uint32_t ph = (it / kStages2) & 1;
+          if (!wait1(empty + s, ph ^ 1, limit, abort_flag)) {
+            fail(0x211);
+            ok = false;
+            break;
+          }
+          if (leader) mbar_expect_tx(xfull + s, 2 * Cfg::kXHalf);
+          mbar_expect_tx(pfull + s, kPackedStage);
+          tma_load_2d_pair(xs + s * Cfg::kXHalf, &tm_x, mapa_shared(smem_u32(xfull + s), 0), kb * kBK,
+                           t_t * BT + static_cast<int>(rank) * (BT / 2));
+          tma_load_2d(ps + s * kPackedStage, &tm_w, pfull + s, kb * (kBK / 4),
+                      n_t * 2 * kBN + static_cast<int>(rank) * kBN);
+        }
+      }
+      for (int j = (it > kStages2 ? it - kStages2 : 0); j < it; ++j)
+        (void)wait_drain(pfull + (j % kStages2), (j / kStages2) & 1, limit);
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer (leader) -------------------------
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = i8_idesc(2 * kBN, BT);
+      int it = 0, tc = 0;
+      bool ok = true;
+      for (int tile = pair; tile < tiles && ok; tile += pairs, ++tc) {
+        const int a = tc & 1;
+        if (!wait1(acce + a, ((tc >> 1) & 1) ^ 1, limit, abort_flag)) {
+          fail(0x311);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + static_cast<uint32_t>(a * BT);
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % kStages2;
+          const uint32_t ph = (it / kStages2) & 1;
+          if (!wait1(xfull + s, ph, limit, abort_flag) || !wait1(expd + s, ph, limit, abort_flag)) {
+            fail(0x312);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t xa = smem_u32(xs + s * Cfg::kXHalf), ea = smem_u32(es + s * kExpStage);
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k)
+            mma_i8_pair(d, sw128_desc(ea + 32 * k), sw128_desc(xa + 32 * k), idesc, (kb | k) != 0);
+          mma_commit_pair(empty + s, 0x3);
+        }
+        if (ok) mma_commit_pair(accf + a, 0x3);
+      }
+      mma_commit_pair(drain, 0x1);
+      (void)wait_drain(drain, 0, limit);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------ expansion (both CTAs) -----------------------
+    const int r = threadIdx.x - 128;
+    int it = 0;
+    bool ok = true;
+    for (int tile = pair; tile < tiles && ok; tile += pairs) {
+      for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        const int s = it % kStages2;
+        const uint32_t ph = (it / kStages2) & 1;
+        if (!wait_warp(pfull + s, ph, limit, abort_flag)) {
+          if (lane == 0) fail(0x411);
+          ok = false;
+          break;
+        }
+        const uint4* src = reinterpret_cast<const uint4*>(ps + s * kPackedStage + r * 32);
+        const uint4 p0 = src[0], p1 = src[1];
+        const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+        uint8_t* row = es + s * kExpStage + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(row + ((j ^ (r & 7)) << 4)) = expand16(w[j]);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(expd + s), 0));
+      }
+    }
+  } else if (warp >= 8) {
+    // ------------------------------ epilogue (both CTAs) ------------------------
+    const int q = warp & 3;
+    const float g = __ldg(gamma);
+    int tc = 0;
+    for (int tile = pair; tile < tiles; tile += pairs, ++tc) {
+      const int a = tc & 1;
+      const int n_t = tile % n_tiles, t_t = tile / n_tiles;
+      const int n = n_t * 2 * kBN + static_cast<int>(rank) * kBN + 32 * q + lane;
+      float* cf = cfac + a * BT;
+      for (int j = threadIdx.x - 256; j < BT; j += 128) {
+        const int t = t_t * BT + j;
+        cf[j] = (t < M && ydt != BL_I32) ? dequant_factor(g, __ldg(scale + t)) : 0.0f;
+      }
+      const uint32_t ok_w = wait_warp(accf + a, (tc >> 1) & 1, limit, abort_flag) ? 1u : 0u;
+      uint32_t ok_all;
+      asm volatile(
+          "{\n\t.reg .pred pi, po;\n\t"
+          "setp.ne.u32 pi, %1, 0;\n\t"
+          "bar.red.and.pred po, 1, 128, pi;\n\t"
+          "selp.u32 %0, 1, 0, po;\n\t}"
+          : "=r"(ok_all)
+          : "r"(ok_w)
+          : "memory");
+      if (!ok_all) {
+        if (!ok_w && lane == 0) fail(0x511);
+        break;
+      }
+      tc_fence_after();
+#pragma unroll 1
+      for (int j0 = 0; j0 < BT; j0 += 32) {
+        uint32_t acc[32];
+        tmem_load<32>(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(a * BT + j0), acc);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int t = t_t * BT + j0 + j;
+          if (t < M && n < N) {
+            const int64_t o = static_cast<int64_t>(t) * N + n;
+            const int v = static_cast<int>(acc[j]);
+            if (ydt == BL_I32) {
+              static_cast<int32_t*>(y)[o] = v;
+            } else {
+              const float yv = __fmul_rn(__int2float_rn(v), cf[j0 + j]);
+              if (ydt == BL_F32)
+                static_cast<float*>(y)[o] = yv;
+              else
+                static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(yv);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(acce + a), 0));
+    }
+  }
+
+  __syncthreads();
+  tc_fence_before();
+  cluster_sync_all();  // no CTA leaves while its peer may still signal its barriers
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(Cfg::kTmemCols)
+                 : "memory");
+  }
+}
+
 // T5 -> 2-bit transcoding (for the tensor-core path on base-3 weights): one
 // thread writes one 16-byte segment (64 weights) of a 2-bit row.  The base-3
 // digit of a weight is its 2-bit code (both are q + 1); invalid bytes (>= 243)
@@ -444,6 +701,31 @@ cudaError_t launch_gemm_bt(const int8_t* xq, const uint8_t* w, int64_t rb, const
   return cudaGetLastError();
 }
 
+template <int BT>
+cudaError_t launch_gemm_2sm(const int8_t* xq, const uint8_t* w, int64_t rb, const float* gamma, const float* scale,
+                            void* y, int ydt, int64_t M, int64_t N, int64_t K, void* ws, long long limit,
+                            cudaStream_t st) {
+  CUtensorMap tx, tw;
+  if (!encode_2d_u8(&tx, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(K), 128,
+                    BT / 2, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (!encode_2d_u8(&tw, w, static_cast<uint64_t>(rb), static_cast<uint64_t>(N), static_cast<uint64_t>(rb),
+                    kBK / 4, kBN, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  auto kern = gemm_i2_2sm_kernel<BT>;
+  const size_t smem = Gemm2Cfg<BT>::kSmem;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = ((N + 2 * kBN - 1) / (2 * kBN)) * ((M + BT - 1) / BT);
+  const int64_t pairs_max = device_sms() / 2;
+  const int64_t pairs = tiles < pairs_max ? tiles : pairs_max;
+  kern<<<static_cast<unsigned>(2 * pairs), kGemmThreads, smem, st>>>(tx, tw, gamma, scale, y, ydt,
+                                                                     static_cast<int>(M), static_cast<int>(N),
+                                                                     static_cast<int>(K), static_cast<WsHeader*>(ws),
+                                                                     limit);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 int gemm_token_tile(int64_t M) {
@@ -458,6 +740,8 @@ cudaError_t launch_gemm_i2(const int8_t* xq, const uint8_t* w, int64_t rb, const
                            void* y, int ydt, int64_t M, int64_t N, int64_t K, void* ws, long long limit_cycles,
                            int skip_producer, cudaStream_t st) {
   const long long limit = limit_cycles > 0 ? limit_cycles : kTimeoutCycles;
+  if (M > 128 && !skip_producer)
+    return launch_gemm_2sm<256>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ws, limit, st);
   switch (gemm_token_tile(M)) {
     case 16: return launch_gemm_bt<16>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ws, limit, skip_producer, st);
     case 32: return launch_gemm_bt<32>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ws, limit, skip_producer, st);

@@ -20,9 +20,9 @@
 
 namespace bl {
 
-constexpr int kGemvThreads = 256;
+constexpr int kGemvThreads = 768;  // one CTA per SM: the token prologue runs once per SM
 constexpr int kGemvWarps = kGemvThreads / 32;
-constexpr int kGemvDepth = 4;  // row-block items whose loads are in flight per warp
+constexpr int kGemvDepth = 6;  // row-block items whose loads are in flight per warp
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   uint4 v;
@@ -35,6 +35,13 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 // Activation bytes per token in shared memory for one packed row of rowbytes.
 __host__ __device__ inline int64_t gemv_x_bytes(int fmt, int64_t rowbytes) {
   return fmt == BL_PACK_I2 ? rowbytes * 4 : rowbytes * 8;
+}
+
+// dp4a with unsigned bytes in a and signed bytes in b.
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
 
 template <int XDT>
@@ -66,7 +73,7 @@ __device__ __forceinline__ uint32_t x_slot(int fmt, uint32_t k, uint32_t segs) {
 }
 
 template <int FMT, int MT, int XDT>
-__global__ void __launch_bounds__(kGemvThreads, 3)
+__global__ void __launch_bounds__(kGemvThreads, 1)
     gemv_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
                 int64_t N, int64_t K, const void* __restrict__ x, float* __restrict__ scale,
                 void* __restrict__ y, int ydt, int write_scale) {
@@ -211,10 +218,13 @@ __global__ void __launch_bounds__(kGemvThreads, 3)
     if (XDT != BL_I8 && write_scale && blockIdx.x == 0 && threadIdx.x == 0) scale[m] = s_tok[m];
   }
 
-  // 3. stream the items, kGemvDepth loads always in flight.
-  int acc[MT];
+  // 3. stream the items, kGemvDepth loads always in flight.  2-bit: the digit
+  //    of weight position j of each byte is taken in place, w & (3 << 2j), so
+  //    each byte holds d 4^j; accumulator j collects 4^j sum d x, and the
+  //    factor comes off exactly at the end of the row.
+  int acc[MT], acc1[MT], acc2[MT], acc3[MT];
 #pragma unroll
-  for (int m = 0; m < MT; ++m) acc[m] = 0;
+  for (int m = 0; m < MT; ++m) acc[m] = acc1[m] = acc2[m] = acc3[m] = 0;
   int64_t c_ri = 0;
   uint32_t c_blk = 0;
   while (c_ri < nrows) {
@@ -228,7 +238,15 @@ __global__ void __launch_bounds__(kGemvThreads, 3)
         const uint32_t wd[4] = {cur.x, cur.y, cur.z, cur.w};
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-          if constexpr (FMT == BL_PACK_I2) {
+          if constexpr (FMT == BL_PACK_I2 && MT == 1) {
+            const uint32_t c0 = wd[w] & 0x03030303u, c1 = wd[w] & 0x0c0c0c0cu;
+            const uint32_t c2 = wd[w] & 0x30303030u, c3 = wd[w] & 0xc0c0c0c0u;
+            const uint4 X = *reinterpret_cast<const uint4*>(xs + ((w * segs) + s) * 16);
+            acc[0] = dp4a_us(c0, X.x, acc[0]);
+            acc1[0] = dp4a_us(c1, X.y, acc1[0]);
+            acc2[0] = dp4a_us(c2, X.z, acc2[0]);
+            acc3[0] = dp4a_us(c3, X.w, acc3[0]);
+          } else if constexpr (FMT == BL_PACK_I2) {  // several tokens: digits shifted down once
             const uint32_t c0 = wd[w] & 0x03030303u, c1 = (wd[w] >> 2) & 0x03030303u;
             const uint32_t c2 = (wd[w] >> 4) & 0x03030303u, c3 = (wd[w] >> 6) & 0x03030303u;
 #pragma unroll
@@ -257,8 +275,9 @@ __global__ void __launch_bounds__(kGemvThreads, 3)
         const int64_t r = r0 + c_ri * TW;
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-          const int a = __reduce_add_sync(0xffffffffu, acc[m]) - corr[m];
-          acc[m] = 0;
+          const int lane_sum = acc[m] + (acc1[m] >> 2) + (acc2[m] >> 4) + (acc3[m] >> 6);
+          const int a = __reduce_add_sync(0xffffffffu, lane_sum) - corr[m];
+          acc[m] = acc1[m] = acc2[m] = acc3[m] = 0;
           if (lane == 0) {
             const int64_t o = m * N + r;
             if (ydt == BL_I32)

@@ -119,6 +119,40 @@ __device__ __forceinline__ double chunk_sum_smem(const uint8_t* stage, int L) {
   return t;
 }
 
+// Part of the fixed-order chunk sum done by one of four warps: lanes
+// l = L + 32 v for v in {sub, sub + 4}, summed in order and combined at tree
+// level 128 (v with v + 4), giving p'[sub].
+template <int WDT>
+__device__ __forceinline__ double chunk_part_smem(const uint8_t* stage, int L, int sub) {
+  constexpr int ES = (WDT == BL_F32) ? 4 : 2;
+  double p[2] = {0.0, 0.0};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int v = sub + 4 * h;
+#pragma unroll 2
+    for (int i = 0; i < 4; ++i) {
+      float x[8];
+      const uint8_t* src = stage + (2048 * i + 256 * v + 8 * L) * ES;
+      if constexpr (WDT == BL_F32) {
+        const float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 16);
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+      } else {
+        const uint4 a = *reinterpret_cast<const uint4*>(src);
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          x[2 * k] = __uint_as_float(w[k] << 16);
+          x[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) p[h] = __dadd_rn(p[h], static_cast<double>(fabsf(x[j])));
+    }
+  }
+  return __dadd_rn(p[0], p[1]);  // level 128
+}
+
 // Bulk-staged absmean: one persistent CTA per SM.  A producer thread keeps
 // kBulkStages whole chunks in flight with cp.async.bulk (global -> shared);
 // consumer warp w owns stage w: it reduces the chunks j = w, w + S, w + 2S, ...
@@ -129,7 +163,8 @@ __device__ __forceinline__ double chunk_sum_smem(const uint8_t* stage, int L) {
 // directly from global memory.  All waits are bounded; on expiry the timeout
 // flag is set and gamma is not meaningful.
 constexpr int kBulkStages = 6;
-constexpr int kBulkConsumers = kBulkStages;
+constexpr int kAbsWarpsPerStage = 4;
+constexpr int kBulkConsumers = kBulkStages * kAbsWarpsPerStage;
 constexpr int kBulkThreads = 32 * (kBulkConsumers + 1);
 constexpr long long kBulkWaitCycles = 1ll << 32;
 constexpr int kTernConsumers = kBulkStages;  // one consumer warp per stage, as above
@@ -145,6 +180,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1)
   uint64_t* empty = full + kBulkStages;
   __shared__ int abort_flag;
   __shared__ double p[kLanes];
+  __shared__ double xchg[kBulkStages][kAbsWarpsPerStage][32];
   __shared__ bool last;
   const int warp = threadIdx.x >> 5, L = threadIdx.x & 31;
   const int64_t G = gridDim.x, b = blockIdx.x;
@@ -173,22 +209,42 @@ __global__ void __launch_bounds__(kBulkThreads, 1)
       }
     }
   } else {
-    for (int64_t j = warp; b + j * G < Cfull; j += kBulkConsumers) {
-      const int s = static_cast<int>(j % kBulkStages);
+    // consumer group s (warps 4s .. 4s + 3) owns stage s
+    const int s = warp / kAbsWarpsPerStage, sub = warp % kAbsWarpsPerStage;
+    for (int64_t j = s; b + j * G < Cfull; j += kBulkStages) {
       const uint32_t ph = static_cast<uint32_t>((j / kBulkStages) & 1);
-      if (!wait_warp(full + s, ph, kBulkWaitCycles, abort_v)) {
+      const bool okw = wait_warp(full + s, ph, kBulkWaitCycles, abort_v);
+      if (!okw && L == 0) {
+        set_flag(hdr, kFlagTimeout, 0x602);
+        *abort_v = 1;
+      }
+      const double part = okw ? chunk_part_smem<WDT>(smem + s * CB, L, sub) : 0.0;
+      xchg[s][sub][L] = part;
+      // the four warps of the group meet here and agree whether to go on
+      uint32_t ok_all;
+      asm volatile(
+          "{\n\t.reg .pred pi, po;\n\t"
+          "setp.ne.u32 pi, %1, 0;\n\t"
+          "bar.red.and.pred po, %2, %3, pi;\n\t"
+          "selp.u32 %0, 1, 0, po;\n\t}"
+          : "=r"(ok_all)
+          : "r"(okw ? 1u : 0u), "r"(1 + s), "n"(32 * kAbsWarpsPerStage)
+          : "memory");
+      const bool ok = ok_all != 0;
+      if (sub == 0) {
+        double q0 = xchg[s][0][L], q1 = xchg[s][1][L];
+        const double q2 = xchg[s][2][L], q3 = xchg[s][3][L];
+        q0 = __dadd_rn(q0, q2);  // level 64
+        q1 = __dadd_rn(q1, q3);
+        double t = __dadd_rn(q0, q1);  // level 32
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) t = __dadd_rn(t, __shfl_down_sync(0xffffffffu, t, o));
         if (L == 0) {
-          set_flag(hdr, kFlagTimeout, 0x602);
-          *abort_v = 1;
+          if (ok) partials[b + j * G] = t;
+          mbar_arrive(empty + s);  // the whole group has read the stage and the exchange slots
         }
-        break;
       }
-      const double t = chunk_sum_smem<WDT>(smem + s * CB, L);
-      __syncwarp();
-      if (L == 0) {
-        partials[b + j * G] = t;
-        mbar_arrive(empty + s);
-      }
+      if (!ok) break;
     }
     if (warp == 0 && Cfull < C && (C - 1) % G == b) {  // the partial last chunk
       const double t = chunk_sum_warp<WDT>(W, T, C - 1, L);
