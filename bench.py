@@ -237,6 +237,38 @@ def time_oracle(wl, phase, budget_s, min_steps=1, rows_frac=1.0):
 # GPU arm
 # ----------------------------------------------------------------------------
 
+def graph_ms(stream, steps, body, sampler=None, world=1):
+    """Device time (ms) of ``steps`` calls of ``body(i)`` captured into one CUDA
+    graph, with CUDA events only at its two ends (events between the kernels
+    would add their own cost to every launch).  One untimed replay first; the
+    timed replay is bracketed by barrier + synchronize on both sides."""
+    import contextlib
+    import torch
+    e0 = torch.cuda.Event(enable_timing=True, external=True)
+    e1 = torch.cuda.Event(enable_timing=True, external=True)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+        e0.record(stream)
+        for i in range(steps):
+            body(i)
+        e1.record(stream)
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with (sampler if sampler is not None else contextlib.nullcontext()):
+        with torch.cuda.stream(stream):
+            g.replay()
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = e0.elapsed_time(e1)
+    del g
+    return ms
+
+
 def run_gpu(args, wl, rank, world, local_rank):
     import numpy as np
     import torch
@@ -296,73 +328,43 @@ def run_gpu(args, wl, rank, world, local_rank):
 
     ops = ["absmean", "ternarize_pack", "forward"] if args.phase == "all" else ["forward"]
 
-    def step(i, evs=None):
-        for li, L in enumerate(layers):
-            def mark(op_i):
-                if evs is not None:
-                    evs[(li, op_i)].record(stream)
-            if args.phase == "all":
-                mark(0)
-                B.bitlinear_absmean(L["W"], L["gamma"], L["ws"], stream)
-                mark(1)
-                B.bitlinear_ternarize_pack(L["W"], L["gamma"], eps, fmt, L["packed"], None, stream)
-                mark(2)
-                packed = L["packed"]
-            else:
-                mark(0)
-                packed = L["copies"][i % rot]
+    def run_op(op, L, i):
+        if op == "absmean":
+            B.bitlinear_absmean(L["W"], L["gamma"], L["ws"], stream)
+        elif op == "ternarize_pack":
+            B.bitlinear_ternarize_pack(L["W"], L["gamma"], eps, fmt, L["packed"], None, stream)
+        else:
+            packed = L["packed"] if args.phase == "all" else L["copies"][i % rot]
             B.bitlinear_forward(packed, fmt, L["gamma"], L["N"], L["K"], L["x"], L["scale"], L["y"],
                                 L["fws"], stream)
-            mark(len(ops))
 
-    def new_events():
-        d = {}
-        for li in range(len(layers)):
-            for oi in range(len(ops) + 1):
-                d[(li, oi)] = torch.cuda.Event(enable_timing=True, external=True)
-        return d
+    def step(i):
+        for L in layers:
+            for op in ops:
+                run_op(op, L, i)
 
-    # warm-up (eager), then capture the K timed steps into one graph
+    # warm-up (eager), then the K timed steps as one graph
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
             step(i)
     stream.synchronize()
-
-    step_events = [new_events() for _ in range(args.steps)]
-    t_start = torch.cuda.Event(enable_timing=True, external=True)
-    t_end = torch.cuda.Event(enable_timing=True, external=True)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream, capture_error_mode="relaxed"):
-        t_start.record(stream)
-        for i in range(args.steps):
-            step(i, step_events[i])
-        t_end.record(stream)
-    with torch.cuda.stream(stream):
-        graph.replay()          # one untimed replay (first-launch costs of the graph)
-    torch.cuda.synchronize()
-
     sampler = ClockSampler(local_rank)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    with sampler:
-        with torch.cuda.stream(stream):
-            graph.replay()
-        torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    ms = t_start.elapsed_time(t_end)
+    ms = graph_ms(stream, args.steps, step, sampler=sampler, world=world)
     for L in layers:
         st = B.bitlinear_device_status(L["fws"], stream)
         if st != B.BL_OK:
             raise RuntimeError(f"device status {B.status_string(st)}")
 
-    # per-op device time (ms per launch) from the events inside the graph
-    per_op = {op: [] for op in ops}
-    for evs in step_events:
-        for li in range(len(layers)):
-            for oi, op in enumerate(ops):
-                per_op[op].append((li, evs[(li, oi)].elapsed_time(evs[(li, oi + 1)])))
+    # each kernel's average launch duration: a graph of K steps of that call
+    # alone, over every layer in turn (so the inputs of consecutive launches
+    # together exceed L2), timed at its two ends
+    per_op_ms = {}
+    for op in ops:
+        if len(ops) == 1:
+            per_op_ms[op] = ms / (args.steps * len(layers))
+            continue
+        t = graph_ms(stream, args.steps, lambda i, op=op: [run_op(op, L, i) for L in layers])
+        per_op_ms[op] = t / (args.steps * len(layers))
     step_bytes = sum(sum(L["bytes"][op] for op in ops) for L in layers)
 
     ms_max = max_over_ranks(ms, world, dev)
@@ -390,9 +392,10 @@ def run_gpu(args, wl, rank, world, local_rank):
     stream.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
 
-    del graph
     prefill = run_prefill(args, dev, stream, rank_seed, l2) if args.prefill else None
-    res = dict(prefill=prefill, ms_total=ms_max, per_op=per_op, step_bytes=step_bytes, layers=layers, ops=ops,
+    decode = run_decode(args, dev, stream, rank_seed, l2) if args.decode else None
+    res = dict(prefill=prefill, decode=decode, ms_total=ms_max, per_op_ms=per_op_ms, step_bytes=step_bytes,
+               layers=layers, ops=ops,
                clocks=sampler.summary(), e2e_ms=e2e_ms, e2e_steps=e2e_steps, h2d=h2d, d2h=d2h,
                rot=rot, l2=l2, launches_per_step=len(layers) * len(ops))
     return res
@@ -431,42 +434,122 @@ def run_prefill(args, dev, stream, rank_seed, l2):
     ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(rot)]
     fws = torch.zeros(B.bitlinear_forward_workspace_bytes(M, N, K, 0, B.BL_I8), dtype=torch.uint8, device=dev)
 
-    def step(i, ev=None):
+    def act(i):
         r = i % rot
-        if ev is not None:
-            ev[0].record(stream)
         B.bitlinear_quantize_acts(xs[r], xq[r], sc[r], stream)
-        if ev is not None:
-            ev[1].record(stream)
+
+    def gemm(i):
+        r = i % rot
         B.bitlinear_forward(pk[r], 0, gamma, N, K, xq[r], sc[r], ys[r], fws, stream)
-        if ev is not None:
-            ev[2].record(stream)
 
     steps = max(1, args.prefill_steps)
     with torch.cuda.stream(stream):
         for i in range(3):
-            step(i)
+            act(i)
+            gemm(i)
     stream.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(steps)]
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
-        for i in range(steps):
-            step(i, evs[i])
-    with torch.cuda.stream(stream):
-        g.replay()
-    torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        g.replay()
-    torch.cuda.synchronize()
+    # each call timed as a graph of `steps` launches of it alone (rotating inputs)
+    act_ms = graph_ms(stream, steps, act) / steps
+    gemm_ms = graph_ms(stream, steps, gemm) / steps
     st = B.bitlinear_device_status(fws, stream)
     if st != B.BL_OK:
         raise RuntimeError(f"prefill device status {B.status_string(st)}")
-    act_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    gemm_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    del g
     ops = 2.0 * M * N * K
     return dict(M=M, K=K, N=N, act_ms=act_ms, gemm_ms=gemm_ms, ops=ops, rot=rot, steps=steps,
                 act_bytes=M * K * 2 + M * K + 4 * M)
+
+
+DECODE_SHAPES = {"3b": ("3b_decode", "3B decode: M=1, K=3200->N=8640 and K=8640->N=3200"),
+                 "70b": ("70b_decode", "70B decode: M=1, K=8192->N=28672 and K=28672->N=8192")}
+
+
+def run_decode(args, dev, stream, rank_seed, l2):
+    """Decode GEMV alone (steps 4-6, M=1) on weights packed beforehand, for the
+    3B and 70B layer shapes, 2-bit and base-3: a graph of ``decode_steps``
+    forward calls per layer over packed copies rotated so that consecutive reads
+    exceed 4x L2, timed at its two ends.  Per layer: average launch duration,
+    GB/s of algorithmic bytes and the fraction of the HBM peak."""
+    import numpy as np
+    import torch
+
+    from bitlinear_b1_fwd_b200 import binding as B
+    from bitlinear_b1_fwd_b200 import synth
+
+    out = {}
+    for key, (wname, desc) in DECODE_SHAPES.items():
+        wl = WORKLOADS[wname]
+        for fmt in (0, 1):
+            rows = []
+            for i, (N, K) in enumerate(wl["layers"]):
+                Wh = synth.normal_f32(1000 + wl["seed"] + 100 * i + rank_seed, (N, K), wl["sigma"])
+                xh = synth.to_bf16_bits(synth.normal_f32(2000 + wl["seed"] + 100 * i + rank_seed, (1, K)))
+                rb = B.bitlinear_packed_row_bytes(K, fmt)
+                W = torch.from_numpy(Wh).to(dev)
+                del Wh
+                gamma = torch.empty(1, dtype=torch.float32, device=dev)
+                ws = torch.zeros(B.bitlinear_quantize_weights_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+                p0 = torch.empty((N, rb), dtype=torch.uint8, device=dev)
+                with torch.cuda.stream(stream):
+                    B.bitlinear_quantize_weights(W, 1e-5, fmt, p0, None, gamma, ws, stream)
+                stream.synchronize()
+                del W
+                rot = max(2, -(-4 * l2 // (N * rb)))
+                copies = [p0] + [p0.clone() for _ in range(rot - 1)]
+                x = torch.from_numpy(xh.view(np.int16)).to(dev).view(torch.bfloat16)
+                y = torch.empty((1, N), dtype=torch.bfloat16, device=dev)
+                scale = torch.empty(1, dtype=torch.float32, device=dev)
+                fws = torch.zeros(B.bitlinear_forward_workspace_bytes(1, N, K, fmt, B.BL_BF16), dtype=torch.uint8,
+                                  device=dev)
+
+                def fwd(j, copies=copies, gamma=gamma, N=N, K=K, x=x, scale=scale, y=y, fws=fws, fmt=fmt):
+                    B.bitlinear_forward(copies[j % len(copies)], fmt, gamma, N, K, x, scale, y, fws, stream)
+
+                with torch.cuda.stream(stream):
+                    for j in range(3):
+                        fwd(j)
+                steps = max(1, args.decode_steps)
+                us = graph_ms(stream, steps, fwd) / steps * 1e3
+                st = B.bitlinear_device_status(fws, stream)
+                if st != B.BL_OK:
+                    raise RuntimeError(f"decode device status {B.status_string(st)}")
+                nbytes = layer_bytes(N, K, 1, rb)["forward"]
+                rows.append(dict(N=N, K=K, us=us, bytes=nbytes, rot=rot))
+                del copies, p0
+            out[f"{key}_{['2bit', 'base3'][fmt]}"] = dict(desc=desc, rows=rows)
+    return out
+
+
+def decode_summary(d):
+    if d is None:
+        return None
+    peak, kind = measured_peaks()
+    res = {}
+    for name, v in d.items():
+        rows = v["rows"]
+        tot_b = sum(r["bytes"] for r in rows)
+        tot_us = sum(r["us"] for r in rows)
+        gbs = tot_b / (tot_us * 1e-6) / 1e9
+        fmt = 1 if name.endswith("base3") else 0
+        res[name] = {"workload": v["desc"] + (", base-3 pack" if fmt else ", 2-bit pack"),
+                     "kernel": gemv_kernel_name(fmt, [(r["N"], r["K"]) for r in rows]), "GB_s": gbs, "frac_of_hbm": gbs / peak,
+                     "per_layer": [{"N": r["N"], "K": r["K"], "us_per_launch": r["us"], "bytes_per_launch": r["bytes"],
+                                    "GB_s": r["bytes"] / (r["us"] * 1e-6) / 1e9,
+                                    "frac_of_hbm": r["bytes"] / (r["us"] * 1e-6) / 1e9 / peak} for r in rows],
+                     "l2": f"packed copies rotated (>= 4x L2): {[r['rot'] for r in rows]}"}
+    return {"peak": peak, "peak_kind": kind, "unit": "GB/s", "shapes": res,
+            "launch_duration": "CUDA events at the two ends of a graph of back-to-back forward calls"}
+
+
+def gemv_kernel_name(fmt, layers):
+    """The decode kernel the forward dispatches to (M <= 4): the lean 2-bit
+    kernel for rows of at most 8192 packed bytes, else the general one."""
+    lean = fmt == 0 and all(((K + 3) // 4 + 15) // 16 * 16 <= 8192 for (_, K) in layers)
+    return "gemv_i2_kernel" if lean else "gemv_kernel"
+
+
+def gemm_kernel_name(M):
+    """The tensor-core kernel the forward dispatches to for M tokens (M > 4)."""
+    return "gemm_i2_2sm_kernel" if M > 128 else "gemm_i2_kernel"
 
 
 def prefill_summary(p):
@@ -482,9 +565,9 @@ def prefill_summary(p):
             "value": tops, "unit": "TOPS (int8)", "forward_TOPS_incl_act_quant": fwd_tops,
             "gemm_us": p["gemm_ms"] * 1e3, "act_quant_us": p["act_ms"] * 1e3,
             "act_quant_GB_s": act_gbs, "act_quant_frac_of_hbm": act_gbs / hbm,
-            "roofline": {"bound": "tensor", "kernel": "gemm_i2_kernel", "achieved": tops, "peak": peak,
+            "roofline": {"bound": "tensor", "kernel": gemm_kernel_name(p["M"]), "achieved": tops, "peak": peak,
                          "peak_kind": kind, "unit": "TOPS", "frac": tops / peak,
-                         "traffic": profiled_traffic("gemm_i2_kernel", "3b_prefill")},
+                         "traffic": profiled_traffic(gemm_kernel_name(p["M"]), "3b_prefill")},
             "steps": p["steps"], "l2": f"inputs rotated over {p['rot']} copies (> 2x L2)"}
 
 
@@ -500,6 +583,9 @@ def main():
     ap.add_argument("--prefill", action=argparse.BooleanOptionalAction, default=True,
                     help="also time the 3B prefill layer (INT8 TOPS of the tensor-core product)")
     ap.add_argument("--prefill-steps", type=int, default=20)
+    ap.add_argument("--decode", action=argparse.BooleanOptionalAction, default=True,
+                    help="also time the decode GEMV alone on packed 3B and 70B layers (2-bit and base-3)")
+    ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--cpu-budget", type=float, default=10.0,
                     help="seconds of oracle time for the cpu_baseline sample (0 = skip)")
     args = ap.parse_args()
@@ -553,23 +639,21 @@ def main():
         peak, peak_kind = measured_peaks()
         # per-op summary and the dominant kernel
         stages = {}
+        nl = len(res["layers"])
         for op in res["ops"]:
-            times = [t for (_, t) in res["per_op"][op]]
+            per_launch = res["per_op_ms"][op]
             nb = sum(L["bytes"][op] for L in res["layers"])
-            tot = sum(times) / args.steps
-            stages[op] = {"ms_per_step": tot, "bytes_per_step": nb, "GB_s": nb / (tot * 1e-3) / 1e9,
-                          "frac_of_hbm": nb / (tot * 1e-3) / 1e9 / peak,
-                          "per_layer_us": [statistics.mean(t for (li, t) in res["per_op"][op] if li == j) * 1e3
-                                           for j in range(len(res["layers"]))]}
-        dom = max(stages, key=lambda o: stages[o]["ms_per_step"])
-        launches = len(res["layers"]) * args.steps
-        avg_launch_ms = stages[dom]["ms_per_step"] * args.steps / launches
-        bytes_per_launch = stages[dom]["bytes_per_step"] / len(res["layers"])
+            stages[op] = {"us_per_launch": per_launch * 1e3, "bytes_per_step": nb,
+                          "GB_s": nb / (per_launch * nl * 1e-3) / 1e9,
+                          "frac_of_hbm": nb / (per_launch * nl * 1e-3) / 1e9 / peak}
+        dom = max(stages, key=lambda o: stages[o]["us_per_launch"])
+        avg_launch_ms = res["per_op_ms"][dom]
+        bytes_per_launch = stages[dom]["bytes_per_step"] / nl
         achieved = bytes_per_launch / (avg_launch_ms * 1e-3) / 1e9
         flat = wl["fmt"] == 0 and all(K % 64 == 0 for (_, K) in wl["layers"])
-        kernel_name = {"absmean": "absmean_bulk_kernel",
+        kernel_name = {"absmean": "absmean_kernel",
                        "ternarize_pack": "ternarize_flat_kernel" if flat else "ternarize_pack_kernel",
-                       "forward": "gemv_kernel"}[dom]
+                       "forward": gemv_kernel_name(wl["fmt"], wl["layers"])}[dom]
         traffic = profiled_traffic(kernel_name, args.workload)
         cpu = None
         if args.cpu_budget > 0 and world == 1:
@@ -589,12 +673,15 @@ def main():
                            kernels_per_step=res["launches_per_step"]),
             "roofline": {"bound": "hbm", "kernel": kernel_name, "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": traffic, "bytes_per_launch": bytes_per_launch},
+                         "traffic": traffic, "bytes_per_launch": bytes_per_launch,
+                         "launch_duration": "CUDA events at the two ends of a graph of K steps of this call alone "
+                                            "over every layer (K x layers back-to-back launches)"},
             "stages": stages,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": res["h2d"],
                     "d2h_bytes_per_step": res["d2h"], "steps": res["e2e_steps"]},
             "prefill": prefill_summary(res["prefill"]),
+            "decode_gemv": decode_summary(res["decode"]),
             "gpu_launches": res["launches_per_step"] * args.steps,
             "clocks": res["clocks"],
         }

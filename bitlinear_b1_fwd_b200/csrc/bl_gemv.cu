@@ -22,7 +22,8 @@ namespace bl {
 
 constexpr int kGemvThreads = 768;  // one CTA per SM: the token prologue runs once per SM
 constexpr int kGemvWarps = kGemvThreads / 32;
-constexpr int kGemvDepth = 6;  // row-block items whose loads are in flight per warp
+constexpr int kGemvBatch = 4;         // items per load batch; two batches per warp alternate
+constexpr int kGemvTileRows = 1024;   // rows whose sums a CTA holds in shared memory at a time
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   uint4 v;
@@ -35,6 +36,11 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 // Activation bytes per token in shared memory for one packed row of rowbytes.
 __host__ __device__ inline int64_t gemv_x_bytes(int fmt, int64_t rowbytes) {
   return fmt == BL_PACK_I2 ? rowbytes * 4 : rowbytes * 8;
+}
+
+// Dynamic shared memory of one CTA for mt tokens.
+__host__ __device__ inline int64_t gemv_smem_bytes(int fmt, int64_t rowbytes, int mt) {
+  return mt * gemv_x_bytes(fmt, rowbytes) + int64_t{4} * mt * kGemvTileRows + (fmt == BL_PACK_T5 ? 256 * 8 : 0);
 }
 
 // dp4a with unsigned bytes in a and signed bytes in b.
@@ -72,6 +78,35 @@ __device__ __forceinline__ uint32_t x_slot(int fmt, uint32_t k, uint32_t segs) {
   }
 }
 
+// The four bytes q[0..3] (low byte of each) as one word, q[0] in the low byte.
+__device__ __forceinline__ uint32_t pack4(const int* q) {
+  return __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
+}
+
+// The 2-bit layout's 16-byte slot of the 16 codes q[0..15] of one packed word:
+// byte 4j + b = q[4b + j], a 4 x 4 byte transpose of P_b = q[4b .. 4b + 3].
+__device__ __forceinline__ uint4 i2_slot(uint32_t P0, uint32_t P1, uint32_t P2, uint32_t P3) {
+  const uint32_t t0 = __byte_perm(P0, P1, 0x5140), t1 = __byte_perm(P2, P3, 0x5140);
+  const uint32_t t2 = __byte_perm(P0, P1, 0x7362), t3 = __byte_perm(P2, P3, 0x7362);
+  return make_uint4(__byte_perm(t0, t1, 0x5410), __byte_perm(t0, t1, 0x7632), __byte_perm(t2, t3, 0x5410),
+                    __byte_perm(t2, t3, 0x7632));
+}
+
+// Work split.  CTA b owns the rows [row0, row0 + nrows) (the N rows shared
+// out as evenly as the grid allows); they are contiguous in memory, and the CTA
+// takes them in tiles of at most kGemvTileRows rows.  A tile is a run of
+// S = rows x segs 16-byte segments; its work items are the 32-segment blocks
+// of that run (512 bytes each, not aligned to rows), dealt round-robin to the
+// warps, so at any time the CTA streams one contiguous window of up to
+// 2 kGemvBatch x kGemvWarps blocks (96 KB).  Each warp loads its items in
+// batches of kGemvBatch (the loads of a batch are issued together and waited
+// for together), two batches alternating: while one is reduced the other is
+// in flight.  Lane L
+// of an item takes segment 32 j + L; a block covers at most two rows when a
+// row has 32 segments or more (any number otherwise).  Each item's INT32 sums
+// are reduced per row across the warp and added into the tile's shared row
+// sums (integer addition: the order does not matter); after the tile the CTA
+// dequantizes the row sums and stores them coalesced.
 template <int FMT, int MT, int XDT>
 __global__ void __launch_bounds__(kGemvThreads, 1)
     gemv_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
@@ -79,53 +114,60 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
                 void* __restrict__ y, int ydt, int write_scale) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int64_t xb = gemv_x_bytes(FMT, rowbytes);
-  uint8_t* xs = smem;                                     // [MT][xb]
-  uint2* lut = reinterpret_cast<uint2*>(smem + MT * xb);  // base 3 only
+  uint8_t* xs = smem;                                                 // [MT][xb]
+  int* racc = reinterpret_cast<int*>(smem + MT * xb);                 // [MT][kGemvTileRows]
+  uint2* lut = reinterpret_cast<uint2*>(racc + MT * kGemvTileRows);   // base 3 only
   __shared__ float red_f[MT][kGemvWarps];
   __shared__ int red_i[MT][kGemvWarps];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t segs = static_cast<uint32_t>(rowbytes >> 4);
   const uint32_t nb = (segs + 31) >> 5;  // 32-segment blocks per row
-  const int64_t TW = static_cast<int64_t>(gridDim.x) * kGemvWarps;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kGemvWarps + warp;
-  const int64_t nrows = r0 < N ? (N - 1 - r0) / TW + 1 : 0;
+  const int64_t G = gridDim.x, b = blockIdx.x;
+  const int64_t per = N / G, extra = N % G;
+  const int64_t row0 = b * per + (b < extra ? b : extra);
+  const int64_t nrows = per + (b < extra ? 1 : 0);
 
-  // The warp's items are (row r0 + ri TW, 32-segment block blk), in order;
-  // the lane's segment of an item is 32 blk + lane.  Two cursors walk them:
-  // one for the loads in flight, one for the item being reduced.
-  int64_t l_ri = 0;
-  uint32_t l_blk = 0;
-  const uint8_t* l_row = packed + r0 * rowbytes;
+  // The warp's items in a tile are j = warp + W k.  Two cursors walk them: one
+  // for the loads in flight, one for the item being reduced.  (A tile has at
+  // most kGemvTileRows x segs < 2^22 segments: 32-bit counts.)
+  uint32_t S = 0, nitems = 0, l_j = 0;
+  const uint4* tile = nullptr;
+  auto start_tile = [&](int64_t t0) {
+    const uint32_t nr = static_cast<uint32_t>((nrows - t0) < kGemvTileRows ? (nrows - t0) : kGemvTileRows);
+    S = nr * segs;
+    nitems = (S + 31) >> 5;
+    l_j = warp;
+    tile = reinterpret_cast<const uint4*>(packed + (row0 + t0) * rowbytes);
+  };
   auto load_next = [&](uint4& dst) {
-    const uint32_t s = 32 * l_blk + lane;
-    if (s < segs) dst = ld_stream(reinterpret_cast<const uint4*>(l_row) + s);
-    if (++l_blk == nb) {
-      l_blk = 0;
-      ++l_ri;
-      l_row += TW * rowbytes;
-    }
+    const uint32_t g = 32 * l_j + lane;
+    if (g < S) dst = ld_stream(tile + g);
+    l_j += kGemvWarps;
   };
 
-  // 1. the first kGemvDepth items' loads go out before the prologue
-  uint4 buf[kGemvDepth];
+  auto issue = [&](uint4(&b)[kGemvBatch]) {
 #pragma unroll
-  for (int d = 0; d < kGemvDepth; ++d) {
-    buf[d] = make_uint4(0, 0, 0, 0);
-    if (l_ri < nrows) load_next(buf[d]);
-  }
+    for (int d = 0; d < kGemvBatch; ++d)
+      if (l_j < nitems) load_next(b[d]);
+  };
 
-  // 2. prologue: zero the activation area, per-token absmax, then scatter the
-  //    INT8 codes into the layout above.
-  {
+  // 1. the first tile's first batch goes out before the prologue
+  start_tile(0);
+  uint4 bufA[kGemvBatch], bufB[kGemvBatch];
+#pragma unroll
+  for (int d = 0; d < kGemvBatch; ++d) bufA[d] = bufB[d] = make_uint4(0, 0, 0, 0);
+  issue(bufA);
+
+  // 2. prologue: per-token absmax, then the INT8 codes in the layout above
+  for (int i = threadIdx.x; i < MT * kGemvTileRows; i += blockDim.x) racc[i] = 0;
+  if constexpr (FMT == BL_PACK_T5) {
     uint4* z = reinterpret_cast<uint4*>(xs);
     for (int64_t i = threadIdx.x; i < MT * xb / 16; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
-  }
-  if constexpr (FMT == BL_PACK_T5) {
-    for (int b = threadIdx.x; b < 256; b += blockDim.x) {
+    for (int e = threadIdx.x; e < 256; e += blockDim.x) {
       uint32_t lo = 0, hi = 0;
-      if (b < 243) {
-        int v = b;
+      if (e < 243) {
+        int v = e;
 #pragma unroll
         for (int i = 0; i < 5; ++i) {
           const uint32_t w = static_cast<uint8_t>(static_cast<int8_t>(v % 3 - 1));
@@ -134,7 +176,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
           else hi = w;
         }
       }
-      lut[b] = make_uint2(lo, hi);
+      lut[e] = make_uint2(lo, hi);
     }
   }
   const bool vec = (K % 8) == 0;
@@ -157,7 +199,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
       if (lane == 0) red_f[m][warp] = amax;
     }
   }
-  __syncthreads();  // zeroed activations, table and per-warp maxima are visible
+  __syncthreads();  // zeroed sums and activations, table and per-warp maxima are visible
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
     if constexpr (XDT != BL_I8) {
@@ -174,7 +216,48 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     int part = 0;
     uint8_t* xm = xs + m * xb;
     const float c127 = (XDT == BL_I8) ? 0.0f : __fdiv_rn(127.0f, s_tok[m]);
-    if (vec) {
+    if constexpr (FMT == BL_PACK_I2) {
+      // one packed word's 16 codes per step, written as one 16-byte slot
+      // (codes past K, under padding digits, are 0)
+      for (uint32_t g = threadIdx.x; g < 4 * segs; g += blockDim.x) {
+        const int64_t k0 = 16 * static_cast<int64_t>(g);
+        const bool full = k0 + 16 <= K && (K % 16) == 0;
+        uint32_t P[4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // eight codes at a time
+          const int64_t kh = k0 + 8 * h;
+          int q[8];
+          if (full) {
+            if constexpr (XDT == BL_I8) {
+              const uint2 raw = __ldg(reinterpret_cast<const uint2*>(static_cast<const int8_t*>(x) + m * K + kh));
+#pragma unroll
+              for (int j = 0; j < 8; ++j) q[j] = static_cast<int8_t>((j < 4 ? raw.x : raw.y) >> (8 * (j & 3)));
+            } else {
+              float e[8];
+              load8_aligned<XDT>(x, m * K + kh, e);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) q[j] = quant_act_fast(e[j], s_tok[m], c127);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int64_t k = kh + j;
+              if (k < K)
+                q[j] = (XDT == BL_I8) ? static_cast<int>(static_cast<const int8_t*>(x)[m * K + k])
+                                      : quant_act_fast(load_x<XDT>(x, m * K + k), s_tok[m], c127);
+              else
+                q[j] = 0;
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) part += q[j];
+          P[2 * h] = pack4(q);
+          P[2 * h + 1] = pack4(q + 4);
+        }
+        const uint32_t s = g >> 2, w = g & 3;
+        *reinterpret_cast<uint4*>(xm + (w * segs + s) * 16) = i2_slot(P[0], P[1], P[2], P[3]);
+      }
+    } else if (vec) {
       for (int64_t v = threadIdx.x; v < K / 8; v += blockDim.x) {
         int q[8];
         if constexpr (XDT == BL_I8) {
@@ -213,87 +296,372 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     int t = 0;
 #pragma unroll
     for (int w = 0; w < kGemvWarps; ++w) t += red_i[m][w];
-    corr[m] = (FMT == BL_PACK_I2) ? t : 0;  // 2-bit digits are q + 1: subtract sum x once
+    corr[m] = (FMT == BL_PACK_I2) ? t : 0;  // 2-bit digits are q + 1: subtract sum x once per row
     cfac[m] = dequant_factor(g, s_tok[m]);
     if (XDT != BL_I8 && write_scale && blockIdx.x == 0 && threadIdx.x == 0) scale[m] = s_tok[m];
   }
 
-  // 3. stream the items, kGemvDepth loads always in flight.  2-bit: the digit
-  //    of weight position j of each byte is taken in place, w & (3 << 2j), so
-  //    each byte holds d 4^j; accumulator j collects 4^j sum d x, and the
-  //    factor comes off exactly at the end of the row.
-  int acc[MT], acc1[MT], acc2[MT], acc3[MT];
+  // 3. per tile: stream the items, one batch of loads in flight while the
+  //    other is reduced.
+  const bool wide = segs >= 32;                            // a block spans at most two rows
+  const uint32_t dq = (32u * kGemvWarps) / segs, dr = (32u * kGemvWarps) % segs;  // one step of a warp
+  for (int64_t t0 = 0; t0 < nrows; t0 += kGemvTileRows) {
+    if (t0 > 0) {
+      start_tile(t0);
+      issue(bufA);
+    }
+    const uint32_t nr = S / segs;
+    uint32_t c_j = warp;
+    uint32_t r0 = (32u * c_j) / segs, s0 = 32u * c_j - r0 * segs;  // row and segment of lane 0
+    auto consume = [&](const uint4(&b)[kGemvBatch]) {
 #pragma unroll
-  for (int m = 0; m < MT; ++m) acc[m] = acc1[m] = acc2[m] = acc3[m] = 0;
-  int64_t c_ri = 0;
-  uint32_t c_blk = 0;
-  while (c_ri < nrows) {
+      for (int d = 0; d < kGemvBatch; ++d) {
+        if (c_j >= nitems) break;
+        const uint4 cur = b[d];
+        const uint32_t g = 32 * c_j + lane;
+        uint32_t r, sg;
+        if (wide) {
+          sg = s0 + lane;
+          r = r0;
+          if (sg >= segs) {
+            sg -= segs;
+            ++r;
+          }
+        } else {
+          r = g / segs;
+          sg = g - r * segs;
+        }
+        int v[MT];
 #pragma unroll
-    for (int d = 0; d < kGemvDepth; ++d) {
-      if (c_ri >= nrows) break;
-      const uint4 cur = buf[d];
-      if (l_ri < nrows) load_next(buf[d]);
-      const uint32_t s = 32 * c_blk + lane;
-      if (s < segs) {
-        const uint32_t wd[4] = {cur.x, cur.y, cur.z, cur.w};
+        for (int m = 0; m < MT; ++m) v[m] = 0;
+        if (g < S) {
+          const uint32_t wd[4] = {cur.x, cur.y, cur.z, cur.w};
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          if constexpr (FMT == BL_PACK_I2 && MT == 1) {
-            const uint32_t c0 = wd[w] & 0x03030303u, c1 = wd[w] & 0x0c0c0c0cu;
-            const uint32_t c2 = wd[w] & 0x30303030u, c3 = wd[w] & 0xc0c0c0c0u;
-            const uint4 X = *reinterpret_cast<const uint4*>(xs + ((w * segs) + s) * 16);
-            acc[0] = dp4a_us(c0, X.x, acc[0]);
-            acc1[0] = dp4a_us(c1, X.y, acc1[0]);
-            acc2[0] = dp4a_us(c2, X.z, acc2[0]);
-            acc3[0] = dp4a_us(c3, X.w, acc3[0]);
-          } else if constexpr (FMT == BL_PACK_I2) {  // several tokens: digits shifted down once
-            const uint32_t c0 = wd[w] & 0x03030303u, c1 = (wd[w] >> 2) & 0x03030303u;
-            const uint32_t c2 = (wd[w] >> 4) & 0x03030303u, c3 = (wd[w] >> 6) & 0x03030303u;
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-              const uint4 X = *reinterpret_cast<const uint4*>(xs + m * xb + ((w * segs) + s) * 16);
-              acc[m] = __dp4a(static_cast<int>(c0), static_cast<int>(X.x), acc[m]);
-              acc[m] = __dp4a(static_cast<int>(c1), static_cast<int>(X.y), acc[m]);
-              acc[m] = __dp4a(static_cast<int>(c2), static_cast<int>(X.z), acc[m]);
-              acc[m] = __dp4a(static_cast<int>(c3), static_cast<int>(X.w), acc[m]);
-            }
-          } else {
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-              const uint2 Lw = lut[(wd[w] >> (8 * b)) & 0xffu];
+          for (int w = 0; w < 4; ++w) {
+            if constexpr (FMT == BL_PACK_I2) {
+              const uint32_t c0 = wd[w] & 0x03030303u, c1 = (wd[w] >> 2) & 0x03030303u;
+              const uint32_t c2 = (wd[w] >> 4) & 0x03030303u, c3 = (wd[w] >> 6) & 0x03030303u;
 #pragma unroll
               for (int m = 0; m < MT; ++m) {
-                const uint2 X = *reinterpret_cast<const uint2*>(xs + m * xb + (((4 * w + b) * segs) + s) * 8);
-                acc[m] = __dp4a(static_cast<int>(Lw.x), static_cast<int>(X.x), acc[m]);
-                acc[m] = __dp4a(static_cast<int>(Lw.y), static_cast<int>(X.y), acc[m]);
+                const uint4 X = *reinterpret_cast<const uint4*>(xs + m * xb + ((w * segs) + sg) * 16);
+                v[m] = dp4a_us(c0, X.x, v[m]);
+                v[m] = dp4a_us(c1, X.y, v[m]);
+                v[m] = dp4a_us(c2, X.z, v[m]);
+                v[m] = dp4a_us(c3, X.w, v[m]);
+              }
+            } else {
+#pragma unroll
+              for (int bb = 0; bb < 4; ++bb) {
+                const uint2 Lw = lut[(wd[w] >> (8 * bb)) & 0xffu];
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                  const uint2 X = *reinterpret_cast<const uint2*>(xs + m * xb + (((4 * w + bb) * segs) + sg) * 8);
+                  v[m] = __dp4a(static_cast<int>(Lw.x), static_cast<int>(X.x), v[m]);
+                  v[m] = __dp4a(static_cast<int>(Lw.y), static_cast<int>(X.y), v[m]);
+                }
               }
             }
           }
         }
-      }
-      if (c_blk == nb - 1) {  // the row is complete: reduce, dequantize, store
-        const int64_t r = r0 + c_ri * TW;
+        // per-row sums of the block into the tile's row sums
+        if (wide) {
+          const uint32_t bnd = segs - s0;  // lanes >= bnd are in row r0 + 1
+          const uint32_t lo = bnd >= 32 ? 0xffffffffu : ((1u << bnd) - 1u);
+          const uint32_t mask = (static_cast<uint32_t>(lane) < bnd) ? lo : ~lo;
 #pragma unroll
-        for (int m = 0; m < MT; ++m) {
-          const int lane_sum = acc[m] + (acc1[m] >> 2) + (acc2[m] >> 4) + (acc3[m] >> 6);
-          const int a = __reduce_add_sync(0xffffffffu, lane_sum) - corr[m];
-          acc[m] = acc1[m] = acc2[m] = acc3[m] = 0;
-          if (lane == 0) {
-            const int64_t o = m * N + r;
-            if (ydt == BL_I32)
-              static_cast<int32_t*>(y)[o] = a;
-            else if (ydt == BL_F32)
-              static_cast<float*>(y)[o] = __fmul_rn(__int2float_rn(a), cfac[m]);
-            else
-              static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(a), cfac[m]));
+          for (int m = 0; m < MT; ++m) {
+            const int t = __reduce_add_sync(mask, v[m]);
+            if ((lane == 0 || static_cast<uint32_t>(lane) == bnd) && r < nr) atomicAdd(racc + m * kGemvTileRows + r, t);
+          }
+        } else {
+          const int key = g < S ? static_cast<int>(r) : -1;
+          const uint32_t mask = __match_any_sync(0xffffffffu, key);
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            const int t = __reduce_add_sync(mask, v[m]);
+            if (key >= 0 && (__ffs(mask) - 1) == lane) atomicAdd(racc + m * kGemvTileRows + key, t);
           }
         }
-        c_blk = 0;
-        ++c_ri;
-      } else {
-        ++c_blk;
+        c_j += kGemvWarps;
+        r0 += dq;
+        s0 += dr;
+        if (s0 >= segs) {
+          s0 -= segs;
+          ++r0;
+        }
+      }
+    };
+    while (c_j < nitems) {
+      issue(bufB);
+      consume(bufA);
+      issue(bufA);
+      consume(bufB);
+    }
+    __syncthreads();  // every part of every row of the tile has been added
+    for (int r = threadIdx.x; r < static_cast<int>(nr); r += blockDim.x) {
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const int a = racc[m * kGemvTileRows + r] - corr[m];
+        racc[m * kGemvTileRows + r] = 0;
+        const int64_t o = m * N + row0 + t0 + r;
+        if (ydt == BL_I32)
+          static_cast<int32_t*>(y)[o] = a;
+        else if (ydt == BL_F32)
+          static_cast<float*>(y)[o] = __fmul_rn(__int2float_rn(a), cfac[m]);
+        else
+          static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(a), cfac[m]));
       }
     }
+    __syncthreads();  // the row sums are zero again for the next tile
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 2-bit decode GEMV, lean form (rows of at most 2 kI2Plane bytes).  A work
+// item is one 64-segment (1 KB) block of a row; lane L takes the segments
+// 64 blk + 2L and 64 blk + 2L + 1 (two 16-byte loads, a warp reads 1 KB
+// contiguous).  A block lies in one row (the last block of a row is partial:
+// lanes past the row's end load nothing and add 0), so each item ends in one
+// warp reduction and one shared atomic into the row sum.  The activations of
+// a token sit in 8 planes of kI2Plane bytes, plane 2w + h holding, for the
+// segments s with s mod 2 = h, the 16 bytes of packed word w (the digit order
+// of the word, as in the general layout) at (s >> 1) * 16: the 32 lanes of a
+// warp read 32 consecutive 16-byte slots of a plane (no bank conflicts), and
+// the 8 planes of a lane are a compile-time distance apart.  The digits are
+// masked in place (w & (3 << 2j)), so accumulator j collects 4^j sum d x and
+// the factors come off exactly at the end of the item.  Work split and load
+// batching as in gemv_kernel: CTA-owned row ranges, items dealt round-robin
+// to the warps, two batches of kI2Batch items alternating.
+// ---------------------------------------------------------------------------
+constexpr int kI2Plane = 4096;  // bytes per activation plane: segments per row <= 2 kI2Plane / 16
+constexpr int kI2Batch = 2;     // items per load batch
+
+__host__ __device__ inline int64_t gemv_i2_smem_bytes(int mt) {
+  return int64_t{8} * kI2Plane * mt + int64_t{4} * mt * kGemvTileRows;
+}
+
+template <int MT, int XDT>
+__global__ void __launch_bounds__(kGemvThreads, 1)
+    gemv_i2_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
+                   int64_t N, int64_t K, const void* __restrict__ x, float* __restrict__ scale,
+                   void* __restrict__ y, int ydt, int write_scale) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint8_t* xs = smem;                                           // [MT][8][kI2Plane]
+  int* racc = reinterpret_cast<int*>(smem + MT * 8 * kI2Plane);  // [MT][kGemvTileRows]
+  __shared__ float red_f[MT][kGemvWarps];
+  __shared__ int red_i[MT][kGemvWarps];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t segs = static_cast<uint32_t>(rowbytes >> 4);
+  const uint32_t nb = (segs + 63) >> 6;  // 1 KB blocks per row
+  const int64_t G = gridDim.x, b = blockIdx.x;
+  const int64_t per = N / G, extra = N % G;
+  const int64_t row0 = b * per + (b < extra ? b : extra);
+  const int64_t nrows = per + (b < extra ? 1 : 0);
+  const uint32_t dq = kGemvWarps / nb, dr = kGemvWarps % nb;  // one step of a warp in (row, block)
+  const uint32_t s_lane = 2u * lane;                            // first segment of the lane in a block
+
+  // load cursor: item (l_row, l_blk) of the tile, l_row < l_rows
+  uint32_t l_row = 0, l_blk = 0, l_rows = 0;
+  const uint8_t* tile = packed;
+  auto start_tile = [&](int64_t t0) {
+    l_rows = static_cast<uint32_t>((nrows - t0) < kGemvTileRows ? (nrows - t0) : kGemvTileRows);
+    l_row = warp / nb;
+    l_blk = warp % nb;
+    tile = packed + (row0 + t0) * rowbytes;
+  };
+  auto issue = [&](uint4(&bf)[kI2Batch][2]) {
+#pragma unroll
+    for (int d = 0; d < kI2Batch; ++d) {
+      bf[d][0] = bf[d][1] = make_uint4(0, 0, 0, 0);
+      if (l_row < l_rows) {
+        const uint32_t s = 64u * l_blk + s_lane;
+        const uint4* p = reinterpret_cast<const uint4*>(tile + static_cast<int64_t>(l_row) * rowbytes) + s;
+        if (s < segs) bf[d][0] = ld_stream(p);
+        if (s + 1 < segs) bf[d][1] = ld_stream(p + 1);
+        l_blk += dr;
+        l_row += dq;
+        if (l_blk >= nb) {
+          l_blk -= nb;
+          ++l_row;
+        }
+      }
+    }
+  };
+
+  // 1. the first tile's first batch goes out before the prologue
+  start_tile(0);
+  uint4 bufA[kI2Batch][2], bufB[kI2Batch][2];
+  issue(bufA);
+
+  // 2. prologue: per-token absmax, then the INT8 codes in the plane layout
+  for (int i = threadIdx.x; i < MT * kGemvTileRows; i += blockDim.x) racc[i] = 0;
+  float s_tok[MT];
+  if constexpr (XDT != BL_I8) {
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      float amax = 0.0f;
+      if ((K % 8) == 0) {
+        for (int64_t v = threadIdx.x; v < K / 8; v += blockDim.x) {
+          float e[8];
+          load8_aligned<XDT>(x, m * K + 8 * v, e);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(e[j]));
+        }
+      } else {
+        for (int64_t k = threadIdx.x; k < K; k += blockDim.x) amax = fmaxf(amax, fabsf(load_x<XDT>(x, m * K + k)));
+      }
+      amax = warp_maxf(amax);
+      if (lane == 0) red_f[m][warp] = amax;
+    }
+  }
+  __syncthreads();  // zeroed row sums and per-warp maxima are visible
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    if constexpr (XDT != BL_I8) {
+      float a = red_f[m][0];
+#pragma unroll
+      for (int w = 1; w < kGemvWarps; ++w) a = fmaxf(a, red_f[m][w]);
+      s_tok[m] = fmaxf(a, 1e-6f);
+    } else {
+      s_tok[m] = __ldg(scale + m);
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    int part = 0;
+    uint8_t* xm = xs + m * 8 * kI2Plane;
+    const float c127 = (XDT == BL_I8) ? 0.0f : __fdiv_rn(127.0f, s_tok[m]);
+    for (uint32_t g = threadIdx.x; g < 4 * segs; g += blockDim.x) {  // one packed word's 16 codes
+      const int64_t k0 = 16 * static_cast<int64_t>(g);
+      const bool full = k0 + 16 <= K && (K % 16) == 0;
+      uint32_t P[4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t kh = k0 + 8 * h;
+        int q[8];
+        if (full) {
+          if constexpr (XDT == BL_I8) {
+            const uint2 raw = __ldg(reinterpret_cast<const uint2*>(static_cast<const int8_t*>(x) + m * K + kh));
+#pragma unroll
+            for (int j = 0; j < 8; ++j) q[j] = static_cast<int8_t>((j < 4 ? raw.x : raw.y) >> (8 * (j & 3)));
+          } else {
+            float e[8];
+            load8_aligned<XDT>(x, m * K + kh, e);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) q[j] = quant_act_fast(e[j], s_tok[m], c127);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int64_t k = kh + j;
+            if (k < K)
+              q[j] = (XDT == BL_I8) ? static_cast<int>(static_cast<const int8_t*>(x)[m * K + k])
+                                    : quant_act_fast(load_x<XDT>(x, m * K + k), s_tok[m], c127);
+            else
+              q[j] = 0;
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) part += q[j];
+        P[2 * h] = pack4(q);
+        P[2 * h + 1] = pack4(q + 4);
+      }
+      const uint32_t s = g >> 2, w = g & 3;
+      *reinterpret_cast<uint4*>(xm + (2 * w + (s & 1)) * kI2Plane + (s >> 1) * 16) = i2_slot(P[0], P[1], P[2], P[3]);
+    }
+    part = __reduce_add_sync(0xffffffffu, part);
+    if (lane == 0) red_i[m][warp] = part;
+  }
+  __syncthreads();  // activations and per-warp sums are visible
+  const float g = __ldg(gamma);
+  float cfac[MT];
+  int corr[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    int t = 0;
+#pragma unroll
+    for (int w = 0; w < kGemvWarps; ++w) t += red_i[m][w];
+    corr[m] = t;  // digits are q + 1: subtract sum x once per row
+    cfac[m] = dequant_factor(g, s_tok[m]);
+    if (XDT != BL_I8 && write_scale && blockIdx.x == 0 && threadIdx.x == 0) scale[m] = s_tok[m];
+  }
+
+  // 3. per tile: one batch of loads in flight while the other is reduced
+  const uint8_t* xl = xs + (s_lane >> 1) * 16;  // this lane's slot in block 0 of plane 0
+  for (int64_t t0 = 0; t0 < nrows; t0 += kGemvTileRows) {
+    if (t0 > 0) {
+      start_tile(t0);
+      issue(bufA);
+    }
+    const uint32_t nr = l_rows;
+    uint32_t c_row = warp / nb, c_blk = warp % nb;
+    auto consume = [&](const uint4(&bf)[kI2Batch][2]) {
+#pragma unroll
+      for (int d = 0; d < kI2Batch; ++d) {
+        if (c_row >= nr) break;
+        int a0[MT], a1[MT], a2[MT], a3[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) a0[m] = a1[m] = a2[m] = a3[m] = 0;
+        const uint8_t* xb = xl + c_blk * 512;  // block blk: slots 32 blk .. 32 blk + 31 of each plane
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t wd[4] = {bf[d][h].x, bf[d][h].y, bf[d][h].z, bf[d][h].w};
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const uint32_t c0 = wd[w] & 0x03030303u, c1 = wd[w] & 0x0c0c0c0cu;
+            const uint32_t c2 = wd[w] & 0x30303030u, c3 = wd[w] & 0xc0c0c0c0u;
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+              const uint4 X = *reinterpret_cast<const uint4*>(xb + (m * 8 + 2 * w + h) * kI2Plane);
+              a0[m] = dp4a_us(c0, X.x, a0[m]);
+              a1[m] = dp4a_us(c1, X.y, a1[m]);
+              a2[m] = dp4a_us(c2, X.z, a2[m]);
+              a3[m] = dp4a_us(c3, X.w, a3[m]);
+            }
+          }
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const int v = a0[m] + (a1[m] >> 2) + (a2[m] >> 4) + (a3[m] >> 6);
+          const int t = __reduce_add_sync(0xffffffffu, v);
+          if (lane == 0) atomicAdd(racc + m * kGemvTileRows + c_row, t);
+        }
+        c_blk += dr;
+        c_row += dq;
+        if (c_blk >= nb) {
+          c_blk -= nb;
+          ++c_row;
+        }
+      }
+    };
+    const uint32_t first_row = warp / nb;
+    if (first_row < nr) {
+      for (;;) {
+        issue(bufB);
+        consume(bufA);
+        if (c_row >= nr) break;
+        issue(bufA);
+        consume(bufB);
+        if (c_row >= nr) break;
+      }
+    }
+    __syncthreads();  // every part of every row of the tile has been added
+    for (int r = threadIdx.x; r < static_cast<int>(nr); r += blockDim.x) {
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const int a = racc[m * kGemvTileRows + r] - corr[m];
+        racc[m * kGemvTileRows + r] = 0;
+        const int64_t o = m * N + row0 + t0 + r;
+        if (ydt == BL_I32)
+          static_cast<int32_t*>(y)[o] = a;
+        else if (ydt == BL_F32)
+          static_cast<float*>(y)[o] = __fmul_rn(__int2float_rn(a), cfac[m]);
+        else
+          static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(a), cfac[m]));
+      }
+    }
+    __syncthreads();  // the row sums are zero again for the next tile
   }
 }
 
@@ -301,11 +669,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
 // Host side.
 // ---------------------------------------------------------------------------
 int gemv_max_tokens(int fmt, int64_t rowbytes) {
-  const int64_t xb = gemv_x_bytes(fmt, rowbytes);
-  const int64_t budget = kGemvSmemBudget - (fmt == BL_PACK_T5 ? 256 * 8 : 0);
-  int64_t mt = budget / xb;
-  if (mt > kGemvMaxTokens) mt = kGemvMaxTokens;
-  return static_cast<int>(mt);
+  int mt = kGemvMaxTokens;
+  while (mt > 0 && gemv_smem_bytes(fmt, rowbytes, mt) > kGemvSmemBudget) --mt;
+  return mt;
 }
 
 template <int FMT, int MT, int XDT>
@@ -313,7 +679,7 @@ static cudaError_t launch_gemv_t(const uint8_t* packed, int64_t rowbytes, const 
                                  int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
                                  int write_scale, cudaStream_t st) {
   auto kern = gemv_kernel<FMT, MT, XDT>;
-  const size_t smem = static_cast<size_t>(MT * gemv_x_bytes(FMT, rowbytes)) + (FMT == BL_PACK_T5 ? 256 * 8 : 0);
+  const size_t smem = static_cast<size_t>(gemv_smem_bytes(FMT, rowbytes, MT));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kGemvSmemBudget));
   if (e != cudaSuccess) return e;
@@ -322,13 +688,40 @@ static cudaError_t launch_gemv_t(const uint8_t* packed, int64_t rowbytes, const 
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGemvThreads, smem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
-  int64_t need = (N + kGemvWarps - 1) / kGemvWarps;
+  int64_t need = N;  // every CTA owns at least one row
   int64_t grid = static_cast<int64_t>(sms) * per_sm;
   if (grid > need) grid = need;
   if (grid < 1) grid = 1;
   kern<<<static_cast<unsigned>(grid), kGemvThreads, smem, st>>>(packed, rowbytes, gamma, N, K, x, scale,
                                                                  y, ydt, write_scale);
   return cudaGetLastError();
+}
+
+template <int MT, int XDT>
+static cudaError_t launch_gemv_i2_t(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N,
+                                    int64_t K, const void* x, float* scale, void* y, int ydt, int write_scale,
+                                    cudaStream_t st) {
+  auto kern = gemv_i2_kernel<MT, XDT>;
+  const size_t smem = static_cast<size_t>(gemv_i2_smem_bytes(MT));
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t sms = device_sms();
+  const int64_t grid = N < sms ? N : sms;  // every CTA owns at least one row
+  kern<<<static_cast<unsigned>(grid), kGemvThreads, smem, st>>>(packed, rowbytes, gamma, N, K, x, scale, y, ydt,
+                                                                 write_scale);
+  return cudaGetLastError();
+}
+
+template <int XDT>
+static cudaError_t launch_gemv_i2_mt(int mt, const uint8_t* packed, int64_t rowbytes, const float* gamma,
+                                     int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
+                                     int write_scale, cudaStream_t st) {
+  switch (mt) {
+    case 1: return launch_gemv_i2_t<1, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
+    case 2: return launch_gemv_i2_t<2, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
+    case 3: return launch_gemv_i2_t<3, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
+    default: return launch_gemv_i2_t<4, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
+  }
 }
 
 template <int FMT, int XDT>
@@ -350,6 +743,9 @@ cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int6
   const int64_t rowbytes = (fmt == BL_PACK_I2) ? ((K + 3) / 4 + 15) / 16 * 16 : ((K + 4) / 5 + 15) / 16 * 16;
   const int mt_max = gemv_max_tokens(fmt, rowbytes);
   if (mt_max < 1) return cudaErrorInvalidValue;
+  // 2-bit rows of up to 2 kI2Plane bytes take the lean kernel (its shared
+  // memory, 8 planes per token, fits kGemvMaxTokens tokens within the budget)
+  const bool lean = fmt == BL_PACK_I2 && rowbytes <= 2 * kI2Plane;
   const int esz = (xdt == BL_F32) ? 4 : (xdt == BL_BF16 ? 2 : 1);
   const int ysz = (ydt == BL_BF16) ? 2 : 4;
   for (int64_t m0 = 0; m0 < M; m0 += mt_max) {
@@ -358,7 +754,11 @@ cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int6
     float* sm = scale + m0;
     void* ym = static_cast<uint8_t*>(y) + m0 * N * ysz;
     cudaError_t e;
-    if (fmt == BL_PACK_I2) {
+    if (lean) {
+      if (xdt == BL_F32) e = launch_gemv_i2_mt<BL_F32>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
+      else if (xdt == BL_BF16) e = launch_gemv_i2_mt<BL_BF16>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
+      else e = launch_gemv_i2_mt<BL_I8>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, st);
+    } else if (fmt == BL_PACK_I2) {
       if (xdt == BL_F32) e = launch_gemv_mt<BL_PACK_I2, BL_F32>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
       else if (xdt == BL_BF16) e = launch_gemv_mt<BL_PACK_I2, BL_BF16>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
       else e = launch_gemv_mt<BL_PACK_I2, BL_I8>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, st);

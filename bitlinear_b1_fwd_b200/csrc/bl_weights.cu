@@ -8,7 +8,6 @@
 
 #include "bl_common.cuh"
 #include "bl_kernels.h"
-#include "bl_sm100.cuh"
 
 namespace bl {
 
@@ -18,12 +17,9 @@ namespace bl {
 // 8192c + 2048i + 8l + j for i = 0..3, j = 0..7; the 256 lane sums meet in the
 // stride-halving tree p[l] += p[l + s], s = 128..1.
 //
-// One warp computes one chunk: lane L holds the eight lanes l = L + 32v
-// (v = 0..7) in registers, so the tree levels s = 128, 64, 32 pair registers
-// of the same thread (v with v + 4, v + 2, v + 1) and only s = 16..1 cross
-// lanes (shuffles).  For fixed (i, v) the warp reads 256 consecutive elements
-// (1 KB of fp32), each lane 32 contiguous bytes.  Warps stride over the chunks
-// (persistent grid), so no CTA waits on another within a chunk.
+// The kernel below gives lane l of a chunk to thread l of a 256-thread CTA;
+// for fixed i the CTA reads 2048 consecutive elements, each thread 32
+// contiguous bytes.
 //
 // When all warps of a CTA are done, the CTA takes a ticket; the CTA with the
 // last ticket combines the C chunk sums, zero-padded to P = 2^ceil(log2 C), by
@@ -36,234 +32,11 @@ namespace bl {
 //   - the last 8 levels run in shared memory and warp shuffles.
 // ---------------------------------------------------------------------------
 
-template <int WDT>
-__device__ __forceinline__ double chunk_sum_warp(const void* __restrict__ W, int64_t T, int64_t c, int L) {
-  double p[8];
-#pragma unroll
-  for (int v = 0; v < 8; ++v) p[v] = 0.0;
-  const int64_t c0 = c * kChunk;
-  const bool full = c0 + kChunk <= T;
-#pragma unroll
-  for (int h = 0; h < 8; ++h) {  // (i, half) = (h / 2, h % 2): lanes v = 4 (h % 2) .. + 3
-    const int i = h >> 1, v0 = 4 * (h & 1);
-    float x[4][8];
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int64_t e0 = c0 + 2048 * i + 256 * (v0 + v) + 8 * L;
-      if (full) {
-        load8_aligned<WDT>(W, e0, x[v]);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) x[v][j] = (e0 + j < T) ? load_elem<WDT>(W, e0 + j) : 0.0f;
-      }
-    }
-#pragma unroll
-    for (int v = 0; v < 4; ++v)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) p[v0 + v] = __dadd_rn(p[v0 + v], static_cast<double>(fabsf(x[v][j])));
-  }
-  // lane levels 128, 64, 32: registers of this thread
-#pragma unroll
-  for (int v = 0; v < 4; ++v) p[v] = __dadd_rn(p[v], p[v + 4]);
-  p[0] = __dadd_rn(p[0], p[2]);
-  p[1] = __dadd_rn(p[1], p[3]);
-  double t = __dadd_rn(p[0], p[1]);
-  // lane levels 16..1: across the warp
-#pragma unroll
-  for (int s = 16; s >= 1; s >>= 1) t = __dadd_rn(t, __shfl_down_sync(0xffffffffu, t, s));
-  return t;
-}
-
-// The same fixed-order chunk sum, reading a chunk staged in shared memory.
-template <int WDT>
-__device__ __forceinline__ double chunk_sum_smem(const uint8_t* stage, int L) {
-  constexpr int ES = (WDT == BL_F32) ? 4 : 2;
-  double p[8];
-#pragma unroll
-  for (int v = 0; v < 8; ++v) p[v] = 0.0;
-#pragma unroll
-  for (int hv = 0; hv < 2; ++hv)
-#pragma unroll 1
-  for (int i = 0; i < 4; ++i) {
-    const int v0 = 4 * hv;
-    float x[4][8];
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const uint8_t* src = stage + (2048 * i + 256 * (v0 + v) + 8 * L) * ES;
-      if constexpr (WDT == BL_F32) {
-        const float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 16);
-        x[v][0] = a.x; x[v][1] = a.y; x[v][2] = a.z; x[v][3] = a.w;
-        x[v][4] = b.x; x[v][5] = b.y; x[v][6] = b.z; x[v][7] = b.w;
-      } else {
-        const uint4 a = *reinterpret_cast<const uint4*>(src);
-        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          x[v][2 * k] = __uint_as_float(w[k] << 16);
-          x[v][2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
-        }
-      }
-    }
-#pragma unroll
-    for (int v = 0; v < 4; ++v)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) p[v0 + v] = __dadd_rn(p[v0 + v], static_cast<double>(fabsf(x[v][j])));
-  }
-#pragma unroll
-  for (int v = 0; v < 4; ++v) p[v] = __dadd_rn(p[v], p[v + 4]);
-  p[0] = __dadd_rn(p[0], p[2]);
-  p[1] = __dadd_rn(p[1], p[3]);
-  double t = __dadd_rn(p[0], p[1]);
-#pragma unroll
-  for (int s = 16; s >= 1; s >>= 1) t = __dadd_rn(t, __shfl_down_sync(0xffffffffu, t, s));
-  return t;
-}
-
-// Part of the fixed-order chunk sum done by one of four warps: lanes
-// l = L + 32 v for v in {sub, sub + 4}, summed in order and combined at tree
-// level 128 (v with v + 4), giving p'[sub].
-template <int WDT>
-__device__ __forceinline__ double chunk_part_smem(const uint8_t* stage, int L, int sub) {
-  constexpr int ES = (WDT == BL_F32) ? 4 : 2;
-  double p[2] = {0.0, 0.0};
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int v = sub + 4 * h;
-#pragma unroll 2
-    for (int i = 0; i < 4; ++i) {
-      float x[8];
-      const uint8_t* src = stage + (2048 * i + 256 * v + 8 * L) * ES;
-      if constexpr (WDT == BL_F32) {
-        const float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 16);
-        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-      } else {
-        const uint4 a = *reinterpret_cast<const uint4*>(src);
-        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          x[2 * k] = __uint_as_float(w[k] << 16);
-          x[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) p[h] = __dadd_rn(p[h], static_cast<double>(fabsf(x[j])));
-    }
-  }
-  return __dadd_rn(p[0], p[1]);  // level 128
-}
-
-// Bulk-staged absmean: one persistent CTA per SM.  A producer thread keeps
-// kBulkStages whole chunks in flight with cp.async.bulk (global -> shared);
-// consumer warp w owns stage w: it reduces the chunks j = w, w + S, w + 2S, ...
-// of its CTA's list from shared memory, in order, and releases the stage.
-// (Every waiter of a stage barrier is then at most one phase ahead of it, which
-// a parity wait needs: a waiter two phases ahead would see the phase before
-// last, of the same parity, and go on early.)  A partial last chunk is read
-// directly from global memory.  All waits are bounded; on expiry the timeout
-// flag is set and gamma is not meaningful.
-constexpr int kBulkStages = 6;
-constexpr int kAbsWarpsPerStage = 4;
-constexpr int kBulkConsumers = kBulkStages * kAbsWarpsPerStage;
-constexpr int kBulkThreads = 32 * (kBulkConsumers + 1);
-constexpr long long kBulkWaitCycles = 1ll << 32;
-constexpr int kTernConsumers = kBulkStages;  // one consumer warp per stage, as above
-constexpr int kTernThreads = 32 * (kTernConsumers + 1);
-
-template <int WDT>
-__global__ void __launch_bounds__(kBulkThreads, 1)
-    absmean_bulk_kernel(const void* __restrict__ W, int64_t T, int64_t C, int64_t Cfull, int lgR,
-                        double* __restrict__ partials, WsHeader* __restrict__ hdr, float* __restrict__ gamma) {
-  constexpr uint32_t CB = kChunk * ((WDT == BL_F32) ? 4 : 2);  // bytes per chunk
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBulkStages * CB);
-  uint64_t* empty = full + kBulkStages;
-  __shared__ int abort_flag;
-  __shared__ double p[kLanes];
-  __shared__ double xchg[kBulkStages][kAbsWarpsPerStage][32];
-  __shared__ bool last;
-  const int warp = threadIdx.x >> 5, L = threadIdx.x & 31;
-  const int64_t G = gridDim.x, b = blockIdx.x;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kBulkStages; ++s) {
-      mbar_init(full + s, 1);
-      mbar_init(empty + s, 1);
-    }
-    abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncthreads();
-  volatile int* abort_v = &abort_flag;
-  if (warp == kBulkConsumers) {
-    if (L == 0) {  // producer
-      for (int64_t j = 0; b + j * G < Cfull; ++j) {
-        const int s = static_cast<int>(j % kBulkStages);
-        const uint32_t ph = static_cast<uint32_t>((j / kBulkStages) & 1);
-        if (!wait1(empty + s, ph ^ 1, kBulkWaitCycles, abort_v)) {
-          set_flag(hdr, kFlagTimeout, 0x601);
-          *abort_v = 1;
-          break;
-        }
-        mbar_expect_tx(full + s, CB);
-        bulk_load(smem + s * CB, static_cast<const uint8_t*>(W) + (b + j * G) * CB, CB, full + s);
-      }
-    }
-  } else {
-    // consumer group s (warps 4s .. 4s + 3) owns stage s
-    const int s = warp / kAbsWarpsPerStage, sub = warp % kAbsWarpsPerStage;
-    for (int64_t j = s; b + j * G < Cfull; j += kBulkStages) {
-      const uint32_t ph = static_cast<uint32_t>((j / kBulkStages) & 1);
-      const bool okw = wait_warp(full + s, ph, kBulkWaitCycles, abort_v);
-      if (!okw && L == 0) {
-        set_flag(hdr, kFlagTimeout, 0x602);
-        *abort_v = 1;
-      }
-      const double part = okw ? chunk_part_smem<WDT>(smem + s * CB, L, sub) : 0.0;
-      xchg[s][sub][L] = part;
-      // the four warps of the group meet here and agree whether to go on
-      uint32_t ok_all;
-      asm volatile(
-          "{\n\t.reg .pred pi, po;\n\t"
-          "setp.ne.u32 pi, %1, 0;\n\t"
-          "bar.red.and.pred po, %2, %3, pi;\n\t"
-          "selp.u32 %0, 1, 0, po;\n\t}"
-          : "=r"(ok_all)
-          : "r"(okw ? 1u : 0u), "r"(1 + s), "n"(32 * kAbsWarpsPerStage)
-          : "memory");
-      const bool ok = ok_all != 0;
-      if (sub == 0) {
-        double q0 = xchg[s][0][L], q1 = xchg[s][1][L];
-        const double q2 = xchg[s][2][L], q3 = xchg[s][3][L];
-        q0 = __dadd_rn(q0, q2);  // level 64
-        q1 = __dadd_rn(q1, q3);
-        double t = __dadd_rn(q0, q1);  // level 32
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) t = __dadd_rn(t, __shfl_down_sync(0xffffffffu, t, o));
-        if (L == 0) {
-          if (ok) partials[b + j * G] = t;
-          mbar_arrive(empty + s);  // the whole group has read the stage and the exchange slots
-        }
-      }
-      if (!ok) break;
-    }
-    if (warp == 0 && Cfull < C && (C - 1) % G == b) {  // the partial last chunk
-      const double t = chunk_sum_warp<WDT>(W, T, C - 1, L);
-      if (L == 0) partials[C - 1] = t;
-    }
-  }
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const unsigned ticket = atomicAdd(&hdr->ticket, 1u);
-    last = (ticket == gridDim.x - 1);
-  }
-  __syncthreads();
-  if (!last) return;
-
-  // ---- finish: this CTA is the last one; every partial is visible ----
-  // (the 256 residue classes are strided over the CTA's threads, whatever
-  // their number)
-  __threadfence();
+// The last CTA's combination of the C chunk sums into gamma (see above), by
+// the threads of the calling CTA whatever their number; p is a shared array of
+// kLanes doubles.  Resets the ticket for the next call on the workspace.
+__device__ __forceinline__ void absmean_finish(const double* __restrict__ partials, int64_t C, int lgR, int64_t T,
+                                               double* p, WsHeader* __restrict__ hdr, float* __restrict__ gamma) {
   const int64_t R = int64_t{1} << lgR;  // P / 256, or 1 when P <= 256
   for (int l = threadIdx.x; l < kLanes; l += blockDim.x) {
     double st[kFinishMaxLevels + 1];
@@ -309,6 +82,77 @@ __global__ void __launch_bounds__(kBulkThreads, 1)
       hdr->ticket = 0u;  // ready for the next call on this workspace
     }
   }
+}
+
+// Streaming absmean: persistent CTAs of 256 threads, kAbsCtasPerSm per SM;
+// thread l is lane l of the fixed order.  CTA b takes the chunks b, b + G, ...:
+// each thread loads its 32 elements of the chunk (the i = 0..3 runs of 8, as
+// 16-byte loads straight into registers) and adds them in order; the lane sums
+// go to a shared array (two copies, by chunk parity), one barrier, and warp
+// (k mod 8) of the CTA takes the chunk's tree (levels 128, 64, 32 in
+// registers, 16..1 by shuffles) while the other warps load the next chunk.
+// The copy written for chunk k is written again for chunk k + 2 only after the
+// barrier of chunk k + 1, which the tree warp of chunk k reaches after its
+// reads.  Reads from L2 or HBM straight to registers (no shared staging):
+// with 4 CTAs per SM, 128 KB per SM can be in flight.
+constexpr int kAbsCtasPerSm = 4;
+
+template <int WDT>
+__global__ void __launch_bounds__(kLanes, kAbsCtasPerSm)
+    absmean_kernel(const void* __restrict__ W, int64_t T, int64_t C, int lgR, double* __restrict__ partials,
+                   WsHeader* __restrict__ hdr, float* __restrict__ gamma) {
+  __shared__ double lsum[2][kLanes];
+  __shared__ double p[kLanes];
+  __shared__ bool last;
+  const int l = threadIdx.x, warp = l >> 5, L = l & 31;
+  const int64_t G = gridDim.x;
+  int k = 0;
+  for (int64_t c = blockIdx.x; c < C; c += G, ++k) {
+    const int64_t c0 = c * kChunk;
+    float v[4][8];
+    if (c0 + kChunk <= T) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) load8_aligned<WDT>(W, c0 + 2048 * i + 8 * l, v[i]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int64_t e0 = c0 + 2048 * i + 8 * l;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[i][j] = (e0 + j < T) ? load_elem<WDT>(W, e0 + j) : 0.0f;
+      }
+    }
+    double acc = 0.0;  // +0.0 for elements past T leaves the sum unchanged
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc = __dadd_rn(acc, static_cast<double>(fabsf(v[i][j])));
+    double* ls = lsum[k & 1];
+    ls[l] = acc;
+    __syncthreads();
+    if (warp == (k & 7)) {
+      double q[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) q[u] = ls[L + 32 * u];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) q[u] = __dadd_rn(q[u], q[u + 4]);  // level 128
+      q[0] = __dadd_rn(q[0], q[2]);                                   // level 64
+      q[1] = __dadd_rn(q[1], q[3]);
+      double t = __dadd_rn(q[0], q[1]);                               // level 32
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) t = __dadd_rn(t, __shfl_down_sync(0xffffffffu, t, o));
+      if (L == 0) partials[c] = t;
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned ticket = atomicAdd(&hdr->ticket, 1u);
+    last = (ticket == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  absmean_finish(partials, C, lgR, T, p, hdr, gamma);
 }
 
 // ---------------------------------------------------------------------------
@@ -431,120 +275,40 @@ __global__ void __launch_bounds__(256)
 
 // Flat 2-bit ternarize + pack, for K % 64 == 0.  The row stride is then K / 4
 // bytes with no padding, so packed byte p of the matrix holds the weights
-// 4p .. 4p + 3 of W in row-major order: each 8192-weight span of W becomes
-// 2048 consecutive packed bytes.  One persistent CTA per SM: a producer keeps
-// kBulkStages spans in flight with cp.async.bulk, walking the spans from the
-// end of W backwards (the absmean kernel streamed W front to back, so the
-// last spans it read are the likeliest to still be in L2); consumer warp w owns
-// stage w (as in the absmean kernel) and turns each staged span into packed
-// bytes (lane L takes weights 4(32a + L)..+3,
-// so the 16-byte shared loads of a warp are contiguous), collects them in its
-// own shared buffer and writes them with one bulk store.  A partial last span
-// is read directly from global memory.
+// 4p .. 4p + 3 of W in row-major order and the matrix is one stream.  A thread
+// turns a group of 16 consecutive weights (16-byte loads straight into
+// registers) into 4 packed bytes (one 32-bit store) and, if asked, 16 int8
+// codes (one 16-byte store); it keeps two groups in flight, and a persistent
+// grid of kTernCtasPerSm CTAs per SM walks the groups from the end of W
+// backwards (the absmean kernel streamed W front to back, so the last groups it
+// read are the likeliest to still be in L2).
+constexpr int kTernCtasPerSm = 4;
+
 template <int WDT>
-__global__ void __launch_bounds__(kTernThreads, 1)
-    ternarize_flat_kernel(const void* __restrict__ W, int64_t T, int64_t Sfull, const float* __restrict__ gamma,
-                          float eps, uint8_t* __restrict__ packed, int8_t* __restrict__ codes,
-                          WsHeader* __restrict__ hdr) {
-  constexpr int ES = (WDT == BL_F32) ? 4 : 2;
-  constexpr uint32_t CB = kChunk * ES;       // bytes of W per span
-  constexpr uint32_t OB = kChunk / 4;        // packed bytes per span
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* outb = smem + kBulkStages * CB;   // [kTernConsumers][OB]
-  uint64_t* full = reinterpret_cast<uint64_t*>(outb + kTernConsumers * OB);
-  uint64_t* empty = full + kBulkStages;
-  __shared__ int abort_flag;
-  const int warp = threadIdx.x >> 5, L = threadIdx.x & 31;
-  const int64_t G = gridDim.x, b = blockIdx.x;
+__global__ void __launch_bounds__(256, kTernCtasPerSm)
+    ternarize_flat_kernel(const void* __restrict__ W, int64_t T, const float* __restrict__ gamma, float eps,
+                          uint8_t* __restrict__ packed, int8_t* __restrict__ codes) {
   const float thr = ternary_threshold(__ldg(gamma), eps);
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kBulkStages; ++s) {
-      mbar_init(full + s, 1);
-      mbar_init(empty + s, 1);
-    }
-    abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncthreads();
-  volatile int* abort_v = &abort_flag;
-  if (warp == kTernConsumers) {
-    if (L == 0) {  // producer: spans Sfull - 1 - b - jG, j = 0, 1, ...
-      for (int64_t j = 0; b + j * G < Sfull; ++j) {
-        const int s = static_cast<int>(j % kBulkStages);
-        const uint32_t ph = static_cast<uint32_t>((j / kBulkStages) & 1);
-        if (!wait1(empty + s, ph ^ 1, kBulkWaitCycles, abort_v)) {
-          set_flag(hdr, kFlagTimeout, 0x611);
-          *abort_v = 1;
-          break;
-        }
-        const int64_t span = Sfull - 1 - (b + j * G);
-        mbar_expect_tx(full + s, CB);
-        bulk_load(smem + s * CB, static_cast<const uint8_t*>(W) + span * CB, CB, full + s);
-      }
-    }
-  } else {
-    uint8_t* ob = outb + warp * OB;
-    for (int64_t j = warp; b + j * G < Sfull; j += kTernConsumers) {
-      const int s = static_cast<int>(j % kBulkStages);
-      const uint32_t ph = static_cast<uint32_t>((j / kBulkStages) & 1);
-      if (!wait_warp(full + s, ph, kBulkWaitCycles, abort_v)) {
-        if (L == 0) {
-          set_flag(hdr, kFlagTimeout, 0x612);
-          *abort_v = 1;
-        }
-        break;
-      }
-      const int64_t span = Sfull - 1 - (b + j * G);
-      if (j >= kTernConsumers) {  // this warp's previous bulk store has read its buffer
-        if (L == 0) bulk_wait_read<0>();
-        __syncwarp();
-      }
-      const uint8_t* st = smem + s * CB;
-#pragma unroll 4
-      for (int a = 0; a < static_cast<int>(OB / 32); ++a) {
-        const int p = 32 * a + L;  // packed byte of the span
-        float v[4];
-        if constexpr (WDT == BL_F32) {
-          const float4 f = *reinterpret_cast<const float4*>(st + 16 * p);
-          v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
-        } else {
-          const uint2 u = *reinterpret_cast<const uint2*>(st + 8 * p);
-          v[0] = __uint_as_float(u.x << 16); v[1] = __uint_as_float(u.x & 0xffff0000u);
-          v[2] = __uint_as_float(u.y << 16); v[3] = __uint_as_float(u.y & 0xffff0000u);
-        }
-        uint32_t byte = 0, cw = 0;
+  const int64_t ng = T / 16;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t gi = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; gi < ng; gi += 2 * stride) {
+    float v[2][16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t d = ternary_digit(v[i], thr);
-          byte |= d << (2 * i);
-          cw |= ((d - 1u) & 0xffu) << (8 * i);
-        }
-        ob[p] = static_cast<uint8_t>(byte);
-        if (codes != nullptr) reinterpret_cast<uint32_t*>(codes + span * kChunk)[p] = cw;
-      }
-      __syncwarp();
-      if (L == 0) mbar_arrive(empty + s);  // the stage has been read
-      fence_proxy_async_smem();            // this lane's bytes are visible to the bulk store
-      __syncwarp();
-      if (L == 0) {
-        bulk_store(packed + span * OB, ob, OB);
-        bulk_commit();
-      }
+    for (int u = 0; u < 2; ++u) {
+      const int64_t g = ng - 1 - (gi + u * stride);
+      if (g >= 0) load16_aligned<WDT>(W, 16 * g, v[u]);
     }
-    if (L == 0) bulk_wait<0>();
-    if (warp == 0 && b == 0 && Sfull * kChunk < T) {  // the partial last span
-      const int64_t e0 = Sfull * kChunk, nbytes = (T - e0) / 4;
-      for (int64_t p = L; p < nbytes; p += 32) {
-        uint32_t byte = 0, cw = 0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t d = ternary_digit(load_elem<WDT>(W, e0 + 4 * p + i), thr);
-          byte |= d << (2 * i);
-          cw |= ((d - 1u) & 0xffu) << (8 * i);
-        }
-        packed[e0 / 4 + p] = static_cast<uint8_t>(byte);
-        if (codes != nullptr) *reinterpret_cast<uint32_t*>(codes + e0 + 4 * p) = cw;
-      }
+    for (int u = 0; u < 2; ++u) {
+      const int64_t g = ng - 1 - (gi + u * stride);
+      if (g < 0) continue;
+      uint32_t word = 0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) word |= ternary_digit(v[u][i], thr) << (2 * i);
+      reinterpret_cast<uint32_t*>(packed)[g] = word;
+      if (codes != nullptr)
+        reinterpret_cast<uint4*>(codes)[g] = make_uint4(codes4_word(v[u], thr), codes4_word(v[u] + 4, thr),
+                                                        codes4_word(v[u] + 8, thr), codes4_word(v[u] + 12, thr));
     }
   }
 }
@@ -628,28 +392,14 @@ cudaError_t launch_absmean(const void* W, int wdt, int64_t N, int64_t K, void* w
   if (lgR > kFinishMaxLevels) return cudaErrorInvalidValue;
   WsHeader* hdr = static_cast<WsHeader*>(ws);
   double* partials = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + BL_WS_HEADER_BYTES);
-  // bulk-staged path: one CTA per SM (at most one per chunk)
-  {
-    const int64_t Cfull = T / kChunk;
-    const int64_t grid = C < device_sms() ? C : device_sms();
-    const uint32_t cb = kChunk * (wdt == BL_F32 ? 4 : 2);
-    const size_t smem = static_cast<size_t>(kBulkStages) * cb + 16 * kBulkStages;
-    cudaError_t e;
-    if (wdt == BL_F32) {
-      e = cudaFuncSetAttribute(absmean_bulk_kernel<BL_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      absmean_bulk_kernel<BL_F32><<<static_cast<unsigned>(grid), kBulkThreads, smem, st>>>(W, T, C, Cfull, lgR,
-                                                                                        partials, hdr, gamma);
-    } else {
-      e = cudaFuncSetAttribute(absmean_bulk_kernel<BL_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      absmean_bulk_kernel<BL_BF16><<<static_cast<unsigned>(grid), kBulkThreads, smem, st>>>(W, T, C, Cfull, lgR,
-                                                                                         partials, hdr, gamma);
-    }
-    return cudaGetLastError();
-  }
+  // persistent streaming grid: kAbsCtasPerSm CTAs per SM (at most one per chunk)
+  const int64_t cap = static_cast<int64_t>(device_sms()) * kAbsCtasPerSm;
+  const int64_t grid = C < cap ? C : cap;
+  if (wdt == BL_F32)
+    absmean_kernel<BL_F32><<<static_cast<unsigned>(grid), kLanes, 0, st>>>(W, T, C, lgR, partials, hdr, gamma);
+  else
+    absmean_kernel<BL_BF16><<<static_cast<unsigned>(grid), kLanes, 0, st>>>(W, T, C, lgR, partials, hdr, gamma);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_ternarize_pack(const void* W, int wdt, int64_t N, int64_t K, const float* gamma,
@@ -657,24 +407,15 @@ cudaError_t launch_ternarize_pack(const void* W, int wdt, int64_t N, int64_t K, 
                                   cudaStream_t st) {
   if (fmt == BL_PACK_I2 && (K % 64) == 0 && packed != nullptr) {
     const int64_t T = N * K;
-    const int64_t Sfull = T / kChunk;
-    const int64_t grid = Sfull < 1 ? 1 : (Sfull < device_sms() ? Sfull : device_sms());
-    const uint32_t cb = kChunk * (wdt == BL_F32 ? 4 : 2);
-    const size_t smem = static_cast<size_t>(kBulkStages) * cb + kTernConsumers * (kChunk / 4) + 16 * kBulkStages;
-    cudaError_t e;
-    if (wdt == BL_F32) {
-      e = cudaFuncSetAttribute(ternarize_flat_kernel<BL_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      ternarize_flat_kernel<BL_F32><<<static_cast<unsigned>(grid), kTernThreads, smem, st>>>(
-          W, T, Sfull, gamma, eps, packed, codes, static_cast<WsHeader*>(ws));
-    } else {
-      e = cudaFuncSetAttribute(ternarize_flat_kernel<BL_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      ternarize_flat_kernel<BL_BF16><<<static_cast<unsigned>(grid), kTernThreads, smem, st>>>(
-          W, T, Sfull, gamma, eps, packed, codes, static_cast<WsHeader*>(ws));
-    }
+    const int64_t ng = T / 16;
+    const int64_t cap = static_cast<int64_t>(device_sms()) * kTernCtasPerSm;
+    int64_t grid = (ng + 511) / 512;  // two groups per thread
+    if (grid > cap) grid = cap;
+    if (grid < 1) grid = 1;
+    if (wdt == BL_F32)
+      ternarize_flat_kernel<BL_F32><<<static_cast<unsigned>(grid), 256, 0, st>>>(W, T, gamma, eps, packed, codes);
+    else
+      ternarize_flat_kernel<BL_BF16><<<static_cast<unsigned>(grid), 256, 0, st>>>(W, T, gamma, eps, packed, codes);
     return cudaGetLastError();
   }
   const bool vec_ok = (wdt == BL_F32) ? (K % 4 == 0) : (K % 8 == 0);
