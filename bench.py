@@ -540,7 +540,7 @@ def decode_summary(d):
             "launch_duration": "CUDA events at the two ends of a graph of back-to-back forward calls"}
 
 
-def gemv_kernel_name(fmt, layers):
+def gemv_kernel_name(fmt, layers, M=1):
     """The decode kernel the forward dispatches to (M <= 4): the lean 2-bit
     kernel for rows of at most 8192 packed bytes, else the general one."""
     lean = fmt == 0 and all(((K + 3) // 4 + 15) // 16 * 16 <= 8192 for (_, K) in layers)
@@ -653,7 +653,7 @@ def main():
         flat = wl["fmt"] == 0 and all(K % 64 == 0 for (_, K) in wl["layers"])
         kernel_name = {"absmean": "absmean_kernel",
                        "ternarize_pack": "ternarize_flat_kernel" if flat else "ternarize_pack_kernel",
-                       "forward": gemv_kernel_name(wl["fmt"], wl["layers"])}[dom]
+                       "forward": gemv_kernel_name(wl["fmt"], wl["layers"], wl["M"])}[dom]
         traffic = profiled_traffic(kernel_name, args.workload)
         cpu = None
         if args.cpu_budget > 0 and world == 1:

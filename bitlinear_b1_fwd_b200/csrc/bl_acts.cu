@@ -2,19 +2,107 @@
 //
 // "BitNet b1.58深度解析：三值权重如何重塑大模型推理" §3.2 and §5.2: each token
 // (one row of x over K) is scaled by its own max |x| (floored at 1e-6) and
-// x_q = clamp(round(x / s * 127), -127, 127).  One warp per token: a max
-// reduction (warp shuffles) and a second pass that writes
-// the INT8 codes, 8 per lane-iteration, with 16-byte loads when K allows.
+// x_q = clamp(round(x / s * 127), -127, 127).  Rows of up to 8 K (bf16) or
+// 4 K (fp32) elements: one CTA per token, read once into registers.  Other
+// rows: one warp per token, two passes whose loads go out kActBatch at a time.
 #include "bl_common.cuh"
 #include "bl_kernels.h"
 
 namespace bl {
 
 constexpr int kActThreads = 256;
+constexpr int kActBatch = 4;  // 16-byte loads in flight per lane in the two-pass kernel
 
-// One warp per token: the absmax over the row (16-byte loads, warp shuffles),
-// then a second pass over the same row (mostly L1 hits) that writes the codes,
-// 8 per lane-iteration.  No shared memory, no block barriers.
+__device__ __forceinline__ uint2 codes8(const float* e, float s, float c127) {
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    lo |= static_cast<uint32_t>(quant_act_fast(e[j], s, c127) & 0xff) << (8 * j);
+    hi |= static_cast<uint32_t>(quant_act_fast(e[j + 4], s, c127) & 0xff) << (8 * j);
+  }
+  return make_uint2(lo, hi);
+}
+
+__device__ __forceinline__ void bf16x8(const uint4 r, float* e) {
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    e[2 * i] = __uint_as_float(w[i] << 16);
+    e[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// Rows with K % 8 == 0 (bf16) or K % 4 == 0 (fp32) and at most
+// kActRowThreads NV 16-byte words: one CTA per token, read once.  Thread t
+// issues its NV loads (words t, t + T, ...) together; the absmax meets across
+// the CTA (warp shuffles, one barrier) and the codes come from registers.
+// Many small CTAs per SM, each at its own phase, keep loads in flight while
+// others compute.
+constexpr int kActRowThreads = 128;
+
+template <int XDT, int NV>
+__global__ void __launch_bounds__(kActRowThreads)
+    act_quant_row_kernel(const void* __restrict__ x, int64_t M, int64_t K, int8_t* __restrict__ xq,
+                         float* __restrict__ scale) {
+  constexpr int EPW = (XDT == BL_F32) ? 4 : 8;  // elements per 16-byte word
+  __shared__ float red[kActRowThreads / 32];
+  const int t = threadIdx.x, lane = t & 31;
+  const int nv = static_cast<int>(K / EPW);
+  for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+    const uint4* row = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(x) + m * K * (16 / EPW));
+    uint4 r[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int v = t + kActRowThreads * i;
+      r[i] = v < nv ? __ldg(row + v) : make_uint4(0, 0, 0, 0);
+    }
+    auto elems = [&](int i, float* e) {
+      if constexpr (XDT == BL_F32) {
+        e[0] = __uint_as_float(r[i].x); e[1] = __uint_as_float(r[i].y);
+        e[2] = __uint_as_float(r[i].z); e[3] = __uint_as_float(r[i].w);
+      } else {
+        bf16x8(r[i], e);
+      }
+    };
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      float e[8];
+      elems(i, e);
+#pragma unroll
+      for (int j = 0; j < EPW; ++j) amax = fmaxf(amax, fabsf(e[j]));
+    }
+    amax = warp_maxf(amax);
+    if (lane == 0) red[t >> 5] = amax;
+    __syncthreads();
+    float a = red[0];
+#pragma unroll
+    for (int w = 1; w < kActRowThreads / 32; ++w) a = fmaxf(a, red[w]);
+    __syncthreads();  // red is free for the next token
+    const float s = fmaxf(a, 1e-6f);
+    const float c127 = __fdiv_rn(127.0f, s);
+    int8_t* out = xq + m * K;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int v = t + kActRowThreads * i;
+      if (v < nv) {
+        float e[8];
+        elems(i, e);
+        if constexpr (XDT == BL_F32) {
+          uint32_t w = 0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) w |= static_cast<uint32_t>(quant_act_fast(e[j], s, c127) & 0xff) << (8 * j);
+          reinterpret_cast<uint32_t*>(out)[v] = w;
+        } else {
+          reinterpret_cast<uint2*>(out)[v] = codes8(e, s, c127);
+        }
+      }
+    }
+    if (t == 0) scale[m] = s;
+  }
+}
+
+// Any row: the absmax pass and the code pass, kActBatch loads per lane in flight.
 template <int XDT>
 __global__ void __launch_bounds__(kActThreads)
     act_quant_kernel(const void* __restrict__ x, int64_t M, int64_t K, int8_t* __restrict__ xq,
@@ -22,16 +110,27 @@ __global__ void __launch_bounds__(kActThreads)
   const int lane = threadIdx.x & 31;
   const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t tw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t nv = K / 8;
   for (int64_t m = gw; m < M; m += tw) {
     const int64_t base = m * K;
     float amax = 0.0f;
     if (vec) {
-#pragma unroll 4
-      for (int64_t v = lane; v < K / 8; v += 32) {
-        float e[8];
-        load8_aligned<XDT>(x, base + 8 * v, e);
+      for (int64_t v0 = lane; v0 < nv; v0 += 32 * kActBatch) {
+        float e[kActBatch][8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(e[j]));
+        for (int b = 0; b < kActBatch; ++b) {
+          const int64_t v = v0 + 32 * b;
+          if (v < nv) {
+            load8_aligned<XDT>(x, base + 8 * v, e[b]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) e[b][j] = 0.0f;
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < kActBatch; ++b)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(e[b][j]));
       }
     } else {
       for (int64_t k = lane; k < K; k += 32) amax = fmaxf(amax, fabsf(load_elem<XDT>(x, base + k)));
@@ -40,17 +139,18 @@ __global__ void __launch_bounds__(kActThreads)
     const float s = fmaxf(amax, 1e-6f);
     const float c127 = __fdiv_rn(127.0f, s);
     if (vec) {
-#pragma unroll 4
-      for (int64_t v = lane; v < K / 8; v += 32) {
-        float e[8];
-        load8_aligned<XDT>(x, base + 8 * v, e);
-        uint32_t lo = 0, hi = 0;
+      for (int64_t v0 = lane; v0 < nv; v0 += 32 * kActBatch) {
+        float e[kActBatch][8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          lo |= static_cast<uint32_t>(quant_act_fast(e[j], s, c127) & 0xff) << (8 * j);
-          hi |= static_cast<uint32_t>(quant_act_fast(e[j + 4], s, c127) & 0xff) << (8 * j);
+        for (int b = 0; b < kActBatch; ++b) {
+          const int64_t v = v0 + 32 * b;
+          if (v < nv) load8_aligned<XDT>(x, base + 8 * v, e[b]);
         }
-        *reinterpret_cast<uint2*>(xq + base + 8 * v) = make_uint2(lo, hi);
+#pragma unroll
+        for (int b = 0; b < kActBatch; ++b) {
+          const int64_t v = v0 + 32 * b;
+          if (v < nv) *reinterpret_cast<uint2*>(xq + base + 8 * v) = codes8(e[b], s, c127);
+        }
       }
     } else {
       for (int64_t k = lane; k < K; k += 32)
@@ -64,13 +164,46 @@ cudaError_t launch_act_quant(const void* x, int xdt, int64_t M, int64_t K, int8_
                              cudaStream_t st) {
   const int64_t warps_per_cta = kActThreads / 32;
   const int64_t need = (M + warps_per_cta - 1) / warps_per_cta;
-  const int64_t cap = static_cast<int64_t>(device_sms()) * (2048 / kActThreads);
-  const unsigned grid = static_cast<unsigned>(need < cap ? need : cap);
+  auto grid_for = [&](const void* kern) -> unsigned {
+    int per_sm = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kActThreads, 0) != cudaSuccess ||
+        per_sm < 1)
+      per_sm = 1;
+    const int64_t cap = static_cast<int64_t>(device_sms()) * per_sm;
+    return static_cast<unsigned>(need < cap ? need : cap);
+  };
   const bool vec = (K % 8) == 0;
+  const int epw = (xdt == BL_F32) ? 4 : 8;
+  const int64_t nv = K / epw;
+  if ((K % epw) == 0 && nv <= kActRowThreads * 8) {
+    int per_sm = 1;
+#define BL_AQ(XDT, NV)                                                                                  \
+  if (nv <= kActRowThreads * (NV)) {                                                                    \
+    auto kern = act_quant_row_kernel<XDT, NV>;                                                          \
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kActRowThreads, 0) != cudaSuccess || \
+        per_sm < 1)                                                                                     \
+      per_sm = 1;                                                                                       \
+    const int64_t cap = static_cast<int64_t>(device_sms()) * per_sm;                                    \
+    kern<<<static_cast<unsigned>(M < cap ? M : cap), kActRowThreads, 0, st>>>(x, M, K, xq, scale);      \
+    return cudaGetLastError();                                                                          \
+  }
+    if (xdt == BL_F32) {
+      BL_AQ(BL_F32, 2)
+      BL_AQ(BL_F32, 4)
+      BL_AQ(BL_F32, 8)
+    } else {
+      BL_AQ(BL_BF16, 2)
+      BL_AQ(BL_BF16, 4)
+      BL_AQ(BL_BF16, 8)
+    }
+#undef BL_AQ
+  }
   if (xdt == BL_F32)
-    act_quant_kernel<BL_F32><<<grid, kActThreads, 0, st>>>(x, M, K, xq, scale, vec);
+    act_quant_kernel<BL_F32><<<grid_for(reinterpret_cast<const void*>(act_quant_kernel<BL_F32>)), kActThreads, 0,
+                               st>>>(x, M, K, xq, scale, vec);
   else
-    act_quant_kernel<BL_BF16><<<grid, kActThreads, 0, st>>>(x, M, K, xq, scale, vec);
+    act_quant_kernel<BL_BF16><<<grid_for(reinterpret_cast<const void*>(act_quant_kernel<BL_BF16>)), kActThreads,
+                                0, st>>>(x, M, K, xq, scale, vec);
   return cudaGetLastError();
 }
 

@@ -67,16 +67,6 @@ __device__ __forceinline__ int quant_act(float x, float s) {
   return __float2int_rn(t);
 }
 
-// |x| widened to fp64 exactly, with integer operations for normal values (the
-// fp32 exponent rebiased by 1023 - 127 = 896, the significand moved up by
-// 29 bits); zeros and subnormals take the conversion instruction.
-__device__ __forceinline__ double widen_abs(float x) {
-  const uint32_t a = __float_as_uint(x) & 0x7fffffffu;
-  if (a < 0x00800000u) return a == 0u ? 0.0 : static_cast<double>(__uint_as_float(a));
-  const unsigned long long b = (static_cast<unsigned long long>(a) << 29) + (896ull << 52);
-  return __longlong_as_double(static_cast<long long>(b));
-}
-
 // Round to the nearest integer, ties to even, for |t| < 2^22: adding 1.5 * 2^23
 // rounds in the adder (round-to-nearest-even) and leaves the integer in the low
 // significand bits.  Returns the rounded value as float and as int.
@@ -86,17 +76,19 @@ __device__ __forceinline__ float round_magic(float t, int* qi) {
   return __fsub_rn(r, 12582912.0f);
 }
 
-// The same code as quant_act without a division per element.  With
-// c127 = fl(127 / s), t_a = fl(x c127) differs from t = fl(fl(x / s) 127) by
-// less than 4.0001 * 2^-24 |t| (two roundings on each side), so when t_a is
-// farther than |t_a| 2^-21 from every half-integer both round to the same
-// integer and t is not a tie; otherwise (rare) the exact quotient decides.
+// The same code as quant_act without a division per element, for |x| <= s.
+// With c127 = fl(127 / s), t_a = fl(x c127) differs from t = fl(fl(x / s) 127)
+// by less than 4.0001 * 2^-24 |t| (two roundings on each side), and
+// |t_a| <= 127 (1 + 2^-22), so |t_a - t| < 2^-14: when t_a is farther than
+// 2^-14 from every half-integer (|t_a - rint(t_a)| < 1/2 - 2^-14; the
+// difference is exact) both round to the same integer, t is not a tie, and
+// the code is within [-127, 127] with no clamp; otherwise (rare) the exact
+// quotient decides.
 __device__ __forceinline__ int quant_act_fast(float x, float s, float c127) {
-  const float ta = __fmul_rn(x, c127);  // |ta| <= 127 (1 + 2^-22): the magic rounding applies
+  const float ta = __fmul_rn(x, c127);
   int qi;
   const float qa = round_magic(ta, &qi);
-  const float dist = __fsub_rn(0.5f, fabsf(__fsub_rn(ta, qa)));  // to the nearest half-integer
-  if (dist > __fmaf_rn(fabsf(ta), 0x1p-21f, 0x1p-126f)) return min(max(qi, -127), 127);
+  if (fabsf(__fsub_rn(ta, qa)) < 0.49993896484375f) return qi;
   return quant_act(x, s);
 }
 
