@@ -13,14 +13,14 @@ namespace bl {
 constexpr int kActThreads = 256;
 constexpr int kActBatch = 4;  // 16-byte loads in flight per lane in the two-pass kernel
 
+__device__ __forceinline__ uint32_t pack_codes4(const int* q) {
+  return __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
+}
+
 __device__ __forceinline__ uint2 codes8(const float* e, float s, float c127) {
-  uint32_t lo = 0, hi = 0;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    lo |= static_cast<uint32_t>(quant_act_fast(e[j], s, c127) & 0xff) << (8 * j);
-    hi |= static_cast<uint32_t>(quant_act_fast(e[j + 4], s, c127) & 0xff) << (8 * j);
-  }
-  return make_uint2(lo, hi);
+  int q[8];
+  quant_act_fast_n<8>(e, s, c127, q);
+  return make_uint2(pack_codes4(q), pack_codes4(q + 4));
 }
 
 __device__ __forceinline__ void bf16x8(const uint4 r, float* e) {
@@ -89,10 +89,9 @@ __global__ void __launch_bounds__(kActRowThreads)
         float e[8];
         elems(i, e);
         if constexpr (XDT == BL_F32) {
-          uint32_t w = 0;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) w |= static_cast<uint32_t>(quant_act_fast(e[j], s, c127) & 0xff) << (8 * j);
-          reinterpret_cast<uint32_t*>(out)[v] = w;
+          int q[4];
+          quant_act_fast_n<4>(e, s, c127, q);
+          reinterpret_cast<uint32_t*>(out)[v] = pack_codes4(q);
         } else {
           reinterpret_cast<uint2*>(out)[v] = codes8(e, s, c127);
         }

@@ -84,12 +84,33 @@ __device__ __forceinline__ float round_magic(float t, int* qi) {
 // difference is exact) both round to the same integer, t is not a tie, and
 // the code is within [-127, 127] with no clamp; otherwise (rare) the exact
 // quotient decides.
+static __device__ __noinline__ int quant_act_slow(float x, float s) { return quant_act(x, s); }
+
 __device__ __forceinline__ int quant_act_fast(float x, float s, float c127) {
   const float ta = __fmul_rn(x, c127);
   int qi;
   const float qa = round_magic(ta, &qi);
   if (fabsf(__fsub_rn(ta, qa)) < 0.49993896484375f) return qi;
-  return quant_act(x, s);
+  return quant_act_slow(x, s);
+}
+
+// The codes of N elements (N <= 32) by the rule above, the exact quotient
+// taken in one rare branch for the elements near a tie only (so the common
+// case evaluates no division).
+template <int N>
+__device__ __forceinline__ void quant_act_fast_n(const float* e, float s, float c127, int* q) {
+  uint32_t near = 0;
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    const float ta = __fmul_rn(e[j], c127);
+    const float qa = round_magic(ta, &q[j]);
+    if (!(fabsf(__fsub_rn(ta, qa)) < 0.49993896484375f)) near |= 1u << j;
+  }
+  if (near != 0) {
+#pragma unroll
+    for (int j = 0; j < N; ++j)
+      if ((near >> j) & 1u) q[j] = quant_act_slow(e[j], s);
+  }
 }
 
 // Dequantization factor c = (gamma * s) / 127 and the dequantized value.

@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
               float e[8];
               load8_aligned<XDT>(x, m * K + kh, e);
 #pragma unroll
-              for (int j = 0; j < 8; ++j) q[j] = quant_act_fast(e[j], s_tok[m], c127);
+              quant_act_fast_n<8>(e, s_tok[m], c127, q);
             }
           } else {
 #pragma unroll
@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
           float e[8];
           load8_aligned<XDT>(x, m * K + 8 * v, e);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) q[j] = quant_act_fast(e[j], s_tok[m], c127);
+          quant_act_fast_n<8>(e, s_tok[m], c127, q);
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -489,92 +489,166 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     }
   };
 
-  // 1. the first tile's first batch goes out before the prologue
+  // 1. one token of bf16 or int8 (K % 16 == 0): each thread's activation loads
+  //    go out first and x is read once; the first batch of weights follows
+  //    once the codes are written (weight loads issued earlier delay the
+  //    activations and stall the prologue's warps at the load instructions).
+  //    Otherwise the first batch of weights goes out before the prologue.
+  constexpr bool kOnePassType = (MT == 1) && (XDT == BL_BF16 || XDT == BL_I8);
+  constexpr int kXW = (XDT == BL_BF16) ? 2 : 1;  // 16-byte words per 16 activations
+  const bool one_pass = kOnePassType && (K % 16) == 0;
+  uint4 xraw[3][kXW];  // packed words g = tid + 768 u: 4 segs <= 2048 words (rows <= 8 KB)
+  const float g_w = __ldg(gamma);  // (loaded with the activations, ahead of the weight stream)
+  if (one_pass) {
+#pragma unroll
+    for (int u = 0; u < 3; ++u) {
+      const int64_t k0 = 16 * (static_cast<int64_t>(threadIdx.x) + static_cast<int64_t>(kGemvThreads) * u);
+#pragma unroll
+      for (int i = 0; i < kXW; ++i)
+        xraw[u][i] = k0 < K ? __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(x) + k0 * kXW) + i)
+                            : make_uint4(0, 0, 0, 0);
+    }
+  }
   start_tile(0);
   uint4 bufA[kI2Batch][2], bufB[kI2Batch][2];
-  issue(bufA);
+  if (!one_pass) issue(bufA);
 
   // 2. prologue: per-token absmax, then the INT8 codes in the plane layout
   for (int i = threadIdx.x; i < MT * kGemvTileRows; i += blockDim.x) racc[i] = 0;
   float s_tok[MT];
-  if constexpr (XDT != BL_I8) {
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
+  if (one_pass) {
+    // the absmax (bf16) and the codes from the registers loaded above
+    auto elem = [&](int u, int jj) -> float {  // bf16 element jj (0..15) of word u
+      const uint4 w4 = xraw[u][(jj >> 3) % kXW];
+      const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+      const uint32_t wd = wv[(jj >> 1) & 3];
+      return __uint_as_float((jj & 1) ? (wd & 0xffff0000u) : (wd << 16));
+    };
+    if constexpr (XDT == BL_BF16) {
       float amax = 0.0f;
-      if ((K % 8) == 0) {
-        for (int64_t v = threadIdx.x; v < K / 8; v += blockDim.x) {
-          float e[8];
-          load8_aligned<XDT>(x, m * K + 8 * v, e);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(e[j]));
-        }
-      } else {
-        for (int64_t k = threadIdx.x; k < K; k += blockDim.x) amax = fmaxf(amax, fabsf(load_x<XDT>(x, m * K + k)));
-      }
+      for (int u = 0; u < 3; ++u)
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) amax = fmaxf(amax, fabsf(elem(u, jj)));
       amax = warp_maxf(amax);
-      if (lane == 0) red_f[m][warp] = amax;
-    }
-  }
-  __syncthreads();  // zeroed row sums and per-warp maxima are visible
-#pragma unroll
-  for (int m = 0; m < MT; ++m) {
-    if constexpr (XDT != BL_I8) {
-      float a = red_f[m][0];
-#pragma unroll
-      for (int w = 1; w < kGemvWarps; ++w) a = fmaxf(a, red_f[m][w]);
-      s_tok[m] = fmaxf(a, 1e-6f);
+      if (lane == 0) red_f[0][warp] = amax;
+      __syncthreads();  // zeroed row sums and per-warp maxima are visible
+      s_tok[0] = fmaxf(warp_maxf(lane < kGemvWarps ? red_f[0][lane] : 0.0f), 1e-6f);
     } else {
-      s_tok[m] = __ldg(scale + m);
+      s_tok[0] = __ldg(scale);
     }
-  }
-#pragma unroll
-  for (int m = 0; m < MT; ++m) {
+    const float c127 = (XDT == BL_I8) ? 0.0f : __fdiv_rn(127.0f, s_tok[0]);
     int part = 0;
-    uint8_t* xm = xs + m * 8 * kI2Plane;
-    const float c127 = (XDT == BL_I8) ? 0.0f : __fdiv_rn(127.0f, s_tok[m]);
-    for (uint32_t g = threadIdx.x; g < 4 * segs; g += blockDim.x) {  // one packed word's 16 codes
-      const int64_t k0 = 16 * static_cast<int64_t>(g);
-      const bool full = k0 + 16 <= K && (K % 16) == 0;
+#pragma unroll
+    for (int u = 0; u < 3; ++u) {
+      const uint32_t g = threadIdx.x + kGemvThreads * u;
+      if (g >= 4 * segs) break;
       uint32_t P[4];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int64_t kh = k0 + 8 * h;
+      for (int hh = 0; hh < 2; ++hh) {  // eight codes at a time
         int q[8];
-        if (full) {
-          if constexpr (XDT == BL_I8) {
-            const uint2 raw = __ldg(reinterpret_cast<const uint2*>(static_cast<const int8_t*>(x) + m * K + kh));
+        if constexpr (XDT == BL_I8) {
+          const uint4 w4 = xraw[u][0];
+          const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-            for (int j = 0; j < 8; ++j) q[j] = static_cast<int8_t>((j < 4 ? raw.x : raw.y) >> (8 * (j & 3)));
-          } else {
-            float e[8];
-            load8_aligned<XDT>(x, m * K + kh, e);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) q[j] = quant_act_fast(e[j], s_tok[m], c127);
-          }
+          for (int jj = 0; jj < 8; ++jj) q[jj] = static_cast<int8_t>(wv[2 * hh + (jj >> 2)] >> (8 * (jj & 3)));
         } else {
+          float e[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int64_t k = kh + j;
-            if (k < K)
-              q[j] = (XDT == BL_I8) ? static_cast<int>(static_cast<const int8_t*>(x)[m * K + k])
-                                    : quant_act_fast(load_x<XDT>(x, m * K + k), s_tok[m], c127);
-            else
-              q[j] = 0;
-          }
+          for (int jj = 0; jj < 8; ++jj) e[jj] = elem(u, 8 * hh + jj);  // 0 past K: a padding word codes 0
+          quant_act_fast_n<8>(e, s_tok[0], c127, q);
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) part += q[j];
-        P[2 * h] = pack4(q);
-        P[2 * h + 1] = pack4(q + 4);
+        for (int jj = 0; jj < 8; ++jj) part += q[jj];
+        P[2 * hh] = pack4(q);
+        P[2 * hh + 1] = pack4(q + 4);
       }
       const uint32_t s = g >> 2, w = g & 3;
-      *reinterpret_cast<uint4*>(xm + (2 * w + (s & 1)) * kI2Plane + (s >> 1) * 16) = i2_slot(P[0], P[1], P[2], P[3]);
+      *reinterpret_cast<uint4*>(xs + (2 * w + (s & 1)) * kI2Plane + (s >> 1) * 16) = i2_slot(P[0], P[1], P[2], P[3]);
     }
     part = __reduce_add_sync(0xffffffffu, part);
-    if (lane == 0) red_i[m][warp] = part;
+    if (lane == 0) red_i[0][warp] = part;
+    issue(bufA);  // the codes are written: now the first batch of weights
+  } else {
+    if constexpr (XDT != BL_I8) {
+  #pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        float amax = 0.0f;
+        if ((K % 8) == 0) {
+          for (int64_t v = threadIdx.x; v < K / 8; v += blockDim.x) {
+            float e[8];
+            load8_aligned<XDT>(x, m * K + 8 * v, e);
+  #pragma unroll
+            for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(e[j]));
+          }
+        } else {
+          for (int64_t k = threadIdx.x; k < K; k += blockDim.x) amax = fmaxf(amax, fabsf(load_x<XDT>(x, m * K + k)));
+        }
+        amax = warp_maxf(amax);
+        if (lane == 0) red_f[m][warp] = amax;
+      }
+    }
+    __syncthreads();  // zeroed row sums and per-warp maxima are visible
+  #pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      if constexpr (XDT != BL_I8) {
+        float a = red_f[m][0];
+  #pragma unroll
+        for (int w = 1; w < kGemvWarps; ++w) a = fmaxf(a, red_f[m][w]);
+        s_tok[m] = fmaxf(a, 1e-6f);
+      } else {
+        s_tok[m] = __ldg(scale + m);
+      }
+    }
+  #pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      int part = 0;
+      uint8_t* xm = xs + m * 8 * kI2Plane;
+      const float c127 = (XDT == BL_I8) ? 0.0f : __fdiv_rn(127.0f, s_tok[m]);
+      for (uint32_t g = threadIdx.x; g < 4 * segs; g += blockDim.x) {  // one packed word's 16 codes
+        const int64_t k0 = 16 * static_cast<int64_t>(g);
+        const bool full = k0 + 16 <= K && (K % 16) == 0;
+        uint32_t P[4];
+  #pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int64_t kh = k0 + 8 * h;
+          int q[8];
+          if (full) {
+            if constexpr (XDT == BL_I8) {
+              const uint2 raw = __ldg(reinterpret_cast<const uint2*>(static_cast<const int8_t*>(x) + m * K + kh));
+  #pragma unroll
+              for (int j = 0; j < 8; ++j) q[j] = static_cast<int8_t>((j < 4 ? raw.x : raw.y) >> (8 * (j & 3)));
+            } else {
+              float e[8];
+              load8_aligned<XDT>(x, m * K + kh, e);
+  #pragma unroll
+              quant_act_fast_n<8>(e, s_tok[m], c127, q);
+            }
+          } else {
+  #pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int64_t k = kh + j;
+              if (k < K)
+                q[j] = (XDT == BL_I8) ? static_cast<int>(static_cast<const int8_t*>(x)[m * K + k])
+                                      : quant_act_fast(load_x<XDT>(x, m * K + k), s_tok[m], c127);
+              else
+                q[j] = 0;
+            }
+          }
+  #pragma unroll
+          for (int j = 0; j < 8; ++j) part += q[j];
+          P[2 * h] = pack4(q);
+          P[2 * h + 1] = pack4(q + 4);
+        }
+        const uint32_t s = g >> 2, w = g & 3;
+        *reinterpret_cast<uint4*>(xm + (2 * w + (s & 1)) * kI2Plane + (s >> 1) * 16) = i2_slot(P[0], P[1], P[2], P[3]);
+      }
+      part = __reduce_add_sync(0xffffffffu, part);
+      if (lane == 0) red_i[m][warp] = part;
+    }
   }
   __syncthreads();  // activations and per-warp sums are visible
-  const float g = __ldg(gamma);
+  const float g = g_w;
   float cfac[MT];
   int corr[MT];
 #pragma unroll
