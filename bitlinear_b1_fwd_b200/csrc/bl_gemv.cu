@@ -122,7 +122,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t segs = static_cast<uint32_t>(rowbytes >> 4);
-  const uint32_t nb = (segs + 31) >> 5;  // 32-segment blocks per row
   const int64_t G = gridDim.x, b = blockIdx.x;
   const int64_t per = N / G, extra = N % G;
   const int64_t row0 = b * per + (b < extra ? b : extra);
@@ -235,8 +234,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
             } else {
               float e[8];
               load8_aligned<XDT>(x, m * K + kh, e);
-#pragma unroll
-              quant_act_fast_n<8>(e, s_tok[m], c127, q);
+quant_act_fast_n<8>(e, s_tok[m], c127, q);
             }
           } else {
 #pragma unroll
@@ -267,7 +265,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
         } else {
           float e[8];
           load8_aligned<XDT>(x, m * K + 8 * v, e);
-#pragma unroll
           quant_act_fast_n<8>(e, s_tok[m], c127, q);
         }
 #pragma unroll
@@ -621,8 +618,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
             } else {
               float e[8];
               load8_aligned<XDT>(x, m * K + kh, e);
-  #pragma unroll
-              quant_act_fast_n<8>(e, s_tok[m], c127, q);
+  quant_act_fast_n<8>(e, s_tok[m], c127, q);
             }
           } else {
   #pragma unroll
