@@ -21,6 +21,7 @@
 // wait is bounded: on expiry the kernel sets the workspace timeout flag, drains
 // what it issued, frees its tensor memory and returns.
 #include <cuda.h>
+#include <cstring>
 
 #include "bl_common.cuh"
 #include "bl_kernels.h"
@@ -359,14 +360,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // CTAs report to the leader by remote arrives.  MMA completion is committed to
 // the barriers of both CTAs.  Every wait is bounded as in the one-SM kernel.
 // ---------------------------------------------------------------------------
-constexpr int kStages2 = 6;
+constexpr int kStagesA = 7;  // TMA ring: x half + packed tile per stage
+constexpr int kStagesB = 3;  // expanded-weight ring
+constexpr uint32_t kYStage = 32 * 128 * 4;  // output staging: 32 tokens x 128 rows, up to 4 bytes each
 
 template <int BT>
 struct Gemm2Cfg {
   static constexpr uint32_t kXHalf = (BT / 2) * 128;
   static constexpr uint32_t kTmemCols = 2 * BT;  // BT >= 128: a power of two
-  static constexpr size_t kSmem =
-      1024 + kStages2 * (kXHalf + kExpStage + kPackedStage) + 8 * (4 * kStages2 + 5) + 16 + 2 * 4 * BT;
+  static constexpr size_t kSmem = 1024 + kStagesB * kExpStage + kStagesA * (kXHalf + kPackedStage) +
+                                  2 * kYStage + 8 * (3 * kStagesA + 2 * kStagesB + 5) + 16 + 2 * 4 * BT;
 };
 
 __device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -392,20 +395,23 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t mask) {
 template <int BT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_i2_2sm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                       const float* __restrict__ gamma, const float* __restrict__ scale, void* __restrict__ y,
-                       int ydt, int M, int N, int K, WsHeader* __restrict__ hdr, long long limit) {
+                       const __grid_constant__ CUtensorMap tm_y, int y_tma, const float* __restrict__ gamma,
+                       const float* __restrict__ scale, void* __restrict__ y, int ydt, int M, int N, int K,
+                       WsHeader* __restrict__ hdr, long long limit) {
   using Cfg = Gemm2Cfg<BT>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* base = smem_raw + pad;
-  uint8_t* xs = base;                              // kStages2 x [BT/2 x 128 B], swizzled
-  uint8_t* es = xs + kStages2 * Cfg::kXHalf;       // kStages2 x [128 x 128 B], swizzled
-  uint8_t* ps = es + kStages2 * kExpStage;         // kStages2 x [128 x 32 B]
-  uint64_t* xfull = reinterpret_cast<uint64_t*>(ps + kStages2 * kPackedStage);  // leader: x of both CTAs
-  uint64_t* pfull = xfull + kStages2;              // local: packed tile
-  uint64_t* expd = pfull + kStages2;               // leader: expansion of both CTAs (8 warps)
-  uint64_t* empty = expd + kStages2;               // local: the MMAs read the stage
-  uint64_t* accf = empty + kStages2;               // local: accumulator ready (2)
+  uint8_t* es = base;                              // kStagesB x [128 x 128 B], swizzled
+  uint8_t* xs = es + kStagesB * kExpStage;         // kStagesA x [BT/2 x 128 B], swizzled
+  uint8_t* ps = xs + kStagesA * Cfg::kXHalf;       // kStagesA x [128 x 32 B]
+  uint8_t* ystage = ps + kStagesA * kPackedStage;  // 2 x [32 tokens x 128 rows] output staging
+  uint64_t* xfull = reinterpret_cast<uint64_t*>(ystage + 2 * kYStage);  // leader: x of both CTAs
+  uint64_t* pfull = xfull + kStagesA;              // local: packed tile
+  uint64_t* emptyA = pfull + kStagesA;             // local: MMAs read x, expansion read packed (1 + 4)
+  uint64_t* expd = emptyA + kStagesA;              // leader: expansion of both CTAs (8 warps)
+  uint64_t* emptyB = expd + kStagesB;              // local: the MMAs read the expanded stage
+  uint64_t* accf = emptyB + kStagesB;              // local: accumulator ready (2)
   uint64_t* acce = accf + 2;                       // leader: epilogues of both CTAs done (2)
   uint64_t* drain = acce + 2;                      // leader
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -422,11 +428,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const int pair = blockIdx.x >> 1, pairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages2; ++s) {
+    for (int s = 0; s < kStagesA; ++s) {
       mbar_init(xfull + s, 1);
       mbar_init(pfull + s, 1);
+      mbar_init(emptyA + s, 1 + 4);
+    }
+    for (int s = 0; s < kStagesB; ++s) {
       mbar_init(expd + s, 8);
-      mbar_init(empty + s, 1);
+      mbar_init(emptyB + s, 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(accf + a, 1);
@@ -460,9 +469,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       for (int tile = pair; tile < tiles && ok; tile += pairs) {
         const int n_t = tile % n_tiles, t_t = tile / n_tiles;
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
-          const int s = it % kStages2;
-          const uint32_t ph = (it / kStages2) & 1;
-          if (!wait1(empty + s, ph ^ 1, limit, abort_flag)) {
+          const int s = it % kStagesA;
+          const uint32_t ph = (it / kStagesA) & 1;
+          if (!wait1(emptyA + s, ph ^ 1, limit, abort_flag)) {
             fail(0x211);
             ok = false;
             break;
@@ -475,8 +484,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                       n_t * 2 * kBN + static_cast<int>(rank) * kBN);
         }
       }
-      for (int j = (it > kStages2 ? it - kStages2 : 0); j < it; ++j)
-        (void)wait_drain(pfull + (j % kStages2), (j / kStages2) & 1, limit);
+      for (int j = (it > kStagesA ? it - kStagesA : 0); j < it; ++j)
+        (void)wait_drain(pfull + (j % kStagesA), (j / kStagesA) & 1, limit);
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer (leader) -------------------------
@@ -493,19 +502,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         const uint32_t d = tmem + static_cast<uint32_t>(a * BT);
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
-          const int s = it % kStages2;
-          const uint32_t ph = (it / kStages2) & 1;
-          if (!wait1(xfull + s, ph, limit, abort_flag) || !wait1(expd + s, ph, limit, abort_flag)) {
+          const int sa = it % kStagesA, sb = it % kStagesB;
+          const uint32_t pha = (it / kStagesA) & 1, phb = (it / kStagesB) & 1;
+          if (!wait1(xfull + sa, pha, limit, abort_flag) || !wait1(expd + sb, phb, limit, abort_flag)) {
             fail(0x312);
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t xa = smem_u32(xs + s * Cfg::kXHalf), ea = smem_u32(es + s * kExpStage);
+          const uint32_t xa = smem_u32(xs + sa * Cfg::kXHalf), ea = smem_u32(es + sb * kExpStage);
 #pragma unroll
           for (int k = 0; k < kBK / 32; ++k)
             mma_i8_pair(d, sw128_desc(ea + 32 * k), sw128_desc(xa + 32 * k), idesc, (kb | k) != 0);
-          mma_commit_pair(empty + s, 0x3);
+          mma_commit_pair(emptyA + sa, 0x3);
+          mma_commit_pair(emptyB + sb, 0x3);
         }
         if (ok) mma_commit_pair(accf + a, 0x3);
       }
@@ -519,35 +529,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     bool ok = true;
     for (int tile = pair; tile < tiles && ok; tile += pairs) {
       for (int kb = 0; kb < kblocks; ++kb, ++it) {
-        const int s = it % kStages2;
-        const uint32_t ph = (it / kStages2) & 1;
-        if (!wait_warp(pfull + s, ph, limit, abort_flag)) {
+        const int sa = it % kStagesA, sb = it % kStagesB;
+        const uint32_t pha = (it / kStagesA) & 1, phb = (it / kStagesB) & 1;
+        if (!wait_warp(pfull + sa, pha, limit, abort_flag) || !wait_warp(emptyB + sb, phb ^ 1, limit, abort_flag)) {
           if (lane == 0) fail(0x411);
           ok = false;
           break;
         }
-        const uint4* src = reinterpret_cast<const uint4*>(ps + s * kPackedStage + r * 32);
+        const uint4* src = reinterpret_cast<const uint4*>(ps + sa * kPackedStage + r * 32);
         const uint4 p0 = src[0], p1 = src[1];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(emptyA + sa);  // the packed tile has been read
         const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-        uint8_t* row = es + s * kExpStage + (r >> 3) * 1024 + (r & 7) * 128;
+        uint8_t* row = es + sb * kExpStage + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
         for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(row + ((j ^ (r & 7)) << 4)) = expand16(w[j]);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(expd + s), 0));
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(expd + sb), 0));
       }
     }
   } else if (warp >= 8) {
     // ------------------------------ epilogue (both CTAs) ------------------------
-    const int q = warp & 3;
+    // Each 32-token chunk of the tile's accumulator is converted into a shared
+    // staging buffer laid out as the output tile [32 tokens x 128 rows] and
+    // written by one TMA tensor store (the TMA unit clips rows past N and
+    // tokens past M); two buffers alternate, a buffer being rewritten only after
+    // the store issued from it two chunks before has read it.  Without a tensor
+    // map for y (a row of y not a multiple of 16 bytes) the lanes store directly.
+    const int q = warp & 3, et = threadIdx.x - 256;
+    const uint32_t esz = (ydt == BL_BF16) ? 2u : 4u;
     const float g = __ldg(gamma);
-    int tc = 0;
+    int tc = 0, chunk = 0;
     for (int tile = pair; tile < tiles; tile += pairs, ++tc) {
       const int a = tc & 1;
       const int n_t = tile % n_tiles, t_t = tile / n_tiles;
-      const int n = n_t * 2 * kBN + static_cast<int>(rank) * kBN + 32 * q + lane;
+      const int nbase = n_t * 2 * kBN + static_cast<int>(rank) * kBN;
+      const int n = nbase + 32 * q + lane;
       float* cf = cfac + a * BT;
-      for (int j = threadIdx.x - 256; j < BT; j += 128) {
+      for (int j = et; j < BT; j += 128) {
         const int t = t_t * BT + j;
         cf[j] = (t < M && ydt != BL_I32) ? dequant_factor(g, __ldg(scale + t)) : 0.0f;
       }
@@ -567,23 +587,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
 #pragma unroll 1
-      for (int j0 = 0; j0 < BT; j0 += 32) {
+      for (int j0 = 0; j0 < BT; j0 += 32, ++chunk) {
         uint32_t acc[32];
         tmem_load<32>(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(a * BT + j0), acc);
+        const int t0 = t_t * BT + j0;
+        if (y_tma) {
+          uint8_t* sb = ystage + (chunk & 1) * kYStage;
+          if (chunk >= 2) {  // the store issued from this buffer two chunks ago has read it
+            if (et == 0) bulk_wait_read<1>();
+            asm volatile("bar.sync 2, 128;" ::: "memory");
+          }
+          uint8_t* col = sb + (32 * q + lane) * esz;  // this lane's row in the staged tile
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int t = t_t * BT + j0 + j;
-          if (t < M && n < N) {
-            const int64_t o = static_cast<int64_t>(t) * N + n;
+          for (int j = 0; j < 32; ++j) {
             const int v = static_cast<int>(acc[j]);
             if (ydt == BL_I32) {
-              static_cast<int32_t*>(y)[o] = v;
+              *reinterpret_cast<int32_t*>(col + j * 128 * 4) = v;
             } else {
               const float yv = __fmul_rn(__int2float_rn(v), cf[j0 + j]);
               if (ydt == BL_F32)
-                static_cast<float*>(y)[o] = yv;
+                *reinterpret_cast<float*>(col + j * 128 * 4) = yv;
               else
-                static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(yv);
+                *reinterpret_cast<__nv_bfloat16*>(col + j * 128 * 2) = __float2bfloat16_rn(yv);
+            }
+          }
+          fence_proxy_async_smem();
+          asm volatile("bar.sync 2, 128;" ::: "memory");
+          if (et == 0 && nbase < N && t0 < M) {
+            tma_store_2d(&tm_y, sb, nbase, t0);
+          }
+          if (et == 0) bulk_commit();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int t = t0 + j;
+            if (t < M && n < N) {
+              const int64_t o = static_cast<int64_t>(t) * N + n;
+              const int v = static_cast<int>(acc[j]);
+              if (ydt == BL_I32) {
+                static_cast<int32_t*>(y)[o] = v;
+              } else {
+                const float yv = __fmul_rn(__int2float_rn(v), cf[j0 + j]);
+                if (ydt == BL_F32)
+                  static_cast<float*>(y)[o] = yv;
+                else
+                  static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(yv);
+              }
             }
           }
         }
@@ -592,6 +641,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(acce + a), 0));
     }
+    if (y_tma && et == 0) bulk_wait<0>();  // every output store has landed before the CTA leaves
   }
 
   __syncthreads();
@@ -678,6 +728,24 @@ bool encode_2d_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t out
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tensor map of y for the TMA-store epilogue: [M x N] of the output type, box
+// 128 rows x 32 tokens.  False when a row of y is not a multiple of 16 bytes.
+bool encode_y(CUtensorMap* m, void* y, int ydt, int64_t M, int64_t N) {
+  const uint64_t esz = (ydt == BL_BF16) ? 2 : 4;
+  if ((static_cast<uint64_t>(N) * esz) % 16 != 0) return false;
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const CUtensorMapDataType dt = ydt == BL_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                 : ydt == BL_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                                 : CU_TENSOR_MAP_DATA_TYPE_INT32;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * esz};
+  const cuuint32_t box[2] = {128, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int BT>
 cudaError_t launch_gemm_bt(const int8_t* xq, const uint8_t* w, int64_t rb, const float* gamma, const float* scale,
                            void* y, int ydt, int64_t M, int64_t N, int64_t K, void* ws, long long limit,
@@ -712,6 +780,9 @@ cudaError_t launch_gemm_2sm(const int8_t* xq, const uint8_t* w, int64_t rb, cons
   if (!encode_2d_u8(&tw, w, static_cast<uint64_t>(rb), static_cast<uint64_t>(N), static_cast<uint64_t>(rb),
                     kBK / 4, kBN, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
+  CUtensorMap ty;
+  const int y_tma = encode_y(&ty, y, ydt, M, N) ? 1 : 0;
+  if (!y_tma) memset(&ty, 0, sizeof(ty));
   auto kern = gemm_i2_2sm_kernel<BT>;
   const size_t smem = Gemm2Cfg<BT>::kSmem;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -719,7 +790,7 @@ cudaError_t launch_gemm_2sm(const int8_t* xq, const uint8_t* w, int64_t rb, cons
   const int64_t tiles = ((N + 2 * kBN - 1) / (2 * kBN)) * ((M + BT - 1) / BT);
   const int64_t pairs_max = device_sms() / 2;
   const int64_t pairs = tiles < pairs_max ? tiles : pairs_max;
-  kern<<<static_cast<unsigned>(2 * pairs), kGemmThreads, smem, st>>>(tx, tw, gamma, scale, y, ydt,
+  kern<<<static_cast<unsigned>(2 * pairs), kGemmThreads, smem, st>>>(tx, tw, ty, y_tma, gamma, scale, y, ydt,
                                                                      static_cast<int>(M), static_cast<int>(N),
                                                                      static_cast<int>(K), static_cast<WsHeader*>(ws),
                                                                      limit);
