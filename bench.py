@@ -55,9 +55,24 @@ WORKLOADS = {
 # helpers
 # ----------------------------------------------------------------------------
 
-def csrc_digest() -> str:
+KERNEL_SOURCE = {"absmean_kernel": "bl_weights.cu", "ternarize_flat_kernel": "bl_weights.cu",
+                 "ternarize_pack_kernel": "bl_weights.cu", "gemv_i2_kernel": "bl_gemv.cu",
+                 "gemv_kernel": "bl_gemv.cu", "act_quant_row_kernel": "bl_acts.cu",
+                 "act_quant_kernel": "bl_acts.cu", "gemm_i2_2sm_kernel": "bl_gemm_sm100.cu",
+                 "gemm_i2_kernel": "bl_gemm_sm100.cu"}
+
+
+def csrc_digest(kernel: str | None = None) -> str:
+    """Digest of the sources a kernel is built from (its .cu file and the
+    shared headers), or of every source when no kernel is named."""
+    csrc = os.path.join(ROOT, "bitlinear_b1_fwd_b200", "csrc")
+    if kernel is None:
+        files = sorted(glob.glob(os.path.join(csrc, "*")))
+    else:
+        files = sorted([os.path.join(csrc, KERNEL_SOURCE[kernel])] + glob.glob(os.path.join(csrc, "*.cuh")) +
+                       glob.glob(os.path.join(csrc, "*.h")))
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "bitlinear_b1_fwd_b200", "csrc", "*"))):
+    for p in files:
         with open(p, "rb") as f:
             h.update(os.path.basename(p).encode() + f.read())
     return h.hexdigest()[:16]
@@ -91,7 +106,7 @@ def measured_int8_peak():
 def profiled_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
     the current kernel sources (else None)."""
-    digest = csrc_digest()
+    digest = csrc_digest(kernel)
     for p in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
         kv = {}
         with open(p) as f:
