@@ -131,16 +131,19 @@ struct GemmCfg {
   static constexpr uint32_t kXStage = BT * 128;
   static constexpr uint32_t kTmemCols = (2 * BT < 32) ? 32 : 2 * BT;
   static constexpr uint32_t kChunk = BT < 32 ? BT : 32;  // accumulator columns per tcgen05.ld
-  static constexpr size_t kSmem =
-      1024 + kStages * (kXStage + kExpStage + kPackedStage) + 8 * (3 * kStages + 5) + 16 + 2 * 4 * BT;
+  // output staging for the TMA-store epilogue: 2 x [kChunk tokens x 128 rows],
+  // up to 4 bytes each (none for 256-token tiles, which do not fit it)
+  static constexpr uint32_t kYStage1 = (BT <= 128) ? kChunk * 128 * 4 : 0;
+  static constexpr size_t kSmem = 1024 + kStages * (kXStage + kExpStage + kPackedStage) + 2 * kYStage1 +
+                                  8 * (3 * kStages + 5) + 16 + 2 * 4 * BT;
 };
 
 template <int BT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_i2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                   const float* __restrict__ gamma, const float* __restrict__ scale, void* __restrict__ y,
-                   int ydt, int M, int N, int K, WsHeader* __restrict__ hdr, long long limit,
-                   int skip_producer) {
+                   const __grid_constant__ CUtensorMap tm_y, int y_tma, const float* __restrict__ gamma,
+                   const float* __restrict__ scale, void* __restrict__ y, int ydt, int M, int N, int K,
+                   WsHeader* __restrict__ hdr, long long limit, int skip_producer) {
   using Cfg = GemmCfg<BT>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -148,7 +151,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* xs = base;                              // kStages x [BT x 128 B], swizzled
   uint8_t* es = xs + kStages * Cfg::kXStage;       // kStages x [128 x 128 B], swizzled
   uint8_t* ps = es + kStages * kExpStage;          // kStages x [128 x 32 B]
-  uint64_t* full = reinterpret_cast<uint64_t*>(ps + kStages * kPackedStage);
+  uint8_t* ystage = ps + kStages * kPackedStage;   // 2 x [kChunk tokens x 128 rows] output staging
+  uint64_t* full = reinterpret_cast<uint64_t*>(ystage + 2 * Cfg::kYStage1);
   uint64_t* expd = full + kStages;
   uint64_t* empty = expd + kStages;
   uint64_t* accf = empty + kStages;  // 2
@@ -281,16 +285,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp >= 8) {
     // ------------------------------ epilogue -----------------------------------
+    // (with a tensor map for y, chunks of the accumulator leave through a
+    // shared staging tile and TMA tensor stores, as in the two-SM kernel)
     const int q = warp & 3;  // TMEM lane quarter this warp may read
+    const int et = threadIdx.x - 256;
+    const uint32_t esz = (ydt == BL_BF16) ? 2u : 4u;
+    const bool use_tma = y_tma != 0 && Cfg::kYStage1 != 0;
     const float g = __ldg(gamma);
-    int tc = 0;
+    int tc = 0, chunk = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
       const int a = tc & 1;
       const int n_t = tile % n_tiles, t_t = tile / n_tiles;
       const int n = n_t * kBN + 32 * q + lane;
       // dequant factor c_t = (gamma s_t) / 127 of each token of the tile, once
       float* cf = cfac + a * BT;
-      for (int j = threadIdx.x - 256; j < BT; j += 128) {
+      for (int j = et; j < BT; j += 128) {
         const int t = t_t * BT + j;
         cf[j] = (t < M && ydt != BL_I32) ? dequant_factor(g, __ldg(scale + t)) : 0.0f;
       }
@@ -311,24 +320,51 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
 #pragma unroll 1
-      for (int j0 = 0; j0 < BT; j0 += Cfg::kChunk) {
+      for (int j0 = 0; j0 < BT; j0 += Cfg::kChunk, ++chunk) {
         uint32_t acc[Cfg::kChunk];
         tmem_load<Cfg::kChunk>(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(a * BT + j0),
                                acc);
+        const int t0 = t_t * BT + j0;
+        if (use_tma) {
+          uint8_t* sb = ystage + (chunk & 1) * Cfg::kYStage1;
+          if (chunk >= 2) {  // the store issued from this buffer two chunks ago has read it
+            if (et == 0) bulk_wait_read<1>();
+            asm volatile("bar.sync 2, 128;" ::: "memory");
+          }
+          uint8_t* col = sb + (32 * q + lane) * esz;  // this lane's row in the staged tile
 #pragma unroll
-        for (int j = 0; j < static_cast<int>(Cfg::kChunk); ++j) {
-          const int t = t_t * BT + j0 + j;
-          if (t < M && n < N) {
-            const int64_t o = static_cast<int64_t>(t) * N + n;
+          for (int j = 0; j < static_cast<int>(Cfg::kChunk); ++j) {
             const int v = static_cast<int>(acc[j]);
             if (ydt == BL_I32) {
-              static_cast<int32_t*>(y)[o] = v;
+              *reinterpret_cast<int32_t*>(col + j * 128 * 4) = v;
             } else {
               const float yv = __fmul_rn(__int2float_rn(v), cf[j0 + j]);
               if (ydt == BL_F32)
-                static_cast<float*>(y)[o] = yv;
+                *reinterpret_cast<float*>(col + j * 128 * 4) = yv;
               else
-                static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(yv);
+                *reinterpret_cast<__nv_bfloat16*>(col + j * 128 * 2) = __float2bfloat16_rn(yv);
+            }
+          }
+          fence_proxy_async_smem();
+          asm volatile("bar.sync 2, 128;" ::: "memory");
+          if (et == 0 && n_t * kBN < N && t0 < M) tma_store_2d(&tm_y, sb, n_t * kBN, t0);
+          if (et == 0) bulk_commit();
+        } else {
+#pragma unroll
+          for (int j = 0; j < static_cast<int>(Cfg::kChunk); ++j) {
+            const int t = t0 + j;
+            if (t < M && n < N) {
+              const int64_t o = static_cast<int64_t>(t) * N + n;
+              const int v = static_cast<int>(acc[j]);
+              if (ydt == BL_I32) {
+                static_cast<int32_t*>(y)[o] = v;
+              } else {
+                const float yv = __fmul_rn(__int2float_rn(v), cf[j0 + j]);
+                if (ydt == BL_F32)
+                  static_cast<float*>(y)[o] = yv;
+                else
+                  static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(yv);
+              }
             }
           }
         }
@@ -337,6 +373,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(acce + a);
     }
+    if (use_tma && et == 0) bulk_wait<0>();  // every output store has landed before the CTA leaves
   }
 
   __syncthreads();
@@ -729,8 +766,9 @@ bool encode_2d_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t out
 }
 
 // Tensor map of y for the TMA-store epilogue: [M x N] of the output type, box
-// 128 rows x 32 tokens.  False when a row of y is not a multiple of 16 bytes.
-bool encode_y(CUtensorMap* m, void* y, int ydt, int64_t M, int64_t N) {
+// 128 rows x `tokens` tokens.  False when a row of y is not a multiple of 16
+// bytes.
+bool encode_y(CUtensorMap* m, void* y, int ydt, int64_t M, int64_t N, uint32_t tokens) {
   const uint64_t esz = (ydt == BL_BF16) ? 2 : 4;
   if ((static_cast<uint64_t>(N) * esz) % 16 != 0) return false;
   EncodeTiledFn fn = encode_fn();
@@ -740,7 +778,7 @@ bool encode_y(CUtensorMap* m, void* y, int ydt, int64_t M, int64_t N) {
                                                  : CU_TENSOR_MAP_DATA_TYPE_INT32;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * esz};
-  const cuuint32_t box[2] = {128, 32};
+  const cuuint32_t box[2] = {128, tokens};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, dt, 2, y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -757,6 +795,9 @@ cudaError_t launch_gemm_bt(const int8_t* xq, const uint8_t* w, int64_t rb, const
   if (!encode_2d_u8(&tw, w, static_cast<uint64_t>(rb), static_cast<uint64_t>(N), static_cast<uint64_t>(rb),
                     kBK / 4, kBN, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
+  CUtensorMap ty;
+  const int y_tma = (GemmCfg<BT>::kYStage1 != 0 && encode_y(&ty, y, ydt, M, N, GemmCfg<BT>::kChunk)) ? 1 : 0;
+  if (!y_tma) memset(&ty, 0, sizeof(ty));
   auto kern = gemm_i2_kernel<BT>;
   const size_t smem = GemmCfg<BT>::kSmem;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -764,7 +805,8 @@ cudaError_t launch_gemm_bt(const int8_t* xq, const uint8_t* w, int64_t rb, const
   const int64_t tiles = ((N + kBN - 1) / kBN) * ((M + BT - 1) / BT);
   const int sms = device_sms();
   const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
-  kern<<<grid, kGemmThreads, smem, st>>>(tx, tw, gamma, scale, y, ydt, static_cast<int>(M), static_cast<int>(N),
+  kern<<<grid, kGemmThreads, smem, st>>>(tx, tw, ty, y_tma, gamma, scale, y, ydt, static_cast<int>(M),
+                                         static_cast<int>(N),
                                          static_cast<int>(K), static_cast<WsHeader*>(ws), limit, skip_producer);
   return cudaGetLastError();
 }
@@ -781,7 +823,7 @@ cudaError_t launch_gemm_2sm(const int8_t* xq, const uint8_t* w, int64_t rb, cons
                     kBK / 4, kBN, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   CUtensorMap ty;
-  const int y_tma = encode_y(&ty, y, ydt, M, N) ? 1 : 0;
+  const int y_tma = encode_y(&ty, y, ydt, M, N, 32) ? 1 : 0;
   if (!y_tma) memset(&ty, 0, sizeof(ty));
   auto kern = gemm_i2_2sm_kernel<BT>;
   const size_t smem = Gemm2Cfg<BT>::kSmem;
