@@ -44,6 +44,7 @@ template <int XDT, int NV>
 __global__ void __launch_bounds__(kActRowThreads)
     act_quant_row_kernel(const void* __restrict__ x, int64_t M, int64_t K, int8_t* __restrict__ xq,
                          float* __restrict__ scale) {
+  pdl_enter(x, xq, scale);
   constexpr int EPW = (XDT == BL_F32) ? 4 : 8;  // elements per 16-byte word
   __shared__ float red[kActRowThreads / 32];
   const int t = threadIdx.x, lane = t & 31;
@@ -54,7 +55,7 @@ __global__ void __launch_bounds__(kActRowThreads)
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       const int v = t + kActRowThreads * i;
-      r[i] = v < nv ? __ldg(row + v) : make_uint4(0, 0, 0, 0);
+      r[i] = v < nv ? __ldcg(row + v) : make_uint4(0, 0, 0, 0);
     }
     auto elems = [&](int i, float* e) {
       if constexpr (XDT == BL_F32) {
@@ -106,6 +107,7 @@ template <int XDT>
 __global__ void __launch_bounds__(kActThreads)
     act_quant_kernel(const void* __restrict__ x, int64_t M, int64_t K, int8_t* __restrict__ xq,
                      float* __restrict__ scale, bool vec) {
+  pdl_enter(x, xq, scale);
   const int lane = threadIdx.x & 31;
   const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t tw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -183,7 +185,7 @@ cudaError_t launch_act_quant(const void* x, int xdt, int64_t M, int64_t K, int8_
         per_sm < 1)                                                                                     \
       per_sm = 1;                                                                                       \
     const int64_t cap = static_cast<int64_t>(device_sms()) * per_sm;                                    \
-    kern<<<static_cast<unsigned>(M < cap ? M : cap), kActRowThreads, 0, st>>>(x, M, K, xq, scale);      \
+    { const cudaError_t le_ = launch_pdl(kern, static_cast<unsigned>(M < cap ? M : cap), kActRowThreads, 0, st, x, M, K, xq, scale); if (le_ != cudaSuccess) return le_; }      \
     return cudaGetLastError();                                                                          \
   }
     if (xdt == BL_F32) {
@@ -198,11 +200,9 @@ cudaError_t launch_act_quant(const void* x, int xdt, int64_t M, int64_t K, int8_
 #undef BL_AQ
   }
   if (xdt == BL_F32)
-    act_quant_kernel<BL_F32><<<grid_for(reinterpret_cast<const void*>(act_quant_kernel<BL_F32>)), kActThreads, 0,
-                               st>>>(x, M, K, xq, scale, vec);
+    { const cudaError_t le_ = launch_pdl(act_quant_kernel<BL_F32>, grid_for(reinterpret_cast<const void*>(act_quant_kernel<BL_F32>)), kActThreads, 0, st, x, M, K, xq, scale, vec); if (le_ != cudaSuccess) return le_; }
   else
-    act_quant_kernel<BL_BF16><<<grid_for(reinterpret_cast<const void*>(act_quant_kernel<BL_BF16>)), kActThreads,
-                                0, st>>>(x, M, K, xq, scale, vec);
+    { const cudaError_t le_ = launch_pdl(act_quant_kernel<BL_BF16>, grid_for(reinterpret_cast<const void*>(act_quant_kernel<BL_BF16>)), kActThreads, 0, st, x, M, K, xq, scale, vec); if (le_ != cudaSuccess) return le_; }
   return cudaGetLastError();
 }
 

@@ -33,9 +33,9 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) {
 template <int DT>
 __device__ __forceinline__ float load_elem(const void* p, int64_t i) {
   if constexpr (DT == BL_F32) {
-    return __ldg(static_cast<const float*>(p) + i);
+    return __ldcg(static_cast<const float*>(p) + i);
   } else {
-    return bf16_bits_to_f32(__ldg(static_cast<const uint16_t*>(p) + i));
+    return bf16_bits_to_f32(__ldcg(static_cast<const uint16_t*>(p) + i));
   }
 }
 
@@ -45,17 +45,68 @@ template <int DT>
 __device__ __forceinline__ void load8_aligned(const void* p, int64_t e, float v[8]) {
   if constexpr (DT == BL_F32) {
     const float4* q = reinterpret_cast<const float4*>(static_cast<const float*>(p) + e);
-    float4 a = __ldg(q), b = __ldg(q + 1);
+    float4 a = __ldcg(q), b = __ldcg(q + 1);
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
   } else {
-    uint4 a = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p) + e));
+    uint4 a = __ldcg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p) + e));
     uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       v[2 * i] = __uint_as_float(w[i] << 16);
       v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
     }
+  }
+}
+
+// Programmatic dependent launch: every kernel of the library lets the next
+// kernel in its stream be scheduled as soon as it starts (all of them run as
+// one wave of persistent CTAs, so that kernel's CTAs only take SM room this
+// grid no longer needs), and waits for the previous kernel to complete (with
+// its memory visible) before it reads or writes anything.  Without the launch
+// attribute both instructions are no-ops.
+// A grid launched this way is alive while its predecessor still writes, so
+// nothing it reads may go through the non-coherent read-only path (whose
+// contract is data constant for the kernel's whole life): inputs are read
+// with L2-coherent loads (ld.global.cg), and the pointers a kernel touches
+// are passed through an opaque move issued after the wait, so that no load
+// through them is derived from a restrict kernel parameter (which the
+// compiler may turn into a read-only-path load) or issued before the wait.
+template <typename P>
+__device__ __forceinline__ void pdl_after(P& p) {
+  uint64_t v;
+  asm volatile("mov.b64 %0, %1;" : "=l"(v) : "l"((uint64_t)(p)) : "memory");
+  p = (P)(v);
+}
+
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... P>
+__device__ __forceinline__ void pdl_wait(P&... ptrs) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  (pdl_after(ptrs), ...);
+}
+
+template <typename... P>
+__device__ __forceinline__ void pdl_enter(P&... ptrs) {
+  pdl_launch_dependents();
+  pdl_wait(ptrs...);
+}
+
+// Bulk prefetch of [p, p + bytes) into L2 (p 16-byte aligned, bytes a
+// multiple of 16), one instruction per 16 KB from threads 0, 1, ...  A
+// prefetch returns no data and L2 is the point of coherence, so it may be
+// issued before the wait: a later load still sees whatever the previous
+// kernel writes there.
+__device__ __forceinline__ void l2_prefetch_bulk(const void* p, int64_t bytes) {
+  constexpr int64_t kPiece = 16384;
+  const int64_t off = static_cast<int64_t>(threadIdx.x) * kPiece;
+  if (off < bytes) {
+    const uint32_t sz = static_cast<uint32_t>(bytes - off < kPiece ? bytes - off : kPiece);
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(static_cast<const uint8_t*>(p) + off), "r"(sz)
+                 : "memory");
   }
 }
 

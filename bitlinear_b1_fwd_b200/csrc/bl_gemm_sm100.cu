@@ -144,6 +144,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                    const __grid_constant__ CUtensorMap tm_y, int y_tma, const float* __restrict__ gamma,
                    const float* __restrict__ scale, void* __restrict__ y, int ydt, int M, int N, int K,
                    WsHeader* __restrict__ hdr, long long limit, int skip_producer) {
+  pdl_enter(gamma, scale, y, hdr);
   using Cfg = GemmCfg<BT>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -291,7 +292,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int et = threadIdx.x - 256;
     const uint32_t esz = (ydt == BL_BF16) ? 2u : 4u;
     const bool use_tma = y_tma != 0 && Cfg::kYStage1 != 0;
-    const float g = __ldg(gamma);
+    const float g = __ldcg(gamma);
     int tc = 0, chunk = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
       const int a = tc & 1;
@@ -301,7 +302,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       float* cf = cfac + a * BT;
       for (int j = et; j < BT; j += 128) {
         const int t = t_t * BT + j;
-        cf[j] = (t < M && ydt != BL_I32) ? dequant_factor(g, __ldg(scale + t)) : 0.0f;
+        cf[j] = (t < M && ydt != BL_I32) ? dequant_factor(g, __ldcg(scale + t)) : 0.0f;
       }
       const uint32_t ok_w = wait_warp(accf + a, (tc >> 1) & 1, limit, abort_flag) ? 1u : 0u;
       // the four epilogue warps agree (and see each other's factors) before going on
@@ -435,6 +436,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                        const __grid_constant__ CUtensorMap tm_y, int y_tma, const float* __restrict__ gamma,
                        const float* __restrict__ scale, void* __restrict__ y, int ydt, int M, int N, int K,
                        WsHeader* __restrict__ hdr, long long limit) {
+  pdl_enter(gamma, scale, y, hdr);
   using Cfg = Gemm2Cfg<BT>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -596,7 +598,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // map for y (a row of y not a multiple of 16 bytes) the lanes store directly.
     const int q = warp & 3, et = threadIdx.x - 256;
     const uint32_t esz = (ydt == BL_BF16) ? 2u : 4u;
-    const float g = __ldg(gamma);
+    const float g = __ldcg(gamma);
     int tc = 0, chunk = 0;
     for (int tile = pair; tile < tiles; tile += pairs, ++tc) {
       const int a = tc & 1;
@@ -606,7 +608,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       float* cf = cfac + a * BT;
       for (int j = et; j < BT; j += 128) {
         const int t = t_t * BT + j;
-        cf[j] = (t < M && ydt != BL_I32) ? dequant_factor(g, __ldg(scale + t)) : 0.0f;
+        cf[j] = (t < M && ydt != BL_I32) ? dequant_factor(g, __ldcg(scale + t)) : 0.0f;
       }
       const uint32_t ok_w = wait_warp(accf + a, (tc >> 1) & 1, limit, abort_flag) ? 1u : 0u;
       uint32_t ok_all;
@@ -698,6 +700,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 __global__ void __launch_bounds__(256)
     t5_to_i2_kernel(const uint8_t* __restrict__ t5, int64_t N, int64_t K, int64_t rb5, uint8_t* __restrict__ i2,
                     int64_t rb2) {
+  pdl_enter(t5, i2);
   __shared__ uint16_t lut[256];
   for (int b = threadIdx.x; b < 256; b += blockDim.x) {
     uint32_t v = b, d = 0;
@@ -805,9 +808,9 @@ cudaError_t launch_gemm_bt(const int8_t* xq, const uint8_t* w, int64_t rb, const
   const int64_t tiles = ((N + kBN - 1) / kBN) * ((M + BT - 1) / BT);
   const int sms = device_sms();
   const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
-  kern<<<grid, kGemmThreads, smem, st>>>(tx, tw, ty, y_tma, gamma, scale, y, ydt, static_cast<int>(M),
+  { const cudaError_t le_ = launch_pdl(kern, grid, kGemmThreads, smem, st, tx, tw, ty, y_tma, gamma, scale, y, ydt, static_cast<int>(M),
                                          static_cast<int>(N),
-                                         static_cast<int>(K), static_cast<WsHeader*>(ws), limit, skip_producer);
+                                         static_cast<int>(K), static_cast<WsHeader*>(ws), limit, skip_producer); if (le_ != cudaSuccess) return le_; }
   return cudaGetLastError();
 }
 
@@ -832,10 +835,10 @@ cudaError_t launch_gemm_2sm(const int8_t* xq, const uint8_t* w, int64_t rb, cons
   const int64_t tiles = ((N + 2 * kBN - 1) / (2 * kBN)) * ((M + BT - 1) / BT);
   const int64_t pairs_max = device_sms() / 2;
   const int64_t pairs = tiles < pairs_max ? tiles : pairs_max;
-  kern<<<static_cast<unsigned>(2 * pairs), kGemmThreads, smem, st>>>(tx, tw, ty, y_tma, gamma, scale, y, ydt,
+  { const cudaError_t le_ = launch_pdl(kern, static_cast<unsigned>(2 * pairs), kGemmThreads, smem, st, tx, tw, ty, y_tma, gamma, scale, y, ydt,
                                                                      static_cast<int>(M), static_cast<int>(N),
                                                                      static_cast<int>(K), static_cast<WsHeader*>(ws),
-                                                                     limit);
+                                                                     limit); if (le_ != cudaSuccess) return le_; }
   return cudaGetLastError();
 }
 
@@ -871,7 +874,7 @@ cudaError_t launch_t5_to_i2(const uint8_t* t5, int64_t N, int64_t K, int64_t rb5
   int64_t grid = (work + 255) / 256;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  t5_to_i2_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(t5, N, K, rb5, i2, rb2);
+  { const cudaError_t le_ = launch_pdl(t5_to_i2_kernel, static_cast<unsigned>(grid), 256, 0, st, t5, N, K, rb5, i2, rb2); if (le_ != cudaSuccess) return le_; }
   return cudaGetLastError();
 }
 

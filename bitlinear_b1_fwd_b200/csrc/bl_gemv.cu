@@ -27,7 +27,7 @@ constexpr int kGemvTileRows = 1024;   // rows whose sums a CTA holds in shared m
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
@@ -112,6 +112,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     gemv_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
                 int64_t N, int64_t K, const void* __restrict__ x, float* __restrict__ scale,
                 void* __restrict__ y, int ydt, int write_scale) {
+  pdl_enter(packed, gamma, x, scale, y);
   extern __shared__ __align__(16) uint8_t smem[];
   const int64_t xb = gemv_x_bytes(FMT, rowbytes);
   uint8_t* xs = smem;                                                 // [MT][xb]
@@ -159,6 +160,12 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   issue(bufA);
 
   // 2. prologue: per-token absmax, then the INT8 codes in the layout above
+  //    gamma (and the scales of int8 tokens) are read once per CTA into
+  //    shared memory: a load by every warp sends thousands of requests to one
+  //    L2 line
+  __shared__ float sh_gs[1 + MT];
+  if (threadIdx.x <= MT && (threadIdx.x == 0 || XDT == BL_I8))
+    sh_gs[threadIdx.x] = __ldcg(threadIdx.x == 0 ? gamma : scale + (threadIdx.x - 1));
   for (int i = threadIdx.x; i < MT * kGemvTileRows; i += blockDim.x) racc[i] = 0;
   if constexpr (FMT == BL_PACK_T5) {
     uint4* z = reinterpret_cast<uint4*>(xs);
@@ -207,7 +214,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
       for (int w = 1; w < kGemvWarps; ++w) a = fmaxf(a, red_f[m][w]);
       s_tok[m] = fmaxf(a, 1e-6f);
     } else {
-      s_tok[m] = __ldg(scale + m);
+      s_tok[m] = sh_gs[1 + m];
     }
   }
 #pragma unroll
@@ -228,7 +235,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
           int q[8];
           if (full) {
             if constexpr (XDT == BL_I8) {
-              const uint2 raw = __ldg(reinterpret_cast<const uint2*>(static_cast<const int8_t*>(x) + m * K + kh));
+              const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(static_cast<const int8_t*>(x) + m * K + kh));
 #pragma unroll
               for (int j = 0; j < 8; ++j) q[j] = static_cast<int8_t>((j < 4 ? raw.x : raw.y) >> (8 * (j & 3)));
             } else {
@@ -259,7 +266,7 @@ quant_act_fast_n<8>(e, s_tok[m], c127, q);
       for (int64_t v = threadIdx.x; v < K / 8; v += blockDim.x) {
         int q[8];
         if constexpr (XDT == BL_I8) {
-          const uint2 raw = __ldg(reinterpret_cast<const uint2*>(static_cast<const int8_t*>(x) + m * K + 8 * v));
+          const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(static_cast<const int8_t*>(x) + m * K + 8 * v));
 #pragma unroll
           for (int j = 0; j < 8; ++j) q[j] = static_cast<int8_t>((j < 4 ? raw.x : raw.y) >> (8 * (j & 3)));
         } else {
@@ -285,7 +292,7 @@ quant_act_fast_n<8>(e, s_tok[m], c127, q);
     if (lane == 0) red_i[m][warp] = part;
   }
   __syncthreads();  // activations and per-warp sums are visible
-  const float g = __ldg(gamma);
+  const float g = sh_gs[0];
   float cfac[MT];
   int corr[MT];
 #pragma unroll
@@ -432,6 +439,7 @@ quant_act_fast_n<8>(e, s_tok[m], c127, q);
 // ---------------------------------------------------------------------------
 constexpr int kI2Plane = 4096;  // bytes per activation plane: segments per row <= 2 kI2Plane / 16
 constexpr int kI2Batch = 2;     // items per load batch
+constexpr int64_t kI2Prefetch = 65536;  // bytes per CTA prefetched into L2 before the wait
 
 __host__ __device__ inline int64_t gemv_i2_smem_bytes(int mt) {
   return int64_t{8} * kI2Plane * mt + int64_t{4} * mt * kGemvTileRows;
@@ -442,6 +450,18 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     gemv_i2_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
                    int64_t N, int64_t K, const void* __restrict__ x, float* __restrict__ scale,
                    void* __restrict__ y, int ydt, int write_scale) {
+  const int64_t G = gridDim.x, b = blockIdx.x;
+  const int64_t per = N / G, extra = N % G;
+  const int64_t row0 = b * per + (b < extra ? b : extra);
+  const int64_t nrows = per + (b < extra ? 1 : 0);
+  // 0. while the previous kernel finishes: the first kI2Prefetch bytes of
+  //    this CTA's rows move into L2 (the weights do not depend on it)
+  pdl_launch_dependents();
+  {
+    const int64_t bytes = nrows * rowbytes;
+    l2_prefetch_bulk(packed + row0 * rowbytes, bytes < kI2Prefetch ? bytes : kI2Prefetch);
+  }
+  pdl_wait(packed, gamma, x, scale, y);
   extern __shared__ __align__(16) uint8_t smem[];
   uint8_t* xs = smem;                                           // [MT][8][kI2Plane]
   int* racc = reinterpret_cast<int*>(smem + MT * 8 * kI2Plane);  // [MT][kGemvTileRows]
@@ -451,10 +471,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t segs = static_cast<uint32_t>(rowbytes >> 4);
   const uint32_t nb = (segs + 63) >> 6;  // 1 KB blocks per row
-  const int64_t G = gridDim.x, b = blockIdx.x;
-  const int64_t per = N / G, extra = N % G;
-  const int64_t row0 = b * per + (b < extra ? b : extra);
-  const int64_t nrows = per + (b < extra ? 1 : 0);
   const uint32_t dq = kGemvWarps / nb, dr = kGemvWarps % nb;  // one step of a warp in (row, block)
   const uint32_t s_lane = 2u * lane;                            // first segment of the lane in a block
 
@@ -495,14 +511,19 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   constexpr int kXW = (XDT == BL_BF16) ? 2 : 1;  // 16-byte words per 16 activations
   const bool one_pass = kOnePassType && (K % 16) == 0;
   uint4 xraw[3][kXW];  // packed words g = tid + 768 u: 4 segs <= 2048 words (rows <= 8 KB)
-  const float g_w = __ldg(gamma);  // (loaded with the activations, ahead of the weight stream)
+  // gamma (and the scales of int8 tokens) once per CTA through shared memory,
+  // loaded with the activations ahead of the weight stream: a load by every
+  // warp sends thousands of requests to one L2 line
+  __shared__ float sh_gs[1 + MT];
+  if (threadIdx.x <= MT && (threadIdx.x == 0 || XDT == BL_I8))
+    sh_gs[threadIdx.x] = __ldcg(threadIdx.x == 0 ? gamma : scale + (threadIdx.x - 1));
   if (one_pass) {
 #pragma unroll
     for (int u = 0; u < 3; ++u) {
       const int64_t k0 = 16 * (static_cast<int64_t>(threadIdx.x) + static_cast<int64_t>(kGemvThreads) * u);
 #pragma unroll
       for (int i = 0; i < kXW; ++i)
-        xraw[u][i] = k0 < K ? __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(x) + k0 * kXW) + i)
+        xraw[u][i] = k0 < K ? __ldcg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(x) + k0 * kXW) + i)
                             : make_uint4(0, 0, 0, 0);
     }
   }
@@ -532,7 +553,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
       __syncthreads();  // zeroed row sums and per-warp maxima are visible
       s_tok[0] = fmaxf(warp_maxf(lane < kGemvWarps ? red_f[0][lane] : 0.0f), 1e-6f);
     } else {
-      s_tok[0] = __ldg(scale);
+      s_tok[0] = 0.0f;  // int8 tokens: the given scale, read after the barrier below
     }
     const float c127 = (XDT == BL_I8) ? 0.0f : __fdiv_rn(127.0f, s_tok[0]);
     int part = 0;
@@ -594,7 +615,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
         for (int w = 1; w < kGemvWarps; ++w) a = fmaxf(a, red_f[m][w]);
         s_tok[m] = fmaxf(a, 1e-6f);
       } else {
-        s_tok[m] = __ldg(scale + m);
+        s_tok[m] = 0.0f;  // int8 tokens: the given scale, read after the barrier below
       }
     }
   #pragma unroll
@@ -612,7 +633,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
           int q[8];
           if (full) {
             if constexpr (XDT == BL_I8) {
-              const uint2 raw = __ldg(reinterpret_cast<const uint2*>(static_cast<const int8_t*>(x) + m * K + kh));
+              const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(static_cast<const int8_t*>(x) + m * K + kh));
   #pragma unroll
               for (int j = 0; j < 8; ++j) q[j] = static_cast<int8_t>((j < 4 ? raw.x : raw.y) >> (8 * (j & 3)));
             } else {
@@ -644,11 +665,12 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     }
   }
   __syncthreads();  // activations and per-warp sums are visible
-  const float g = g_w;
+  const float g = sh_gs[0];
   float cfac[MT];
   int corr[MT];
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
+    if constexpr (XDT == BL_I8) s_tok[m] = sh_gs[1 + m];
     int t = 0;
 #pragma unroll
     for (int w = 0; w < kGemvWarps; ++w) t += red_i[m][w];
@@ -762,8 +784,8 @@ static cudaError_t launch_gemv_t(const uint8_t* packed, int64_t rowbytes, const 
   int64_t grid = static_cast<int64_t>(sms) * per_sm;
   if (grid > need) grid = need;
   if (grid < 1) grid = 1;
-  kern<<<static_cast<unsigned>(grid), kGemvThreads, smem, st>>>(packed, rowbytes, gamma, N, K, x, scale,
-                                                                 y, ydt, write_scale);
+  { const cudaError_t le_ = launch_pdl(kern, static_cast<unsigned>(grid), kGemvThreads, smem, st, packed, rowbytes, gamma, N, K, x, scale,
+                                                                 y, ydt, write_scale); if (le_ != cudaSuccess) return le_; }
   return cudaGetLastError();
 }
 
@@ -777,8 +799,8 @@ static cudaError_t launch_gemv_i2_t(const uint8_t* packed, int64_t rowbytes, con
   if (e != cudaSuccess) return e;
   const int64_t sms = device_sms();
   const int64_t grid = N < sms ? N : sms;  // every CTA owns at least one row
-  kern<<<static_cast<unsigned>(grid), kGemvThreads, smem, st>>>(packed, rowbytes, gamma, N, K, x, scale, y, ydt,
-                                                                 write_scale);
+  { const cudaError_t le_ = launch_pdl(kern, static_cast<unsigned>(grid), kGemvThreads, smem, st, packed, rowbytes, gamma, N, K, x, scale, y, ydt,
+                                                                 write_scale); if (le_ != cudaSuccess) return le_; }
   return cudaGetLastError();
 }
 

@@ -6,6 +6,24 @@
 
 namespace bl {
 
+// Launch with programmatic stream serialization (see pdl_enter): the kernel
+// may be scheduled while the previous kernel in the stream finishes.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // absmean: the last CTA folds 2^lgR chunk sums per lane (lgR <= 11 allows
 // 2^19 chunks of 8192 elements, so N*K <= 2^32).
 constexpr int kFinishMaxLevels = 11;

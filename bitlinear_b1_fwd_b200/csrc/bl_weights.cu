@@ -101,6 +101,7 @@ template <int WDT>
 __global__ void __launch_bounds__(kLanes, kAbsCtasPerSm)
     absmean_kernel(const void* __restrict__ W, int64_t T, int64_t C, int lgR, double* __restrict__ partials,
                    WsHeader* __restrict__ hdr, float* __restrict__ gamma) {
+  pdl_enter(W, partials, hdr, gamma);
   __shared__ double lsum[2][kLanes];
   __shared__ double p[kLanes];
   __shared__ bool last;
@@ -197,9 +198,13 @@ __global__ void __launch_bounds__(256)
     ternarize_pack_kernel(const void* __restrict__ W, int64_t N, int64_t K,
                           const float* __restrict__ gamma, float eps, uint8_t* __restrict__ packed,
                           int8_t* __restrict__ codes, int64_t rowbytes, bool vec_ok) {
+  pdl_enter(W, gamma, packed, codes);
   constexpr int PER = (FMT == BL_PACK_I2) ? 4 : 5;
   constexpr int WPS = 16 * PER;  // weights per segment
-  const float thr = ternary_threshold(__ldg(gamma), eps);
+  __shared__ float sh_thr;  // gamma once per CTA: a load by every warp hits one L2 line thousands of times
+  if (threadIdx.x == 0) sh_thr = ternary_threshold(__ldcg(gamma), eps);
+  __syncthreads();
+  const float thr = sh_thr;
   const int64_t segs = rowbytes / 16;
   const int64_t total = N * segs;
   for (int64_t it = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; it < total;
@@ -278,7 +283,10 @@ __global__ void __launch_bounds__(256)
 // 4p .. 4p + 3 of W in row-major order and the matrix is one stream.  A thread
 // turns a group of 16 consecutive weights (16-byte loads straight into
 // registers) into 4 packed bytes (one 32-bit store) and, if asked, 16 int8
-// codes (one 16-byte store); it keeps two groups in flight, and a persistent
+// codes (one 16-byte store).  It works on 64 bytes of W (two groups of bf16,
+// one of fp32) while the loads of the next 64 are in flight (issued ahead in program order: the loads are
+// L2-coherent asm loads, which the compiler does not move across the stores
+// of the groups before them), and a persistent
 // grid of kTernCtasPerSm CTAs per SM walks the groups from the end of W
 // backwards (the absmean kernel streamed W front to back, so the last groups it
 // read are the likeliest to still be in L2).
@@ -288,28 +296,63 @@ template <int WDT>
 __global__ void __launch_bounds__(256, kTernCtasPerSm)
     ternarize_flat_kernel(const void* __restrict__ W, int64_t T, const float* __restrict__ gamma, float eps,
                           uint8_t* __restrict__ packed, int8_t* __restrict__ codes) {
-  const float thr = ternary_threshold(__ldg(gamma), eps);
+  pdl_enter(W, gamma, packed, codes);
   const int64_t ng = T / 16;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t gi = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; gi < ng; gi += 2 * stride) {
-    float v[2][16];
+  // raw 16-byte words of the thread's U groups (64 bytes of W); the next U
+  // groups' loads go out before the current ones are turned into codes
+  constexpr int RW = (WDT == BL_F32) ? 4 : 2;  // 16-byte words per group
+  constexpr int EW = 16 / RW;                   // weights per word
+  constexpr int U = (WDT == BL_F32) ? 1 : 2;    // groups per step
+  auto fetch = [&](int64_t gi, uint4 (&r)[U][RW]) {
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < U; ++u) {
       const int64_t g = ng - 1 - (gi + u * stride);
-      if (g >= 0) load16_aligned<WDT>(W, 16 * g, v[u]);
-    }
+      const uint4* q = static_cast<const uint4*>(W) + g * RW;  // group g: 16 weights, RW words
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+      for (int i = 0; i < RW; ++i) r[u][i] = g >= 0 ? __ldcg(q + i) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  int64_t gi = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  uint4 cur[U][RW];
+  if (gi < ng) fetch(gi, cur);  // (the first loads go out before the threshold is known)
+  __shared__ float sh_thr;      // gamma once per CTA: a load by every warp hits one L2 line thousands of times
+  if (threadIdx.x == 0) sh_thr = ternary_threshold(__ldcg(gamma), eps);
+  __syncthreads();
+  const float thr = sh_thr;
+  for (; gi < ng; gi += U * stride) {
+    uint4 nxt[U][RW];
+    fetch(gi + U * stride, nxt);  // (zeros past the last group)
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
       const int64_t g = ng - 1 - (gi + u * stride);
       if (g < 0) continue;
-      uint32_t word = 0;
+      uint32_t word = 0, cw[4];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) word |= ternary_digit(v[u][i], thr) << (2 * i);
+      for (int i = 0; i < RW; ++i) {
+        const uint32_t w[4] = {cur[u][i].x, cur[u][i].y, cur[u][i].z, cur[u][i].w};
+        float v[EW];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if constexpr (WDT == BL_F32) {
+            v[j] = __uint_as_float(w[j]);
+          } else {
+            v[2 * j] = __uint_as_float(w[j] << 16);
+            v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < EW; ++j) word |= ternary_digit(v[j], thr) << (2 * (EW * i + j));
+#pragma unroll
+        for (int j = 0; j < EW / 4; ++j) cw[EW / 4 * i + j] = codes4_word(v + 4 * j, thr);
+      }
       reinterpret_cast<uint32_t*>(packed)[g] = word;
-      if (codes != nullptr)
-        reinterpret_cast<uint4*>(codes)[g] = make_uint4(codes4_word(v[u], thr), codes4_word(v[u] + 4, thr),
-                                                        codes4_word(v[u] + 8, thr), codes4_word(v[u] + 12, thr));
+      if (codes != nullptr) reinterpret_cast<uint4*>(codes)[g] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
     }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int i = 0; i < RW; ++i) cur[u][i] = nxt[u][i];
   }
 }
 
@@ -319,6 +362,7 @@ template <int FMT>
 __global__ void __launch_bounds__(256)
     pack_kernel(const int8_t* __restrict__ codes, int64_t N, int64_t K, uint8_t* __restrict__ packed,
                 int64_t rowbytes, void* ws) {
+  pdl_enter(codes, packed, ws);
   constexpr int PER = (FMT == BL_PACK_I2) ? 4 : 5;
   constexpr int WPS = 16 * PER;
   const int64_t segs = rowbytes / 16;
@@ -341,7 +385,7 @@ __global__ void __launch_bounds__(256)
         for (int ii = 0; ii < PER; ++ii) {
           const int i = (FMT == BL_PACK_I2) ? ii : PER - 1 - ii;
           const int kk = (FMT == BL_PACK_I2) ? 16 * w + 4 * b + i : 20 * w + 5 * b + i;
-          int c = (k0 + kk < K) ? static_cast<int>(__ldg(src + kk)) : 0;
+          int c = (k0 + kk < K) ? static_cast<int>(__ldcg(src + kk)) : 0;
           if (c < -1 || c > 1) {
             bad = true;
             c = 0;
@@ -396,10 +440,10 @@ cudaError_t launch_absmean(const void* W, int wdt, int64_t N, int64_t K, void* w
   const int64_t cap = static_cast<int64_t>(device_sms()) * kAbsCtasPerSm;
   const int64_t grid = C < cap ? C : cap;
   if (wdt == BL_F32)
-    absmean_kernel<BL_F32><<<static_cast<unsigned>(grid), kLanes, 0, st>>>(W, T, C, lgR, partials, hdr, gamma);
-  else
-    absmean_kernel<BL_BF16><<<static_cast<unsigned>(grid), kLanes, 0, st>>>(W, T, C, lgR, partials, hdr, gamma);
-  return cudaGetLastError();
+    return launch_pdl(absmean_kernel<BL_F32>, static_cast<unsigned>(grid), kLanes, 0, st, W, T, C, lgR, partials,
+                      hdr, gamma);
+  return launch_pdl(absmean_kernel<BL_BF16>, static_cast<unsigned>(grid), kLanes, 0, st, W, T, C, lgR, partials, hdr,
+                    gamma);
 }
 
 cudaError_t launch_ternarize_pack(const void* W, int wdt, int64_t N, int64_t K, const float* gamma,
@@ -413,35 +457,31 @@ cudaError_t launch_ternarize_pack(const void* W, int wdt, int64_t N, int64_t K, 
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
     if (wdt == BL_F32)
-      ternarize_flat_kernel<BL_F32><<<static_cast<unsigned>(grid), 256, 0, st>>>(W, T, gamma, eps, packed, codes);
-    else
-      ternarize_flat_kernel<BL_BF16><<<static_cast<unsigned>(grid), 256, 0, st>>>(W, T, gamma, eps, packed, codes);
-    return cudaGetLastError();
+      return launch_pdl(ternarize_flat_kernel<BL_F32>, static_cast<unsigned>(grid), 256, 0, st, W, T, gamma, eps,
+                        packed, codes);
+    return launch_pdl(ternarize_flat_kernel<BL_BF16>, static_cast<unsigned>(grid), 256, 0, st, W, T, gamma, eps,
+                      packed, codes);
   }
   const bool vec_ok = (wdt == BL_F32) ? (K % 4 == 0) : (K % 8 == 0);
   const int64_t work = N * (rowbytes / 16);
   const int threads = 256;
   const int grid = grid_for(work, threads, 4);
-#define BL_TP(WDT, FMT)                                                                            \
-  ternarize_pack_kernel<WDT, FMT><<<grid, threads, 0, st>>>(W, N, K, gamma, eps, packed, codes, \
-                                                            rowbytes, vec_ok)
+#define BL_TP(WDT, FMT)                                                                                     \
+  return launch_pdl(ternarize_pack_kernel<WDT, FMT>, grid, threads, 0, st, W, N, K, gamma, eps, packed, codes, \
+                    rowbytes, vec_ok)
   if (wdt == BL_F32 && fmt == BL_PACK_I2) BL_TP(BL_F32, BL_PACK_I2);
   else if (wdt == BL_F32) BL_TP(BL_F32, BL_PACK_T5);
   else if (fmt == BL_PACK_I2) BL_TP(BL_BF16, BL_PACK_I2);
   else BL_TP(BL_BF16, BL_PACK_T5);
 #undef BL_TP
-  return cudaGetLastError();
 }
 
 cudaError_t launch_pack(const int8_t* codes, int64_t N, int64_t K, int fmt, uint8_t* packed,
                         int64_t rowbytes, void* ws, cudaStream_t st) {
   const int64_t work = N * (rowbytes / 16);
   const int grid = grid_for(work, 256, 8);
-  if (fmt == BL_PACK_I2)
-    pack_kernel<BL_PACK_I2><<<grid, 256, 0, st>>>(codes, N, K, packed, rowbytes, ws);
-  else
-    pack_kernel<BL_PACK_T5><<<grid, 256, 0, st>>>(codes, N, K, packed, rowbytes, ws);
-  return cudaGetLastError();
+  if (fmt == BL_PACK_I2) return launch_pdl(pack_kernel<BL_PACK_I2>, grid, 256, 0, st, codes, N, K, packed, rowbytes, ws);
+  return launch_pdl(pack_kernel<BL_PACK_T5>, grid, 256, 0, st, codes, N, K, packed, rowbytes, ws);
 }
 
 }  // namespace bl
