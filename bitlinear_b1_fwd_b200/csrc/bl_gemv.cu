@@ -758,6 +758,242 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Base-3 decode GEMV for one token, column-stationary.  A row of segs 16-byte
+// segments (80 weights each) is cut into nb = ceil(segs / 32) columns of 32
+// segments; warp w < nb kc (kc = kGemvWarps / nb) keeps column c = w mod nb
+// and takes the rows j, j + kc, ... of its CTA (j = w / nb), so lane L holds
+// the 80 activation codes of segment 32 c + L in registers for the whole
+// kernel: xlo[p] = the codes of digits 0..3 of packed byte p of the segment,
+// xhi[j] byte i = the code of digit 4 of packed byte 4 j + i.  At any time the
+// CTA's warps read kc whole rows, one contiguous window.  A packed byte b is
+// decoded by one 4-byte shared lookup: byte j of the entry is the digit
+// d_j = floor(b / 3^j) mod 3 (j < 4) and bits 2..3 of byte 0 hold d_4.  The
+// table has one copy per lane (copy L in bank L), so a warp's 32 lookups are
+// one conflict-free shared access whatever the bytes.  Per packed word: four
+// lookups, four dp4a on the masked entries (digits 0..3 against xlo) and one
+// dp4a on the gathered d_4 (4 d_4 in each byte, against xhi; the factor 4 is
+// taken off at the end).  Digits are q + 1, so sum q x = sum d x - sum x with
+// the sum of the token's codes subtracted once per row.  Bytes 243..255 are
+// not produced by the packer; they decode as five zero weights.
+// ---------------------------------------------------------------------------
+constexpr int kT5Batch = 4;                 // rows per load batch; two batches alternate
+constexpr int kT5LutBytes = 256 * 32 * 4;   // 32 copies of 256 4-byte entries
+constexpr int64_t kT5Prefetch = 65536;      // bytes per CTA prefetched into L2 before the wait
+
+__host__ __device__ inline int64_t gemv_t5_smem_bytes(int64_t rowbytes) {
+  return kT5LutBytes + (rowbytes / 16) * 80 + int64_t{4} * kGemvTileRows;
+}
+
+template <int XDT>
+__global__ void __launch_bounds__(kGemvThreads, 1)
+    gemv_t5_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
+                   int64_t N, int64_t K, const void* __restrict__ x, float* __restrict__ scale,
+                   void* __restrict__ y, int ydt, int write_scale) {
+  const int64_t G = gridDim.x, b = blockIdx.x;
+  const int64_t per = N / G, extra = N % G;
+  const int64_t row0 = b * per + (b < extra ? b : extra);
+  const int nrows = static_cast<int>(per + (b < extra ? 1 : 0));  // <= kGemvTileRows (host-checked)
+  // 0. while the previous kernel finishes: the table, the zeroed row sums and
+  //    an L2 prefetch of the first kT5Prefetch bytes of this CTA's rows
+  pdl_launch_dependents();
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem);           // [256][32]
+  int8_t* xq = reinterpret_cast<int8_t*>(smem + kT5LutBytes);   // [segs * 80] codes, 0 past K
+  const uint32_t segs = static_cast<uint32_t>(rowbytes >> 4);
+  int* racc = reinterpret_cast<int*>(xq + segs * 80);           // [kGemvTileRows]
+  __shared__ float red_f[kGemvWarps];
+  __shared__ int red_i[kGemvWarps];
+  __shared__ float sh_gs[2];
+  {
+    const int64_t bytes = static_cast<int64_t>(nrows) * rowbytes;
+    l2_prefetch_bulk(packed + row0 * rowbytes, bytes < kT5Prefetch ? bytes : kT5Prefetch);
+  }
+  for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
+    const int e = i >> 5;
+    uint32_t d[5] = {1, 1, 1, 1, 1};  // bytes past 242: five zero weights
+    if (e < 243) {
+      int v = e;
+#pragma unroll
+      for (int j = 0; j < 5; ++j) {
+        d[j] = static_cast<uint32_t>(v % 3);
+        v /= 3;
+      }
+    }
+    lut[i] = (d[0] | (d[4] << 2)) | (d[1] << 8) | (d[2] << 16) | (d[3] << 24);
+  }
+  for (int i = threadIdx.x; i < kGemvTileRows; i += blockDim.x) racc[i] = 0;
+  pdl_wait(packed, gamma, x, scale, y);
+  if (threadIdx.x == 0) sh_gs[0] = __ldcg(gamma);
+  if (XDT == BL_I8 && threadIdx.x == 1) sh_gs[1] = __ldcg(scale);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nthr = blockDim.x;
+
+  // 1. the token's INT8 codes: per-token absmax (fp32 / bf16) or the given
+  //    scale (int8); codes past K are 0
+  const uint32_t nq8 = segs * 10;  // groups of eight codes in shared memory
+  const bool vec = (K % 8) == 0;
+  if constexpr (XDT != BL_I8) {
+    float amax = 0.0f;
+    if (vec) {
+      for (int64_t v = threadIdx.x; v < K / 8; v += nthr) {
+        float e[8];
+        load8_aligned<XDT>(x, 8 * v, e);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(e[j]));
+      }
+    } else {
+      for (int64_t k = threadIdx.x; k < K; k += nthr) amax = fmaxf(amax, fabsf(load_x<XDT>(x, k)));
+    }
+    amax = warp_maxf(amax);
+    if (lane == 0) red_f[warp] = amax;
+  }
+  __syncthreads();  // per-warp maxima, the table and the zeroed row sums are visible
+  float s_tok;
+  if constexpr (XDT != BL_I8) {
+    s_tok = fmaxf(warp_maxf(lane < kGemvWarps ? red_f[lane] : 0.0f), 1e-6f);
+  } else {
+    s_tok = sh_gs[1];
+  }
+  const float c127 = (XDT == BL_I8) ? 0.0f : __fdiv_rn(127.0f, s_tok);
+  int part = 0;
+  for (uint32_t v = threadIdx.x; v < nq8; v += nthr) {
+    const int64_t k0 = 8 * static_cast<int64_t>(v);
+    int q[8];
+    if (vec && k0 + 8 <= K) {
+      if constexpr (XDT == BL_I8) {
+        const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(static_cast<const int8_t*>(x) + k0));
+#pragma unroll
+        for (int j = 0; j < 8; ++j) q[j] = static_cast<int8_t>((j < 4 ? raw.x : raw.y) >> (8 * (j & 3)));
+      } else {
+        float e[8];
+        load8_aligned<XDT>(x, k0, e);
+        quant_act_fast_n<8>(e, s_tok, c127, q);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int64_t k = k0 + j;
+        q[j] = (k >= K) ? 0
+               : (XDT == BL_I8) ? static_cast<int>(static_cast<const int8_t*>(x)[k])
+                                : quant_act_fast(load_x<XDT>(x, k), s_tok, c127);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) part += q[j];
+    *reinterpret_cast<uint2*>(xq + k0) = make_uint2(pack4(q), pack4(q + 4));
+  }
+  part = __reduce_add_sync(0xffffffffu, part);
+  if (lane == 0) red_i[warp] = part;
+  __syncthreads();  // the codes, per-warp sums, gamma and the given scale are visible
+  const int corr = __reduce_add_sync(0xffffffffu, lane < kGemvWarps ? red_i[lane] : 0);
+  const float cfac = dequant_factor(sh_gs[0], s_tok);
+  if (XDT != BL_I8 && write_scale && blockIdx.x == 0 && threadIdx.x == 0) scale[0] = s_tok;
+
+  // 2. this lane's activations: segment s = 32 c + lane of the warp's column
+  const int nb = static_cast<int>((segs + 31) >> 5);
+  const int kc = kGemvWarps / nb;
+  const int c = warp % nb, j0 = warp / nb;
+  const uint32_t s = 32u * c + lane;
+  const bool active = warp < nb * kc;
+  const bool mine = active && s < segs;  // lanes past the row's end load nothing and add 0
+  uint32_t xlo[16], xhi[4];
+  {
+    uint32_t w[20];
+    if (mine) {
+      const uint4* xp = reinterpret_cast<const uint4*>(xq + 80 * s);
+#pragma unroll
+      for (int i = 0; i < 5; ++i) {
+        const uint4 t = xp[i];
+        w[4 * i] = t.x;
+        w[4 * i + 1] = t.y;
+        w[4 * i + 2] = t.z;
+        w[4 * i + 3] = t.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 20; ++i) w[i] = 0;
+    }
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {  // codes 5p .. 5p + 3 of the segment
+      const int o = 5 * p;
+      xlo[p] = __byte_perm(w[o >> 2], w[(o >> 2) + 1], 0x3210 + 0x1111 * (o & 3));
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {  // code 5p + 4 of packed bytes p = 4j .. 4j + 3
+      uint32_t h = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = 20 * j + 5 * i + 4;
+        h |= ((w[t >> 2] >> (8 * (t & 3))) & 0xffu) << (8 * i);
+      }
+      xhi[j] = h;
+    }
+  }
+
+  // 3. the warp's rows j0, j0 + kc, ...: kT5Batch loads in flight per batch,
+  //    two batches alternating
+  const uint32_t* lut_l = lut + lane;  // this lane's copy: entry e at lut_l[32 e]
+  const int nmine = (active && j0 < nrows) ? (nrows - 1 - j0) / kc + 1 : 0;
+  const uint8_t* src = packed + (row0 + j0) * rowbytes + 16 * static_cast<int64_t>(s);
+  const int64_t step = static_cast<int64_t>(kc) * rowbytes;
+  int issued = 0, done = 0;
+  uint4 bufA[kT5Batch], bufB[kT5Batch];
+  auto issue = [&](uint4(&bf)[kT5Batch]) {
+#pragma unroll
+    for (int d = 0; d < kT5Batch; ++d) {
+      bf[d] = make_uint4(0, 0, 0, 0);
+      if (mine && issued + d < nmine) bf[d] = ld_stream(reinterpret_cast<const uint4*>(src + (issued + d) * step));
+    }
+    issued += kT5Batch;
+  };
+  auto consume = [&](const uint4(&bf)[kT5Batch]) {
+#pragma unroll
+    for (int d = 0; d < kT5Batch; ++d) {
+      if (done + d >= nmine) break;  // (uniform across the warp)
+      const uint32_t wd[4] = {bf[d].x, bf[d].y, bf[d].z, bf[d].w};
+      int v = 0, vh = 0;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint32_t L[4];
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) L[bb] = lut_l[32 * __byte_perm(wd[w], 0, 0x4440 + bb)];
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) v = dp4a_us(L[bb] & 0x03030303u, xlo[4 * w + bb], v);
+        const uint32_t H =
+            __byte_perm(__byte_perm(L[0], L[1], 0x0040), __byte_perm(L[2], L[3], 0x0040), 0x5410) & 0x0c0c0c0cu;
+        vh = dp4a_us(H, xhi[w], vh);
+      }
+      const int t = __reduce_add_sync(0xffffffffu, v + (vh >> 2));  // vh is 4 sum d_4 x: exact
+      if (lane == 0) atomicAdd(racc + j0 + (done + d) * kc, t);
+    }
+    done += kT5Batch;
+  };
+  if (nmine > 0) {
+    issue(bufA);
+    for (;;) {
+      issue(bufB);
+      consume(bufA);
+      if (done >= nmine) break;
+      issue(bufA);
+      consume(bufB);
+      if (done >= nmine) break;
+    }
+  }
+  __syncthreads();  // every part of every row has been added
+  for (int r = threadIdx.x; r < nrows; r += nthr) {
+    const int a = racc[r] - corr;
+    const int64_t o = row0 + r;
+    if (ydt == BL_I32)
+      static_cast<int32_t*>(y)[o] = a;
+    else if (ydt == BL_F32)
+      static_cast<float*>(y)[o] = __fmul_rn(__int2float_rn(a), cfac);
+    else
+      static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(a), cfac));
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Host side.
 // ---------------------------------------------------------------------------
 int gemv_max_tokens(int fmt, int64_t rowbytes) {
@@ -816,6 +1052,31 @@ static cudaError_t launch_gemv_i2_mt(int mt, const uint8_t* packed, int64_t rowb
   }
 }
 
+// The base-3 column-stationary kernel: rows of at most 32 kGemvWarps
+// segments and at most kGemvTileRows rows per CTA.
+static bool gemv_t5_fits(int64_t rowbytes, int64_t N) {
+  const int64_t sms = device_sms();
+  const int64_t grid = N < sms ? N : sms;
+  return rowbytes / 16 <= 32 * kGemvWarps && (N + grid - 1) / grid <= kGemvTileRows &&
+         gemv_t5_smem_bytes(rowbytes) <= kGemvSmemBudget;
+}
+
+template <int XDT>
+static cudaError_t launch_gemv_t5_t(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N,
+                                    int64_t K, const void* x, float* scale, void* y, int ydt, int write_scale,
+                                    cudaStream_t st) {
+  auto kern = gemv_t5_kernel<XDT>;
+  const size_t smem = static_cast<size_t>(gemv_t5_smem_bytes(rowbytes));
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t sms = device_sms();
+  const int64_t grid = N < sms ? N : sms;  // every CTA owns at least one row
+  e = launch_pdl(kern, static_cast<unsigned>(grid), kGemvThreads, smem, st, packed, rowbytes, gamma, N, K, x, scale,
+                 y, ydt, write_scale);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 template <int FMT, int XDT>
 static cudaError_t launch_gemv_mt(int mt, const uint8_t* packed, int64_t rowbytes, const float* gamma,
                                   int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
@@ -846,7 +1107,11 @@ cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int6
     float* sm = scale + m0;
     void* ym = static_cast<uint8_t*>(y) + m0 * N * ysz;
     cudaError_t e;
-    if (lean) {
+    if (fmt == BL_PACK_T5 && mt == 1 && M == 1 && gemv_t5_fits(rowbytes, N)) {
+      if (xdt == BL_F32) e = launch_gemv_t5_t<BL_F32>(packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
+      else if (xdt == BL_BF16) e = launch_gemv_t5_t<BL_BF16>(packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
+      else e = launch_gemv_t5_t<BL_I8>(packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, st);
+    } else if (lean) {
       if (xdt == BL_F32) e = launch_gemv_i2_mt<BL_F32>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
       else if (xdt == BL_BF16) e = launch_gemv_i2_mt<BL_BF16>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
       else e = launch_gemv_i2_mt<BL_I8>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, st);

@@ -324,3 +324,31 @@ def test_quantize_acts_near_ties(orc):
         y, sm = forward(packed, I2, np.float32(1.0), K, K, x[m:m + 1], B.BL_I32)
         assert np.array_equal(y[0], xq_ref[m].astype(np.int32))
         assert sm[0] == s_ref[m]
+
+
+# --- one-token base-3 decode: the column-stationary kernel and its limits ---------
+
+@pytest.mark.parametrize("N,K,xkind", [(300, 1000, "int8"), (65, 129, "int8"), (97, 8193, "bf16"),
+                                       (37, 61440, "bf16"), (37, 61441, "f32"), (5, 80 * 33, "f32")])
+def test_forward_t5_one_token(orc, N, K, xkind):
+    """Rows of 1..768 segments (the kernel's limit: 61440 weights) and one past
+    it (the general kernel), ragged K, fp32 / bf16 tokens quantized inside and
+    int8 tokens with their given scale."""
+    W = synth.normal_f32(N * 13 + K, (N, K), 0.02)
+    x = synth.normal_f32(K * 5 + N, (1, K))
+    g, _, packed = quantize_weights(W, T5, codes=False)
+    if xkind == "int8":
+        xq, s = orc.act_quant(x)
+        check_forward(orc, packed, T5, g, N, K, xq, scale=s)
+    else:
+        check_forward(orc, packed, T5, g, N, K, synth.to_bf16_bits(x) if xkind == "bf16" else x)
+
+
+def test_forward_t5_many_rows_per_cta(orc):
+    """More rows than one CTA's row sums hold (N > 148 x 1024 on a B200): the
+    general kernel takes the call, with the same results."""
+    N, K = 160_000, 40
+    W = synth.normal_f32(91, (N, K), 0.02)
+    x = synth.normal_f32(92, (1, K))
+    g, _, packed = quantize_weights(W, T5, codes=False)
+    check_forward(orc, packed, T5, g, N, K, x, ydts=(B.BL_I32, B.BL_BF16))
