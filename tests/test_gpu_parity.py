@@ -352,3 +352,31 @@ def test_forward_t5_many_rows_per_cta(orc):
     x = synth.normal_f32(92, (1, K))
     g, _, packed = quantize_weights(W, T5, codes=False)
     check_forward(orc, packed, T5, g, N, K, x, ydts=(B.BL_I32, B.BL_BF16))
+
+
+# --- one-token 2-bit decode: the lean kernel and its limits ----------------------------
+
+@pytest.mark.parametrize("N,K,xkind", [(300, 1000, "int8"), (150, 4104, "int8"), (97, 8193, "bf16"),
+                                       (149, 32768, "bf16"), (37, 32769, "f32"), (5, 64, "f32"),
+                                       (2000, 2048, "bf16")])
+def test_forward_i2_one_token(orc, N, K, xkind):
+    """Rows of 16 B .. 8 KB (the lean kernel's limit: K = 32768) and one past
+    it (the general kernel), CTAs with one to many rows, ragged K, fp32 / bf16
+    tokens quantized inside and int8 tokens with their given scale."""
+    W = synth.normal_f32(N * 11 + K, (N, K), 0.02)
+    x = synth.normal_f32(K * 7 + N, (1, K))
+    g, _, packed = quantize_weights(W, I2, codes=False)
+    if xkind == "int8":
+        xq, s = orc.act_quant(x)
+        check_forward(orc, packed, I2, g, N, K, xq, scale=s)
+    else:
+        check_forward(orc, packed, I2, g, N, K, synth.to_bf16_bits(x) if xkind == "bf16" else x)
+
+
+def test_forward_i2_many_rows_per_cta(orc):
+    """More rows than one CTA's row sums hold: the lean kernel's row tiles."""
+    N, K = 160_000, 64
+    W = synth.normal_f32(93, (N, K), 0.02)
+    x = synth.to_bf16_bits(synth.normal_f32(94, (1, K)))
+    g, _, packed = quantize_weights(W, I2, codes=False)
+    check_forward(orc, packed, I2, g, N, K, x, ydts=(B.BL_I32, B.BL_BF16))
