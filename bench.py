@@ -591,6 +591,53 @@ def prefill_summary(p):
             "steps": p["steps"], "l2": f"inputs rotated over {p['rot']} copies (> 2x L2)"}
 
 
+# Small standalone cases for ncu captures: one call repeated a few times on one
+# shape, with seeded N(0, sigma) latent weights and N(0, 1) bf16 tokens drawn on
+# the device.  Launch order: the weight preparation (absmean, ternarize + pack)
+# once, then three forwards; a "quantize" case runs the preparation three times.
+PROFILE_CASES = {
+    "quantize_3b_up": dict(N=8640, K=3200, fmt=0, M=1, sigma=0.02, op="quantize"),
+    "decode_3b_up": dict(N=8640, K=3200, fmt=0, M=1, sigma=0.02, op="forward"),
+    "decode_70b_up": dict(N=28672, K=8192, fmt=0, M=1, sigma=0.01, op="forward"),
+    "decode_70b_down": dict(N=8192, K=28672, fmt=0, M=1, sigma=0.01, op="forward"),
+    "decode_70b_up_t5": dict(N=28672, K=8192, fmt=1, M=1, sigma=0.01, op="forward"),
+    "prefill_3b": dict(N=8640, K=3200, fmt=0, M=4096, sigma=0.02, op="forward"),
+}
+
+
+def run_profile_case(name):
+    import torch
+
+    from bitlinear_b1_fwd_b200 import binding as B
+    from bitlinear_b1_fwd_b200 import build as libbuild
+
+    c = PROFILE_CASES[name]
+    libbuild.build()
+    dev = torch.device("cuda", 0)
+    N, K, M, fmt = c["N"], c["K"], c["M"], c["fmt"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    W = torch.randn(N, K, generator=g, device=dev) * c["sigma"]
+    x = torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16)
+    packed = torch.empty((N, B.bitlinear_packed_row_bytes(K, fmt)), dtype=torch.uint8, device=dev)
+    gamma = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = torch.zeros(B.bitlinear_quantize_weights_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+    for _ in range(3 if c["op"] == "quantize" else 1):
+        B.bitlinear_quantize_weights(W, 1e-5, fmt, packed, None, gamma, ws)
+    status = [B.bitlinear_device_status(ws)]
+    if c["op"] == "forward":
+        scale = torch.empty(M, dtype=torch.float32, device=dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        fws = torch.zeros(B.bitlinear_forward_workspace_bytes(M, N, K, fmt, B.BL_BF16), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            B.bitlinear_forward(packed, fmt, gamma, N, K, x, scale, y, fws)
+        status.append(B.bitlinear_device_status(fws))
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": name, **c, "status": status}))
+    if any(status):
+        sys.exit(1)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -608,7 +655,12 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--cpu-budget", type=float, default=10.0,
                     help="seconds of oracle time for the cpu_baseline sample (0 = skip)")
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES), default=None,
+                    help="run one small standalone case (for ncu captures) and exit")
     args = ap.parse_args()
+    if args.profile_case:
+        run_profile_case(args.profile_case)
+        return
     wl = WORKLOADS[args.workload]
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
