@@ -409,7 +409,8 @@ def run_gpu(args, wl, rank, world, local_rank):
 
     prefill = run_prefill(args, dev, stream, rank_seed, l2) if args.prefill else None
     decode = run_decode(args, dev, stream, rank_seed, l2) if args.decode else None
-    res = dict(prefill=prefill, decode=decode, ms_total=ms_max, per_op_ms=per_op_ms, step_bytes=step_bytes,
+    sweep = run_sweep(args, dev, stream, l2) if args.sweep else None
+    res = dict(prefill=prefill, decode=decode, sweep=sweep, ms_total=ms_max, per_op_ms=per_op_ms, step_bytes=step_bytes,
                layers=layers, ops=ops,
                clocks=sampler.summary(), e2e_ms=e2e_ms, e2e_steps=e2e_steps, h2d=h2d, d2h=d2h,
                rot=rot, l2=l2, launches_per_step=len(layers) * len(ops))
@@ -534,6 +535,108 @@ def run_decode(args, dev, stream, rank_seed, l2):
     return out
 
 
+def run_sweep(args, dev, stream, l2):
+    """Config sweeps (opt-in): the 70B layers (2-bit) over M = 1, 2, 4, ..., 8192
+    and the 3B block's six BitLinears (Q, K, V, O, up, down, each with its
+    own per-token quantization) as one graph per block at M = 1, 16, 128, 1024.
+    Latent weights N(0, sigma) and bf16 tokens N(0, 1) are drawn on the device
+    with a seeded generator (parity on the host-generated recipe is the tests'
+    job); packed weights and tokens rotate over copies past 4x L2 where they
+    fit.  Each point: a graph of back-to-back calls timed at its two ends."""
+    import torch
+
+    from bitlinear_b1_fwd_b200 import binding as B
+    from bitlinear_b1_fwd_b200 import synth
+
+    peak_gbs, _ = measured_peaks()
+    peak_tops, _ = measured_int8_peak()
+    g = torch.Generator(device=dev)
+
+    def prep(N, K, sigma, seed):
+        g.manual_seed(seed)
+        W = torch.randn(N, K, generator=g, device=dev) * sigma
+        rb = B.bitlinear_packed_row_bytes(K, 0)
+        packed = torch.empty((N, rb), dtype=torch.uint8, device=dev)
+        gamma = torch.empty(1, dtype=torch.float32, device=dev)
+        ws = torch.zeros(B.bitlinear_quantize_weights_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+        with torch.cuda.stream(stream):
+            B.bitlinear_quantize_weights(W, 1e-5, 0, packed, None, gamma, ws, stream)
+        stream.synchronize()
+        return packed, gamma, rb
+
+    def point(N, K, M, rb, us):
+        nbytes = N * rb + M * K * 2 + M * N * 2 + 4 * M + 4
+        ops = 2.0 * M * N * K
+        gbs = nbytes / (us * 1e-6) / 1e9
+        tops = ops / (us * 1e-6) / 1e12
+        kern = gemv_kernel_name(0, [(N, K)], M) if M <= 4 else gemm_kernel_name(M)
+        return {"M": M, "us": us, "GB_s": gbs, "frac_of_hbm": gbs / peak_gbs, "TOPS": tops,
+                "frac_of_int8": tops / peak_tops, "kernel": kern}
+
+    out = {"layer_70b": {}, "block_3b": []}
+    for li, c in enumerate(synth.LAYER_70B):
+        N, K = c["N"], c["K"]
+        p0, gamma, rb = prep(N, K, c["w_sigma"], 1005 + 100 * li)
+        pk = [p0] + [p0.clone() for _ in range(max(0, -(-4 * l2 // (N * rb)) - 1))]
+        pts = []
+        for M in synth.LAYER_70B_M:
+            xr = max(1, min(4, -(-4 * l2 // (M * K * 2))))
+            g.manual_seed(2005 + 100 * li + M)
+            xs = [torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16) for _ in range(xr)]
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            sc = torch.empty(M, dtype=torch.float32, device=dev)
+            fws = torch.zeros(B.bitlinear_forward_workspace_bytes(M, N, K, 0, B.BL_BF16), dtype=torch.uint8,
+                              device=dev)
+
+            def fwd(j, M=M, xs=xs, y=y, sc=sc, fws=fws):
+                B.bitlinear_forward(pk[j % len(pk)], 0, gamma, N, K, xs[j % len(xs)], sc, y, fws, stream)
+
+            with torch.cuda.stream(stream):
+                for j in range(3):
+                    fwd(j)
+            steps = 100 if M <= 16 else (30 if M <= 512 else 6)
+            us = graph_ms(stream, steps, fwd) / steps * 1e3
+            if B.bitlinear_device_status(fws, stream) != B.BL_OK:
+                raise RuntimeError("sweep device status")
+            pts.append(point(N, K, M, rb, us))
+            del xs, y, fws
+        out["layer_70b"][c["name"]] = {"N": N, "K": K, "points": pts}
+        del pk, p0
+    blk = [prep(c["N"], c["K"], 0.02, 1004 + 100 * i) for i, c in enumerate(synth.BLOCK_3B)]
+    blk_bytes = sum(c["N"] * rb for c, (_, _, rb) in zip(synth.BLOCK_3B, blk))
+    rot = max(1, -(-4 * l2 // blk_bytes))
+    copies = [[p] + [p.clone() for _ in range(rot - 1)] for (p, _, _) in blk]
+    for M in synth.BLOCK_3B_M:
+        g.manual_seed(2004 + M)
+        xs = [torch.randn(M, c["K"], generator=g, device=dev).to(torch.bfloat16) for c in synth.BLOCK_3B]
+        ys = [torch.empty((M, c["N"]), dtype=torch.bfloat16, device=dev) for c in synth.BLOCK_3B]
+        scs = [torch.empty(M, dtype=torch.float32, device=dev) for _ in synth.BLOCK_3B]
+        fwss = [torch.zeros(B.bitlinear_forward_workspace_bytes(M, c["N"], c["K"], 0, B.BL_BF16),
+                            dtype=torch.uint8, device=dev) for c in synth.BLOCK_3B]
+
+        def block(j, M=M, xs=xs, ys=ys, scs=scs, fwss=fwss):
+            for i, c in enumerate(synth.BLOCK_3B):
+                B.bitlinear_forward(copies[i][j % rot], 0, blk[i][1], c["N"], c["K"], xs[i], scs[i], ys[i],
+                                    fwss[i], stream)
+
+        with torch.cuda.stream(stream):
+            for j in range(3):
+                block(j)
+        steps = 50 if M <= 128 else 10
+        us = graph_ms(stream, steps, block) / steps * 1e3
+        nbytes = sum(c["N"] * rb + M * c["K"] * 2 + M * c["N"] * 2 + 4 * M + 4
+                     for c, (_, _, rb) in zip(synth.BLOCK_3B, blk))
+        ops = sum(2.0 * M * c["N"] * c["K"] for c in synth.BLOCK_3B)
+        out["block_3b"].append({"M": M, "us_per_block": us, "GB_s": nbytes / (us * 1e-6) / 1e9,
+                                "frac_of_hbm": nbytes / (us * 1e-6) / 1e9 / peak_gbs,
+                                "TOPS": ops / (us * 1e-6) / 1e12,
+                                "frac_of_int8": ops / (us * 1e-6) / 1e12 / peak_tops})
+        del xs, ys, scs, fwss
+    out["note"] = ("graphs of back-to-back forward calls timed at their two ends; bytes = packed weights + bf16 x + "
+                   "bf16 y; TOPS = 2 M N K; fractions of the measured HBM copy rate and of the int8 peak")
+    return out
+
+
 def decode_summary(d):
     if d is None:
         return None
@@ -602,6 +705,8 @@ PROFILE_CASES = {
     "decode_70b_down": dict(N=8192, K=28672, fmt=0, M=1, sigma=0.01, op="forward"),
     "decode_70b_up_t5": dict(N=28672, K=8192, fmt=1, M=1, sigma=0.01, op="forward"),
     "prefill_3b": dict(N=8640, K=3200, fmt=0, M=4096, sigma=0.02, op="forward"),
+    "batch16_70b_up": dict(N=28672, K=8192, fmt=0, M=16, sigma=0.01, op="forward"),
+    "batch16_70b_down": dict(N=8192, K=28672, fmt=0, M=16, sigma=0.01, op="forward"),
 }
 
 
@@ -655,6 +760,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--cpu-budget", type=float, default=10.0,
                     help="seconds of oracle time for the cpu_baseline sample (0 = skip)")
+    ap.add_argument("--sweep", action=argparse.BooleanOptionalAction, default=False,
+                    help="also time the 70B layers over M = 1..8192 and the 3B block at M = 1, 16, 128, 1024")
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES), default=None,
                     help="run one small standalone case (for ncu captures) and exit")
     args = ap.parse_args()
@@ -754,6 +861,7 @@ def main():
                     "d2h_bytes_per_step": res["d2h"], "steps": res["e2e_steps"]},
             "prefill": prefill_summary(res["prefill"]),
             "decode_gemv": decode_summary(res["decode"]),
+            "sweep": res["sweep"],
             "gpu_launches": res["launches_per_step"] * args.steps,
             "clocks": res["clocks"],
         }

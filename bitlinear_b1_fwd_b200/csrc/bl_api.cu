@@ -69,6 +69,8 @@ size_t bitlinear_forward_workspace_bytes(int64_t M, int64_t N, int64_t K, int fm
   if (uses_gemm(M, K)) {
     if (xdt != BL_I8) bytes += round256(static_cast<size_t>(M * K));
     if (fmt == BL_PACK_T5) bytes += round256(static_cast<size_t>(N * bitlinear_packed_row_bytes(K, BL_PACK_I2)));
+    const int ks = bl::gemm_split_k(M, N, K);
+    if (ks > 1) bytes += round256(static_cast<size_t>(ks) * M * N * sizeof(int32_t));
   }
   return bytes;
 }
@@ -170,8 +172,10 @@ bl_status bitlinear_forward(const uint8_t* packed, int fmt, const float* gamma, 
     if (bl::launch_t5_to_i2(packed, N, K, bitlinear_packed_row_bytes(K, fmt), scratch, rb2, st) != cudaSuccess)
       return BL_ERR_CUDA;
     w2 = scratch;
+    scratch += round256(static_cast<size_t>(N * rb2));
   }
-  return cuda_status(bl::launch_gemm_i2(xq, w2, rb2, gamma, scale, y, ydt, M, N, K, ws, 0, 0, st));
+  int32_t* part = bl::gemm_split_k(M, N, K) > 1 ? reinterpret_cast<int32_t*>(scratch) : nullptr;
+  return cuda_status(bl::launch_gemm_i2(xq, w2, rb2, gamma, scale, y, ydt, M, N, K, part, ws, 0, 0, st));
 }
 
 bl_status bitlinear_selftest_wait_timeout(void* ws, size_t ws_bytes, void* stream) {
@@ -181,7 +185,7 @@ bl_status bitlinear_selftest_wait_timeout(void* ws, size_t ws_bytes, void* strea
   uint8_t* op = static_cast<uint8_t*>(ws) + BL_WS_HEADER_BYTES;
   const float* g = reinterpret_cast<const float*>(op);
   return cuda_status(bl::launch_gemm_i2(reinterpret_cast<const int8_t*>(op), op, 32, g, g, op, BL_I32, 16, 128,
-                                        128, ws, int64_t{1} << 20, 1, static_cast<cudaStream_t>(stream)));
+                                        128, nullptr, ws, int64_t{1} << 20, 1, static_cast<cudaStream_t>(stream)));
 }
 
 bl_status bitlinear_device_status(void* ws, void* stream) {

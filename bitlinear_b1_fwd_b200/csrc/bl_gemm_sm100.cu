@@ -17,9 +17,13 @@
 //     accumulator in tensor memory, double-buffered across tiles;
 //   - four epilogue warps read the accumulator with tcgen05.ld, dequantize
 //     and store, overlapping the next tile's main loop.
-// The kernel is persistent (one CTA per SM, tiles strided by the grid).  Every
-// wait is bounded: on expiry the kernel sets the workspace timeout flag, drains
-// what it issued, frees its tensor memory and returns.
+// The kernels are persistent (one CTA or CTA pair per SM, work strided by the
+// grid).  For 5..128 tokens the one-SM kernel keeps a deep ring of TMA stages
+// apart from the ring of expanded tiles, and splits each tile's K range when
+// there are too few tiles for the SMs (INT32 partial sums, added by a small
+// reduction kernel).  Every wait is bounded: on expiry the kernel sets the
+// workspace timeout flag, drains what it issued, frees its tensor memory and
+// returns.
 #include <cuda.h>
 #include <cstring>
 
@@ -31,7 +35,6 @@ namespace bl {
 namespace {
 
 constexpr int kGemmThreads = 384;  // warp 0 TMA, 1 MMA, 4-7 expansion, 8-11 epilogue
-constexpr int kStages = 4;
 constexpr int kBN = 128;  // weight rows per tile = MMA M
 constexpr int kBK = 128;  // K per stage = 4 MMAs of K = 32
 constexpr uint32_t kPackedStage = kBN * kBK / 4;  // 4096 bytes
@@ -126,39 +129,76 @@ __device__ __forceinline__ uint4 expand16(uint32_t w) {
   return o;
 }
 
+// One-SM tiles (5..128 tokens).  A work unit is a tile of 128 weight rows x BT
+// tokens over a range of k-blocks (128 K each): with ks > 1 the k-blocks of a
+// tile are cut into ks parts (units = tiles x ks, so that a small layer still
+// spreads over every SM), each unit writes its INT32 partial sums to
+// part[kz][t][n] and splitk_reduce_kernel adds the parts and dequantizes.
+// Three rings decouple the streams:
+//   - packed tiles of 128 rows x 128 B (four k-blocks: one full 128-byte line
+//     per row and TMA request; 128-byte swizzled, so that the expansion's
+//     16-byte reads of eight rows hit eight different bank groups), kSP
+//     stages, released by the expansion warps;
+//   - x_q tiles [BT x 128 B] per k-block, kSX stages, released by the MMAs;
+//   - expanded int8 tiles per k-block, kSB stages, released by the MMAs.
+// The expansion warps take whole k-blocks in turn (warp v the k-blocks with
+// index v mod kExp): one warp's pass over a k-block is a chain of long
+// latencies (barrier test, shared loads, stores, proxy fence, arrive), and
+// with the k-blocks dealt out several of them are in flight at once (rows
+// dealt out instead left one k-block per ~0.5 us).  Each waiter takes its
+// stages in order and waits for a stage's release before its data, so with
+// kSB >= kExp and kSB + 3 <= 4 kSP no waiter is two phases ahead of a
+// barrier.
+constexpr size_t kGemmSmemBudget = 227 * 1024;  // dynamic shared memory per CTA
+constexpr int kGroup = 4;                                 // k-blocks per packed tile
+constexpr uint32_t kPackedTile = kBN * kGroup * kBK / 4;  // 16384 bytes
+constexpr int kSXMax = 16;     // x_q ring, at most
+
 template <int BT>
 struct GemmCfg {
   static constexpr uint32_t kXStage = BT * 128;
   static constexpr uint32_t kTmemCols = (2 * BT < 32) ? 32 : 2 * BT;
   static constexpr uint32_t kChunk = BT < 32 ? BT : 32;  // accumulator columns per tcgen05.ld
-  // output staging for the TMA-store epilogue: 2 x [kChunk tokens x 128 rows],
-  // up to 4 bytes each (none for 256-token tiles, which do not fit it)
-  static constexpr uint32_t kYStage1 = (BT <= 128) ? kChunk * 128 * 4 : 0;
-  static constexpr size_t kSmem = 1024 + kStages * (kXStage + kExpStage + kPackedStage) + 2 * kYStage1 +
-                                  8 * (3 * kStages + 5) + 16 + 2 * 4 * BT;
+  static constexpr uint32_t kYStage1 = kChunk * 128 * 4;  // output staging (TMA-store epilogue), x2
+  static constexpr int kExp = BT <= 32 ? 8 : 4;                  // expansion warps
+  static constexpr int kSB = BT <= 32 ? 8 : (BT <= 64 ? 5 : 4);  // expanded-tile ring (>= kExp)
+  static constexpr int kSP = BT == 32 ? 3 : 4;                   // packed-tile ring
+  static constexpr int kThreads = 32 * (4 + kExp + 4);  // TMA, MMA, 2 idle | expansion | epilogue
+  static_assert(kSB >= kExp && kSB + 3 <= 4 * kSP, "ring depths");
+  static constexpr size_t kFixed = 1024 + kSB * kExpStage + kSP * kPackedTile + 2 * kYStage1 +
+                                   8 * (2 * kSXMax + 2 * kSP + 2 * kSB + 5) + 16 + 2 * 4 * BT;
+  static_assert(kFixed + 2 * kXStage <= kGemmSmemBudget, "shared memory");
+  static constexpr size_t kFit = (kGemmSmemBudget - kFixed) / kXStage;
+  static constexpr int kSX = kFit > kSXMax ? kSXMax : static_cast<int>(kFit);
+  static constexpr size_t kSmem = kFixed + kSX * kXStage;
+  static_assert(kSX >= 2, "x_q ring");
 };
 
 template <int BT>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(GemmCfg<BT>::kThreads, 1)
     gemm_i2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                    const __grid_constant__ CUtensorMap tm_y, int y_tma, const float* __restrict__ gamma,
-                   const float* __restrict__ scale, void* __restrict__ y, int ydt, int M, int N, int K,
-                   WsHeader* __restrict__ hdr, long long limit, int skip_producer) {
-  pdl_enter(gamma, scale, y, hdr);
+                   const float* __restrict__ scale, void* __restrict__ y, int ydt, int M, int N, int K, int ks,
+                   int32_t* __restrict__ part, WsHeader* __restrict__ hdr, long long limit, int skip_producer) {
+  pdl_enter(gamma, scale, y, part, hdr);
   using Cfg = GemmCfg<BT>;
+  constexpr int SX = Cfg::kSX, SP = Cfg::kSP, SB = Cfg::kSB;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* base = smem_raw + pad;
-  uint8_t* xs = base;                              // kStages x [BT x 128 B], swizzled
-  uint8_t* es = xs + kStages * Cfg::kXStage;       // kStages x [128 x 128 B], swizzled
-  uint8_t* ps = es + kStages * kExpStage;          // kStages x [128 x 32 B]
-  uint8_t* ystage = ps + kStages * kPackedStage;   // 2 x [kChunk tokens x 128 rows] output staging
-  uint64_t* full = reinterpret_cast<uint64_t*>(ystage + 2 * Cfg::kYStage1);
-  uint64_t* expd = full + kStages;
-  uint64_t* empty = expd + kStages;
-  uint64_t* accf = empty + kStages;  // 2
-  uint64_t* acce = accf + 2;         // 2
-  uint64_t* drain = acce + 2;        // 1
+  uint8_t* es = base;                              // SB x [128 x 128 B], swizzled (1024-aligned)
+  uint8_t* ps = es + SB * kExpStage;               // SP x [128 rows x 128 B] packed
+  uint8_t* xs = ps + SP * kPackedTile;             // SX x [BT x 128 B], swizzled
+  uint8_t* ystage = xs + SX * Cfg::kXStage;        // 2 x [kChunk tokens x 128 rows] output staging
+  uint64_t* xfull = reinterpret_cast<uint64_t*>(ystage + 2 * Cfg::kYStage1);
+  uint64_t* xempty = xfull + SX;
+  uint64_t* pfull = xempty + SX;
+  uint64_t* pempty = pfull + SP;
+  uint64_t* expd = pempty + SP;
+  uint64_t* emptyB = expd + SB;
+  uint64_t* accf = emptyB + SB;  // 2
+  uint64_t* acce = accf + 2;     // 2
+  uint64_t* drain = acce + 2;    // 1
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* cfac = reinterpret_cast<float*>(tmem_slot + 4);  // [2][BT] dequant factors per accumulator buffer
@@ -167,13 +207,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int kblocks = (K + kBK - 1) / kBK;
   const int n_tiles = (N + kBN - 1) / kBN;
   const int t_tiles = (M + BT - 1) / BT;
-  const int tiles = n_tiles * t_tiles;
+  const int units = n_tiles * t_tiles * ks;  // ks <= kblocks (host-checked): no unit is empty
+  struct Unit {
+    int n_t, t_t, kz, kb0, kb1;
+  };
+  auto unit_of = [&](int u) {
+    Unit w;
+    w.n_t = u % n_tiles;
+    const int r = u / n_tiles;
+    w.kz = r % ks;
+    w.t_t = r / ks;
+    w.kb0 = static_cast<int>((static_cast<int64_t>(w.kz) * kblocks) / ks);
+    w.kb1 = static_cast<int>((static_cast<int64_t>(w.kz + 1) * kblocks) / ks);
+    return w;
+  };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(full + s, 1);
-      mbar_init(expd + s, 4);
-      mbar_init(empty + s, 1);
+    for (int s = 0; s < SX; ++s) {
+      mbar_init(xfull + s, 1);
+      mbar_init(xempty + s, 1);
+    }
+    for (int s = 0; s < SP; ++s) {
+      mbar_init(pfull + s, 1);
+      mbar_init(pempty + s, kGroup);  // one arrival per k-block of the tile
+    }
+    for (int b = 0; b < SB; ++b) {
+      mbar_init(expd + b, 1);  // the warp that expanded it
+      mbar_init(emptyB + b, 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(accf + a, 1);
@@ -201,27 +261,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
+    // per unit: for each group of kGroup k-blocks its packed tile, then the
+    // x_q tile of each of its k-blocks
     if (lane == 0 && !skip_producer) {
-      int it = 0;
+      int ix = 0, ip = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-        const int n_t = tile % n_tiles, t_t = tile / n_tiles;
-        for (int kb = 0; kb < kblocks; ++kb, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
-          if (!wait1(empty + s, ph ^ 1, limit, abort_flag)) {
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const Unit w = unit_of(u);
+        for (int kb = w.kb0; kb < w.kb1 && ok; ++kb) {
+          if ((kb - w.kb0) % kGroup == 0) {
+            const int s = ip % SP;
+            if (!wait1(pempty + s, ((ip / SP) & 1) ^ 1, limit, abort_flag)) {
+              fail(0x203);
+              ok = false;
+              break;
+            }
+            mbar_expect_tx(pfull + s, kPackedTile);
+            tma_load_2d(ps + s * kPackedTile, &tm_w, pfull + s, kb * (kBK / 4), w.n_t * kBN);
+            ++ip;
+          }
+          const int s = ix % SX;
+          if (!wait1(xempty + s, ((ix / SX) & 1) ^ 1, limit, abort_flag)) {
             fail(0x201);
             ok = false;
             break;
           }
-          mbar_expect_tx(full + s, Cfg::kXStage + kPackedStage);
-          tma_load_2d(xs + s * Cfg::kXStage, &tm_x, full + s, kb * kBK, t_t * BT);
-          tma_load_2d(ps + s * kPackedStage, &tm_w, full + s, kb * (kBK / 4), n_t * kBN);
+          mbar_expect_tx(xfull + s, Cfg::kXStage);
+          tma_load_2d(xs + s * Cfg::kXStage, &tm_x, xfull + s, kb * kBK, w.t_t * BT);
+          ++ix;
         }
       }
       // copies still in flight land before the CTA leaves (bounded)
-      for (int j = (it > kStages ? it - kStages : 0); j < it; ++j)
-        (void)wait_drain(full + (j % kStages), (j / kStages) & 1, limit);
+      for (int j = (ix > SX ? ix - SX : 0); j < ix; ++j) (void)wait_drain(xfull + (j % SX), (j / SX) & 1, limit);
+      for (int j = (ip > SP ? ip - SP : 0); j < ip; ++j) (void)wait_drain(pfull + (j % SP), (j / SP) & 1, limit);
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ---------------------------------
@@ -229,7 +301,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       constexpr uint32_t idesc = i8_idesc(kBN, BT);
       int it = 0, tc = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tc) {
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++tc) {
+        const Unit w = unit_of(u);
         const int a = tc & 1;
         if (!wait1(acce + a, ((tc >> 1) & 1) ^ 1, limit, abort_flag)) {
           fail(0x301);
@@ -237,20 +310,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         const uint32_t d = tmem + static_cast<uint32_t>(a * BT);
-        for (int kb = 0; kb < kblocks; ++kb, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
-          if (!wait1(full + s, ph, limit, abort_flag) || !wait1(expd + s, ph, limit, abort_flag)) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+          const int s = it % SX, b = it % SB;
+          if (!wait1(xfull + s, (it / SX) & 1, limit, abort_flag) || !wait1(expd + b, (it / SB) & 1, limit, abort_flag)) {
             fail(0x302);
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t xa = smem_u32(xs + s * Cfg::kXStage), ea = smem_u32(es + s * kExpStage);
+          const uint32_t xa = smem_u32(xs + s * Cfg::kXStage), ea = smem_u32(es + b * kExpStage);
 #pragma unroll
           for (int k = 0; k < kBK / 32; ++k)
-            mma_i8(d, sw128_desc(ea + 32 * k), sw128_desc(xa + 32 * k), idesc, (kb | k) != 0);
-          mma_commit(empty + s);
+            mma_i8(d, sw128_desc(ea + 32 * k), sw128_desc(xa + 32 * k), idesc, (kb != w.kb0 || k != 0) ? 1u : 0u);
+          mma_commit(xempty + s);  // the x_q tile has been read
+          mma_commit(emptyB + b);  // the expanded tile has been read
         }
         if (ok) mma_commit(accf + a);
       }
@@ -258,52 +331,77 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mma_commit(drain);
       (void)wait_drain(drain, 0, limit);
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= 4 && warp < 4 + Cfg::kExp) {
     // ------------------------------ expansion ----------------------------------
-    const int r = threadIdx.x - 128;  // weight row of the tile, 0..127
-    int it = 0;
+    // warp v expands the k-blocks it with it % kExp == v, whole: lane L the
+    // rows L, L + 32, L + 64, L + 96
+    const int v = warp - 4;
+    int it = 0, ip = 0;  // k-blocks and packed tiles of the CTA so far (every warp counts all)
     bool ok = true;
-    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-      for (int kb = 0; kb < kblocks; ++kb, ++it) {
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
-        if (!wait_warp(full + s, ph, limit, abort_flag)) {
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      const Unit w = unit_of(u);
+      const int nk = w.kb1 - w.kb0;
+      for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+        const int i = kb - w.kb0, j = i % kGroup;
+        const int gsz = (nk - (i - j)) < kGroup ? (nk - (i - j)) : kGroup;  // k-blocks of this packed tile
+        const int tile_ip = ip;
+        if (j == gsz - 1) ++ip;
+        if (it % Cfg::kExp != v) continue;
+        const int sp = tile_ip % SP, b = it % SB;
+        if (!wait_warp(emptyB + b, ((it / SB) & 1) ^ 1, limit, abort_flag)) {
+          if (lane == 0) fail(0x402);
+          ok = false;
+          break;
+        }
+        if (!wait_warp(pfull + sp, (tile_ip / SP) & 1, limit, abort_flag)) {
           if (lane == 0) fail(0x401);
           ok = false;
           break;
         }
-        const uint4* src = reinterpret_cast<const uint4*>(ps + s * kPackedStage + r * 32);
-        const uint4 p0 = src[0], p1 = src[1];
-        const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-        uint8_t* row = es + s * kExpStage + (r >> 3) * 1024 + (r & 7) * 128;
+        const uint8_t* pt = ps + sp * kPackedTile;
+        uint8_t* et_ = es + b * kExpStage;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<uint4*>(row + ((j ^ (r & 7)) << 4)) = expand16(w[j]);
+        for (int rr = 0; rr < 4; ++rr) {
+          const int r = lane + 32 * rr;
+          const uint8_t* prow = pt + (r >> 3) * 1024 + (r & 7) * 128;  // swizzled 128-byte row
+          const uint4 p0 = *reinterpret_cast<const uint4*>(prow + (((2 * j) ^ (r & 7)) << 4));
+          const uint4 p1 = *reinterpret_cast<const uint4*>(prow + (((2 * j + 1) ^ (r & 7)) << 4));
+          const uint32_t wd[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+          uint8_t* row = et_ + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = expand16(wd[c]);
+        }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
-        if (lane == 0) mbar_arrive(expd + s);
+        if (lane == 0) {
+          mbar_arrive(expd + b);
+          // the last k-block of a short tile also stands for its missing ones
+          mbar_arrive_n(pempty + sp, j == gsz - 1 ? static_cast<uint32_t>(kGroup - gsz + 1) : 1u);
+        }
       }
     }
-  } else if (warp >= 8) {
+  } else if (warp >= 4 + Cfg::kExp) {
     // ------------------------------ epilogue -----------------------------------
-    // (with a tensor map for y, chunks of the accumulator leave through a
-    // shared staging tile and TMA tensor stores, as in the two-SM kernel)
+    // (ks == 1: dequantize and store, through a shared staging tile and TMA
+    // tensor stores when y has a tensor map; ks > 1: the raw INT32 partial
+    // sums to part[kz][t][n], coalesced along n)
     const int q = warp & 3;  // TMEM lane quarter this warp may read
-    const int et = threadIdx.x - 256;
+    const int et = threadIdx.x - 32 * (4 + Cfg::kExp);
     const uint32_t esz = (ydt == BL_BF16) ? 2u : 4u;
-    const bool use_tma = y_tma != 0 && Cfg::kYStage1 != 0;
+    const bool use_tma = y_tma != 0 && ks == 1;
     const float g = __ldcg(gamma);
     int tc = 0, chunk = 0;
-    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++tc) {
+      const Unit w = unit_of(u);
       const int a = tc & 1;
-      const int n_t = tile % n_tiles, t_t = tile / n_tiles;
-      const int n = n_t * kBN + 32 * q + lane;
+      const int n = w.n_t * kBN + 32 * q + lane;
       // dequant factor c_t = (gamma s_t) / 127 of each token of the tile, once
       float* cf = cfac + a * BT;
-      for (int j = et; j < BT; j += 128) {
-        const int t = t_t * BT + j;
-        cf[j] = (t < M && ydt != BL_I32) ? dequant_factor(g, __ldcg(scale + t)) : 0.0f;
-      }
+      if (ks == 1)
+        for (int j = et; j < BT; j += 128) {
+          const int t = w.t_t * BT + j;
+          cf[j] = (t < M && ydt != BL_I32) ? dequant_factor(g, __ldcg(scale + t)) : 0.0f;
+        }
       const uint32_t ok_w = wait_warp(accf + a, (tc >> 1) & 1, limit, abort_flag) ? 1u : 0u;
       // the four epilogue warps agree (and see each other's factors) before going on
       uint32_t ok_all;
@@ -325,8 +423,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t acc[Cfg::kChunk];
         tmem_load<Cfg::kChunk>(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(a * BT + j0),
                                acc);
-        const int t0 = t_t * BT + j0;
-        if (use_tma) {
+        const int t0 = w.t_t * BT + j0;
+        if (ks > 1) {
+          if (n < N) {
+#pragma unroll
+            for (int j = 0; j < static_cast<int>(Cfg::kChunk); ++j)
+              if (t0 + j < M) part[(static_cast<int64_t>(w.kz) * M + t0 + j) * N + n] = static_cast<int32_t>(acc[j]);
+          }
+        } else if (use_tma) {
           uint8_t* sb = ystage + (chunk & 1) * Cfg::kYStage1;
           if (chunk >= 2) {  // the store issued from this buffer two chunks ago has read it
             if (et == 0) bulk_wait_read<1>();
@@ -348,7 +452,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           fence_proxy_async_smem();
           asm volatile("bar.sync 2, 128;" ::: "memory");
-          if (et == 0 && n_t * kBN < N && t0 < M) tma_store_2d(&tm_y, sb, n_t * kBN, t0);
+          if (et == 0 && w.n_t * kBN < N && t0 < M) tma_store_2d(&tm_y, sb, w.n_t * kBN, t0);
           if (et == 0) bulk_commit();
         } else {
 #pragma unroll
@@ -383,6 +487,57 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(Cfg::kTmemCols)
                  : "memory");
+  }
+}
+
+// The ks partial sums of each output (exact INT32 addition, any order), then
+// the dequantization y = acc * (gamma s_t) / 127 as in the GEMM epilogues.
+// Four consecutive outputs per thread when N % 4 == 0.
+__global__ void __launch_bounds__(256)
+    splitk_reduce_kernel(const int32_t* __restrict__ part, int ks, int M, int N, const float* __restrict__ gamma,
+                         const float* __restrict__ scale, void* __restrict__ y, int ydt) {
+  pdl_enter(part, gamma, scale, y);
+  __shared__ float sh_g;  // gamma once per CTA
+  if (threadIdx.x == 0) sh_g = __ldcg(gamma);
+  __syncthreads();
+  const float g = sh_g;
+  const int64_t plane = static_cast<int64_t>(M) * N;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  auto emit = [&](int64_t o, int t, int v) {
+    if (ydt == BL_I32) {
+      static_cast<int32_t*>(y)[o] = v;
+    } else {
+      const float yv = __fmul_rn(__int2float_rn(v), dequant_factor(g, __ldcg(scale + t)));
+      if (ydt == BL_F32)
+        static_cast<float*>(y)[o] = yv;
+      else
+        static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(yv);
+    }
+  };
+  if ((N % 4) == 0) {
+    const int64_t n4 = plane / 4;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4; i += stride) {
+      int4 s = __ldcg(reinterpret_cast<const int4*>(part) + i);
+      for (int kz = 1; kz < ks; ++kz) {
+        const int4 p = __ldcg(reinterpret_cast<const int4*>(part + kz * plane) + i);
+        s.x += p.x;
+        s.y += p.y;
+        s.z += p.z;
+        s.w += p.w;
+      }
+      const int64_t o = 4 * i;
+      const int t = static_cast<int>(o / N);
+      emit(o, t, s.x);
+      emit(o + 1, t, s.y);
+      emit(o + 2, t, s.z);
+      emit(o + 3, t, s.w);
+    }
+  } else {
+    for (int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; o < plane; o += stride) {
+      int s = __ldcg(part + o);
+      for (int kz = 1; kz < ks; ++kz) s += __ldcg(part + kz * plane + o);
+      emit(o, static_cast<int>(o / N), s);
+    }
   }
 }
 
@@ -789,28 +944,37 @@ bool encode_y(CUtensorMap* m, void* y, int ydt, int64_t M, int64_t N, uint32_t t
 
 template <int BT>
 cudaError_t launch_gemm_bt(const int8_t* xq, const uint8_t* w, int64_t rb, const float* gamma, const float* scale,
-                           void* y, int ydt, int64_t M, int64_t N, int64_t K, void* ws, long long limit,
-                           int skip_producer, cudaStream_t st) {
+                           void* y, int ydt, int64_t M, int64_t N, int64_t K, int ks, int32_t* part, void* ws,
+                           long long limit, int skip_producer, cudaStream_t st) {
   CUtensorMap tx, tw;
   if (!encode_2d_u8(&tx, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(K), 128, BT,
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (!encode_2d_u8(&tw, w, static_cast<uint64_t>(rb), static_cast<uint64_t>(N), static_cast<uint64_t>(rb),
-                    kBK / 4, kBN, CU_TENSOR_MAP_SWIZZLE_NONE))
+                    kGroup * kBK / 4, kBN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   CUtensorMap ty;
-  const int y_tma = (GemmCfg<BT>::kYStage1 != 0 && encode_y(&ty, y, ydt, M, N, GemmCfg<BT>::kChunk)) ? 1 : 0;
+  const int y_tma = (ks == 1 && encode_y(&ty, y, ydt, M, N, GemmCfg<BT>::kChunk)) ? 1 : 0;
   if (!y_tma) memset(&ty, 0, sizeof(ty));
   auto kern = gemm_i2_kernel<BT>;
   const size_t smem = GemmCfg<BT>::kSmem;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int64_t tiles = ((N + kBN - 1) / kBN) * ((M + BT - 1) / BT);
+  const int64_t units = ((N + kBN - 1) / kBN) * ((M + BT - 1) / BT) * ks;
   const int sms = device_sms();
-  const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
-  { const cudaError_t le_ = launch_pdl(kern, grid, kGemmThreads, smem, st, tx, tw, ty, y_tma, gamma, scale, y, ydt, static_cast<int>(M),
-                                         static_cast<int>(N),
-                                         static_cast<int>(K), static_cast<WsHeader*>(ws), limit, skip_producer); if (le_ != cudaSuccess) return le_; }
+  const unsigned grid = static_cast<unsigned>(units < sms ? units : sms);
+  e = launch_pdl(kern, grid, GemmCfg<BT>::kThreads, smem, st, tx, tw, ty, y_tma, gamma, scale, y, ydt, static_cast<int>(M),
+                 static_cast<int>(N), static_cast<int>(K), ks, part, static_cast<WsHeader*>(ws), limit,
+                 skip_producer);
+  if (e != cudaSuccess) return e;
+  if (ks > 1) {
+    const int64_t work = (N % 4 == 0) ? M * N / 4 : M * N;
+    int64_t rgrid = (work + 255) / 256;
+    if (rgrid > 8 * sms) rgrid = 8 * sms;
+    e = launch_pdl(splitk_reduce_kernel, static_cast<unsigned>(rgrid), 256, 0, st, static_cast<const int32_t*>(part),
+                   ks, static_cast<int>(M), static_cast<int>(N), gamma, scale, y, ydt);
+    if (e != cudaSuccess) return e;
+  }
   return cudaGetLastError();
 }
 
@@ -852,18 +1016,40 @@ int gemm_token_tile(int64_t M) {
   return 16;
 }
 
+// Split of the k-blocks of each one-SM tile: the ks in 1..16 (at most the
+// number of k-blocks) with the smallest per-SM makespan in k-blocks, waves x
+// (k-blocks per unit + 4), plus 12 for the reduction pass when ks > 1.
+int gemm_split_k(int64_t M, int64_t N, int64_t K) {
+  if (M > 128) return 1;
+  const int64_t bt = gemm_token_tile(M);
+  const int64_t tiles = ((N + kBN - 1) / kBN) * ((M + bt - 1) / bt);
+  const int64_t kblocks = (K + kBK - 1) / kBK;
+  const int64_t sms = device_sms();
+  int best = 1;
+  int64_t best_cost = -1;
+  for (int ks = 1; ks <= 16 && ks <= kblocks; ++ks) {
+    const int64_t waves = (tiles * ks + sms - 1) / sms;
+    const int64_t cost = waves * ((kblocks + ks - 1) / ks + 4) + (ks > 1 ? 12 : 0);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = ks;
+    }
+  }
+  return best;
+}
+
 cudaError_t launch_gemm_i2(const int8_t* xq, const uint8_t* w, int64_t rb, const float* gamma, const float* scale,
-                           void* y, int ydt, int64_t M, int64_t N, int64_t K, void* ws, long long limit_cycles,
-                           int skip_producer, cudaStream_t st) {
+                           void* y, int ydt, int64_t M, int64_t N, int64_t K, int32_t* part, void* ws,
+                           long long limit_cycles, int skip_producer, cudaStream_t st) {
   const long long limit = limit_cycles > 0 ? limit_cycles : kTimeoutCycles;
   if (M > 128 && !skip_producer)
     return launch_gemm_2sm<256>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ws, limit, st);
+  const int ks = (part != nullptr && !skip_producer) ? gemm_split_k(M, N, K) : 1;
   switch (gemm_token_tile(M)) {
-    case 16: return launch_gemm_bt<16>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ws, limit, skip_producer, st);
-    case 32: return launch_gemm_bt<32>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ws, limit, skip_producer, st);
-    case 64: return launch_gemm_bt<64>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ws, limit, skip_producer, st);
-    case 128: return launch_gemm_bt<128>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ws, limit, skip_producer, st);
-    default: return launch_gemm_bt<256>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ws, limit, skip_producer, st);
+    case 16: return launch_gemm_bt<16>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ks, part, ws, limit, skip_producer, st);
+    case 32: return launch_gemm_bt<32>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ks, part, ws, limit, skip_producer, st);
+    case 64: return launch_gemm_bt<64>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ks, part, ws, limit, skip_producer, st);
+    default: return launch_gemm_bt<128>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ks, part, ws, limit, skip_producer, st);
   }
 }
 

@@ -104,7 +104,10 @@ BL_API size_t bitlinear_quantize_weights_workspace_bytes(int64_t N, int64_t K);
 
 /* Workspace bytes needed by bitlinear_forward for these sizes and formats (the
  * header, plus x_q when activations are quantized ahead of the tensor-core
- * path, plus a 2-bit copy of base-3 weights for that path). */
+ * path, plus a 2-bit copy of base-3 weights for that path, plus the INT32
+ * partial sums when a layer with few tokens (5..128) is split along K so
+ * that it spreads over every SM; the split depends on the device's SM
+ * count, so query on the device that runs the call). */
 BL_API size_t bitlinear_forward_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int xdt);
 
 /* Zero the status header of a workspace (enqueued on `stream`). */
