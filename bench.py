@@ -57,7 +57,7 @@ WORKLOADS = {
 
 KERNEL_SOURCE = {"absmean_kernel": "bl_weights.cu", "ternarize_flat_kernel": "bl_weights.cu",
                  "ternarize_pack_kernel": "bl_weights.cu", "gemv_i2_kernel": "bl_gemv.cu",
-                 "gemv_kernel": "bl_gemv.cu", "gemv_t5_kernel": "bl_gemv.cu", "act_quant_row_kernel": "bl_acts.cu",
+                 "gemv_kernel": "bl_gemv.cu", "gemv_t5_kernel": "bl_gemv.cu", "gemv_i2_mt_kernel": "bl_gemv.cu", "act_quant_row_kernel": "bl_acts.cu",
                  "act_quant_kernel": "bl_acts.cu", "gemm_i2_2sm_kernel": "bl_gemm_sm100.cu",
                  "gemm_i2_kernel": "bl_gemm_sm100.cu"}
 
@@ -659,13 +659,17 @@ def decode_summary(d):
 
 
 def gemv_kernel_name(fmt, layers, M=1):
-    """The decode kernel the forward dispatches to (M <= 4): the lean 2-bit
-    kernel for rows of at most 8192 packed bytes; for one token of base 3,
+    """The decode kernel the forward dispatches to (M <= 4): for 2..4 tokens
+    of 2-bit rows of at most 8192 bytes (and at most 1024 rows per CTA) the
+    column-stationary multi-token kernel, else the lean 2-bit kernel for rows
+    of at most 8192 packed bytes; for one token of base 3,
     the column-stationary kernel for rows of at most 768 segments and at most
     1024 rows per CTA (148 CTAs); else the general one."""
     if fmt == 0:
-        lean = all(((K + 3) // 4 + 15) // 16 * 16 <= 8192 for (_, K) in layers)
-        return "gemv_i2_kernel" if lean else "gemv_kernel"
+        rbs = [((K + 3) // 4 + 15) // 16 * 16 for (_, K) in layers]
+        if 2 <= M <= 4 and all(rb <= 8192 and -(-N // min(N, 148)) <= 1024 for rb, (N, _) in zip(rbs, layers)):
+            return "gemv_i2_mt_kernel"
+        return "gemv_i2_kernel" if all(rb <= 8192 for rb in rbs) else "gemv_kernel"
     t5 = M == 1 and all(((K + 4) // 5 + 15) // 16 <= 768 and -(-N // min(N, 148)) <= 1024 for (N, K) in layers)
     return "gemv_t5_kernel" if t5 else "gemv_kernel"
 

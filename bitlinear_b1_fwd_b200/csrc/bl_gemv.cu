@@ -758,6 +758,232 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// 2-bit decode GEMV for 2..4 tokens, column-stationary.  As in gemv_t5_kernel,
+// a row of segs 16-byte segments (64 weights each) is cut into nb columns of
+// 32 segments; warp w < nb kc (kc = kMtWarps / nb) keeps column w mod nb and
+// takes every kc-th row of its CTA, so lane L holds, for each of the MT tokens,
+// the 64 codes of segment 32 c + L in registers (16 words, in the digit order
+// of the packed words) for the whole kernel: the weights are read once and no
+// token code is read from shared memory per row.  Per row and packed word:
+// four digit masks (taken in place), then four dp4a per token into four
+// accumulators whose factors 4^j come off exactly at the end of the row, one
+// warp reduction and one shared atomic per token.  Digits are q + 1, so the
+// sum of each token's codes is subtracted once per row.
+// ---------------------------------------------------------------------------
+constexpr int kMtThreads = 512;               // 16 warps: 16 MT + load registers per lane
+constexpr int kMtWarps = kMtThreads / 32;
+constexpr int kMtBatch = 2;                   // rows per load batch; two batches alternate
+constexpr int64_t kMtPrefetch = 65536;        // bytes per CTA prefetched into L2 before the wait
+
+__host__ __device__ inline int64_t gemv_mt_smem_bytes(int64_t rowbytes, int mt) {
+  return int64_t{4} * rowbytes * mt + int64_t{4} * kGemvTileRows * mt;  // codes | row sums
+}
+
+template <int MT, int XDT>
+__global__ void __launch_bounds__(kMtThreads, 1)
+    gemv_i2_mt_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
+                      int64_t N, int64_t K, const void* __restrict__ x, float* __restrict__ scale,
+                      void* __restrict__ y, int ydt, int write_scale) {
+  const int64_t G = gridDim.x, b = blockIdx.x;
+  const int64_t per = N / G, extra = N % G;
+  const int64_t row0 = b * per + (b < extra ? b : extra);
+  const int nrows = static_cast<int>(per + (b < extra ? 1 : 0));  // <= kGemvTileRows (host-checked)
+  const uint32_t segs = static_cast<uint32_t>(rowbytes >> 4);
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint8_t* xs = smem;                                             // [MT][4][segs][16] codes
+  int* racc = reinterpret_cast<int*>(xs + 4 * rowbytes * MT);     // [MT][kGemvTileRows]
+  __shared__ float red_f[MT][kMtWarps];
+  __shared__ int red_i[MT][kMtWarps];
+  __shared__ float sh_gs[1 + MT];
+  // 0. while the previous kernel finishes: zeroed row sums and an L2 prefetch
+  pdl_launch_dependents();
+  {
+    const int64_t bytes = static_cast<int64_t>(nrows) * rowbytes;
+    l2_prefetch_bulk(packed + row0 * rowbytes, bytes < kMtPrefetch ? bytes : kMtPrefetch);
+  }
+  for (int i = threadIdx.x; i < MT * kGemvTileRows; i += blockDim.x) racc[i] = 0;
+  pdl_wait(packed, gamma, x, scale, y);
+  if (threadIdx.x <= MT && (threadIdx.x == 0 || XDT == BL_I8))
+    sh_gs[threadIdx.x] = __ldcg(threadIdx.x == 0 ? gamma : scale + (threadIdx.x - 1));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nthr = blockDim.x;
+
+  // 1. the tokens' INT8 codes in the general 2-bit layout (packed word w of
+  //    segment s: 16 codes at (w segs + s) 16, byte 4 j + b = x[64 s + 16 w + 4 b + j])
+  const bool vec = (K % 8) == 0;
+  if constexpr (XDT != BL_I8) {
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      float amax = 0.0f;
+      if (vec) {
+        for (int64_t v = threadIdx.x; v < K / 8; v += nthr) {
+          float e[8];
+          load8_aligned<XDT>(x, m * K + 8 * v, e);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(e[j]));
+        }
+      } else {
+        for (int64_t k = threadIdx.x; k < K; k += nthr) amax = fmaxf(amax, fabsf(load_x<XDT>(x, m * K + k)));
+      }
+      amax = warp_maxf(amax);
+      if (lane == 0) red_f[m][warp] = amax;
+    }
+  }
+  __syncthreads();  // per-warp maxima, zeroed row sums, gamma and the given scales are visible
+  float s_tok[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    if constexpr (XDT != BL_I8) {
+      float a = red_f[m][0];
+#pragma unroll
+      for (int w = 1; w < kMtWarps; ++w) a = fmaxf(a, red_f[m][w]);
+      s_tok[m] = fmaxf(a, 1e-6f);
+    } else {
+      s_tok[m] = sh_gs[1 + m];
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    int part = 0;
+    const float c127 = (XDT == BL_I8) ? 0.0f : __fdiv_rn(127.0f, s_tok[m]);
+    uint8_t* xm = xs + 4 * rowbytes * m;
+    for (uint32_t g = threadIdx.x; g < 4 * segs; g += nthr) {  // one packed word's 16 codes
+      const int64_t k0 = 16 * static_cast<int64_t>(g);
+      uint32_t P[4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t kh = k0 + 8 * h;
+        int q[8];
+        if (vec && kh + 8 <= K) {
+          if constexpr (XDT == BL_I8) {
+            const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(static_cast<const int8_t*>(x) + m * K + kh));
+#pragma unroll
+            for (int j = 0; j < 8; ++j) q[j] = static_cast<int8_t>((j < 4 ? raw.x : raw.y) >> (8 * (j & 3)));
+          } else {
+            float e[8];
+            load8_aligned<XDT>(x, m * K + kh, e);
+            quant_act_fast_n<8>(e, s_tok[m], c127, q);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int64_t k = kh + j;
+            q[j] = (k >= K) ? 0
+                   : (XDT == BL_I8) ? static_cast<int>(static_cast<const int8_t*>(x)[m * K + k])
+                                    : quant_act_fast(load_x<XDT>(x, m * K + k), s_tok[m], c127);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) part += q[j];
+        P[2 * h] = pack4(q);
+        P[2 * h + 1] = pack4(q + 4);
+      }
+      const uint32_t s = g >> 2, w = g & 3;
+      *reinterpret_cast<uint4*>(xm + (w * segs + s) * 16) = i2_slot(P[0], P[1], P[2], P[3]);
+    }
+    part = __reduce_add_sync(0xffffffffu, part);
+    if (lane == 0) red_i[m][warp] = part;
+  }
+  __syncthreads();  // the codes and per-warp sums are visible
+  int corr[MT];
+  float cfac[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    int t = 0;
+#pragma unroll
+    for (int w = 0; w < kMtWarps; ++w) t += red_i[m][w];
+    corr[m] = t;
+    cfac[m] = dequant_factor(sh_gs[0], s_tok[m]);
+    if (XDT != BL_I8 && write_scale && blockIdx.x == 0 && threadIdx.x == 0) scale[m] = s_tok[m];
+  }
+
+  // 2. this lane's codes: segment s = 32 c + lane of the warp's column
+  const int nb = static_cast<int>((segs + 31) >> 5);
+  const int kc = kMtWarps / nb;
+  const int c = warp % nb, j0 = warp / nb;
+  const uint32_t s = 32u * c + lane;
+  const bool active = warp < nb * kc;
+  const bool mine = active && s < segs;  // lanes past the row's end load nothing and add 0
+  uint4 X[MT][4];
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+      X[m][w] = mine ? *reinterpret_cast<const uint4*>(xs + 4 * rowbytes * m + (w * segs + s) * 16)
+                     : make_uint4(0, 0, 0, 0);
+
+  // 3. the warp's rows j0, j0 + kc, ...: kMtBatch loads in flight per batch,
+  //    two batches alternating
+  const int nmine = (active && j0 < nrows) ? (nrows - 1 - j0) / kc + 1 : 0;
+  const uint8_t* src = packed + (row0 + j0) * rowbytes + 16 * static_cast<int64_t>(s);
+  const int64_t step = static_cast<int64_t>(kc) * rowbytes;
+  int issued = 0, done = 0;
+  uint4 bufA[kMtBatch], bufB[kMtBatch];
+  auto issue = [&](uint4(&bf)[kMtBatch]) {
+#pragma unroll
+    for (int d = 0; d < kMtBatch; ++d) {
+      bf[d] = make_uint4(0, 0, 0, 0);
+      if (mine && issued + d < nmine) bf[d] = ld_stream(reinterpret_cast<const uint4*>(src + (issued + d) * step));
+    }
+    issued += kMtBatch;
+  };
+  auto consume = [&](const uint4(&bf)[kMtBatch]) {
+#pragma unroll
+    for (int d = 0; d < kMtBatch; ++d) {
+      if (done + d >= nmine) break;  // (uniform across the warp)
+      const uint32_t wd[4] = {bf[d].x, bf[d].y, bf[d].z, bf[d].w};
+      int a0[MT], a1[MT], a2[MT], a3[MT];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) a0[m] = a1[m] = a2[m] = a3[m] = 0;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const uint32_t c0 = wd[w] & 0x03030303u, c1 = wd[w] & 0x0c0c0c0cu;
+        const uint32_t c2 = wd[w] & 0x30303030u, c3 = wd[w] & 0xc0c0c0c0u;
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          a0[m] = dp4a_us(c0, X[m][w].x, a0[m]);
+          a1[m] = dp4a_us(c1, X[m][w].y, a1[m]);
+          a2[m] = dp4a_us(c2, X[m][w].z, a2[m]);
+          a3[m] = dp4a_us(c3, X[m][w].w, a3[m]);
+        }
+      }
+      const int r = j0 + (done + d) * kc;
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const int t = __reduce_add_sync(0xffffffffu, a0[m] + (a1[m] >> 2) + (a2[m] >> 4) + (a3[m] >> 6));
+        if (lane == 0) atomicAdd(racc + m * kGemvTileRows + r, t);
+      }
+    }
+    done += kMtBatch;
+  };
+  if (nmine > 0) {
+    issue(bufA);
+    for (;;) {
+      issue(bufB);
+      consume(bufA);
+      if (done >= nmine) break;
+      issue(bufA);
+      consume(bufB);
+      if (done >= nmine) break;
+    }
+  }
+  __syncthreads();  // every part of every row has been added
+  for (int r = threadIdx.x; r < nrows; r += nthr) {
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      const int a = racc[m * kGemvTileRows + r] - corr[m];
+      const int64_t o = m * N + row0 + r;
+      if (ydt == BL_I32)
+        static_cast<int32_t*>(y)[o] = a;
+      else if (ydt == BL_F32)
+        static_cast<float*>(y)[o] = __fmul_rn(__int2float_rn(a), cfac[m]);
+      else
+        static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(a), cfac[m]));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Base-3 decode GEMV for one token, column-stationary.  A row of segs 16-byte
 // segments (80 weights each) is cut into nb = ceil(segs / 32) columns of 32
 // segments; warp w < nb kc (kc = kGemvWarps / nb) keeps column c = w mod nb
@@ -1052,6 +1278,42 @@ static cudaError_t launch_gemv_i2_mt(int mt, const uint8_t* packed, int64_t rowb
   }
 }
 
+// The multi-token column-stationary kernel: 2-bit rows of at most
+// 32 kMtWarps segments and at most kGemvTileRows rows per CTA.
+static bool gemv_mt_fits(int64_t rowbytes, int64_t N, int mt) {
+  const int64_t sms = device_sms();
+  const int64_t grid = N < sms ? N : sms;
+  return rowbytes / 16 <= 32 * kMtWarps && (N + grid - 1) / grid <= kGemvTileRows &&
+         gemv_mt_smem_bytes(rowbytes, mt) <= kGemvSmemBudget;
+}
+
+template <int MT, int XDT>
+static cudaError_t launch_gemv_mt_cs(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N,
+                                     int64_t K, const void* x, float* scale, void* y, int ydt, int write_scale,
+                                     cudaStream_t st) {
+  auto kern = gemv_i2_mt_kernel<MT, XDT>;
+  const size_t smem = static_cast<size_t>(gemv_mt_smem_bytes(rowbytes, MT));
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t sms = device_sms();
+  const int64_t grid = N < sms ? N : sms;  // every CTA owns at least one row
+  e = launch_pdl(kern, static_cast<unsigned>(grid), kMtThreads, smem, st, packed, rowbytes, gamma, N, K, x, scale, y,
+                 ydt, write_scale);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <int XDT>
+static cudaError_t launch_gemv_mt_cs_n(int mt, const uint8_t* packed, int64_t rowbytes, const float* gamma,
+                                       int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
+                                       int write_scale, cudaStream_t st) {
+  switch (mt) {
+    case 2: return launch_gemv_mt_cs<2, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
+    case 3: return launch_gemv_mt_cs<3, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
+    default: return launch_gemv_mt_cs<4, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
+  }
+}
+
 // The base-3 column-stationary kernel: rows of at most 32 kGemvWarps
 // segments and at most kGemvTileRows rows per CTA.
 static bool gemv_t5_fits(int64_t rowbytes, int64_t N) {
@@ -1107,7 +1369,11 @@ cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int6
     float* sm = scale + m0;
     void* ym = static_cast<uint8_t*>(y) + m0 * N * ysz;
     cudaError_t e;
-    if (fmt == BL_PACK_T5 && mt == 1 && M == 1 && gemv_t5_fits(rowbytes, N)) {
+    if (fmt == BL_PACK_I2 && mt >= 2 && mt <= 4 && gemv_mt_fits(rowbytes, N, mt)) {
+      if (xdt == BL_F32) e = launch_gemv_mt_cs_n<BL_F32>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
+      else if (xdt == BL_BF16) e = launch_gemv_mt_cs_n<BL_BF16>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
+      else e = launch_gemv_mt_cs_n<BL_I8>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, st);
+    } else if (fmt == BL_PACK_T5 && mt == 1 && M == 1 && gemv_t5_fits(rowbytes, N)) {
       if (xdt == BL_F32) e = launch_gemv_t5_t<BL_F32>(packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
       else if (xdt == BL_BF16) e = launch_gemv_t5_t<BL_BF16>(packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
       else e = launch_gemv_t5_t<BL_I8>(packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, st);
