@@ -75,6 +75,10 @@ def lib() -> C.CDLL:
             L.orc_forward.restype = i
             L.orc_onebit.argtypes = [p, i64, p, p, p]
             L.orc_onebit.restype = None
+            L.orc_layernorm.argtypes = [p, i, p, p, f, i64, i64, p]
+            L.orc_layernorm.restype = None
+            L.orc_layernorm_quant.argtypes = [p, i, p, p, f, i64, i64, p, p, p]
+            L.orc_layernorm_quant.restype = None
             L.orc_f32_to_bf16.argtypes = [f]
             L.orc_f32_to_bf16.restype = C.c_uint16
             L.orc_bf16_to_f32.argtypes = [C.c_uint16]
@@ -249,3 +253,29 @@ def f32_to_bf16(v: float) -> int:
 
 def bf16_to_f32(h: int) -> np.float32:
     return np.float32(lib().orc_bf16_to_f32(int(h)))
+
+
+# --- pre-norm: LayerNorm + per-token INT8 quantization ---------------------------
+
+def layernorm(x: np.ndarray, g: np.ndarray, b: np.ndarray, eps: float = 1e-5) -> np.ndarray:
+    """LayerNorm of each token (fixed-order fp64 mean and variance), bf16 bits out."""
+    x = np.ascontiguousarray(x)
+    M, K = x.shape
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    b = np.ascontiguousarray(b, dtype=np.float32)
+    y = np.empty((M, K), np.uint16)
+    lib().orc_layernorm(_ptr(x), _dt(x), _ptr(g), _ptr(b), float(eps), M, K, _ptr(y))
+    return y
+
+
+def layernorm_quant(x: np.ndarray, g: np.ndarray, b: np.ndarray, eps: float = 1e-5):
+    """LayerNorm then per-token absmax INT8: returns (y bf16 bits, x_q, scale)."""
+    x = np.ascontiguousarray(x)
+    M, K = x.shape
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    b = np.ascontiguousarray(b, dtype=np.float32)
+    y = np.empty((M, K), np.uint16)
+    xq = np.empty((M, K), np.int8)
+    s = np.empty((M,), np.float32)
+    lib().orc_layernorm_quant(_ptr(x), _dt(x), _ptr(g), _ptr(b), float(eps), M, K, _ptr(y), _ptr(xq), _ptr(s))
+    return y, xq, s

@@ -347,3 +347,62 @@ void orc_onebit(const float *w, int64_t n, int8_t *b, float *alpha,
   *beta = (float)(sa / (double)n);
   for (int64_t i = 0; i < n; ++i) b[i] = (int8_t)(w[i] > a ? 1 : -1);
 }
+
+/* ------------------------------------------------------------------------ */
+/* Pre-norm + step 4: LayerNorm of each token, then per-token absmax INT8.  */
+/* [P5] "The BitLinear Recipe" step 1 (the input is quantized with absmax   */
+/* scaling after LayerNorm, whose output has a stable scale); [P3] §5.5    */
+/* (the training configuration keeps LayerNorm in high precision, bf16 for */
+/* the activations between layers).                                       */
+/* Readings: LayerNorm over a token's K values with elementwise fp32      */
+/* weight g and bias b and eps added to the (biased) variance; the mean    */
+/* and the variance are sums in fp64 in a fixed order -- lane l in         */
+/* [0, 256) adds the elements l, l + 256, l + 512, ... of the token in turn */
+/* from 0.0, and the 256 lane sums combine by the stride-halving tree      */
+/* p[l] += p[l + s], s = 128, ..., 1 (lanes with no element hold 0.0) --   */
+/* mu = S1 / K, var = S2 / K with S2 the sum of (x - mu)^2 in that order,  */
+/* r = 1 / sqrt(var + eps) (fp64, correctly rounded); y = ((x - mu) r) g + b */
+/* in fp64, one rounding per operation, then rounded to fp32 and to bf16;  */
+/* the bf16 y is then quantized exactly as orc_act_quant does.             */
+/* ------------------------------------------------------------------------ */
+
+static double token_tree_sum(const double *lane_sum) {
+  double p[256];
+  for (int l = 0; l < 256; ++l) p[l] = lane_sum[l];
+  for (int s = 128; s >= 1; s >>= 1)
+    for (int l = 0; l < s; ++l) p[l] = p[l] + p[l + s];
+  return p[0];
+}
+
+void orc_layernorm(const void *x, int dt, const float *g, const float *b, float eps, int64_t M,
+                   int64_t K, uint16_t *y) {
+  double lane[256];
+  for (int64_t m = 0; m < M; ++m) {
+    for (int l = 0; l < 256; ++l) {
+      double acc = 0.0;
+      for (int64_t k = l; k < K; k += 256) acc = acc + (double)load_f(x, dt, m * K + k);
+      lane[l] = acc;
+    }
+    const double mu = token_tree_sum(lane) / (double)K;
+    for (int l = 0; l < 256; ++l) {
+      double acc = 0.0;
+      for (int64_t k = l; k < K; k += 256) {
+        const double d = (double)load_f(x, dt, m * K + k) - mu;
+        acc = acc + d * d;
+      }
+      lane[l] = acc;
+    }
+    const double var = token_tree_sum(lane) / (double)K;
+    const double r = 1.0 / sqrt(var + (double)eps);
+    for (int64_t k = 0; k < K; ++k) {
+      const double v = (((double)load_f(x, dt, m * K + k) - mu) * r) * (double)g[k] + (double)b[k];
+      y[m * K + k] = orc_f32_to_bf16((float)v);
+    }
+  }
+}
+
+void orc_layernorm_quant(const void *x, int dt, const float *g, const float *b, float eps,
+                         int64_t M, int64_t K, uint16_t *y, int8_t *xq, float *scale) {
+  orc_layernorm(x, dt, g, b, eps, M, K, y);
+  orc_act_quant(y, ORC_BF16, M, K, xq, scale);
+}
