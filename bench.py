@@ -58,7 +58,7 @@ WORKLOADS = {
 KERNEL_SOURCE = {"absmean_kernel": "bl_weights.cu", "ternarize_flat_kernel": "bl_weights.cu",
                  "ternarize_pack_kernel": "bl_weights.cu", "gemv_i2_kernel": "bl_gemv.cu",
                  "gemv_kernel": "bl_gemv.cu", "gemv_t5_kernel": "bl_gemv.cu", "gemv_i2_mt_kernel": "bl_gemv.cu", "act_quant_row_kernel": "bl_acts.cu",
-                 "act_quant_kernel": "bl_acts.cu", "gemm_i2_2sm_kernel": "bl_gemm_sm100.cu",
+                 "act_quant_kernel": "bl_acts.cu", "ln_quant_kernel": "bl_acts.cu", "gemm_i2_2sm_kernel": "bl_gemm_sm100.cu",
                  "gemm_i2_kernel": "bl_gemm_sm100.cu"}
 
 
@@ -458,13 +458,23 @@ def run_prefill(args, dev, stream, rank_seed, l2):
         r = i % rot
         B.bitlinear_forward(pk[r], 0, gamma, N, K, xq[r], sc[r], ys[r], fws, stream)
 
+    # pre-norm variant of step 4: LayerNorm of each token, then INT8 (seeded N(1, 0.1) / N(0, 0.1) parameters)
+    ln_w = torch.from_numpy(synth.normal_f32(95, (K,), 0.1) + np.float32(1.0)).to(dev)
+    ln_b = torch.from_numpy(synth.normal_f32(96, (K,), 0.1)).to(dev)
+
+    def lnq(i):
+        r = i % rot
+        B.bitlinear_layernorm_quantize_acts(xs[r], ln_w, ln_b, 1e-5, xq[r], sc[r], None, stream)
+
     steps = max(1, args.prefill_steps)
     with torch.cuda.stream(stream):
         for i in range(3):
+            lnq(i)
             act(i)
             gemm(i)
     stream.synchronize()
     # each call timed as a graph of `steps` launches of it alone (rotating inputs)
+    ln_ms = graph_ms(stream, steps, lnq) / steps
     act_ms = graph_ms(stream, steps, act) / steps
     gemm_ms = graph_ms(stream, steps, gemm) / steps
     st = B.bitlinear_device_status(fws, stream)
@@ -472,7 +482,7 @@ def run_prefill(args, dev, stream, rank_seed, l2):
         raise RuntimeError(f"prefill device status {B.status_string(st)}")
     ops = 2.0 * M * N * K
     return dict(M=M, K=K, N=N, act_ms=act_ms, gemm_ms=gemm_ms, ops=ops, rot=rot, steps=steps,
-                act_bytes=M * K * 2 + M * K + 4 * M)
+                act_bytes=M * K * 2 + M * K + 4 * M, ln_ms=ln_ms, ln_bytes=M * K * 2 + 2 * K * 4 + M * K + 4 * M)
 
 
 DECODE_SHAPES = {"3b": ("3b_decode", "3B decode: M=1, K=3200->N=8640 and K=8640->N=3200"),
@@ -692,6 +702,9 @@ def prefill_summary(p):
             "value": tops, "unit": "TOPS (int8)", "forward_TOPS_incl_act_quant": fwd_tops,
             "gemm_us": p["gemm_ms"] * 1e3, "act_quant_us": p["act_ms"] * 1e3,
             "act_quant_GB_s": act_gbs, "act_quant_frac_of_hbm": act_gbs / hbm,
+            "layernorm_act_quant": {"kernel": "ln_quant_kernel", "us": p["ln_ms"] * 1e3,
+                                    "GB_s": p["ln_bytes"] / (p["ln_ms"] * 1e-3) / 1e9,
+                                    "frac_of_hbm": p["ln_bytes"] / (p["ln_ms"] * 1e-3) / 1e9 / hbm},
             "roofline": {"bound": "tensor", "kernel": gemm_kernel_name(p["M"]), "achieved": tops, "peak": peak,
                          "peak_kind": kind, "unit": "TOPS", "frac": tops / peak,
                          "traffic": profiled_traffic(gemm_kernel_name(p["M"]), "3b_prefill")},

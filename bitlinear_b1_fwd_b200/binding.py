@@ -36,6 +36,7 @@ SIGNATURES = {
     "bitlinear_ternarize_pack": (_I, [_P, _I, _I64, _I64, _P, _F, _I, _P, _P, _P]),
     "bitlinear_pack": (_I, [_P, _I64, _I64, _I, _P, _P, _SZ, _P]),
     "bitlinear_quantize_acts": (_I, [_P, _I, _I64, _I64, _P, _P, _P]),
+    "bitlinear_layernorm_quantize_acts": (_I, [_P, _I, _P, _P, _F, _I64, _I64, _P, _P, _P, _P]),
     "bitlinear_forward": (_I, [_P, _I, _P, _I64, _I64, _P, _I, _P, _I64, _P, _I, _P, _SZ, _P]),
     "bitlinear_selftest_wait_timeout": (_I, [_P, _SZ, _P]),
     "bitlinear_device_status": (_I, [_P, _P]),
@@ -170,6 +171,15 @@ def bitlinear_quantize_acts(x, xq, scale, stream=None) -> None:
     M, K = x.shape
     _check(lib().bitlinear_quantize_acts(_ptr(x), dtype_code(x), M, K, _ptr(xq), _ptr(scale),
                                          _stream(stream)), "bitlinear_quantize_acts")
+
+
+def bitlinear_layernorm_quantize_acts(x, ln_w, ln_b, eps, xq, scale, y=None, stream=None) -> None:
+    """LayerNorm of each token (y: optional bf16 output), then per-token INT8."""
+    _contig(x, ln_w, ln_b, xq, scale, y)
+    M, K = x.shape
+    _check(lib().bitlinear_layernorm_quantize_acts(_ptr(x), dtype_code(x), _ptr(ln_w), _ptr(ln_b), float(eps), M, K,
+                                                   _ptr(y), _ptr(xq), _ptr(scale), _stream(stream)),
+           "bitlinear_layernorm_quantize_acts")
 
 
 def bitlinear_forward(packed, fmt, gamma, N, K, x, scale, y, ws, stream=None) -> None:

@@ -161,6 +161,95 @@ __global__ void __launch_bounds__(kActThreads)
   }
 }
 
+// Pre-norm + step 4: LayerNorm of each token, then per-token absmax INT8
+// ([P5] "The BitLinear Recipe" step 1: the input is quantized after
+// LayerNorm; [P3] §5.5: LayerNorm kept in high precision, bf16 activations).
+// One CTA of kLnThreads per token.  The mean and the variance are fp64 sums
+// in a fixed order: thread l adds the elements l, l + 256, ... in turn from
+// 0.0, and the 256 partial sums combine by the stride-halving tree p[l] +=
+// p[l + s], s = 128, ..., 1.  r = 1 / sqrt(var + eps) in fp64; y = ((x - mu) r)
+// g + b in fp64 with one rounding per operation, then fp32 and bf16 (RNE).
+// The bf16 y is quantized exactly as act_quant_row_kernel does (absmax over
+// the token, the division-free exact rounding).  Four passes over the token,
+// the later ones from L1/L2.
+constexpr int kLnThreads = 256;
+
+template <int XDT>
+__global__ void __launch_bounds__(kLnThreads)
+    ln_quant_kernel(const void* __restrict__ x, const float* __restrict__ g, const float* __restrict__ b, float eps,
+                    int64_t M, int64_t K, uint16_t* __restrict__ y, int8_t* __restrict__ xq,
+                    float* __restrict__ scale) {
+  pdl_enter(x, g, b, y, xq, scale);
+  __shared__ double p[kLnThreads];
+  __shared__ float red[kLnThreads / 32];
+  const int l = threadIdx.x, lane = l & 31, warp = l >> 5;
+  auto tree = [&](double v) -> double {
+    p[l] = v;
+    __syncthreads();
+#pragma unroll
+    for (int s = kLnThreads / 2; s >= 1; s >>= 1) {
+      if (l < s) p[l] = __dadd_rn(p[l], p[l + s]);
+      __syncthreads();
+    }
+    const double t = p[0];
+    __syncthreads();  // p is free for the next sum
+    return t;
+  };
+  for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+    const int64_t base = m * K;
+    double a = 0.0;
+    for (int64_t k = l; k < K; k += kLnThreads) a = __dadd_rn(a, static_cast<double>(load_elem<XDT>(x, base + k)));
+    const double mu = __ddiv_rn(tree(a), static_cast<double>(K));
+    a = 0.0;
+    for (int64_t k = l; k < K; k += kLnThreads) {
+      const double d = __dsub_rn(static_cast<double>(load_elem<XDT>(x, base + k)), mu);
+      a = __dadd_rn(a, __dmul_rn(d, d));
+    }
+    const double var = __ddiv_rn(tree(a), static_cast<double>(K));
+    const double r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(var, static_cast<double>(eps))));
+    auto yk = [&](int64_t k) -> __nv_bfloat16 {
+      const double d = __dsub_rn(static_cast<double>(load_elem<XDT>(x, base + k)), mu);
+      const double v = __dadd_rn(__dmul_rn(__dmul_rn(d, r), static_cast<double>(__ldcg(g + k))),
+                                 static_cast<double>(__ldcg(b + k)));
+      return __float2bfloat16_rn(__double2float_rn(v));
+    };
+    float amax = 0.0f;
+    for (int64_t k = l; k < K; k += kLnThreads) {
+      const __nv_bfloat16 v = yk(k);
+      amax = fmaxf(amax, fabsf(__bfloat162float(v)));
+      if (y != nullptr) y[base + k] = __bfloat16_as_ushort(v);
+    }
+    amax = warp_maxf(amax);
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    float am = red[0];
+#pragma unroll
+    for (int w = 1; w < kLnThreads / 32; ++w) am = fmaxf(am, red[w]);
+    __syncthreads();  // red is free for the next token
+    const float s = fmaxf(am, 1e-6f);
+    const float c127 = __fdiv_rn(127.0f, s);
+    for (int64_t k = l; k < K; k += kLnThreads)
+      xq[base + k] = static_cast<int8_t>(quant_act_fast(__bfloat162float(yk(k)), s, c127));
+    if (l == 0) scale[m] = s;
+  }
+}
+
+cudaError_t launch_ln_quant(const void* x, int xdt, const float* g, const float* b, float eps, int64_t M, int64_t K,
+                            uint16_t* y, int8_t* xq, float* scale, cudaStream_t st) {
+  int per_sm = 1;
+  const void* kp = xdt == BL_F32 ? reinterpret_cast<const void*>(ln_quant_kernel<BL_F32>)
+                                 : reinterpret_cast<const void*>(ln_quant_kernel<BL_BF16>);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kp, kLnThreads, 0) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  const int64_t cap = static_cast<int64_t>(device_sms()) * per_sm;
+  const unsigned grid = static_cast<unsigned>(M < cap ? M : cap);
+  cudaError_t e = (xdt == BL_F32)
+                      ? launch_pdl(ln_quant_kernel<BL_F32>, grid, kLnThreads, 0, st, x, g, b, eps, M, K, y, xq, scale)
+                      : launch_pdl(ln_quant_kernel<BL_BF16>, grid, kLnThreads, 0, st, x, g, b, eps, M, K, y, xq, scale);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 cudaError_t launch_act_quant(const void* x, int xdt, int64_t M, int64_t K, int8_t* xq, float* scale,
                              cudaStream_t st) {
   const int64_t warps_per_cta = kActThreads / 32;

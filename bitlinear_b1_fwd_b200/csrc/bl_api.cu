@@ -139,6 +139,19 @@ bl_status bitlinear_quantize_acts(const void* x, int xdt, int64_t M, int64_t K, 
   return cuda_status(bl::launch_act_quant(x, xdt, M, K, xq, scale, static_cast<cudaStream_t>(stream)));
 }
 
+bl_status bitlinear_layernorm_quantize_acts(const void* x, int xdt, const float* ln_w, const float* ln_b, float eps,
+                                            int64_t M, int64_t K, uint16_t* y, int8_t* xq, float* scale,
+                                            void* stream) {
+  if (!float_dt(xdt) || M < 0 || K < 1 || K > kMaxK) return BL_ERR_INVALID_VALUE;
+  if (!(eps > 0.0f) || !std::isfinite(eps)) return BL_ERR_INVALID_VALUE;
+  if (M == 0) return BL_OK;
+  if (x == nullptr || ln_w == nullptr || ln_b == nullptr || xq == nullptr || scale == nullptr)
+    return BL_ERR_INVALID_VALUE;
+  if (!aligned(x, 16) || !aligned(ln_w, 4) || !aligned(ln_b, 4) || !aligned(y, 2) || !aligned(scale, 4))
+    return BL_ERR_MISALIGNED;
+  return cuda_status(bl::launch_ln_quant(x, xdt, ln_w, ln_b, eps, M, K, y, xq, scale, static_cast<cudaStream_t>(stream)));
+}
+
 bl_status bitlinear_forward(const uint8_t* packed, int fmt, const float* gamma, int64_t N, int64_t K,
                             const void* x, int xdt, float* scale, int64_t M, void* y, int ydt, void* ws,
                             size_t ws_bytes, void* stream) {

@@ -46,6 +46,8 @@ cudaError_t launch_ternarize_pack(const void* W, int wdt, int64_t N, int64_t K, 
                                   cudaStream_t st);
 cudaError_t launch_pack(const int8_t* codes, int64_t N, int64_t K, int fmt, uint8_t* packed,
                         int64_t rowbytes, void* ws, cudaStream_t st);
+cudaError_t launch_ln_quant(const void* x, int xdt, const float* g, const float* b, float eps, int64_t M, int64_t K,
+                            uint16_t* y, int8_t* xq, float* scale, cudaStream_t st);
 cudaError_t launch_act_quant(const void* x, int xdt, int64_t M, int64_t K, int8_t* xq, float* scale,
                              cudaStream_t st);
 int gemv_max_tokens(int fmt, int64_t rowbytes);

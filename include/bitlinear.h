@@ -176,6 +176,24 @@ BL_API bl_status bitlinear_pack(const int8_t *codes, int64_t N, int64_t K, int f
 BL_API bl_status bitlinear_quantize_acts(const void *x, int xdt, int64_t M, int64_t K, int8_t *xq,
                                   float *scale, void *stream);
 
+/* Pre-norm + step 4: LayerNorm of each token, then per-token absmax INT8.
+ * [P5] "The BitLinear Recipe" step 1 (the input is quantized with absmax
+ * scaling after LayerNorm); [P3] §5.5 (LayerNorm kept in high precision,
+ * bf16 activations between layers).  Computes, for each token (row of x):
+ * mu and the biased variance as fp64 sums in a fixed order (element k goes to
+ * lane k mod 256, each lane adds its elements in turn, the 256 lane sums
+ * combine by the stride-halving tree s = 128, ..., 1), r = 1 / sqrt(var + eps),
+ * y = ((x - mu) r) ln_w + ln_b in fp64, rounded to fp32 and then to bf16, and
+ * the INT8 codes of the bf16 y exactly as bitlinear_quantize_acts does.
+ *   x      [M, K] fp32 or bf16 (16-byte aligned); ln_w, ln_b [K] fp32.
+ *   eps    > 0 (PyTorch's LayerNorm default is 1e-5).
+ *   y      [M, K] bf16 bits output of the LayerNorm, or NULL.
+ *   xq     [M, K] int8 output;  scale [M] fp32 output.
+ * Feeds bitlinear_forward with xdt = BL_I8. */
+BL_API bl_status bitlinear_layernorm_quantize_acts(const void *x, int xdt, const float *ln_w, const float *ln_b,
+                                                float eps, int64_t M, int64_t K, uint16_t *y, int8_t *xq,
+                                                float *scale, void *stream);
+
 /* BitLinear forward, y = dequant(x_q . W_q^T) (steps 4-6).
  * [P3] §4.2 (add / subtract / skip), §3.3 (INT32 accumulation), §5.3.
  *   packed  [N, row_bytes] from bitlinear_quantize_weights / bitlinear_pack.

@@ -380,3 +380,52 @@ def test_forward_i2_many_rows_per_cta(orc):
     x = synth.to_bf16_bits(synth.normal_f32(94, (1, K)))
     g, _, packed = quantize_weights(W, I2, codes=False)
     check_forward(orc, packed, I2, g, N, K, x, ydts=(B.BL_I32, B.BL_BF16))
+
+
+# --- pre-norm: LayerNorm of each token, then per-token INT8 ---------------------------
+
+def _ln_cases():
+    yield "tiny_f32_outliers", synth.tiny_inputs()[1]
+    yield "3b_decode_bf16", synth.decode_3b_inputs(0)[1]
+    yield "3b_prefill_bf16_outlier_channels", synth.prefill_3b_inputs()[1]
+    yield "ragged_3x20001_f32", synth.normal_f32(71, (3, 20001))
+    yield "k1_f32", synth.normal_f32(72, (4, 1))
+    yield "70b_down_bf16", synth.to_bf16_bits(synth.normal_f32(73, (2, 28672)))
+    c = synth.normal_f32(74, (4, 300))
+    c[1] = 0.375  # a constant token: y = ln_b
+    c[2] = 0.0
+    yield "constant_and_zero_tokens", c
+
+
+@pytest.mark.parametrize("name,x", list(_ln_cases()), ids=lambda v: v if isinstance(v, str) else "")
+def test_layernorm_quantize_acts(orc, name, x):
+    """bf16 LayerNorm output, INT8 codes and scales bit-exact against the oracle."""
+    M, K = x.shape
+    g = synth.normal_f32(80 + K % 11, (K,), 1.0)
+    b = synth.normal_f32(81 + K % 13, (K,), 0.1)
+    y_ref, xq_ref, s_ref = orc.layernorm_quant(x, g, b, 1e-5)
+    y = torch.empty((M, K), dtype=torch.int16, device="cuda")
+    xq = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    s = torch.empty((M,), dtype=torch.float32, device="cuda")
+    B.bitlinear_layernorm_quantize_acts(dev(x), dev(g), dev(b), 1e-5, xq, s, y)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(y).view(np.uint16), y_ref)
+    assert np.array_equal(host(xq), xq_ref)
+    assert np.array_equal(host(s).view(np.uint32), s_ref.view(np.uint32))
+
+
+def test_layernorm_quantize_acts_feeds_forward(orc):
+    """The codes and scales go straight into the forward as int8 tokens."""
+    W, x = synth.decode_3b_inputs(0)
+    c = synth.DECODE_3B[0]
+    K = c["K"]
+    g = synth.normal_f32(90, (K,), 1.0)
+    b = synth.normal_f32(91, (K,), 0.1)
+    _, xq_ref, s_ref = orc.layernorm_quant(x, g, b, 1e-5)
+    xq = torch.empty(x.shape, dtype=torch.int8, device="cuda")
+    s = torch.empty((x.shape[0],), dtype=torch.float32, device="cuda")
+    B.bitlinear_layernorm_quantize_acts(dev(x), dev(g), dev(b), 1e-5, xq, s)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(xq), xq_ref)
+    gam, _, packed = quantize_weights(W, I2, codes=False)
+    check_forward(orc, packed, I2, gam, c["N"], K, xq_ref, scale=s_ref)
