@@ -723,6 +723,7 @@ PROFILE_CASES = {
     "decode_70b_up_t5": dict(N=28672, K=8192, fmt=1, M=1, sigma=0.01, op="forward"),
     "prefill_3b": dict(N=8640, K=3200, fmt=0, M=4096, sigma=0.02, op="forward"),
     "batch16_70b_up": dict(N=28672, K=8192, fmt=0, M=16, sigma=0.01, op="forward"),
+    "lnquant_3b_prefill": dict(N=8640, K=3200, fmt=0, M=4096, sigma=0.02, op="lnquant"),
     "batch16_70b_down": dict(N=8192, K=28672, fmt=0, M=16, sigma=0.01, op="forward"),
 }
 
@@ -747,6 +748,13 @@ def run_profile_case(name):
     for _ in range(3 if c["op"] == "quantize" else 1):
         B.bitlinear_quantize_weights(W, 1e-5, fmt, packed, None, gamma, ws)
     status = [B.bitlinear_device_status(ws)]
+    if c["op"] == "lnquant":
+        ln_w = torch.randn(K, generator=g, device=dev) * 0.1 + 1.0
+        ln_b = torch.randn(K, generator=g, device=dev) * 0.1
+        xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+        sc = torch.empty(M, dtype=torch.float32, device=dev)
+        for _ in range(3):
+            B.bitlinear_layernorm_quantize_acts(x, ln_w, ln_b, 1e-5, xq, sc)
     if c["op"] == "forward":
         scale = torch.empty(M, dtype=torch.float32, device=dev)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
