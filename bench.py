@@ -548,7 +548,8 @@ def run_decode(args, dev, stream, rank_seed, l2):
 def run_sweep(args, dev, stream, l2):
     """Config sweeps (opt-in): the 70B layers (2-bit) over M = 1, 2, 4, ..., 8192
     and the 3B block's six BitLinears (Q, K, V, O, up, down, each with its
-    own per-token quantization) as one graph per block at M = 1, 16, 128, 1024.
+    own per-token quantization) as one graph per block at M = 1, 16, 128, 1024,
+    and the same block with Q, K and V as one grouped call on a shared input.
     Latent weights N(0, sigma) and bf16 tokens N(0, 1) are drawn on the device
     with a seeded generator (parity on the host-generated recipe is the tests'
     job); packed weights and tokens rotate over copies past 4x L2 where they
@@ -583,7 +584,7 @@ def run_sweep(args, dev, stream, l2):
         return {"M": M, "us": us, "GB_s": gbs, "frac_of_hbm": gbs / peak_gbs, "TOPS": tops,
                 "frac_of_int8": tops / peak_tops, "kernel": kern}
 
-    out = {"layer_70b": {}, "block_3b": []}
+    out = {"layer_70b": {}, "block_3b": [], "block_3b_fused_qkv": []}
     for li, c in enumerate(synth.LAYER_70B):
         N, K = c["N"], c["K"]
         p0, gamma, rb = prep(N, K, c["w_sigma"], 1005 + 100 * li)
@@ -641,7 +642,34 @@ def run_sweep(args, dev, stream, l2):
                                 "frac_of_hbm": nbytes / (us * 1e-6) / 1e9 / peak_gbs,
                                 "TOPS": ops / (us * 1e-6) / 1e12,
                                 "frac_of_int8": ops / (us * 1e-6) / 1e12 / peak_tops})
-        del xs, ys, scs, fwss
+        # the same block with Q, K and V as one grouped call on one shared input
+        qkv_rows = [c["N"] for c in synth.BLOCK_3B[:3]]
+        qkv = [torch.cat([copies[i][r] for i in range(3)], dim=0) for r in range(rot)]
+        qkv_g = torch.cat([blk[i][1] for i in range(3)])
+        y_qkv = torch.empty((M, sum(qkv_rows)), dtype=torch.bfloat16, device=dev)
+        ws_qkv = torch.zeros(B.bitlinear_forward_grouped_workspace_bytes(M, qkv_rows, synth.BLOCK_3B[0]["K"], 0,
+                                                                         B.BL_BF16), dtype=torch.uint8, device=dev)
+
+        def block_fused(j, M=M, xs=xs, ys=ys, scs=scs, fwss=fwss, y_qkv=y_qkv, ws_qkv=ws_qkv):
+            B.bitlinear_forward_grouped(qkv[j % rot], 0, qkv_g, qkv_rows, synth.BLOCK_3B[0]["K"], xs[0], scs[0],
+                                        y_qkv, ws_qkv, stream)
+            for i, c in enumerate(synth.BLOCK_3B[3:], start=3):
+                B.bitlinear_forward(copies[i][j % rot], 0, blk[i][1], c["N"], c["K"], xs[i], scs[i], ys[i],
+                                    fwss[i], stream)
+
+        with torch.cuda.stream(stream):
+            for j in range(3):
+                block_fused(j)
+        us_f = graph_ms(stream, steps, block_fused) / steps * 1e3
+        if B.bitlinear_device_status(ws_qkv, stream) != B.BL_OK:
+            raise RuntimeError("fused block device status")
+        nbytes_f = nbytes - 2 * M * synth.BLOCK_3B[0]["K"] * 2
+        out["block_3b_fused_qkv"].append({"M": M, "us_per_block": us_f, "GB_s": nbytes_f / (us_f * 1e-6) / 1e9,
+                                          "frac_of_hbm": nbytes_f / (us_f * 1e-6) / 1e9 / peak_gbs,
+                                          "TOPS": ops / (us_f * 1e-6) / 1e12,
+                                          "frac_of_int8": ops / (us_f * 1e-6) / 1e12 / peak_tops,
+                                          "vs_separate": us / us_f})
+        del xs, ys, scs, fwss, qkv, y_qkv, ws_qkv
     out["note"] = ("graphs of back-to-back forward calls timed at their two ends; bytes = packed weights + bf16 x + "
                    "bf16 y; TOPS = 2 M N K; fractions of the measured HBM copy rate and of the int8 peak")
     return out

@@ -38,6 +38,8 @@ SIGNATURES = {
     "bitlinear_quantize_acts": (_I, [_P, _I, _I64, _I64, _P, _P, _P]),
     "bitlinear_layernorm_quantize_acts": (_I, [_P, _I, _P, _P, _F, _I64, _I64, _P, _P, _P, _P]),
     "bitlinear_forward": (_I, [_P, _I, _P, _I64, _I64, _P, _I, _P, _I64, _P, _I, _P, _SZ, _P]),
+    "bitlinear_forward_grouped_workspace_bytes": (_SZ, [_I64, _I64, _P, _I64, _I, _I]),
+    "bitlinear_forward_grouped": (_I, [_P, _I, _P, _I64, _P, _I64, _P, _I, _P, _I64, _P, _I, _P, _SZ, _P]),
     "bitlinear_selftest_wait_timeout": (_I, [_P, _SZ, _P]),
     "bitlinear_device_status": (_I, [_P, _P]),
     "bitlinear_status_string": (C.c_char_p, [_I]),
@@ -120,6 +122,16 @@ def bitlinear_forward_workspace_bytes(M: int, N: int, K: int, fmt: int, xdt: int
     return int(lib().bitlinear_forward_workspace_bytes(M, N, K, fmt, xdt))
 
 
+def _rows_array(group_rows):
+    rows = [int(r) for r in group_rows]
+    return (C.c_int64 * len(rows))(*rows), len(rows)
+
+
+def bitlinear_forward_grouped_workspace_bytes(M: int, group_rows, K: int, fmt: int, xdt: int) -> int:
+    arr, n = _rows_array(group_rows)
+    return int(lib().bitlinear_forward_grouped_workspace_bytes(M, n, arr, K, fmt, xdt))
+
+
 # --- entry points -------------------------------------------------------------
 
 def bitlinear_workspace_init(ws: torch.Tensor, stream=None) -> None:
@@ -189,6 +201,16 @@ def bitlinear_forward(packed, fmt, gamma, N, K, x, scale, y, ws, stream=None) ->
                                    _ptr(scale), M, _ptr(y), dtype_code(y), _ptr(ws),
                                    ws.numel() * ws.element_size(), _stream(stream)),
            "bitlinear_forward")
+
+
+def bitlinear_forward_grouped(packed, fmt, gammas, group_rows, K, x, scale, y, ws, stream=None) -> None:
+    _contig(packed, gammas, x, scale, y, ws)
+    M = x.shape[0]
+    arr, n = _rows_array(group_rows)
+    _check(lib().bitlinear_forward_grouped(_ptr(packed), fmt, _ptr(gammas), n, arr, K, _ptr(x), dtype_code(x),
+                                           _ptr(scale), M, _ptr(y), dtype_code(y), _ptr(ws),
+                                           ws.numel() * ws.element_size(), _stream(stream)),
+           "bitlinear_forward_grouped")
 
 
 def bitlinear_device_status(ws, stream=None) -> int:

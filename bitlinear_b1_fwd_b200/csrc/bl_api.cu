@@ -169,7 +169,7 @@ bl_status bitlinear_forward(const uint8_t* packed, int fmt, const float* gamma, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (!uses_gemm(M, K)) {
     if (bl::gemv_max_tokens(fmt, bitlinear_packed_row_bytes(K, fmt)) < 1) return BL_ERR_UNSUPPORTED;
-    return cuda_status(bl::launch_gemv(packed, fmt, gamma, N, K, x, xdt, scale, M, y, ydt, st));
+    return cuda_status(bl::launch_gemv(packed, fmt, gamma, N, K, x, xdt, scale, M, y, ydt, bl::one_group(N), st));
   }
   uint8_t* scratch = static_cast<uint8_t*>(ws) + BL_WS_HEADER_BYTES;
   const int8_t* xq = static_cast<const int8_t*>(x);
@@ -188,7 +188,96 @@ bl_status bitlinear_forward(const uint8_t* packed, int fmt, const float* gamma, 
     scratch += round256(static_cast<size_t>(N * rb2));
   }
   int32_t* part = bl::gemm_split_k(M, N, K) > 1 ? reinterpret_cast<int32_t*>(scratch) : nullptr;
-  return cuda_status(bl::launch_gemm_i2(xq, w2, rb2, gamma, scale, y, ydt, M, N, K, part, ws, 0, 0, st));
+  return cuda_status(bl::launch_gemm_i2(xq, w2, rb2, gamma, scale, y, ydt, M, N, K, N, part, ws, 0, 0, st));
+}
+
+// Several weight matrices sharing one token batch (for example a block's Q, K
+// and V projections): their packed rows are concatenated, each group has its
+// own gamma, and y holds the groups' outputs side by side.
+static int64_t group_total(int64_t ngroups, const int64_t* group_rows) {
+  if (ngroups < 1 || ngroups > bl::kMaxRowGroups || group_rows == nullptr) return -1;
+  int64_t n = 0;
+  for (int64_t g = 0; g < ngroups; ++g) {
+    if (group_rows[g] < 1) return -1;
+    n += group_rows[g];
+  }
+  return n;
+}
+
+size_t bitlinear_forward_grouped_workspace_bytes(int64_t M, int64_t ngroups, const int64_t* group_rows, int64_t K,
+                                                 int fmt, int xdt) {
+  const int64_t N = group_total(ngroups, group_rows);
+  if (N < 1 || M < 0 || !nk_ok(N, K) || !fmt_ok(fmt)) return 0;
+  size_t bytes = BL_WS_HEADER_BYTES;
+  if (uses_gemm(M, K)) {
+    if (xdt != BL_I8) bytes += round256(static_cast<size_t>(M * K));
+    size_t most = 0;  // the groups run one after another and share the rest
+    for (int64_t g = 0; g < ngroups; ++g) {
+      const int64_t Ng = group_rows[g];
+      size_t e = 0;
+      if (fmt == BL_PACK_T5) e += round256(static_cast<size_t>(Ng * bitlinear_packed_row_bytes(K, BL_PACK_I2)));
+      const int ks = bl::gemm_split_k(M, Ng, K);
+      if (ks > 1) e += round256(static_cast<size_t>(ks) * M * Ng * sizeof(int32_t));
+      if (e > most) most = e;
+    }
+    bytes += most;
+  }
+  return bytes;
+}
+
+bl_status bitlinear_forward_grouped(const uint8_t* packed, int fmt, const float* gammas, int64_t ngroups,
+                                    const int64_t* group_rows, int64_t K, const void* x, int xdt, float* scale,
+                                    int64_t M, void* y, int ydt, void* ws, size_t ws_bytes, void* stream) {
+  if (!fmt_ok(fmt) || !(float_dt(xdt) || xdt == BL_I8) || !(float_dt(ydt) || ydt == BL_I32))
+    return BL_ERR_INVALID_VALUE;
+  const int64_t N = group_total(ngroups, group_rows);
+  if (N < 1 || M < 0 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
+  if (M == 0) return BL_OK;
+  if (packed == nullptr || gammas == nullptr || x == nullptr || scale == nullptr || y == nullptr || ws == nullptr)
+    return BL_ERR_INVALID_VALUE;
+  if (!aligned(packed, 16) || !aligned(x, 16) || !aligned(y, 16) || !aligned(scale, 4) || !aligned(gammas, 4) ||
+      !aligned(ws, 16))
+    return BL_ERR_MISALIGNED;
+  if (ws_bytes < bitlinear_forward_grouped_workspace_bytes(M, ngroups, group_rows, K, fmt, xdt))
+    return BL_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t rb = bitlinear_packed_row_bytes(K, fmt);
+  if (!uses_gemm(M, K)) {  // one GEMV launch over every group's rows
+    if (bl::gemv_max_tokens(fmt, rb) < 1) return BL_ERR_UNSUPPORTED;
+    bl::RowGroups rg{};
+    rg.n = static_cast<int>(ngroups);
+    int64_t end = 0;
+    for (int64_t g = 0; g < ngroups; ++g) rg.end[g] = (end += group_rows[g]);
+    return cuda_status(bl::launch_gemv(packed, fmt, gammas, N, K, x, xdt, scale, M, y, ydt, rg, st));
+  }
+  // one activation quantization, then each group's product into its columns of y
+  uint8_t* scratch = static_cast<uint8_t*>(ws) + BL_WS_HEADER_BYTES;
+  const int8_t* xq = static_cast<const int8_t*>(x);
+  if (xdt != BL_I8) {
+    if (bl::launch_act_quant(x, xdt, M, K, reinterpret_cast<int8_t*>(scratch), scale, st) != cudaSuccess)
+      return BL_ERR_CUDA;
+    xq = reinterpret_cast<const int8_t*>(scratch);
+    scratch += round256(static_cast<size_t>(M * K));
+  }
+  const int64_t rb2 = bitlinear_packed_row_bytes(K, BL_PACK_I2);
+  const size_t ysize = (ydt == BL_BF16) ? 2 : 4;
+  int64_t off = 0;
+  for (int64_t g = 0; g < ngroups; ++g) {
+    const int64_t Ng = group_rows[g];
+    uint8_t* s2 = scratch;
+    const uint8_t* w2 = packed + off * rb;
+    if (fmt == BL_PACK_T5) {
+      if (bl::launch_t5_to_i2(w2, Ng, K, rb, s2, rb2, st) != cudaSuccess) return BL_ERR_CUDA;
+      w2 = s2;
+      s2 += round256(static_cast<size_t>(Ng * rb2));
+    }
+    int32_t* part = bl::gemm_split_k(M, Ng, K) > 1 ? reinterpret_cast<int32_t*>(s2) : nullptr;
+    const bl_status e = cuda_status(bl::launch_gemm_i2(xq, w2, rb2, gammas + g, scale, static_cast<uint8_t*>(y) + off * ysize,
+                                                       ydt, M, Ng, K, N, part, ws, 0, 0, st));
+    if (e != BL_OK) return e;
+    off += Ng;
+  }
+  return BL_OK;
 }
 
 bl_status bitlinear_selftest_wait_timeout(void* ws, size_t ws_bytes, void* stream) {
@@ -198,7 +287,7 @@ bl_status bitlinear_selftest_wait_timeout(void* ws, size_t ws_bytes, void* strea
   uint8_t* op = static_cast<uint8_t*>(ws) + BL_WS_HEADER_BYTES;
   const float* g = reinterpret_cast<const float*>(op);
   return cuda_status(bl::launch_gemm_i2(reinterpret_cast<const int8_t*>(op), op, 32, g, g, op, BL_I32, 16, 128,
-                                        128, nullptr, ws, int64_t{1} << 20, 1, static_cast<cudaStream_t>(stream)));
+                                        128, 128, nullptr, ws, int64_t{1} << 20, 1, static_cast<cudaStream_t>(stream)));
 }
 
 bl_status bitlinear_device_status(void* ws, void* stream) {

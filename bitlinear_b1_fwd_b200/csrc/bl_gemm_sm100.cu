@@ -178,7 +178,7 @@ template <int BT>
 __global__ void __launch_bounds__(GemmCfg<BT>::kThreads, 1)
     gemm_i2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                    const __grid_constant__ CUtensorMap tm_y, int y_tma, const float* __restrict__ gamma,
-                   const float* __restrict__ scale, void* __restrict__ y, int ydt, int M, int N, int K, int ks,
+                   const float* __restrict__ scale, void* __restrict__ y, int ydt, int M, int N, int K, int ldy, int ks,
                    int32_t* __restrict__ part, WsHeader* __restrict__ hdr, long long limit, int skip_producer) {
   pdl_enter(gamma, scale, y, part, hdr);
   using Cfg = GemmCfg<BT>;
@@ -459,7 +459,7 @@ __global__ void __launch_bounds__(GemmCfg<BT>::kThreads, 1)
           for (int j = 0; j < static_cast<int>(Cfg::kChunk); ++j) {
             const int t = t0 + j;
             if (t < M && n < N) {
-              const int64_t o = static_cast<int64_t>(t) * N + n;
+              const int64_t o = static_cast<int64_t>(t) * ldy + n;
               const int v = static_cast<int>(acc[j]);
               if (ydt == BL_I32) {
                 static_cast<int32_t*>(y)[o] = v;
@@ -494,7 +494,7 @@ __global__ void __launch_bounds__(GemmCfg<BT>::kThreads, 1)
 // the dequantization y = acc * (gamma s_t) / 127 as in the GEMM epilogues.
 // Four consecutive outputs per thread when N % 4 == 0.
 __global__ void __launch_bounds__(256)
-    splitk_reduce_kernel(const int32_t* __restrict__ part, int ks, int M, int N, const float* __restrict__ gamma,
+    splitk_reduce_kernel(const int32_t* __restrict__ part, int ks, int M, int N, int ldy, const float* __restrict__ gamma,
                          const float* __restrict__ scale, void* __restrict__ y, int ydt) {
   pdl_enter(part, gamma, scale, y);
   __shared__ float sh_g;  // gamma once per CTA
@@ -527,16 +527,18 @@ __global__ void __launch_bounds__(256)
       }
       const int64_t o = 4 * i;
       const int t = static_cast<int>(o / N);
-      emit(o, t, s.x);
-      emit(o + 1, t, s.y);
-      emit(o + 2, t, s.z);
-      emit(o + 3, t, s.w);
+      const int64_t yo = static_cast<int64_t>(t) * ldy + (o - static_cast<int64_t>(t) * N);  // row stride ldy
+      emit(yo, t, s.x);
+      emit(yo + 1, t, s.y);
+      emit(yo + 2, t, s.z);
+      emit(yo + 3, t, s.w);
     }
   } else {
     for (int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; o < plane; o += stride) {
       int s = __ldcg(part + o);
       for (int kz = 1; kz < ks; ++kz) s += __ldcg(part + kz * plane + o);
-      emit(o, static_cast<int>(o / N), s);
+      const int t = static_cast<int>(o / N);
+      emit(static_cast<int64_t>(t) * ldy + (o - static_cast<int64_t>(t) * N), t, s);
     }
   }
 }
@@ -589,7 +591,7 @@ template <int BT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_i2_2sm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                        const __grid_constant__ CUtensorMap tm_y, int y_tma, const float* __restrict__ gamma,
-                       const float* __restrict__ scale, void* __restrict__ y, int ydt, int M, int N, int K,
+                       const float* __restrict__ scale, void* __restrict__ y, int ydt, int M, int N, int K, int ldy,
                        WsHeader* __restrict__ hdr, long long limit) {
   pdl_enter(gamma, scale, y, hdr);
   using Cfg = Gemm2Cfg<BT>;
@@ -816,7 +818,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           for (int j = 0; j < 32; ++j) {
             const int t = t0 + j;
             if (t < M && n < N) {
-              const int64_t o = static_cast<int64_t>(t) * N + n;
+              const int64_t o = static_cast<int64_t>(t) * ldy + n;
               const int v = static_cast<int>(acc[j]);
               if (ydt == BL_I32) {
                 static_cast<int32_t*>(y)[o] = v;
@@ -926,16 +928,16 @@ bool encode_2d_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t out
 // Tensor map of y for the TMA-store epilogue: [M x N] of the output type, box
 // 128 rows x `tokens` tokens.  False when a row of y is not a multiple of 16
 // bytes.
-bool encode_y(CUtensorMap* m, void* y, int ydt, int64_t M, int64_t N, uint32_t tokens) {
+bool encode_y(CUtensorMap* m, void* y, int ydt, int64_t M, int64_t N, int64_t ldy, uint32_t tokens) {
   const uint64_t esz = (ydt == BL_BF16) ? 2 : 4;
-  if ((static_cast<uint64_t>(N) * esz) % 16 != 0) return false;
+  if ((static_cast<uint64_t>(ldy) * esz) % 16 != 0 || (reinterpret_cast<uintptr_t>(y) % 16) != 0) return false;
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const CUtensorMapDataType dt = ydt == BL_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                  : ydt == BL_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                                                  : CU_TENSOR_MAP_DATA_TYPE_INT32;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * esz};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldy) * esz};
   const cuuint32_t box[2] = {128, tokens};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, dt, 2, y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -944,7 +946,7 @@ bool encode_y(CUtensorMap* m, void* y, int ydt, int64_t M, int64_t N, uint32_t t
 
 template <int BT>
 cudaError_t launch_gemm_bt(const int8_t* xq, const uint8_t* w, int64_t rb, const float* gamma, const float* scale,
-                           void* y, int ydt, int64_t M, int64_t N, int64_t K, int ks, int32_t* part, void* ws,
+                           void* y, int ydt, int64_t M, int64_t N, int64_t K, int64_t ldy, int ks, int32_t* part, void* ws,
                            long long limit, int skip_producer, cudaStream_t st) {
   CUtensorMap tx, tw;
   if (!encode_2d_u8(&tx, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(K), 128, BT,
@@ -954,7 +956,7 @@ cudaError_t launch_gemm_bt(const int8_t* xq, const uint8_t* w, int64_t rb, const
                     kGroup * kBK / 4, kBN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   CUtensorMap ty;
-  const int y_tma = (ks == 1 && encode_y(&ty, y, ydt, M, N, GemmCfg<BT>::kChunk)) ? 1 : 0;
+  const int y_tma = (ks == 1 && encode_y(&ty, y, ydt, M, N, ldy, GemmCfg<BT>::kChunk)) ? 1 : 0;
   if (!y_tma) memset(&ty, 0, sizeof(ty));
   auto kern = gemm_i2_kernel<BT>;
   const size_t smem = GemmCfg<BT>::kSmem;
@@ -964,7 +966,7 @@ cudaError_t launch_gemm_bt(const int8_t* xq, const uint8_t* w, int64_t rb, const
   const int sms = device_sms();
   const unsigned grid = static_cast<unsigned>(units < sms ? units : sms);
   e = launch_pdl(kern, grid, GemmCfg<BT>::kThreads, smem, st, tx, tw, ty, y_tma, gamma, scale, y, ydt, static_cast<int>(M),
-                 static_cast<int>(N), static_cast<int>(K), ks, part, static_cast<WsHeader*>(ws), limit,
+                 static_cast<int>(N), static_cast<int>(K), static_cast<int>(ldy), ks, part, static_cast<WsHeader*>(ws), limit,
                  skip_producer);
   if (e != cudaSuccess) return e;
   if (ks > 1) {
@@ -972,7 +974,7 @@ cudaError_t launch_gemm_bt(const int8_t* xq, const uint8_t* w, int64_t rb, const
     int64_t rgrid = (work + 255) / 256;
     if (rgrid > 8 * sms) rgrid = 8 * sms;
     e = launch_pdl(splitk_reduce_kernel, static_cast<unsigned>(rgrid), 256, 0, st, static_cast<const int32_t*>(part),
-                   ks, static_cast<int>(M), static_cast<int>(N), gamma, scale, y, ydt);
+                   ks, static_cast<int>(M), static_cast<int>(N), static_cast<int>(ldy), gamma, scale, y, ydt);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
@@ -980,7 +982,7 @@ cudaError_t launch_gemm_bt(const int8_t* xq, const uint8_t* w, int64_t rb, const
 
 template <int BT>
 cudaError_t launch_gemm_2sm(const int8_t* xq, const uint8_t* w, int64_t rb, const float* gamma, const float* scale,
-                            void* y, int ydt, int64_t M, int64_t N, int64_t K, void* ws, long long limit,
+                            void* y, int ydt, int64_t M, int64_t N, int64_t K, int64_t ldy, void* ws, long long limit,
                             cudaStream_t st) {
   CUtensorMap tx, tw;
   if (!encode_2d_u8(&tx, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(K), 128,
@@ -990,7 +992,7 @@ cudaError_t launch_gemm_2sm(const int8_t* xq, const uint8_t* w, int64_t rb, cons
                     kBK / 4, kBN, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   CUtensorMap ty;
-  const int y_tma = encode_y(&ty, y, ydt, M, N, 32) ? 1 : 0;
+  const int y_tma = encode_y(&ty, y, ydt, M, N, ldy, 32) ? 1 : 0;
   if (!y_tma) memset(&ty, 0, sizeof(ty));
   auto kern = gemm_i2_2sm_kernel<BT>;
   const size_t smem = Gemm2Cfg<BT>::kSmem;
@@ -1001,7 +1003,8 @@ cudaError_t launch_gemm_2sm(const int8_t* xq, const uint8_t* w, int64_t rb, cons
   const int64_t pairs = tiles < pairs_max ? tiles : pairs_max;
   { const cudaError_t le_ = launch_pdl(kern, static_cast<unsigned>(2 * pairs), kGemmThreads, smem, st, tx, tw, ty, y_tma, gamma, scale, y, ydt,
                                                                      static_cast<int>(M), static_cast<int>(N),
-                                                                     static_cast<int>(K), static_cast<WsHeader*>(ws),
+                                                                     static_cast<int>(K), static_cast<int>(ldy),
+                                                                     static_cast<WsHeader*>(ws),
                                                                      limit); if (le_ != cudaSuccess) return le_; }
   return cudaGetLastError();
 }
@@ -1039,17 +1042,17 @@ int gemm_split_k(int64_t M, int64_t N, int64_t K) {
 }
 
 cudaError_t launch_gemm_i2(const int8_t* xq, const uint8_t* w, int64_t rb, const float* gamma, const float* scale,
-                           void* y, int ydt, int64_t M, int64_t N, int64_t K, int32_t* part, void* ws,
+                           void* y, int ydt, int64_t M, int64_t N, int64_t K, int64_t ldy, int32_t* part, void* ws,
                            long long limit_cycles, int skip_producer, cudaStream_t st) {
   const long long limit = limit_cycles > 0 ? limit_cycles : kTimeoutCycles;
   if (M > 128 && !skip_producer)
-    return launch_gemm_2sm<256>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ws, limit, st);
+    return launch_gemm_2sm<256>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ldy, ws, limit, st);
   const int ks = (part != nullptr && !skip_producer) ? gemm_split_k(M, N, K) : 1;
   switch (gemm_token_tile(M)) {
-    case 16: return launch_gemm_bt<16>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ks, part, ws, limit, skip_producer, st);
-    case 32: return launch_gemm_bt<32>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ks, part, ws, limit, skip_producer, st);
-    case 64: return launch_gemm_bt<64>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ks, part, ws, limit, skip_producer, st);
-    default: return launch_gemm_bt<128>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ks, part, ws, limit, skip_producer, st);
+    case 16: return launch_gemm_bt<16>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ldy, ks, part, ws, limit, skip_producer, st);
+    case 32: return launch_gemm_bt<32>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ldy, ks, part, ws, limit, skip_producer, st);
+    case 64: return launch_gemm_bt<64>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ldy, ks, part, ws, limit, skip_producer, st);
+    default: return launch_gemm_bt<128>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ldy, ks, part, ws, limit, skip_producer, st);
   }
 }
 

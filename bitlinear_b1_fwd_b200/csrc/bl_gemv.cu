@@ -111,7 +111,7 @@ template <int FMT, int MT, int XDT>
 __global__ void __launch_bounds__(kGemvThreads, 1)
     gemv_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
                 int64_t N, int64_t K, const void* __restrict__ x, float* __restrict__ scale,
-                void* __restrict__ y, int ydt, int write_scale) {
+                void* __restrict__ y, int ydt, int write_scale, const RowGroups rg) {
   pdl_enter(packed, gamma, x, scale, y);
   extern __shared__ __align__(16) uint8_t smem[];
   const int64_t xb = gemv_x_bytes(FMT, rowbytes);
@@ -166,6 +166,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   __shared__ float sh_gs[1 + MT];
   if (threadIdx.x <= MT && (threadIdx.x == 0 || XDT == BL_I8))
     sh_gs[threadIdx.x] = __ldcg(threadIdx.x == 0 ? gamma : scale + (threadIdx.x - 1));
+  __shared__ float sh_gam[kMaxRowGroups];  // gamma of each row group
+  if (threadIdx.x < rg.n) sh_gam[threadIdx.x] = __ldcg(gamma + threadIdx.x);
   for (int i = threadIdx.x; i < MT * kGemvTileRows; i += blockDim.x) racc[i] = 0;
   if constexpr (FMT == BL_PACK_T5) {
     uint4* z = reinterpret_cast<uint4*>(xs);
@@ -408,12 +410,13 @@ quant_act_fast_n<8>(e, s_tok[m], c127, q);
         const int a = racc[m * kGemvTileRows + r] - corr[m];
         racc[m * kGemvTileRows + r] = 0;
         const int64_t o = m * N + row0 + t0 + r;
+        const float cf = rg.n == 1 ? cfac[m] : dequant_factor(sh_gam[row_group(rg, row0 + t0 + r)], s_tok[m]);
         if (ydt == BL_I32)
           static_cast<int32_t*>(y)[o] = a;
         else if (ydt == BL_F32)
-          static_cast<float*>(y)[o] = __fmul_rn(__int2float_rn(a), cfac[m]);
+          static_cast<float*>(y)[o] = __fmul_rn(__int2float_rn(a), cf);
         else
-          static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(a), cfac[m]));
+          static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(a), cf));
       }
     }
     __syncthreads();  // the row sums are zero again for the next tile
@@ -449,7 +452,7 @@ template <int MT, int XDT>
 __global__ void __launch_bounds__(kGemvThreads, 1)
     gemv_i2_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
                    int64_t N, int64_t K, const void* __restrict__ x, float* __restrict__ scale,
-                   void* __restrict__ y, int ydt, int write_scale) {
+                   void* __restrict__ y, int ydt, int write_scale, const RowGroups rg) {
   const int64_t G = gridDim.x, b = blockIdx.x;
   const int64_t per = N / G, extra = N % G;
   const int64_t row0 = b * per + (b < extra ? b : extra);
@@ -517,6 +520,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   __shared__ float sh_gs[1 + MT];
   if (threadIdx.x <= MT && (threadIdx.x == 0 || XDT == BL_I8))
     sh_gs[threadIdx.x] = __ldcg(threadIdx.x == 0 ? gamma : scale + (threadIdx.x - 1));
+  __shared__ float sh_gam[kMaxRowGroups];  // gamma of each row group
+  if (threadIdx.x < rg.n) sh_gam[threadIdx.x] = __ldcg(gamma + threadIdx.x);
   if (one_pass) {
 #pragma unroll
     for (int u = 0; u < 3; ++u) {
@@ -745,12 +750,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
         const int a = racc[m * kGemvTileRows + r] - corr[m];
         racc[m * kGemvTileRows + r] = 0;
         const int64_t o = m * N + row0 + t0 + r;
+        const float cf = rg.n == 1 ? cfac[m] : dequant_factor(sh_gam[row_group(rg, row0 + t0 + r)], s_tok[m]);
         if (ydt == BL_I32)
           static_cast<int32_t*>(y)[o] = a;
         else if (ydt == BL_F32)
-          static_cast<float*>(y)[o] = __fmul_rn(__int2float_rn(a), cfac[m]);
+          static_cast<float*>(y)[o] = __fmul_rn(__int2float_rn(a), cf);
         else
-          static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(a), cfac[m]));
+          static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(a), cf));
       }
     }
     __syncthreads();  // the row sums are zero again for the next tile
@@ -783,7 +789,7 @@ template <int MT, int XDT>
 __global__ void __launch_bounds__(kMtThreads, 1)
     gemv_i2_mt_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
                       int64_t N, int64_t K, const void* __restrict__ x, float* __restrict__ scale,
-                      void* __restrict__ y, int ydt, int write_scale) {
+                      void* __restrict__ y, int ydt, int write_scale, const RowGroups rg) {
   const int64_t G = gridDim.x, b = blockIdx.x;
   const int64_t per = N / G, extra = N % G;
   const int64_t row0 = b * per + (b < extra ? b : extra);
@@ -805,6 +811,8 @@ __global__ void __launch_bounds__(kMtThreads, 1)
   pdl_wait(packed, gamma, x, scale, y);
   if (threadIdx.x <= MT && (threadIdx.x == 0 || XDT == BL_I8))
     sh_gs[threadIdx.x] = __ldcg(threadIdx.x == 0 ? gamma : scale + (threadIdx.x - 1));
+  __shared__ float sh_gam[kMaxRowGroups];  // gamma of each row group
+  if (threadIdx.x < rg.n) sh_gam[threadIdx.x] = __ldcg(gamma + threadIdx.x);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nthr = blockDim.x;
 
@@ -973,12 +981,13 @@ __global__ void __launch_bounds__(kMtThreads, 1)
     for (int m = 0; m < MT; ++m) {
       const int a = racc[m * kGemvTileRows + r] - corr[m];
       const int64_t o = m * N + row0 + r;
+      const float cf = rg.n == 1 ? cfac[m] : dequant_factor(sh_gam[row_group(rg, row0 + r)], s_tok[m]);
       if (ydt == BL_I32)
         static_cast<int32_t*>(y)[o] = a;
       else if (ydt == BL_F32)
-        static_cast<float*>(y)[o] = __fmul_rn(__int2float_rn(a), cfac[m]);
+        static_cast<float*>(y)[o] = __fmul_rn(__int2float_rn(a), cf);
       else
-        static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(a), cfac[m]));
+        static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(a), cf));
     }
   }
 }
@@ -1014,7 +1023,7 @@ template <int XDT>
 __global__ void __launch_bounds__(kGemvThreads, 1)
     gemv_t5_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
                    int64_t N, int64_t K, const void* __restrict__ x, float* __restrict__ scale,
-                   void* __restrict__ y, int ydt, int write_scale) {
+                   void* __restrict__ y, int ydt, int write_scale, const RowGroups rg) {
   const int64_t G = gridDim.x, b = blockIdx.x;
   const int64_t per = N / G, extra = N % G;
   const int64_t row0 = b * per + (b < extra ? b : extra);
@@ -1051,6 +1060,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   pdl_wait(packed, gamma, x, scale, y);
   if (threadIdx.x == 0) sh_gs[0] = __ldcg(gamma);
   if (XDT == BL_I8 && threadIdx.x == 1) sh_gs[1] = __ldcg(scale);
+  __shared__ float sh_gam[kMaxRowGroups];  // gamma of each row group
+  if (threadIdx.x < rg.n) sh_gam[threadIdx.x] = __ldcg(gamma + threadIdx.x);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nthr = blockDim.x;
@@ -1210,12 +1221,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   for (int r = threadIdx.x; r < nrows; r += nthr) {
     const int a = racc[r] - corr;
     const int64_t o = row0 + r;
+    const float cf = rg.n == 1 ? cfac : dequant_factor(sh_gam[row_group(rg, o)], s_tok);
     if (ydt == BL_I32)
       static_cast<int32_t*>(y)[o] = a;
     else if (ydt == BL_F32)
-      static_cast<float*>(y)[o] = __fmul_rn(__int2float_rn(a), cfac);
+      static_cast<float*>(y)[o] = __fmul_rn(__int2float_rn(a), cf);
     else
-      static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(a), cfac));
+      static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(a), cf));
   }
 }
 
@@ -1231,7 +1243,7 @@ int gemv_max_tokens(int fmt, int64_t rowbytes) {
 template <int FMT, int MT, int XDT>
 static cudaError_t launch_gemv_t(const uint8_t* packed, int64_t rowbytes, const float* gamma,
                                  int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
-                                 int write_scale, cudaStream_t st) {
+                                 int write_scale, const RowGroups& rg, cudaStream_t st) {
   auto kern = gemv_kernel<FMT, MT, XDT>;
   const size_t smem = static_cast<size_t>(gemv_smem_bytes(FMT, rowbytes, MT));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1247,14 +1259,14 @@ static cudaError_t launch_gemv_t(const uint8_t* packed, int64_t rowbytes, const 
   if (grid > need) grid = need;
   if (grid < 1) grid = 1;
   { const cudaError_t le_ = launch_pdl(kern, static_cast<unsigned>(grid), kGemvThreads, smem, st, packed, rowbytes, gamma, N, K, x, scale,
-                                                                 y, ydt, write_scale); if (le_ != cudaSuccess) return le_; }
+                                                                 y, ydt, write_scale, rg); if (le_ != cudaSuccess) return le_; }
   return cudaGetLastError();
 }
 
 template <int MT, int XDT>
 static cudaError_t launch_gemv_i2_t(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N,
                                     int64_t K, const void* x, float* scale, void* y, int ydt, int write_scale,
-                                    cudaStream_t st) {
+                                    const RowGroups& rg, cudaStream_t st) {
   auto kern = gemv_i2_kernel<MT, XDT>;
   const size_t smem = static_cast<size_t>(gemv_i2_smem_bytes(MT));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -1262,19 +1274,19 @@ static cudaError_t launch_gemv_i2_t(const uint8_t* packed, int64_t rowbytes, con
   const int64_t sms = device_sms();
   const int64_t grid = N < sms ? N : sms;  // every CTA owns at least one row
   { const cudaError_t le_ = launch_pdl(kern, static_cast<unsigned>(grid), kGemvThreads, smem, st, packed, rowbytes, gamma, N, K, x, scale, y, ydt,
-                                                                 write_scale); if (le_ != cudaSuccess) return le_; }
+                                                                 write_scale, rg); if (le_ != cudaSuccess) return le_; }
   return cudaGetLastError();
 }
 
 template <int XDT>
 static cudaError_t launch_gemv_i2_mt(int mt, const uint8_t* packed, int64_t rowbytes, const float* gamma,
                                      int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
-                                     int write_scale, cudaStream_t st) {
+                                     int write_scale, const RowGroups& rg, cudaStream_t st) {
   switch (mt) {
-    case 1: return launch_gemv_i2_t<1, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
-    case 2: return launch_gemv_i2_t<2, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
-    case 3: return launch_gemv_i2_t<3, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
-    default: return launch_gemv_i2_t<4, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
+    case 1: return launch_gemv_i2_t<1, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
+    case 2: return launch_gemv_i2_t<2, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
+    case 3: return launch_gemv_i2_t<3, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
+    default: return launch_gemv_i2_t<4, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
   }
 }
 
@@ -1290,7 +1302,7 @@ static bool gemv_mt_fits(int64_t rowbytes, int64_t N, int mt) {
 template <int MT, int XDT>
 static cudaError_t launch_gemv_mt_cs(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N,
                                      int64_t K, const void* x, float* scale, void* y, int ydt, int write_scale,
-                                     cudaStream_t st) {
+                                     const RowGroups& rg, cudaStream_t st) {
   auto kern = gemv_i2_mt_kernel<MT, XDT>;
   const size_t smem = static_cast<size_t>(gemv_mt_smem_bytes(rowbytes, MT));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -1298,7 +1310,7 @@ static cudaError_t launch_gemv_mt_cs(const uint8_t* packed, int64_t rowbytes, co
   const int64_t sms = device_sms();
   const int64_t grid = N < sms ? N : sms;  // every CTA owns at least one row
   e = launch_pdl(kern, static_cast<unsigned>(grid), kMtThreads, smem, st, packed, rowbytes, gamma, N, K, x, scale, y,
-                 ydt, write_scale);
+                 ydt, write_scale, rg);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -1306,11 +1318,11 @@ static cudaError_t launch_gemv_mt_cs(const uint8_t* packed, int64_t rowbytes, co
 template <int XDT>
 static cudaError_t launch_gemv_mt_cs_n(int mt, const uint8_t* packed, int64_t rowbytes, const float* gamma,
                                        int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
-                                       int write_scale, cudaStream_t st) {
+                                       int write_scale, const RowGroups& rg, cudaStream_t st) {
   switch (mt) {
-    case 2: return launch_gemv_mt_cs<2, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
-    case 3: return launch_gemv_mt_cs<3, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
-    default: return launch_gemv_mt_cs<4, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
+    case 2: return launch_gemv_mt_cs<2, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
+    case 3: return launch_gemv_mt_cs<3, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
+    default: return launch_gemv_mt_cs<4, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
   }
 }
 
@@ -1326,7 +1338,7 @@ static bool gemv_t5_fits(int64_t rowbytes, int64_t N) {
 template <int XDT>
 static cudaError_t launch_gemv_t5_t(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N,
                                     int64_t K, const void* x, float* scale, void* y, int ydt, int write_scale,
-                                    cudaStream_t st) {
+                                    const RowGroups& rg, cudaStream_t st) {
   auto kern = gemv_t5_kernel<XDT>;
   const size_t smem = static_cast<size_t>(gemv_t5_smem_bytes(rowbytes));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -1334,7 +1346,7 @@ static cudaError_t launch_gemv_t5_t(const uint8_t* packed, int64_t rowbytes, con
   const int64_t sms = device_sms();
   const int64_t grid = N < sms ? N : sms;  // every CTA owns at least one row
   e = launch_pdl(kern, static_cast<unsigned>(grid), kGemvThreads, smem, st, packed, rowbytes, gamma, N, K, x, scale,
-                 y, ydt, write_scale);
+                 y, ydt, write_scale, rg);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -1342,19 +1354,19 @@ static cudaError_t launch_gemv_t5_t(const uint8_t* packed, int64_t rowbytes, con
 template <int FMT, int XDT>
 static cudaError_t launch_gemv_mt(int mt, const uint8_t* packed, int64_t rowbytes, const float* gamma,
                                   int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
-                                  int write_scale, cudaStream_t st) {
+                                  int write_scale, const RowGroups& rg, cudaStream_t st) {
   switch (mt) {
-    case 1: return launch_gemv_t<FMT, 1, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
-    case 2: return launch_gemv_t<FMT, 2, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
-    case 3: return launch_gemv_t<FMT, 3, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
-    default: return launch_gemv_t<FMT, 4, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, st);
+    case 1: return launch_gemv_t<FMT, 1, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
+    case 2: return launch_gemv_t<FMT, 2, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
+    case 3: return launch_gemv_t<FMT, 3, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
+    default: return launch_gemv_t<FMT, 4, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
   }
 }
 
 // Runs the GEMV over all M tokens in groups that fit in shared memory.
 cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int64_t N, int64_t K,
                         const void* x, int xdt, float* scale, int64_t M, void* y, int ydt,
-                        cudaStream_t st) {
+                        const RowGroups& rg, cudaStream_t st) {
   const int64_t rowbytes = (fmt == BL_PACK_I2) ? ((K + 3) / 4 + 15) / 16 * 16 : ((K + 4) / 5 + 15) / 16 * 16;
   const int mt_max = gemv_max_tokens(fmt, rowbytes);
   if (mt_max < 1) return cudaErrorInvalidValue;
@@ -1370,25 +1382,25 @@ cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int6
     void* ym = static_cast<uint8_t*>(y) + m0 * N * ysz;
     cudaError_t e;
     if (fmt == BL_PACK_I2 && mt >= 2 && mt <= 4 && gemv_mt_fits(rowbytes, N, mt)) {
-      if (xdt == BL_F32) e = launch_gemv_mt_cs_n<BL_F32>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
-      else if (xdt == BL_BF16) e = launch_gemv_mt_cs_n<BL_BF16>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
-      else e = launch_gemv_mt_cs_n<BL_I8>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, st);
+      if (xdt == BL_F32) e = launch_gemv_mt_cs_n<BL_F32>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, rg, st);
+      else if (xdt == BL_BF16) e = launch_gemv_mt_cs_n<BL_BF16>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, rg, st);
+      else e = launch_gemv_mt_cs_n<BL_I8>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, rg, st);
     } else if (fmt == BL_PACK_T5 && mt == 1 && M == 1 && gemv_t5_fits(rowbytes, N)) {
-      if (xdt == BL_F32) e = launch_gemv_t5_t<BL_F32>(packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
-      else if (xdt == BL_BF16) e = launch_gemv_t5_t<BL_BF16>(packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
-      else e = launch_gemv_t5_t<BL_I8>(packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, st);
+      if (xdt == BL_F32) e = launch_gemv_t5_t<BL_F32>(packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, rg, st);
+      else if (xdt == BL_BF16) e = launch_gemv_t5_t<BL_BF16>(packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, rg, st);
+      else e = launch_gemv_t5_t<BL_I8>(packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, rg, st);
     } else if (lean) {
-      if (xdt == BL_F32) e = launch_gemv_i2_mt<BL_F32>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
-      else if (xdt == BL_BF16) e = launch_gemv_i2_mt<BL_BF16>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
-      else e = launch_gemv_i2_mt<BL_I8>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, st);
+      if (xdt == BL_F32) e = launch_gemv_i2_mt<BL_F32>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, rg, st);
+      else if (xdt == BL_BF16) e = launch_gemv_i2_mt<BL_BF16>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, rg, st);
+      else e = launch_gemv_i2_mt<BL_I8>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, rg, st);
     } else if (fmt == BL_PACK_I2) {
-      if (xdt == BL_F32) e = launch_gemv_mt<BL_PACK_I2, BL_F32>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
-      else if (xdt == BL_BF16) e = launch_gemv_mt<BL_PACK_I2, BL_BF16>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
-      else e = launch_gemv_mt<BL_PACK_I2, BL_I8>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, st);
+      if (xdt == BL_F32) e = launch_gemv_mt<BL_PACK_I2, BL_F32>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, rg, st);
+      else if (xdt == BL_BF16) e = launch_gemv_mt<BL_PACK_I2, BL_BF16>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, rg, st);
+      else e = launch_gemv_mt<BL_PACK_I2, BL_I8>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, rg, st);
     } else {
-      if (xdt == BL_F32) e = launch_gemv_mt<BL_PACK_T5, BL_F32>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
-      else if (xdt == BL_BF16) e = launch_gemv_mt<BL_PACK_T5, BL_BF16>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, st);
-      else e = launch_gemv_mt<BL_PACK_T5, BL_I8>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, st);
+      if (xdt == BL_F32) e = launch_gemv_mt<BL_PACK_T5, BL_F32>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, rg, st);
+      else if (xdt == BL_BF16) e = launch_gemv_mt<BL_PACK_T5, BL_BF16>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, rg, st);
+      else e = launch_gemv_mt<BL_PACK_T5, BL_I8>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, rg, st);
     }
     if (e != cudaSuccess) return e;
   }

@@ -53,16 +53,36 @@ cudaError_t launch_act_quant(const void* x, int xdt, int64_t M, int64_t K, int8_
 int gemv_max_tokens(int fmt, int64_t rowbytes);
 // tcgen05 GEMM on 2-bit weights; limit_cycles <= 0 uses the default wait limit.
 int gemm_token_tile(int64_t M);
-// part: ks x M x N INT32 partial sums for the split-K one-SM path
-// (ks = gemm_split_k(M, N, K)), or nullptr to keep every tile whole.
+// y: row t of the output at y + t ldy (ldy >= N).  part: ks x M x N INT32
+// partial sums for the split-K one-SM path (ks = gemm_split_k(M, N, K)), or
+// nullptr to keep every tile whole.
 cudaError_t launch_gemm_i2(const int8_t* xq, const uint8_t* w, int64_t rb, const float* gamma, const float* scale,
-                           void* y, int ydt, int64_t M, int64_t N, int64_t K, int32_t* part, void* ws,
+                           void* y, int ydt, int64_t M, int64_t N, int64_t K, int64_t ldy, int32_t* part, void* ws,
                            long long limit_cycles, int skip_producer, cudaStream_t st);
 int gemm_split_k(int64_t M, int64_t N, int64_t K);
 cudaError_t launch_t5_to_i2(const uint8_t* t5, int64_t N, int64_t K, int64_t rb5, uint8_t* i2, int64_t rb2,
                             cudaStream_t st);
+// Output rows in up to kMaxRowGroups consecutive groups, each with its own
+// gamma (row n belongs to the first group g with n < end[g]).
+constexpr int kMaxRowGroups = 8;
+struct RowGroups {
+  int n;
+  int64_t end[kMaxRowGroups];
+};
+__host__ __device__ inline int row_group(const RowGroups& rg, int64_t row) {
+  int g = 0;
+  while (g + 1 < rg.n && row >= rg.end[g]) ++g;
+  return g;
+}
+inline RowGroups one_group(int64_t N) {
+  RowGroups rg{};
+  rg.n = 1;
+  rg.end[0] = N;
+  return rg;
+}
+
 cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int64_t N, int64_t K,
                         const void* x, int xdt, float* scale, int64_t M, void* y, int ydt,
-                        cudaStream_t st);
+                        const RowGroups& rg, cudaStream_t st);
 
 }  // namespace bl

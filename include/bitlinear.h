@@ -207,6 +207,27 @@ BL_API bl_status bitlinear_forward(const uint8_t *packed, int fmt, const float *
                             int64_t K, const void *x, int xdt, float *scale, int64_t M, void *y,
                             int ydt, void *ws, size_t ws_bytes, void *stream);
 
+/* Several BitLinear layers that share their input, in one call (for example
+ * a block's Q, K and V projections).  [P3] §5.4 replaces the attention's Q, K,
+ * V and output projections by BitLinear layers of the same input size; each
+ * keeps its own gamma.  Row group g (group_rows[g] rows, at most
+ * BL_MAX_ROW_GROUPS groups) is a weight matrix; its packed rows follow those of
+ * group g - 1 in `packed`, gammas[g] is its gamma, and its outputs are the
+ * columns sum(group_rows[0..g-1]) .. + group_rows[g] - 1 of y [M, sum of
+ * group_rows].  The result equals bitlinear_forward per group: for at most 4
+ * tokens one GEMV launch covers every group; otherwise the tokens are
+ * quantized once and each group's tensor-core product writes its columns.
+ *   gammas      [ngroups] fp32 device array.
+ *   group_rows  [ngroups] host array, each >= 1.
+ *   ws          at least bitlinear_forward_grouped_workspace_bytes(...). */
+#define BL_MAX_ROW_GROUPS 8
+BL_API size_t bitlinear_forward_grouped_workspace_bytes(int64_t M, int64_t ngroups, const int64_t *group_rows,
+                                                     int64_t K, int fmt, int xdt);
+BL_API bl_status bitlinear_forward_grouped(const uint8_t *packed, int fmt, const float *gammas, int64_t ngroups,
+                                        const int64_t *group_rows, int64_t K, const void *x, int xdt,
+                                        float *scale, int64_t M, void *y, int ydt, void *ws, size_t ws_bytes,
+                                        void *stream);
+
 /* Failure-detection self test: launches the tensor-core kernel with its data
  * producer switched off and a wait limit of about a millisecond, so that its
  * bounded waits run out; the kernel then records BL_ERR_DEVICE_TIMEOUT in the

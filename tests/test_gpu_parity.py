@@ -429,3 +429,92 @@ def test_layernorm_quantize_acts_feeds_forward(orc):
     assert np.array_equal(host(xq), xq_ref)
     gam, _, packed = quantize_weights(W, I2, codes=False)
     check_forward(orc, packed, I2, gam, c["N"], K, xq_ref, scale=s_ref)
+
+
+# --- several layers sharing their input (a block's Q, K, V projections) -------------
+
+def _grouped_weights(orc, rows, K, fmt, seed):
+    """Each group quantized on its own (its own gamma); packed rows concatenated."""
+    gammas, packs = [], []
+    for i, n in enumerate(rows):
+        W = synth.normal_f32(seed + i, (n, K), 0.02 * (i + 1))
+        g, _, packed = quantize_weights(W, fmt, codes=False)
+        gammas.append(g)
+        packs.append(packed)
+    return np.array(gammas, np.float32), np.concatenate(packs, axis=0)
+
+
+def check_forward_grouped(orc, rows, K, fmt, x, scale=None, ydts=(B.BL_I32, B.BL_F32, B.BL_BF16)):
+    gammas, packed = _grouped_weights(orc, rows, K, fmt, 300 + K)
+    M, N = x.shape[0], sum(rows)
+    for ydt in ydts:
+        xd = dev(x)
+        sd = dev(scale) if scale is not None else torch.full((M,), -1.0, dtype=torch.float32, device="cuda")
+        tdt = {B.BL_F32: torch.float32, B.BL_BF16: torch.bfloat16, B.BL_I32: torch.int32}[ydt]
+        y = torch.empty((M, N), dtype=tdt, device="cuda")
+        y.view(torch.uint8).fill_(0xCD)
+        need = B.bitlinear_forward_grouped_workspace_bytes(M, rows, K, fmt, B.dtype_code(xd))
+        ws = torch.zeros(max(256, need), dtype=torch.uint8, device="cuda")
+        B.bitlinear_forward_grouped(dev(packed), fmt, dev(gammas), rows, K, xd, sd, y, ws)
+        torch.cuda.synchronize()
+        assert B.bitlinear_device_status(ws) == B.BL_OK
+        yh, sh = host(y), host(sd)
+        off = 0
+        for g, n in enumerate(rows):
+            y_ref, s_ref = orc.forward(packed[off:off + n], fmt, gammas[g], n, K, x, ydt=ydt, scale=scale)
+            assert np.array_equal(sh, s_ref)
+            got = yh[:, off:off + n]
+            if ydt == B.BL_I32:
+                assert np.array_equal(got, y_ref), (g, n)
+            elif ydt == B.BL_F32:
+                assert_f32_rel(got, y_ref)
+            else:
+                assert_bf16_ulp(got, y_ref)
+            off += n
+        assert off == N
+
+
+@pytest.mark.parametrize("M", [1, 3, 4, 5, 16, 40, 130])
+@pytest.mark.parametrize("fmt", [I2, T5])
+def test_forward_grouped_qkv(orc, M, fmt):
+    """Three groups of ragged sizes (unaligned column offsets included), one
+    GEMV launch for up to 4 tokens, one product per group beyond."""
+    K = 640
+    x = synth.to_bf16_bits(synth.normal_f32(310 + M, (M, K)))
+    check_forward_grouped(orc, [200, 72, 131], K, fmt, x)
+
+
+def test_forward_grouped_aligned_columns_int8_tokens(orc):
+    """Row counts that keep every group's columns 16-byte aligned (the tensor
+    map store path), int8 tokens with given scales."""
+    M, K = 24, 1024
+    xf = synth.normal_f32(320, (M, K))
+    xq, s = orc.act_quant(xf)
+    check_forward_grouped(orc, [256, 128, 384], K, I2, xq.astype(np.int8), scale=s)
+
+
+def test_forward_grouped_one_group_matches_forward(orc):
+    """A single group is the plain forward."""
+    K, n = 512, 333
+    x = synth.normal_f32(321, (2, K))
+    check_forward_grouped(orc, [n], K, T5, x)
+
+
+def test_forward_grouped_eight_groups_decode(orc):
+    """The most groups one call takes, at one token, with one-row groups in it."""
+    K = 384
+    x = synth.to_bf16_bits(synth.normal_f32(322, (1, K)))
+    check_forward_grouped(orc, [1, 64, 3, 128, 1, 200, 17, 90], K, I2, x)
+
+
+def test_forward_grouped_rejects_bad_groups():
+    g = torch.ones(9, dtype=torch.float32, device="cuda")
+    x = torch.zeros((1, 64), dtype=torch.bfloat16, device="cuda")
+    s = torch.empty(1, dtype=torch.float32, device="cuda")
+    y = torch.empty((1, 9), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    p = torch.zeros((9, 16), dtype=torch.uint8, device="cuda")
+    for rows in ([1] * 9, [3, 0, 6], []):
+        with pytest.raises(B.BitLinearError) as e:
+            B.bitlinear_forward_grouped(p, I2, g, rows, 64, x, s, y, ws)
+        assert e.value.status == B.BL_ERR_INVALID_VALUE
