@@ -27,7 +27,7 @@ SRC = os.path.join(HERE, "bitlinear_oracle.c")
 LIB_PATH = os.path.join(HERE, "liboracle.so")
 
 F32, BF16, I8, I32 = 0, 1, 2, 3
-PACK_I2, PACK_T5 = 0, 1
+PACK_I2, PACK_T5, PACK_B1 = 0, 1, 2
 
 _lib = None
 _lock = threading.Lock()
@@ -55,6 +55,10 @@ def lib() -> C.CDLL:
             p, i64, f, d, i = C.c_void_p, C.c_int64, C.c_float, C.c_double, C.c_int
             L.orc_absmean_sum.argtypes = [p, i, i64, i64]
             L.orc_absmean_sum.restype = d
+            L.orc_signed_sum.argtypes = [p, i, i64, i64]
+            L.orc_signed_sum.restype = d
+            L.orc_binarize_weights.argtypes = [p, i, i64, i64, p, p, p]
+            L.orc_binarize_weights.restype = None
             L.orc_gamma.argtypes = [p, i, i64, i64]
             L.orc_gamma.restype = f
             L.orc_ternarize.argtypes = [p, i, i64, i64, f, f, p]
@@ -152,7 +156,7 @@ def pack(codes: np.ndarray, fmt: int) -> np.ndarray:
     out = np.empty((N, packed_row_bytes(K, fmt)), np.uint8)
     rc = lib().orc_pack(_ptr(codes), N, K, fmt, _ptr(out))
     if rc != 0:
-        raise ValueError("code outside {-1, 0, 1}")
+        raise ValueError("code outside {-1, 0, 1} ({-1, 1} for the 1-bit format)")
     return out
 
 
@@ -245,6 +249,24 @@ def onebit(w: np.ndarray):
     be = C.c_float()
     lib().orc_onebit(_ptr(w), w.size, _ptr(b), C.byref(a), C.byref(be))
     return b, np.float32(a.value), np.float32(be.value)
+
+
+# --- 1-bit variant: alpha, beta and the {-1, +1} codes of a whole matrix ----------
+
+def signed_sum(W: np.ndarray) -> float:
+    """fp64 sum of w over W [N, K] in the fixed reduction order of step 1."""
+    N, K = W.shape
+    return lib().orc_signed_sum(_ptr(W), _dt(W), N, K)
+
+
+def binarize_weights(W: np.ndarray):
+    """1-bit weights of W [N, K]: returns (alpha, beta, codes int8 in {-1, +1})."""
+    N, K = W.shape
+    codes = np.empty((N, K), np.int8)
+    a = C.c_float()
+    b = C.c_float()
+    lib().orc_binarize_weights(_ptr(W), _dt(W), N, K, C.byref(a), C.byref(b), _ptr(codes))
+    return np.float32(a.value), np.float32(b.value), codes
 
 
 def f32_to_bf16(v: float) -> int:

@@ -38,6 +38,7 @@
 
 #define ORC_PACK_I2 0 /* 2 bits per weight, 4 weights per byte */
 #define ORC_PACK_T5 1 /* 5 trits per byte, base 3 */
+#define ORC_PACK_B1 2 /* 1 bit per weight, 8 weights per byte (1-bit BitNet) */
 
 /* ------------------------------------------------------------------------ */
 /* dtype helpers                                                            */
@@ -88,14 +89,20 @@ static float load_f(const void *p, int dt, int64_t i) {
 #define ORC_CHUNK 8192
 #define ORC_LANES 256
 
-static double chunk_sum(const void *W, int dt, int64_t T, int64_t c) {
+/* absval = 1: the terms are |w|; absval = 0: the terms are w (the signed  */
+/* sum of the 1-bit variant below takes the same order).                    */
+static double chunk_sum(const void *W, int dt, int64_t T, int64_t c,
+                        int absval) {
   double p[ORC_LANES];
   for (int l = 0; l < ORC_LANES; ++l) {
     double acc = 0.0;
     for (int i = 0; i < 4; ++i)
       for (int j = 0; j < 8; ++j) {
         int64_t e = c * ORC_CHUNK + 2048 * (int64_t)i + 8 * (int64_t)l + j;
-        if (e < T) acc += (double)fabsf(load_f(W, dt, e));
+        if (e < T) {
+          float w = load_f(W, dt, e);
+          acc += (double)(absval ? fabsf(w) : w);
+        }
       }
     p[l] = acc;
   }
@@ -104,7 +111,8 @@ static double chunk_sum(const void *W, int dt, int64_t T, int64_t c) {
   return p[0];
 }
 
-double orc_absmean_sum(const void *W, int dt, int64_t N, int64_t K) {
+static double fixed_order_sum(const void *W, int dt, int64_t N, int64_t K,
+                              int absval) {
   int64_t T = N * K;
   if (T <= 0) return 0.0;
   int64_t C = (T + ORC_CHUNK - 1) / ORC_CHUNK;
@@ -112,12 +120,20 @@ double orc_absmean_sum(const void *W, int dt, int64_t N, int64_t K) {
   while (P < C) P *= 2;
   double *q = (double *)calloc((size_t)P, sizeof(double));
   if (!q) return NAN;
-  for (int64_t c = 0; c < C; ++c) q[c] = chunk_sum(W, dt, T, c);
+  for (int64_t c = 0; c < C; ++c) q[c] = chunk_sum(W, dt, T, c, absval);
   for (int64_t s = P / 2; s >= 1; s /= 2)
     for (int64_t c = 0; c < s; ++c) q[c] += q[c + s];
   double S = q[0];
   free(q);
   return S;
+}
+
+double orc_absmean_sum(const void *W, int dt, int64_t N, int64_t K) {
+  return fixed_order_sum(W, dt, N, K, 1);
+}
+
+double orc_signed_sum(const void *W, int dt, int64_t N, int64_t K) {
+  return fixed_order_sum(W, dt, N, K, 0);
 }
 
 float orc_gamma(const void *W, int dt, int64_t N, int64_t K) {
@@ -159,7 +175,13 @@ void orc_ternarize(const void *W, int dt, int64_t N, int64_t K, float gamma,
 /* 2-bit format, 121 in base 3).                                            */
 /* ------------------------------------------------------------------------ */
 
-static int per_byte(int fmt) { return fmt == ORC_PACK_I2 ? 4 : 5; }
+/* The 1-bit format (ORC_PACK_B1) follows the same byte order: bit i of     */
+/* byte j holds weight 8 j + i, 1 for +1 and 0 for -1; pad bits are 0 (the  */
+/* pages give 8 weights per byte and no bit order, so this is a reading).   */
+
+static int per_byte(int fmt) {
+  return fmt == ORC_PACK_I2 ? 4 : (fmt == ORC_PACK_T5 ? 5 : 8);
+}
 
 int64_t orc_packed_row_bytes(int64_t K, int fmt) {
   int64_t per = per_byte(fmt);
@@ -167,7 +189,7 @@ int64_t orc_packed_row_bytes(int64_t K, int fmt) {
   return (used + 15) / 16 * 16;
 }
 
-/* returns 0, or -1 if a code is outside {-1, 0, 1} */
+/* returns 0, or -1 if a code is outside {-1, 0, 1} ({-1, 1} for 1 bit) */
 int orc_pack(const int8_t *codes, int64_t N, int64_t K, int fmt,
              uint8_t *packed) {
   int per = per_byte(fmt);
@@ -181,6 +203,11 @@ int orc_pack(const int8_t *codes, int64_t N, int64_t K, int fmt,
         if (k < K) {
           q = codes[n * K + k];
           if (q < -1 || q > 1) return -1;
+          if (fmt == ORC_PACK_B1 && q == 0) return -1;
+        }
+        if (fmt == ORC_PACK_B1) {
+          if (q > 0) byte |= 1u << i;
+          continue;
         }
         unsigned digit = (unsigned)(q + 1);
         if (fmt == ORC_PACK_I2)
@@ -206,6 +233,15 @@ int orc_unpack(const uint8_t *packed, int64_t N, int64_t K, int fmt,
       if (fmt == ORC_PACK_T5 && byte >= 243) return -1;
       for (int i = 0; i < per; ++i) {
         unsigned digit;
+        if (fmt == ORC_PACK_B1) {
+          unsigned bit = (byte >> i) & 1u;
+          int64_t kb = j * per + i;
+          if (kb < K)
+            codes[n * K + kb] = (int8_t)(bit ? 1 : -1);
+          else if (bit != 0)
+            return -2;
+          continue;
+        }
         if (fmt == ORC_PACK_I2) {
           digit = (byte >> (2 * i)) & 3u;
           if (digit == 3) return -1;
@@ -346,6 +382,30 @@ void orc_onebit(const float *w, int64_t n, int8_t *b, float *alpha,
   *alpha = a;
   *beta = (float)(sa / (double)n);
   for (int64_t i = 0; i < n; ++i) b[i] = (int8_t)(w[i] > a ? 1 : -1);
+}
+
+/* ------------------------------------------------------------------------ */
+/* 1-bit BitNet weights for a whole matrix (the 1-bit variant of steps 1-2). */
+/* [P1]/[P5] "The BitLinear Recipe" step 2 (alpha = mean of the weights;    */
+/* a weight above alpha becomes +1, one below -1) and step 4 (beta = mean   */
+/* |W| rescales the output, in place of gamma).                             */
+/* Readings: alpha and beta are fp64 sums in the fixed order of step 1 (for */
+/* alpha the terms are w, for beta |w|), divided by N K and rounded to fp32; */
+/* beta is therefore gamma.  A weight equal to alpha maps to -1 (the pages  */
+/* do not say); w > alpha in fp32 is the sign of w - alpha, since the fp32  */
+/* difference of two distinct floats is never 0.  The forward is then steps */
+/* 4-6 unchanged with codes in {-1, +1} and beta as the weight factor.      */
+/* ------------------------------------------------------------------------ */
+
+void orc_binarize_weights(const void *W, int dt, int64_t N, int64_t K,
+                          float *alpha, float *beta, int8_t *codes) {
+  double S = orc_signed_sum(W, dt, N, K);
+  float a = (float)(S / (double)(N * K));
+  *alpha = a;
+  *beta = orc_gamma(W, dt, N, K);
+  if (codes != NULL)
+    for (int64_t e = 0; e < N * K; ++e)
+      codes[e] = (int8_t)(load_f(W, dt, e) > a ? 1 : -1);
 }
 
 /* ------------------------------------------------------------------------ */
