@@ -56,6 +56,7 @@ WORKLOADS = {
 # ----------------------------------------------------------------------------
 
 KERNEL_SOURCE = {"absmean_kernel": "bl_weights.cu", "ternarize_flat_kernel": "bl_weights.cu",
+                 "binarize_pack_kernel": "bl_weights.cu",
                  "ternarize_pack_kernel": "bl_weights.cu", "gemv_i2_kernel": "bl_gemv.cu",
                  "gemv_kernel": "bl_gemv.cu", "gemv_t5_kernel": "bl_gemv.cu", "gemv_i2_mt_kernel": "bl_gemv.cu", "act_quant_row_kernel": "bl_acts.cu",
                  "act_quant_kernel": "bl_acts.cu", "ln_quant_kernel": "bl_acts.cu", "gemm_i2_2sm_kernel": "bl_gemm_sm100.cu",
@@ -491,7 +492,8 @@ DECODE_SHAPES = {"3b": ("3b_decode", "3B decode: M=1, K=3200->N=8640 and K=8640-
 
 def run_decode(args, dev, stream, rank_seed, l2):
     """Decode GEMV alone (steps 4-6, M=1) on weights packed beforehand, for the
-    3B and 70B layer shapes, 2-bit and base-3: a graph of ``decode_steps``
+    3B and 70B layer shapes, 2-bit, base-3 and 1-bit (the 1-bit BitNet variant,
+    weights from bitlinear_binarize_weights): a graph of ``decode_steps``
     forward calls per layer over packed copies rotated so that consecutive reads
     exceed 4x L2, timed at its two ends.  Per layer: average launch duration,
     GB/s of algorithmic bytes and the fraction of the HBM peak."""
@@ -504,7 +506,7 @@ def run_decode(args, dev, stream, rank_seed, l2):
     out = {}
     for key, (wname, desc) in DECODE_SHAPES.items():
         wl = WORKLOADS[wname]
-        for fmt in (0, 1):
+        for fmt in (0, 1, 2):
             rows = []
             for i, (N, K) in enumerate(wl["layers"]):
                 Wh = synth.normal_f32(1000 + wl["seed"] + 100 * i + rank_seed, (N, K), wl["sigma"])
@@ -513,10 +515,16 @@ def run_decode(args, dev, stream, rank_seed, l2):
                 W = torch.from_numpy(Wh).to(dev)
                 del Wh
                 gamma = torch.empty(1, dtype=torch.float32, device=dev)
-                ws = torch.zeros(B.bitlinear_quantize_weights_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
                 p0 = torch.empty((N, rb), dtype=torch.uint8, device=dev)
-                with torch.cuda.stream(stream):
-                    B.bitlinear_quantize_weights(W, 1e-5, fmt, p0, None, gamma, ws, stream)
+                if fmt == B.BL_PACK_B1:
+                    ws = torch.zeros(B.bitlinear_binarize_weights_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+                    alpha = torch.empty(1, dtype=torch.float32, device=dev)
+                    with torch.cuda.stream(stream):
+                        B.bitlinear_binarize_weights(W, p0, None, gamma, alpha, ws, stream)
+                else:
+                    ws = torch.zeros(B.bitlinear_quantize_weights_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+                    with torch.cuda.stream(stream):
+                        B.bitlinear_quantize_weights(W, 1e-5, fmt, p0, None, gamma, ws, stream)
                 stream.synchronize()
                 del W
                 rot = max(2, -(-4 * l2 // (N * rb)))
@@ -541,7 +549,7 @@ def run_decode(args, dev, stream, rank_seed, l2):
                 nbytes = layer_bytes(N, K, 1, rb)["forward"]
                 rows.append(dict(N=N, K=K, us=us, bytes=nbytes, rot=rot))
                 del copies, p0
-            out[f"{key}_{['2bit', 'base3'][fmt]}"] = dict(desc=desc, rows=rows)
+            out[f"{key}_{['2bit', 'base3', '1bit'][fmt]}"] = dict(desc=desc, rows=rows)
     return out
 
 
@@ -685,8 +693,8 @@ def decode_summary(d):
         tot_b = sum(r["bytes"] for r in rows)
         tot_us = sum(r["us"] for r in rows)
         gbs = tot_b / (tot_us * 1e-6) / 1e9
-        fmt = 1 if name.endswith("base3") else 0
-        res[name] = {"workload": v["desc"] + (", base-3 pack" if fmt else ", 2-bit pack"),
+        fmt = 1 if name.endswith("base3") else (2 if name.endswith("1bit") else 0)
+        res[name] = {"workload": v["desc"] + [", 2-bit pack", ", base-3 pack", ", 1-bit weights (8 per byte)"][fmt],
                      "kernel": gemv_kernel_name(fmt, [(r["N"], r["K"]) for r in rows]), "GB_s": gbs, "frac_of_hbm": gbs / peak,
                      "per_layer": [{"N": r["N"], "K": r["K"], "us_per_launch": r["us"], "bytes_per_launch": r["bytes"],
                                     "GB_s": r["bytes"] / (r["us"] * 1e-6) / 1e9,
@@ -703,6 +711,8 @@ def gemv_kernel_name(fmt, layers, M=1):
     of at most 8192 packed bytes; for one token of base 3,
     the column-stationary kernel for rows of at most 768 segments and at most
     1024 rows per CTA (148 CTAs); else the general one."""
+    if fmt == 2:  # 1-bit rows of at most 4096 bytes: the lean kernel's 1-bit form
+        return "gemv_i2_kernel" if all(((K + 7) // 8 + 15) // 16 * 16 <= 4096 for (_, K) in layers) else "gemv_kernel"
     if fmt == 0:
         rbs = [((K + 3) // 4 + 15) // 16 * 16 for (_, K) in layers]
         if 2 <= M <= 4 and all(rb <= 8192 and -(-N // min(N, 148)) <= 1024 for rb, (N, _) in zip(rbs, layers)):
@@ -753,6 +763,8 @@ PROFILE_CASES = {
     "batch16_70b_up": dict(N=28672, K=8192, fmt=0, M=16, sigma=0.01, op="forward"),
     "lnquant_3b_prefill": dict(N=8640, K=3200, fmt=0, M=4096, sigma=0.02, op="lnquant"),
     "batch16_70b_down": dict(N=8192, K=28672, fmt=0, M=16, sigma=0.01, op="forward"),
+    "binarize_3b_up": dict(N=8640, K=3200, fmt=2, M=1, sigma=0.02, op="quantize"),
+    "decode_70b_up_1bit": dict(N=28672, K=8192, fmt=2, M=1, sigma=0.01, op="forward"),
 }
 
 
@@ -772,9 +784,15 @@ def run_profile_case(name):
     x = torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16)
     packed = torch.empty((N, B.bitlinear_packed_row_bytes(K, fmt)), dtype=torch.uint8, device=dev)
     gamma = torch.empty(1, dtype=torch.float32, device=dev)
-    ws = torch.zeros(B.bitlinear_quantize_weights_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
-    for _ in range(3 if c["op"] == "quantize" else 1):
-        B.bitlinear_quantize_weights(W, 1e-5, fmt, packed, None, gamma, ws)
+    if fmt == B.BL_PACK_B1:  # the 1-bit variant: beta (in gamma's place) and alpha
+        alpha = torch.empty(1, dtype=torch.float32, device=dev)
+        ws = torch.zeros(B.bitlinear_binarize_weights_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+        for _ in range(3 if c["op"] == "quantize" else 1):
+            B.bitlinear_binarize_weights(W, packed, None, gamma, alpha, ws)
+    else:
+        ws = torch.zeros(B.bitlinear_quantize_weights_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+        for _ in range(3 if c["op"] == "quantize" else 1):
+            B.bitlinear_quantize_weights(W, 1e-5, fmt, packed, None, gamma, ws)
     status = [B.bitlinear_device_status(ws)]
     if c["op"] == "lnquant":
         ln_w = torch.randn(K, generator=g, device=dev) * 0.1 + 1.0

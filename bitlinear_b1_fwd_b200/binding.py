@@ -20,7 +20,7 @@ BL_OK, BL_ERR_INVALID_VALUE, BL_ERR_UNSUPPORTED, BL_ERR_MISALIGNED = 0, 1, 2, 3
 BL_ERR_WORKSPACE_TOO_SMALL, BL_ERR_CUDA, BL_ERR_DEVICE_TIMEOUT, BL_ERR_BAD_CODE = 4, 5, 6, 7
 BL_ERR_SCRATCH_LIMIT = 8
 BL_F32, BL_BF16, BL_I8, BL_I32 = 0, 1, 2, 3
-BL_PACK_I2, BL_PACK_T5 = 0, 1
+BL_PACK_I2, BL_PACK_T5, BL_PACK_B1 = 0, 1, 2
 BL_WS_HEADER_BYTES = 256
 
 # (name, restype, argtypes) of every exported entry point
@@ -35,6 +35,8 @@ SIGNATURES = {
     "bitlinear_absmean_noalloc": (_I, [_P, _I, _I64, _I64, _P, _P]),
     "bitlinear_ternarize_pack": (_I, [_P, _I, _I64, _I64, _P, _F, _I, _P, _P, _P]),
     "bitlinear_pack": (_I, [_P, _I64, _I64, _I, _P, _P, _SZ, _P]),
+    "bitlinear_binarize_weights_workspace_bytes": (_SZ, [_I64, _I64]),
+    "bitlinear_binarize_weights": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _P, _P, _SZ, _P]),
     "bitlinear_quantize_acts": (_I, [_P, _I, _I64, _I64, _P, _P, _P]),
     "bitlinear_layernorm_quantize_acts": (_I, [_P, _I, _P, _P, _F, _I64, _I64, _P, _P, _P, _P]),
     "bitlinear_forward": (_I, [_P, _I, _P, _I64, _I64, _P, _I, _P, _I64, _P, _I, _P, _SZ, _P]),
@@ -118,6 +120,10 @@ def bitlinear_quantize_weights_workspace_bytes(N: int, K: int) -> int:
     return int(lib().bitlinear_quantize_weights_workspace_bytes(N, K))
 
 
+def bitlinear_binarize_weights_workspace_bytes(N: int, K: int) -> int:
+    return int(lib().bitlinear_binarize_weights_workspace_bytes(N, K))
+
+
 def bitlinear_forward_workspace_bytes(M: int, N: int, K: int, fmt: int, xdt: int) -> int:
     return int(lib().bitlinear_forward_workspace_bytes(M, N, K, fmt, xdt))
 
@@ -192,6 +198,14 @@ def bitlinear_layernorm_quantize_acts(x, ln_w, ln_b, eps, xq, scale, y=None, str
     _check(lib().bitlinear_layernorm_quantize_acts(_ptr(x), dtype_code(x), _ptr(ln_w), _ptr(ln_b), float(eps), M, K,
                                                    _ptr(y), _ptr(xq), _ptr(scale), _stream(stream)),
            "bitlinear_layernorm_quantize_acts")
+
+
+def bitlinear_binarize_weights(W, packed, codes, beta, alpha, ws, stream=None) -> None:
+    _contig(W, packed, codes, beta, alpha, ws)
+    N, K = W.shape
+    _check(lib().bitlinear_binarize_weights(_ptr(W), dtype_code(W), N, K, _ptr(packed), _ptr(codes), _ptr(beta),
+                                            _ptr(alpha), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "bitlinear_binarize_weights")
 
 
 def bitlinear_forward(packed, fmt, gamma, N, K, x, scale, y, ws, stream=None) -> None:

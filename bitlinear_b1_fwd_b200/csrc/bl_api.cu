@@ -16,7 +16,8 @@ constexpr int kVersion = 100;  // 0.1.0
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 inline size_t round256(size_t v) { return (v + 255) / 256 * 256; }
 inline bool float_dt(int dt) { return dt == BL_F32 || dt == BL_BF16; }
-inline bool fmt_ok(int fmt) { return fmt == BL_PACK_I2 || fmt == BL_PACK_T5; }
+inline bool fmt_ok(int fmt) { return fmt == BL_PACK_I2 || fmt == BL_PACK_T5 || fmt == BL_PACK_B1; }
+inline bool tern_fmt_ok(int fmt) { return fmt == BL_PACK_I2 || fmt == BL_PACK_T5; }  // ternary formats
 
 inline bl_status cuda_status(cudaError_t e) { return e == cudaSuccess ? BL_OK : BL_ERR_CUDA; }
 
@@ -49,7 +50,7 @@ const char* bitlinear_status_string(int status) {
 
 int64_t bitlinear_packed_row_bytes(int64_t K, int fmt) {
   if (K < 1 || K > kMaxK || !fmt_ok(fmt)) return -1;
-  const int64_t per = fmt == BL_PACK_I2 ? 4 : 5;
+  const int64_t per = fmt == BL_PACK_I2 ? 4 : (fmt == BL_PACK_T5 ? 5 : 8);
   return ((K + per - 1) / per + 15) / 16 * 16;
 }
 
@@ -62,15 +63,20 @@ size_t bitlinear_quantize_weights_workspace_bytes(int64_t N, int64_t K) {
 // The tensor-core path serves more tokens than one GEMV launch holds, when the
 // x_q rows can be a TMA tensor (row stride a multiple of 16 bytes).
 bool uses_gemm(int64_t M, int64_t K) { return M > bl::kGemvMaxTokens && (K % 16) == 0; }
+// 1-bit rows longer than the 1-bit GEMV takes (4096 bytes: K > 32768) are
+// transcoded to 2 bits in the workspace for the decode path too.
+bool b1_via_i2(int fmt, int64_t K) { return fmt == BL_PACK_B1 && (K + 7) / 8 > 4096; }
 
 size_t bitlinear_forward_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int xdt) {
   if (M < 0 || !nk_ok(N, K) || !fmt_ok(fmt)) return 0;
   size_t bytes = BL_WS_HEADER_BYTES;
   if (uses_gemm(M, K)) {
     if (xdt != BL_I8) bytes += round256(static_cast<size_t>(M * K));
-    if (fmt == BL_PACK_T5) bytes += round256(static_cast<size_t>(N * bitlinear_packed_row_bytes(K, BL_PACK_I2)));
+    if (fmt != BL_PACK_I2) bytes += round256(static_cast<size_t>(N * bitlinear_packed_row_bytes(K, BL_PACK_I2)));
     const int ks = bl::gemm_split_k(M, N, K);
     if (ks > 1) bytes += round256(static_cast<size_t>(ks) * M * N * sizeof(int32_t));
+  } else if (b1_via_i2(fmt, K)) {
+    bytes += round256(static_cast<size_t>(N * bitlinear_packed_row_bytes(K, BL_PACK_I2)));
   }
   return bytes;
 }
@@ -85,7 +91,7 @@ bl_status bitlinear_quantize_weights(const void* W, int wdt, int64_t N, int64_t 
                                      size_t ws_bytes, void* stream) {
   if (W == nullptr || gamma == nullptr || ws == nullptr || (packed == nullptr && codes == nullptr))
     return BL_ERR_INVALID_VALUE;
-  if (!float_dt(wdt) || !fmt_ok(fmt) || N < 1 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
+  if (!float_dt(wdt) || !tern_fmt_ok(fmt) || N < 1 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
   if (!(eps > 0.0f) || !std::isfinite(eps)) return BL_ERR_INVALID_VALUE;
   if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(codes, 16) || !aligned(gamma, 4) ||
       !aligned(ws, 16))
@@ -110,13 +116,34 @@ bl_status bitlinear_absmean(const void* W, int wdt, int64_t N, int64_t K, float*
 bl_status bitlinear_ternarize_pack(const void* W, int wdt, int64_t N, int64_t K, const float* gamma,
                                    float eps, int fmt, uint8_t* packed, int8_t* codes, void* stream) {
   if (W == nullptr || gamma == nullptr || (packed == nullptr && codes == nullptr)) return BL_ERR_INVALID_VALUE;
-  if (!float_dt(wdt) || !fmt_ok(fmt) || N < 1 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
+  if (!float_dt(wdt) || !tern_fmt_ok(fmt) || N < 1 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
   if (!(eps > 0.0f) || !std::isfinite(eps)) return BL_ERR_INVALID_VALUE;
   if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(codes, 16) || !aligned(gamma, 4))
     return BL_ERR_MISALIGNED;
   const int64_t rb = bitlinear_packed_row_bytes(K, fmt);
   return cuda_status(bl::launch_ternarize_pack(W, wdt, N, K, gamma, eps, fmt, packed, codes, rb, nullptr,
                                                static_cast<cudaStream_t>(stream)));
+}
+
+size_t bitlinear_binarize_weights_workspace_bytes(int64_t N, int64_t K) {
+  if (N < 1 || !nk_ok(N, K)) return 0;
+  const int64_t chunks = (N * K + bl::kChunk - 1) / bl::kChunk;
+  return BL_WS_HEADER_BYTES + round256(static_cast<size_t>(2 * chunks) * sizeof(double));
+}
+
+bl_status bitlinear_binarize_weights(const void* W, int wdt, int64_t N, int64_t K, uint8_t* packed, int8_t* codes,
+                                     float* beta, float* alpha, void* ws, size_t ws_bytes, void* stream) {
+  if (W == nullptr || beta == nullptr || alpha == nullptr || ws == nullptr || (packed == nullptr && codes == nullptr))
+    return BL_ERR_INVALID_VALUE;
+  if (!float_dt(wdt) || N < 1 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
+  if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(codes, 16) || !aligned(beta, 4) || !aligned(alpha, 4) ||
+      !aligned(ws, 16))
+    return BL_ERR_MISALIGNED;
+  if (ws_bytes < bitlinear_binarize_weights_workspace_bytes(N, K)) return BL_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (bl::launch_absmean(W, wdt, N, K, ws, beta, st, alpha) != cudaSuccess) return BL_ERR_CUDA;
+  const int64_t rb = bitlinear_packed_row_bytes(K, BL_PACK_B1);
+  return cuda_status(bl::launch_binarize_pack(W, wdt, N, K, alpha, packed, codes, rb, st));
 }
 
 bl_status bitlinear_pack(const int8_t* codes, int64_t N, int64_t K, int fmt, uint8_t* packed, void* ws,
@@ -168,6 +195,14 @@ bl_status bitlinear_forward(const uint8_t* packed, int fmt, const float* gamma, 
   if (ws_bytes < bitlinear_forward_workspace_bytes(M, N, K, fmt, xdt)) return BL_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (!uses_gemm(M, K)) {
+    if (b1_via_i2(fmt, K)) {
+      uint8_t* w2 = static_cast<uint8_t*>(ws) + BL_WS_HEADER_BYTES;
+      const int64_t rb2 = bitlinear_packed_row_bytes(K, BL_PACK_I2);
+      if (bl::launch_b1_to_i2(packed, N, K, bitlinear_packed_row_bytes(K, fmt), w2, rb2, st) != cudaSuccess)
+        return BL_ERR_CUDA;
+      packed = w2;
+      fmt = BL_PACK_I2;
+    }
     if (bl::gemv_max_tokens(fmt, bitlinear_packed_row_bytes(K, fmt)) < 1) return BL_ERR_UNSUPPORTED;
     return cuda_status(bl::launch_gemv(packed, fmt, gamma, N, K, x, xdt, scale, M, y, ydt, bl::one_group(N), st));
   }
@@ -181,9 +216,11 @@ bl_status bitlinear_forward(const uint8_t* packed, int fmt, const float* gamma, 
   }
   const int64_t rb2 = bitlinear_packed_row_bytes(K, BL_PACK_I2);
   const uint8_t* w2 = packed;
-  if (fmt == BL_PACK_T5) {
-    if (bl::launch_t5_to_i2(packed, N, K, bitlinear_packed_row_bytes(K, fmt), scratch, rb2, st) != cudaSuccess)
-      return BL_ERR_CUDA;
+  if (fmt != BL_PACK_I2) {
+    const int64_t rb = bitlinear_packed_row_bytes(K, fmt);
+    const cudaError_t e = fmt == BL_PACK_T5 ? bl::launch_t5_to_i2(packed, N, K, rb, scratch, rb2, st)
+                                            : bl::launch_b1_to_i2(packed, N, K, rb, scratch, rb2, st);
+    if (e != cudaSuccess) return BL_ERR_CUDA;
     w2 = scratch;
     scratch += round256(static_cast<size_t>(N * rb2));
   }
@@ -215,12 +252,14 @@ size_t bitlinear_forward_grouped_workspace_bytes(int64_t M, int64_t ngroups, con
     for (int64_t g = 0; g < ngroups; ++g) {
       const int64_t Ng = group_rows[g];
       size_t e = 0;
-      if (fmt == BL_PACK_T5) e += round256(static_cast<size_t>(Ng * bitlinear_packed_row_bytes(K, BL_PACK_I2)));
+      if (fmt != BL_PACK_I2) e += round256(static_cast<size_t>(Ng * bitlinear_packed_row_bytes(K, BL_PACK_I2)));
       const int ks = bl::gemm_split_k(M, Ng, K);
       if (ks > 1) e += round256(static_cast<size_t>(ks) * M * Ng * sizeof(int32_t));
       if (e > most) most = e;
     }
     bytes += most;
+  } else if (b1_via_i2(fmt, K)) {
+    bytes += round256(static_cast<size_t>(N * bitlinear_packed_row_bytes(K, BL_PACK_I2)));
   }
   return bytes;
 }
@@ -243,7 +282,14 @@ bl_status bitlinear_forward_grouped(const uint8_t* packed, int fmt, const float*
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t rb = bitlinear_packed_row_bytes(K, fmt);
   if (!uses_gemm(M, K)) {  // one GEMV launch over every group's rows
-    if (bl::gemv_max_tokens(fmt, rb) < 1) return BL_ERR_UNSUPPORTED;
+    if (b1_via_i2(fmt, K)) {
+      uint8_t* w2 = static_cast<uint8_t*>(ws) + BL_WS_HEADER_BYTES;
+      if (bl::launch_b1_to_i2(packed, N, K, rb, w2, bitlinear_packed_row_bytes(K, BL_PACK_I2), st) != cudaSuccess)
+        return BL_ERR_CUDA;
+      packed = w2;
+      fmt = BL_PACK_I2;
+    }
+    if (bl::gemv_max_tokens(fmt, bitlinear_packed_row_bytes(K, fmt)) < 1) return BL_ERR_UNSUPPORTED;
     bl::RowGroups rg{};
     rg.n = static_cast<int>(ngroups);
     int64_t end = 0;
@@ -266,8 +312,10 @@ bl_status bitlinear_forward_grouped(const uint8_t* packed, int fmt, const float*
     const int64_t Ng = group_rows[g];
     uint8_t* s2 = scratch;
     const uint8_t* w2 = packed + off * rb;
-    if (fmt == BL_PACK_T5) {
-      if (bl::launch_t5_to_i2(w2, Ng, K, rb, s2, rb2, st) != cudaSuccess) return BL_ERR_CUDA;
+    if (fmt != BL_PACK_I2) {
+      const cudaError_t ce = fmt == BL_PACK_T5 ? bl::launch_t5_to_i2(w2, Ng, K, rb, s2, rb2, st)
+                                               : bl::launch_b1_to_i2(w2, Ng, K, rb, s2, rb2, st);
+      if (ce != cudaSuccess) return BL_ERR_CUDA;
       w2 = s2;
       s2 += round256(static_cast<size_t>(Ng * rb2));
     }

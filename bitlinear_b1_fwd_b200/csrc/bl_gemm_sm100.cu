@@ -895,6 +895,46 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// 1-bit -> 2-bit transcoding (for the tensor-core path, and for decode rows
+// too long for the 1-bit GEMV): one thread writes one 16-byte segment (64
+// weights) of a 2-bit row from 8 bytes of the 1-bit row.  A set bit (+1) is
+// digit 2, a clear bit (-1) digit 0; weights past K are digit 1 (weight 0).
+__device__ __forceinline__ uint32_t spread16_to_2bit(uint32_t h) {  // bit i -> bit 2i
+  uint32_t x = h & 0xffffu;
+  x = (x | (x << 8)) & 0x00ff00ffu;
+  x = (x | (x << 4)) & 0x0f0f0f0fu;
+  x = (x | (x << 2)) & 0x33333333u;
+  x = (x | (x << 1)) & 0x55555555u;
+  return x;
+}
+
+__global__ void __launch_bounds__(256)
+    b1_to_i2_kernel(const uint8_t* __restrict__ b1, int64_t N, int64_t K, int64_t rb1, uint8_t* __restrict__ i2,
+                    int64_t rb2) {
+  pdl_enter(b1, i2);
+  const int64_t segs = rb2 / 16;
+  for (int64_t gid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; gid < N * segs;
+       gid += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = gid / segs, sg = gid - n * segs;
+    const uint8_t* row = b1 + n * rb1;
+    uint32_t out[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {  // 16 weights: two bytes of the 1-bit row
+      const int64_t j = 8 * sg + 2 * w;
+      const uint32_t bits = (j < rb1 ? __ldcg(row + j) : 0u) | ((j + 1 < rb1 ? __ldcg(row + j + 1) : 0u) << 8);
+      uint32_t d = spread16_to_2bit(bits) << 1;  // +1 -> 10, -1 -> 00
+      const int64_t k0 = 64 * sg + 16 * w;
+      if (k0 + 16 > K) {
+        const int64_t valid = K - k0 < 0 ? 0 : K - k0;  // weights of the word below K
+        const uint32_t keep = valid >= 16 ? 0xffffffffu : ((1u << (2 * valid)) - 1u);
+        d = (d & keep) | (0x55555555u & ~keep);
+      }
+      out[w] = d;
+    }
+    *reinterpret_cast<uint4*>(i2 + n * rb2 + sg * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
 // ---- host side --------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -1054,6 +1094,18 @@ cudaError_t launch_gemm_i2(const int8_t* xq, const uint8_t* w, int64_t rb, const
     case 64: return launch_gemm_bt<64>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ldy, ks, part, ws, limit, skip_producer, st);
     default: return launch_gemm_bt<128>(xq, w, rb, gamma, scale, y, ydt, M, N, K, ldy, ks, part, ws, limit, skip_producer, st);
   }
+}
+
+cudaError_t launch_b1_to_i2(const uint8_t* b1, int64_t N, int64_t K, int64_t rb1, uint8_t* i2, int64_t rb2,
+                            cudaStream_t st) {
+  const int64_t work = N * (rb2 / 16);
+  const int64_t cap = static_cast<int64_t>(device_sms()) * 8;
+  int64_t grid = (work + 255) / 256;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  const cudaError_t e = launch_pdl(b1_to_i2_kernel, static_cast<unsigned>(grid), 256, 0, st, b1, N, K, rb1, i2, rb2);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
 }
 
 cudaError_t launch_t5_to_i2(const uint8_t* t5, int64_t N, int64_t K, int64_t rb5, uint8_t* i2, int64_t rb2,

@@ -423,6 +423,32 @@ quant_act_fast_n<8>(e, s_tok[m], c127, q);
   }
 }
 
+// 1-bit activation layout, one-pass prologue: lane pair (2t, 2t + 1) holds the
+// 16-code groups e and e + 1 (e even), the two halves of packed word e >> 1
+// (P: the group's codes, four per word).  Each lane builds, for the activation
+// words i of the word, its two bytes (codes i and 8 + i of its half: bytes 2hb
+// and 2hb + 1, hb = e & 1), trades the halves the other lane stores with
+// it, and writes the four words of its plane (words 0-3 for hb = 0, 4-7 for
+// hb = 1).  Every lane of the warp takes part in the exchange; `valid` only
+// gates the store.
+template <int kPB>
+__device__ __forceinline__ void b1_put_half_t(uint8_t* xm, const uint32_t (&P)[4], uint32_t e, bool valid) {
+  // hh[t]: own bytes of words 2t (low half) and 2t + 1 (high half)
+  const uint32_t hh[4] = {__byte_perm(P[0], P[2], 0x5140), __byte_perm(P[0], P[2], 0x7362),
+                          __byte_perm(P[1], P[3], 0x5140), __byte_perm(P[1], P[3], 0x7362)};
+  const uint32_t hb = e & 1u;
+  const uint32_t oA = hb ? hh[2] : hh[0], oB = hb ? hh[3] : hh[1];  // kept: this lane's words
+  const uint32_t sA = hb ? hh[0] : hh[2], sB = hb ? hh[1] : hh[3];  // sent: the other lane's words
+  const uint32_t rA = __shfl_xor_sync(0xffffffffu, sA, 1), rB = __shfl_xor_sync(0xffffffffu, sB, 1);
+  const uint32_t loA = hb ? rA : oA, hiA = hb ? oA : rA, loB = hb ? rB : oB, hiB = hb ? oB : rB;
+  if (valid) {
+    const uint32_t g = e >> 1, s = g >> 2, w = g & 3u;
+    *reinterpret_cast<uint4*>(xm + (4 * w + 2 * (s & 1u) + hb) * kPB + (s >> 1) * 16) =
+        make_uint4(__byte_perm(loA, hiA, 0x5410), __byte_perm(loA, hiA, 0x7632), __byte_perm(loB, hiB, 0x5410),
+                   __byte_perm(loB, hiB, 0x7632));
+  }
+}
+
 // ---------------------------------------------------------------------------
 // 2-bit decode GEMV, lean form (rows of at most 2 kI2Plane bytes).  A work
 // item is one 64-segment (1 KB) block of a row; lane L takes the segments
@@ -448,11 +474,25 @@ __host__ __device__ inline int64_t gemv_i2_smem_bytes(int mt) {
   return int64_t{8} * kI2Plane * mt + int64_t{4} * mt * kGemvTileRows;
 }
 
-template <int MT, int XDT>
+// The same kernel serves the 1-bit format (FMT = BL_PACK_B1, rows of at most
+// kI2Plane bytes): a 16-byte segment then holds 128 weights, bit i of byte j
+// of a packed word being weight 8 j + i of its 32.  The token's codes sit in
+// 16 planes of kI2Plane / 2 bytes, plane 4w + 2h + p holding, for the segments
+// s with s mod 2 = h, four activation words of packed word w at (s >> 1) * 16:
+// word i (i = 4p .. 4p + 3) has in byte j the code of weight 8 j + i, so that
+// the mask w & (0x01010101 << i) and one dp4a collect 2^i times the sum of the
+// codes over the +1 weights among weights i, 8 + i, 16 + i, 24 + i.  Eight
+// accumulators per token, 2^i off exactly at the end of the item; with S the
+// sum over the +1 weights and X the sum of the token's codes the product is
+// 2 S - X.
+template <int FMT, int MT, int XDT>
 __global__ void __launch_bounds__(kGemvThreads, 1)
     gemv_i2_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
                    int64_t N, int64_t K, const void* __restrict__ x, float* __restrict__ scale,
                    void* __restrict__ y, int ydt, int write_scale, const RowGroups rg) {
+  constexpr bool kB1 = FMT == BL_PACK_B1;
+  constexpr int kNP = kB1 ? 16 : 8;                   // activation planes per token
+  constexpr int kPB = kB1 ? kI2Plane / 2 : kI2Plane;  // bytes per plane
   const int64_t G = gridDim.x, b = blockIdx.x;
   const int64_t per = N / G, extra = N % G;
   const int64_t row0 = b * per + (b < extra ? b : extra);
@@ -466,7 +506,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   }
   pdl_wait(packed, gamma, x, scale, y);
   extern __shared__ __align__(16) uint8_t smem[];
-  uint8_t* xs = smem;                                           // [MT][8][kI2Plane]
+  uint8_t* xs = smem;                                           // [MT][kNP][kPB]
   int* racc = reinterpret_cast<int*>(smem + MT * 8 * kI2Plane);  // [MT][kGemvTileRows]
   __shared__ float red_f[MT][kGemvWarps];
   __shared__ int red_i[MT][kGemvWarps];
@@ -564,8 +604,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     int part = 0;
 #pragma unroll
     for (int u = 0; u < 3; ++u) {
-      const uint32_t g = threadIdx.x + kGemvThreads * u;
-      if (g >= 4 * segs) break;
+      const uint32_t g = threadIdx.x + kGemvThreads * u;  // 16 codes: 16 g .. 16 g + 15
+      if (!kB1 && g >= 4 * segs) break;  // (1-bit: every lane goes on, for the pair exchange)
       uint32_t P[4];
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {  // eight codes at a time
@@ -586,8 +626,12 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
         P[2 * hh] = pack4(q);
         P[2 * hh + 1] = pack4(q + 4);
       }
-      const uint32_t s = g >> 2, w = g & 3;
-      *reinterpret_cast<uint4*>(xs + (2 * w + (s & 1)) * kI2Plane + (s >> 1) * 16) = i2_slot(P[0], P[1], P[2], P[3]);
+      if constexpr (kB1) {
+        b1_put_half_t<kPB>(xs, P, g, g < 8 * segs);
+      } else {
+        const uint32_t s = g >> 2, w = g & 3;
+        *reinterpret_cast<uint4*>(xs + (2 * w + (s & 1)) * kI2Plane + (s >> 1) * 16) = i2_slot(P[0], P[1], P[2], P[3]);
+      }
     }
     part = __reduce_add_sync(0xffffffffu, part);
     if (lane == 0) red_i[0][warp] = part;
@@ -626,8 +670,48 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   #pragma unroll
     for (int m = 0; m < MT; ++m) {
       int part = 0;
-      uint8_t* xm = xs + m * 8 * kI2Plane;
+      uint8_t* xm = xs + m * kNP * kPB;
       const float c127 = (XDT == BL_I8) ? 0.0f : __fdiv_rn(127.0f, s_tok[m]);
+      if constexpr (kB1) {
+        for (uint32_t g = threadIdx.x; g < 4 * segs; g += blockDim.x) {  // one packed word's 32 codes
+          const int64_t k0 = 32 * static_cast<int64_t>(g);
+          int q[32];
+  #pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int64_t kh = k0 + 8 * h;
+            if (kh + 8 <= K && (K % 8) == 0) {
+              if constexpr (XDT == BL_I8) {
+                const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(static_cast<const int8_t*>(x) + m * K + kh));
+  #pragma unroll
+                for (int j = 0; j < 8; ++j) q[8 * h + j] = static_cast<int8_t>((j < 4 ? raw.x : raw.y) >> (8 * (j & 3)));
+              } else {
+                float e[8];
+                load8_aligned<XDT>(x, m * K + kh, e);
+                quant_act_fast_n<8>(e, s_tok[m], c127, q + 8 * h);
+              }
+            } else {
+  #pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int64_t k = kh + j;
+                q[8 * h + j] = k >= K ? 0
+                               : (XDT == BL_I8) ? static_cast<int>(static_cast<const int8_t*>(x)[m * K + k])
+                                                : quant_act_fast(load_x<XDT>(x, m * K + k), s_tok[m], c127);
+              }
+            }
+          }
+          uint32_t X[8];
+  #pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            int qq[4] = {q[i], q[8 + i], q[16 + i], q[24 + i]};
+            X[i] = pack4(qq);
+            part += qq[0] + qq[1] + qq[2] + qq[3];
+          }
+          const uint32_t s = g >> 2, w = g & 3;
+          uint8_t* dst = xm + (4 * w + 2 * (s & 1)) * kPB + (s >> 1) * 16;
+          *reinterpret_cast<uint4*>(dst) = make_uint4(X[0], X[1], X[2], X[3]);
+          *reinterpret_cast<uint4*>(dst + kPB) = make_uint4(X[4], X[5], X[6], X[7]);
+        }
+      } else {
       for (uint32_t g = threadIdx.x; g < 4 * segs; g += blockDim.x) {  // one packed word's 16 codes
         const int64_t k0 = 16 * static_cast<int64_t>(g);
         const bool full = k0 + 16 <= K && (K % 16) == 0;
@@ -665,6 +749,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
         const uint32_t s = g >> 2, w = g & 3;
         *reinterpret_cast<uint4*>(xm + (2 * w + (s & 1)) * kI2Plane + (s >> 1) * 16) = i2_slot(P[0], P[1], P[2], P[3]);
       }
+      }
       part = __reduce_add_sync(0xffffffffu, part);
       if (lane == 0) red_i[m][warp] = part;
     }
@@ -697,6 +782,43 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
 #pragma unroll
       for (int d = 0; d < kI2Batch; ++d) {
         if (c_row >= nr) break;
+        if constexpr (kB1) {
+          int ab[8][MT];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int m = 0; m < MT; ++m) ab[i][m] = 0;
+          const uint8_t* xb = xl + c_blk * 512;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t wd[4] = {bf[d][h].x, bf[d][h].y, bf[d][h].z, bf[d][h].w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+#pragma unroll
+              for (int m = 0; m < MT; ++m) {
+                const uint8_t* xp = xb + (m * kNP + 4 * w + 2 * h) * kPB;
+                const uint4 X0 = *reinterpret_cast<const uint4*>(xp);
+                const uint4 X1 = *reinterpret_cast<const uint4*>(xp + kPB);
+                ab[0][m] = dp4a_us(wd[w] & 0x01010101u, X0.x, ab[0][m]);
+                ab[1][m] = dp4a_us(wd[w] & 0x02020202u, X0.y, ab[1][m]);
+                ab[2][m] = dp4a_us(wd[w] & 0x04040404u, X0.z, ab[2][m]);
+                ab[3][m] = dp4a_us(wd[w] & 0x08080808u, X0.w, ab[3][m]);
+                ab[4][m] = dp4a_us(wd[w] & 0x10101010u, X1.x, ab[4][m]);
+                ab[5][m] = dp4a_us(wd[w] & 0x20202020u, X1.y, ab[5][m]);
+                ab[6][m] = dp4a_us(wd[w] & 0x40404040u, X1.z, ab[6][m]);
+                ab[7][m] = dp4a_us(wd[w] & 0x80808080u, X1.w, ab[7][m]);
+              }
+            }
+          }
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            int v = ab[0][m];
+#pragma unroll
+            for (int i = 1; i < 8; ++i) v += ab[i][m] >> i;
+            const int t = __reduce_add_sync(0xffffffffu, v);
+            if (lane == 0) atomicAdd(racc + m * kGemvTileRows + c_row, t);
+          }
+        } else {
         int a0[MT], a1[MT], a2[MT], a3[MT];
 #pragma unroll
         for (int m = 0; m < MT; ++m) a0[m] = a1[m] = a2[m] = a3[m] = 0;
@@ -724,6 +846,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
           const int t = __reduce_add_sync(0xffffffffu, v);
           if (lane == 0) atomicAdd(racc + m * kGemvTileRows + c_row, t);
         }
+        }
         c_blk += dr;
         c_row += dq;
         if (c_blk >= nb) {
@@ -747,7 +870,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     for (int r = threadIdx.x; r < static_cast<int>(nr); r += blockDim.x) {
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
-        const int a = racc[m * kGemvTileRows + r] - corr[m];
+        const int a = (kB1 ? 2 : 1) * racc[m * kGemvTileRows + r] - corr[m];
         racc[m * kGemvTileRows + r] = 0;
         const int64_t o = m * N + row0 + t0 + r;
         const float cf = rg.n == 1 ? cfac[m] : dequant_factor(sh_gam[row_group(rg, row0 + t0 + r)], s_tok[m]);
@@ -1263,11 +1386,11 @@ static cudaError_t launch_gemv_t(const uint8_t* packed, int64_t rowbytes, const 
   return cudaGetLastError();
 }
 
-template <int MT, int XDT>
+template <int FMT, int MT, int XDT>
 static cudaError_t launch_gemv_i2_t(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N,
                                     int64_t K, const void* x, float* scale, void* y, int ydt, int write_scale,
                                     const RowGroups& rg, cudaStream_t st) {
-  auto kern = gemv_i2_kernel<MT, XDT>;
+  auto kern = gemv_i2_kernel<FMT, MT, XDT>;
   const size_t smem = static_cast<size_t>(gemv_i2_smem_bytes(MT));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -1278,16 +1401,25 @@ static cudaError_t launch_gemv_i2_t(const uint8_t* packed, int64_t rowbytes, con
   return cudaGetLastError();
 }
 
-template <int XDT>
+template <int FMT, int XDT>
 static cudaError_t launch_gemv_i2_mt(int mt, const uint8_t* packed, int64_t rowbytes, const float* gamma,
                                      int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
                                      int write_scale, const RowGroups& rg, cudaStream_t st) {
   switch (mt) {
-    case 1: return launch_gemv_i2_t<1, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
-    case 2: return launch_gemv_i2_t<2, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
-    case 3: return launch_gemv_i2_t<3, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
-    default: return launch_gemv_i2_t<4, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
+    case 1: return launch_gemv_i2_t<FMT, 1, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
+    case 2: return launch_gemv_i2_t<FMT, 2, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
+    case 3: return launch_gemv_i2_t<FMT, 3, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
+    default: return launch_gemv_i2_t<FMT, 4, XDT>(packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
   }
+}
+
+template <int XDT>
+static cudaError_t launch_gemv_lean(int fmt, int mt, const uint8_t* packed, int64_t rowbytes, const float* gamma,
+                                    int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
+                                    int write_scale, const RowGroups& rg, cudaStream_t st) {
+  if (fmt == BL_PACK_B1)
+    return launch_gemv_i2_mt<BL_PACK_B1, XDT>(mt, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
+  return launch_gemv_i2_mt<BL_PACK_I2, XDT>(mt, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
 }
 
 // The multi-token column-stationary kernel: 2-bit rows of at most
@@ -1367,12 +1499,16 @@ static cudaError_t launch_gemv_mt(int mt, const uint8_t* packed, int64_t rowbyte
 cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int64_t N, int64_t K,
                         const void* x, int xdt, float* scale, int64_t M, void* y, int ydt,
                         const RowGroups& rg, cudaStream_t st) {
-  const int64_t rowbytes = (fmt == BL_PACK_I2) ? ((K + 3) / 4 + 15) / 16 * 16 : ((K + 4) / 5 + 15) / 16 * 16;
+  const int per = (fmt == BL_PACK_I2) ? 4 : (fmt == BL_PACK_T5 ? 5 : 8);
+  const int64_t rowbytes = ((K + per - 1) / per + 15) / 16 * 16;
   const int mt_max = gemv_max_tokens(fmt, rowbytes);
   if (mt_max < 1) return cudaErrorInvalidValue;
-  // 2-bit rows of up to 2 kI2Plane bytes take the lean kernel (its shared
-  // memory, 8 planes per token, fits kGemvMaxTokens tokens within the budget)
-  const bool lean = fmt == BL_PACK_I2 && rowbytes <= 2 * kI2Plane;
+  // 2-bit rows of up to 2 kI2Plane bytes and 1-bit rows of up to kI2Plane
+  // bytes take the lean kernel (its shared memory, 8 x kI2Plane bytes per
+  // token, fits kGemvMaxTokens tokens within the budget); longer 1-bit rows
+  // are not served here (the caller transcodes them to 2 bits)
+  const bool lean = (fmt == BL_PACK_I2 && rowbytes <= 2 * kI2Plane) || (fmt == BL_PACK_B1 && rowbytes <= kI2Plane);
+  if (fmt == BL_PACK_B1 && !lean) return cudaErrorInvalidValue;
   const int esz = (xdt == BL_F32) ? 4 : (xdt == BL_BF16 ? 2 : 1);
   const int ysz = (ydt == BL_BF16) ? 2 : 4;
   for (int64_t m0 = 0; m0 < M; m0 += mt_max) {
@@ -1390,9 +1526,9 @@ cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int6
       else if (xdt == BL_BF16) e = launch_gemv_t5_t<BL_BF16>(packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, rg, st);
       else e = launch_gemv_t5_t<BL_I8>(packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, rg, st);
     } else if (lean) {
-      if (xdt == BL_F32) e = launch_gemv_i2_mt<BL_F32>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, rg, st);
-      else if (xdt == BL_BF16) e = launch_gemv_i2_mt<BL_BF16>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, rg, st);
-      else e = launch_gemv_i2_mt<BL_I8>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, rg, st);
+      if (xdt == BL_F32) e = launch_gemv_lean<BL_F32>(fmt, mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, rg, st);
+      else if (xdt == BL_BF16) e = launch_gemv_lean<BL_BF16>(fmt, mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, rg, st);
+      else e = launch_gemv_lean<BL_I8>(fmt, mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 0, rg, st);
     } else if (fmt == BL_PACK_I2) {
       if (xdt == BL_F32) e = launch_gemv_mt<BL_PACK_I2, BL_F32>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, rg, st);
       else if (xdt == BL_BF16) e = launch_gemv_mt<BL_PACK_I2, BL_BF16>(mt, packed, rowbytes, gamma, N, K, xm, sm, ym, ydt, 1, rg, st);

@@ -37,8 +37,14 @@ constexpr int64_t kGemvSmemBudget = 200 * 1024;
 constexpr int kGemvMaxTokens = 4;
 
 // ws: a workspace whose header ticket is zero; partial sums follow the header.
+// alpha: when given, the mean of the weights in the same order (the 1-bit
+// variant; then the partial sums take 2 C doubles).
 cudaError_t launch_absmean(const void* W, int wdt, int64_t N, int64_t K, void* ws, float* gamma,
-                           cudaStream_t st);
+                           cudaStream_t st, float* alpha = nullptr);
+cudaError_t launch_binarize_pack(const void* W, int wdt, int64_t N, int64_t K, const float* alpha, uint8_t* packed,
+                                 int8_t* codes, int64_t rowbytes, cudaStream_t st);
+cudaError_t launch_b1_to_i2(const uint8_t* b1, int64_t N, int64_t K, int64_t rb1, uint8_t* i2, int64_t rb2,
+                            cudaStream_t st);
 // ws: a workspace header for device flags, or nullptr (then a bounded wait
 // that runs out goes unreported).
 cudaError_t launch_ternarize_pack(const void* W, int wdt, int64_t N, int64_t K, const float* gamma,

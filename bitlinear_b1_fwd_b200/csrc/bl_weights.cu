@@ -97,12 +97,16 @@ __device__ __forceinline__ void absmean_finish(const double* __restrict__ partia
 // with 4 CTAs per SM, 128 KB per SM can be in flight.
 constexpr int kAbsCtasPerSm = 4;
 
-template <int WDT>
+// With MEAN (the 1-bit variant) the kernel also adds the signed weights in the
+// same order, into partials[C + c], and the last CTA writes alpha = fp32(S / T)
+// beside gamma (= beta).
+template <int WDT, bool MEAN>
 __global__ void __launch_bounds__(kLanes, kAbsCtasPerSm)
     absmean_kernel(const void* __restrict__ W, int64_t T, int64_t C, int lgR, double* __restrict__ partials,
-                   WsHeader* __restrict__ hdr, float* __restrict__ gamma) {
-  pdl_enter(W, partials, hdr, gamma);
-  __shared__ double lsum[2][kLanes];
+                   WsHeader* __restrict__ hdr, float* __restrict__ gamma, float* __restrict__ alpha) {
+  pdl_enter(W, partials, hdr, gamma, alpha);
+  constexpr int NS = MEAN ? 2 : 1;  // sums per lane
+  __shared__ double lsum[2][NS][kLanes];
   __shared__ double p[kLanes];
   __shared__ bool last;
   const int l = threadIdx.x, warp = l >> 5, L = l & 31;
@@ -122,26 +126,33 @@ __global__ void __launch_bounds__(kLanes, kAbsCtasPerSm)
         for (int j = 0; j < 8; ++j) v[i][j] = (e0 + j < T) ? load_elem<WDT>(W, e0 + j) : 0.0f;
       }
     }
-    double acc = 0.0;  // +0.0 for elements past T leaves the sum unchanged
+    double acc = 0.0, acc_s = 0.0;  // +0.0 for elements past T leaves the sums unchanged
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc = __dadd_rn(acc, static_cast<double>(fabsf(v[i][j])));
-    double* ls = lsum[k & 1];
-    ls[l] = acc;
+      for (int j = 0; j < 8; ++j) {
+        acc = __dadd_rn(acc, static_cast<double>(fabsf(v[i][j])));
+        if constexpr (MEAN) acc_s = __dadd_rn(acc_s, static_cast<double>(v[i][j]));
+      }
+    lsum[k & 1][0][l] = acc;
+    if constexpr (MEAN) lsum[k & 1][NS - 1][l] = acc_s;
     __syncthreads();
     if (warp == (k & 7)) {
-      double q[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) q[u] = ls[L + 32 * u];
+      for (int z = 0; z < NS; ++z) {
+        const double* ls = lsum[k & 1][z];
+        double q[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) q[u] = __dadd_rn(q[u], q[u + 4]);  // level 128
-      q[0] = __dadd_rn(q[0], q[2]);                                   // level 64
-      q[1] = __dadd_rn(q[1], q[3]);
-      double t = __dadd_rn(q[0], q[1]);                               // level 32
+        for (int u = 0; u < 8; ++u) q[u] = ls[L + 32 * u];
 #pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) t = __dadd_rn(t, __shfl_down_sync(0xffffffffu, t, o));
-      if (L == 0) partials[c] = t;
+        for (int u = 0; u < 4; ++u) q[u] = __dadd_rn(q[u], q[u + 4]);  // level 128
+        q[0] = __dadd_rn(q[0], q[2]);                                   // level 64
+        q[1] = __dadd_rn(q[1], q[3]);
+        double t = __dadd_rn(q[0], q[1]);                               // level 32
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) t = __dadd_rn(t, __shfl_down_sync(0xffffffffu, t, o));
+        if (L == 0) partials[z * C + c] = t;
+      }
     }
   }
   __threadfence();
@@ -154,6 +165,10 @@ __global__ void __launch_bounds__(kLanes, kAbsCtasPerSm)
   if (!last) return;
   __threadfence();
   absmean_finish(partials, C, lgR, T, p, hdr, gamma);
+  if constexpr (MEAN) {
+    __syncthreads();  // warp 0 has read p
+    absmean_finish(partials + C, C, lgR, T, p, hdr, alpha);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -356,6 +371,76 @@ __global__ void __launch_bounds__(256, kTernCtasPerSm)
   }
 }
 
+// ---------------------------------------------------------------------------
+// 1-bit binarize and pack ("QAT and BitNet: A Deep Dive into 1-bit and
+// 1.58-bit Quantization-Aware Training", "The BitLinear Recipe" step 2): a
+// weight above alpha is +1, any other -1.  Bit i of byte j of a row holds
+// weight 8 j + i (1 for +1); bits past K are 0.  One thread writes one 16-byte
+// segment (128 weights) of a packed row, one 32-bit word (32 weights) at a
+// time, with 16-byte loads of W when the row allows them; segments are walked
+// from the end of W backwards (the scale kernel just streamed W front to back).
+// ---------------------------------------------------------------------------
+template <int WDT>
+__global__ void __launch_bounds__(256)
+    binarize_pack_kernel(const void* __restrict__ W, int64_t N, int64_t K, const float* __restrict__ alpha,
+                         uint8_t* __restrict__ packed, int8_t* __restrict__ codes, int64_t rowbytes, bool vec_ok) {
+  pdl_enter(W, alpha, packed, codes);
+  __shared__ float sh_alpha;  // once per CTA
+  if (threadIdx.x == 0) sh_alpha = __ldcg(alpha);
+  __syncthreads();
+  const float a = sh_alpha;
+  const int64_t segs = rowbytes / 16;
+  const int64_t total = N * segs;
+  for (int64_t it = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; it < total;
+       it += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t gid = total - 1 - it;
+    const int64_t n = gid / segs;
+    const int64_t sg = gid - n * segs;
+    uint32_t out[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int64_t k0 = sg * 128 + 32 * w;
+      const int64_t base = n * K + k0;
+      uint32_t word = 0;
+      if (vec_ok && k0 + 32 <= K) {
+        float v[32];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) load8_aligned<WDT>(W, base + 8 * g, v + 8 * g);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) word |= (v[i] > a ? 1u : 0u) << i;
+        if (codes != nullptr) {
+          uint32_t cw[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            uint32_t c = 0;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) c |= (v[4 * j + b] > a ? 0x01u : 0xffu) << (8 * b);
+            cw[j] = c;
+          }
+          if ((K % 16) == 0) {
+            uint4* dst = reinterpret_cast<uint4*>(codes + base);
+            dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) codes[base + i] = static_cast<int8_t>(v[i] > a ? 1 : -1);
+          }
+        }
+      } else {
+        for (int i = 0; i < 32; ++i) {
+          if (k0 + i >= K) break;
+          const bool plus = load_elem<WDT>(W, base + i) > a;
+          word |= (plus ? 1u : 0u) << i;
+          if (codes != nullptr) codes[base + i] = static_cast<int8_t>(plus ? 1 : -1);
+        }
+      }
+      out[w] = word;
+    }
+    if (packed != nullptr)
+      *reinterpret_cast<uint4*>(packed + n * rowbytes + sg * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
 // Pack int8 codes (same segment mapping).  A code outside {-1, 0, 1} packs as
 // weight 0 and raises the bad-code flag.
 template <int FMT>
@@ -363,7 +448,7 @@ __global__ void __launch_bounds__(256)
     pack_kernel(const int8_t* __restrict__ codes, int64_t N, int64_t K, uint8_t* __restrict__ packed,
                 int64_t rowbytes, void* ws) {
   pdl_enter(codes, packed, ws);
-  constexpr int PER = (FMT == BL_PACK_I2) ? 4 : 5;
+  constexpr int PER = (FMT == BL_PACK_I2) ? 4 : (FMT == BL_PACK_T5 ? 5 : 8);
   constexpr int WPS = 16 * PER;
   const int64_t segs = rowbytes / 16;
   const int64_t total = N * segs;
@@ -383,9 +468,14 @@ __global__ void __launch_bounds__(256)
         uint32_t byte = 0;
 #pragma unroll
         for (int ii = 0; ii < PER; ++ii) {
-          const int i = (FMT == BL_PACK_I2) ? ii : PER - 1 - ii;
-          const int kk = (FMT == BL_PACK_I2) ? 16 * w + 4 * b + i : 20 * w + 5 * b + i;
+          const int i = (FMT == BL_PACK_T5) ? PER - 1 - ii : ii;
+          const int kk = 4 * PER * w + PER * b + i;
           int c = (k0 + kk < K) ? static_cast<int>(__ldcg(src + kk)) : 0;
+          if constexpr (FMT == BL_PACK_B1) {  // {-1, +1}; pad bits 0
+            if (k0 + kk < K && c != 1 && c != -1) bad = true;
+            byte |= (c == 1 ? 1u : 0u) << i;
+            continue;
+          }
           if (c < -1 || c > 1) {
             bad = true;
             c = 0;
@@ -427,7 +517,7 @@ static int grid_for(int64_t work, int threads, int per_sm_ctas) {
 }
 
 cudaError_t launch_absmean(const void* W, int wdt, int64_t N, int64_t K, void* ws, float* gamma,
-                           cudaStream_t st) {
+                           cudaStream_t st, float* alpha) {
   const int64_t T = N * K;
   const int64_t C = (T + kChunk - 1) / kChunk;
   int lgP = 0;
@@ -439,11 +529,15 @@ cudaError_t launch_absmean(const void* W, int wdt, int64_t N, int64_t K, void* w
   // persistent streaming grid: kAbsCtasPerSm CTAs per SM (at most one per chunk)
   const int64_t cap = static_cast<int64_t>(device_sms()) * kAbsCtasPerSm;
   const int64_t grid = C < cap ? C : cap;
+  const unsigned g = static_cast<unsigned>(grid);
+  if (alpha != nullptr) {
+    if (wdt == BL_F32)
+      return launch_pdl(absmean_kernel<BL_F32, true>, g, kLanes, 0, st, W, T, C, lgR, partials, hdr, gamma, alpha);
+    return launch_pdl(absmean_kernel<BL_BF16, true>, g, kLanes, 0, st, W, T, C, lgR, partials, hdr, gamma, alpha);
+  }
   if (wdt == BL_F32)
-    return launch_pdl(absmean_kernel<BL_F32>, static_cast<unsigned>(grid), kLanes, 0, st, W, T, C, lgR, partials,
-                      hdr, gamma);
-  return launch_pdl(absmean_kernel<BL_BF16>, static_cast<unsigned>(grid), kLanes, 0, st, W, T, C, lgR, partials, hdr,
-                    gamma);
+    return launch_pdl(absmean_kernel<BL_F32, false>, g, kLanes, 0, st, W, T, C, lgR, partials, hdr, gamma, alpha);
+  return launch_pdl(absmean_kernel<BL_BF16, false>, g, kLanes, 0, st, W, T, C, lgR, partials, hdr, gamma, alpha);
 }
 
 cudaError_t launch_ternarize_pack(const void* W, int wdt, int64_t N, int64_t K, const float* gamma,
@@ -481,7 +575,18 @@ cudaError_t launch_pack(const int8_t* codes, int64_t N, int64_t K, int fmt, uint
   const int64_t work = N * (rowbytes / 16);
   const int grid = grid_for(work, 256, 8);
   if (fmt == BL_PACK_I2) return launch_pdl(pack_kernel<BL_PACK_I2>, grid, 256, 0, st, codes, N, K, packed, rowbytes, ws);
+  if (fmt == BL_PACK_B1) return launch_pdl(pack_kernel<BL_PACK_B1>, grid, 256, 0, st, codes, N, K, packed, rowbytes, ws);
   return launch_pdl(pack_kernel<BL_PACK_T5>, grid, 256, 0, st, codes, N, K, packed, rowbytes, ws);
+}
+
+cudaError_t launch_binarize_pack(const void* W, int wdt, int64_t N, int64_t K, const float* alpha, uint8_t* packed,
+                                 int8_t* codes, int64_t rowbytes, cudaStream_t st) {
+  const bool vec_ok = (K % 8) == 0;
+  const int64_t work = N * (rowbytes / 16);
+  const int grid = grid_for(work, 256, 4);
+  if (wdt == BL_F32)
+    return launch_pdl(binarize_pack_kernel<BL_F32>, grid, 256, 0, st, W, N, K, alpha, packed, codes, rowbytes, vec_ok);
+  return launch_pdl(binarize_pack_kernel<BL_BF16>, grid, 256, 0, st, W, N, K, alpha, packed, codes, rowbytes, vec_ok);
 }
 
 }  // namespace bl

@@ -85,7 +85,9 @@ typedef enum { BL_F32 = 0, BL_BF16 = 1, BL_I8 = 2, BL_I32 = 3 } bl_dtype;
 
 typedef enum {
   BL_PACK_I2 = 0, /* 2 bits per weight, 4 weights per byte */
-  BL_PACK_T5 = 1  /* 5 trits per byte in base 3 (3^5 = 243 <= 256) */
+  BL_PACK_T5 = 1, /* 5 trits per byte in base 3 (3^5 = 243 <= 256) */
+  BL_PACK_B1 = 2  /* 1-bit BitNet: 1 bit per weight, 8 per byte; bit i of byte j
+                     is weight 8j + i, 1 for +1 and 0 for -1, pad bits 0 */
 } bl_pack;
 
 /* Bytes at the start of every workspace that hold the device status flags.
@@ -93,7 +95,7 @@ typedef enum {
  * or cudaMemset); the library keeps them consistent afterwards. */
 #define BL_WS_HEADER_BYTES 256
 
-/* Row stride of a packed matrix: ceil(K / per) bytes (per = 4 or 5) rounded up
+/* Row stride of a packed matrix: ceil(K / per) bytes (per = 4, 5 or 8) rounded up
  * to a multiple of 16.  [P3] §4.1 (70B x 0.25 B = 17.5 GB; 5 per byte ~14 GB).
  * Returns -1 for K < 1 or an unknown format. */
 BL_API int64_t bitlinear_packed_row_bytes(int64_t K, int fmt);
@@ -104,7 +106,8 @@ BL_API size_t bitlinear_quantize_weights_workspace_bytes(int64_t N, int64_t K);
 
 /* Workspace bytes needed by bitlinear_forward for these sizes and formats (the
  * header, plus x_q when activations are quantized ahead of the tensor-core
- * path, plus a 2-bit copy of base-3 weights for that path, plus the INT32
+ * path, plus a 2-bit copy of base-3 or 1-bit weights for that path (and of
+ * 1-bit rows longer than 4096 bytes for any M), plus the INT32
  * partial sums when a layer with few tokens (5..128) is split along K so
  * that it spreads over every SM; the split depends on the device's SM
  * count, so query on the device that runs the call). */
@@ -164,10 +167,31 @@ BL_API bl_status bitlinear_ternarize_pack(const void *W, int wdt, int64_t N, int
                                    const float *gamma, float eps, int fmt, uint8_t *packed,
                                    int8_t *codes, void *stream);
 
+/* 1-bit BitNet weights (the 1-bit variant of steps 1-3).  [P5] "The BitLinear
+ * Recipe" steps 2 and 4: alpha = mean of the weights, a weight above alpha
+ * becomes +1 and any other -1 (a weight equal to alpha gives -1, a reading:
+ * the pages do not say), beta = mean |W| rescales the output.  alpha and beta
+ * are fp64 sums in the same fixed order as gamma's (for alpha the terms are
+ * w), divided by N K and rounded to fp32; beta equals the gamma of
+ * bitlinear_absmean.  The forward then takes fmt = BL_PACK_B1 with beta in
+ * place of gamma.
+ *   W       [N, K] fp32 or bf16.
+ *   packed  [N, bitlinear_packed_row_bytes(K, BL_PACK_B1)] uint8 output, or NULL.
+ *   codes   [N, K] int8 output in {-1, +1}, or NULL (not both NULL).
+ *   beta, alpha  [1] fp32 device outputs.
+ *   ws      at least bitlinear_binarize_weights_workspace_bytes(N, K) (two
+ *           fp64 partial sums per 8192-element chunk). */
+BL_API size_t bitlinear_binarize_weights_workspace_bytes(int64_t N, int64_t K);
+BL_API bl_status bitlinear_binarize_weights(const void *W, int wdt, int64_t N, int64_t K, uint8_t *packed,
+                                         int8_t *codes, float *beta, float *alpha, void *ws, size_t ws_bytes,
+                                         void *stream);
+
 /* Pack int8 codes in {-1, 0, 1} (step 3).  [P3] §2.3, §6.3.
  *   codes  [N, K] int8; packed [N, row_bytes] uint8 output.
  *   ws     at least BL_WS_HEADER_BYTES; a code outside {-1, 0, 1} is packed
- *          as weight 0 and sets BL_ERR_BAD_CODE in the workspace flag. */
+ *          as weight 0 and sets BL_ERR_BAD_CODE in the workspace flag.
+ * With fmt = BL_PACK_B1 the codes must be -1 or +1; any other code packs as -1
+ * and sets BL_ERR_BAD_CODE. */
 BL_API bl_status bitlinear_pack(const int8_t *codes, int64_t N, int64_t K, int fmt, uint8_t *packed,
                          void *ws, size_t ws_bytes, void *stream);
 
@@ -196,8 +220,10 @@ BL_API bl_status bitlinear_layernorm_quantize_acts(const void *x, int xdt, const
 
 /* BitLinear forward, y = dequant(x_q . W_q^T) (steps 4-6).
  * [P3] §4.2 (add / subtract / skip), §3.3 (INT32 accumulation), §5.3.
- *   packed  [N, row_bytes] from bitlinear_quantize_weights / bitlinear_pack.
- *   gamma   [1] fp32 device pointer.
+ *   packed  [N, row_bytes] from bitlinear_quantize_weights / bitlinear_pack
+ *           (fmt BL_PACK_I2 | BL_PACK_T5), or from bitlinear_binarize_weights
+ *           (fmt BL_PACK_B1: weights in {-1, +1}).
+ *   gamma   [1] fp32 device pointer (beta for BL_PACK_B1).
  *   x       [M, K]: fp32 or bf16 (quantized inside; `scale` [M] is written),
  *           or int8 x_q (xdt = BL_I8; `scale` [M] is read).
  *   y       [M, N]: ydt = BL_F32 | BL_BF16, or BL_I32 for the raw INT32

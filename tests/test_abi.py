@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(bl):
 
 def test_row_bytes_match_oracle(bl, orc):
     for K in (1, 4, 5, 63, 64, 65, 256, 3200, 8192, 8640, 28672, 1 << 20):
-        for fmt in (0, 1):
+        for fmt in (0, 1, 2):
             assert bl.bitlinear_packed_row_bytes(K, fmt) == orc.packed_row_bytes(K, fmt)
     assert bl.bitlinear_packed_row_bytes(0, 0) == -1
     assert bl.bitlinear_packed_row_bytes(5, 7) == -1
@@ -57,6 +57,18 @@ def test_workspace_sizes(bl):
     assert bl.bitlinear_quantize_weights_workspace_bytes(0, 5) == 0
     assert bl.bitlinear_forward_workspace_bytes(1, 8640, 3200, 0, 1) >= bl.BL_WS_HEADER_BYTES
     assert bl.bitlinear_forward_workspace_bytes(1, 8640, 0, 0, 1) == 0
+
+
+def test_onebit_workspace_sizes(bl):
+    # two fp64 partial sums per 8192-element chunk
+    assert bl.bitlinear_binarize_weights_workspace_bytes(512, 256) == 256 + 256
+    assert bl.bitlinear_binarize_weights_workspace_bytes(8640, 3200) == 256 + (2 * 3375 * 8 + 255) // 256 * 256
+    assert bl.bitlinear_binarize_weights_workspace_bytes(0, 5) == 0
+    # decode of 1-bit rows up to 4096 bytes needs only the header; longer rows a 2-bit copy
+    assert bl.bitlinear_forward_workspace_bytes(1, 8192, 28672, 2, 1) == bl.BL_WS_HEADER_BYTES
+    assert bl.bitlinear_forward_workspace_bytes(1, 300, 40000, 2, 1) == 256 + (300 * 10000 + 255) // 256 * 256
+    # the tensor-core path transcodes 1-bit weights like base-3 ones
+    assert bl.bitlinear_forward_workspace_bytes(64, 256, 1024, 2, 2) == bl.bitlinear_forward_workspace_bytes(64, 256, 1024, 1, 2)
 
 
 def test_status_strings(bl):
@@ -84,6 +96,16 @@ def test_host_validation_without_gpu(bl):
     assert L.bitlinear_quantize_weights(p, 0, 4, 4, 1e-5, 0, null, null, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
     assert L.bitlinear_quantize_weights(odd, 0, 4, 4, 1e-5, 0, p, null, p, p, 4096, null) == bl.BL_ERR_MISALIGNED
     assert L.bitlinear_quantize_weights(p, 0, 4, 4, 1e-5, 0, p, null, p, p, 100, null) == bl.BL_ERR_WORKSPACE_TOO_SMALL
+    # the 1-bit format is not a ternary format
+    assert L.bitlinear_quantize_weights(p, 0, 4, 4, 1e-5, 2, p, null, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_ternarize_pack(p, 0, 4, 4, p, 1e-5, 2, p, null, null) == bl.BL_ERR_INVALID_VALUE
+    # binarize_weights
+    assert L.bitlinear_binarize_weights(p, 0, 4, 4, null, null, p, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_binarize_weights(p, 0, 4, 4, p, null, null, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_binarize_weights(p, 2, 4, 4, p, null, p, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_binarize_weights(p, 0, 0, 4, p, null, p, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_binarize_weights(odd, 0, 4, 4, p, null, p, p, p, 4096, null) == bl.BL_ERR_MISALIGNED
+    assert L.bitlinear_binarize_weights(p, 0, 4, 4, p, null, p, p, p, 100, null) == bl.BL_ERR_WORKSPACE_TOO_SMALL
     # ternarize_pack
     assert L.bitlinear_ternarize_pack(p, 0, 4, 4, null, 1e-5, 0, p, null, null) == bl.BL_ERR_INVALID_VALUE
     assert L.bitlinear_ternarize_pack(p, 0, 4, 4, p, -1.0, 0, p, null, null) == bl.BL_ERR_INVALID_VALUE
@@ -91,7 +113,7 @@ def test_host_validation_without_gpu(bl):
     assert L.bitlinear_pack(p, 4, 4, 0, p, p, 10, null) == bl.BL_ERR_WORKSPACE_TOO_SMALL
     assert L.bitlinear_pack(null, 0, 4, 0, null, null, 0, null) == bl.BL_OK
     assert L.bitlinear_pack(odd, 4, 4, 0, p, p, 4096, null) == bl.BL_ERR_MISALIGNED
-    assert L.bitlinear_pack(p, 4, 4, 2, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_pack(p, 4, 4, 3, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
     assert L.bitlinear_pack(p, 0, 4, 0, p, p, 4096, null) == bl.BL_OK          # empty: nothing to do
     # quantize_acts
     assert L.bitlinear_quantize_acts(p, 2, 4, 4, p, p, null) == bl.BL_ERR_INVALID_VALUE
