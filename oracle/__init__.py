@@ -59,6 +59,10 @@ def lib() -> C.CDLL:
             L.orc_signed_sum.restype = d
             L.orc_binarize_weights.argtypes = [p, i, i64, i64, p, p, p]
             L.orc_binarize_weights.restype = None
+            L.orc_backward_dx.argtypes = [p, i64, i64, p, i, i64, f, p]
+            L.orc_backward_dx.restype = None
+            L.orc_backward_dw.argtypes = [p, i, p, p, f, i64, i64, i64, p]
+            L.orc_backward_dw.restype = None
             L.orc_gamma.argtypes = [p, i, i64, i64]
             L.orc_gamma.restype = f
             L.orc_ternarize.argtypes = [p, i, i64, i64, f, f, p]
@@ -267,6 +271,44 @@ def binarize_weights(W: np.ndarray):
     b = C.c_float()
     lib().orc_binarize_weights(_ptr(W), _dt(W), N, K, C.byref(a), C.byref(b), _ptr(codes))
     return np.float32(a.value), np.float32(b.value), codes
+
+
+# --- STE backward -------------------------------------------------------------------
+
+def backward_dx(codes: np.ndarray, dy: np.ndarray, g: float, parallel: bool = False) -> np.ndarray:
+    """dx [M, K] = gamma * dy [M, N] . W_q [N, K] (fp64 in the fixed chunk order, fp32 out)."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    dy = np.ascontiguousarray(dy)
+    N, K = codes.shape
+    M = dy.shape[0]
+    assert dy.shape == (M, N)
+    dx = np.empty((M, K), np.float32)
+    L = lib()
+    if not parallel or M < 2:
+        L.orc_backward_dx(_ptr(codes), N, K, _ptr(dy), _dt(dy), M, float(g), _ptr(dx))
+        return dx
+    toks = [r for r in np.array_split(np.arange(M), _threads()) if len(r)]
+
+    def run(r):
+        a, b = int(r[0]), int(r[-1]) + 1
+        L.orc_backward_dx(_ptr(codes), N, K, _ptr(dy) + a * N * dy.itemsize, _dt(dy), b - a, float(g),
+                          _ptr(dx) + a * K * 4)
+    with ThreadPoolExecutor(len(toks)) as ex:
+        list(ex.map(run, toks))
+    return dx
+
+
+def backward_dw(dy: np.ndarray, xq: np.ndarray, scale: np.ndarray, g: float) -> np.ndarray:
+    """dW [N, K] = gamma * dy^T . x_deq, x_deq = x_q * s / 127 (fp64 in token order, fp32 out)."""
+    dy = np.ascontiguousarray(dy)
+    xq = np.ascontiguousarray(xq, dtype=np.int8)
+    scale = np.ascontiguousarray(scale, dtype=np.float32)
+    M, N = dy.shape
+    K = xq.shape[1]
+    assert xq.shape == (M, K) and scale.shape == (M,)
+    dw = np.empty((N, K), np.float32)
+    lib().orc_backward_dw(_ptr(dy), _dt(dy), _ptr(xq), _ptr(scale), float(g), M, N, K, _ptr(dw))
+    return dw
 
 
 def f32_to_bf16(v: float) -> int:

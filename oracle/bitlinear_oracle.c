@@ -409,6 +409,67 @@ void orc_binarize_weights(const void *W, int dt, int64_t N, int64_t K,
 }
 
 /* ------------------------------------------------------------------------ */
+/* STE backward of the BitLinear layer (the training side).                 */
+/* [P3] §5.3 (BitLinear: out = F.linear(x_deq, W_eff) * gamma with W_eff =  */
+/* W_ternary + W - W.detach(), the straight-through estimator taking the    */
+/* quantizer as the identity in the backward pass); [P1]/[P5] "How          */
+/* Gradients Flow: Fake Quantization and STE" (forward with the quantized   */
+/* values, backward as if rounding were the identity).                     */
+/* Readings: both quantizers pass the gradient straight through and gamma  */
+/* is a constant of the step (no gradient through mean |W|), so for an     */
+/* upstream gradient dy [M, N]:                                             */
+/*   dx[m][k] = gamma * sum_n dy[m][n] * W_q[n][k]                          */
+/*   dW[n][k] = gamma * sum_m dy[m][n] * x_deq[m][k],                       */
+/*              x_deq[m][k] = x_q[m][k] * s_m / 127 (the forward's codes).  */
+/* Arithmetic: fp64, one rounding per operation, then fp32.  dx: the rows  */
+/* n are taken in chunks of 256 (n in [256 r, 256 r + 256)); within a chunk */
+/* the terms +dy, -dy or nothing (add / subtract / skip) go into a sum from */
+/* 0.0 in row order, and the chunk sums go into S from 0.0 in chunk order; */
+/* dx = fp32(gamma * S).  dW: c_m = s_m / 127, each term is                */
+/* (dy[m][n] * x_q[m][k]) * c_m, added from 0.0 in token order into T;     */
+/* dW = fp32(gamma * T).                                                    */
+/* ------------------------------------------------------------------------ */
+
+#define ORC_DX_CHUNK 256
+
+void orc_backward_dx(const int8_t *codes, int64_t N, int64_t K,
+                     const void *dy, int dydt, int64_t M, float gamma,
+                     float *dx) {
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t k = 0; k < K; ++k) {
+      double S = 0.0;
+      for (int64_t r0 = 0; r0 < N; r0 += ORC_DX_CHUNK) {
+        double P = 0.0;
+        for (int64_t n = r0; n < N && n < r0 + ORC_DX_CHUNK; ++n) {
+          int q = codes[n * K + k];
+          double g = (double)load_f(dy, dydt, m * N + n);
+          if (q == 1)
+            P += g;
+          else if (q == -1)
+            P -= g;
+        }
+        S += P;
+      }
+      dx[m * K + k] = (float)((double)gamma * S);
+    }
+}
+
+void orc_backward_dw(const void *dy, int dydt, const int8_t *xq,
+                     const float *scale, float gamma, int64_t M, int64_t N,
+                     int64_t K, float *dw) {
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) {
+      double T = 0.0;
+      for (int64_t m = 0; m < M; ++m) {
+        double c = (double)scale[m] / 127.0;
+        double t = (double)load_f(dy, dydt, m * N + n) * (double)xq[m * K + k];
+        T += t * c;
+      }
+      dw[n * K + k] = (float)((double)gamma * T);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Pre-norm + step 4: LayerNorm of each token, then per-token absmax INT8.  */
 /* [P5] "The BitLinear Recipe" step 1 (the input is quantized with absmax   */
 /* scaling after LayerNorm, whose output has a stable scale); [P3] §5.5    */
