@@ -60,7 +60,9 @@ KERNEL_SOURCE = {"absmean_kernel": "bl_weights.cu", "ternarize_flat_kernel": "bl
                  "ternarize_pack_kernel": "bl_weights.cu", "gemv_i2_kernel": "bl_gemv.cu",
                  "gemv_kernel": "bl_gemv.cu", "gemv_t5_kernel": "bl_gemv.cu", "gemv_i2_mt_kernel": "bl_gemv.cu", "act_quant_row_kernel": "bl_acts.cu",
                  "act_quant_kernel": "bl_acts.cu", "ln_quant_kernel": "bl_acts.cu", "gemm_i2_2sm_kernel": "bl_gemm_sm100.cu",
-                 "gemm_i2_kernel": "bl_gemm_sm100.cu"}
+                 "gemm_i2_kernel": "bl_gemm_sm100.cu", "b1_to_i2_kernel": "bl_gemm_sm100.cu",
+                 "backward_dx_partial_kernel": "bl_backward.cu", "backward_dx_reduce_kernel": "bl_backward.cu",
+                 "backward_dw_kernel": "bl_backward.cu"}
 
 
 def csrc_digest(kernel: str | None = None) -> str:
@@ -411,7 +413,8 @@ def run_gpu(args, wl, rank, world, local_rank):
     prefill = run_prefill(args, dev, stream, rank_seed, l2) if args.prefill else None
     decode = run_decode(args, dev, stream, rank_seed, l2) if args.decode else None
     sweep = run_sweep(args, dev, stream, l2) if args.sweep else None
-    res = dict(prefill=prefill, decode=decode, sweep=sweep, ms_total=ms_max, per_op_ms=per_op_ms, step_bytes=step_bytes,
+    backward = run_backward(args, dev, stream, rank_seed, l2) if args.decode else None
+    res = dict(prefill=prefill, decode=decode, sweep=sweep, backward=backward, ms_total=ms_max, per_op_ms=per_op_ms, step_bytes=step_bytes,
                layers=layers, ops=ops,
                clocks=sampler.summary(), e2e_ms=e2e_ms, e2e_steps=e2e_steps, h2d=h2d, d2h=d2h,
                rot=rot, l2=l2, launches_per_step=len(layers) * len(ops))
@@ -551,6 +554,65 @@ def run_decode(args, dev, stream, rank_seed, l2):
                 del copies, p0
             out[f"{key}_{['2bit', 'base3', '1bit'][fmt]}"] = dict(desc=desc, rows=rows)
     return out
+
+
+def run_backward(args, dev, stream, rank_seed, l2):
+    """STE backward for one token on the 3B decode layers (2-bit): dx reads the
+    packed weights (plus dy) and writes dx; dW reads dy and x_q and writes N K
+    fp32.  Each call alone in a graph of back-to-back launches, packed copies
+    and dW outputs rotated past 4x L2; GB/s of the algorithmic bytes."""
+    import torch
+
+    from bitlinear_b1_fwd_b200 import binding as B
+
+    peak, kind = measured_peaks()
+    wl = WORKLOADS["3b_decode"]
+    g = torch.Generator(device=dev)
+    out = []
+    for i, (N, K) in enumerate(wl["layers"]):
+        g.manual_seed(3000 + 100 * i + rank_seed)
+        W = torch.randn(N, K, generator=g, device=dev) * wl["sigma"]
+        rb = B.bitlinear_packed_row_bytes(K, 0)
+        p0 = torch.empty((N, rb), dtype=torch.uint8, device=dev)
+        gamma = torch.empty(1, dtype=torch.float32, device=dev)
+        ws = torch.zeros(B.bitlinear_quantize_weights_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+        with torch.cuda.stream(stream):
+            B.bitlinear_quantize_weights(W, 1e-5, 0, p0, None, gamma, ws, stream)
+        stream.synchronize()
+        del W
+        rot = max(2, -(-4 * l2 // (N * rb)))
+        copies = [p0] + [p0.clone() for _ in range(rot - 1)]
+        dy = (torch.randn(1, N, generator=g, device=dev) * 1e-3).to(torch.bfloat16)
+        xq = torch.randint(-127, 128, (1, K), generator=g, device=dev, dtype=torch.int8)
+        sc = torch.rand(1, generator=g, device=dev) + 0.5
+        dx = torch.empty((1, K), dtype=torch.float32, device=dev)
+        dws = torch.zeros(B.bitlinear_backward_dx_workspace_bytes(1, N, K, 0), dtype=torch.uint8, device=dev)
+        rot_w = max(2, -(-4 * l2 // (N * K * 4)))
+        dw = [torch.empty((N, K), dtype=torch.float32, device=dev) for _ in range(rot_w)]
+
+        def f_dx(j, copies=copies, gamma=gamma, N=N, K=K, dy=dy, dx=dx, dws=dws):
+            B.bitlinear_backward_dx(copies[j % len(copies)], 0, gamma, N, K, dy, dx, dws, stream)
+
+        def f_dw(j, dy=dy, xq=xq, sc=sc, gamma=gamma, dw=dw):
+            B.bitlinear_backward_dw(dy, xq, sc, gamma, dw[j % len(dw)], stream)
+
+        steps = max(1, args.decode_steps // 4)
+        res = {"N": N, "K": K}
+        for name, fn, nbytes in (("dx", f_dx, N * rb + 2 * N + 4 * K + 4),
+                                 ("dw", f_dw, 4 * N * K + 2 * N + K + 8)):
+            with torch.cuda.stream(stream):
+                for j in range(3):
+                    fn(j)
+            us = graph_ms(stream, steps, fn) / steps * 1e3
+            res[name] = {"us": us, "bytes": nbytes, "GB_s": nbytes / (us * 1e-6) / 1e9,
+                         "frac_of_hbm": nbytes / (us * 1e-6) / 1e9 / peak}
+        if B.bitlinear_device_status(dws, stream) != B.BL_OK:
+            raise RuntimeError("backward device status")
+        out.append(res)
+        del copies, p0, dw
+    return {"workload": "3B decode layers, one bf16 gradient token, 2-bit weights", "peak": peak, "peak_kind": kind,
+            "layers": out, "note": "fp64 sums in a fixed order, fp32 out; bytes: dx = packed + dy + dx, "
+                                   "dw = N K fp32 + dy + x_q"}
 
 
 def run_sweep(args, dev, stream, l2):
@@ -932,6 +994,7 @@ def main():
                     "d2h_bytes_per_step": res["d2h"], "steps": res["e2e_steps"]},
             "prefill": prefill_summary(res["prefill"]),
             "decode_gemv": decode_summary(res["decode"]),
+            "backward": res.get("backward"),
             "sweep": res["sweep"],
             "gpu_launches": res["launches_per_step"] * args.steps,
             "clocks": res["clocks"],

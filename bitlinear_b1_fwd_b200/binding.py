@@ -42,6 +42,9 @@ SIGNATURES = {
     "bitlinear_forward": (_I, [_P, _I, _P, _I64, _I64, _P, _I, _P, _I64, _P, _I, _P, _SZ, _P]),
     "bitlinear_forward_grouped_workspace_bytes": (_SZ, [_I64, _I64, _P, _I64, _I, _I]),
     "bitlinear_forward_grouped": (_I, [_P, _I, _P, _I64, _P, _I64, _P, _I, _P, _I64, _P, _I, _P, _SZ, _P]),
+    "bitlinear_backward_dx_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
+    "bitlinear_backward_dx": (_I, [_P, _I, _P, _I64, _I64, _P, _I, _I64, _P, _P, _SZ, _P]),
+    "bitlinear_backward_dw": (_I, [_P, _I, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "bitlinear_selftest_wait_timeout": (_I, [_P, _SZ, _P]),
     "bitlinear_device_status": (_I, [_P, _P]),
     "bitlinear_status_string": (C.c_char_p, [_I]),
@@ -225,6 +228,27 @@ def bitlinear_forward_grouped(packed, fmt, gammas, group_rows, K, x, scale, y, w
                                            _ptr(scale), M, _ptr(y), dtype_code(y), _ptr(ws),
                                            ws.numel() * ws.element_size(), _stream(stream)),
            "bitlinear_forward_grouped")
+
+
+def bitlinear_backward_dx_workspace_bytes(M: int, N: int, K: int, fmt: int) -> int:
+    return int(lib().bitlinear_backward_dx_workspace_bytes(M, N, K, fmt))
+
+
+def bitlinear_backward_dx(packed, fmt, gamma, N, K, dy, dx, ws, stream=None) -> None:
+    _contig(packed, gamma, dy, dx, ws)
+    M = dy.shape[0]
+    _check(lib().bitlinear_backward_dx(_ptr(packed), fmt, _ptr(gamma), N, K, _ptr(dy), dtype_code(dy), M, _ptr(dx),
+                                       _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "bitlinear_backward_dx")
+
+
+def bitlinear_backward_dw(dy, xq, scale, gamma, dw, stream=None) -> None:
+    _contig(dy, xq, scale, gamma, dw)
+    M, N = dy.shape
+    K = xq.shape[1]
+    _check(lib().bitlinear_backward_dw(_ptr(dy), dtype_code(dy), _ptr(xq), _ptr(scale), _ptr(gamma), M, N, K,
+                                       _ptr(dw), _stream(stream)),
+           "bitlinear_backward_dw")
 
 
 def bitlinear_device_status(ws, stream=None) -> int:

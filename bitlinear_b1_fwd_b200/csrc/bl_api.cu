@@ -328,6 +328,51 @@ bl_status bitlinear_forward_grouped(const uint8_t* packed, int fmt, const float*
   return BL_OK;
 }
 
+// STE backward.
+size_t bitlinear_backward_dx_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt) {
+  if (N < 1 || M < 0 || !nk_ok(N, K) || !fmt_ok(fmt)) return 0;
+  size_t bytes = BL_WS_HEADER_BYTES;
+  if (fmt != BL_PACK_I2) bytes += round256(static_cast<size_t>(N * bitlinear_packed_row_bytes(K, BL_PACK_I2)));
+  const int64_t mt = M < bl::backward_dx_tokens_per_pass() ? M : bl::backward_dx_tokens_per_pass();
+  bytes += round256(static_cast<size_t>(bl::backward_dx_chunks(N) * mt * K) * sizeof(double));
+  return bytes;
+}
+
+bl_status bitlinear_backward_dx(const uint8_t* packed, int fmt, const float* gamma, int64_t N, int64_t K,
+                                const void* dy, int dydt, int64_t M, float* dx, void* ws, size_t ws_bytes,
+                                void* stream) {
+  if (!fmt_ok(fmt) || !float_dt(dydt) || M < 0 || N < 1 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
+  if (M == 0) return BL_OK;
+  if (packed == nullptr || gamma == nullptr || dy == nullptr || dx == nullptr || ws == nullptr)
+    return BL_ERR_INVALID_VALUE;
+  if (!aligned(packed, 16) || !aligned(dy, 16) || !aligned(dx, 16) || !aligned(gamma, 4) || !aligned(ws, 16))
+    return BL_ERR_MISALIGNED;
+  if (ws_bytes < bitlinear_backward_dx_workspace_bytes(M, N, K, fmt)) return BL_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* scratch = static_cast<uint8_t*>(ws) + BL_WS_HEADER_BYTES;
+  const int64_t rb2 = bitlinear_packed_row_bytes(K, BL_PACK_I2);
+  const uint8_t* w2 = packed;
+  if (fmt != BL_PACK_I2) {
+    const int64_t rb = bitlinear_packed_row_bytes(K, fmt);
+    const cudaError_t e = fmt == BL_PACK_T5 ? bl::launch_t5_to_i2(packed, N, K, rb, scratch, rb2, st)
+                                            : bl::launch_b1_to_i2(packed, N, K, rb, scratch, rb2, st);
+    if (e != cudaSuccess) return BL_ERR_CUDA;
+    w2 = scratch;
+    scratch += round256(static_cast<size_t>(N * rb2));
+  }
+  return cuda_status(bl::launch_backward_dx(w2, rb2, gamma, N, K, dy, dydt, M, dx, reinterpret_cast<double*>(scratch), st));
+}
+
+bl_status bitlinear_backward_dw(const void* dy, int dydt, const int8_t* xq, const float* scale, const float* gamma,
+                                int64_t M, int64_t N, int64_t K, float* dw, void* stream) {
+  if (!float_dt(dydt) || M < 0 || N < 1 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
+  if (dw == nullptr || gamma == nullptr || (M > 0 && (dy == nullptr || xq == nullptr || scale == nullptr)))
+    return BL_ERR_INVALID_VALUE;
+  if (!aligned(dy, 16) || !aligned(xq, 16) || !aligned(dw, 16) || !aligned(scale, 4) || !aligned(gamma, 4))
+    return BL_ERR_MISALIGNED;
+  return cuda_status(bl::launch_backward_dw(dy, dydt, xq, scale, gamma, M, N, K, dw, static_cast<cudaStream_t>(stream)));
+}
+
 bl_status bitlinear_selftest_wait_timeout(void* ws, size_t ws_bytes, void* stream) {
   // 16 tokens x 128 rows x 128 K: the header plus 8 KB of operand space that is never touched
   if (ws == nullptr || ws_bytes < BL_WS_HEADER_BYTES + 8192) return BL_ERR_INVALID_VALUE;

@@ -1,0 +1,239 @@
+// bl_backward.cu -- STE backward of the BitLinear layer.
+//
+// "BitNet b1.58深度解析：三值权重如何重塑大模型推理" §5.3: the layer computes
+// F.linear(x_deq, W_eff) * gamma with W_eff = W_ternary + W - W.detach(), the
+// straight-through estimator taking each quantizer as the identity in the
+// backward pass ("QAT and BitNet: A Deep Dive into 1-bit and 1.58-bit
+// Quantization-Aware Training", "How Gradients Flow: Fake Quantization and
+// STE").  With gamma a constant of the step and an upstream gradient dy [M, N]:
+//   dx[m, k] = gamma * sum_n dy[m, n] W_q[n, k]
+//   dW[n, k] = gamma * sum_m dy[m, n] x_q[m, k] s_m / 127
+// Both sums run in fp64 (one rounding per operation, no contraction) in a
+// fixed order and are rounded to fp32 once at the end:
+//   dx: rows in chunks of 64, each chunk summed from 0.0 in row order
+//       (+dy for weight +1, -dy for -1, nothing for 0), the chunk sums added
+//       from 0.0 in chunk order, then gamma * S;
+//   dW: c_m = s_m / 127, terms (dy[m, n] x_q[m, k]) c_m added from 0.0 in token
+//       order, then gamma * T.
+// dx reads the packed 2-bit weights once per pass of up to two tokens; dW
+// writes N K fp32 values (the HBM-bound part for few tokens).
+#include "bl_common.cuh"
+#include "bl_kernels.h"
+
+namespace bl {
+
+constexpr int kDxChunk = 64;   // rows per partial sum (enough units to fill every SM)
+constexpr int kDxTokens = 2;   // tokens per pass: 16 weights x 2 tokens of fp64 sums per thread
+
+template <int DYT>
+__device__ __forceinline__ double load_grad(const void* p, int64_t i) {
+  return static_cast<double>(load_elem<DYT>(p, i));
+}
+
+// Partial sums: thread (chunk r, word column c) adds, for rows n of chunk r in
+// order, the 16 weights of packed word c of row n times dy[m, n] for the MT
+// tokens of the pass.  A warp's lanes take 32 consecutive columns of one
+// chunk, so each row is one 128-byte read.  part[r][m][k] (fp64).
+template <int DYT, int MT>
+__global__ void __launch_bounds__(256)
+    backward_dx_partial_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, int64_t N, int64_t K,
+                               const void* __restrict__ dy, int64_t m0, double* __restrict__ part) {
+  pdl_enter(packed, dy, part);
+  const int64_t words = (K + 15) / 16;  // packed 32-bit words holding weights below K
+  const int64_t chunks = (N + kDxChunk - 1) / kDxChunk;
+  const int64_t units = words * chunks;
+  for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < units;
+       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = u / words, c = u - r * words;
+    double acc[MT][16];
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) acc[m][i] = 0.0;
+    const int64_t n1 = (r + 1) * kDxChunk < N ? (r + 1) * kDxChunk : N;
+    const uint32_t* col = reinterpret_cast<const uint32_t*>(packed) + c;
+    const int64_t stride = rowbytes / 4;
+    // the rows' words (and gradients) are loaded 16 at a time ahead of the
+    // adds, so that a thread keeps 16 loads in flight
+    for (int64_t nb = r * kDxChunk; nb < n1; nb += 16) {
+      uint32_t wv[16];
+      double gv[MT][16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int64_t n = nb + j;
+        wv[j] = n < n1 ? __ldcg(col + n * stride) : 0x55555555u;  // past the chunk: weight 0
+#pragma unroll
+        for (int m = 0; m < MT; ++m) gv[m][j] = n < n1 ? load_grad<DYT>(dy, (m0 + m) * N + n) : 0.0;
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+      const uint32_t w = wv[j];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const double g = gv[m][j];
+        const double ng = -g;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t d = (w >> (2 * i)) & 3u;  // digit q + 1
+          if (d == 2u)
+            acc[m][i] = __dadd_rn(acc[m][i], g);
+          else if (d == 0u)
+            acc[m][i] = __dadd_rn(acc[m][i], ng);
+        }
+      }
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      double* dst = part + (r * MT + m) * K + 16 * c;
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (16 * c + i < K) dst[i] = acc[m][i];
+    }
+  }
+}
+
+// dx[m0 + m, k] = fp32(gamma * sum_r part[r][m][k]), r in order.
+template <int MT>
+__global__ void __launch_bounds__(256)
+    backward_dx_reduce_kernel(const double* __restrict__ part, int64_t chunks, int64_t K, const float* __restrict__ gamma,
+                              int64_t m0, float* __restrict__ dx) {
+  pdl_enter(part, gamma, dx);
+  __shared__ double sh_g;
+  if (threadIdx.x == 0) sh_g = static_cast<double>(__ldcg(gamma));
+  __syncthreads();
+  const double g = sh_g;
+  const int64_t total = MT * K;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = e / K, k = e - m * K;
+    double S = 0.0;
+#pragma unroll 8
+    for (int64_t r = 0; r < chunks; ++r) S = __dadd_rn(S, __ldcg(part + (r * MT + m) * K + k));
+    dx[(m0 + m) * K + k] = __double2float_rn(__dmul_rn(g, S));
+  }
+}
+
+// dW: thread owns four consecutive outputs (n, k0 .. k0 + 3) and adds the M
+// tokens in order; c_m = s_m / 127 is computed once per CTA per token block in
+// shared memory.  The grid-stride loop runs the same number of iterations in
+// every thread of a CTA (the barriers of the token blocks are uniform).
+constexpr int kDwTokBlock = 256;
+
+template <int DYT>
+__global__ void __launch_bounds__(256)
+    backward_dw_kernel(const void* __restrict__ dy, const int8_t* __restrict__ xq, const float* __restrict__ scale,
+                       const float* __restrict__ gamma, int64_t M, int64_t N, int64_t K, float* __restrict__ dw) {
+  pdl_enter(dy, xq, scale, gamma, dw);
+  __shared__ double sh_c[kDwTokBlock];
+  __shared__ double sh_g;
+  if (threadIdx.x == 0) sh_g = static_cast<double>(__ldcg(gamma));
+  const int64_t kq = (K + 3) / 4;
+  const int64_t total = N * kq;
+  const bool vec = (K % 4) == 0;
+  auto term4 = [&](int64_t m, int64_t n, int64_t k0, double c, double (&T)[4]) {
+    const double g = load_grad<DYT>(dy, m * N + n);
+    int q[4];
+    if (vec) {
+      const uint32_t w = __ldcg(reinterpret_cast<const uint32_t*>(xq + m * K + k0));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) q[i] = static_cast<int8_t>(w >> (8 * i));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) q[i] = (k0 + i < K) ? static_cast<int>(__ldcg(xq + m * K + k0 + i)) : 0;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) T[i] = __dadd_rn(T[i], __dmul_rn(__dmul_rn(g, static_cast<double>(q[i])), c));
+  };
+  auto store4 = [&](int64_t n, int64_t k0, const double (&T)[4], double g) {
+    float o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = __double2float_rn(__dmul_rn(g, T[i]));
+    float* dst = dw + n * K + k0;
+    if (vec) {
+      *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (k0 + i < K) dst[i] = o[i];
+    }
+  };
+  if (M <= kDwTokBlock) {  // every token's factor in shared memory once; no barrier in the loop
+    if (threadIdx.x < M) sh_c[threadIdx.x] = __ddiv_rn(static_cast<double>(__ldcg(scale + threadIdx.x)), 127.0);
+    __syncthreads();
+    const double g = sh_g;
+    for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+      const int64_t n = e / kq, k0 = 4 * (e - n * kq);
+      double T[4] = {0.0, 0.0, 0.0, 0.0};
+      for (int64_t m = 0; m < M; ++m) term4(m, n, k0, sh_c[m], T);
+      store4(n, k0, T, g);
+    }
+    return;
+  }
+  for (int64_t base = blockIdx.x * static_cast<int64_t>(blockDim.x); base < total;
+       base += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t e = base + threadIdx.x;
+    const bool active = e < total;
+    const int64_t n = active ? e / kq : 0;
+    const int64_t k0 = active ? 4 * (e - n * kq) : 0;
+    double T[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int64_t t0 = 0; t0 < M; t0 += kDwTokBlock) {
+      const int64_t tn = (M - t0) < kDwTokBlock ? (M - t0) : kDwTokBlock;
+      __syncthreads();  // the previous block's factors have been read
+      if (threadIdx.x < tn) sh_c[threadIdx.x] = __ddiv_rn(static_cast<double>(__ldcg(scale + t0 + threadIdx.x)), 127.0);
+      __syncthreads();
+      if (active)
+        for (int64_t j = 0; j < tn; ++j) term4(t0 + j, n, k0, sh_c[j], T);
+    }
+    if (active) store4(n, k0, T, sh_g);
+  }
+}
+
+// ---- host side --------------------------------------------------------------------
+int64_t backward_dx_chunks(int64_t N) { return (N + kDxChunk - 1) / kDxChunk; }
+int backward_dx_tokens_per_pass() { return kDxTokens; }
+
+static unsigned grid_of(int64_t work, int per_sm) {
+  const int64_t cap = static_cast<int64_t>(device_sms()) * per_sm;
+  int64_t g = (work + 255) / 256;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return static_cast<unsigned>(g);
+}
+
+cudaError_t launch_backward_dx(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
+                               const void* dy, int dydt, int64_t M, float* dx, double* part, cudaStream_t st) {
+  const int64_t chunks = backward_dx_chunks(N);
+  const int64_t words = (K + 15) / 16;
+  for (int64_t m0 = 0; m0 < M; m0 += kDxTokens) {
+    const int mt = (M - m0) < kDxTokens ? static_cast<int>(M - m0) : kDxTokens;
+    const unsigned gp = grid_of(words * chunks, 8);
+    const unsigned gr = grid_of(mt * K, 8);
+    cudaError_t e;
+    if (dydt == BL_F32) {
+      e = mt == 2 ? launch_pdl(backward_dx_partial_kernel<BL_F32, 2>, gp, 256, 0, st, packed, rowbytes, N, K, dy, m0, part)
+                  : launch_pdl(backward_dx_partial_kernel<BL_F32, 1>, gp, 256, 0, st, packed, rowbytes, N, K, dy, m0, part);
+    } else {
+      e = mt == 2 ? launch_pdl(backward_dx_partial_kernel<BL_BF16, 2>, gp, 256, 0, st, packed, rowbytes, N, K, dy, m0, part)
+                  : launch_pdl(backward_dx_partial_kernel<BL_BF16, 1>, gp, 256, 0, st, packed, rowbytes, N, K, dy, m0, part);
+    }
+    if (e != cudaSuccess) return e;
+    e = mt == 2 ? launch_pdl(backward_dx_reduce_kernel<2>, gr, 256, 0, st, part, chunks, K, gamma, m0, dx)
+                : launch_pdl(backward_dx_reduce_kernel<1>, gr, 256, 0, st, part, chunks, K, gamma, m0, dx);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_backward_dw(const void* dy, int dydt, const int8_t* xq, const float* scale, const float* gamma,
+                               int64_t M, int64_t N, int64_t K, float* dw, cudaStream_t st) {
+  const unsigned g = grid_of(N * ((K + 3) / 4), 8);
+  cudaError_t e = dydt == BL_F32
+                      ? launch_pdl(backward_dw_kernel<BL_F32>, g, 256, 0, st, dy, xq, scale, gamma, M, N, K, dw)
+                      : launch_pdl(backward_dw_kernel<BL_BF16>, g, 256, 0, st, dy, xq, scale, gamma, M, N, K, dw);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace bl

@@ -87,6 +87,15 @@ inline RowGroups one_group(int64_t N) {
   return rg;
 }
 
+// STE backward: dx through fp64 partial sums part [chunks][2][K] (chunks =
+// backward_dx_chunks(N)); dW straight into dw [N, K].
+int64_t backward_dx_chunks(int64_t N);
+int backward_dx_tokens_per_pass();
+cudaError_t launch_backward_dx(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
+                               const void* dy, int dydt, int64_t M, float* dx, double* part, cudaStream_t st);
+cudaError_t launch_backward_dw(const void* dy, int dydt, const int8_t* xq, const float* scale, const float* gamma,
+                               int64_t M, int64_t N, int64_t K, float* dw, cudaStream_t st);
+
 cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int64_t N, int64_t K,
                         const void* x, int xdt, float* scale, int64_t M, void* y, int ydt,
                         const RowGroups& rg, cudaStream_t st);

@@ -254,6 +254,31 @@ BL_API bl_status bitlinear_forward_grouped(const uint8_t *packed, int fmt, const
                                         float *scale, int64_t M, void *y, int ydt, void *ws, size_t ws_bytes,
                                         void *stream);
 
+/* STE backward of the BitLinear layer (the training side).  [P3] §5.3 (the
+ * layer's F.linear(x_deq, W_eff) * gamma with W_eff = W_ternary + W -
+ * W.detach(): the quantizer is the identity in the backward pass); [P5] "How
+ * Gradients Flow: Fake Quantization and STE".  Both quantizers pass the
+ * gradient straight through and gamma is a constant of the step, so for an
+ * upstream gradient dy [M, N] (fp32 or bf16):
+ *   dx [M, K] = gamma * dy . W_q        (bitlinear_backward_dx)
+ *   dW [N, K] = gamma * dy^T . x_deq    (bitlinear_backward_dw),
+ *   x_deq[m, k] = x_q[m, k] * s_m / 127 (the forward's codes and scales).
+ * Both are fp64 sums in a fixed order rounded once to fp32: dx adds the rows
+ * in chunks of 64 (each chunk from 0.0 in row order; chunk sums from 0.0 in
+ * chunk order) then multiplies by gamma; dW adds (dy x_q) (s_m / 127) from
+ * 0.0 in token order then multiplies by gamma.  A CUDA-core path for few
+ * tokens: dx reads the packed weights once per two tokens.
+ *   packed, fmt, gamma  as for bitlinear_forward (gamma: beta for BL_PACK_B1).
+ *   dx    [M, K] fp32 output;  dw [N, K] fp32 output (16-byte aligned).
+ *   ws    at least bitlinear_backward_dx_workspace_bytes(M, N, K, fmt). */
+BL_API size_t bitlinear_backward_dx_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt);
+BL_API bl_status bitlinear_backward_dx(const uint8_t *packed, int fmt, const float *gamma, int64_t N, int64_t K,
+                                    const void *dy, int dydt, int64_t M, float *dx, void *ws, size_t ws_bytes,
+                                    void *stream);
+BL_API bl_status bitlinear_backward_dw(const void *dy, int dydt, const int8_t *xq, const float *scale,
+                                    const float *gamma, int64_t M, int64_t N, int64_t K, float *dw,
+                                    void *stream);
+
 /* Failure-detection self test: launches the tensor-core kernel with its data
  * producer switched off and a wait limit of about a millisecond, so that its
  * bounded waits run out; the kernel then records BL_ERR_DEVICE_TIMEOUT in the

@@ -422,7 +422,7 @@ void orc_binarize_weights(const void *W, int dt, int64_t N, int64_t K,
 /*   dW[n][k] = gamma * sum_m dy[m][n] * x_deq[m][k],                       */
 /*              x_deq[m][k] = x_q[m][k] * s_m / 127 (the forward's codes).  */
 /* Arithmetic: fp64, one rounding per operation, then fp32.  dx: the rows  */
-/* n are taken in chunks of 256 (n in [256 r, 256 r + 256)); within a chunk */
+/* n are taken in chunks of 64 (n in [64 r, 64 r + 64)); within a chunk     */
 /* the terms +dy, -dy or nothing (add / subtract / skip) go into a sum from */
 /* 0.0 in row order, and the chunk sums go into S from 0.0 in chunk order; */
 /* dx = fp32(gamma * S).  dW: c_m = s_m / 127, each term is                */
@@ -430,7 +430,7 @@ void orc_binarize_weights(const void *W, int dt, int64_t N, int64_t K,
 /* dW = fp32(gamma * T).                                                    */
 /* ------------------------------------------------------------------------ */
 
-#define ORC_DX_CHUNK 256
+#define ORC_DX_CHUNK 64
 
 void orc_backward_dx(const int8_t *codes, int64_t N, int64_t K,
                      const void *dy, int dydt, int64_t M, float gamma,

@@ -71,6 +71,14 @@ def test_onebit_workspace_sizes(bl):
     assert bl.bitlinear_forward_workspace_bytes(64, 256, 1024, 2, 2) == bl.bitlinear_forward_workspace_bytes(64, 256, 1024, 1, 2)
 
 
+def test_backward_workspace_sizes(bl):
+    # header + fp64 partials [ceil(N / 64)][min(M, 2)][K], + a 2-bit copy for base 3 / 1-bit
+    assert bl.bitlinear_backward_dx_workspace_bytes(1, 512, 256, 0) == 256 + 8 * 1 * 256 * 8
+    assert bl.bitlinear_backward_dx_workspace_bytes(5, 777, 1000, 0) == 256 + (13 * 2 * 1000 * 8 + 255) // 256 * 256
+    assert bl.bitlinear_backward_dx_workspace_bytes(1, 512, 256, 1) == 256 + 512 * 64 + 8 * 256 * 8
+    assert bl.bitlinear_backward_dx_workspace_bytes(1, 0, 256, 0) == 0
+
+
 def test_status_strings(bl):
     for s in range(8):
         assert bl.status_string(s).startswith("BL_")
@@ -135,6 +143,17 @@ def test_host_validation_without_gpu(bl):
     assert L.bitlinear_forward(*args(M=0)) == bl.BL_OK
     assert L.bitlinear_forward(*args(N=0)) == bl.BL_OK
     assert L.bitlinear_forward(*args(M=0, x=null, y=null, scale=null, ws=null)) == bl.BL_OK
+    # STE backward
+    assert L.bitlinear_backward_dx(p, 0, p, 4, 4, p, 2, 1, p, p, 1 << 20, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_backward_dx(p, 5, p, 4, 4, p, 0, 1, p, p, 1 << 20, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_backward_dx(null, 0, p, 4, 4, p, 0, 1, p, p, 1 << 20, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_backward_dx(p, 0, p, 4, 4, odd, 0, 1, p, p, 1 << 20, null) == bl.BL_ERR_MISALIGNED
+    assert L.bitlinear_backward_dx(p, 0, p, 4, 4, p, 0, 1, p, p, 8, null) == bl.BL_ERR_WORKSPACE_TOO_SMALL
+    assert L.bitlinear_backward_dx(null, 0, null, 4, 4, null, 0, 0, null, null, 0, null) == bl.BL_OK
+    assert L.bitlinear_backward_dw(p, 3, p, p, p, 1, 4, 4, p, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_backward_dw(p, 0, p, p, p, 1, 0, 4, p, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_backward_dw(p, 0, p, p, p, 1, 4, 4, null, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_backward_dw(p, 0, p, p, p, 1, 4, 4, odd, null) == bl.BL_ERR_MISALIGNED
     # workspace helpers
     assert L.bitlinear_workspace_init(null, 4096, null) == bl.BL_ERR_INVALID_VALUE
     assert L.bitlinear_device_status(null, null) == bl.BL_ERR_INVALID_VALUE

@@ -1,0 +1,126 @@
+"""GPU parity of the STE backward through the C ABI against the oracle.
+
+Both sides add in fp64 in the same fixed order and round once to fp32, so dx
+and dW are compared bit for bit (the fp32 tolerance of the spec, 1e-6
+relative, is the fallback bar; the kernels meet the stricter one)."""
+import numpy as np
+import pytest
+import torch
+
+from bitlinear_b1_fwd_b200 import binding as B
+from bitlinear_b1_fwd_b200 import synth
+from gpu_helpers import dev, host, quantize_weights
+
+pytestmark = pytest.mark.gpu
+
+I2, T5, B1 = B.BL_PACK_I2, B.BL_PACK_T5, B.BL_PACK_B1
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from bitlinear_b1_fwd_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+    torch.cuda.init()
+
+
+def _weights(orc, N, K, fmt, seed):
+    W = synth.normal_f32(seed, (N, K), 0.02)
+    if fmt == B1:
+        Wd = dev(W)
+        packed = torch.empty((N, B.bitlinear_packed_row_bytes(K, B1)), dtype=torch.uint8, device="cuda")
+        beta = torch.empty(1, dtype=torch.float32, device="cuda")
+        alpha = torch.empty(1, dtype=torch.float32, device="cuda")
+        ws = torch.zeros(B.bitlinear_binarize_weights_workspace_bytes(N, K), dtype=torch.uint8, device="cuda")
+        B.bitlinear_binarize_weights(Wd, packed, None, beta, alpha, ws)
+        torch.cuda.synchronize()
+        g, packed = np.float32(beta.item()), host(packed)
+    else:
+        g, _, packed = quantize_weights(W, fmt, codes=False)
+    return g, packed, orc.unpack(packed, N, K, fmt)
+
+
+def run_dx(packed, fmt, g, N, K, dy):
+    M = dy.shape[0]
+    dx = torch.full((M, K), float("nan"), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(B.bitlinear_backward_dx_workspace_bytes(M, N, K, fmt), dtype=torch.uint8, device="cuda")
+    B.bitlinear_backward_dx(dev(packed), fmt, torch.tensor([float(g)], device="cuda"), N, K, dev(dy), dx, ws)
+    torch.cuda.synchronize()
+    assert B.bitlinear_device_status(ws) == B.BL_OK
+    return host(dx)
+
+
+@pytest.mark.parametrize("M,N,K,fmt,dydt", [
+    (1, 512, 256, I2, "f32"),
+    (3, 777, 1000, I2, "bf16"),     # K % 16 != 0: a partial last word; 13 row chunks, the last partial
+    (2, 3200, 3200, T5, "f32"),     # base 3 through the 2-bit transcoding
+    (5, 300, 129, B1, "f32"),       # 1-bit (codes in {-1, +1}); three passes of two tokens
+    (1, 8640, 3200, I2, "bf16"),    # 3B up-projection shape, one token
+    (4, 1, 64, I2, "f32"),          # one row
+])
+def test_backward_dx(orc, M, N, K, fmt, dydt):
+    g, packed, codes = _weights(orc, N, K, fmt, 720 + K)
+    dy = synth.normal_f32(721 + M, (M, N), 1e-3)
+    if dydt == "bf16":
+        dy = synth.to_bf16_bits(dy)
+    dx = run_dx(packed, fmt, g, N, K, dy)
+    ref = orc.backward_dx(codes, dy, g, parallel=True)
+    assert np.array_equal(dx.view(np.uint32), ref.view(np.uint32))
+
+
+def run_dw(dy, xq, s, g, N, K):
+    M = dy.shape[0]
+    dw = torch.full((N, K), float("nan"), dtype=torch.float32, device="cuda")
+    B.bitlinear_backward_dw(dev(dy), dev(xq), dev(s), torch.tensor([float(g)], device="cuda"), dw)
+    torch.cuda.synchronize()
+    return host(dw)
+
+
+@pytest.mark.parametrize("M,N,K,dydt", [
+    (1, 512, 256, "f32"),
+    (3, 777, 1001, "bf16"),   # K % 4 != 0: scalar loads and stores
+    (300, 64, 128, "f32"),    # two blocks of token factors
+    (1, 3200, 3200, "bf16"),  # 3B attention shape, one token
+])
+def test_backward_dw(orc, M, N, K, dydt):
+    x = synth.entry_outliers(synth.normal_f32(730 + M, (M, K)), 731, 0.01, 20.0)
+    xq, s = orc.act_quant(x)
+    dy = synth.normal_f32(732 + M, (M, N), 1e-3)
+    if dydt == "bf16":
+        dy = synth.to_bf16_bits(dy)
+    g = np.float32(0.0173)
+    dw = run_dw(dy, xq, s, g, N, K)
+    ref = orc.backward_dw(dy, xq, s, g)
+    assert np.array_equal(dw.view(np.uint32), ref.view(np.uint32))
+
+
+def test_backward_dw_no_tokens_writes_zeros():
+    N, K = 10, 16
+    dw = torch.full((N, K), float("nan"), dtype=torch.float32, device="cuda")
+    dy = torch.empty((0, N), dtype=torch.float32, device="cuda")
+    xq = torch.empty((0, K), dtype=torch.int8, device="cuda")
+    s = torch.empty((0,), dtype=torch.float32, device="cuda")
+    B.bitlinear_backward_dw(dy, xq, s, torch.tensor([0.5], device="cuda"), dw)
+    torch.cuda.synchronize()
+    assert not host(dw).any()
+
+
+def test_backward_after_forward_chain(orc):
+    """The forward's own codes and scales feed dW: quantize, forward (bf16
+    tokens), then both gradients, all through the C ABI."""
+    M, N, K = 2, 640, 512
+    W = synth.normal_f32(740, (N, K), 0.02)
+    x = synth.to_bf16_bits(synth.normal_f32(741, (M, K)))
+    g, _, packed = quantize_weights(W, I2, codes=False)
+    xq = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    s = torch.empty((M,), dtype=torch.float32, device="cuda")
+    B.bitlinear_quantize_acts(dev(x), xq, s)
+    dy = synth.normal_f32(742, (M, N), 1e-2)
+    dw = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    B.bitlinear_backward_dw(dev(dy), xq, s, torch.tensor([float(g)], device="cuda"), dw)
+    dx = run_dx(packed, I2, g, N, K, dy)
+    xq_ref, s_ref = orc.act_quant(x)
+    assert np.array_equal(host(xq), xq_ref)
+    assert np.array_equal(host(dw).view(np.uint32), orc.backward_dw(dy, xq_ref, s_ref, g).view(np.uint32))
+    codes = orc.unpack(packed, N, K, I2)
+    assert np.array_equal(dx.view(np.uint32), orc.backward_dx(codes, dy, g).view(np.uint32))

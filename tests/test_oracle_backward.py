@@ -17,7 +17,7 @@ def _codes(rng, N, K, p0=0.3):
     return np.where(u < p0, 0, np.where(u < (1 + p0) / 2, 1, -1)).astype(np.int8)
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 5, 7), (3, 777, 100), (2, 1000, 33)])
+@pytest.mark.parametrize("M,N,K", [(1, 5, 7), (3, 777, 100), (2, 1000, 33), (1, 64, 16), (1, 65, 16)])
 def test_dx_exact_on_integers(orc, M, N, K):
     """Integer dy and gamma = 0.5: every partial sum is an exact integer, so
     the chunk order is immaterial and dx = 0.5 (dy . W_q) exactly."""
