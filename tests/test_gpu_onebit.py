@@ -179,3 +179,33 @@ def test_forward_grouped_b1(orc, M):
         assert np.array_equal(host(s), s_ref)
         assert_f32_rel(yh[:, off:off + n], y_ref)
         off += n
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_forward_grouped_b1_long_rows(orc, M):
+    """1-bit groups with rows longer than the 1-bit GEMV takes (K = 40000):
+    transcoded to 2 bits in the workspace, then the general GEMV kernel with
+    the row-group table."""
+    K, rows = 40000, [96, 40, 130]
+    betas, packs = [], []
+    for i, n in enumerate(rows):
+        _, b, _, p = binarize(synth.normal_f32(640 + i, (n, K), 0.01 * (i + 1)), codes=False)
+        betas.append(b)
+        packs.append(p)
+    packed = np.concatenate(packs, axis=0)
+    x = synth.to_bf16_bits(synth.normal_f32(650 + M, (M, K)))
+    N = sum(rows)
+    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    s = torch.empty(M, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(B.bitlinear_forward_grouped_workspace_bytes(M, rows, K, B1, B.BL_BF16), dtype=torch.uint8,
+                     device="cuda")
+    B.bitlinear_forward_grouped(dev(packed), B1, dev(np.array(betas, np.float32)), rows, K, dev(x), s, y, ws)
+    torch.cuda.synchronize()
+    assert B.bitlinear_device_status(ws) == B.BL_OK
+    yh = host(y)
+    off = 0
+    for g, n in enumerate(rows):
+        y_ref, s_ref = orc.forward(packs[g], B1, betas[g], n, K, x, ydt=0)
+        assert np.array_equal(host(s), s_ref)
+        assert_f32_rel(yh[:, off:off + n], y_ref)
+        off += n
