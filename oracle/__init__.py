@@ -25,6 +25,11 @@ import numpy as np
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "bitlinear_oracle.c")
 LIB_PATH = os.path.join(HERE, "liboracle.so")
+# A test of the pins themselves builds copies of the oracle with one planted
+# mistake each and points this variable at such a copy (never set otherwise).
+_PLANTED = os.environ.get("BL_ORACLE_PLANTED_LIB")
+if _PLANTED:
+    LIB_PATH = _PLANTED
 
 F32, BF16, I8, I32 = 0, 1, 2, 3
 PACK_I2, PACK_T5, PACK_B1 = 0, 1, 2
@@ -35,6 +40,8 @@ _lock = threading.Lock()
 
 def build(force: bool = False) -> str:
     """Compile the oracle with gcc (IEEE arithmetic: no fast-math, no FMA)."""
+    if _PLANTED:
+        return LIB_PATH  # a prebuilt copy with a planted mistake
     if (not force and os.path.exists(LIB_PATH)
             and os.path.getmtime(LIB_PATH) >= os.path.getmtime(SRC)):
         return LIB_PATH
