@@ -17,6 +17,12 @@
  *   acc[m, n] = sum_k W_q[n, k] x_q[m, k]  (INT32)    [P3] §4.2 §3.3
  *   y[m, n] = acc[m, n] * (gamma * s_m / 127)         [P3] §3.2 §5.3, [P5]
  *
+ * Around that path: the pre-norm LayerNorm feeding x_q ([P5] recipe step 1),
+ * several layers on one input (a block's Q, K, V: [P3] §5.4), the 1-bit
+ * variant (alpha = mean W, codes sign(W - alpha), beta = mean |W|, 8 weights
+ * per byte: [P5] recipe steps 2 and 4) and the straight-through backward
+ * (dx = gamma dy W_q, dW = gamma dy^T x_deq: [P3] §5.3).
+ *
  * Exact conventions (where the pages are silent):
  *   - gamma: |w| summed in fp64 in a fixed order (below), divided by N*K in
  *     fp64, rounded to fp32.  Order: elements in row-major order e = n*K + k;
@@ -34,7 +40,8 @@
  *   - 2-bit format: digit q + 1 (-1 -> 00, 0 -> 01, +1 -> 10) of weight k in
  *     bits 2*(k % 4) of byte k / 4.  Base-3 format: byte j of a row is
  *     sum_i (q[5j + i] + 1) * 3^i.  Every row is padded to a multiple of 16
- *     bytes with digits of weight 0 (0x55 / 121).  Row stride =
+ *     bytes with digits of weight 0 (0x55 / 121).  1-bit format: bit k % 8 of
+ *     byte k / 8 is 1 for +1 and 0 for -1, pad bits 0.  Row stride =
  *     bitlinear_packed_row_bytes(K, fmt).
  *
  * Conventions of every call:
