@@ -827,6 +827,7 @@ PROFILE_CASES = {
     "batch16_70b_down": dict(N=8192, K=28672, fmt=0, M=16, sigma=0.01, op="forward"),
     "binarize_3b_up": dict(N=8640, K=3200, fmt=2, M=1, sigma=0.02, op="quantize"),
     "decode_70b_up_1bit": dict(N=28672, K=8192, fmt=2, M=1, sigma=0.01, op="forward"),
+    "backward_3b_up": dict(N=8640, K=3200, fmt=0, M=1, sigma=0.02, op="backward"),
 }
 
 
@@ -870,6 +871,18 @@ def run_profile_case(name):
         for _ in range(3):
             B.bitlinear_forward(packed, fmt, gamma, N, K, x, scale, y, fws)
         status.append(B.bitlinear_device_status(fws))
+    if c["op"] == "backward":  # STE backward for M tokens: dx from the packed weights, dW from x_q
+        dy = (torch.randn(M, N, generator=g, device=dev) * 1e-3).to(torch.bfloat16)
+        xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+        sc = torch.empty(M, dtype=torch.float32, device=dev)
+        B.bitlinear_quantize_acts(x, xq, sc)
+        dx = torch.empty((M, K), dtype=torch.float32, device=dev)
+        dw = torch.empty((N, K), dtype=torch.float32, device=dev)
+        bws = torch.zeros(B.bitlinear_backward_dx_workspace_bytes(M, N, K, fmt), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            B.bitlinear_backward_dx(packed, fmt, gamma, N, K, dy, dx, bws)
+            B.bitlinear_backward_dw(dy, xq, sc, gamma, dw)
+        status.append(B.bitlinear_device_status(bws))
     torch.cuda.synchronize()
     print(json.dumps({"profile_case": name, **c, "status": status}))
     if any(status):
