@@ -165,3 +165,39 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         binding.lib()
+
+
+def _prototypes():
+    """name -> (return type, [parameter types]) for every BL_API function."""
+    text = re.sub(r"/\*.*?\*/", " ", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"BL_API\s+([^;]*?)\b(bitlinear_\w+)\s*\(([^)]*)\)\s*;", text, flags=re.S):
+        ret, name, params = " ".join(m.group(1).split()), m.group(2), " ".join(m.group(3).split())
+        if params in ("", "void"):
+            types = []
+        else:
+            types = [re.sub(r"\s*\b\w+$", "", p.strip()).strip() if not p.strip().endswith("*") else p.strip()
+                     for p in params.split(",")]
+        out[name] = (ret, types)
+    return out
+
+
+def _ctype_of(c_type: str):
+    t = c_type.replace("const ", "").strip()
+    if "*" in t:
+        return C.c_char_p if t.startswith("char") else C.c_void_p
+    return {"int64_t": C.c_int64, "size_t": C.c_size_t, "int": C.c_int, "float": C.c_float,
+            "bl_status": C.c_int}[t]
+
+
+def test_binding_signatures_match_the_header(bl):
+    """Every ctypes signature has the header's parameter count, widths and
+    return type (a mismatch would pass wrong values silently)."""
+    protos = _prototypes()
+    assert set(protos) == set(declared_functions())
+    for name, (ret, params) in protos.items():
+        res, args = bl.SIGNATURES[name]
+        assert len(args) == len(params), (name, params, args)
+        for i, (p, a) in enumerate(zip(params, args)):
+            assert _ctype_of(p) == a, (name, i, p, a)
+        assert _ctype_of(ret) == res, (name, ret, res)
