@@ -36,3 +36,22 @@ def test_forward_from_cpp(abi_binary):
     r = subprocess.run([abi_binary, "--gpu"], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stdout + r.stderr
     assert r.stdout.startswith("OK")
+
+
+def test_header_is_plain_c99(tmp_path):
+    """The header compiles as strict C99 (-Wall -Wextra -pedantic -Werror) and a
+    C program links against the library and calls it."""
+    from bitlinear_b1_fwd_b200 import build
+    lib = build.build()
+    src = tmp_path / "c_client.c"
+    src.write_text('#include "bitlinear.h"\n'
+                   "int main(void) {\n"
+                   "  if (bitlinear_packed_row_bytes(3200, BL_PACK_I2) != 800) return 1;\n"
+                   "  if (bitlinear_forward(0, BL_PACK_I2, 0, 4, 4, 0, BL_BF16, 0, 1, 0, BL_BF16, 0, 0, 0)\n"
+                   "      != BL_ERR_INVALID_VALUE) return 2;\n"
+                   "  return bitlinear_version() >= 100 ? 0 : 3;\n"
+                   "}\n")
+    exe = str(tmp_path / "c_client")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", exe, lib, f"-Wl,-rpath,{LIBDIR}"], check=True)
+    assert subprocess.run([exe], timeout=60).returncode == 0
