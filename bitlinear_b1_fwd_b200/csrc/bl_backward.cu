@@ -8,13 +8,14 @@
 // STE").  With gamma a constant of the step and an upstream gradient dy [M, N]:
 //   dx[m, k] = gamma * sum_n dy[m, n] W_q[n, k]
 //   dW[n, k] = gamma * sum_m dy[m, n] x_q[m, k] s_m / 127
-// Both sums run in fp64 (one rounding per operation, no contraction) in a
-// fixed order and are rounded to fp32 once at the end:
-//   dx: rows in chunks of 64, each chunk summed from 0.0 in row order
-//       (+dy for weight +1, -dy for -1, nothing for 0), the chunk sums added
-//       from 0.0 in chunk order, then gamma * S;
-//   dW: c_m = s_m / 127, terms (dy[m, n] x_q[m, k]) c_m added from 0.0 in token
-//       order, then gamma * T.
+// dx is defined by the exact sum over the rows rounded once to fp64 (no
+// order), then gamma * S in fp64 and fp32; this kernel adds in fp64 in an
+// order of its own (rows in chunks of 64, +dy for weight +1, -dy for -1,
+// nothing for 0; the chunk sums in chunk order), which stays within one fp32
+// ulp plus gamma N 2^-52 sum |dy| of the definition.
+// dW: c_m = s_m / 127, terms (dy[m, n] x_q[m, k]) c_m added in fp64 from 0.0
+// in token order (the plain order of the sum), then gamma * T, rounded once
+// to fp32.
 // dx reads the packed 2-bit weights once per pass of up to two tokens; dW
 // writes N K fp32 values (the HBM-bound part for few tokens).
 #include "bl_common.cuh"

@@ -421,35 +421,108 @@ void orc_binarize_weights(const void *W, int dt, int64_t N, int64_t K,
 /*   dx[m][k] = gamma * sum_n dy[m][n] * W_q[n][k]                          */
 /*   dW[n][k] = gamma * sum_m dy[m][n] * x_deq[m][k],                       */
 /*              x_deq[m][k] = x_q[m][k] * s_m / 127 (the forward's codes).  */
-/* Arithmetic: fp64, one rounding per operation, then fp32.  dx: the rows  */
-/* n are taken in chunks of 64 (n in [64 r, 64 r + 64)); within a chunk     */
-/* the terms +dy, -dy or nothing (add / subtract / skip) go into a sum from */
-/* 0.0 in row order, and the chunk sums go into S from 0.0 in chunk order; */
-/* dx = fp32(gamma * S).  dW: c_m = s_m / 127, each term is                */
-/* (dy[m][n] * x_q[m][k]) * c_m, added from 0.0 in token order into T;     */
-/* dW = fp32(gamma * T).                                                    */
+/* dx: the pages fix no summation order, so none is taken: S is the exact   */
+/* real sum of the terms +dy, -dy or nothing (add / subtract / skip),       */
+/* rounded once to fp64 (nearest, ties to even); dx = fp32(gamma * S) with  */
+/* the product in fp64.  Any summation order gives the same S.             */
+/* dW: c_m = s_m / 127, each term is (dy[m][n] * x_q[m][k]) * c_m, added    */
+/* from 0.0 in token order (the plain order of the sum) into T;            */
+/* dW = fp32(gamma * T).  Gradients are finite.                            */
 /* ------------------------------------------------------------------------ */
 
-#define ORC_DX_CHUNK 64
+/* Exact sum of fp32 values.  Every finite fp32 value is an integer multiple */
+/* of 2^-149 (the smallest subnormal) and below 2^128, i.e. an integer below */
+/* 2^277 in that unit; 2^31 terms stay below 2^308.  The integer is held as  */
+/* ORC_XLIMBS little-endian base-2^32 digits in int64 slots, so a digit may   */
+/* run ahead of its carries for 2^29 additions (each adds less than 2^32).   */
+#define ORC_XLIMBS 10
+typedef struct {
+  int64_t d[ORC_XLIMBS];
+  int64_t adds;
+} orc_xsum;
+
+static void xsum_normalize(orc_xsum *a) {
+  for (int i = 0; i + 1 < ORC_XLIMBS; ++i) {
+    int64_t low = a->d[i] & (int64_t)0xffffffff;
+    int64_t carry = (a->d[i] - low) / ((int64_t)1 << 32); /* exact: floor */
+    a->d[i] = low;
+    a->d[i + 1] += carry;
+  }
+  a->adds = 0;
+}
+
+/* a += sign * v exactly (sign = +1 or -1). */
+static void xsum_add(orc_xsum *a, float v, int sign) {
+  uint32_t u;
+  memcpy(&u, &v, sizeof u);
+  uint32_t e = (u >> 23) & 0xffu, f = u & 0x7fffffu;
+  uint64_t mant = e ? (f | 0x800000u) : f;
+  int shift = e ? (int)e - 1 : 0; /* value = mant * 2^(shift - 149) */
+  if (u >> 31) sign = -sign;
+  uint64_t t = mant << (shift & 31);
+  int i = shift >> 5;
+  int64_t lo = (int64_t)(t & 0xffffffffu), hi = (int64_t)(t >> 32);
+  a->d[i] += sign * lo;
+  a->d[i + 1] += sign * hi;
+  if (++a->adds == ((int64_t)1 << 29)) xsum_normalize(a);
+}
+
+/* The exact sum rounded once to fp64 (nearest, ties to even). */
+static double xsum_round(orc_xsum *a) {
+  xsum_normalize(a);
+  double sign = 1.0;
+  uint32_t mag[ORC_XLIMBS];
+  if (a->d[ORC_XLIMBS - 1] < 0) { /* magnitude = 0 - a, digit by digit */
+    sign = -1.0;
+    int64_t borrow = 0;
+    for (int i = 0; i < ORC_XLIMBS; ++i) {
+      int64_t v = -a->d[i] - borrow;
+      borrow = v < 0;
+      mag[i] = (uint32_t)(v + (borrow ? ((int64_t)1 << 32) : 0));
+    }
+  } else {
+    for (int i = 0; i < ORC_XLIMBS; ++i) mag[i] = (uint32_t)a->d[i];
+  }
+  int top = -1; /* index of the highest set bit */
+  for (int i = ORC_XLIMBS - 1; i >= 0 && top < 0; --i)
+    if (mag[i])
+      for (int b = 31; b >= 0; --b)
+        if ((mag[i] >> b) & 1u) { top = 32 * i + b; break; }
+  if (top < 0) return 0.0;
+#define XBIT(n) ((mag[(n) >> 5] >> ((n) & 31)) & 1u)
+  if (top <= 52) { /* fits in the fp64 significand: exact */
+    uint64_t v = 0;
+    for (int n = top; n >= 0; --n) v = (v << 1) | XBIT(n);
+    return sign * ldexp((double)v, -149);
+  }
+  uint64_t sig = 0;
+  for (int n = top; n >= top - 52; --n) sig = (sig << 1) | XBIT(n);
+  int round_bit = (int)XBIT(top - 53), sticky = 0;
+  for (int n = top - 54; n >= 0 && !sticky; --n) sticky = (int)XBIT(n);
+#undef XBIT
+  int exp = top - 52 - 149;
+  if (round_bit && (sticky || (sig & 1u))) {
+    ++sig;
+    if (sig == ((uint64_t)1 << 53)) { sig >>= 1; ++exp; }
+  }
+  return sign * ldexp((double)sig, exp);
+}
 
 void orc_backward_dx(const int8_t *codes, int64_t N, int64_t K,
                      const void *dy, int dydt, int64_t M, float gamma,
                      float *dx) {
   for (int64_t m = 0; m < M; ++m)
     for (int64_t k = 0; k < K; ++k) {
-      double S = 0.0;
-      for (int64_t r0 = 0; r0 < N; r0 += ORC_DX_CHUNK) {
-        double P = 0.0;
-        for (int64_t n = r0; n < N && n < r0 + ORC_DX_CHUNK; ++n) {
-          int q = codes[n * K + k];
-          double g = (double)load_f(dy, dydt, m * N + n);
-          if (q == 1)
-            P += g;
-          else if (q == -1)
-            P -= g;
-        }
-        S += P;
+      orc_xsum acc;
+      memset(&acc, 0, sizeof acc);
+      for (int64_t n = 0; n < N; ++n) {
+        int q = codes[n * K + k];
+        if (q == 1)
+          xsum_add(&acc, load_f(dy, dydt, m * N + n), +1);
+        else if (q == -1)
+          xsum_add(&acc, load_f(dy, dydt, m * N + n), -1);
       }
+      double S = xsum_round(&acc);
       dx[m * K + k] = (float)((double)gamma * S);
     }
 }

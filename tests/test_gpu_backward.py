@@ -1,8 +1,10 @@
 """GPU parity of the STE backward through the C ABI against the oracle.
 
-Both sides add in fp64 in the same fixed order and round once to fp32, so dx
-and dW are compared bit for bit (the fp32 tolerance of the spec, 1e-6
-relative, is the fallback bar; the kernels meet the stricter one)."""
+dW: both sides add in fp64 in token order and round once to fp32, so dW is
+compared bit for bit.  dx: the oracle's sum over the rows is exact (no order),
+rounded once to fp64; the kernel may add in any order, so dx is compared
+within one fp32 ulp plus the fp64 rounding bound of an N-term sum
+(gamma N 2^-52 sum |dy|), see ``assert_dx_close``."""
 import numpy as np
 import pytest
 import torch
@@ -40,6 +42,26 @@ def _weights(orc, N, K, fmt, seed):
     return g, packed, orc.unpack(packed, N, K, fmt)
 
 
+def _widen(dy):
+    return (dy.astype(np.uint32) << 16).view(np.float32) if dy.dtype == np.uint16 else dy
+
+
+def assert_dx_close(dx, ref, codes, dy, g):
+    """dx against the exact-sum oracle: a sum of N terms in fp64 in any order
+    is within (N - 1) 2^-53 sum |term| of the exact sum; scaled by gamma (one
+    more fp64 rounding) and rounded to fp32, two such values differ by at most
+    one fp32 ulp of the larger plus gamma N 2^-52 sum |q dy|."""
+    N = codes.shape[0]
+    mag = np.abs(_widen(dy)).astype(np.float64) @ np.abs(codes).astype(np.float64)
+    big = np.maximum(np.abs(dx), np.abs(ref)).astype(np.float32)
+    tol = np.spacing(big).astype(np.float64) + float(g) * N * 2.0 ** -52 * mag
+    err = np.abs(dx.astype(np.float64) - ref.astype(np.float64))
+    bad = ~(err <= tol)
+    assert not bad.any(), f"{bad.sum()} dx entries outside the bound; first at {np.argwhere(bad)[:3].tolist()}"
+    # the bound is loose only where the sum cancels; report how many are bit-equal
+    return float(np.mean(dx.view(np.uint32) == ref.view(np.uint32)))
+
+
 def run_dx(packed, fmt, g, N, K, dy):
     M = dy.shape[0]
     dx = torch.full((M, K), float("nan"), dtype=torch.float32, device="cuda")
@@ -65,7 +87,7 @@ def test_backward_dx(orc, M, N, K, fmt, dydt):
         dy = synth.to_bf16_bits(dy)
     dx = run_dx(packed, fmt, g, N, K, dy)
     ref = orc.backward_dx(codes, dy, g, parallel=True)
-    assert np.array_equal(dx.view(np.uint32), ref.view(np.uint32))
+    assert_dx_close(dx, ref, codes, dy, g)
 
 
 def run_dw(dy, xq, s, g, N, K):
@@ -123,4 +145,4 @@ def test_backward_after_forward_chain(orc):
     assert np.array_equal(host(xq), xq_ref)
     assert np.array_equal(host(dw).view(np.uint32), orc.backward_dw(dy, xq_ref, s_ref, g).view(np.uint32))
     codes = orc.unpack(packed, N, K, I2)
-    assert np.array_equal(dx.view(np.uint32), orc.backward_dx(codes, dy, g).view(np.uint32))
+    assert_dx_close(dx, orc.backward_dx(codes, dy, g), codes, dy, g)

@@ -1,10 +1,16 @@
 """Pins for the oracle's STE backward (CPU only).
 
-The pins: exact integer arithmetic (integer gradients and a power-of-two gamma
-make every sum exact, so the fp32 results equal numpy's int64 products), torch
-autograd of the pages' straight-through construction (W_eff = W_q + W -
-W.detach(), the same for the activations, gamma held constant) in float64,
-bf16 gradients equal to their fp32 widening, and the degenerate cases."""
+The pins: the exact sum of dx checked against Python's ``math.fsum`` (the
+correctly rounded fp64 sum of its inputs, which is dx's definition before the
+gamma product) on wide-range gradients, hand cases where any fixed fp64 order
+loses bits (cancellation, a rounding decided by a far-away term, subnormals),
+exact integer arithmetic (integer gradients and a power-of-two gamma make every
+sum exact, so the fp32 results equal numpy's int64 products), torch autograd of
+the pages' straight-through construction (W_eff = W_q + W - W.detach(), the
+same for the activations, gamma held constant) in float64, bf16 gradients
+equal to their fp32 widening, and the degenerate cases."""
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -19,14 +25,62 @@ def _codes(rng, N, K, p0=0.3):
 
 @pytest.mark.parametrize("M,N,K", [(1, 5, 7), (3, 777, 100), (2, 1000, 33), (1, 64, 16), (1, 65, 16)])
 def test_dx_exact_on_integers(orc, M, N, K):
-    """Integer dy and gamma = 0.5: every partial sum is an exact integer, so
-    the chunk order is immaterial and dx = 0.5 (dy . W_q) exactly."""
+    """Integer dy and gamma = 0.5: the sum is an exact integer and
+    dx = 0.5 (dy . W_q) exactly."""
     rng = np.random.default_rng(N)
     codes = _codes(rng, N, K)
     dy = rng.integers(-1000, 1001, size=(M, N)).astype(np.float32)
     dx = orc.backward_dx(codes, dy, 0.5)
     want = (dy.astype(np.int64) @ codes.astype(np.int64)).astype(np.float64) * 0.5
     assert np.array_equal(dx, want.astype(np.float32))
+
+
+def _fsum_dx(codes, dy, g):
+    """dx by its definition with a library routine for the exact sum:
+    fp32(gamma * fsum(q dy)), fsum being the correctly rounded fp64 sum."""
+    M, N = dy.shape
+    K = codes.shape[1]
+    out = np.empty((M, K), np.float32)
+    for m in range(M):
+        for k in range(K):
+            terms = [float(dy[m, n]) * int(codes[n, k]) for n in range(N) if codes[n, k]]
+            out[m, k] = np.float32(float(np.float32(g)) * math.fsum(terms))
+    return out
+
+
+@pytest.mark.parametrize("g", [1.0, 0.37, 3.0e-3])
+def test_dx_is_the_exact_sum_rounded_once(orc, g):
+    """Gradients spread over 2^-60 .. 2^60, so every fixed fp64 order loses
+    bits somewhere: dx equals fp32(gamma * fsum(q dy)) bit for bit."""
+    rng = np.random.default_rng(11)
+    M, N, K = 3, 400, 24
+    codes = _codes(rng, N, K)
+    dy = (rng.standard_normal((M, N)) * np.exp2(rng.integers(-60, 61, size=(M, N)))).astype(np.float32)
+    dy[:, ::7] = -np.roll(dy, 1, axis=1)[:, ::7]  # planted cancellations
+    assert np.array_equal(orc.backward_dx(codes, dy, g).view(np.uint32), _fsum_dx(codes, dy, g).view(np.uint32))
+
+
+def test_dx_hand_cases(orc):
+    one = np.ones((4, 1), np.int8)
+    # cancellation: 1e30 + 1 - 1e30 is 1 exactly (0 in left-to-right fp64)
+    dy = np.array([[1e30, 1.0, -1e30, 0.0]], np.float32)
+    assert orc.backward_dx(one, dy, 1.0)[0, 0] == 1.0
+    # 1 + 2^-24 + 2^-53 + 2^-80: the far term makes fp64 round up, past fp32's tie
+    dy = np.array([[1.0, 2.0 ** -24, 2.0 ** -53, 2.0 ** -80]], np.float32)
+    assert orc.backward_dx(one, dy, 1.0)[0, 0] == np.float32(1.0 + 2.0 ** -23)
+    # without the far term it is an fp32 tie, to even
+    dy = np.array([[1.0, 2.0 ** -24, 0.0, 0.0]], np.float32)
+    assert orc.backward_dx(one, dy, 1.0)[0, 0] == np.float32(1.0)
+    # subnormals add exactly
+    tiny = np.float32(2.0 ** -149)
+    dy = np.array([[tiny, tiny, tiny, -tiny]], np.float32)
+    assert orc.backward_dx(one, dy, 1.0)[0, 0] == np.float32(2.0 ** -148)
+    # largest magnitudes: 3 x FLT_MAX - 2 x FLT_MAX, and the sign of -q dy
+    big = np.finfo(np.float32).max
+    dy = np.array([[big, big, big, 0.0]], np.float32)
+    codes = np.array([[1], [1], [-1], [0]], np.int8)
+    assert orc.backward_dx(codes, dy, 1.0)[0, 0] == big
+    assert orc.backward_dx(codes, -dy, 0.5)[0, 0] == -big / 2
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 6, 9), (5, 40, 300), (64, 3, 17)])

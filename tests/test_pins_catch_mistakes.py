@@ -37,7 +37,10 @@ MISTAKES = [
     ("onebit_alpha_of_abs", "return fixed_order_sum(W, dt, N, K, 0);", "return fixed_order_sum(W, dt, N, K, 1);"),
     ("onebit_bits_reversed", "if (q > 0) byte |= 1u << i;", "if (q > 0) byte |= 0x80u >> i;"),
     ("backward_dx_without_gamma", "dx[m * K + k] = (float)((double)gamma * S);", "dx[m * K + k] = (float)S;"),
-    ("backward_dx_sign", "P -= g;", "P += g;"),
+    ("backward_dx_sign", "load_f(dy, dydt, m * N + n), -1);", "load_f(dy, dydt, m * N + n), +1);"),
+    ("exact_sum_drops_high_digit", "a->d[i + 1] += sign * hi;", "a->d[i + 1] += 0 * hi;"),
+    ("exact_sum_without_sticky_bit", "if (round_bit && (sticky || (sig & 1u))) {", "if (round_bit && (sig & 1u)) {"),
+    ("exact_sum_subnormal_shift", "int shift = e ? (int)e - 1 : 0;", "int shift = e ? (int)e : 0;"),
     ("backward_dw_without_scale", "T += t * c;", "T += t;"),
     ("backward_dw_k_reversed", "(double)xq[m * K + k];", "(double)xq[m * K + (K - 1 - k)];"),
     ("layernorm_unbiased_variance", "const double var = token_tree_sum(lane) / (double)K;",
