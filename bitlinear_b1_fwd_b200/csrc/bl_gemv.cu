@@ -16,6 +16,7 @@
 // sums meet by warp reduction; the dequantization y = acc * (gamma s / 127)
 // ("§5.3") is fused into the store.
 #include "bl_common.cuh"
+#include "bl_gemv.cuh"
 #include "bl_kernels.h"
 
 namespace bl {
@@ -25,13 +26,6 @@ constexpr int kGemvWarps = kGemvThreads / 32;
 constexpr int kGemvBatch = 4;         // items per load batch; two batches per warp alternate
 constexpr int kGemvTileRows = 1024;   // rows whose sums a CTA holds in shared memory at a time
 
-__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
-  uint4 v;
-  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
 
 // Activation bytes per token in shared memory for one packed row of rowbytes.
 __host__ __device__ inline int64_t gemv_x_bytes(int fmt, int64_t rowbytes) {
@@ -43,12 +37,6 @@ __host__ __device__ inline int64_t gemv_smem_bytes(int fmt, int64_t rowbytes, in
   return mt * gemv_x_bytes(fmt, rowbytes) + int64_t{4} * mt * kGemvTileRows + (fmt == BL_PACK_T5 ? 256 * 8 : 0);
 }
 
-// dp4a with unsigned bytes in a and signed bytes in b.
-__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
-  int d;
-  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
 
 template <int XDT>
 __device__ __forceinline__ float load_x(const void* x, int64_t i) {
@@ -78,19 +66,7 @@ __device__ __forceinline__ uint32_t x_slot(int fmt, uint32_t k, uint32_t segs) {
   }
 }
 
-// The four bytes q[0..3] (low byte of each) as one word, q[0] in the low byte.
-__device__ __forceinline__ uint32_t pack4(const int* q) {
-  return __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
-}
 
-// The 2-bit layout's 16-byte slot of the 16 codes q[0..15] of one packed word:
-// byte 4j + b = q[4b + j], a 4 x 4 byte transpose of P_b = q[4b .. 4b + 3].
-__device__ __forceinline__ uint4 i2_slot(uint32_t P0, uint32_t P1, uint32_t P2, uint32_t P3) {
-  const uint32_t t0 = __byte_perm(P0, P1, 0x5140), t1 = __byte_perm(P2, P3, 0x5140);
-  const uint32_t t2 = __byte_perm(P0, P1, 0x7362), t3 = __byte_perm(P2, P3, 0x7362);
-  return make_uint4(__byte_perm(t0, t1, 0x5410), __byte_perm(t0, t1, 0x7632), __byte_perm(t2, t3, 0x5410),
-                    __byte_perm(t2, t3, 0x7632));
-}
 
 // Work split.  CTA b owns the rows [row0, row0 + nrows) (the N rows shared
 // out as evenly as the grid allows); they are contiguous in memory, and the CTA
@@ -1509,6 +1485,8 @@ cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int6
   // are not served here (the caller transcodes them to 2 bits)
   const bool lean = (fmt == BL_PACK_I2 && rowbytes <= 2 * kI2Plane) || (fmt == BL_PACK_B1 && rowbytes <= kI2Plane);
   if (fmt == BL_PACK_B1 && !lean) return cudaErrorInvalidValue;
+  if (fmt == BL_PACK_I2 && M == 1 && gemv1_fits(N, K, rowbytes, xdt))
+    return launch_gemv1(packed, rowbytes, gamma, N, K, x, xdt, scale, y, ydt, rg, st);
   const int esz = (xdt == BL_F32) ? 4 : (xdt == BL_BF16 ? 2 : 1);
   const int ysz = (ydt == BL_BF16) ? 2 : 4;
   for (int64_t m0 = 0; m0 < M; m0 += mt_max) {

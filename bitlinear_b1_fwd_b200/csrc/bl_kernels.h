@@ -96,6 +96,14 @@ cudaError_t launch_backward_dx(const uint8_t* packed, int64_t rowbytes, const fl
 cudaError_t launch_backward_dw(const void* dy, int dydt, const int8_t* xq, const float* scale, const float* gamma,
                                int64_t M, int64_t N, int64_t K, float* dw, cudaStream_t st);
 
+// One-token 2-bit GEMV (column-stationary, early start): K % 16 == 0, rows of
+// at most 8192 bytes, and fp32 tokens only when K is small enough for the raw
+// token words of a thread to fit (see gemv1_fits).
+bool gemv1_fits(int64_t N, int64_t K, int64_t rowbytes, int xdt);
+cudaError_t launch_gemv1(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
+                         const void* x, int xdt, float* scale, void* y, int ydt, const RowGroups& rg,
+                         cudaStream_t st);
+
 cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int64_t N, int64_t K,
                         const void* x, int xdt, float* scale, int64_t M, void* y, int ydt,
                         const RowGroups& rg, cudaStream_t st);
