@@ -204,7 +204,7 @@ bl_status bitlinear_forward(const uint8_t* packed, int fmt, const float* gamma, 
       fmt = BL_PACK_I2;
     }
     if (bl::gemv_max_tokens(fmt, bitlinear_packed_row_bytes(K, fmt)) < 1) return BL_ERR_UNSUPPORTED;
-    return cuda_status(bl::launch_gemv(packed, fmt, gamma, N, K, x, xdt, scale, M, y, ydt, bl::one_group(N), st));
+    return cuda_status(bl::launch_gemv(packed, fmt, gamma, N, K, x, xdt, scale, M, y, ydt, bl::one_group(N), ws, st));
   }
   uint8_t* scratch = static_cast<uint8_t*>(ws) + BL_WS_HEADER_BYTES;
   const int8_t* xq = static_cast<const int8_t*>(x);
@@ -294,7 +294,7 @@ bl_status bitlinear_forward_grouped(const uint8_t* packed, int fmt, const float*
     rg.n = static_cast<int>(ngroups);
     int64_t end = 0;
     for (int64_t g = 0; g < ngroups; ++g) rg.end[g] = (end += group_rows[g]);
-    return cuda_status(bl::launch_gemv(packed, fmt, gammas, N, K, x, xdt, scale, M, y, ydt, rg, st));
+    return cuda_status(bl::launch_gemv(packed, fmt, gammas, N, K, x, xdt, scale, M, y, ydt, rg, ws, st));
   }
   // one activation quantization, then each group's product into its columns of y
   uint8_t* scratch = static_cast<uint8_t*>(ws) + BL_WS_HEADER_BYTES;

@@ -1474,7 +1474,7 @@ static cudaError_t launch_gemv_mt(int mt, const uint8_t* packed, int64_t rowbyte
 // Runs the GEMV over all M tokens in groups that fit in shared memory.
 cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int64_t N, int64_t K,
                         const void* x, int xdt, float* scale, int64_t M, void* y, int ydt,
-                        const RowGroups& rg, cudaStream_t st) {
+                        const RowGroups& rg, void* ws, cudaStream_t st) {
   const int per = (fmt == BL_PACK_I2) ? 4 : (fmt == BL_PACK_T5 ? 5 : 8);
   const int64_t rowbytes = ((K + per - 1) / per + 15) / 16 * 16;
   const int mt_max = gemv_max_tokens(fmt, rowbytes);
@@ -1486,7 +1486,7 @@ cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int6
   const bool lean = (fmt == BL_PACK_I2 && rowbytes <= 2 * kI2Plane) || (fmt == BL_PACK_B1 && rowbytes <= kI2Plane);
   if (fmt == BL_PACK_B1 && !lean) return cudaErrorInvalidValue;
   if (fmt == BL_PACK_I2 && M == 1 && gemv1_fits(N, K, rowbytes, xdt))
-    return launch_gemv1(packed, rowbytes, gamma, N, K, x, xdt, scale, y, ydt, rg, st);
+    return launch_gemv1(packed, rowbytes, gamma, N, K, x, xdt, scale, y, ydt, rg, ws, st);
   const int esz = (xdt == BL_F32) ? 4 : (xdt == BL_BF16 ? 2 : 1);
   const int ysz = (ydt == BL_BF16) ? 2 : 4;
   for (int64_t m0 = 0; m0 < M; m0 += mt_max) {

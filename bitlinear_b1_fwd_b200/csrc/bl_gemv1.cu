@@ -32,21 +32,19 @@
 #include "bl_common.cuh"
 #include "bl_gemv.cuh"
 #include "bl_kernels.h"
+#include "bl_sm100.cuh"
 
 #ifndef BL_G1_PREFETCH
 #define BL_G1_PREFETCH 65536  // bytes of each CTA's rows prefetched into L2 before the wait
+#endif
+#ifndef BL_G1_PREFETCH2
+#define BL_G1_PREFETCH2 0  // bytes prefetched into L2 after the wait, while the token is quantized
 #endif
 
 namespace bl {
 
 constexpr int kG1MaxThreads = 512;
-constexpr int64_t kG1MaxSmem = 96 * 1024;  // two CTAs (of consecutive launches) per SM
-
-// Shared memory: the raw token (K elements), its codes (64 per segment) and
-// the CTA's row sums.
-__host__ __device__ inline int64_t gemv1_smem_bytes(int64_t rowbytes, int64_t K, int xsize, int64_t rows_per_cta) {
-  return (K * xsize + 15) / 16 * 16 + rowbytes * 4 + 4 * rows_per_cta;
-}
+constexpr int64_t kG1MaxSmem = 110 * 1024;  // two CTAs (of consecutive launches) per SM
 
 // 16-byte words of raw activations per 16 elements.
 template <int XDT>
@@ -54,22 +52,44 @@ constexpr int g1_xwords() {
   return XDT == BL_F32 ? 4 : (XDT == BL_BF16 ? 2 : 1);
 }
 
-constexpr int kG1Depth = 6;  // 16-byte weight loads in flight per thread
+// Stages of a thread's row ring: rows copied ahead into shared memory by
+// cp.async (no registers held, and no per-warp limit on loads in flight).
+constexpr int kG1StagesMax = 8;
+constexpr long long kG1WaitCycles = 1ll << 30;  // bound of the token wait (~0.5 s)
 
-// 16-byte copy global -> shared without registers (L2 only).
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+// 16-byte copy global -> shared (at a shared-window address) without
+// registers, through L2 only.
+__device__ __forceinline__ void cp_async16_s(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_add_s(uint32_t a, int v) {
+  asm volatile("red.shared.add.s32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
-// sum over the 64 weights of a segment of d x, d the stored digit: the mask
+// Bytes of the token region: the raw token, and later its codes in the slot
+// layout (4 x 16 bytes per segment), whichever is larger.
+__host__ __device__ inline int64_t g1_xregion(int64_t K, int xwords, int64_t rowbytes) {
+  const int64_t raw = K * xwords;  // xwords 16-byte words per 16 elements: K * xwords bytes
+  return ((raw > rowbytes * 4 ? raw : rowbytes * 4) + 15) / 16 * 16;
+}
+
+// a0 + sum over the 64 weights of a segment of d x, d the stored digit: the mask
 // w & (3 << 2j) leaves digit j of every byte in place (4^j d), so accumulator
 // j collects 4^j sum d x and the factor comes off exactly with a shift.
 // X[w] byte 4j + b holds the code of weight 16 w + 4 b + j of the segment.
-__device__ __forceinline__ int dot_seg_i2(const uint4 wv, const uint4 (&X)[4]) {
+__device__ __forceinline__ int dot_seg_i2(const uint4 wv, const uint4 (&X)[4], int a0) {
   const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
-  int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+  int a1 = 0, a2 = 0, a3 = 0;
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
     a0 = dp4a_us(wd[w] & 0x03030303u, X[w].x, a0);
@@ -80,20 +100,59 @@ __device__ __forceinline__ int dot_seg_i2(const uint4 wv, const uint4 (&X)[4]) {
   return a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6);
 }
 
+// The INT8 codes of 16 activations e[0..15] against scale s (c127 =
+// fl(127 / s)), returned as the 16-byte slot of their packed word (byte
+// 4j + b = code of element 4b + j).  Each code is rint(fl(fl(e / s) 127)),
+// taken division-free as in quant_act_fast: t_a = fl(e c127) is within 2^-14
+// of t, so rint(t_a) = rint(t) unless t_a lies within 2^-14 of a
+// half-integer.  rint(t_a) comes from the adder (t_a + 1.5 * 2^23 rounds to
+// nearest even and leaves the code in the low byte of the sum's bits, two's
+// complement, |code| <= 127), the margin is checked once per eight elements
+// on the largest |t_a - rint(t_a)| (an exact difference), and only a group
+// with an element that close to a tie takes the exact quotient.
+__device__ __forceinline__ uint4 g1_codes16(const float (&e)[16], float s, float c127) {
+  uint32_t r[16];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float worst = 0.0f;
+#pragma unroll
+    for (int j = 8 * h; j < 8 * h + 8; ++j) {
+      const float ta = __fmul_rn(e[j], c127);
+      const float r2 = __fadd_rn(ta, 12582912.0f);
+      worst = fmaxf(worst, fabsf(__fsub_rn(ta, __fsub_rn(r2, 12582912.0f))));
+      r[j] = __float_as_uint(r2);
+    }
+    if (!(worst < 0.49993896484375f)) {  // rare: some element is near a tie
+#pragma unroll
+      for (int j = 8 * h; j < 8 * h + 8; ++j) {
+        const float ta = __fmul_rn(e[j], c127);
+        if (!(fabsf(__fsub_rn(ta, rintf(ta))) < 0.49993896484375f))
+          r[j] = static_cast<uint32_t>(quant_act_slow(e[j], s));
+      }
+    }
+  }
+  uint32_t w[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    w[j] = __byte_perm(__byte_perm(r[j], r[4 + j], 0x0040), __byte_perm(r[8 + j], r[12 + j], 0x0040), 0x5410);
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // XC: 16-element chunks of the token per thread (the chunks of segment c are
-// 4c .. 4c + 3; chunk g of thread t is t + T u, u < XC).
-template <int XDT, int XC>
+// 4c .. 4c + 3; chunk g of thread t is t + T u, u < XC).  S: stages of the
+// thread's row ring.  ALIGNED: segs % 32 == 0, so every warp lies in one row.
+template <int XDT, int XC, int S, bool ALIGNED>
 __global__ void __launch_bounds__(kG1MaxThreads, 2)
     gemv1_i2_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
                     int64_t N, int64_t K, const void* __restrict__ x, float* __restrict__ scale,
-                    void* __restrict__ y, int ydt, int write_scale, const RowGroups rg, int R) {
-  constexpr int D = kG1Depth;
+                    void* __restrict__ y, int ydt, int write_scale, const RowGroups rg, int R, void* ws) {
   constexpr int kXW = g1_xwords<XDT>();
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ uint32_t red[kG1MaxThreads / 32];
   __shared__ float sh_gam[kMaxRowGroups];
   __shared__ int64_t sh_end[kMaxRowGroups];
   __shared__ float sh_s;
+  __shared__ __align__(8) uint64_t xbar;  // completion of the token's bulk copy
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int T = blockDim.x;
@@ -110,11 +169,18 @@ __global__ void __launch_bounds__(kG1MaxThreads, 2)
   const uint32_t step = static_cast<uint32_t>(R * rowbytes);  // bytes between a thread's rows (<= 8 KB)
   const int kch = static_cast<int>(K >> 4);  // chunks holding weights (K % 16 == 0)
   const int nch = 4 * segs;                  // chunks of the packed rows (the last ones are padding)
-  uint8_t* xraw = smem;                                             // [K] raw token
-  uint8_t* xs = smem + (K * kXW + 15) / 16 * 16;                    // [4][segs] 16-byte code slots
-  int* rsum = reinterpret_cast<int*>(xs + rowbytes * 4);           // [nrows]
+  const uint32_t xbytes = static_cast<uint32_t>(K * kXW);  // raw token bytes (a multiple of 16)
+  // shared memory: the token region (first the raw token, then its codes in
+  // the slot layout [4][segs] x 16 bytes), the row ring [S][T] x 16 bytes,
+  // the row sums [nrows]
+  const int64_t xreg = g1_xregion(K, kXW, rowbytes);
+  uint8_t* xbuf = smem;
+  const uint32_t ring_s = smem_u32(smem + xreg) + 16u * tid;       // slot 0 of this thread
+  const uint32_t tstride = 16u * T;                                 // bytes between its slots
+  int* rsum = reinterpret_cast<int*>(smem + xreg + static_cast<int64_t>(S) * T * 16);
 
-  // 0. before the wait: the first bytes of the CTA's rows into L2
+  // 0. before the wait: the first bytes of the CTA's rows into L2, the row
+  //    sums zeroed, the token barrier set up
   {
     const int64_t bytes = static_cast<int64_t>(nrows) * rowbytes;
     l2_prefetch_bulk(packed + row0 * rowbytes, bytes < BL_G1_PREFETCH ? bytes : BL_G1_PREFETCH);
@@ -123,59 +189,77 @@ __global__ void __launch_bounds__(kG1MaxThreads, 2)
 #pragma unroll
   for (int i = 0; i < kMaxRowGroups; ++i)
     if (tid == i) sh_end[i] = rg.end[i];
+  if (tid == 0) {
+    mbar_init(&xbar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
   pdl_wait(packed, gamma, x, scale, y);
   pdl_launch_dependents();
 
-  // 1. the token into shared memory, and the first D rows of this thread
-  //    into registers, all in flight together
-#pragma unroll
-  for (int u = 0; u < XC; ++u) {
-    const int g = tid + T * u;
-    if (g < kch)
-#pragma unroll
-      for (int i = 0; i < kXW; ++i)
-        cp_async16(xraw + (static_cast<int64_t>(g) * kXW + i) * 16,
-                   static_cast<const uint8_t*>(x) + (static_cast<int64_t>(g) * kXW + i) * 16);
+  // 1. while the token is read and quantized the memory system would idle:
+  //    the next part of the CTA's rows moves into L2 meanwhile
+  if (BL_G1_PREFETCH2 > 0) {
+    const int64_t bytes = static_cast<int64_t>(nrows) * rowbytes;
+    const int64_t lo = bytes < BL_G1_PREFETCH ? bytes : BL_G1_PREFETCH;
+    const int64_t hi = bytes < lo + BL_G1_PREFETCH2 ? bytes : lo + BL_G1_PREFETCH2;
+    if (hi > lo) l2_prefetch_bulk(packed + row0 * rowbytes + lo, hi - lo);
   }
-  const uint8_t* lp = packed + row0 * rowbytes + static_cast<int64_t>(tid) * 16;  // next load
-  uint4 buf[D];
-#pragma unroll
-  for (int j = 0; j < D; ++j) {
-    buf[j] = make_uint4(0, 0, 0, 0);
-    if (j < nr) buf[j] = ld_stream(reinterpret_cast<const uint4*>(lp));
-    lp += step;
+  // 1. the token by one bulk copy; the rows follow once it has landed (row
+  //    copies issued alongside slow the token's copy several fold, and the
+  //    token is on the critical path while the rows have the whole
+  //    quantization to arrive)
+  if (tid == 0) {
+    mbar_expect_tx(&xbar, xbytes);
+    bulk_load(xbuf, x, xbytes, &xbar);
   }
   if (tid < rg.n) sh_gam[tid] = __ldcg(gamma + tid);
   if (XDT == BL_I8 && tid == 0) sh_s = __ldcg(scale);
-  cp_async_wait_all();
-  __syncthreads();  // the raw token, zeroed row sums, gammas and the given scale are visible
+  // every thread waits (bounded) for the token; if any gives up, the CTA
+  // records the timeout, lets the copy land (bounded) and leaves
+  const bool got = wait_drain(&xbar, 0, kG1WaitCycles);
+  if (__syncthreads_or(!got)) {  // also: zeroed row sums, gammas and the given scale are visible
+    if (tid == 0) {
+      set_flag(ws, kFlagTimeout, 0x601);
+      wait_drain(&xbar, 0, kG1WaitCycles);
+    }
+    return;
+  }
+  // the thread's first S - 1 rows (one cp.async group each, empty past its rows)
+  const uint8_t* gp = packed + row0 * rowbytes + static_cast<int64_t>(tid) * 16;  // next row to copy
+#pragma unroll
+  for (int j = 0; j < S - 1; ++j) {
+    if (j < nr) cp_async16_s(ring_s + j * tstride, gp);
+    cp_async_commit();
+    gp += step;
+  }
 
-  // 2. per-token absmax (fmaxf, so a NaN is ignored; the result is a
-  //    non-negative float, whose bits order like unsigned integers)
+  // 2. per-token absmax.  The inputs are finite, so the magnitude bits
+  //    (sign cleared) order like unsigned integers: the maximum is taken on
+  //    them, two bf16 values per 32-bit word at a time.
   float s;
   if constexpr (XDT != BL_I8) {
-    float amax = 0.0f;
+    uint32_t mx = 0;  // fp32: magnitude bits; bf16: two 16-bit magnitudes
 #pragma unroll
     for (int u = 0; u < XC; ++u) {
       const int g = tid + T * u;
       if (g < kch)
 #pragma unroll
         for (int i = 0; i < kXW; ++i) {
-          const uint4 v = *reinterpret_cast<const uint4*>(xraw + (static_cast<int64_t>(g) * kXW + i) * 16);
+          const uint4 v = *reinterpret_cast<const uint4*>(xbuf + (static_cast<int64_t>(g) * kXW + i) * 16);
           if constexpr (XDT == BL_F32) {
-            amax = fmaxf(fmaxf(amax, fabsf(__uint_as_float(v.x))), fabsf(__uint_as_float(v.y)));
-            amax = fmaxf(fmaxf(amax, fabsf(__uint_as_float(v.z))), fabsf(__uint_as_float(v.w)));
+            const uint32_t a = max(v.x & 0x7fffffffu, v.y & 0x7fffffffu);
+            const uint32_t b2 = max(v.z & 0x7fffffffu, v.w & 0x7fffffffu);
+            mx = max(mx, max(a, b2));
           } else {
-            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              amax = fmaxf(amax, fabsf(__uint_as_float(wv[h] << 16)));
-              amax = fmaxf(amax, fabsf(__uint_as_float(wv[h] & 0xffff0000u)));
-            }
+            const uint32_t a = __vmaxu2(v.x & 0x7fff7fffu, v.y & 0x7fff7fffu);
+            const uint32_t b2 = __vmaxu2(v.z & 0x7fff7fffu, v.w & 0x7fff7fffu);
+            mx = __vmaxu2(mx, __vmaxu2(a, b2));
           }
         }
     }
-    const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+    if constexpr (XDT == BL_BF16) mx = max(mx & 0xffffu, mx >> 16) << 16;  // as fp32 bits
+    const uint32_t m = __reduce_max_sync(0xffffffffu, mx);
     if (lane == 0) red[warp] = m;
     __syncthreads();
     uint32_t mm = 0;
@@ -185,89 +269,110 @@ __global__ void __launch_bounds__(kG1MaxThreads, 2)
     s = sh_s;
   }
 
-  // 3. the codes, written in the slot layout of the packed words
+  // 3. the codes of the thread's chunks (from the raw token), then, once every
+  //    thread has read its raw chunks, written over the token region in the
+  //    slot layout of the packed words
   {
     const float c127 = (XDT == BL_I8) ? 0.0f : __fdiv_rn(127.0f, s);
+    uint4 slot[XC];
 #pragma unroll
     for (int u = 0; u < XC; ++u) {
       const int g = tid + T * u;
-      if (g < nch) {
-        uint32_t P[4] = {0u, 0u, 0u, 0u};  // padding chunks (past K): code 0
-        if (g < kch) {
-          const uint8_t* src = xraw + static_cast<int64_t>(g) * kXW * 16;
-          if constexpr (XDT == BL_I8) {
-            const uint4 v = *reinterpret_cast<const uint4*>(src);
-            P[0] = v.x;
-            P[1] = v.y;
-            P[2] = v.z;
-            P[3] = v.w;
+      uint32_t P[4] = {0u, 0u, 0u, 0u};  // padding chunks (past K): code 0
+      if (g < kch) {
+        const uint8_t* src = xbuf + static_cast<int64_t>(g) * kXW * 16;
+        if constexpr (XDT == BL_I8) {
+          const uint4 v = *reinterpret_cast<const uint4*>(src);
+          P[0] = v.x;
+          P[1] = v.y;
+          P[2] = v.z;
+          P[3] = v.w;
+        } else {
+          float e[16];
+          if constexpr (XDT == BL_F32) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * i);
+              e[4 * i] = __uint_as_float(v.x); e[4 * i + 1] = __uint_as_float(v.y);
+              e[4 * i + 2] = __uint_as_float(v.z); e[4 * i + 3] = __uint_as_float(v.w);
+            }
           } else {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {  // eight elements at a time
-              float e[8];
-              if constexpr (XDT == BL_F32) {
-                const uint4 v0 = *reinterpret_cast<const uint4*>(src + 32 * h);
-                const uint4 v1 = *reinterpret_cast<const uint4*>(src + 32 * h + 16);
-                e[0] = __uint_as_float(v0.x); e[1] = __uint_as_float(v0.y);
-                e[2] = __uint_as_float(v0.z); e[3] = __uint_as_float(v0.w);
-                e[4] = __uint_as_float(v1.x); e[5] = __uint_as_float(v1.y);
-                e[6] = __uint_as_float(v1.z); e[7] = __uint_as_float(v1.w);
-              } else {
-                const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * h);
-                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+            for (int i = 0; i < 2; ++i) {
+              const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * i);
+              const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  e[2 * k] = __uint_as_float(wv[k] << 16);
-                  e[2 * k + 1] = __uint_as_float(wv[k] & 0xffff0000u);
-                }
+              for (int k = 0; k < 4; ++k) {
+                e[8 * i + 2 * k] = __uint_as_float(wv[k] << 16);
+                e[8 * i + 2 * k + 1] = __uint_as_float(wv[k] & 0xffff0000u);
               }
-              int q[8];
-              quant_act_fast_n<8>(e, s, c127, q);
-              P[2 * h] = pack4(q);
-              P[2 * h + 1] = pack4(q + 4);
             }
           }
+          slot[u] = g1_codes16(e, s, c127);
+          continue;
         }
-        *reinterpret_cast<uint4*>(xs + (static_cast<int64_t>(g & 3) * segs + (g >> 2)) * 16) =
-            i2_slot(P[0], P[1], P[2], P[3]);
       }
+      slot[u] = i2_slot(P[0], P[1], P[2], P[3]);
+    }
+    __syncthreads();  // every raw chunk has been read
+#pragma unroll
+    for (int u = 0; u < XC; ++u) {
+      const int g = tid + T * u;
+      if (g < nch) *reinterpret_cast<uint4*>(xbuf + (static_cast<int64_t>(g & 3) * segs + (g >> 2)) * 16) = slot[u];
     }
   }
   __syncthreads();
 
   // 4. this thread's 64 codes and their sum (digits are q + 1: the sum is
-  //    taken off once per row)
+  //    taken off once per row, as the starting value of the row's sum)
   uint4 X[4];
   int csum = 0;
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
-    X[w] = active ? *reinterpret_cast<const uint4*>(xs + (static_cast<int64_t>(w) * segs + c) * 16)
+    X[w] = active ? *reinterpret_cast<const uint4*>(xbuf + (static_cast<int64_t>(w) * segs + c) * 16)
                   : make_uint4(0, 0, 0, 0);
     csum = __dp4a(static_cast<int>(X[w].x), 0x01010101, csum);
     csum = __dp4a(static_cast<int>(X[w].y), 0x01010101, csum);
     csum = __dp4a(static_cast<int>(X[w].z), 0x01010101, csum);
     csum = __dp4a(static_cast<int>(X[w].w), 0x01010101, csum);
   }
+  const int init = -csum;
   // lanes with the same first row share a row at every step
-  const uint32_t gmask = __match_any_sync(0xffffffffu, active ? r0 : -1 - lane);
-  const bool leader = (__ffs(gmask) - 1) == lane;
+  const uint32_t gmask = ALIGNED ? 0xffffffffu : __match_any_sync(0xffffffffu, active ? r0 : -1 - lane);
+  const bool leader = ALIGNED ? lane == 0 : (__ffs(gmask) - 1) == lane;
+  uint32_t rs = smem_u32(rsum + r0);    // this thread's next row sum
+  const uint32_t rstep = 4u * R;
 
-  // 5. the stream: consume the oldest load, refill its slot D rows ahead (the
-  //    lanes of a group take the same branches: same rows)
-  int* rs = rsum + r0;
-  for (int k0 = 0; k0 < nr; k0 += D) {
+  // 5. the stream: copy row k + S - 1 into the slot freed by row k - 1, wait
+  //    for row k, consume it (the lanes of a group take the same branches:
+  //    same rows); each thread reads back only its own slots.  Blocks of S
+  //    rows with no guard while every refill is a row of the thread, then
+  //    the rest one by one.
+  auto consume = [&](const uint4 wv) {
+    int v = dot_seg_i2(wv, X, init);
+    v = __reduce_add_sync(gmask, v);
+    if (leader) red_add_s(rs, v);
+    rs += rstep;
+  };
+  int k = 0;
+  for (; k < nr - 2 * S + 2; k += S) {
 #pragma unroll
-    for (int j = 0; j < D; ++j) {
-      if (k0 + j < nr) {
-        const uint4 wv = buf[j];
-        if (k0 + j + D < nr) buf[j] = ld_stream(reinterpret_cast<const uint4*>(lp));
-        lp += step;
-        const int v = __reduce_add_sync(gmask, dot_seg_i2(wv, X) - csum);
-        if (leader) atomicAdd(rs, v);
-        rs += R;
-      }
+    for (int j = 0; j < S; ++j) {
+      cp_async16_s(ring_s + ((j + S - 1) % S) * tstride, gp);
+      cp_async_commit();
+      gp += step;
+      cp_async_wait<S - 1>();
+      consume(lds128(ring_s + j * tstride));
     }
   }
+  for (; k < nr; ++k) {
+    if (k + S - 1 < nr) cp_async16_s(ring_s + ((k + S - 1) % S) * tstride, gp);
+    cp_async_commit();
+    gp += step;
+    cp_async_wait<S - 1>();
+    consume(lds128(ring_s + (k % S) * tstride));
+  }
+  cp_async_wait<0>();
   __syncthreads();  // every row sum is complete
 
   // 6. dequantize and store the CTA's outputs (coalesced)
@@ -294,7 +399,7 @@ __global__ void __launch_bounds__(kG1MaxThreads, 2)
 // Launch geometry: R rows per step, threads rounded up to whole warps, and
 // the token chunks per thread (1, 2 or 4).
 struct Gemv1Geom {
-  int R, threads, xc;
+  int R, threads, xc, stages;
   int64_t grid, rows_per_cta, smem;
 };
 
@@ -304,16 +409,20 @@ static bool gemv1_geom(int64_t N, int64_t K, int64_t rowbytes, int xdt, Gemv1Geo
   const int64_t sms = device_sms();
   g->grid = N < sms ? N : sms;
   g->rows_per_cta = (N + g->grid - 1) / g->grid;
-  const int xsize = xdt == BL_F32 ? 4 : (xdt == BL_BF16 ? 2 : 1);
-  g->smem = gemv1_smem_bytes(rowbytes, K, xsize, g->rows_per_cta);
-  if (g->smem > kG1MaxSmem) return false;
   int64_t R = kG1MaxThreads / segs;
   if (R > g->rows_per_cta) R = g->rows_per_cta;
   g->R = static_cast<int>(R);
   g->threads = static_cast<int>((R * segs + 31) / 32 * 32);
   const int64_t per = (4 * segs + g->threads - 1) / g->threads;
   g->xc = per <= 1 ? 1 : (per <= 2 ? 2 : 4);
-  return true;
+  const int xwords = xdt == BL_F32 ? 4 : (xdt == BL_BF16 ? 2 : 1);
+  const int64_t fixed = g1_xregion(K, xwords, rowbytes) + 4 * g->rows_per_cta;
+  for (int st : {kG1StagesMax, 6}) {  // the deepest ring that keeps two CTAs per SM
+    g->stages = st;
+    g->smem = fixed + int64_t{16} * st * g->threads;
+    if (g->smem <= kG1MaxSmem) return true;
+  }
+  return false;
 }
 
 bool gemv1_fits(int64_t N, int64_t K, int64_t rowbytes, int xdt) {
@@ -321,11 +430,11 @@ bool gemv1_fits(int64_t N, int64_t K, int64_t rowbytes, int xdt) {
   return gemv1_geom(N, K, rowbytes, xdt, &g);
 }
 
-template <int XDT, int XC>
+template <int XDT, int XC, int S>
 static cudaError_t launch_gemv1_t(const Gemv1Geom& g, const uint8_t* packed, int64_t rowbytes, const float* gamma,
                                   int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
-                                  int write_scale, const RowGroups& rg, cudaStream_t st) {
-  auto kern = gemv1_i2_kernel<XDT, XC>;
+                                  int write_scale, const RowGroups& rg, void* ws, cudaStream_t st) {
+  auto kern = (rowbytes / 16) % 32 == 0 ? gemv1_i2_kernel<XDT, XC, S, true> : gemv1_i2_kernel<XDT, XC, S, false>;
   const size_t smem = static_cast<size_t>(g.smem);
   if (smem > 48 * 1024) {
     const cudaError_t e =
@@ -333,28 +442,38 @@ static cudaError_t launch_gemv1_t(const Gemv1Geom& g, const uint8_t* packed, int
     if (e != cudaSuccess) return e;
   }
   const cudaError_t e = launch_pdl(kern, static_cast<unsigned>(g.grid), static_cast<unsigned>(g.threads), smem, st,
-                                   packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, g.R);
+                                   packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, g.R, ws);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+template <int XDT, int XC>
+static cudaError_t launch_gemv1_s(const Gemv1Geom& g, const uint8_t* packed, int64_t rowbytes, const float* gamma,
+                                  int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
+                                  int write_scale, const RowGroups& rg, void* ws, cudaStream_t st) {
+  if (g.stages == kG1StagesMax)
+    return launch_gemv1_t<XDT, XC, kG1StagesMax>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg,
+                                                 ws, st);
+  return launch_gemv1_t<XDT, XC, 6>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
 }
 
 template <int XDT>
 static cudaError_t launch_gemv1_x(const Gemv1Geom& g, const uint8_t* packed, int64_t rowbytes, const float* gamma,
                                   int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
-                                  int write_scale, const RowGroups& rg, cudaStream_t st) {
-  if (g.xc == 1) return launch_gemv1_t<XDT, 1>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
-  if (g.xc == 2) return launch_gemv1_t<XDT, 2>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
-  return launch_gemv1_t<XDT, 4>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, st);
+                                  int write_scale, const RowGroups& rg, void* ws, cudaStream_t st) {
+  if (g.xc == 1) return launch_gemv1_s<XDT, 1>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
+  if (g.xc == 2) return launch_gemv1_s<XDT, 2>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
+  return launch_gemv1_s<XDT, 4>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
 }
 
 cudaError_t launch_gemv1(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
-                         const void* x, int xdt, float* scale, void* y, int ydt, const RowGroups& rg,
+                         const void* x, int xdt, float* scale, void* y, int ydt, const RowGroups& rg, void* ws,
                          cudaStream_t st) {
   Gemv1Geom g;
   if (!gemv1_geom(N, K, rowbytes, xdt, &g)) return cudaErrorInvalidValue;
-  if (xdt == BL_F32) return launch_gemv1_x<BL_F32>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 1, rg, st);
-  if (xdt == BL_BF16) return launch_gemv1_x<BL_BF16>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 1, rg, st);
-  return launch_gemv1_x<BL_I8>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 0, rg, st);
+  if (xdt == BL_F32) return launch_gemv1_x<BL_F32>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 1, rg, ws, st);
+  if (xdt == BL_BF16) return launch_gemv1_x<BL_BF16>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 1, rg, ws, st);
+  return launch_gemv1_x<BL_I8>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 0, rg, ws, st);
 }
 
 }  // namespace bl

@@ -100,12 +100,13 @@ cudaError_t launch_backward_dw(const void* dy, int dydt, const int8_t* xq, const
 // at most 8192 bytes, and fp32 tokens only when K is small enough for the raw
 // token words of a thread to fit (see gemv1_fits).
 bool gemv1_fits(int64_t N, int64_t K, int64_t rowbytes, int xdt);
+// ws: a workspace header for the device flags (a bounded wait that runs out).
 cudaError_t launch_gemv1(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
-                         const void* x, int xdt, float* scale, void* y, int ydt, const RowGroups& rg,
+                         const void* x, int xdt, float* scale, void* y, int ydt, const RowGroups& rg, void* ws,
                          cudaStream_t st);
 
 cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int64_t N, int64_t K,
                         const void* x, int xdt, float* scale, int64_t M, void* y, int ydt,
-                        const RowGroups& rg, cudaStream_t st);
+                        const RowGroups& rg, void* ws, cudaStream_t st);
 
 }  // namespace bl
