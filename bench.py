@@ -1,19 +1,21 @@
 #!/usr/bin/env python3
 """BitLinear forward throughput on B200: one JSON line on rank 0.
 
-A step is one pass of the whole hot path over one batch of synthetic input:
-for every layer of the workload, the absmean scale (step 1), ternarize + pack
-(steps 2-3) and the forward (per-token INT8 quantization, ternary x INT8
-product, dequantization: steps 4-6), each through the C ABI of
-libbitlinear.so.  ``--phase forward`` times steps 4-6 alone on weights packed
-beforehand (an inference server's per-token work).
+A step is one pass of the per-token hot path over one batch of synthetic
+input: for every layer of the workload, the forward on weights packed
+beforehand (per-token INT8 quantization, ternary x INT8 product,
+dequantization: steps 4-6), through the C ABI of libbitlinear.so.  Weight
+preparation (absmean, ternarize + pack: steps 1-3) is offline -- done once per
+weight matrix, not per token -- and is timed on its own as a secondary section
+(``--phase all`` puts it back into every step).
 
 Timing: W untimed warm-up steps; then exactly K steps captured into one CUDA
-graph with timing events between the library calls, replayed once between
-barrier + synchronize on both sides; the device time is the max over ranks.
-The weights are larger than L2 (phase all) or rotated over enough packed copies
-to exceed 4x L2 (phase forward).  Multi-GPU: one process per GPU (torchrun),
-every rank runs its own independent replica of the workload (weak scaling).
+graph with CUDA events at its two ends, replayed once untimed and once timed
+between barrier + synchronize on both sides; the device time is the max over
+ranks.  The packed weights are rotated over enough copies to exceed 4x L2 (the
+fp32 latent weights of ``--phase all`` exceed L2 on their own).  Multi-GPU:
+one process per GPU (torchrun), every rank runs its own independent replica of
+the workload (weak scaling).
 
 ``--impl reference`` times the CPU oracle instead (rank 0 only), each step a
 bounded sample of the same workload.
@@ -57,7 +59,7 @@ WORKLOADS = {
 
 KERNEL_SOURCE = {"absmean_kernel": "bl_weights.cu", "ternarize_flat_kernel": "bl_weights.cu",
                  "binarize_pack_kernel": "bl_weights.cu",
-                 "ternarize_pack_kernel": "bl_weights.cu", "gemv_i2_kernel": "bl_gemv.cu",
+                 "ternarize_pack_kernel": "bl_weights.cu", "gemv_i2_kernel": "bl_gemv.cu", "gemv1_i2_kernel": "bl_gemv1.cu",
                  "gemv_kernel": "bl_gemv.cu", "gemv_t5_kernel": "bl_gemv.cu", "gemv_i2_mt_kernel": "bl_gemv.cu", "act_quant_row_kernel": "bl_acts.cu",
                  "act_quant_kernel": "bl_acts.cu", "ln_quant_kernel": "bl_acts.cu", "gemm_i2_2sm_kernel": "bl_gemm_sm100.cu",
                  "gemm_i2_kernel": "bl_gemm_sm100.cu", "b1_to_i2_kernel": "bl_gemm_sm100.cu",
@@ -214,35 +216,60 @@ def layer_bytes(N, K, M, rb, w_es=4, x_es=2, y_es=2):
 # CPU oracle timing (the baseline and the reference arm)
 # ----------------------------------------------------------------------------
 
-def oracle_layer_inputs(wl, rows_frac=1.0):
+def oracle_layer_inputs(wl, phase, rows_frac=1.0):
+    """Seeded inputs of the workload's layers (the first rows_frac of each
+    layer's weight rows); for ``phase == "forward"`` the weights are also
+    quantized and packed here, outside any timed region (offline work)."""
+    import oracle
     from bitlinear_b1_fwd_b200 import synth
     out = []
     for i, (N, K) in enumerate(wl["layers"]):
         n = max(1, int(N * rows_frac))
         W = synth.normal_f32(1000 + wl["seed"] + 100 * i, (N, K), wl["sigma"])[:n]
         x = synth.to_bf16_bits(synth.normal_f32(2000 + wl["seed"] + 100 * i, (wl["M"], K)))
-        out.append((W, x))
+        L = dict(W=W, x=x)
+        if phase == "forward":
+            L["g"] = oracle.gamma(W)
+            L["packed"] = oracle.pack(oracle.ternarize(W, L["g"]), wl["fmt"])
+        out.append(L)
     return out
 
 
 def oracle_step(orc, wl, inputs, phase):
-    """One oracle pass over the inputs; returns algorithmic bytes processed."""
+    """One oracle pass over the inputs; returns the algorithmic bytes processed."""
     total = 0
-    for (W, x) in inputs:
-        n, K = W.shape
+    for L in inputs:
+        n, K = L["W"].shape
         rb = orc.packed_row_bytes(K, wl["fmt"])
         b = layer_bytes(n, K, wl["M"], rb)
-        g = orc.gamma(W)
-        packed = orc.pack(orc.ternarize(W, g), wl["fmt"])
-        orc.forward(packed, wl["fmt"], g, n, K, x, ydt=orc.BF16)
+        if phase == "all":
+            g = orc.gamma(L["W"])
+            packed = orc.pack(orc.ternarize(L["W"], g), wl["fmt"])
+        else:
+            g, packed = L["g"], L["packed"]
+        orc.forward(packed, wl["fmt"], g, n, K, L["x"], ydt=orc.BF16)
         total += b["forward"] + (b["absmean"] + b["ternarize_pack"] if phase == "all" else 0)
     return total
+
+
+def host_cpu():
+    """The host's logical core count and CPU model."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": os.cpu_count(), "cpu_model": model}
 
 
 def time_oracle(wl, phase, budget_s, min_steps=1, rows_frac=1.0):
     import oracle
     oracle.build()
-    inputs = oracle_layer_inputs(wl, rows_frac)
+    inputs = oracle_layer_inputs(wl, phase, rows_frac)
     steps, nbytes, t0 = 0, 0, time.perf_counter()
     while steps < min_steps or time.perf_counter() - t0 < budget_s:
         nbytes += oracle_step(oracle, wl, inputs, phase)
@@ -314,7 +341,8 @@ def run_gpu(args, wl, rank, world, local_rank):
         L = dict(N=N, K=K, rb=rb)
         L["W"] = torch.from_numpy(Wh).to(dev)
         L["x"] = torch.from_numpy(xh.view(np.int16)).to(dev).view(torch.bfloat16)
-        L["W_host"] = torch.from_numpy(Wh).pin_memory()
+        if args.phase == "all":  # the step copies the latent weights from the host too
+            L["W_host"] = torch.from_numpy(Wh).pin_memory()
         L["x_host"] = torch.from_numpy(xh.view(np.int16)).view(torch.bfloat16).pin_memory()
         L["gamma"] = torch.empty(1, dtype=torch.float32, device=dev)
         L["ws"] = torch.zeros(B.bitlinear_quantize_weights_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
@@ -331,18 +359,16 @@ def run_gpu(args, wl, rank, world, local_rank):
     stream = torch.cuda.Stream(device=dev)
     eps = 1e-5
 
-    # phase forward: pack once, then rotate over copies of the packed weights
-    rot = 1
-    if args.phase == "forward":
-        with torch.cuda.stream(stream):
-            for L in layers:
-                B.bitlinear_quantize_weights(L["W"], eps, fmt, L["packed"], None, L["gamma"], L["ws"], stream)
-        stream.synchronize()
-        packed_bytes = sum(L["N"] * L["rb"] for L in layers)
-        rot = max(1, -(-4 * l2 // packed_bytes))
+    # weight preparation once (offline work), then copies of the packed
+    # weights rotated so that consecutive steps read more than 4x L2
+    with torch.cuda.stream(stream):
         for L in layers:
-            L["copies"] = [L["packed"]] + [L["packed"].clone() for _ in range(rot - 1)]
-            del L["W"]
+            B.bitlinear_quantize_weights(L["W"], eps, fmt, L["packed"], None, L["gamma"], L["ws"], stream)
+    stream.synchronize()
+    packed_bytes = sum(L["N"] * L["rb"] for L in layers)
+    rot = max(2, -(-4 * l2 // packed_bytes))
+    for L in layers:
+        L["copies"] = [L["packed"]] + [L["packed"].clone() for _ in range(rot - 1)]
 
     ops = ["absmean", "ternarize_pack", "forward"] if args.phase == "all" else ["forward"]
 
@@ -373,12 +399,13 @@ def run_gpu(args, wl, rank, world, local_rank):
         if st != B.BL_OK:
             raise RuntimeError(f"device status {B.status_string(st)}")
 
-    # each kernel's average launch duration: a graph of K steps of that call
-    # alone, over every layer in turn (so the inputs of consecutive launches
-    # together exceed L2), timed at its two ends
+    # each op's average launch duration: a graph of K steps of that call alone
+    # over every layer in turn (the inputs of consecutive launches together
+    # exceed L2), timed at its two ends; the offline weight preparation is
+    # timed this way in every run
     per_op_ms = {}
-    for op in ops:
-        if len(ops) == 1:
+    for op in ("absmean", "ternarize_pack", "forward"):
+        if op == "forward" and ops == ["forward"]:
             per_op_ms[op] = ms / (args.steps * len(layers))
             continue
         t = graph_ms(stream, args.steps, lambda i, op=op: [run_op(op, L, i) for L in layers])
@@ -387,7 +414,9 @@ def run_gpu(args, wl, rank, world, local_rank):
 
     ms_max = max_over_ranks(ms, world, dev)
 
-    # ---- end to end through the public API from pinned host buffers ----
+    # ---- end to end through the public API: each step copies its token(s)
+    # (and, for --phase all, the latent weights) from pinned host memory and
+    # reads y back ----
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     h2d = sum((L["W_host"].numel() * 4 if args.phase == "all" else 0) + L["x_host"].numel() * 2 for L in layers)
     d2h = sum(L["y_host"].numel() * 2 for L in layers)
@@ -414,8 +443,8 @@ def run_gpu(args, wl, rank, world, local_rank):
     decode = run_decode(args, dev, stream, rank_seed, l2) if args.decode else None
     sweep = run_sweep(args, dev, stream, l2) if args.sweep else None
     backward = run_backward(args, dev, stream, rank_seed, l2) if args.decode else None
-    res = dict(prefill=prefill, decode=decode, sweep=sweep, backward=backward, ms_total=ms_max, per_op_ms=per_op_ms, step_bytes=step_bytes,
-               layers=layers, ops=ops,
+    res = dict(prefill=prefill, decode=decode, sweep=sweep, backward=backward, ms_total=ms_max, per_op_ms=per_op_ms,
+               step_bytes=step_bytes, layers=layers, ops=ops,
                clocks=sampler.summary(), e2e_ms=e2e_ms, e2e_steps=e2e_steps, h2d=h2d, d2h=d2h,
                rot=rot, l2=l2, launches_per_step=len(layers) * len(ops))
     return res
@@ -767,7 +796,8 @@ def decode_summary(d):
 
 
 def gemv_kernel_name(fmt, layers, M=1):
-    """The decode kernel the forward dispatches to (M <= 4): for 2..4 tokens
+    """The decode kernel the forward dispatches to (M <= 4): for one token of
+    2-bit rows the one-token column-stationary kernel where it fits; for 2..4 tokens
     of 2-bit rows of at most 8192 bytes (and at most 1024 rows per CTA) the
     column-stationary multi-token kernel, else the lean 2-bit kernel for rows
     of at most 8192 packed bytes; for one token of base 3,
@@ -777,6 +807,12 @@ def gemv_kernel_name(fmt, layers, M=1):
         return "gemv_i2_kernel" if all(((K + 7) // 8 + 15) // 16 * 16 <= 4096 for (_, K) in layers) else "gemv_kernel"
     if fmt == 0:
         rbs = [((K + 3) // 4 + 15) // 16 * 16 for (_, K) in layers]
+        # one bf16 token, K % 16 == 0, rows of at most 8192 bytes and the
+        # token, its codes and the row sums within 96 KB of shared memory
+        if M == 1 and all(K % 16 == 0 and rb <= 8192 and
+                          K * 2 + rb * 4 + 4 * -(-N // min(N, 148)) <= 96 * 1024
+                          for rb, (N, K) in zip(rbs, layers)):
+            return "gemv1_i2_kernel"
         if 2 <= M <= 4 and all(rb <= 8192 and -(-N // min(N, 148)) <= 1024 for rb, (N, _) in zip(rbs, layers)):
             return "gemv_i2_mt_kernel"
         return "gemv_i2_kernel" if all(rb <= 8192 for rb in rbs) else "gemv_kernel"
@@ -896,7 +932,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="3b_decode")
-    ap.add_argument("--phase", choices=["all", "forward"], default="all")
+    ap.add_argument("--phase", choices=["forward", "all"], default="forward")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--prefill", action=argparse.BooleanOptionalAction, default=True,
                     help="also time the 3B prefill layer (INT8 TOPS of the tensor-core product)")
@@ -919,6 +955,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    # one config dict, printed unchanged by both arms
     config = {"workload": args.workload, "desc": wl["desc"], "phase": args.phase, "M": wl["M"],
               "layers_NK": wl["layers"], "pack": ["2-bit", "base-3"][wl["fmt"]],
               "parallelism": f"replicas x{args.gpus}"}
@@ -934,20 +971,22 @@ def main():
         per_step_full = dt / s / probe_frac
         budget = 120.0 / max(1, args.steps + args.warmup)
         frac = min(1.0, max(1e-4, budget / per_step_full))
-        inputs = oracle_layer_inputs(wl, frac)
+        inputs = oracle_layer_inputs(wl, args.phase, frac)
         for _ in range(args.warmup):
             oracle_step(oracle, wl, inputs, args.phase)
         t0 = time.perf_counter()
         nbytes = sum(oracle_step(oracle, wl, inputs, args.phase) for _ in range(args.steps))
         dt = time.perf_counter() - t0
         val = nbytes / dt / 1e9
-        sample = f"first {frac:.4%} of each layer's weight rows per step, all steps of the path"
+        what = "the forward on weights packed beforehand" if args.phase == "forward" else "all steps of the path"
+        sample = f"first {frac:.4%} of each layer's weight rows per step, {what}"
         print(json.dumps({
             "impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64+i32",
             "data": "synthetic", "config": config,
-            "cpu_baseline": {"value": val, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": val, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample,
+                             **host_cpu()},
             "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }))
         return
@@ -962,46 +1001,61 @@ def main():
         ms = res["ms_total"] / args.steps
         value = whole_job_gbs(res["step_bytes"], world, ms)
         peak, peak_kind = measured_peaks()
-        # per-op summary and the dominant kernel
-        stages = {}
         nl = len(res["layers"])
-        for op in res["ops"]:
+
+        def stage(op):
             per_launch = res["per_op_ms"][op]
             nb = sum(L["bytes"][op] for L in res["layers"])
-            stages[op] = {"us_per_launch": per_launch * 1e3, "bytes_per_step": nb,
-                          "GB_s": nb / (per_launch * nl * 1e-3) / 1e9,
-                          "frac_of_hbm": nb / (per_launch * nl * 1e-3) / 1e9 / peak}
-        dom = max(stages, key=lambda o: stages[o]["us_per_launch"])
+            return {"us_per_launch": per_launch * 1e3, "bytes_per_step": nb,
+                    "GB_s": nb / (per_launch * nl * 1e-3) / 1e9,
+                    "frac_of_hbm": nb / (per_launch * nl * 1e-3) / 1e9 / peak}
+
+        stages = {op: stage(op) for op in res["ops"]}
+        flat = wl["fmt"] == 0 and all(K % 64 == 0 for (_, K) in wl["layers"])
+        names = {"absmean": "absmean_kernel",
+                 "ternarize_pack": "ternarize_flat_kernel" if flat else "ternarize_pack_kernel",
+                 "forward": gemv_kernel_name(wl["fmt"], wl["layers"], wl["M"])}
+        # the roofline is the forward's (the per-token kernel the metric names);
+        # with --phase all, the step's dominant kernel
+        dom = "forward" if args.phase == "forward" else max(stages, key=lambda o: stages[o]["us_per_launch"])
         avg_launch_ms = res["per_op_ms"][dom]
         bytes_per_launch = stages[dom]["bytes_per_step"] / nl
         achieved = bytes_per_launch / (avg_launch_ms * 1e-3) / 1e9
-        flat = wl["fmt"] == 0 and all(K % 64 == 0 for (_, K) in wl["layers"])
-        kernel_name = {"absmean": "absmean_kernel",
-                       "ternarize_pack": "ternarize_flat_kernel" if flat else "ternarize_pack_kernel",
-                       "forward": gemv_kernel_name(wl["fmt"], wl["layers"], wl["M"])}[dom]
+        kernel_name = names[dom]
         traffic = profiled_traffic(kernel_name, args.workload)
+        weight_prep = {op: dict(stage(op), kernel=names[op]) for op in ("absmean", "ternarize_pack")} \
+            if args.phase == "forward" else None
+        if weight_prep is not None:
+            for op in weight_prep:
+                nb = sum(L["bytes"][op] for L in res["layers"])
+                weight_prep[op]["bytes_per_step"] = nb
         cpu = None
         if args.cpu_budget > 0 and world == 1:
             v, s, dt = time_oracle(wl, args.phase, args.cpu_budget)
+            what = "forwards on weights packed beforehand" if args.phase == "forward" else "full oracle steps"
             cpu = {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                   "sample": f"{s} full oracle steps of the same workload ({dt:.1f} s, 1 thread)"}
+                   "sample": f"{s} {what} of the same workload ({dt:.1f} s, 1 thread)", **host_cpu()}
         e2e_value = whole_job_gbs(res["step_bytes"], world, res["e2e_ms"])
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "i8xternary->i32 (fp32 scales, fp64 gamma)",
             "data": "synthetic (seeded N(0,sigma) latent weights, N(0,1) bf16 activations)",
-            "config": dict(config, l2=("inputs larger than L2 (fp32 latent weights "
-                                       f"{sum(L['N'] * L['K'] * 4 for L in res['layers']) / 1e6:.0f} MB per step)"
-                                       if args.phase == "all" else
-                                       f"packed weights rotated over {res['rot']} copies (>= 4x L2)"),
-                           kernels_per_step=res["launches_per_step"]),
+            "config": config,
+            "l2": (f"packed weights rotated over {res['rot']} copies (>= 4x L2)" if args.phase == "forward" else
+                   "inputs larger than L2 (fp32 latent weights "
+                   f"{sum(L['N'] * L['K'] * 4 for L in res['layers']) / 1e6:.0f} MB per step)"),
+            "kernels_per_step": res["launches_per_step"],
             "roofline": {"bound": "hbm", "kernel": kernel_name, "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic, "bytes_per_launch": bytes_per_launch,
-                         "launch_duration": "CUDA events at the two ends of a graph of K steps of this call alone "
-                                            "over every layer (K x layers back-to-back launches)"},
+                         "launch_duration": ("CUDA events at the two ends of the graph of K steps "
+                                             "(K x layers back-to-back forward launches)"
+                                             if args.phase == "forward" else
+                                             "CUDA events at the two ends of a graph of K steps of this "
+                                             "call alone over every layer")},
             "stages": stages,
+            "weight_prep": weight_prep,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": res["h2d"],
                     "d2h_bytes_per_step": res["d2h"], "steps": res["e2e_steps"]},

@@ -160,7 +160,10 @@ BL_API bl_status bitlinear_absmean(const void *W, int wdt, int64_t N, int64_t K,
  * The partial sums live in a 256 KiB device array owned by the library (held
  * on every GPU that loads it, until the process exits); nothing is allocated.
  * The first call on a device looks up the array's device address (once per
- * device), so make that first call before any stream capture.  Every call
+ * device, with that device current) and keeps it, so make that first call
+ * before any stream capture.  The kept address belongs to the device context
+ * of that first call: after cudaDeviceReset it is stale, so a process that
+ * resets a device must not call this entry point on it again.  Every call
  * shares the one array and resets its counter: calls whose kernels overlap on
  * the GPU (different streams, or different host threads) race and must be
  * serialized by the caller. */
