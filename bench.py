@@ -61,7 +61,7 @@ KERNEL_SOURCE = {"absmean_kernel": "bl_weights.cu", "ternarize_flat_kernel": "bl
                  "binarize_pack_kernel": "bl_weights.cu",
                  "ternarize_pack_kernel": "bl_weights.cu", "gemv_i2_kernel": "bl_gemv.cu", "gemv1_i2_kernel": "bl_gemv1.cu",
                  "gemv_kernel": "bl_gemv.cu", "gemv_t5_kernel": "bl_gemv.cu", "gemv_i2_mt_kernel": "bl_gemv.cu", "act_quant_row_kernel": "bl_acts.cu",
-                 "act_quant_kernel": "bl_acts.cu", "ln_quant_kernel": "bl_acts.cu", "gemm_i2_2sm_kernel": "bl_gemm_sm100.cu",
+                 "act_quant_kernel": "bl_acts.cu", "ln_quant_kernel": "bl_acts.cu", "ln_quant_reg_kernel": "bl_acts.cu", "gemm_i2_2sm_kernel": "bl_gemm_sm100.cu",
                  "gemm_i2_kernel": "bl_gemm_sm100.cu", "b1_to_i2_kernel": "bl_gemm_sm100.cu",
                  "backward_dx_partial_kernel": "bl_backward.cu", "backward_dx_reduce_kernel": "bl_backward.cu",
                  "backward_dw_kernel": "bl_backward.cu"}
@@ -838,7 +838,8 @@ def prefill_summary(p):
             "value": tops, "unit": "TOPS (int8)", "forward_TOPS_incl_act_quant": fwd_tops,
             "gemm_us": p["gemm_ms"] * 1e3, "act_quant_us": p["act_ms"] * 1e3,
             "act_quant_GB_s": act_gbs, "act_quant_frac_of_hbm": act_gbs / hbm,
-            "layernorm_act_quant": {"kernel": "ln_quant_kernel", "us": p["ln_ms"] * 1e3,
+            "layernorm_act_quant": {"kernel": "ln_quant_reg_kernel" if p["K"] % 2 == 0 and p["K"] <= 4096
+                                    else "ln_quant_kernel", "us": p["ln_ms"] * 1e3,
                                     "GB_s": p["ln_bytes"] / (p["ln_ms"] * 1e-3) / 1e9,
                                     "frac_of_hbm": p["ln_bytes"] / (p["ln_ms"] * 1e-3) / 1e9 / hbm},
             "roofline": {"bound": "tensor", "kernel": gemm_kernel_name(p["M"]), "achieved": tops, "peak": peak,

@@ -5,6 +5,8 @@
 // x_q = clamp(round(x / s * 127), -127, 127).  Rows of up to 8 K (bf16) or
 // 4 K (fp32) elements: one CTA per token, read once into registers.  Other
 // rows: one warp per token, two passes whose loads go out kActBatch at a time.
+#include <type_traits>
+
 #include "bl_common.cuh"
 #include "bl_kernels.h"
 
@@ -234,8 +236,163 @@ __global__ void __launch_bounds__(kLnThreads)
   }
 }
 
+
+// The same LayerNorm + INT8 with the token held in registers (K even and
+// ceil(K / 256) <= NI).  R18's lane l is a set of elements, not a thread:
+// here thread t of a 128-thread CTA computes lanes 2t and 2t + 1, loading
+// the element pairs (2t + 256 i, 2t + 1 + 256 i) with one 4-byte (bf16) or
+// 8-byte (fp32) load each, and adds each lane's elements in R18's order.  A
+// tree of the 256 lane sums takes one shared-memory write and one barrier:
+// every warp then reads the eight sums of its lane's subtree and adds them in
+// the tree's order (levels 128, 64, 32), and levels 16..1 run by shuffles --
+// each warp computes the same total, so no broadcast is needed.  y is
+// computed once and kept for the absmax and the codes.
+constexpr int kLnRegThreads = 128;
+
+template <int XDT, int NI>
+__global__ void __launch_bounds__(kLnRegThreads, 4)
+    ln_quant_reg_kernel(const void* __restrict__ x, const float* __restrict__ g, const float* __restrict__ b,
+                        float eps, int64_t M, int64_t K, uint16_t* __restrict__ y, int8_t* __restrict__ xq,
+                        float* __restrict__ scale) {
+  pdl_enter(x, g, b, y, xq, scale);
+  __shared__ __align__(16) double p1[256];
+  __shared__ __align__(16) double p2[256];
+  __shared__ float red[kLnRegThreads / 32];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  // the tree of the 256 lane sums held in p, R18's order
+  auto tree = [&](const double* p) -> double {
+    const int L = lane;
+    const double q0 = __dadd_rn(p[L], p[L + 128]), q1 = __dadd_rn(p[L + 64], p[L + 192]);
+    const double q2 = __dadd_rn(p[L + 32], p[L + 160]), q3 = __dadd_rn(p[L + 96], p[L + 224]);
+    double v = __dadd_rn(__dadd_rn(q0, q1), __dadd_rn(q2, q3));
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) v = __dadd_rn(v, __shfl_down_sync(0xffffffffu, v, s));
+    return __shfl_sync(0xffffffffu, v, 0);
+  };
+  // the element pair i of lanes (2t, 2t + 1) as two floats
+  constexpr bool kF32 = XDT == BL_F32;
+  using Pair = typename std::conditional<kF32, float2, uint32_t>::type;
+  auto lo = [](const Pair& v) -> float {
+    if constexpr (kF32) return v.x; else return __uint_as_float(v << 16);
+  };
+  auto hi = [](const Pair& v) -> float {
+    if constexpr (kF32) return v.y; else return __uint_as_float(v & 0xffff0000u);
+  };
+  const double dK = static_cast<double>(K);
+  for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+    const int64_t base = m * K;
+    Pair xr[NI];  // the token's pairs; later y's bf16 pairs
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+      const int64_t k = 2 * t + 256 * i;
+      if constexpr (kF32) {
+        xr[i] = k < K ? __ldcg(reinterpret_cast<const float2*>(static_cast<const float*>(x) + base + k))
+                      : make_float2(0.0f, 0.0f);
+      } else {
+        xr[i] = k < K ? __ldcg(reinterpret_cast<const unsigned int*>(static_cast<const uint16_t*>(x) + base + k))
+                      : 0u;
+      }
+    }
+    // mean: each lane's elements in turn from 0.0
+    double sa = 0.0, sb = 0.0;
+#pragma unroll
+    for (int i = 0; i < NI; ++i)
+      if (2 * t + 256 * i < K) {
+        sa = __dadd_rn(sa, static_cast<double>(lo(xr[i])));
+        sb = __dadd_rn(sb, static_cast<double>(hi(xr[i])));
+      }
+    reinterpret_cast<double2*>(p1)[t] = make_double2(sa, sb);
+    __syncthreads();
+    const double mu = __ddiv_rn(tree(p1), dK);
+    // variance: (x - mu)^2 in the same order
+    sa = sb = 0.0;
+#pragma unroll
+    for (int i = 0; i < NI; ++i)
+      if (2 * t + 256 * i < K) {
+        const double da = __dsub_rn(static_cast<double>(lo(xr[i])), mu);
+        const double db = __dsub_rn(static_cast<double>(hi(xr[i])), mu);
+        sa = __dadd_rn(sa, __dmul_rn(da, da));
+        sb = __dadd_rn(sb, __dmul_rn(db, db));
+      }
+    reinterpret_cast<double2*>(p2)[t] = make_double2(sa, sb);
+    __syncthreads();
+    const double var = __ddiv_rn(tree(p2), dK);
+    const double r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(var, static_cast<double>(eps))));
+    // y = ((x - mu) r) g + b, fp64 -> fp32 -> bf16, stored and kept (bf16 pairs)
+    uint32_t yr[NI];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+      const int64_t k = 2 * t + 256 * i;
+      yr[i] = 0u;
+      if (k < K) {
+        const float2 gg = __ldcg(reinterpret_cast<const float2*>(g + k));
+        const float2 bb = __ldcg(reinterpret_cast<const float2*>(b + k));
+        const double va = __dadd_rn(__dmul_rn(__dmul_rn(__dsub_rn(static_cast<double>(lo(xr[i])), mu), r),
+                                              static_cast<double>(gg.x)),
+                                    static_cast<double>(bb.x));
+        const double vb = __dadd_rn(__dmul_rn(__dmul_rn(__dsub_rn(static_cast<double>(hi(xr[i])), mu), r),
+                                              static_cast<double>(gg.y)),
+                                    static_cast<double>(bb.y));
+        const uint32_t ha = __bfloat16_as_ushort(__float2bfloat16_rn(__double2float_rn(va)));
+        const uint32_t hb = __bfloat16_as_ushort(__float2bfloat16_rn(__double2float_rn(vb)));
+        yr[i] = ha | (hb << 16);
+        if (y != nullptr) *reinterpret_cast<uint32_t*>(y + base + k) = yr[i];
+        amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(ha << 16)), fabsf(__uint_as_float(hb << 16))));
+      }
+    }
+    amax = warp_maxf(amax);
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    float am = red[0];
+#pragma unroll
+    for (int w = 1; w < kLnRegThreads / 32; ++w) am = fmaxf(am, red[w]);
+    const float s = fmaxf(am, 1e-6f);
+    const float c127 = __fdiv_rn(127.0f, s);
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+      const int64_t k = 2 * t + 256 * i;
+      if (k < K) {
+        const uint32_t qa = static_cast<uint8_t>(quant_act_fast(__uint_as_float(yr[i] << 16), s, c127));
+        const uint32_t qb = static_cast<uint8_t>(quant_act_fast(__uint_as_float(yr[i] & 0xffff0000u), s, c127));
+        *reinterpret_cast<uint16_t*>(xq + base + k) = static_cast<uint16_t>(qa | (qb << 8));
+      }
+    }
+    if (t == 0) scale[m] = s;
+    // red, p1 and p2 are free for the next token once every warp is past here
+    __syncthreads();
+  }
+}
+
+template <int XDT, int NI>
+static cudaError_t launch_ln_quant_reg(const void* x, const float* g, const float* b, float eps, int64_t M, int64_t K,
+                                       uint16_t* y, int8_t* xq, float* scale, cudaStream_t st) {
+  int per_sm = 1;
+  auto kern = ln_quant_reg_kernel<XDT, NI>;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kLnRegThreads, 0) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  const int64_t cap = static_cast<int64_t>(device_sms()) * per_sm;
+  const unsigned grid = static_cast<unsigned>(M < cap ? M : cap);
+  const cudaError_t e = launch_pdl(kern, grid, kLnRegThreads, 0, st, x, g, b, eps, M, K, y, xq, scale);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 cudaError_t launch_ln_quant(const void* x, int xdt, const float* g, const float* b, float eps, int64_t M, int64_t K,
                             uint16_t* y, int8_t* xq, float* scale, cudaStream_t st) {
+  // the register form: K even (vector loads and stores of element pairs), the
+  // token in registers, g and b 8-byte aligned (float2 loads), y 4-byte and
+  // x_q 2-byte aligned (pair stores)
+  const bool pairs = (K % 2) == 0 && (reinterpret_cast<uintptr_t>(g) & 7) == 0 &&
+                     (reinterpret_cast<uintptr_t>(b) & 7) == 0 && (reinterpret_cast<uintptr_t>(y) & 3) == 0 &&
+                     (reinterpret_cast<uintptr_t>(xq) & 1) == 0;
+  if (pairs && K <= 256 * 8)
+    return xdt == BL_F32 ? launch_ln_quant_reg<BL_F32, 8>(x, g, b, eps, M, K, y, xq, scale, st)
+                         : launch_ln_quant_reg<BL_BF16, 8>(x, g, b, eps, M, K, y, xq, scale, st);
+  if (pairs && K <= 256 * 16)
+    return xdt == BL_F32 ? launch_ln_quant_reg<BL_F32, 16>(x, g, b, eps, M, K, y, xq, scale, st)
+                         : launch_ln_quant_reg<BL_BF16, 16>(x, g, b, eps, M, K, y, xq, scale, st);
+
   int per_sm = 1;
   const void* kp = xdt == BL_F32 ? reinterpret_cast<const void*>(ln_quant_kernel<BL_F32>)
                                  : reinterpret_cast<const void*>(ln_quant_kernel<BL_BF16>);
