@@ -865,6 +865,11 @@ PROFILE_CASES = {
     "binarize_3b_up": dict(N=8640, K=3200, fmt=2, M=1, sigma=0.02, op="quantize"),
     "decode_70b_up_1bit": dict(N=28672, K=8192, fmt=2, M=1, sigma=0.01, op="forward"),
     "backward_3b_up": dict(N=8640, K=3200, fmt=0, M=1, sigma=0.02, op="backward"),
+    "batch4_70b_up": dict(N=28672, K=8192, fmt=0, M=4, sigma=0.01, op="forward"),
+    "batch2_70b_up_t5": dict(N=28672, K=8192, fmt=1, M=2, sigma=0.01, op="forward"),
+    "batch16_70b_up_t5": dict(N=28672, K=8192, fmt=1, M=16, sigma=0.01, op="forward"),
+    "batch16_70b_up_1bit": dict(N=28672, K=8192, fmt=2, M=16, sigma=0.01, op="forward"),
+    "backward_3b_down": dict(N=3200, K=8640, fmt=0, M=1, sigma=0.02, op="backward"),
 }
 
 

@@ -10,87 +10,99 @@
 //   dW[n, k] = gamma * sum_m dy[m, n] x_q[m, k] s_m / 127
 // dx is defined by the exact sum over the rows rounded once to fp64 (no
 // order), then gamma * S in fp64 and fp32; this kernel adds in fp64 in an
-// order of its own (rows in chunks of 64, +dy for weight +1, -dy for -1,
-// nothing for 0; the chunk sums in chunk order), which stays within one fp32
-// ulp plus gamma N 2^-52 sum |dy| of the definition.
+// order of its own (+dy for weight +1, -dy for -1, nothing for 0; per tile a
+// warp's rows in order, the tile's warps in order, the row blocks in order),
+// which stays within one fp32 ulp plus gamma N 2^-52 sum |dy| of the
+// definition.
 // dW: c_m = s_m / 127, terms (dy[m, n] x_q[m, k]) c_m added in fp64 from 0.0
 // in token order (the plain order of the sum), then gamma * T, rounded once
 // to fp32.
-// dx reads the packed 2-bit weights once per pass of up to two tokens; dW
-// writes N K fp32 values (the HBM-bound part for few tokens).
+// dx reads the packed 2-bit weights once per pass of up to two tokens in 2-D
+// tiles (512 columns x at least 64 rows: about two CTAs per SM, partial sums
+// a few percent of the weight bytes); dW writes N K fp32 values (the
+// HBM-bound part for few tokens).
 #include "bl_common.cuh"
 #include "bl_kernels.h"
 
 namespace bl {
 
-constexpr int kDxChunk = 64;   // rows per partial sum (enough units to fill every SM)
-constexpr int kDxTokens = 2;   // tokens per pass: 16 weights x 2 tokens of fp64 sums per thread
+constexpr int kDxMinRows = 64;  // rows per row block, at least (the workspace holds ceil(N / 64) blocks)
+constexpr int kDxTokens = 2;    // tokens per pass: 16 columns x 2 tokens of fp64 sums per lane
+constexpr int kDxWarps = 8;     // warps of a CTA: each takes every 8th row of the row block
+constexpr int kDxAhead = 4;     // rows whose words and gradients are loaded ahead of the adds
 
 template <int DYT>
 __device__ __forceinline__ double load_grad(const void* p, int64_t i) {
   return static_cast<double>(load_elem<DYT>(p, i));
 }
 
-// Partial sums: thread (chunk r, word column c) adds, for rows n of chunk r in
-// order, the 16 weights of packed word c of row n times dy[m, n] for the MT
-// tokens of the pass.  A warp's lanes take 32 consecutive columns of one
-// chunk, so each row is one 128-byte read.  part[r][m][k] (fp64).
+// Partial sums over one tile: CTA (cb, rb) takes the 32 packed words
+// 32 cb .. 32 cb + 31 of each row (columns 512 cb .. 512 cb + 511; lane L one
+// word, so a warp reads a 128-byte piece of a row) of the rows of row block
+// rb; warp w takes every kDxWarps-th row.  A lane adds +dy, -dy or nothing
+// (the stored digit 2, 0 or 1) into 16 fp64 sums per token; the warps' sums
+// meet in shared memory in a fixed order and go to part[rb][m][k] (fp64).
 template <int DYT, int MT>
-__global__ void __launch_bounds__(256)
-    backward_dx_partial_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, int64_t N, int64_t K,
-                               const void* __restrict__ dy, int64_t m0, double* __restrict__ part) {
+__global__ void __launch_bounds__(kDxWarps * 32)
+    backward_dx_tile_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, int64_t N, int64_t K,
+                            const void* __restrict__ dy, int64_t m0, int64_t rows_per_block,
+                            double* __restrict__ part) {
   pdl_enter(packed, dy, part);
-  const int64_t words = (K + 15) / 16;  // packed 32-bit words holding weights below K
-  const int64_t chunks = (N + kDxChunk - 1) / kDxChunk;
-  const int64_t units = words * chunks;
-  for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < units;
-       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = u / words, c = u - r * words;
-    double acc[MT][16];
+  extern __shared__ __align__(16) double sh[];  // [kDxWarps][MT * 16][33]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t words = (K + 15) / 16;                // packed 32-bit words holding weights below K
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * 32 + lane;  // this lane's word
+  const int64_t n0 = static_cast<int64_t>(blockIdx.y) * rows_per_block;
+  const int64_t n1 = n0 + rows_per_block < N ? n0 + rows_per_block : N;
+  const int64_t stride = rowbytes / 4;
+  double acc[MT][16];
 #pragma unroll
-    for (int m = 0; m < MT; ++m)
+  for (int m = 0; m < MT; ++m)
 #pragma unroll
-      for (int i = 0; i < 16; ++i) acc[m][i] = 0.0;
-    const int64_t n1 = (r + 1) * kDxChunk < N ? (r + 1) * kDxChunk : N;
+    for (int i = 0; i < 16; ++i) acc[m][i] = 0.0;
+  if (c < words) {
     const uint32_t* col = reinterpret_cast<const uint32_t*>(packed) + c;
-    const int64_t stride = rowbytes / 4;
-    // the rows' words (and gradients) are loaded 16 at a time ahead of the
-    // adds, so that a thread keeps 16 loads in flight
-    for (int64_t nb = r * kDxChunk; nb < n1; nb += 16) {
-      uint32_t wv[16];
-      double gv[MT][16];
+    for (int64_t nb = n0 + warp; nb < n1; nb += kDxWarps * kDxAhead) {
+      uint32_t wv[kDxAhead];
+      double gv[kDxAhead][MT];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int64_t n = nb + j;
-        wv[j] = n < n1 ? __ldcg(col + n * stride) : 0x55555555u;  // past the chunk: weight 0
+      for (int j = 0; j < kDxAhead; ++j) {
+        const int64_t n = nb + static_cast<int64_t>(kDxWarps) * j;
+        wv[j] = n < n1 ? __ldcg(col + n * stride) : 0x55555555u;  // past the block: weight 0
 #pragma unroll
-        for (int m = 0; m < MT; ++m) gv[m][j] = n < n1 ? load_grad<DYT>(dy, (m0 + m) * N + n) : 0.0;
+        for (int m = 0; m < MT; ++m) gv[j][m] = n < n1 ? load_grad<DYT>(dy, (m0 + m) * N + n) : 0.0;
       }
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-      const uint32_t w = wv[j];
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        const double g = gv[m][j];
-        const double ng = -g;
+      for (int j = 0; j < kDxAhead; ++j) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const uint32_t d = (w >> (2 * i)) & 3u;  // digit q + 1
-          if (d == 2u)
-            acc[m][i] = __dadd_rn(acc[m][i], g);
-          else if (d == 0u)
-            acc[m][i] = __dadd_rn(acc[m][i], ng);
+          const uint32_t d = (wv[j] >> (2 * i)) & 3u;  // digit q + 1
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            if (d == 2u)
+              acc[m][i] = __dadd_rn(acc[m][i], gv[j][m]);
+            else if (d == 0u)
+              acc[m][i] = __dadd_rn(acc[m][i], -gv[j][m]);
+          }
         }
       }
-      }
     }
+  }
+  // the warps' sums, transposed through shared memory (a padded row of 33 per
+  // column keeps both the writes and the reads free of bank conflicts)
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      double* dst = part + (r * MT + m) * K + 16 * c;
+  for (int m = 0; m < MT; ++m)
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        if (16 * c + i < K) dst[i] = acc[m][i];
-    }
+    for (int i = 0; i < 16; ++i) sh[(warp * MT * 16 + m * 16 + i) * 33 + lane] = acc[m][i];
+  __syncthreads();
+  // output o = (m, lane L, i): column 16 (32 cb + L) + i, the warps added in order
+  for (int o = threadIdx.x; o < MT * 32 * 16; o += kDxWarps * 32) {
+    const int m = o / 512, L = (o / 16) & 31, i = o & 15;
+    const int64_t k = 16 * (static_cast<int64_t>(blockIdx.x) * 32 + L) + i;
+    double v = 0.0;
+#pragma unroll
+    for (int w = 0; w < kDxWarps; ++w) v = __dadd_rn(v, sh[(w * MT * 16 + m * 16 + i) * 33 + L]);
+    if (k < K) part[(static_cast<int64_t>(blockIdx.y) * MT + m) * K + k] = v;
   }
 }
 
@@ -192,7 +204,7 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---- host side --------------------------------------------------------------------
-int64_t backward_dx_chunks(int64_t N) { return (N + kDxChunk - 1) / kDxChunk; }
+int64_t backward_dx_chunks(int64_t N) { return (N + kDxMinRows - 1) / kDxMinRows; }
 int backward_dx_tokens_per_pass() { return kDxTokens; }
 
 static unsigned grid_of(int64_t work, int per_sm) {
@@ -203,25 +215,43 @@ static unsigned grid_of(int64_t work, int per_sm) {
   return static_cast<unsigned>(g);
 }
 
+template <int DYT, int MT>
+static cudaError_t launch_dx_tile(dim3 grid, const uint8_t* packed, int64_t rowbytes, int64_t N, int64_t K,
+                                  const void* dy, int64_t m0, int64_t rows, double* part, cudaStream_t st) {
+  auto kern = backward_dx_tile_kernel<DYT, MT>;
+  const size_t smem = static_cast<size_t>(kDxWarps) * MT * 16 * 33 * sizeof(double);
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  return launch_pdl(kern, grid, kDxWarps * 32, smem, st, packed, rowbytes, N, K, dy, m0, rows, part);
+}
+
 cudaError_t launch_backward_dx(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
                                const void* dy, int dydt, int64_t M, float* dx, double* part, cudaStream_t st) {
-  const int64_t chunks = backward_dx_chunks(N);
+  // tiles: 512-column blocks x row blocks of at least kDxMinRows rows, about
+  // two CTAs per SM (the row blocks never outnumber backward_dx_chunks(N),
+  // which the workspace holds)
   const int64_t words = (K + 15) / 16;
+  const int64_t cbs = (words + 31) / 32;
+  int64_t rbs = (2 * static_cast<int64_t>(device_sms()) + cbs - 1) / cbs;
+  int64_t rows = (N + rbs - 1) / rbs;
+  rows = rows < kDxMinRows ? kDxMinRows : (rows + 7) / 8 * 8;
+  rbs = (N + rows - 1) / rows;
+  const dim3 grid(static_cast<unsigned>(cbs), static_cast<unsigned>(rbs));
   for (int64_t m0 = 0; m0 < M; m0 += kDxTokens) {
     const int mt = (M - m0) < kDxTokens ? static_cast<int>(M - m0) : kDxTokens;
-    const unsigned gp = grid_of(words * chunks, 8);
     const unsigned gr = grid_of(mt * K, 8);
     cudaError_t e;
-    if (dydt == BL_F32) {
-      e = mt == 2 ? launch_pdl(backward_dx_partial_kernel<BL_F32, 2>, gp, 256, 0, st, packed, rowbytes, N, K, dy, m0, part)
-                  : launch_pdl(backward_dx_partial_kernel<BL_F32, 1>, gp, 256, 0, st, packed, rowbytes, N, K, dy, m0, part);
-    } else {
-      e = mt == 2 ? launch_pdl(backward_dx_partial_kernel<BL_BF16, 2>, gp, 256, 0, st, packed, rowbytes, N, K, dy, m0, part)
-                  : launch_pdl(backward_dx_partial_kernel<BL_BF16, 1>, gp, 256, 0, st, packed, rowbytes, N, K, dy, m0, part);
-    }
+    if (dydt == BL_F32)
+      e = mt == 2 ? launch_dx_tile<BL_F32, 2>(grid, packed, rowbytes, N, K, dy, m0, rows, part, st)
+                  : launch_dx_tile<BL_F32, 1>(grid, packed, rowbytes, N, K, dy, m0, rows, part, st);
+    else
+      e = mt == 2 ? launch_dx_tile<BL_BF16, 2>(grid, packed, rowbytes, N, K, dy, m0, rows, part, st)
+                  : launch_dx_tile<BL_BF16, 1>(grid, packed, rowbytes, N, K, dy, m0, rows, part, st);
     if (e != cudaSuccess) return e;
-    e = mt == 2 ? launch_pdl(backward_dx_reduce_kernel<2>, gr, 256, 0, st, part, chunks, K, gamma, m0, dx)
-                : launch_pdl(backward_dx_reduce_kernel<1>, gr, 256, 0, st, part, chunks, K, gamma, m0, dx);
+    e = mt == 2 ? launch_pdl(backward_dx_reduce_kernel<2>, gr, 256, 0, st, part, rbs, K, gamma, m0, dx)
+                : launch_pdl(backward_dx_reduce_kernel<1>, gr, 256, 0, st, part, rbs, K, gamma, m0, dx);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();

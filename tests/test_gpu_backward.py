@@ -74,11 +74,13 @@ def run_dx(packed, fmt, g, N, K, dy):
 
 @pytest.mark.parametrize("M,N,K,fmt,dydt", [
     (1, 512, 256, I2, "f32"),
-    (3, 777, 1000, I2, "bf16"),     # K % 16 != 0: a partial last word; 13 row chunks, the last partial
+    (3, 777, 1000, I2, "bf16"),     # K % 16 != 0: a partial last word; row blocks, the last partial
     (2, 3200, 3200, T5, "f32"),     # base 3 through the 2-bit transcoding
     (5, 300, 129, B1, "f32"),       # 1-bit (codes in {-1, +1}); three passes of two tokens
     (1, 8640, 3200, I2, "bf16"),    # 3B up-projection shape, one token
     (4, 1, 64, I2, "f32"),          # one row
+    (128, 640, 512, I2, "bf16"),    # many tokens: 64 passes of two
+    (1, 3200, 8640, I2, "f32"),     # 3B down-projection shape: 17 column blocks
 ])
 def test_backward_dx(orc, M, N, K, fmt, dydt):
     g, packed, codes = _weights(orc, N, K, fmt, 720 + K)
