@@ -145,7 +145,7 @@ template <int XDT, int XC, int S, bool ALIGNED>
 __global__ void __launch_bounds__(kG1MaxThreads, 2)
     gemv1_i2_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
                     int64_t N, int64_t K, const void* __restrict__ x, float* __restrict__ scale,
-                    void* __restrict__ y, int ydt, int write_scale, const RowGroups rg, int R, void* ws) {
+                    void* __restrict__ y, int ydt, int write_scale, const RowGroups rg, int R, int lpr, void* ws) {
   constexpr int kXW = g1_xwords<XDT>();
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ uint32_t red[kG1MaxThreads / 32];
@@ -161,11 +161,17 @@ __global__ void __launch_bounds__(kG1MaxThreads, 2)
   const int64_t per = N / G, extra = N % G;
   const int64_t row0 = b * per + (b < extra ? b : extra);
   const int nrows = static_cast<int>(per + (b < extra ? 1 : 0));
-  const bool active = tid < R * segs;
-  const int r0 = active ? tid / segs : 0;  // this thread's first row (of the CTA's rows)
-  const int c = active ? tid - r0 * segs : 0;
+  // lpr lanes per row (segs, or segs rounded up to whole warps so that every
+  // warp lies in one row); lane c < segs of a row holds column c
+  // (the idle lanes of a row take part in every step with zero codes and no
+  // copies, so all lanes of a warp run the same steps)
+  const int r0_raw = tid / lpr, c_raw = tid - r0_raw * lpr;
+  const bool row_ok = r0_raw < R;
+  const bool col_ok = row_ok && c_raw < segs;
+  const int r0 = row_ok ? r0_raw : 0;  // this thread's first row (of the CTA's rows)
+  const int c = col_ok ? c_raw : 0;
   // rows of this thread: r0, r0 + R, ... below nrows
-  const int nr = (active && r0 < nrows) ? (nrows - r0 + R - 1) / R : 0;
+  const int nr = (row_ok && r0 < nrows) ? (nrows - r0 + R - 1) / R : 0;
   const uint32_t step = static_cast<uint32_t>(R * rowbytes);  // bytes between a thread's rows (<= 8 KB)
   const int kch = static_cast<int>(K >> 4);  // chunks holding weights (K % 16 == 0)
   const int nch = 4 * segs;                  // chunks of the packed rows (the last ones are padding)
@@ -226,10 +232,10 @@ __global__ void __launch_bounds__(kG1MaxThreads, 2)
     return;
   }
   // the thread's first S - 1 rows (one cp.async group each, empty past its rows)
-  const uint8_t* gp = packed + row0 * rowbytes + static_cast<int64_t>(tid) * 16;  // next row to copy
+  const uint8_t* gp = packed + (row0 + r0) * rowbytes + static_cast<int64_t>(c) * 16;  // next row to copy
 #pragma unroll
   for (int j = 0; j < S - 1; ++j) {
-    if (j < nr) cp_async16_s(ring_s + j * tstride, gp);
+    if (col_ok && j < nr) cp_async16_s(ring_s + j * tstride, gp);
     cp_async_commit();
     gp += step;
   }
@@ -329,7 +335,7 @@ __global__ void __launch_bounds__(kG1MaxThreads, 2)
   int csum = 0;
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
-    X[w] = active ? *reinterpret_cast<const uint4*>(xbuf + (static_cast<int64_t>(w) * segs + c) * 16)
+    X[w] = col_ok ? *reinterpret_cast<const uint4*>(xbuf + (static_cast<int64_t>(w) * segs + c) * 16)
                   : make_uint4(0, 0, 0, 0);
     csum = __dp4a(static_cast<int>(X[w].x), 0x01010101, csum);
     csum = __dp4a(static_cast<int>(X[w].y), 0x01010101, csum);
@@ -338,7 +344,7 @@ __global__ void __launch_bounds__(kG1MaxThreads, 2)
   }
   const int init = -csum;
   // lanes with the same first row share a row at every step
-  const uint32_t gmask = ALIGNED ? 0xffffffffu : __match_any_sync(0xffffffffu, active ? r0 : -1 - lane);
+  const uint32_t gmask = ALIGNED ? 0xffffffffu : __match_any_sync(0xffffffffu, row_ok ? r0_raw : -1 - lane);
   const bool leader = ALIGNED ? lane == 0 : (__ffs(gmask) - 1) == lane;
   uint32_t rs = smem_u32(rsum + r0);    // this thread's next row sum
   const uint32_t rstep = 4u * R;
@@ -358,7 +364,7 @@ __global__ void __launch_bounds__(kG1MaxThreads, 2)
   for (; k < nr - 2 * S + 2; k += S) {
 #pragma unroll
     for (int j = 0; j < S; ++j) {
-      cp_async16_s(ring_s + ((j + S - 1) % S) * tstride, gp);
+      if (col_ok) cp_async16_s(ring_s + ((j + S - 1) % S) * tstride, gp);
       cp_async_commit();
       gp += step;
       cp_async_wait<S - 1>();
@@ -366,7 +372,7 @@ __global__ void __launch_bounds__(kG1MaxThreads, 2)
     }
   }
   for (; k < nr; ++k) {
-    if (k + S - 1 < nr) cp_async16_s(ring_s + ((k + S - 1) % S) * tstride, gp);
+    if (col_ok && k + S - 1 < nr) cp_async16_s(ring_s + ((k + S - 1) % S) * tstride, gp);
     cp_async_commit();
     gp += step;
     cp_async_wait<S - 1>();
@@ -399,7 +405,7 @@ __global__ void __launch_bounds__(kG1MaxThreads, 2)
 // Launch geometry: R rows per step, threads rounded up to whole warps, and
 // the token chunks per thread (1, 2 or 4).
 struct Gemv1Geom {
-  int R, threads, xc, stages;
+  int R, lpr, threads, xc, stages;
   int64_t grid, rows_per_cta, smem;
 };
 
@@ -409,10 +415,15 @@ static bool gemv1_geom(int64_t N, int64_t K, int64_t rowbytes, int xdt, Gemv1Geo
   const int64_t sms = device_sms();
   g->grid = N < sms ? N : sms;
   g->rows_per_cta = (N + g->grid - 1) / g->grid;
-  int64_t R = kG1MaxThreads / segs;
+  // rows of at least 32 segments take whole warps (the lanes past the row's
+  // end idle), so that every warp lies in one row and sums with a full mask
+  const int64_t lpr = segs >= 32 ? (segs + 31) / 32 * 32 : segs;
+  if (lpr > kG1MaxThreads) return false;
+  int64_t R = kG1MaxThreads / lpr;
   if (R > g->rows_per_cta) R = g->rows_per_cta;
   g->R = static_cast<int>(R);
-  g->threads = static_cast<int>((R * segs + 31) / 32 * 32);
+  g->lpr = static_cast<int>(lpr);
+  g->threads = static_cast<int>((R * lpr + 31) / 32 * 32);
   const int64_t per = (4 * segs + g->threads - 1) / g->threads;
   g->xc = per <= 1 ? 1 : (per <= 2 ? 2 : 4);
   const int xwords = xdt == BL_F32 ? 4 : (xdt == BL_BF16 ? 2 : 1);
@@ -434,7 +445,7 @@ template <int XDT, int XC, int S>
 static cudaError_t launch_gemv1_t(const Gemv1Geom& g, const uint8_t* packed, int64_t rowbytes, const float* gamma,
                                   int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
                                   int write_scale, const RowGroups& rg, void* ws, cudaStream_t st) {
-  auto kern = (rowbytes / 16) % 32 == 0 ? gemv1_i2_kernel<XDT, XC, S, true> : gemv1_i2_kernel<XDT, XC, S, false>;
+  auto kern = g.lpr % 32 == 0 ? gemv1_i2_kernel<XDT, XC, S, true> : gemv1_i2_kernel<XDT, XC, S, false>;
   const size_t smem = static_cast<size_t>(g.smem);
   if (smem > 48 * 1024) {
     const cudaError_t e =
@@ -442,7 +453,7 @@ static cudaError_t launch_gemv1_t(const Gemv1Geom& g, const uint8_t* packed, int
     if (e != cudaSuccess) return e;
   }
   const cudaError_t e = launch_pdl(kern, static_cast<unsigned>(g.grid), static_cast<unsigned>(g.threads), smem, st,
-                                   packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, g.R, ws);
+                                   packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, g.R, g.lpr, ws);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
