@@ -43,8 +43,14 @@
 
 namespace bl {
 
-constexpr int kG1MaxThreads = 512;
-constexpr int64_t kG1MaxSmem = 110 * 1024;  // two CTAs (of consecutive launches) per SM
+#ifndef BL_G1_MAXT
+#define BL_G1_MAXT 512
+#endif
+#ifndef BL_G1_MAXSMEM
+#define BL_G1_MAXSMEM (110 * 1024)
+#endif
+constexpr int kG1MaxThreads = BL_G1_MAXT;
+constexpr int64_t kG1MaxSmem = BL_G1_MAXSMEM;  // two CTAs (of consecutive launches) per SM
 
 // 16-byte words of raw activations per 16 elements.
 template <int XDT>
@@ -111,16 +117,23 @@ __device__ __forceinline__ int dot_seg_i2(const uint4 wv, const uint4 (&X)[4], i
 // on the largest |t_a - rint(t_a)| (an exact difference), and only a group
 // with an element that close to a tie takes the exact quotient.
 __device__ __forceinline__ uint4 g1_codes16(const float (&e)[16], float s, float c127) {
+  // element pairs through the paired fp32 unit (each lane rounds to nearest
+  // as the scalar operation does); ta - rint(ta) = fma(rint(ta), -1, ta) is
+  // exact, so one rounding of an exact value
+  const float2 c2 = make_float2(c127, c127), mg = make_float2(12582912.0f, 12582912.0f);
+  const float2 nmg = make_float2(-12582912.0f, -12582912.0f), m1 = make_float2(-1.0f, -1.0f);
   uint32_t r[16];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     float worst = 0.0f;
 #pragma unroll
-    for (int j = 8 * h; j < 8 * h + 8; ++j) {
-      const float ta = __fmul_rn(e[j], c127);
-      const float r2 = __fadd_rn(ta, 12582912.0f);
-      worst = fmaxf(worst, fabsf(__fsub_rn(ta, __fsub_rn(r2, 12582912.0f))));
-      r[j] = __float_as_uint(r2);
+    for (int j = 8 * h; j < 8 * h + 8; j += 2) {
+      const float2 ta = __fmul2_rn(make_float2(e[j], e[j + 1]), c2);
+      const float2 r2 = __fadd2_rn(ta, mg);
+      const float2 d = __ffma2_rn(__fadd2_rn(r2, nmg), m1, ta);
+      worst = fmaxf(worst, fmaxf(fabsf(d.x), fabsf(d.y)));
+      r[j] = __float_as_uint(r2.x);
+      r[j + 1] = __float_as_uint(r2.y);
     }
     if (!(worst < 0.49993896484375f)) {  // rare: some element is near a tie
 #pragma unroll
@@ -142,7 +155,7 @@ __device__ __forceinline__ uint4 g1_codes16(const float (&e)[16], float s, float
 // 4c .. 4c + 3; chunk g of thread t is t + T u, u < XC).  S: stages of the
 // thread's row ring.  ALIGNED: segs % 32 == 0, so every warp lies in one row.
 template <int XDT, int XC, int S, bool ALIGNED>
-__global__ void __launch_bounds__(kG1MaxThreads, 2)
+__global__ void __launch_bounds__(kG1MaxThreads, 1024 / kG1MaxThreads)
     gemv1_i2_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
                     int64_t N, int64_t K, const void* __restrict__ x, float* __restrict__ scale,
                     void* __restrict__ y, int ydt, int write_scale, const RowGroups rg, int R, int lpr, void* ws) {
