@@ -74,15 +74,18 @@ __global__ void __launch_bounds__(kDxWarps * 32)
       }
 #pragma unroll
       for (int j = 0; j < kDxAhead; ++j) {
+        // bit 2i of pos / neg: weight i of the word is +1 / -1 (digit 2 / 0)
+        const uint32_t w = wv[j];
+        const uint32_t pos = (w >> 1) & ~w & 0x55555555u;
+        const uint32_t neg = ~(w | (w >> 1)) & 0x55555555u;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const uint32_t d = (wv[j] >> (2 * i)) & 3u;  // digit q + 1
 #pragma unroll
           for (int m = 0; m < MT; ++m) {
-            if (d == 2u)
-              acc[m][i] = __dadd_rn(acc[m][i], gv[j][m]);
-            else if (d == 0u)
-              acc[m][i] = __dadd_rn(acc[m][i], -gv[j][m]);
+            // two independent one-instruction conditionals (predicated adds,
+            // no divergent branch)
+            if (pos & (1u << (2 * i))) acc[m][i] = __dadd_rn(acc[m][i], gv[j][m]);
+            if (neg & (1u << (2 * i))) acc[m][i] = __dadd_rn(acc[m][i], -gv[j][m]);
           }
         }
       }
@@ -106,24 +109,36 @@ __global__ void __launch_bounds__(kDxWarps * 32)
   }
 }
 
-// dx[m0 + m, k] = fp32(gamma * sum_r part[r][m][k]), r in order.
+// dx[m0 + m, k] = fp32(gamma * sum_r part[r][m][k]).  A CTA takes 32
+// columns (lane L column 32 blockIdx.x + L, so each read of a partial row is
+// coalesced) of token m = blockIdx.y; warp w adds the row blocks
+// [w C / 8, (w + 1) C / 8) in order, and the 8 warp sums meet in warp order
+// through shared memory (a fixed order: the result is the same on every run).
 template <int MT>
 __global__ void __launch_bounds__(256)
     backward_dx_reduce_kernel(const double* __restrict__ part, int64_t chunks, int64_t K, const float* __restrict__ gamma,
                               int64_t m0, float* __restrict__ dx) {
   pdl_enter(part, gamma, dx);
+  __shared__ double sh[8][32];
   __shared__ double sh_g;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) sh_g = static_cast<double>(__ldcg(gamma));
+  const int m = blockIdx.y;
+  const int64_t k = static_cast<int64_t>(blockIdx.x) * 32 + lane;
+  const int64_t r0 = chunks * warp / 8, r1 = chunks * (warp + 1) / 8;
+  double S = 0.0;
+  if (k < K) {
+    const double* p = part + m * K + k;
+#pragma unroll 4
+    for (int64_t r = r0; r < r1; ++r) S = __dadd_rn(S, __ldcg(p + r * MT * K));
+  }
+  sh[warp][lane] = S;
   __syncthreads();
-  const double g = sh_g;
-  const int64_t total = MT * K;
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t m = e / K, k = e - m * K;
-    double S = 0.0;
-#pragma unroll 8
-    for (int64_t r = 0; r < chunks; ++r) S = __dadd_rn(S, __ldcg(part + (r * MT + m) * K + k));
-    dx[(m0 + m) * K + k] = __double2float_rn(__dmul_rn(g, S));
+  if (warp == 0 && k < K) {
+    double t = sh[0][lane];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) t = __dadd_rn(t, sh[w][lane]);
+    dx[(m0 + m) * K + k] = __double2float_rn(__dmul_rn(sh_g, t));
   }
 }
 
@@ -241,7 +256,7 @@ cudaError_t launch_backward_dx(const uint8_t* packed, int64_t rowbytes, const fl
   const dim3 grid(static_cast<unsigned>(cbs), static_cast<unsigned>(rbs));
   for (int64_t m0 = 0; m0 < M; m0 += kDxTokens) {
     const int mt = (M - m0) < kDxTokens ? static_cast<int>(M - m0) : kDxTokens;
-    const unsigned gr = grid_of(mt * K, 8);
+    const dim3 gr(static_cast<unsigned>((K + 31) / 32), static_cast<unsigned>(mt));
     cudaError_t e;
     if (dydt == BL_F32)
       e = mt == 2 ? launch_dx_tile<BL_F32, 2>(grid, packed, rowbytes, N, K, dy, m0, rows, part, st)

@@ -850,49 +850,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-// T5 -> 2-bit transcoding (for the tensor-core path on base-3 weights): one
-// thread writes one 16-byte segment (64 weights) of a 2-bit row.  The base-3
-// digit of a weight is its 2-bit code (both are q + 1); invalid bytes (>= 243)
-// read as weight 0, as in the decode kernel.
+// Base-3 rows re-encoded as 2-bit rows (a base-3 digit is the 2-bit code of
+// the same weight), for the tensor-core path.  Item (n, t): the 16 base-3
+// bytes 16t .. 16t + 15 of row n (weights 80t .. 80t + 79; bytes past rb5 read
+// as padding, 121 = five weight-0 digits) become 160 bits, i.e. five 32-bit
+// words at byte 20t of the 2-bit row (words past rb2 are dropped).  A byte's
+// five codes come from a 256-entry table of 10-bit entries with one copy per
+// lane, so the 32 lookups of a warp are one conflict-free access.
 __global__ void __launch_bounds__(256)
     t5_to_i2_kernel(const uint8_t* __restrict__ t5, int64_t N, int64_t K, int64_t rb5, uint8_t* __restrict__ i2,
                     int64_t rb2) {
   pdl_enter(t5, i2);
-  __shared__ uint16_t lut[256];
-  for (int b = threadIdx.x; b < 256; b += blockDim.x) {
-    uint32_t v = b, d = 0;
+  __shared__ uint32_t lut[256][32];
+  for (int e = threadIdx.x; e < 256 * 32; e += blockDim.x) {
+    const int b = e >> 5;
+    uint32_t v = static_cast<uint32_t>(b), d = 0x155u;  // bytes 243..255: five weight-0 digits
     if (b < 243) {
+      d = 0;
       for (int i = 0; i < 5; ++i) {
         d |= (v % 3) << (2 * i);
         v /= 3;
       }
-    } else {
-      d = 0x155;  // five weight-0 digits
     }
-    lut[b] = static_cast<uint16_t>(d);
+    lut[b][e & 31] = d;
   }
   __syncthreads();
-  const int64_t segs = rb2 / 16;
-  for (int64_t gid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; gid < N * segs;
-       gid += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t n = gid / segs, sg = gid - n * segs;
-    const int64_t kb = 64 * sg;
-    uint32_t out[4] = {0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u};
-    const uint8_t* row = t5 + n * rb5;
-    for (int64_t b = kb / 5; b <= (kb + 63) / 5; ++b) {
-      const uint32_t digs = lut[b < rb5 ? row[b] : 121];
+  const int lane = threadIdx.x & 31;
+  // items fit in 32 bits (N K <= 2^32 and an item covers 80 weights): 32-bit
+  // index arithmetic, no 64-bit division per item
+  const uint32_t per_row = static_cast<uint32_t>((rb2 + 19) / 20);
+  const uint32_t words2 = static_cast<uint32_t>(rb2 / 4);
+  const uint32_t items = static_cast<uint32_t>(N) * per_row;
+  for (uint32_t gid = blockIdx.x * blockDim.x + threadIdx.x; gid < items; gid += gridDim.x * blockDim.x) {
+    const uint32_t nn = gid / per_row, t = gid - nn * per_row;
+    const int64_t n = nn;
+    const uint4 v = 16 * static_cast<int64_t>(t) < rb5 ? __ldcg(reinterpret_cast<const uint4*>(t5 + n * rb5 + 16 * t))
+                                 : make_uint4(0x79797979u, 0x79797979u, 0x79797979u, 0x79797979u);
+    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[6] = {0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
-      for (int i = 0; i < 5; ++i) {
-        const int64_t k = 5 * b + i, kk = k - kb;
-        if (kk >= 0 && kk < 64) {
-          const uint32_t code = (k < K) ? ((digs >> (2 * i)) & 3u) : 1u;
-          const int wi = static_cast<int>(kk >> 4), sh = static_cast<int>(2 * (kk & 15));
-          out[wi] = (out[wi] & ~(3u << sh)) | (code << sh);
-        }
-      }
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t d = lut[(wd[i >> 2] >> (8 * (i & 3))) & 0xffu][lane];
+      const int pos = 10 * i, w = pos >> 5, sh = pos & 31;
+      out[w] |= d << sh;
+      if (sh > 22) out[w + 1] |= d >> (32 - sh);
     }
-    *reinterpret_cast<uint4*>(i2 + n * rb2 + sg * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(i2 + n * rb2) + 5 * t;
+#pragma unroll
+    for (int j = 0; j < 5; ++j)
+      if (5 * t + j < words2) dst[j] = out[j];
   }
+  (void)K;  // the padding digits past K are weight-0 codes in both formats
 }
 
 // 1-bit -> 2-bit transcoding (for the tensor-core path, and for decode rows
@@ -912,16 +920,21 @@ __global__ void __launch_bounds__(256)
     b1_to_i2_kernel(const uint8_t* __restrict__ b1, int64_t N, int64_t K, int64_t rb1, uint8_t* __restrict__ i2,
                     int64_t rb2) {
   pdl_enter(b1, i2);
-  const int64_t segs = rb2 / 16;
-  for (int64_t gid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; gid < N * segs;
-       gid += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t n = gid / segs, sg = gid - n * segs;
+  // N segs < 2^32 (N K <= 2^32, a segment covers 64 weights): 32-bit index
+  // arithmetic, no 64-bit division per segment
+  const uint32_t segs = static_cast<uint32_t>(rb2 / 16);
+  const uint32_t items = static_cast<uint32_t>(N) * segs;
+  for (uint32_t gid = blockIdx.x * blockDim.x + threadIdx.x; gid < items; gid += gridDim.x * blockDim.x) {
+    const uint32_t nn = gid / segs, sg32 = gid - nn * segs;
+    const int64_t n = nn, sg = sg32;
     const uint8_t* row = b1 + n * rb1;
     uint32_t out[4];
+    // the segment's eight 1-bit bytes in one load (rb1 is a multiple of 16, so
+    // they are all in the row or all past it)
+    const uint2 raw = 8 * sg < rb1 ? __ldcg(reinterpret_cast<const uint2*>(row + 8 * sg)) : make_uint2(0u, 0u);
 #pragma unroll
     for (int w = 0; w < 4; ++w) {  // 16 weights: two bytes of the 1-bit row
-      const int64_t j = 8 * sg + 2 * w;
-      const uint32_t bits = (j < rb1 ? __ldcg(row + j) : 0u) | ((j + 1 < rb1 ? __ldcg(row + j + 1) : 0u) << 8);
+      const uint32_t bits = ((w < 2 ? raw.x : raw.y) >> (16 * (w & 1))) & 0xffffu;
       uint32_t d = spread16_to_2bit(bits) << 1;  // +1 -> 10, -1 -> 00
       const int64_t k0 = 64 * sg + 16 * w;
       if (k0 + 16 > K) {
@@ -1110,7 +1123,7 @@ cudaError_t launch_b1_to_i2(const uint8_t* b1, int64_t N, int64_t K, int64_t rb1
 
 cudaError_t launch_t5_to_i2(const uint8_t* t5, int64_t N, int64_t K, int64_t rb5, uint8_t* i2, int64_t rb2,
                             cudaStream_t st) {
-  const int64_t work = N * (rb2 / 16);
+  const int64_t work = N * ((rb2 + 19) / 20);
   const int64_t cap = static_cast<int64_t>(device_sms()) * 8;
   int64_t grid = (work + 255) / 256;
   if (grid > cap) grid = cap;
