@@ -63,7 +63,9 @@ KERNEL_SOURCE = {"absmean_kernel": "bl_weights.cu", "ternarize_flat_kernel": "bl
                  "gemv_kernel": "bl_gemv.cu", "gemv_t5_kernel": "bl_gemv.cu", "gemv_i2_mt_kernel": "bl_gemv.cu", "act_quant_row_kernel": "bl_acts.cu",
                  "act_quant_kernel": "bl_acts.cu", "ln_quant_kernel": "bl_acts.cu", "ln_quant_reg_kernel": "bl_acts.cu", "gemm_i2_2sm_kernel": "bl_gemm_sm100.cu",
                  "gemm_i2_kernel": "bl_gemm_sm100.cu", "b1_to_i2_kernel": "bl_gemm_sm100.cu",
-                 "backward_dx_partial_kernel": "bl_backward.cu", "backward_dx_reduce_kernel": "bl_backward.cu",
+                 "t5_to_i2_kernel": "bl_gemm_sm100.cu", "splitk_reduce_kernel": "bl_gemm_sm100.cu",
+                 "pack_kernel": "bl_weights.cu",
+                 "backward_dx_tile_kernel": "bl_backward.cu", "backward_dx_reduce_kernel": "bl_backward.cu",
                  "backward_dw_kernel": "bl_backward.cu"}
 
 
