@@ -245,20 +245,28 @@ __global__ void __launch_bounds__(kLnThreads)
 // tree of the 256 lane sums takes one shared-memory write and one barrier:
 // every warp then reads the eight sums of its lane's subtree and adds them in
 // the tree's order (levels 128, 64, 32), and levels 16..1 run by shuffles --
-// each warp computes the same total, so no broadcast is needed.  y is
-// computed once and kept for the absmax and the codes.
+// each warp computes the same total, so no broadcast is needed.
+// The conversions to and from fp64 run on the SM's narrow conversion pipe, so
+// each is done once: the token's elements are converted once and kept in
+// registers as fp64 for the three passes, g and b are converted once per CTA
+// into shared memory (fp64 pairs (g_k, b_k)), and the next token's elements
+// are loaded while this one is normalised.  y is kept as bf16 pairs for the
+// absmax and the codes.
 constexpr int kLnRegThreads = 128;
 
 template <int XDT, int NI>
-__global__ void __launch_bounds__(kLnRegThreads, 4)
+__global__ void __launch_bounds__(kLnRegThreads, NI > 13 ? 3 : 4)
     ln_quant_reg_kernel(const void* __restrict__ x, const float* __restrict__ g, const float* __restrict__ b,
                         float eps, int64_t M, int64_t K, uint16_t* __restrict__ y, int8_t* __restrict__ xq,
                         float* __restrict__ scale) {
   pdl_enter(x, g, b, y, xq, scale);
+  extern __shared__ __align__(16) double2 gb[];  // [K]: (g_k, b_k) in fp64
   __shared__ __align__(16) double p1[256];
   __shared__ __align__(16) double p2[256];
   __shared__ float red[kLnRegThreads / 32];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  for (int64_t k = t; k < K; k += kLnRegThreads)
+    gb[k] = make_double2(static_cast<double>(__ldcg(g + k)), static_cast<double>(__ldcg(b + k)));
   // the tree of the 256 lane sums held in p, R18's order
   auto tree = [&](const double* p) -> double {
     const int L = lane;
@@ -278,42 +286,56 @@ __global__ void __launch_bounds__(kLnRegThreads, 4)
   auto hi = [](const Pair& v) -> float {
     if constexpr (kF32) return v.y; else return __uint_as_float(v & 0xffff0000u);
   };
-  const double dK = static_cast<double>(K);
-  for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+  auto load_token = [&](int64_t m, Pair (&xr)[NI]) {
     const int64_t base = m * K;
-    Pair xr[NI];  // the token's pairs; later y's bf16 pairs
 #pragma unroll
     for (int i = 0; i < NI; ++i) {
       const int64_t k = 2 * t + 256 * i;
       if constexpr (kF32) {
-        xr[i] = k < K ? __ldcg(reinterpret_cast<const float2*>(static_cast<const float*>(x) + base + k))
-                      : make_float2(0.0f, 0.0f);
+        xr[i] = (m < M && k < K) ? __ldcg(reinterpret_cast<const float2*>(static_cast<const float*>(x) + base + k))
+                                 : make_float2(0.0f, 0.0f);
       } else {
-        xr[i] = k < K ? __ldcg(reinterpret_cast<const unsigned int*>(static_cast<const uint16_t*>(x) + base + k))
-                      : 0u;
+        xr[i] = (m < M && k < K)
+                    ? __ldcg(reinterpret_cast<const unsigned int*>(static_cast<const uint16_t*>(x) + base + k))
+                    : 0u;
       }
     }
+  };
+  const double dK = static_cast<double>(K);
+  Pair xr[NI];  // the token's raw pairs; loaded one token ahead
+  load_token(blockIdx.x, xr);
+  __syncthreads();  // gb is complete
+  for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+    const int64_t base = m * K;
+    double xa[NI], xb[NI];  // lanes 2t and 2t + 1 in fp64 (0 past K)
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+      xa[i] = static_cast<double>(lo(xr[i]));
+      xb[i] = static_cast<double>(hi(xr[i]));
+    }
+    load_token(m + gridDim.x, xr);  // in flight during the three passes
     // mean: each lane's elements in turn from 0.0
     double sa = 0.0, sb = 0.0;
 #pragma unroll
     for (int i = 0; i < NI; ++i)
       if (2 * t + 256 * i < K) {
-        sa = __dadd_rn(sa, static_cast<double>(lo(xr[i])));
-        sb = __dadd_rn(sb, static_cast<double>(hi(xr[i])));
+        sa = __dadd_rn(sa, xa[i]);
+        sb = __dadd_rn(sb, xb[i]);
       }
     reinterpret_cast<double2*>(p1)[t] = make_double2(sa, sb);
     __syncthreads();
     const double mu = __ddiv_rn(tree(p1), dK);
-    // variance: (x - mu)^2 in the same order
+    // variance: (x - mu)^2 in the same order; x - mu kept for y
     sa = sb = 0.0;
 #pragma unroll
-    for (int i = 0; i < NI; ++i)
+    for (int i = 0; i < NI; ++i) {
+      xa[i] = __dsub_rn(xa[i], mu);
+      xb[i] = __dsub_rn(xb[i], mu);
       if (2 * t + 256 * i < K) {
-        const double da = __dsub_rn(static_cast<double>(lo(xr[i])), mu);
-        const double db = __dsub_rn(static_cast<double>(hi(xr[i])), mu);
-        sa = __dadd_rn(sa, __dmul_rn(da, da));
-        sb = __dadd_rn(sb, __dmul_rn(db, db));
+        sa = __dadd_rn(sa, __dmul_rn(xa[i], xa[i]));
+        sb = __dadd_rn(sb, __dmul_rn(xb[i], xb[i]));
       }
+    }
     reinterpret_cast<double2*>(p2)[t] = make_double2(sa, sb);
     __syncthreads();
     const double var = __ddiv_rn(tree(p2), dK);
@@ -326,14 +348,9 @@ __global__ void __launch_bounds__(kLnRegThreads, 4)
       const int64_t k = 2 * t + 256 * i;
       yr[i] = 0u;
       if (k < K) {
-        const float2 gg = __ldcg(reinterpret_cast<const float2*>(g + k));
-        const float2 bb = __ldcg(reinterpret_cast<const float2*>(b + k));
-        const double va = __dadd_rn(__dmul_rn(__dmul_rn(__dsub_rn(static_cast<double>(lo(xr[i])), mu), r),
-                                              static_cast<double>(gg.x)),
-                                    static_cast<double>(bb.x));
-        const double vb = __dadd_rn(__dmul_rn(__dmul_rn(__dsub_rn(static_cast<double>(hi(xr[i])), mu), r),
-                                              static_cast<double>(gg.y)),
-                                    static_cast<double>(bb.y));
+        const double2 ga = gb[k], gbb = gb[k + 1];
+        const double va = __dadd_rn(__dmul_rn(__dmul_rn(xa[i], r), ga.x), ga.y);
+        const double vb = __dadd_rn(__dmul_rn(__dmul_rn(xb[i], r), gbb.x), gbb.y);
         const uint32_t ha = __bfloat16_as_ushort(__float2bfloat16_rn(__double2float_rn(va)));
         const uint32_t hb = __bfloat16_as_ushort(__float2bfloat16_rn(__double2float_rn(vb)));
         yr[i] = ha | (hb << 16);
@@ -369,11 +386,18 @@ static cudaError_t launch_ln_quant_reg(const void* x, const float* g, const floa
                                        uint16_t* y, int8_t* xq, float* scale, cudaStream_t st) {
   int per_sm = 1;
   auto kern = ln_quant_reg_kernel<XDT, NI>;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kLnRegThreads, 0) != cudaSuccess || per_sm < 1)
+  const size_t smem = static_cast<size_t>(K) * sizeof(double2);
+  // the 4 KB of static shared memory plus the dynamic part can pass the 48 KB
+  // default well before the dynamic part alone does: opt in early
+  if (smem > 32 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kLnRegThreads, smem) != cudaSuccess || per_sm < 1)
     per_sm = 1;
   const int64_t cap = static_cast<int64_t>(device_sms()) * per_sm;
   const unsigned grid = static_cast<unsigned>(M < cap ? M : cap);
-  const cudaError_t e = launch_pdl(kern, grid, kLnRegThreads, 0, st, x, g, b, eps, M, K, y, xq, scale);
+  const cudaError_t e = launch_pdl(kern, grid, kLnRegThreads, smem, st, x, g, b, eps, M, K, y, xq, scale);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -389,6 +413,9 @@ cudaError_t launch_ln_quant(const void* x, int xdt, const float* g, const float*
   if (pairs && K <= 256 * 8)
     return xdt == BL_F32 ? launch_ln_quant_reg<BL_F32, 8>(x, g, b, eps, M, K, y, xq, scale, st)
                          : launch_ln_quant_reg<BL_BF16, 8>(x, g, b, eps, M, K, y, xq, scale, st);
+  if (pairs && K <= 256 * 13)  // the 3B hidden size, 3200, without idle registers
+    return xdt == BL_F32 ? launch_ln_quant_reg<BL_F32, 13>(x, g, b, eps, M, K, y, xq, scale, st)
+                         : launch_ln_quant_reg<BL_BF16, 13>(x, g, b, eps, M, K, y, xq, scale, st);
   if (pairs && K <= 256 * 16)
     return xdt == BL_F32 ? launch_ln_quant_reg<BL_F32, 16>(x, g, b, eps, M, K, y, xq, scale, st)
                          : launch_ln_quant_reg<BL_BF16, 16>(x, g, b, eps, M, K, y, xq, scale, st);

@@ -81,6 +81,7 @@ def run_dx(packed, fmt, g, N, K, dy):
     (4, 1, 64, I2, "f32"),          # one row
     (128, 640, 512, I2, "bf16"),    # many tokens: 64 passes of two
     (1, 3200, 8640, I2, "f32"),     # 3B down-projection shape: 17 column blocks
+    (2, 6001, 8192, I2, "bf16"),    # row blocks of 320 rows: three chunks of row pairs, odd last row
 ])
 def test_backward_dx(orc, M, N, K, fmt, dydt):
     g, packed, codes = _weights(orc, N, K, fmt, 720 + K)

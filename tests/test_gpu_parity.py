@@ -391,6 +391,12 @@ def _ln_cases():
     yield "ragged_3x20001_f32", synth.normal_f32(71, (3, 20001))
     yield "k1_f32", synth.normal_f32(72, (4, 1))
     yield "70b_down_bf16", synth.to_bf16_bits(synth.normal_f32(73, (2, 28672)))
+    # the register form's three widths (K <= 2048, <= 3328, <= 4096), fp32 input,
+    # more tokens than resident CTAs (each CTA loads its next token ahead)
+    yield "1300x2048_f32", synth.normal_f32(75, (1300, 2048))
+    yield "900x3000_f32", synth.entry_outliers(synth.normal_f32(76, (900, 3000)), 77, 0.01, 20.0)
+    yield "700x4096_bf16", synth.to_bf16_bits(synth.normal_f32(78, (700, 4096)))
+    yield "5x3330_f32", synth.normal_f32(79, (5, 3330))
     c = synth.normal_f32(74, (4, 300))
     c[1] = 0.375  # a constant token: y = ln_b
     c[2] = 0.0
