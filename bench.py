@@ -130,7 +130,8 @@ def profiled_traffic(kernel: str, workload: str):
 
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML while running."""
+    """Samples SM clock and throttle reasons through NVML while running (every
+    0.2 ms: the timed graphs of short workloads last about a millisecond)."""
 
     REASONS = {
         0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
@@ -138,7 +139,7 @@ class ClockSampler:
         0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.0002):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period, self._stop, self._t = period_s, threading.Event(), None
         try:

@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(kLnThreads)
 // The conversions to and from fp64 run on the SM's narrow conversion pipe, so
 // each is done once: the token's elements are converted once and kept in
 // registers as fp64 for the three passes, g and b are converted once per CTA
-// into shared memory (fp64 pairs (g_k, b_k)), and the next token's elements
+// into shared memory (fp64), and the next token's elements
 // are loaded while this one is normalised.  y is kept as bf16 pairs for the
 // absmax and the codes.
 constexpr int kLnRegThreads = 128;
@@ -260,13 +260,17 @@ __global__ void __launch_bounds__(kLnRegThreads, NI > 13 ? 3 : 4)
                         float eps, int64_t M, int64_t K, uint16_t* __restrict__ y, int8_t* __restrict__ xq,
                         float* __restrict__ scale) {
   pdl_enter(x, g, b, y, xq, scale);
-  extern __shared__ __align__(16) double2 gb[];  // [K]: (g_k, b_k) in fp64
+  extern __shared__ __align__(16) double gbs[];  // [2][K]: g then b in fp64 (a thread reads 16-byte pairs)
   __shared__ __align__(16) double p1[256];
   __shared__ __align__(16) double p2[256];
-  __shared__ float red[kLnRegThreads / 32];
+  __shared__ uint32_t red[kLnRegThreads / 32];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  for (int64_t k = t; k < K; k += kLnRegThreads)
-    gb[k] = make_double2(static_cast<double>(__ldcg(g + k)), static_cast<double>(__ldcg(b + k)));
+  double* gd = gbs;
+  double* bd = gbs + K;
+  for (int64_t k = t; k < K; k += kLnRegThreads) {
+    gd[k] = static_cast<double>(__ldcg(g + k));
+    bd[k] = static_cast<double>(__ldcg(b + k));
+  }
   // the tree of the 256 lane sums held in p, R18's order
   auto tree = [&](const double* p) -> double {
     const int L = lane;
@@ -340,40 +344,68 @@ __global__ void __launch_bounds__(kLnRegThreads, NI > 13 ? 3 : 4)
     __syncthreads();
     const double var = __ddiv_rn(tree(p2), dK);
     const double r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(var, static_cast<double>(eps))));
-    // y = ((x - mu) r) g + b, fp64 -> fp32 -> bf16, stored and kept (bf16 pairs)
+    // y = ((x - mu) r) g + b, fp64 -> fp32 -> bf16 (RNE, the pair in one
+    // conversion), stored and kept (bf16 pairs); the absmax on the magnitude
+    // bits of the pairs (finite values order like unsigned integers)
     uint32_t yr[NI];
-    float amax = 0.0f;
+    uint32_t mx = 0;
 #pragma unroll
     for (int i = 0; i < NI; ++i) {
       const int64_t k = 2 * t + 256 * i;
       yr[i] = 0u;
       if (k < K) {
-        const double2 ga = gb[k], gbb = gb[k + 1];
-        const double va = __dadd_rn(__dmul_rn(__dmul_rn(xa[i], r), ga.x), ga.y);
-        const double vb = __dadd_rn(__dmul_rn(__dmul_rn(xb[i], r), gbb.x), gbb.y);
-        const uint32_t ha = __bfloat16_as_ushort(__float2bfloat16_rn(__double2float_rn(va)));
-        const uint32_t hb = __bfloat16_as_ushort(__float2bfloat16_rn(__double2float_rn(vb)));
-        yr[i] = ha | (hb << 16);
+        const double2 gg = *reinterpret_cast<const double2*>(gd + k);
+        const double2 bb = *reinterpret_cast<const double2*>(bd + k);
+        const double va = __dadd_rn(__dmul_rn(__dmul_rn(xa[i], r), gg.x), bb.x);
+        const double vb = __dadd_rn(__dmul_rn(__dmul_rn(xb[i], r), gg.y), bb.y);
+        const __nv_bfloat162 h = __floats2bfloat162_rn(__double2float_rn(va), __double2float_rn(vb));
+        yr[i] = *reinterpret_cast<const uint32_t*>(&h);
         if (y != nullptr) *reinterpret_cast<uint32_t*>(y + base + k) = yr[i];
-        amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(ha << 16)), fabsf(__uint_as_float(hb << 16))));
+        mx = __vmaxu2(mx, yr[i] & 0x7fff7fffu);
       }
     }
-    amax = warp_maxf(amax);
-    if (lane == 0) red[warp] = amax;
+    mx = __reduce_max_sync(0xffffffffu, max(mx & 0xffffu, mx >> 16) << 16);  // fp32 bits
+    if (lane == 0) red[warp] = mx;
     __syncthreads();
-    float am = red[0];
+    uint32_t am = red[0];
 #pragma unroll
-    for (int w = 1; w < kLnRegThreads / 32; ++w) am = fmaxf(am, red[w]);
-    const float s = fmaxf(am, 1e-6f);
+    for (int w = 1; w < kLnRegThreads / 32; ++w) am = max(am, red[w]);
+    const float s = fmaxf(__uint_as_float(am), 1e-6f);
     const float c127 = __fdiv_rn(127.0f, s);
+    // the codes by quant_act_fast's division-free rule, element pairs through
+    // the paired fp32 unit: t_a = y c127, rint(t_a) from the adder (the code
+    // in the low byte of the sum's bits), t_a - rint(t_a) exact by one fma;
+    // one margin test per thread, the exact quotient only near a tie
+    const float2 c2 = make_float2(c127, c127), mg = make_float2(12582912.0f, 12582912.0f);
+    const float2 nmg = make_float2(-12582912.0f, -12582912.0f), m1 = make_float2(-1.0f, -1.0f);
+    uint32_t qw[NI];
+    float worst = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+      const float2 ta = __fmul2_rn(make_float2(__uint_as_float(yr[i] << 16), __uint_as_float(yr[i] & 0xffff0000u)), c2);
+      const float2 r2 = __fadd2_rn(ta, mg);
+      const float2 d = __ffma2_rn(__fadd2_rn(r2, nmg), m1, ta);
+      worst = fmaxf(worst, fmaxf(fabsf(d.x), fabsf(d.y)));
+      qw[i] = __byte_perm(__float_as_uint(r2.x), __float_as_uint(r2.y), 0x0040);
+    }
+    if (!(worst < 0.49993896484375f)) {  // rare: some element is near a tie
+#pragma unroll
+      for (int i = 0; i < NI; ++i) {
+        const float e2[2] = {__uint_as_float(yr[i] << 16), __uint_as_float(yr[i] & 0xffff0000u)};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float ta = __fmul_rn(e2[h], c127);
+          if (!(fabsf(__fsub_rn(ta, rintf(ta))) < 0.49993896484375f)) {
+            const uint32_t q = static_cast<uint8_t>(quant_act_slow(e2[h], s));
+            qw[i] = h == 0 ? ((qw[i] & 0xff00u) | q) : ((qw[i] & 0x00ffu) | (q << 8));
+          }
+        }
+      }
+    }
 #pragma unroll
     for (int i = 0; i < NI; ++i) {
       const int64_t k = 2 * t + 256 * i;
-      if (k < K) {
-        const uint32_t qa = static_cast<uint8_t>(quant_act_fast(__uint_as_float(yr[i] << 16), s, c127));
-        const uint32_t qb = static_cast<uint8_t>(quant_act_fast(__uint_as_float(yr[i] & 0xffff0000u), s, c127));
-        *reinterpret_cast<uint16_t*>(xq + base + k) = static_cast<uint16_t>(qa | (qb << 8));
-      }
+      if (k < K) *reinterpret_cast<uint16_t*>(xq + base + k) = static_cast<uint16_t>(qw[i]);
     }
     if (t == 0) scale[m] = s;
     // red, p1 and p2 are free for the next token once every warp is past here
@@ -386,7 +418,7 @@ static cudaError_t launch_ln_quant_reg(const void* x, const float* g, const floa
                                        uint16_t* y, int8_t* xq, float* scale, cudaStream_t st) {
   int per_sm = 1;
   auto kern = ln_quant_reg_kernel<XDT, NI>;
-  const size_t smem = static_cast<size_t>(K) * sizeof(double2);
+  const size_t smem = static_cast<size_t>(2 * K) * sizeof(double);
   // the 4 KB of static shared memory plus the dynamic part can pass the 48 KB
   // default well before the dynamic part alone does: opt in early
   if (smem > 32 * 1024) {

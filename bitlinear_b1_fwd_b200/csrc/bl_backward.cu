@@ -19,7 +19,7 @@
 // in token order (the plain order of the sum), then gamma * T, rounded once
 // to fp32.
 // dx reads the packed 2-bit weights once per pass of up to two tokens in 2-D
-// tiles (512 columns x at least 64 rows: about two CTAs per SM, partial sums
+// tiles (512 columns x at least 64 rows: two or three CTAs per SM, partial sums
 // a few percent of the weight bytes); dW writes N K fp32 values (the
 // HBM-bound part for few tokens).
 #include "bl_common.cuh"
@@ -70,7 +70,7 @@ __device__ __forceinline__ double lds_f64(uint32_t addr) {
 // half of a double buffer.  The warps' sums meet in shared memory in a fixed
 // order and go to part[rb][m][k] (fp64).
 template <int DYT, int MT>
-__global__ void __launch_bounds__(kDxWarps * 32, 2)
+__global__ void __launch_bounds__(kDxWarps * 32, MT == 1 ? 3 : 2)
     backward_dx_tile_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, int64_t N, int64_t K,
                             const void* __restrict__ dy, int64_t m0, int64_t rows_per_block,
                             double* __restrict__ part) {
@@ -291,25 +291,37 @@ __global__ void __launch_bounds__(256)
         if (k0 + i < K) dst[i] = o[i];
     }
   };
+  // item e = (row nn, quad qq) with e = nn kq + qq; the grid stride S moves it
+  // by (S / kq, S mod kq) with one carry, so the loop divides only once
+  const uint32_t S = gridDim.x * blockDim.x;
+  const uint32_t Sn = S / kq, Sr = S - Sn * kq;
+  const uint32_t e0 = blockIdx.x * blockDim.x + threadIdx.x;
+  uint32_t nn = e0 / kq, qq = e0 - (e0 / kq) * kq;
+  auto advance = [&]() {
+    nn += Sn;
+    qq += Sr;
+    if (qq >= kq) {
+      qq -= kq;
+      ++nn;
+    }
+  };
   if (M <= kDwTokBlock) {  // every token's factor in shared memory once; no barrier in the loop
     if (threadIdx.x < M) sh_c[threadIdx.x] = __ddiv_rn(static_cast<double>(__ldcg(scale + threadIdx.x)), 127.0);
     __syncthreads();
     const double g = sh_g;
-    for (uint32_t e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
-      const uint32_t nn = e / kq;
-      const int64_t n = nn, k0 = 4 * static_cast<int64_t>(e - nn * kq);
+    for (uint32_t e = e0; e < total; e += S, advance()) {
+      const int64_t n = nn, k0 = 4 * static_cast<int64_t>(qq);
       double T[4] = {0.0, 0.0, 0.0, 0.0};
       for (int64_t m = 0; m < M; ++m) term4(m, n, k0, sh_c[m], T);
       store4(n, k0, T, g);
     }
     return;
   }
-  for (uint32_t base = blockIdx.x * blockDim.x; base < total; base += gridDim.x * blockDim.x) {
+  for (uint32_t base = blockIdx.x * blockDim.x; base < total; base += S, advance()) {
     const uint32_t e = base + threadIdx.x;
     const bool active = e < total;
-    const uint32_t nn = active ? e / kq : 0u;
-    const int64_t n = nn;
-    const int64_t k0 = active ? 4 * static_cast<int64_t>(e - nn * kq) : 0;
+    const int64_t n = active ? static_cast<int64_t>(nn) : 0;
+    const int64_t k0 = active ? 4 * static_cast<int64_t>(qq) : 0;
     double T[4] = {0.0, 0.0, 0.0, 0.0};
     for (int64_t t0 = 0; t0 < M; t0 += kDwTokBlock) {
       const int64_t tn = (M - t0) < kDwTokBlock ? (M - t0) : kDwTokBlock;
@@ -351,11 +363,12 @@ static cudaError_t launch_dx_tile(dim3 grid, const uint8_t* packed, int64_t rowb
 cudaError_t launch_backward_dx(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
                                const void* dy, int dydt, int64_t M, float* dx, double* part, cudaStream_t st) {
   // tiles: 512-column blocks x row blocks of at least kDxMinRows rows, about
-  // two CTAs per SM (the row blocks never outnumber backward_dx_chunks(N),
-  // which the workspace holds)
+  // as many CTAs as fit on the SMs at once (the row blocks never outnumber
+  // backward_dx_chunks(N), which the workspace holds)
   const int64_t words = (K + 15) / 16;
   const int64_t cbs = (words + 31) / 32;
-  int64_t rbs = (2 * static_cast<int64_t>(device_sms()) + cbs - 1) / cbs;
+  const int per_sm = M == 1 ? 3 : 2;  // the one-token tile kernel fits three CTAs per SM
+  int64_t rbs = (per_sm * static_cast<int64_t>(device_sms()) + cbs - 1) / cbs;
   int64_t rows = (N + rbs - 1) / rbs;
   rows = rows < kDxMinRows ? kDxMinRows : (rows + 7) / 8 * 8;
   rbs = (N + rows - 1) / rows;
