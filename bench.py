@@ -59,7 +59,7 @@ WORKLOADS = {
 
 KERNEL_SOURCE = {"absmean_kernel": "bl_weights.cu", "ternarize_flat_kernel": "bl_weights.cu",
                  "binarize_pack_kernel": "bl_weights.cu",
-                 "ternarize_pack_kernel": "bl_weights.cu", "gemv_i2_kernel": "bl_gemv.cu", "gemv1_i2_kernel": "bl_gemv1.cu",
+                 "ternarize_pack_kernel": "bl_weights.cu", "gemv_i2_kernel": "bl_gemv.cu", "gemv1_i2_kernel": "bl_gemv1.cu", "gemv1_t5_kernel": "bl_gemv1.cu",
                  "gemv_kernel": "bl_gemv.cu", "gemv_t5_kernel": "bl_gemv.cu", "gemv_i2_mt_kernel": "bl_gemv.cu", "act_quant_row_kernel": "bl_acts.cu",
                  "act_quant_kernel": "bl_acts.cu", "ln_quant_kernel": "bl_acts.cu", "ln_quant_reg_kernel": "bl_acts.cu", "gemm_i2_2sm_kernel": "bl_gemm_sm100.cu",
                  "gemm_i2_kernel": "bl_gemm_sm100.cu", "b1_to_i2_kernel": "bl_gemm_sm100.cu",
@@ -798,29 +798,58 @@ def decode_summary(d):
             "launch_duration": "CUDA events at the two ends of a graph of back-to-back forward calls"}
 
 
+def gemv1_fits(N, K, rb, t5=False, xwords=2):
+    """Mirror of the library's one-token kernel geometry (bf16 tokens by
+    default): K % 16 == 0, at most 512 lanes per row, at most four 16-byte code
+    chunks per thread, and the (table,) token region, row sums and a ring of 8
+    or 6 stages within 110 KB of shared memory."""
+    segs = rb // 16
+    lpr = segs if segs < 32 else -(-segs // 32) * 32
+    if K % 16 or segs < 1 or lpr > 512:
+        return False
+    grid = min(N, 148)
+    rpc = -(-N // grid)
+    R = min(512 // lpr, rpc)
+    threads = -(-(R * lpr) // 32) * 32
+    if -(-((5 if t5 else 4) * segs) // threads) > 4:
+        return False
+    xreg = -(-max(K * xwords, rb * (5 if t5 else 4)) // 16) * 16
+    fixed = (32768 if t5 else 0) + xreg + 4 * rpc
+    return any(fixed + 16 * st * threads <= 110 * 1024 for st in (8, 6))
+
+
 def gemv_kernel_name(fmt, layers, M=1):
-    """The decode kernel the forward dispatches to (M <= 4): for one token of
-    2-bit rows the one-token column-stationary kernel where it fits; for 2..4 tokens
-    of 2-bit rows of at most 8192 bytes (and at most 1024 rows per CTA) the
-    column-stationary multi-token kernel, else the lean 2-bit kernel for rows
-    of at most 8192 packed bytes; for one token of base 3,
-    the column-stationary kernel for rows of at most 768 segments and at most
-    1024 rows per CTA (148 CTAs); else the general one."""
-    if fmt == 2:  # 1-bit rows of at most 4096 bytes: the lean kernel's 1-bit form
-        return "gemv_i2_kernel" if all(((K + 7) // 8 + 15) // 16 * 16 <= 4096 for (_, K) in layers) else "gemv_kernel"
-    if fmt == 0:
-        rbs = [((K + 3) // 4 + 15) // 16 * 16 for (_, K) in layers]
-        # one bf16 token, K % 16 == 0, rows of at most 8192 bytes and the
-        # token, its codes and the row sums within 96 KB of shared memory
-        if M == 1 and all(K % 16 == 0 and rb <= 8192 and
-                          K * 2 + rb * 4 + 4 * -(-N // min(N, 148)) <= 96 * 1024
-                          for rb, (N, K) in zip(rbs, layers)):
-            return "gemv1_i2_kernel"
-        if 2 <= M <= 4 and all(rb <= 8192 and -(-N // min(N, 148)) <= 1024 for rb, (N, _) in zip(rbs, layers)):
-            return "gemv_i2_mt_kernel"
-        return "gemv_i2_kernel" if all(rb <= 8192 for rb in rbs) else "gemv_kernel"
-    t5 = M == 1 and all(((K + 4) // 5 + 15) // 16 <= 768 and -(-N // min(N, 148)) <= 1024 for (N, K) in layers)
-    return "gemv_t5_kernel" if t5 else "gemv_kernel"
+    """The decode kernel the forward dispatches to (M <= 4), '+'-joined when
+    the layers take different ones: for one token the column-stationary
+    one-token kernels where they fit (2-bit: gemv1_i2_kernel, base 3:
+    gemv1_t5_kernel); for 2..4 tokens of 2-bit rows of at most 8192 bytes
+    (and at most 1024 rows per CTA) the column-stationary multi-token kernel,
+    else the lean 2-bit kernel for rows of at most 8192 packed bytes; for one
+    token of base 3 that the one-token kernel does not take, the older
+    column-stationary kernel for rows of at most 768 segments and at most 1024
+    rows per CTA; else the general one."""
+    def one(N, K):
+        if fmt == 2:  # 1-bit rows of at most 4096 bytes: the lean kernel's 1-bit form
+            return "gemv_i2_kernel" if ((K + 7) // 8 + 15) // 16 * 16 <= 4096 else "gemv_kernel"
+        if fmt == 0:
+            rb = ((K + 3) // 4 + 15) // 16 * 16
+            if M == 1 and rb <= 8192 and gemv1_fits(N, K, rb):
+                return "gemv1_i2_kernel"
+            if 2 <= M <= 4 and rb <= 8192 and -(-N // min(N, 148)) <= 1024:
+                return "gemv_i2_mt_kernel"
+            return "gemv_i2_kernel" if rb <= 8192 else "gemv_kernel"
+        rb = ((K + 4) // 5 + 15) // 16 * 16
+        if M == 1 and gemv1_fits(N, K, rb, t5=True):
+            return "gemv1_t5_kernel"
+        if M == 1 and rb // 16 <= 768 and -(-N // min(N, 148)) <= 1024:
+            return "gemv_t5_kernel"
+        return "gemv_kernel"
+    names = []
+    for (N, K) in layers:
+        n = one(N, K)
+        if n not in names:
+            names.append(n)
+    return "+".join(names)
 
 
 def gemm_kernel_name(M):

@@ -19,7 +19,7 @@
 // in token order (the plain order of the sum), then gamma * T, rounded once
 // to fp32.
 // dx reads the packed 2-bit weights once per pass of up to two tokens in 2-D
-// tiles (512 columns x at least 64 rows: two or three CTAs per SM, partial sums
+// tiles (512 columns x at least 64 rows: about two CTAs per SM, partial sums
 // a few percent of the weight bytes); dW writes N K fp32 values (the
 // HBM-bound part for few tokens).
 #include "bl_common.cuh"
@@ -70,7 +70,7 @@ __device__ __forceinline__ double lds_f64(uint32_t addr) {
 // half of a double buffer.  The warps' sums meet in shared memory in a fixed
 // order and go to part[rb][m][k] (fp64).
 template <int DYT, int MT>
-__global__ void __launch_bounds__(kDxWarps * 32, MT == 1 ? 3 : 2)
+__global__ void __launch_bounds__(kDxWarps * 32, 2)
     backward_dx_tile_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, int64_t N, int64_t K,
                             const void* __restrict__ dy, int64_t m0, int64_t rows_per_block,
                             double* __restrict__ part) {
@@ -335,6 +335,55 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// dW for one token: dW[n, k] depends on row n only through dy[n] and on
+// column k only through the code x_q[k], so each row has at most 256
+// distinct outputs.  A CTA takes rows n = b, b + G, ...: per row its threads
+// first fill a 256-entry table of the outputs for every code (the same fp64
+// operations as backward_dw_kernel: T = 0.0 + (dy x_q) c, then gamma T to
+// fp32), then write the row by lookups (four codes per 32-bit load, one
+// 16-byte store).  Four copies of the table (lane mod 4 picks one) spread a
+// warp's lookups over the banks.
+constexpr int kDw1Copies = 4;
+
+template <int DYT>
+__global__ void __launch_bounds__(256)
+    backward_dw1_kernel(const void* __restrict__ dy, const int8_t* __restrict__ xq, const float* __restrict__ scale,
+                        const float* __restrict__ gamma, int64_t N, int64_t K, float* __restrict__ dw) {
+  pdl_enter(dy, xq, scale, gamma, dw);
+  __shared__ float tab[256][kDw1Copies];  // [code + 128][copy]
+  const double c = __ddiv_rn(static_cast<double>(__ldcg(scale)), 127.0);
+  const double g = static_cast<double>(__ldcg(gamma));
+  const int t = threadIdx.x;
+  const int copy = t & (kDw1Copies - 1);
+  const bool vec = (K % 4) == 0;
+  const uint32_t kq = static_cast<uint32_t>((K + 3) / 4);
+  const double q_t = i32_to_f64(t - 128);  // this thread's code
+  for (int64_t n = blockIdx.x; n < N; n += gridDim.x) {
+    const double a = load_grad<DYT>(dy, n);
+    const float o = __double2float_rn(__dmul_rn(g, __dadd_rn(0.0, __dmul_rn(__dmul_rn(a, q_t), c))));
+    __syncthreads();  // the previous row's lookups are done
+#pragma unroll
+    for (int j = 0; j < kDw1Copies; ++j) tab[t][j] = o;
+    __syncthreads();
+    float* row = dw + n * K;
+    for (uint32_t qd = t; qd < kq; qd += blockDim.x) {
+      const int64_t k0 = 4 * static_cast<int64_t>(qd);
+      if (vec) {
+        const uint32_t w = __ldcg(reinterpret_cast<const uint32_t*>(xq + k0));
+        float4 v;
+        v.x = tab[(w & 0xffu) ^ 0x80u][copy];
+        v.y = tab[((w >> 8) & 0xffu) ^ 0x80u][copy];
+        v.z = tab[((w >> 16) & 0xffu) ^ 0x80u][copy];
+        v.w = tab[(w >> 24) ^ 0x80u][copy];
+        *reinterpret_cast<float4*>(row + k0) = v;
+      } else {
+        for (int i = 0; i < 4 && k0 + i < K; ++i)
+          row[k0 + i] = tab[(static_cast<uint32_t>(static_cast<uint8_t>(xq[k0 + i]))) ^ 0x80u][copy];
+      }
+    }
+  }
+}
+
 // ---- host side --------------------------------------------------------------------
 int64_t backward_dx_chunks(int64_t N) { return (N + kDxMinRows - 1) / kDxMinRows; }
 int backward_dx_tokens_per_pass() { return kDxTokens; }
@@ -363,12 +412,12 @@ static cudaError_t launch_dx_tile(dim3 grid, const uint8_t* packed, int64_t rowb
 cudaError_t launch_backward_dx(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
                                const void* dy, int dydt, int64_t M, float* dx, double* part, cudaStream_t st) {
   // tiles: 512-column blocks x row blocks of at least kDxMinRows rows, about
-  // as many CTAs as fit on the SMs at once (the row blocks never outnumber
-  // backward_dx_chunks(N), which the workspace holds)
+  // two CTAs per SM (more and smaller row blocks measured slower: each
+  // builds its own tables and writes its own partial sums; the row blocks
+  // never outnumber backward_dx_chunks(N), which the workspace holds)
   const int64_t words = (K + 15) / 16;
   const int64_t cbs = (words + 31) / 32;
-  const int per_sm = M == 1 ? 3 : 2;  // the one-token tile kernel fits three CTAs per SM
-  int64_t rbs = (per_sm * static_cast<int64_t>(device_sms()) + cbs - 1) / cbs;
+  int64_t rbs = (2 * static_cast<int64_t>(device_sms()) + cbs - 1) / cbs;
   int64_t rows = (N + rbs - 1) / rbs;
   rows = rows < kDxMinRows ? kDxMinRows : (rows + 7) / 8 * 8;
   rbs = (N + rows - 1) / rows;
@@ -393,6 +442,15 @@ cudaError_t launch_backward_dx(const uint8_t* packed, int64_t rowbytes, const fl
 
 cudaError_t launch_backward_dw(const void* dy, int dydt, const int8_t* xq, const float* scale, const float* gamma,
                                int64_t M, int64_t N, int64_t K, float* dw, cudaStream_t st) {
+  if (M == 1) {  // one token: a 256-entry table of outputs per row
+    const int64_t cap = static_cast<int64_t>(device_sms()) * 8;
+    const unsigned g1 = static_cast<unsigned>(N < cap ? N : cap);
+    const cudaError_t e = dydt == BL_F32
+                              ? launch_pdl(backward_dw1_kernel<BL_F32>, g1, 256, 0, st, dy, xq, scale, gamma, N, K, dw)
+                              : launch_pdl(backward_dw1_kernel<BL_BF16>, g1, 256, 0, st, dy, xq, scale, gamma, N, K, dw);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   const unsigned g = grid_of(N * ((K + 3) / 4), 8);
   cudaError_t e = dydt == BL_F32
                       ? launch_pdl(backward_dw_kernel<BL_F32>, g, 256, 0, st, dy, xq, scale, gamma, M, N, K, dw)

@@ -108,7 +108,7 @@ __device__ __forceinline__ int dot_seg_i2(const uint4 wv, const uint4 (&X)[4], i
 
 // The INT8 codes of 16 activations e[0..15] against scale s (c127 =
 // fl(127 / s)), returned as the 16-byte slot of their packed word (byte
-// 4j + b = code of element 4b + j).  Each code is rint(fl(fl(e / s) 127)),
+// 4j + b = code of element 4b + j), or with SLOT false in element order.  Each code is rint(fl(fl(e / s) 127)),
 // taken division-free as in quant_act_fast: t_a = fl(e c127) is within 2^-14
 // of t, so rint(t_a) = rint(t) unless t_a lies within 2^-14 of a
 // half-integer.  rint(t_a) comes from the adder (t_a + 1.5 * 2^23 rounds to
@@ -116,6 +116,7 @@ __device__ __forceinline__ int dot_seg_i2(const uint4 wv, const uint4 (&X)[4], i
 // complement, |code| <= 127), the margin is checked once per eight elements
 // on the largest |t_a - rint(t_a)| (an exact difference), and only a group
 // with an element that close to a tie takes the exact quotient.
+template <bool SLOT = true>
 __device__ __forceinline__ uint4 g1_codes16(const float (&e)[16], float s, float c127) {
   // element pairs through the paired fp32 unit (each lane rounds to nearest
   // as the scalar operation does); ta - rint(ta) = fma(rint(ta), -1, ta) is
@@ -146,8 +147,13 @@ __device__ __forceinline__ uint4 g1_codes16(const float (&e)[16], float s, float
   }
   uint32_t w[4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
-    w[j] = __byte_perm(__byte_perm(r[j], r[4 + j], 0x0040), __byte_perm(r[8 + j], r[12 + j], 0x0040), 0x5410);
+  for (int j = 0; j < 4; ++j) {
+    if (SLOT)  // byte 4j + b = code of element 4b + j
+      w[j] = __byte_perm(__byte_perm(r[j], r[4 + j], 0x0040), __byte_perm(r[8 + j], r[12 + j], 0x0040), 0x5410);
+    else  // linear: byte 4j + b = code of element 4j + b
+      w[j] = __byte_perm(__byte_perm(r[4 * j], r[4 * j + 1], 0x0040), __byte_perm(r[4 * j + 2], r[4 * j + 3], 0x0040),
+                         0x5410);
+  }
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
@@ -415,6 +421,318 @@ __global__ void __launch_bounds__(kG1MaxThreads, 1024 / kG1MaxThreads)
   if (XDT != BL_I8 && write_scale && b == 0 && tid == 0) scale[0] = s;
 }
 
+// ---------------------------------------------------------------------------
+// One token on base-3 rows (5 weights per byte: digit j of byte b is
+// floor(b / 3^j) mod 3, the stored digit q + 1), in the layout of
+// gemv1_i2_kernel: a 16-byte segment holds 80 weights, thread t keeps the 80
+// activation codes of its column c in registers (xlo[p]: the codes of digits
+// 0..3 of byte p; xhi[j] byte i: the code of digit 4 of byte 4j + i) and
+// reads segment t + i R segs of its CTA's range at step i, so the rows of a
+// step are one contiguous block and the lanes of a row are used as densely
+// as in the 2-bit kernel.  A byte is decoded by one 4-byte shared lookup in
+// the lane's own copy of a 256-entry table (copy L in bank L: a warp's
+// lookups never conflict): byte j of the entry is digit j (j < 4) and bits
+// 2..3 of byte 0 hold digit 4.  Per packed word: four lookups, four dp4a on
+// the masked entries against xlo, and one dp4a on the gathered fifth digits
+// (4 d4 in each byte) against xhi, whose factor 4 comes off at the end.  The
+// table depends on nothing the previous kernel writes, so it is filled before
+// the dependency wait.  Bytes 243..255 are not produced by the packer; they
+// decode as five zero weights.  The token's codes are written in element
+// order over the raw token (80 per segment, 0 past K).
+// ---------------------------------------------------------------------------
+constexpr int kT1LutBytes = 256 * 32 * 4;
+
+__host__ __device__ inline int64_t g1t5_xregion(int64_t K, int xwords, int64_t rowbytes) {
+  const int64_t raw = K * xwords;     // the raw token: xwords 16-byte words per 16 elements
+  const int64_t codes = rowbytes * 5;  // 80 codes per 16-byte segment
+  return ((raw > codes ? raw : codes) + 15) / 16 * 16;
+}
+
+// a0 + sum over the 80 weights of a base-3 segment of d x (d the stored digit)
+__device__ __forceinline__ int dot_seg_t5(const uint4 wv, const uint32_t (&xlo)[16], const uint32_t (&xhi)[4],
+                                          uint32_t lut_l, int a0) {
+  const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+  int v = a0, vh = 0;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    uint32_t L[4];
+#pragma unroll
+    for (int bb = 0; bb < 4; ++bb) {
+      const uint32_t a = lut_l + (__byte_perm(wd[w], 0, 0x4440 + bb) << 7);  // entry e of copy L: 128 e + 4 L
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(L[bb]) : "r"(a) : "memory");
+    }
+#pragma unroll
+    for (int bb = 0; bb < 4; ++bb) v = dp4a_us(L[bb] & 0x03030303u, xlo[4 * w + bb], v);
+    const uint32_t H =
+        __byte_perm(__byte_perm(L[0], L[1], 0x0040), __byte_perm(L[2], L[3], 0x0040), 0x5410) & 0x0c0c0c0cu;
+    vh = dp4a_us(H, xhi[w], vh);
+  }
+  return v + (vh >> 2);
+}
+
+template <int XDT, int XC, int S, bool ALIGNED>
+__global__ void __launch_bounds__(kG1MaxThreads, 1024 / kG1MaxThreads)
+    gemv1_t5_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
+                    int64_t N, int64_t K, const void* __restrict__ x, float* __restrict__ scale,
+                    void* __restrict__ y, int ydt, int write_scale, const RowGroups rg, int R, int lpr, void* ws) {
+  constexpr int kXW = g1_xwords<XDT>();
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ uint32_t red[kG1MaxThreads / 32];
+  __shared__ float sh_gam[kMaxRowGroups];
+  __shared__ int64_t sh_end[kMaxRowGroups];
+  __shared__ float sh_s;
+  __shared__ __align__(8) uint64_t xbar;  // completion of the token's bulk copy
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int T = blockDim.x;
+  const int segs = static_cast<int>(rowbytes >> 4);
+  const int64_t G = gridDim.x, b = blockIdx.x;
+  const int64_t per = N / G, extra = N % G;
+  const int64_t row0 = b * per + (b < extra ? b : extra);
+  const int nrows = static_cast<int>(per + (b < extra ? 1 : 0));
+  const int r0_raw = tid / lpr, c_raw = tid - r0_raw * lpr;
+  const bool row_ok = r0_raw < R;
+  const bool col_ok = row_ok && c_raw < segs;
+  const int r0 = row_ok ? r0_raw : 0;
+  const int c = col_ok ? c_raw : 0;
+  const int nr = (row_ok && r0 < nrows) ? (nrows - r0 + R - 1) / R : 0;
+  const uint32_t step = static_cast<uint32_t>(R * rowbytes);
+  const int kch = static_cast<int>(K >> 4);  // 16-element chunks of the token (K % 16 == 0)
+  const int nch = 5 * segs;                  // 16-code chunks of the codes region (0 past K)
+  const uint32_t xbytes = static_cast<uint32_t>(K * kXW);
+  // shared memory: the table [256][32] x 4 bytes, the token region (the raw
+  // token, then its codes), the row ring [S][T] x 16 bytes, the row sums
+  const int64_t xreg = g1t5_xregion(K, kXW, rowbytes);
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
+  uint8_t* xbuf = smem + kT1LutBytes;
+  const uint32_t ring_s = smem_u32(xbuf + xreg) + 16u * tid;
+  const uint32_t tstride = 16u * T;
+  int* rsum = reinterpret_cast<int*>(xbuf + xreg + static_cast<int64_t>(S) * T * 16);
+
+  // 0. before the wait: the first bytes of the CTA's rows into L2, the
+  //    table, the row sums zeroed, the token barrier set up
+  {
+    const int64_t bytes = static_cast<int64_t>(nrows) * rowbytes;
+    l2_prefetch_bulk(packed + row0 * rowbytes, bytes < BL_G1_PREFETCH ? bytes : BL_G1_PREFETCH);
+  }
+  for (int i = tid; i < 256 * 32; i += T) {
+    const int e = i >> 5;
+    uint32_t d[5] = {1, 1, 1, 1, 1};  // bytes past 242: five zero weights
+    if (e < 243) {
+      int v = e;
+#pragma unroll
+      for (int j = 0; j < 5; ++j) {
+        d[j] = static_cast<uint32_t>(v % 3);
+        v /= 3;
+      }
+    }
+    lut[i] = (d[0] | (d[4] << 2)) | (d[1] << 8) | (d[2] << 16) | (d[3] << 24);
+  }
+  for (int i = tid; i < nrows; i += T) rsum[i] = 0;
+#pragma unroll
+  for (int i = 0; i < kMaxRowGroups; ++i)
+    if (tid == i) sh_end[i] = rg.end[i];
+  if (tid == 0) {
+    mbar_init(&xbar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  pdl_wait(packed, gamma, x, scale, y);
+  pdl_launch_dependents();
+
+  // 1. the token by one bulk copy (bounded wait: on expiry the CTA records the
+  //    timeout, lets the copy land and leaves)
+  if (tid == 0) {
+    mbar_expect_tx(&xbar, xbytes);
+    bulk_load(xbuf, x, xbytes, &xbar);
+  }
+  if (tid < rg.n) sh_gam[tid] = __ldcg(gamma + tid);
+  if (XDT == BL_I8 && tid == 0) sh_s = __ldcg(scale);
+  const bool got = wait_drain(&xbar, 0, kG1WaitCycles);
+  if (__syncthreads_or(!got)) {
+    if (tid == 0) {
+      set_flag(ws, kFlagTimeout, 0x602);
+      wait_drain(&xbar, 0, kG1WaitCycles);
+    }
+    return;
+  }
+  const uint8_t* gp = packed + (row0 + r0) * rowbytes + static_cast<int64_t>(c) * 16;
+#pragma unroll
+  for (int j = 0; j < S - 1; ++j) {
+    if (col_ok && j < nr) cp_async16_s(ring_s + j * tstride, gp);
+    cp_async_commit();
+    gp += step;
+  }
+
+  // 2. per-token absmax on the magnitude bits (finite inputs)
+  float s;
+  if constexpr (XDT != BL_I8) {
+    uint32_t mx = 0;
+#pragma unroll
+    for (int u = 0; u < XC; ++u) {
+      const int g = tid + T * u;
+      if (g < kch)
+#pragma unroll
+        for (int i = 0; i < kXW; ++i) {
+          const uint4 v = *reinterpret_cast<const uint4*>(xbuf + (static_cast<int64_t>(g) * kXW + i) * 16);
+          if constexpr (XDT == BL_F32) {
+            const uint32_t a = max(v.x & 0x7fffffffu, v.y & 0x7fffffffu);
+            const uint32_t b2 = max(v.z & 0x7fffffffu, v.w & 0x7fffffffu);
+            mx = max(mx, max(a, b2));
+          } else {
+            const uint32_t a = __vmaxu2(v.x & 0x7fff7fffu, v.y & 0x7fff7fffu);
+            const uint32_t b2 = __vmaxu2(v.z & 0x7fff7fffu, v.w & 0x7fff7fffu);
+            mx = __vmaxu2(mx, __vmaxu2(a, b2));
+          }
+        }
+    }
+    if constexpr (XDT == BL_BF16) mx = max(mx & 0xffffu, mx >> 16) << 16;
+    const uint32_t m = __reduce_max_sync(0xffffffffu, mx);
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    uint32_t mm = 0;
+    for (int w = 0; w < (T >> 5); ++w) mm = max(mm, red[w]);
+    s = fmaxf(__uint_as_float(mm), 1e-6f);
+  } else {
+    s = sh_s;
+  }
+
+  // 3. the codes of the thread's chunks in element order, written over the
+  //    raw token once every thread has read its raw chunks
+  {
+    const float c127 = (XDT == BL_I8) ? 0.0f : __fdiv_rn(127.0f, s);
+    uint4 cw[XC];
+#pragma unroll
+    for (int u = 0; u < XC; ++u) {
+      const int g = tid + T * u;
+      cw[u] = make_uint4(0u, 0u, 0u, 0u);  // padding chunks (past K): code 0
+      if (g < kch) {
+        const uint8_t* src = xbuf + static_cast<int64_t>(g) * kXW * 16;
+        if constexpr (XDT == BL_I8) {
+          cw[u] = *reinterpret_cast<const uint4*>(src);
+        } else {
+          float e[16];
+          if constexpr (XDT == BL_F32) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * i);
+              e[4 * i] = __uint_as_float(v.x); e[4 * i + 1] = __uint_as_float(v.y);
+              e[4 * i + 2] = __uint_as_float(v.z); e[4 * i + 3] = __uint_as_float(v.w);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * i);
+              const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                e[8 * i + 2 * k] = __uint_as_float(wv[k] << 16);
+                e[8 * i + 2 * k + 1] = __uint_as_float(wv[k] & 0xffff0000u);
+              }
+            }
+          }
+          cw[u] = g1_codes16<false>(e, s, c127);
+        }
+      }
+    }
+    __syncthreads();  // every raw chunk has been read
+#pragma unroll
+    for (int u = 0; u < XC; ++u) {
+      const int g = tid + T * u;
+      if (g < nch) *reinterpret_cast<uint4*>(xbuf + static_cast<int64_t>(g) * 16) = cw[u];
+    }
+  }
+  __syncthreads();
+
+  // 4. this thread's 80 codes (xlo / xhi) and their sum (digits are q + 1:
+  //    the sum is taken off once per row, as the row sum's starting value)
+  uint32_t xlo[16], xhi[4];
+  int csum = 0;
+  {
+    uint32_t w[20];
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+      const uint4 t = col_ok ? *reinterpret_cast<const uint4*>(xbuf + (static_cast<int64_t>(c) * 5 + i) * 16)
+                             : make_uint4(0u, 0u, 0u, 0u);
+      w[4 * i] = t.x;
+      w[4 * i + 1] = t.y;
+      w[4 * i + 2] = t.z;
+      w[4 * i + 3] = t.w;
+    }
+#pragma unroll
+    for (int i = 0; i < 20; ++i) csum = __dp4a(static_cast<int>(w[i]), 0x01010101, csum);
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {  // codes 5p .. 5p + 3 of the segment
+      const int o = 5 * p;
+      xlo[p] = __byte_perm(w[o >> 2], w[(o >> 2) + 1], 0x3210 + 0x1111 * (o & 3));
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {  // code 5p + 4 of bytes p = 4j .. 4j + 3
+      uint32_t h = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = 20 * j + 5 * i + 4;
+        h |= ((w[t >> 2] >> (8 * (t & 3))) & 0xffu) << (8 * i);
+      }
+      xhi[j] = h;
+    }
+  }
+  const int init = -csum;
+  const uint32_t gmask = ALIGNED ? 0xffffffffu : __match_any_sync(0xffffffffu, row_ok ? r0_raw : -1 - lane);
+  const bool leader = ALIGNED ? lane == 0 : (__ffs(gmask) - 1) == lane;
+  uint32_t rs = smem_u32(rsum + r0);
+  const uint32_t rstep = 4u * R;
+  const uint32_t lut_l = smem_u32(lut) + 4u * lane;  // this lane's table copy
+
+  // 5. the stream, as in gemv1_i2_kernel
+  auto consume = [&](const uint4 wv) {
+    int v = dot_seg_t5(wv, xlo, xhi, lut_l, init);
+    v = __reduce_add_sync(gmask, v);
+    if (leader) red_add_s(rs, v);
+    rs += rstep;
+  };
+  int k = 0;
+  for (; k < nr - 2 * S + 2; k += S) {
+#pragma unroll
+    for (int j = 0; j < S; ++j) {
+      if (col_ok) cp_async16_s(ring_s + ((j + S - 1) % S) * tstride, gp);
+      cp_async_commit();
+      gp += step;
+      cp_async_wait<S - 1>();
+      consume(lds128(ring_s + j * tstride));
+    }
+  }
+  for (; k < nr; ++k) {
+    if (col_ok && k + S - 1 < nr) cp_async16_s(ring_s + ((k + S - 1) % S) * tstride, gp);
+    cp_async_commit();
+    gp += step;
+    cp_async_wait<S - 1>();
+    consume(lds128(ring_s + (k % S) * tstride));
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // 6. dequantize and store the CTA's outputs (coalesced)
+  const float cf1 = dequant_factor(sh_gam[0], s);
+  for (int r = tid; r < nrows; r += T) {
+    const int a = rsum[r];
+    const int64_t n = row0 + r;
+    float cf = cf1;
+    if (rg.n > 1) {
+      int gi = 0;
+      while (gi + 1 < rg.n && n >= sh_end[gi]) ++gi;
+      cf = dequant_factor(sh_gam[gi], s);
+    }
+    if (ydt == BL_I32)
+      static_cast<int32_t*>(y)[n] = a;
+    else if (ydt == BL_F32)
+      static_cast<float*>(y)[n] = __fmul_rn(__int2float_rn(a), cf);
+    else
+      static_cast<__nv_bfloat16*>(y)[n] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(a), cf));
+  }
+  if (XDT != BL_I8 && write_scale && b == 0 && tid == 0) scale[0] = s;
+}
+
 // Launch geometry: R rows per step, threads rounded up to whole warps, and
 // the token chunks per thread (1, 2 or 4).
 struct Gemv1Geom {
@@ -422,7 +740,7 @@ struct Gemv1Geom {
   int64_t grid, rows_per_cta, smem;
 };
 
-static bool gemv1_geom(int64_t N, int64_t K, int64_t rowbytes, int xdt, Gemv1Geom* g) {
+static bool gemv1_geom(int64_t N, int64_t K, int64_t rowbytes, int xdt, Gemv1Geom* g, bool t5 = false) {
   const int64_t segs = rowbytes / 16;
   if (K % 16 != 0 || segs < 1 || segs > kG1MaxThreads) return false;
   const int64_t sms = device_sms();
@@ -437,10 +755,14 @@ static bool gemv1_geom(int64_t N, int64_t K, int64_t rowbytes, int xdt, Gemv1Geo
   g->R = static_cast<int>(R);
   g->lpr = static_cast<int>(lpr);
   g->threads = static_cast<int>((R * lpr + 31) / 32 * 32);
-  const int64_t per = (4 * segs + g->threads - 1) / g->threads;
+  // 16-byte chunks of the codes: 4 per 2-bit segment (64 codes), 5 per base-3
+  // segment (80 codes)
+  const int64_t per = ((t5 ? 5 : 4) * segs + g->threads - 1) / g->threads;
+  if (per > 4) return false;
   g->xc = per <= 1 ? 1 : (per <= 2 ? 2 : 4);
   const int xwords = xdt == BL_F32 ? 4 : (xdt == BL_BF16 ? 2 : 1);
-  const int64_t fixed = g1_xregion(K, xwords, rowbytes) + 4 * g->rows_per_cta;
+  const int64_t fixed = (t5 ? kT1LutBytes + g1t5_xregion(K, xwords, rowbytes) : g1_xregion(K, xwords, rowbytes)) +
+                        4 * g->rows_per_cta;
   for (int st : {kG1StagesMax, 6}) {  // the deepest ring that keeps two CTAs per SM
     g->stages = st;
     g->smem = fixed + int64_t{16} * st * g->threads;
@@ -454,11 +776,17 @@ bool gemv1_fits(int64_t N, int64_t K, int64_t rowbytes, int xdt) {
   return gemv1_geom(N, K, rowbytes, xdt, &g);
 }
 
-template <int XDT, int XC, int S>
+bool gemv1_t5_fits(int64_t N, int64_t K, int64_t rowbytes, int xdt) {
+  Gemv1Geom g;
+  return gemv1_geom(N, K, rowbytes, xdt, &g, true);
+}
+
+template <bool T5, int XDT, int XC, int S>
 static cudaError_t launch_gemv1_t(const Gemv1Geom& g, const uint8_t* packed, int64_t rowbytes, const float* gamma,
                                   int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
                                   int write_scale, const RowGroups& rg, void* ws, cudaStream_t st) {
-  auto kern = g.lpr % 32 == 0 ? gemv1_i2_kernel<XDT, XC, S, true> : gemv1_i2_kernel<XDT, XC, S, false>;
+  auto kern = T5 ? (g.lpr % 32 == 0 ? gemv1_t5_kernel<XDT, XC, S, true> : gemv1_t5_kernel<XDT, XC, S, false>)
+                 : (g.lpr % 32 == 0 ? gemv1_i2_kernel<XDT, XC, S, true> : gemv1_i2_kernel<XDT, XC, S, false>);
   const size_t smem = static_cast<size_t>(g.smem);
   if (smem > 48 * 1024) {
     const cudaError_t e =
@@ -471,33 +799,50 @@ static cudaError_t launch_gemv1_t(const Gemv1Geom& g, const uint8_t* packed, int
   return cudaGetLastError();
 }
 
-template <int XDT, int XC>
+template <bool T5, int XDT, int XC>
 static cudaError_t launch_gemv1_s(const Gemv1Geom& g, const uint8_t* packed, int64_t rowbytes, const float* gamma,
                                   int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
                                   int write_scale, const RowGroups& rg, void* ws, cudaStream_t st) {
   if (g.stages == kG1StagesMax)
-    return launch_gemv1_t<XDT, XC, kG1StagesMax>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg,
-                                                 ws, st);
-  return launch_gemv1_t<XDT, XC, 6>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
+    return launch_gemv1_t<T5, XDT, XC, kG1StagesMax>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale,
+                                                     rg, ws, st);
+  return launch_gemv1_t<T5, XDT, XC, 6>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
 }
 
-template <int XDT>
+template <bool T5, int XDT>
 static cudaError_t launch_gemv1_x(const Gemv1Geom& g, const uint8_t* packed, int64_t rowbytes, const float* gamma,
                                   int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
                                   int write_scale, const RowGroups& rg, void* ws, cudaStream_t st) {
-  if (g.xc == 1) return launch_gemv1_s<XDT, 1>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
-  if (g.xc == 2) return launch_gemv1_s<XDT, 2>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
-  return launch_gemv1_s<XDT, 4>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
+  if (g.xc == 1)
+    return launch_gemv1_s<T5, XDT, 1>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
+  if (g.xc == 2)
+    return launch_gemv1_s<T5, XDT, 2>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
+  return launch_gemv1_s<T5, XDT, 4>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
+}
+
+template <bool T5>
+static cudaError_t launch_gemv1_f(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
+                                  const void* x, int xdt, float* scale, void* y, int ydt, const RowGroups& rg,
+                                  void* ws, cudaStream_t st) {
+  Gemv1Geom g;
+  if (!gemv1_geom(N, K, rowbytes, xdt, &g, T5)) return cudaErrorInvalidValue;
+  if (xdt == BL_F32)
+    return launch_gemv1_x<T5, BL_F32>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 1, rg, ws, st);
+  if (xdt == BL_BF16)
+    return launch_gemv1_x<T5, BL_BF16>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 1, rg, ws, st);
+  return launch_gemv1_x<T5, BL_I8>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 0, rg, ws, st);
 }
 
 cudaError_t launch_gemv1(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
                          const void* x, int xdt, float* scale, void* y, int ydt, const RowGroups& rg, void* ws,
                          cudaStream_t st) {
-  Gemv1Geom g;
-  if (!gemv1_geom(N, K, rowbytes, xdt, &g)) return cudaErrorInvalidValue;
-  if (xdt == BL_F32) return launch_gemv1_x<BL_F32>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 1, rg, ws, st);
-  if (xdt == BL_BF16) return launch_gemv1_x<BL_BF16>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 1, rg, ws, st);
-  return launch_gemv1_x<BL_I8>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 0, rg, ws, st);
+  return launch_gemv1_f<false>(packed, rowbytes, gamma, N, K, x, xdt, scale, y, ydt, rg, ws, st);
+}
+
+cudaError_t launch_gemv1_t5(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
+                            const void* x, int xdt, float* scale, void* y, int ydt, const RowGroups& rg, void* ws,
+                            cudaStream_t st) {
+  return launch_gemv1_f<true>(packed, rowbytes, gamma, N, K, x, xdt, scale, y, ydt, rg, ws, st);
 }
 
 }  // namespace bl

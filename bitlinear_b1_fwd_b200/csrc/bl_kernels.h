@@ -104,6 +104,13 @@ bool gemv1_fits(int64_t N, int64_t K, int64_t rowbytes, int xdt);
 cudaError_t launch_gemv1(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
                          const void* x, int xdt, float* scale, void* y, int ydt, const RowGroups& rg, void* ws,
                          cudaStream_t st);
+// The same for one token on base-3 rows (80 weights per 16-byte segment,
+// digits decoded by a per-lane shared table): K % 16 == 0 and the table,
+// token, ring and row sums within the two-CTAs-per-SM budget.
+bool gemv1_t5_fits(int64_t N, int64_t K, int64_t rowbytes, int xdt);
+cudaError_t launch_gemv1_t5(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
+                            const void* x, int xdt, float* scale, void* y, int ydt, const RowGroups& rg, void* ws,
+                            cudaStream_t st);
 
 cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int64_t N, int64_t K,
                         const void* x, int xdt, float* scale, int64_t M, void* y, int ydt,

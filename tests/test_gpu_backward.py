@@ -106,6 +106,8 @@ def run_dw(dy, xq, s, g, N, K):
     (3, 777, 1001, "bf16"),   # K % 4 != 0: scalar loads and stores
     (300, 64, 128, "f32"),    # two blocks of token factors
     (1, 3200, 3200, "bf16"),  # 3B attention shape, one token
+    (1, 777, 1001, "f32"),    # one token (the per-row table kernel), K % 4 != 0
+    (1, 5000, 64, "bf16"),    # one token, more rows than CTAs: each CTA refills its table per row
 ])
 def test_backward_dw(orc, M, N, K, dydt):
     x = synth.entry_outliers(synth.normal_f32(730 + M, (M, K)), 731, 0.01, 20.0)
@@ -114,6 +116,22 @@ def test_backward_dw(orc, M, N, K, dydt):
     if dydt == "bf16":
         dy = synth.to_bf16_bits(dy)
     g = np.float32(0.0173)
+    dw = run_dw(dy, xq, s, g, N, K)
+    ref = orc.backward_dw(dy, xq, s, g)
+    assert np.array_equal(dw.view(np.uint32), ref.view(np.uint32))
+
+
+def test_backward_dw_one_token_every_code():
+    """One token whose codes take all 256 int8 values (including -128, which
+    the API accepts though the quantizer never writes it), zero and negative
+    gradients: every entry of the per-row table is used."""
+    N, K = 300, 512
+    xq = (np.arange(K) % 256 - 128).astype(np.int8).reshape(1, K)
+    s = np.array([0.731], dtype=np.float32)
+    dy = synth.normal_f32(740, (1, N), 1e-2)
+    dy[0, ::7] = 0.0
+    dy[0, 3] = -0.0
+    g = np.float32(0.0419)
     dw = run_dw(dy, xq, s, g, N, K)
     ref = orc.backward_dw(dy, xq, s, g)
     assert np.array_equal(dw.view(np.uint32), ref.view(np.uint32))

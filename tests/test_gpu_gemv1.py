@@ -1,5 +1,6 @@
-"""GPU parity of the one-token 2-bit decode GEMV (the column-stationary
-kernel with K % 16 == 0 and rows of up to 8 KB) against the oracle.
+"""GPU parity of the one-token decode GEMVs (the column-stationary kernels
+with K % 16 == 0: 2-bit rows of up to 8 KB, and base-3 rows where the
+table, token and ring fit) against the oracle.
 
 The cases walk its geometry: segments per row from 1 to 512 (several rows per
 warp, warps that span two rows, one row per warp), one to about a thousand
@@ -18,6 +19,7 @@ from gpu_helpers import assert_bf16_ulp, assert_f32_rel, dev, forward, host, qua
 pytestmark = pytest.mark.gpu
 
 I2 = B.BL_PACK_I2
+T5 = B.BL_PACK_T5
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -28,20 +30,20 @@ def _lib():
     torch.cuda.init()
 
 
-def _check(orc, N, K, xkind, seed, zero_token=False, ydts=(B.BL_I32, B.BL_F32, B.BL_BF16)):
+def _check(orc, N, K, xkind, seed, zero_token=False, ydts=(B.BL_I32, B.BL_F32, B.BL_BF16), fmt=I2):
     W = synth.normal_f32(seed, (N, K), 0.02)
     x = synth.entry_outliers(synth.normal_f32(seed + 1, (1, K)), seed + 2, 0.01, 20.0)
     if zero_token:
         x[:] = 0.0
-    g, _, packed = quantize_weights(W, I2, codes=False)
+    g, _, packed = quantize_weights(W, fmt, codes=False)
     scale = None
     if xkind == "int8":
         x, scale = orc.act_quant(x)
     elif xkind == "bf16":
         x = synth.to_bf16_bits(x)
     for ydt in ydts:
-        y, s = forward(packed, I2, g, N, K, x, ydt, scale)
-        y_ref, s_ref = orc.forward(packed, I2, g, N, K, x, ydt=ydt, scale=scale)
+        y, s = forward(packed, fmt, g, N, K, x, ydt, scale)
+        y_ref, s_ref = orc.forward(packed, fmt, g, N, K, x, ydt=ydt, scale=scale)
         assert np.array_equal(s, s_ref)
         if ydt == B.BL_I32:
             assert np.array_equal(y, y_ref), np.argwhere(y != y_ref)[:5].tolist()
@@ -110,3 +112,26 @@ def test_gemv1_3b_layers_back_to_back(orc):
     # move a code, so the reference takes the same bf16 input)
     out_ref, _ = orc.forward(pd, I2, gd, Nd, Kd, host(h), ydt=B.BL_BF16)
     assert_bf16_ulp(host(out), out_ref)
+
+
+@pytest.mark.parametrize("N,K", [
+    (300, 64),      # one base-3 segment per row (80 weights, 16 of them padding)
+    (1000, 400),    # 5 segments: a warp spans several rows
+    (777, 1600),    # 20 segments
+    (8640, 3200),   # 3B up: 40 segments, 8 rows per step
+    (3200, 8640),   # 3B down: 108 segments, two chunks per thread
+    (900, 8192),    # 70B up rows: 103 segments, four rows per step, 6 ring stages
+    (500, 12800),   # 160 segments: three rows of 160 lanes per step
+    (149, 20480),   # 256 segments (int8 tokens only: bf16 and fp32 ones take the other kernel)
+])
+@pytest.mark.parametrize("xkind", ["bf16", "f32", "int8"])
+def test_gemv1_t5_geometry(orc, N, K, xkind):
+    """Base-3 rows in the column-stationary layout (and, where the token does
+    not fit beside the table, the fallback kernel)."""
+    _check(orc, N, K, xkind, seed=N * 17 + K, fmt=T5)
+
+
+def test_gemv1_t5_zero_token_and_rows_per_cta(orc):
+    _check(orc, 640, 3200, "bf16", seed=7, zero_token=True, fmt=T5)
+    for N in (1, 149, 30_000):
+        _check(orc, N, 400, "bf16", seed=N, fmt=T5, ydts=(B.BL_I32, B.BL_BF16))
