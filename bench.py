@@ -66,7 +66,7 @@ KERNEL_SOURCE = {"absmean_kernel": "bl_weights.cu", "ternarize_flat_kernel": "bl
                  "t5_to_i2_kernel": "bl_gemm_sm100.cu", "splitk_reduce_kernel": "bl_gemm_sm100.cu",
                  "pack_kernel": "bl_weights.cu",
                  "backward_dx_tile_kernel": "bl_backward.cu", "backward_dx_reduce_kernel": "bl_backward.cu",
-                 "backward_dw_kernel": "bl_backward.cu"}
+                 "backward_dw_kernel": "bl_backward.cu", "backward_dw1_kernel": "bl_backward.cu"}
 
 
 def csrc_digest(kernel: str | None = None) -> str:

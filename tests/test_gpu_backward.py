@@ -121,7 +121,7 @@ def test_backward_dw(orc, M, N, K, dydt):
     assert np.array_equal(dw.view(np.uint32), ref.view(np.uint32))
 
 
-def test_backward_dw_one_token_every_code():
+def test_backward_dw_one_token_every_code(orc):
     """One token whose codes take all 256 int8 values (including -128, which
     the API accepts though the quantizer never writes it), zero and negative
     gradients: every entry of the per-row table is used."""
