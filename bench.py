@@ -902,6 +902,10 @@ PROFILE_CASES = {
     "batch16_70b_up_t5": dict(N=28672, K=8192, fmt=1, M=16, sigma=0.01, op="forward"),
     "batch16_70b_up_1bit": dict(N=28672, K=8192, fmt=2, M=16, sigma=0.01, op="forward"),
     "backward_3b_down": dict(N=3200, K=8640, fmt=0, M=1, sigma=0.02, op="backward"),
+    "backward_3b_up_m8": dict(N=8640, K=3200, fmt=0, M=8, sigma=0.02, op="backward"),
+    "decode_70b_down_t5": dict(N=8192, K=28672, fmt=1, M=1, sigma=0.01, op="forward"),
+    "lnquant_70b_down": dict(N=8192, K=28672, fmt=0, M=256, sigma=0.01, op="lnquant"),
+    "pack_3b_up": dict(N=8640, K=3200, fmt=0, M=1, sigma=0.02, op="pack"),
 }
 
 
@@ -931,6 +935,12 @@ def run_profile_case(name):
         for _ in range(3 if c["op"] == "quantize" else 1):
             B.bitlinear_quantize_weights(W, 1e-5, fmt, packed, None, gamma, ws)
     status = [B.bitlinear_device_status(ws)]
+    if c["op"] == "pack":  # A3 alone: int8 codes -> packed rows
+        codes = torch.empty((N, K), dtype=torch.int8, device=dev)
+        B.bitlinear_quantize_weights(W, 1e-5, fmt, packed, codes, gamma, ws)
+        for _ in range(3):
+            B.bitlinear_pack(codes, fmt, packed, ws)
+        status.append(B.bitlinear_device_status(ws))
     if c["op"] == "lnquant":
         ln_w = torch.randn(K, generator=g, device=dev) * 0.1 + 1.0
         ln_b = torch.randn(K, generator=g, device=dev) * 0.1
