@@ -59,7 +59,7 @@ WORKLOADS = {
 
 KERNEL_SOURCE = {"absmean_kernel": "bl_weights.cu", "ternarize_flat_kernel": "bl_weights.cu",
                  "binarize_pack_kernel": "bl_weights.cu",
-                 "ternarize_pack_kernel": "bl_weights.cu", "gemv_i2_kernel": "bl_gemv.cu", "gemv1_i2_kernel": "bl_gemv1.cu", "gemv1_t5_kernel": "bl_gemv1.cu",
+                 "ternarize_pack_kernel": "bl_weights.cu", "gemv_i2_kernel": "bl_gemv.cu", "gemv1_i2_kernel": "bl_gemv1.cu", "gemv1_t5_kernel": "bl_gemv1.cu", "gemv1_b1_kernel": "bl_gemv1.cu",
                  "gemv_kernel": "bl_gemv.cu", "gemv_t5_kernel": "bl_gemv.cu", "gemv_i2_mt_kernel": "bl_gemv.cu", "act_quant_row_kernel": "bl_acts.cu",
                  "act_quant_kernel": "bl_acts.cu", "ln_quant_kernel": "bl_acts.cu", "ln_quant_reg_kernel": "bl_acts.cu", "gemm_i2_2sm_kernel": "bl_gemm_sm100.cu",
                  "gemm_i2_kernel": "bl_gemm_sm100.cu", "b1_to_i2_kernel": "bl_gemm_sm100.cu",
@@ -798,7 +798,7 @@ def decode_summary(d):
             "launch_duration": "CUDA events at the two ends of a graph of back-to-back forward calls"}
 
 
-def gemv1_fits(N, K, rb, t5=False, xwords=2):
+def gemv1_fits(N, K, rb, t5=False, xwords=2, cps=None):
     """Mirror of the library's one-token kernel geometry (bf16 tokens by
     default): K % 16 == 0, at most 512 lanes per row, at most four 16-byte code
     chunks per thread, and the (table,) token region, row sums and a ring of 8
@@ -811,11 +811,13 @@ def gemv1_fits(N, K, rb, t5=False, xwords=2):
     rpc = -(-N // grid)
     R = min(512 // lpr, rpc)
     threads = -(-(R * lpr) // 32) * 32
-    if -(-((5 if t5 else 4) * segs) // threads) > 4:
+    cps = cps or (5 if t5 else 4)  # 16-byte code chunks per segment (1-bit: 8)
+    per = -(-(cps * segs) // threads)
+    if per > 4 or (cps == 8 and per > 2):
         return False
-    xreg = -(-max(K * xwords, rb * (5 if t5 else 4)) // 16) * 16
+    xreg = -(-max(K * xwords, rb * cps) // 16) * 16
     fixed = (32768 if t5 else 0) + xreg + 4 * rpc
-    return any(fixed + 16 * st * threads <= 110 * 1024 for st in (8, 6))
+    return any(fixed + 16 * st * threads <= 110 * 1024 for st in ((6,) if cps == 8 else (8, 6)))
 
 
 def gemv_kernel_name(fmt, layers, M=1):
@@ -829,8 +831,11 @@ def gemv_kernel_name(fmt, layers, M=1):
     column-stationary kernel for rows of at most 768 segments and at most 1024
     rows per CTA; else the general one."""
     def one(N, K):
-        if fmt == 2:  # 1-bit rows of at most 4096 bytes: the lean kernel's 1-bit form
-            return "gemv_i2_kernel" if ((K + 7) // 8 + 15) // 16 * 16 <= 4096 else "gemv_kernel"
+        if fmt == 2:  # 1-bit: the one-token kernel where it fits, else the lean kernel's 1-bit form
+            rb = ((K + 7) // 8 + 15) // 16 * 16
+            if M == 1 and gemv1_fits(N, K, rb, cps=8):
+                return "gemv1_b1_kernel"
+            return "gemv_i2_kernel" if rb <= 4096 else "gemv_kernel"
         if fmt == 0:
             rb = ((K + 3) // 4 + 15) // 16 * 16
             if M == 1 and rb <= 8192 and gemv1_fits(N, K, rb):

@@ -1489,6 +1489,8 @@ cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int6
     return launch_gemv1(packed, rowbytes, gamma, N, K, x, xdt, scale, y, ydt, rg, ws, st);
   if (fmt == BL_PACK_T5 && M == 1 && gemv1_t5_fits(N, K, rowbytes, xdt))
     return launch_gemv1_t5(packed, rowbytes, gamma, N, K, x, xdt, scale, y, ydt, rg, ws, st);
+  if (fmt == BL_PACK_B1 && M == 1 && gemv1_b1_fits(N, K, rowbytes, xdt))
+    return launch_gemv1_b1(packed, rowbytes, gamma, N, K, x, xdt, scale, y, ydt, rg, ws, st);
   const int esz = (xdt == BL_F32) ? 4 : (xdt == BL_BF16 ? 2 : 1);
   const int ysz = (ydt == BL_BF16) ? 2 : 4;
   for (int64_t m0 = 0; m0 < M; m0 += mt_max) {

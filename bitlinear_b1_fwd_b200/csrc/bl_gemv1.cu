@@ -733,6 +733,285 @@ __global__ void __launch_bounds__(kG1MaxThreads, 1024 / kG1MaxThreads)
   if (XDT != BL_I8 && write_scale && b == 0 && tid == 0) scale[0] = s;
 }
 
+// ---------------------------------------------------------------------------
+// One token on 1-bit rows (the 1-bit variant: bit i of byte j of a packed
+// 32-bit word is weight 8 j + i of its 32, set = +1, clear = -1), in the same
+// column-stationary layout: a 16-byte segment holds 128 weights and thread t
+// keeps the 128 activation codes of its column in registers in the bit-plane
+// layout X[w][i] (byte j = the code of weight 32 w + 8 j + i), so a mask of
+// bit i of every byte and one dp4a collect the sum of the codes over the +1
+// weights of plane i, and the product is 2 S - X with X the sum of the
+// token's codes.  The codes
+// are written in element order over the raw token (128 per segment, 0 past
+// K).
+// ---------------------------------------------------------------------------
+__host__ __device__ inline int64_t g1b1_xregion(int64_t K, int xwords, int64_t rowbytes) {
+  const int64_t raw = K * xwords;      // the raw token
+  const int64_t codes = rowbytes * 8;  // 128 codes per 16-byte segment
+  return ((raw > codes ? raw : codes) + 15) / 16 * 16;
+}
+
+// a0 + 2 S over the 128 weights of a 1-bit segment, S the sum of the codes of
+// its +1 weights.  Plane i = 2 m + k is masked in (w >> 2m) at bit k, so two
+// accumulators (factors 1 and 2) hold every plane.
+__device__ __forceinline__ int dot_seg_b1(const uint4 wv, const uint32_t (&X)[4][8], int a0) {
+  const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+  int a_even = 0, a_odd = 0;
+#pragma unroll
+  for (int w = 0; w < 4; ++w)
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const uint32_t v = wd[w] >> (2 * m);
+      a_even = dp4a_us(v & 0x01010101u, X[w][2 * m], a_even);
+      a_odd = dp4a_us(v & 0x02020202u, X[w][2 * m + 1], a_odd);
+    }
+  return a0 + 2 * (a_even + (a_odd >> 1));
+}
+
+template <int XDT, int XC, int S, bool ALIGNED>
+__global__ void __launch_bounds__(kG1MaxThreads, 1024 / kG1MaxThreads)
+    gemv1_b1_kernel(const uint8_t* __restrict__ packed, int64_t rowbytes, const float* __restrict__ gamma,
+                    int64_t N, int64_t K, const void* __restrict__ x, float* __restrict__ scale,
+                    void* __restrict__ y, int ydt, int write_scale, const RowGroups rg, int R, int lpr, void* ws) {
+  constexpr int kXW = g1_xwords<XDT>();
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ uint32_t red[kG1MaxThreads / 32];
+  __shared__ float sh_gam[kMaxRowGroups];
+  __shared__ int64_t sh_end[kMaxRowGroups];
+  __shared__ float sh_s;
+  __shared__ __align__(8) uint64_t xbar;  // completion of the token's bulk copy
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int T = blockDim.x;
+  const int segs = static_cast<int>(rowbytes >> 4);
+  const int64_t G = gridDim.x, b = blockIdx.x;
+  const int64_t per = N / G, extra = N % G;
+  const int64_t row0 = b * per + (b < extra ? b : extra);
+  const int nrows = static_cast<int>(per + (b < extra ? 1 : 0));
+  const int r0_raw = tid / lpr, c_raw = tid - r0_raw * lpr;
+  const bool row_ok = r0_raw < R;
+  const bool col_ok = row_ok && c_raw < segs;
+  const int r0 = row_ok ? r0_raw : 0;
+  const int c = col_ok ? c_raw : 0;
+  const int nr = (row_ok && r0 < nrows) ? (nrows - r0 + R - 1) / R : 0;
+  const uint32_t step = static_cast<uint32_t>(R * rowbytes);
+  const int kch = static_cast<int>(K >> 4);  // 16-element chunks of the token (K % 16 == 0)
+  const int nch = 8 * segs;                  // 16-code chunks of the codes region (0 past K)
+  const uint32_t xbytes = static_cast<uint32_t>(K * kXW);
+  // shared memory: the token region (the raw token, then its codes), the row
+  // ring [S][T] x 16 bytes, the row sums
+  const int64_t xreg = g1b1_xregion(K, kXW, rowbytes);
+  uint8_t* xbuf = smem;
+  const uint32_t ring_s = smem_u32(xbuf + xreg) + 16u * tid;
+  const uint32_t tstride = 16u * T;
+  int* rsum = reinterpret_cast<int*>(xbuf + xreg + static_cast<int64_t>(S) * T * 16);
+
+  // 0. before the wait: the first bytes of the CTA's rows into L2, the row
+  //    sums zeroed, the token barrier set up
+  {
+    const int64_t bytes = static_cast<int64_t>(nrows) * rowbytes;
+    l2_prefetch_bulk(packed + row0 * rowbytes, bytes < BL_G1_PREFETCH ? bytes : BL_G1_PREFETCH);
+  }
+  for (int i = tid; i < nrows; i += T) rsum[i] = 0;
+#pragma unroll
+  for (int i = 0; i < kMaxRowGroups; ++i)
+    if (tid == i) sh_end[i] = rg.end[i];
+  if (tid == 0) {
+    mbar_init(&xbar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  pdl_wait(packed, gamma, x, scale, y);
+  pdl_launch_dependents();
+
+  // 1. the token by one bulk copy (bounded wait: on expiry the CTA records the
+  //    timeout, lets the copy land and leaves)
+  if (tid == 0) {
+    mbar_expect_tx(&xbar, xbytes);
+    bulk_load(xbuf, x, xbytes, &xbar);
+  }
+  if (tid < rg.n) sh_gam[tid] = __ldcg(gamma + tid);
+  if (XDT == BL_I8 && tid == 0) sh_s = __ldcg(scale);
+  const bool got = wait_drain(&xbar, 0, kG1WaitCycles);
+  if (__syncthreads_or(!got)) {
+    if (tid == 0) {
+      set_flag(ws, kFlagTimeout, 0x603);
+      wait_drain(&xbar, 0, kG1WaitCycles);
+    }
+    return;
+  }
+  const uint8_t* gp = packed + (row0 + r0) * rowbytes + static_cast<int64_t>(c) * 16;
+#pragma unroll
+  for (int j = 0; j < S - 1; ++j) {
+    if (col_ok && j < nr) cp_async16_s(ring_s + j * tstride, gp);
+    cp_async_commit();
+    gp += step;
+  }
+
+  // 2. per-token absmax on the magnitude bits (finite inputs)
+  float s;
+  if constexpr (XDT != BL_I8) {
+    uint32_t mx = 0;
+#pragma unroll
+    for (int u = 0; u < XC; ++u) {
+      const int g = tid + T * u;
+      if (g < kch)
+#pragma unroll
+        for (int i = 0; i < kXW; ++i) {
+          const uint4 v = *reinterpret_cast<const uint4*>(xbuf + (static_cast<int64_t>(g) * kXW + i) * 16);
+          if constexpr (XDT == BL_F32) {
+            const uint32_t a = max(v.x & 0x7fffffffu, v.y & 0x7fffffffu);
+            const uint32_t b2 = max(v.z & 0x7fffffffu, v.w & 0x7fffffffu);
+            mx = max(mx, max(a, b2));
+          } else {
+            const uint32_t a = __vmaxu2(v.x & 0x7fff7fffu, v.y & 0x7fff7fffu);
+            const uint32_t b2 = __vmaxu2(v.z & 0x7fff7fffu, v.w & 0x7fff7fffu);
+            mx = __vmaxu2(mx, __vmaxu2(a, b2));
+          }
+        }
+    }
+    if constexpr (XDT == BL_BF16) mx = max(mx & 0xffffu, mx >> 16) << 16;
+    const uint32_t m = __reduce_max_sync(0xffffffffu, mx);
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    uint32_t mm = 0;
+    for (int w = 0; w < (T >> 5); ++w) mm = max(mm, red[w]);
+    s = fmaxf(__uint_as_float(mm), 1e-6f);
+  } else {
+    s = sh_s;
+  }
+
+  // 3. the codes of the thread's chunks in element order, written over the
+  //    raw token once every thread has read its raw chunks
+  {
+    const float c127 = (XDT == BL_I8) ? 0.0f : __fdiv_rn(127.0f, s);
+    uint4 cw[XC];
+#pragma unroll
+    for (int u = 0; u < XC; ++u) {
+      const int g = tid + T * u;
+      cw[u] = make_uint4(0u, 0u, 0u, 0u);  // padding chunks (past K): code 0
+      if (g < kch) {
+        const uint8_t* src = xbuf + static_cast<int64_t>(g) * kXW * 16;
+        if constexpr (XDT == BL_I8) {
+          cw[u] = *reinterpret_cast<const uint4*>(src);
+        } else {
+          float e[16];
+          if constexpr (XDT == BL_F32) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * i);
+              e[4 * i] = __uint_as_float(v.x); e[4 * i + 1] = __uint_as_float(v.y);
+              e[4 * i + 2] = __uint_as_float(v.z); e[4 * i + 3] = __uint_as_float(v.w);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * i);
+              const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                e[8 * i + 2 * k] = __uint_as_float(wv[k] << 16);
+                e[8 * i + 2 * k + 1] = __uint_as_float(wv[k] & 0xffff0000u);
+              }
+            }
+          }
+          cw[u] = g1_codes16<false>(e, s, c127);
+        }
+      }
+    }
+    __syncthreads();  // every raw chunk has been read
+#pragma unroll
+    for (int u = 0; u < XC; ++u) {
+      const int g = tid + T * u;
+      if (g < nch) *reinterpret_cast<uint4*>(xbuf + static_cast<int64_t>(g) * 16) = cw[u];
+    }
+  }
+  __syncthreads();
+
+  // 4. this thread's 128 codes in the bit-plane layout and their sum (the
+  //    product is 2 S - X, S the sum over the +1 weights: X is taken off once
+  //    per row, as the row sum's starting value)
+  uint32_t X[4][8];
+  int csum = 0;
+  {
+    uint32_t lw[32];  // lw[m]: codes 4m .. 4m + 3 of the segment
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint4 t = col_ok ? *reinterpret_cast<const uint4*>(xbuf + (static_cast<int64_t>(c) * 8 + i) * 16)
+                             : make_uint4(0u, 0u, 0u, 0u);
+      lw[4 * i] = t.x;
+      lw[4 * i + 1] = t.y;
+      lw[4 * i + 2] = t.z;
+      lw[4 * i + 3] = t.w;
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) csum = __dp4a(static_cast<int>(lw[i]), 0x01010101, csum);
+    // X[w][i] byte j = code of weight 32 w + 8 j + i = byte (i & 3) of
+    // lw[8 w + 2 j + (i >> 2)]
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int o = 8 * w + (i >> 2);
+        const uint32_t sel = static_cast<uint32_t>(i & 3) | (static_cast<uint32_t>(4 + (i & 3)) << 4);
+        X[w][i] = __byte_perm(__byte_perm(lw[o], lw[o + 2], sel), __byte_perm(lw[o + 4], lw[o + 6], sel), 0x5410);
+      }
+  }
+  const int init = -csum;
+  const uint32_t gmask = ALIGNED ? 0xffffffffu : __match_any_sync(0xffffffffu, row_ok ? r0_raw : -1 - lane);
+  const bool leader = ALIGNED ? lane == 0 : (__ffs(gmask) - 1) == lane;
+  uint32_t rs = smem_u32(rsum + r0);
+  const uint32_t rstep = 4u * R;
+
+  // 5. the stream, as in gemv1_i2_kernel
+  auto consume = [&](const uint4 wv) {
+    int v = dot_seg_b1(wv, X, init);
+    v = __reduce_add_sync(gmask, v);
+    if (leader) red_add_s(rs, v);
+    rs += rstep;
+  };
+  int k = 0;
+  for (; k < nr - 2 * S + 2; k += S) {
+#pragma unroll
+    for (int j = 0; j < S; ++j) {
+      if (col_ok) cp_async16_s(ring_s + ((j + S - 1) % S) * tstride, gp);
+      cp_async_commit();
+      gp += step;
+      cp_async_wait<S - 1>();
+      consume(lds128(ring_s + j * tstride));
+    }
+  }
+  for (; k < nr; ++k) {
+    if (col_ok && k + S - 1 < nr) cp_async16_s(ring_s + ((k + S - 1) % S) * tstride, gp);
+    cp_async_commit();
+    gp += step;
+    cp_async_wait<S - 1>();
+    consume(lds128(ring_s + (k % S) * tstride));
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // 6. dequantize and store the CTA's outputs (coalesced)
+  const float cf1 = dequant_factor(sh_gam[0], s);
+  for (int r = tid; r < nrows; r += T) {
+    const int a = rsum[r];
+    const int64_t n = row0 + r;
+    float cf = cf1;
+    if (rg.n > 1) {
+      int gi = 0;
+      while (gi + 1 < rg.n && n >= sh_end[gi]) ++gi;
+      cf = dequant_factor(sh_gam[gi], s);
+    }
+    if (ydt == BL_I32)
+      static_cast<int32_t*>(y)[n] = a;
+    else if (ydt == BL_F32)
+      static_cast<float*>(y)[n] = __fmul_rn(__int2float_rn(a), cf);
+    else
+      static_cast<__nv_bfloat16*>(y)[n] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(a), cf));
+  }
+  if (XDT != BL_I8 && write_scale && b == 0 && tid == 0) scale[0] = s;
+}
+
 // Launch geometry: R rows per step, threads rounded up to whole warps, and
 // the token chunks per thread (1, 2 or 4).
 struct Gemv1Geom {
@@ -740,7 +1019,7 @@ struct Gemv1Geom {
   int64_t grid, rows_per_cta, smem;
 };
 
-static bool gemv1_geom(int64_t N, int64_t K, int64_t rowbytes, int xdt, Gemv1Geom* g, bool t5 = false) {
+static bool gemv1_geom(int64_t N, int64_t K, int64_t rowbytes, int xdt, Gemv1Geom* g, int fmt = BL_PACK_I2) {
   const int64_t segs = rowbytes / 16;
   if (K % 16 != 0 || segs < 1 || segs > kG1MaxThreads) return false;
   const int64_t sms = device_sms();
@@ -756,14 +1035,23 @@ static bool gemv1_geom(int64_t N, int64_t K, int64_t rowbytes, int xdt, Gemv1Geo
   g->lpr = static_cast<int>(lpr);
   g->threads = static_cast<int>((R * lpr + 31) / 32 * 32);
   // 16-byte chunks of the codes: 4 per 2-bit segment (64 codes), 5 per base-3
-  // segment (80 codes)
-  const int64_t per = ((t5 ? 5 : 4) * segs + g->threads - 1) / g->threads;
+  // segment (80 codes), 8 per 1-bit segment (128 codes)
+  const int cps = fmt == BL_PACK_T5 ? 5 : (fmt == BL_PACK_B1 ? 8 : 4);
+  const int64_t per = (cps * segs + g->threads - 1) / g->threads;
   if (per > 4) return false;
+  // 1-bit rows needing more than two chunks per thread (K above 16384) ran
+  // slower here than in the lean kernel (70B down-projection: 17.5 against
+  // 16.0 us), so they stay there
+  if (fmt == BL_PACK_B1 && per > 2) return false;
   g->xc = per <= 1 ? 1 : (per <= 2 ? 2 : 4);
   const int xwords = xdt == BL_F32 ? 4 : (xdt == BL_BF16 ? 2 : 1);
-  const int64_t fixed = (t5 ? kT1LutBytes + g1t5_xregion(K, xwords, rowbytes) : g1_xregion(K, xwords, rowbytes)) +
-                        4 * g->rows_per_cta;
+  const int64_t xreg = fmt == BL_PACK_T5   ? kT1LutBytes + g1t5_xregion(K, xwords, rowbytes)
+                       : fmt == BL_PACK_B1 ? g1b1_xregion(K, xwords, rowbytes)
+                                           : g1_xregion(K, xwords, rowbytes);
+  const int64_t fixed = xreg + 4 * g->rows_per_cta;
   for (int st : {kG1StagesMax, 6}) {  // the deepest ring that keeps two CTAs per SM
+    // (the 1-bit kernel's 32 code registers leave room for 6 stages only)
+    if (fmt == BL_PACK_B1 && st > 6) continue;
     g->stages = st;
     g->smem = fixed + int64_t{16} * st * g->threads;
     if (g->smem <= kG1MaxSmem) return true;
@@ -778,15 +1066,28 @@ bool gemv1_fits(int64_t N, int64_t K, int64_t rowbytes, int xdt) {
 
 bool gemv1_t5_fits(int64_t N, int64_t K, int64_t rowbytes, int xdt) {
   Gemv1Geom g;
-  return gemv1_geom(N, K, rowbytes, xdt, &g, true);
+  return gemv1_geom(N, K, rowbytes, xdt, &g, BL_PACK_T5);
 }
 
-template <bool T5, int XDT, int XC, int S>
+bool gemv1_b1_fits(int64_t N, int64_t K, int64_t rowbytes, int xdt) {
+  Gemv1Geom g;
+  return gemv1_geom(N, K, rowbytes, xdt, &g, BL_PACK_B1);
+}
+
+template <int FMT, int XDT, int XC, int S>
 static cudaError_t launch_gemv1_t(const Gemv1Geom& g, const uint8_t* packed, int64_t rowbytes, const float* gamma,
                                   int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
                                   int write_scale, const RowGroups& rg, void* ws, cudaStream_t st) {
-  auto kern = T5 ? (g.lpr % 32 == 0 ? gemv1_t5_kernel<XDT, XC, S, true> : gemv1_t5_kernel<XDT, XC, S, false>)
-                 : (g.lpr % 32 == 0 ? gemv1_i2_kernel<XDT, XC, S, true> : gemv1_i2_kernel<XDT, XC, S, false>);
+  const bool al = g.lpr % 32 == 0;
+  auto pick = [al]() {
+    if constexpr (FMT == BL_PACK_T5)
+      return al ? gemv1_t5_kernel<XDT, XC, S, true> : gemv1_t5_kernel<XDT, XC, S, false>;
+    else if constexpr (FMT == BL_PACK_B1)
+      return al ? gemv1_b1_kernel<XDT, XC, S, true> : gemv1_b1_kernel<XDT, XC, S, false>;
+    else
+      return al ? gemv1_i2_kernel<XDT, XC, S, true> : gemv1_i2_kernel<XDT, XC, S, false>;
+  };
+  auto kern = pick();
   const size_t smem = static_cast<size_t>(g.smem);
   if (smem > 48 * 1024) {
     const cudaError_t e =
@@ -799,50 +1100,58 @@ static cudaError_t launch_gemv1_t(const Gemv1Geom& g, const uint8_t* packed, int
   return cudaGetLastError();
 }
 
-template <bool T5, int XDT, int XC>
+template <int FMT, int XDT, int XC>
 static cudaError_t launch_gemv1_s(const Gemv1Geom& g, const uint8_t* packed, int64_t rowbytes, const float* gamma,
                                   int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
                                   int write_scale, const RowGroups& rg, void* ws, cudaStream_t st) {
-  if (g.stages == kG1StagesMax)
-    return launch_gemv1_t<T5, XDT, XC, kG1StagesMax>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale,
-                                                     rg, ws, st);
-  return launch_gemv1_t<T5, XDT, XC, 6>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
+  if constexpr (FMT != BL_PACK_B1) {  // the 1-bit kernel runs with 6 stages only
+    if (g.stages == kG1StagesMax)
+      return launch_gemv1_t<FMT, XDT, XC, kG1StagesMax>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt,
+                                                       write_scale, rg, ws, st);
+  }
+  return launch_gemv1_t<FMT, XDT, XC, 6>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
 }
 
-template <bool T5, int XDT>
+template <int FMT, int XDT>
 static cudaError_t launch_gemv1_x(const Gemv1Geom& g, const uint8_t* packed, int64_t rowbytes, const float* gamma,
                                   int64_t N, int64_t K, const void* x, float* scale, void* y, int ydt,
                                   int write_scale, const RowGroups& rg, void* ws, cudaStream_t st) {
   if (g.xc == 1)
-    return launch_gemv1_s<T5, XDT, 1>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
+    return launch_gemv1_s<FMT, XDT, 1>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
   if (g.xc == 2)
-    return launch_gemv1_s<T5, XDT, 2>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
-  return launch_gemv1_s<T5, XDT, 4>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
+    return launch_gemv1_s<FMT, XDT, 2>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
+  return launch_gemv1_s<FMT, XDT, 4>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, write_scale, rg, ws, st);
 }
 
-template <bool T5>
+template <int FMT>
 static cudaError_t launch_gemv1_f(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
                                   const void* x, int xdt, float* scale, void* y, int ydt, const RowGroups& rg,
                                   void* ws, cudaStream_t st) {
   Gemv1Geom g;
-  if (!gemv1_geom(N, K, rowbytes, xdt, &g, T5)) return cudaErrorInvalidValue;
+  if (!gemv1_geom(N, K, rowbytes, xdt, &g, FMT)) return cudaErrorInvalidValue;
   if (xdt == BL_F32)
-    return launch_gemv1_x<T5, BL_F32>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 1, rg, ws, st);
+    return launch_gemv1_x<FMT, BL_F32>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 1, rg, ws, st);
   if (xdt == BL_BF16)
-    return launch_gemv1_x<T5, BL_BF16>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 1, rg, ws, st);
-  return launch_gemv1_x<T5, BL_I8>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 0, rg, ws, st);
+    return launch_gemv1_x<FMT, BL_BF16>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 1, rg, ws, st);
+  return launch_gemv1_x<FMT, BL_I8>(g, packed, rowbytes, gamma, N, K, x, scale, y, ydt, 0, rg, ws, st);
 }
 
 cudaError_t launch_gemv1(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
                          const void* x, int xdt, float* scale, void* y, int ydt, const RowGroups& rg, void* ws,
                          cudaStream_t st) {
-  return launch_gemv1_f<false>(packed, rowbytes, gamma, N, K, x, xdt, scale, y, ydt, rg, ws, st);
+  return launch_gemv1_f<BL_PACK_I2>(packed, rowbytes, gamma, N, K, x, xdt, scale, y, ydt, rg, ws, st);
 }
 
 cudaError_t launch_gemv1_t5(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
                             const void* x, int xdt, float* scale, void* y, int ydt, const RowGroups& rg, void* ws,
                             cudaStream_t st) {
-  return launch_gemv1_f<true>(packed, rowbytes, gamma, N, K, x, xdt, scale, y, ydt, rg, ws, st);
+  return launch_gemv1_f<BL_PACK_T5>(packed, rowbytes, gamma, N, K, x, xdt, scale, y, ydt, rg, ws, st);
+}
+
+cudaError_t launch_gemv1_b1(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
+                            const void* x, int xdt, float* scale, void* y, int ydt, const RowGroups& rg, void* ws,
+                            cudaStream_t st) {
+  return launch_gemv1_f<BL_PACK_B1>(packed, rowbytes, gamma, N, K, x, xdt, scale, y, ydt, rg, ws, st);
 }
 
 }  // namespace bl

@@ -111,6 +111,12 @@ bool gemv1_t5_fits(int64_t N, int64_t K, int64_t rowbytes, int xdt);
 cudaError_t launch_gemv1_t5(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
                             const void* x, int xdt, float* scale, void* y, int ydt, const RowGroups& rg, void* ws,
                             cudaStream_t st);
+// And on 1-bit rows (128 weights per 16-byte segment, the codes of a column
+// in registers in bit-plane order), within the same budget.
+bool gemv1_b1_fits(int64_t N, int64_t K, int64_t rowbytes, int xdt);
+cudaError_t launch_gemv1_b1(const uint8_t* packed, int64_t rowbytes, const float* gamma, int64_t N, int64_t K,
+                            const void* x, int xdt, float* scale, void* y, int ydt, const RowGroups& rg, void* ws,
+                            cudaStream_t st);
 
 cudaError_t launch_gemv(const uint8_t* packed, int fmt, const float* gamma, int64_t N, int64_t K,
                         const void* x, int xdt, float* scale, int64_t M, void* y, int ydt,

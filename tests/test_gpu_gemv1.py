@@ -1,6 +1,6 @@
 """GPU parity of the one-token decode GEMVs (the column-stationary kernels
-with K % 16 == 0: 2-bit rows of up to 8 KB, and base-3 rows where the
-table, token and ring fit) against the oracle.
+with K % 16 == 0: 2-bit rows of up to 8 KB, and base-3 and 1-bit rows where
+the table, token, codes and ring fit) against the oracle.
 
 The cases walk its geometry: segments per row from 1 to 512 (several rows per
 warp, warps that span two rows, one row per warp), one to about a thousand
@@ -20,6 +20,7 @@ pytestmark = pytest.mark.gpu
 
 I2 = B.BL_PACK_I2
 T5 = B.BL_PACK_T5
+B1 = B.BL_PACK_B1
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -35,7 +36,17 @@ def _check(orc, N, K, xkind, seed, zero_token=False, ydts=(B.BL_I32, B.BL_F32, B
     x = synth.entry_outliers(synth.normal_f32(seed + 1, (1, K)), seed + 2, 0.01, 20.0)
     if zero_token:
         x[:] = 0.0
-    g, _, packed = quantize_weights(W, fmt, codes=False)
+    if fmt == B1:  # the 1-bit variant: beta in gamma's place
+        N_, K_ = W.shape
+        packed_t = torch.empty((N_, B.bitlinear_packed_row_bytes(K_, B1)), dtype=torch.uint8, device="cuda")
+        beta = torch.empty((1,), dtype=torch.float32, device="cuda")
+        alpha = torch.empty((1,), dtype=torch.float32, device="cuda")
+        ws = torch.zeros(B.bitlinear_binarize_weights_workspace_bytes(N_, K_), dtype=torch.uint8, device="cuda")
+        B.bitlinear_binarize_weights(dev(W), packed_t, None, beta, alpha, ws)
+        torch.cuda.synchronize()
+        g, packed = np.float32(beta.item()), host(packed_t)
+    else:
+        g, _, packed = quantize_weights(W, fmt, codes=False)
     scale = None
     if xkind == "int8":
         x, scale = orc.act_quant(x)
@@ -135,3 +146,25 @@ def test_gemv1_t5_zero_token_and_rows_per_cta(orc):
     _check(orc, 640, 3200, "bf16", seed=7, zero_token=True, fmt=T5)
     for N in (1, 149, 30_000):
         _check(orc, N, 400, "bf16", seed=N, fmt=T5, ydts=(B.BL_I32, B.BL_BF16))
+
+
+@pytest.mark.parametrize("N,K", [
+    (300, 128),     # one 1-bit segment per row (128 weights)
+    (1000, 1024),   # 8 segments
+    (777, 3200),    # 25 segments: a warp spans two rows
+    (900, 8192),    # 70B up rows: 64 segments, 8 rows per step
+    (3200, 8640),   # 68 segments in 96 lanes per row, two chunks per thread
+    (500, 16384),   # 128 segments, two chunks per thread
+    (160, 28672),   # 70B down rows: four chunks per thread, so the lean kernel
+])
+@pytest.mark.parametrize("xkind", ["bf16", "f32", "int8"])
+def test_gemv1_b1_geometry(orc, N, K, xkind):
+    """1-bit rows in the column-stationary layout (bit-plane codes in
+    registers), and past its limit the lean kernel."""
+    _check(orc, N, K, xkind, seed=N * 19 + K, fmt=B1)
+
+
+def test_gemv1_b1_zero_token_and_rows_per_cta(orc):
+    _check(orc, 640, 3200, "bf16", seed=9, zero_token=True, fmt=B1)
+    for N in (1, 149, 30_000):
+        _check(orc, N, 1024, "bf16", seed=N + 3, fmt=B1, ydts=(B.BL_I32, B.BL_BF16))
