@@ -909,6 +909,7 @@ PROFILE_CASES = {
     "backward_3b_down": dict(N=3200, K=8640, fmt=0, M=1, sigma=0.02, op="backward"),
     "backward_3b_up_m8": dict(N=8640, K=3200, fmt=0, M=8, sigma=0.02, op="backward"),
     "decode_70b_down_t5": dict(N=8192, K=28672, fmt=1, M=1, sigma=0.01, op="forward"),
+    "decode_70b_down_1bit": dict(N=8192, K=28672, fmt=2, M=1, sigma=0.01, op="forward"),
     "lnquant_70b_down": dict(N=8192, K=28672, fmt=0, M=256, sigma=0.01, op="lnquant"),
     "pack_3b_up": dict(N=8640, K=3200, fmt=0, M=1, sigma=0.02, op="pack"),
 }
