@@ -912,6 +912,7 @@ PROFILE_CASES = {
     "decode_70b_down_1bit": dict(N=8192, K=28672, fmt=2, M=1, sigma=0.01, op="forward"),
     "lnquant_70b_down": dict(N=8192, K=28672, fmt=0, M=256, sigma=0.01, op="lnquant"),
     "pack_3b_up": dict(N=8640, K=3200, fmt=0, M=1, sigma=0.02, op="pack"),
+    "actquant_16x40000": dict(N=16, K=40000, fmt=0, M=16, sigma=0.02, op="actquant"),
 }
 
 
@@ -947,6 +948,11 @@ def run_profile_case(name):
         for _ in range(3):
             B.bitlinear_pack(codes, fmt, packed, ws)
         status.append(B.bitlinear_device_status(ws))
+    if c["op"] == "actquant":  # A4 alone on rows longer than the one-CTA-per-token kernels take
+        xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+        sc = torch.empty(M, dtype=torch.float32, device=dev)
+        for _ in range(3):
+            B.bitlinear_quantize_acts(x, xq, sc)
     if c["op"] == "lnquant":
         ln_w = torch.randn(K, generator=g, device=dev) * 0.1 + 1.0
         ln_b = torch.randn(K, generator=g, device=dev) * 0.1

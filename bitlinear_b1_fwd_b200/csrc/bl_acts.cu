@@ -2,9 +2,10 @@
 //
 // "BitNet b1.58深度解析：三值权重如何重塑大模型推理" §3.2 and §5.2: each token
 // (one row of x over K) is scaled by its own max |x| (floored at 1e-6) and
-// x_q = clamp(round(x / s * 127), -127, 127).  Rows of up to 8 K (bf16) or
-// 4 K (fp32) elements: one CTA per token, read once into registers.  Other
-// rows: one warp per token, two passes whose loads go out kActBatch at a time.
+// x_q = clamp(round(x / s * 127), -127, 127).  Rows of up to 32 K (bf16) or
+// 16 K (fp32) elements with K % 8 (bf16) or K % 4 (fp32) == 0: one CTA per
+// token, read once into registers.  Other rows: one warp per token, two
+// passes whose loads go out kActBatch at a time.
 #include <type_traits>
 
 #include "bl_common.cuh"
@@ -34,19 +35,23 @@ __device__ __forceinline__ void bf16x8(const uint4 r, float* e) {
   }
 }
 
-// Rows with K % 8 == 0 (bf16) or K % 4 == 0 (fp32) and at most
-// kActRowThreads NV 16-byte words: one CTA per token, read once.  Thread t
-// issues its NV loads (words t, t + T, ...) together; the absmax meets across
-// the CTA (warp shuffles, one barrier) and the codes come from registers.
-// Many small CTAs per SM, each at its own phase, keep loads in flight while
-// others compute.
+// Rows with K % 8 == 0 (bf16) or K % 4 == 0 (fp32) and at most T NV 16-byte
+// words: one CTA of T threads per token, read once.  Thread t issues its NV
+// loads (words t, t + T, ...) together; the absmax meets across the CTA (warp
+// shuffles, one barrier) and the codes come from registers.  Rows of up to
+// 8192 bf16 elements take 128-thread CTAs, many per SM, each at its own
+// phase, keeping loads in flight while others compute; longer rows (up to
+// 32768 bf16 elements) take 512-thread CTAs, so that even a few tokens spread
+// over as many threads as their words.
 constexpr int kActRowThreads = 128;
+constexpr int kActLongRowThreads = 512;
 
-template <int XDT, int NV>
-__global__ void __launch_bounds__(kActRowThreads)
+template <int XDT, int NV, int T = kActRowThreads>
+__global__ void __launch_bounds__(T)
     act_quant_row_kernel(const void* __restrict__ x, int64_t M, int64_t K, int8_t* __restrict__ xq,
                          float* __restrict__ scale) {
   pdl_enter(x, xq, scale);
+  constexpr int kActRowThreads = T;  // this instance's CTA size
   constexpr int EPW = (XDT == BL_F32) ? 4 : 8;  // elements per 16-byte word
   __shared__ float red[kActRowThreads / 32];
   const int t = threadIdx.x, lane = t & 31;
@@ -503,6 +508,29 @@ cudaError_t launch_act_quant(const void* x, int xdt, int64_t M, int64_t K, int8_
       BL_AQ(BL_BF16, 8)
     }
 #undef BL_AQ
+  }
+  if ((K % epw) == 0 && nv <= kActLongRowThreads * 8) {
+    int per_sm = 1;
+#define BL_AQL(XDT, NV)                                                                                      \
+  if (nv <= kActLongRowThreads * (NV)) {                                                                     \
+    auto kern = act_quant_row_kernel<XDT, NV, kActLongRowThreads>;                                           \
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kActLongRowThreads, 0) != cudaSuccess || \
+        per_sm < 1)                                                                                          \
+      per_sm = 1;                                                                                            \
+    const int64_t cap = static_cast<int64_t>(device_sms()) * per_sm;                                         \
+    const cudaError_t le_ = launch_pdl(kern, static_cast<unsigned>(M < cap ? M : cap), kActLongRowThreads, 0, \
+                                       st, x, M, K, xq, scale);                                              \
+    if (le_ != cudaSuccess) return le_;                                                                      \
+    return cudaGetLastError();                                                                               \
+  }
+    if (xdt == BL_F32) {
+      BL_AQL(BL_F32, 4)
+      BL_AQL(BL_F32, 8)
+    } else {
+      BL_AQL(BL_BF16, 4)
+      BL_AQL(BL_BF16, 8)
+    }
+#undef BL_AQL
   }
   if (xdt == BL_F32)
     { const cudaError_t le_ = launch_pdl(act_quant_kernel<BL_F32>, grid_for(reinterpret_cast<const void*>(act_quant_kernel<BL_F32>)), kActThreads, 0, st, x, M, K, xq, scale, vec); if (le_ != cudaSuccess) return le_; }

@@ -450,14 +450,30 @@ __global__ void __launch_bounds__(256)
   pdl_enter(codes, packed, ws);
   constexpr int PER = (FMT == BL_PACK_I2) ? 4 : (FMT == BL_PACK_T5 ? 5 : 8);
   constexpr int WPS = 16 * PER;
-  const int64_t segs = rowbytes / 16;
-  const int64_t total = N * segs;
-  for (int64_t gid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; gid < total;
-       gid += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t n = gid / segs;
-    const int64_t sg = gid - n * segs;
+  // N segs < 2^32 (N K <= 2^32): 32-bit item indices
+  const uint32_t segs = static_cast<uint32_t>(rowbytes / 16);
+  const uint32_t total = static_cast<uint32_t>(N) * segs;
+  // K % 16 == 0: every 16-code chunk of a segment starts 16-byte aligned and
+  // lies wholly inside or past the row, so the segment's codes come in with
+  // 16-byte loads (chunks past K read as 0)
+  const bool vec = (K & 15) == 0;
+  for (uint32_t gid = blockIdx.x * blockDim.x + threadIdx.x; gid < total; gid += gridDim.x * blockDim.x) {
+    const uint32_t n32 = gid / segs;
+    const int64_t n = n32;
+    const int64_t sg = gid - n32 * segs;
     const int64_t k0 = sg * WPS;
     const int8_t* src = codes + n * K + k0;
+    uint32_t cw[WPS / 4];
+    if (vec) {
+#pragma unroll
+      for (int j = 0; j < WPS / 16; ++j) {
+        const uint4 v = k0 + 16 * j < K ? __ldcg(reinterpret_cast<const uint4*>(src + 16 * j)) : make_uint4(0, 0, 0, 0);
+        cw[4 * j] = v.x;
+        cw[4 * j + 1] = v.y;
+        cw[4 * j + 2] = v.z;
+        cw[4 * j + 3] = v.w;
+      }
+    }
     bool bad = false;
     uint32_t out[4];
 #pragma unroll
@@ -470,7 +486,8 @@ __global__ void __launch_bounds__(256)
         for (int ii = 0; ii < PER; ++ii) {
           const int i = (FMT == BL_PACK_T5) ? PER - 1 - ii : ii;
           const int kk = 4 * PER * w + PER * b + i;
-          int c = (k0 + kk < K) ? static_cast<int>(__ldcg(src + kk)) : 0;
+          int c = vec ? static_cast<int>(static_cast<int8_t>(cw[kk >> 2] >> (8 * (kk & 3))))
+                      : ((k0 + kk < K) ? static_cast<int>(__ldcg(src + kk)) : 0);
           if constexpr (FMT == BL_PACK_B1) {  // {-1, +1}; pad bits 0
             if (k0 + kk < K && c != 1 && c != -1) bad = true;
             byte |= (c == 1 ? 1u : 0u) << i;

@@ -69,7 +69,7 @@ def test_binarize_packed_only_matches(orc):
 
 def test_pack_b1_from_codes(orc):
     rng = np.random.default_rng(605)
-    for K in (1, 127, 128, 1000):
+    for K in (1, 127, 128, 1000, 1024, 4096):
         codes = np.where(rng.random((7, K)) < 0.5, 1, -1).astype(np.int8)
         packed = torch.full((7, B.bitlinear_packed_row_bytes(K, B1)), 0xAB, dtype=torch.uint8, device="cuda")
         ws = torch.zeros(256, dtype=torch.uint8, device="cuda")

@@ -61,6 +61,14 @@ def _act_cases():
     z[1] = 0.0
     z[2] = 1e-9
     yield "zero_and_tiny_rows", z
+    # long rows: one 512-thread CTA per token (bf16 up to 32768, fp32 up to 16384
+    # elements), and past that the warp-per-token kernel
+    yield "70b_down_16x28672_bf16", synth.to_bf16_bits(
+        synth.entry_outliers(synth.normal_f32(46, (16, 28672)), 47, 0.001, 30.0))
+    yield "long_3x16384_f32", synth.normal_f32(48, (3, 16384))
+    yield "long_2x32768_bf16", synth.to_bf16_bits(synth.normal_f32(49, (2, 32768)))
+    yield "longer_2x40000_bf16", synth.to_bf16_bits(synth.normal_f32(50, (2, 40000)))
+    yield "long_5x9000_f32", synth.normal_f32(51, (5, 9000))
 
 
 @pytest.mark.parametrize("name,x", list(_act_cases()), ids=lambda v: v if isinstance(v, str) else "")
@@ -182,7 +190,7 @@ def test_ternarize_threshold_boundary(orc):
 
 def test_pack_and_bad_codes(orc):
     rng = np.random.default_rng(3)
-    for (N, K) in [(5, 3), (7, 129), (64, 3200), (3, 8193)]:
+    for (N, K) in [(5, 3), (7, 129), (64, 3200), (3, 8193), (3, 48), (9, 4096)]:
         codes = rng.integers(-1, 2, (N, K), dtype=np.int8)
         for fmt in (I2, T5):
             packed = torch.empty((N, B.bitlinear_packed_row_bytes(K, fmt)), dtype=torch.uint8, device="cuda")
@@ -200,6 +208,17 @@ def test_pack_and_bad_codes(orc):
     fixed = bad.copy()
     fixed[2, 17] = 0
     assert np.array_equal(host(packed), orc.pack(fixed, I2))
+    # the same with K % 16 == 0 (codes read 16 at a time), both formats
+    for fmt in (I2, T5):
+        bad = rng.integers(-1, 2, (3, 80), dtype=np.int8)
+        bad[1, 66] = -2
+        ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+        packed = torch.empty((3, B.bitlinear_packed_row_bytes(80, fmt)), dtype=torch.uint8, device="cuda")
+        B.bitlinear_pack(dev(bad), fmt, packed, ws)
+        assert B.bitlinear_device_status(ws) == B.BL_ERR_BAD_CODE
+        fixed = bad.copy()
+        fixed[1, 66] = 0
+        assert np.array_equal(host(packed), orc.pack(fixed, fmt))
 
 
 # --- steps 4-6: forward ------------------------------------------------------------
