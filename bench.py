@@ -336,6 +336,21 @@ def run_gpu(args, wl, rank, world, local_rank):
     rank_seed = rank_seed_offset(rank)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
 
+    # every layer's tokens and outputs sit in one device buffer each (and one
+    # pinned host buffer each), at 256-byte offsets, so the end-to-end step
+    # moves them with one copy each way
+    def offsets(sizes):
+        offs, o = [], 0
+        for n in sizes:
+            offs.append(o)
+            o += -(-n // 128) * 128  # bf16 elements: 256-byte steps
+        return offs, o
+    x_offs, x_tot = offsets([M * K for (_, K) in wl["layers"]])
+    y_offs, y_tot = offsets([M * N for (N, _) in wl["layers"]])
+    xs_dev = torch.zeros(x_tot, dtype=torch.bfloat16, device=dev)
+    ys_dev = torch.zeros(y_tot, dtype=torch.bfloat16, device=dev)
+    xs_host = torch.zeros(x_tot, dtype=torch.bfloat16).pin_memory()
+    ys_host = torch.zeros(y_tot, dtype=torch.bfloat16).pin_memory()
     layers = []
     for i, (N, K) in enumerate(wl["layers"]):
         Wh = synth.normal_f32(1000 + wl["seed"] + 100 * i + rank_seed, (N, K), wl["sigma"])
@@ -343,16 +358,18 @@ def run_gpu(args, wl, rank, world, local_rank):
         rb = B.bitlinear_packed_row_bytes(K, fmt)
         L = dict(N=N, K=K, rb=rb)
         L["W"] = torch.from_numpy(Wh).to(dev)
-        L["x"] = torch.from_numpy(xh.view(np.int16)).to(dev).view(torch.bfloat16)
+        L["x_host"] = xs_host[x_offs[i]:x_offs[i] + M * K].view(M, K)
+        L["x_host"].copy_(torch.from_numpy(xh.view(np.int16)).view(torch.bfloat16).view(M, K))
+        L["x"] = xs_dev[x_offs[i]:x_offs[i] + M * K].view(M, K)
+        L["x"].copy_(L["x_host"])
         if args.phase == "all":  # the step copies the latent weights from the host too
             L["W_host"] = torch.from_numpy(Wh).pin_memory()
-        L["x_host"] = torch.from_numpy(xh.view(np.int16)).view(torch.bfloat16).pin_memory()
         L["gamma"] = torch.empty(1, dtype=torch.float32, device=dev)
         L["ws"] = torch.zeros(B.bitlinear_quantize_weights_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
         L["packed"] = torch.empty((N, rb), dtype=torch.uint8, device=dev)
         L["scale"] = torch.empty(M, dtype=torch.float32, device=dev)
-        L["y"] = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        L["y_host"] = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        L["y"] = ys_dev[y_offs[i]:y_offs[i] + M * N].view(M, N)
+        L["y_host"] = ys_host[y_offs[i]:y_offs[i] + M * N].view(M, N)
         L["fws"] = torch.zeros(B.bitlinear_forward_workspace_bytes(M, N, K, fmt, B.BL_BF16),
                                dtype=torch.uint8, device=dev)
         L["bytes"] = layer_bytes(N, K, M, rb)
@@ -421,8 +438,9 @@ def run_gpu(args, wl, rank, world, local_rank):
     # (and, for --phase all, the latent weights) from pinned host memory and
     # reads y back ----
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
-    h2d = sum((L["W_host"].numel() * 4 if args.phase == "all" else 0) + L["x_host"].numel() * 2 for L in layers)
-    d2h = sum(L["y_host"].numel() * 2 for L in layers)
+    h2d = sum(L["W_host"].numel() * 4 for L in layers) if args.phase == "all" else 0
+    h2d += xs_host.numel() * 2
+    d2h = ys_host.numel() * 2
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -431,13 +449,12 @@ def run_gpu(args, wl, rank, world, local_rank):
     with torch.cuda.stream(stream):
         e0.record(stream)
         for i in range(e2e_steps):
-            for L in layers:
-                if args.phase == "all":
+            if args.phase == "all":
+                for L in layers:
                     L["W"].copy_(L["W_host"], non_blocking=True)
-                L["x"].copy_(L["x_host"], non_blocking=True)
+            xs_dev.copy_(xs_host, non_blocking=True)  # every layer's tokens, one copy
             step(i)
-            for L in layers:
-                L["y_host"].copy_(L["y"], non_blocking=True)
+            ys_host.copy_(ys_dev, non_blocking=True)  # every layer's outputs, one copy
         e1.record(stream)
     stream.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)

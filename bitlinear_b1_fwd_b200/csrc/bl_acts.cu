@@ -4,7 +4,7 @@
 // (one row of x over K) is scaled by its own max |x| (floored at 1e-6) and
 // x_q = clamp(round(x / s * 127), -127, 127).  Rows of up to 32 K (bf16) or
 // 16 K (fp32) elements with K % 8 (bf16) or K % 4 (fp32) == 0: one CTA per
-// token, read once into registers.  Other rows: one warp per token, two
+// token, read once into registers.  Other rows: one CTA per token, two
 // passes whose loads go out kActBatch at a time.
 #include <type_traits>
 
@@ -109,25 +109,26 @@ __global__ void __launch_bounds__(T)
   }
 }
 
-// Any row: the absmax pass and the code pass, kActBatch loads per lane in flight.
+// Any row: one CTA of kActThreads per token, the absmax pass and the code
+// pass over the row, kActBatch 16-byte loads per thread in flight.
 template <int XDT>
 __global__ void __launch_bounds__(kActThreads)
     act_quant_kernel(const void* __restrict__ x, int64_t M, int64_t K, int8_t* __restrict__ xq,
                      float* __restrict__ scale, bool vec) {
   pdl_enter(x, xq, scale);
-  const int lane = threadIdx.x & 31;
-  const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t tw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  __shared__ float red[kActThreads / 32];
+  const int t = threadIdx.x, lane = t & 31;
+  constexpr int T = kActThreads;
   const int64_t nv = K / 8;
-  for (int64_t m = gw; m < M; m += tw) {
+  for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
     const int64_t base = m * K;
     float amax = 0.0f;
     if (vec) {
-      for (int64_t v0 = lane; v0 < nv; v0 += 32 * kActBatch) {
+      for (int64_t v0 = t; v0 < nv; v0 += T * kActBatch) {
         float e[kActBatch][8];
 #pragma unroll
         for (int b = 0; b < kActBatch; ++b) {
-          const int64_t v = v0 + 32 * b;
+          const int64_t v = v0 + T * b;
           if (v < nv) {
             load8_aligned<XDT>(x, base + 8 * v, e[b]);
           } else {
@@ -141,30 +142,36 @@ __global__ void __launch_bounds__(kActThreads)
           for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(e[b][j]));
       }
     } else {
-      for (int64_t k = lane; k < K; k += 32) amax = fmaxf(amax, fabsf(load_elem<XDT>(x, base + k)));
+      for (int64_t k = t; k < K; k += T) amax = fmaxf(amax, fabsf(load_elem<XDT>(x, base + k)));
     }
     amax = warp_maxf(amax);
-    const float s = fmaxf(amax, 1e-6f);
+    if (lane == 0) red[t >> 5] = amax;
+    __syncthreads();
+    float a = red[0];
+#pragma unroll
+    for (int w = 1; w < T / 32; ++w) a = fmaxf(a, red[w]);
+    __syncthreads();  // red is free for the next token
+    const float s = fmaxf(a, 1e-6f);
     const float c127 = __fdiv_rn(127.0f, s);
     if (vec) {
-      for (int64_t v0 = lane; v0 < nv; v0 += 32 * kActBatch) {
+      for (int64_t v0 = t; v0 < nv; v0 += T * kActBatch) {
         float e[kActBatch][8];
 #pragma unroll
         for (int b = 0; b < kActBatch; ++b) {
-          const int64_t v = v0 + 32 * b;
+          const int64_t v = v0 + T * b;
           if (v < nv) load8_aligned<XDT>(x, base + 8 * v, e[b]);
         }
 #pragma unroll
         for (int b = 0; b < kActBatch; ++b) {
-          const int64_t v = v0 + 32 * b;
+          const int64_t v = v0 + T * b;
           if (v < nv) *reinterpret_cast<uint2*>(xq + base + 8 * v) = codes8(e[b], s, c127);
         }
       }
     } else {
-      for (int64_t k = lane; k < K; k += 32)
+      for (int64_t k = t; k < K; k += T)
         xq[base + k] = static_cast<int8_t>(quant_act_fast(load_elem<XDT>(x, base + k), s, c127));
     }
-    if (lane == 0) scale[m] = s;
+    if (t == 0) scale[m] = s;
   }
 }
 
@@ -473,8 +480,7 @@ cudaError_t launch_ln_quant(const void* x, int xdt, const float* g, const float*
 
 cudaError_t launch_act_quant(const void* x, int xdt, int64_t M, int64_t K, int8_t* xq, float* scale,
                              cudaStream_t st) {
-  const int64_t warps_per_cta = kActThreads / 32;
-  const int64_t need = (M + warps_per_cta - 1) / warps_per_cta;
+  const int64_t need = M;  // one CTA per token
   auto grid_for = [&](const void* kern) -> unsigned {
     int per_sm = 1;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kActThreads, 0) != cudaSuccess ||
