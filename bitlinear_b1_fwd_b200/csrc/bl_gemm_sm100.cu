@@ -555,8 +555,8 @@ __global__ void __launch_bounds__(256)
 // CTAs report to the leader by remote arrives.  MMA completion is committed to
 // the barriers of both CTAs.  Every wait is bounded as in the one-SM kernel.
 // ---------------------------------------------------------------------------
-constexpr int kStagesA = 7;  // TMA ring: x half + packed tile per stage
-constexpr int kStagesB = 3;  // expanded-weight ring
+constexpr int kStagesA = 5;  // TMA ring: x half + packed tile per stage
+constexpr int kStagesB = 5;  // expanded-weight ring
 constexpr uint32_t kYStage = 32 * 128 * 4;  // output staging: 32 tokens x 128 rows, up to 4 bytes each
 
 template <int BT>
