@@ -547,8 +547,9 @@ __global__ void __launch_bounds__(256)
 // Two-SM variant for many tokens.  A cluster of two CTAs computes a tile of
 // 256 weight rows x BT tokens with tcgen05.mma.cta_group::2 (M = 256): CTA r
 // stages its own 128 weight rows and tokens r BT/2 .. (r+1) BT/2 - 1, so per
-// SM the staged bytes per MAC fall to about 2/3 of the one-SM tile and six
-// stages fit.  Each CTA's accumulator in tensor memory holds its 128 rows x BT
+// SM the staged bytes per MAC fall to about 2/3 of the one-SM tile: five TMA
+// stages and five expanded stages fit (three expanded stages measured 1-3 %
+// slower).  Each CTA's accumulator in tensor memory holds its 128 rows x BT
 // tokens.  The leader (rank 0) issues the MMAs; the x loads of both CTAs count
 // on the leader's barrier, the packed loads on the local one (the expansion
 // warps of each CTA wait there), and the expansion and epilogue warps of both
