@@ -930,6 +930,7 @@ PROFILE_CASES = {
     "lnquant_70b_down": dict(N=8192, K=28672, fmt=0, M=256, sigma=0.01, op="lnquant"),
     "pack_3b_up": dict(N=8640, K=3200, fmt=0, M=1, sigma=0.02, op="pack"),
     "actquant_16x40000": dict(N=16, K=40000, fmt=0, M=16, sigma=0.02, op="actquant"),
+    "quantize_3b_up_t5": dict(N=8640, K=3200, fmt=1, M=1, sigma=0.02, op="quantize"),
 }
 
 
