@@ -66,3 +66,8 @@ def test_headline_roofline_kernels_have_profiles():
              for p in glob.glob(os.path.join(ROOT, "profiles", "ncu_*.md"))}
     assert (bench.gemv_kernel_name(0, [(8640, 3200), (3200, 8640)]), "3b_decode") in names
     assert (bench.gemm_kernel_name(4096), "3b_prefill") in names
+
+
+def test_every_kernel_has_an_ncu_summary():
+    have = {_fields(p).get("kernel") for p in glob.glob(os.path.join(ROOT, "profiles", "ncu_*.md"))}
+    assert set(bench.KERNEL_SOURCE) <= have, sorted(set(bench.KERNEL_SOURCE) - have)
