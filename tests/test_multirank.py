@@ -17,7 +17,7 @@ sys.path.insert(0, ROOT)
 import bench  # noqa: E402
 
 
-def _worker(rank, world, port, out):
+def _worker(rank, world, port, out_dir):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
@@ -26,17 +26,22 @@ def _worker(rank, world, port, out):
         val = bench.whole_job_gbs(1_000_000, world, got)
         seeds = [None] * world
         dist.all_gather_object(seeds, bench.rank_seed_offset(rank))
-        out[rank] = (got, val, tuple(seeds))
+        with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+            json.dump([got, val, seeds], f)
     finally:
         dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_agree():
+def test_two_gloo_ranks_agree(tmp_path):
+    # the ranks are spawned (never forked: this process already runs threads)
+    # and hand their results back through files
     port = 29500 + (os.getpid() % 1000)
-    with mp.Manager() as m:
-        out = m.dict()
-        mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
-        res = dict(out)
+    mp.spawn(_worker, args=(2, port, str(tmp_path)), nprocs=2, join=True)
+    res = {}
+    for r in range(2):
+        with open(tmp_path / f"rank{r}.json") as f:
+            got, val, seeds = json.load(f)
+        res[r] = (got, val, tuple(seeds))
     assert res[0] == res[1]
     got, val, seeds = res[0]
     assert got == 3.5                                   # the slower rank sets the time
