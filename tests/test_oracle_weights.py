@@ -86,6 +86,23 @@ def test_threshold_form(orc, seed):
     assert codes[0, 0] == 0 and codes[0, 1] == 0     # exactly gamma/2 -> 0 (half-to-even)
 
 
+def test_threshold_form_over_many_scales(orc):
+    """The threshold form at the boundary d/2 for 512 scales spread over three
+    binades: the weights d/2, its fp32 neighbours and their negatives.  A
+    quotient taken as w * fl(1/d) instead of one division disagrees with the
+    threshold on about a fifth of the scales (fl(1/d) carries up to half an
+    ulp of error, enough to move w = d/2 -+ 1 ulp across 1/2)."""
+    gammas = (0.0025 + 0.0175 * synth.uniform(17, 512)).astype(np.float32)
+    eps = np.float32(1e-5)
+    for gamma in gammas:
+        d = np.float32(gamma + eps)
+        half = np.float32(d / np.float32(2))
+        up, down = np.nextafter(half, np.float32(1)), np.nextafter(half, np.float32(0))
+        W = np.array([[half, up, down, -half, -up, -down]], np.float32)
+        codes = orc.ternarize(W, np.float32(gamma), 1e-5)[0]
+        assert codes.tolist() == [0, 1, 0, 0, -1, 0], (float(gamma), codes.tolist())
+
+
 # --- exact value of gamma ---------------------------------------------------
 
 def _exact_abs_sum(W):

@@ -48,6 +48,27 @@ MISTAKES = [
     ("layernorm_without_bias", "* (double)g[k] + (double)b[k];", "* (double)g[k];"),
     ("layernorm_without_eps", "sqrt(var + (double)eps)", "sqrt(var)"),
     ("layernorm_tree_drops_a_level", "for (int s = 128; s >= 1; s >>= 1)", "for (int s = 128; s >= 2; s >>= 1)"),
+    ("ternarize_without_upper_clamp", "if (q > 1.0f) q = 1.0f;", ";"),
+    ("ternarize_without_lower_clamp", "if (q < -1.0f) q = -1.0f;", ";"),
+    ("ternarize_reciprocal_multiply", "float r = load_f(W, dt, e) / d;", "float r = load_f(W, dt, e) * (1.0f / d);"),
+    ("pack_base3_first_weight_most_significant", "byte += digit * pow3;", "byte = byte * 3u + digit;"),
+    ("pack_twos_complement_codes", "unsigned digit = (unsigned)(q + 1);", "unsigned digit = (unsigned)q & 3u;"),
+    ("unpack_accepts_base3_bytes_above_242", "if (fmt == ORC_PACK_T5 && byte >= 243) return -1;", ";"),
+    ("act_quant_signed_max", "float a = fabsf(load_f(x, dt, m * K + k));", "float a = load_f(x, dt, m * K + k);"),
+    ("act_quant_reciprocal_multiply", "float t = load_f(x, dt, m * K + k) / s;",
+     "float t = load_f(x, dt, m * K + k) * (1.0f / s);"),
+    ("matmul_skips_minus_one", "s += (int32_t)codes[n * K + k] * (int32_t)xq[m * K + k];",
+     "s += (codes[n * K + k] > 0) * (int32_t)xq[m * K + k];"),
+    ("dequant_without_gamma", "float c = (gamma * scale[m]) / 127.0f;", "float c = scale[m] / 127.0f;"),
+    ("dequant_reassociated", "float c = (gamma * scale[m]) / 127.0f;", "float c = gamma * (scale[m] / 127.0f);"),
+    ("onebit_beta_of_signed", "sa += (double)fabsf(w[i]);", "sa += (double)w[i];"),
+    ("backward_dx_skips_minus_one", "xsum_add(&acc, load_f(dy, dydt, m * N + n), -1);", ";"),
+    ("layernorm_variance_about_zero", "const double d = (double)load_f(x, dt, m * K + k) - mu;",
+     "const double d = (double)load_f(x, dt, m * K + k);"),
+    ("layernorm_mean_over_lanes", "const double mu = token_tree_sum(lane) / (double)K;",
+     "const double mu = token_tree_sum(lane) / 256.0;"),
+    ("layernorm_without_sqrt", "const double r = 1.0 / sqrt(var + (double)eps);",
+     "const double r = 1.0 / (var + (double)eps);"),
 ]
 
 GCC = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fno-fast-math", "-ffp-contract=off",
