@@ -69,6 +69,10 @@ MISTAKES = [
      "const double mu = token_tree_sum(lane) / 256.0;"),
     ("layernorm_without_sqrt", "const double r = 1.0 / sqrt(var + (double)eps);",
      "const double r = 1.0 / (var + (double)eps);"),
+    ("unpack_accepts_nonzero_padding", "else if (digit != 1)", "else if (0)"),
+    ("unpack_accepts_set_pad_bits", "else if (bit != 0)", "else if (0)"),
+    ("onebit_matrix_compares_with_beta", "codes[e] = (int8_t)(load_f(W, dt, e) > a ? 1 : -1);",
+     "codes[e] = (int8_t)(load_f(W, dt, e) > *beta ? 1 : -1);"),
 ]
 
 GCC = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fno-fast-math", "-ffp-contract=off",
