@@ -11,6 +11,10 @@ namespace {
 
 constexpr int64_t kMaxK = int64_t{1} << 20;
 constexpr int64_t kMaxNK = int64_t{1} << 32;
+// Rows of W (N) and tokens (M) stay below 2^31: the kernels count rows,
+// tokens and per-row work items in 32-bit integers (with K = 1, N up to
+// 2^32 would satisfy N K <= 2^32 but overflow those counts).
+constexpr int64_t kMaxRows = (int64_t{1} << 31) - 1;
 constexpr int kVersion = 100;  // 0.1.0
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -22,9 +26,11 @@ inline bool tern_fmt_ok(int fmt) { return fmt == BL_PACK_I2 || fmt == BL_PACK_T5
 inline bl_status cuda_status(cudaError_t e) { return e == cudaSuccess ? BL_OK : BL_ERR_CUDA; }
 
 bool nk_ok(int64_t N, int64_t K) {
-  if (N < 0 || K < 1 || K > kMaxK) return false;
+  if (N < 0 || N > kMaxRows || K < 1 || K > kMaxK) return false;
   return N <= kMaxNK / K;
 }
+
+inline bool m_ok(int64_t M) { return M >= 0 && M <= kMaxRows; }
 
 }  // namespace
 
@@ -68,7 +74,7 @@ bool uses_gemm(int64_t M, int64_t K) { return M > bl::kGemvMaxTokens && (K % 16)
 bool b1_via_i2(int fmt, int64_t K) { return fmt == BL_PACK_B1 && (K + 7) / 8 > 4096; }
 
 size_t bitlinear_forward_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int xdt) {
-  if (M < 0 || !nk_ok(N, K) || !fmt_ok(fmt)) return 0;
+  if (!m_ok(M) || !nk_ok(N, K) || !fmt_ok(fmt)) return 0;
   size_t bytes = BL_WS_HEADER_BYTES;
   if (uses_gemm(M, K)) {
     if (xdt != BL_I8) bytes += round256(static_cast<size_t>(M * K));
@@ -159,7 +165,7 @@ bl_status bitlinear_pack(const int8_t* codes, int64_t N, int64_t K, int fmt, uin
 
 bl_status bitlinear_quantize_acts(const void* x, int xdt, int64_t M, int64_t K, int8_t* xq, float* scale,
                                   void* stream) {
-  if (!float_dt(xdt) || M < 0 || K < 1 || K > kMaxK) return BL_ERR_INVALID_VALUE;
+  if (!float_dt(xdt) || !m_ok(M) || K < 1 || K > kMaxK) return BL_ERR_INVALID_VALUE;
   if (M == 0) return BL_OK;
   if (x == nullptr || xq == nullptr || scale == nullptr) return BL_ERR_INVALID_VALUE;
   if (!aligned(x, 16) || !aligned(xq, 16) || !aligned(scale, 4)) return BL_ERR_MISALIGNED;
@@ -169,7 +175,7 @@ bl_status bitlinear_quantize_acts(const void* x, int xdt, int64_t M, int64_t K, 
 bl_status bitlinear_layernorm_quantize_acts(const void* x, int xdt, const float* ln_w, const float* ln_b, float eps,
                                             int64_t M, int64_t K, uint16_t* y, int8_t* xq, float* scale,
                                             void* stream) {
-  if (!float_dt(xdt) || M < 0 || K < 1 || K > kMaxK) return BL_ERR_INVALID_VALUE;
+  if (!float_dt(xdt) || !m_ok(M) || K < 1 || K > kMaxK) return BL_ERR_INVALID_VALUE;
   if (!(eps > 0.0f) || !std::isfinite(eps)) return BL_ERR_INVALID_VALUE;
   if (M == 0) return BL_OK;
   if (x == nullptr || ln_w == nullptr || ln_b == nullptr || xq == nullptr || scale == nullptr)
@@ -184,7 +190,7 @@ bl_status bitlinear_forward(const uint8_t* packed, int fmt, const float* gamma, 
                             size_t ws_bytes, void* stream) {
   if (!fmt_ok(fmt) || !(float_dt(xdt) || xdt == BL_I8) || !(float_dt(ydt) || ydt == BL_I32))
     return BL_ERR_INVALID_VALUE;
-  if (M < 0 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
+  if (!m_ok(M) || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
   if (M == 0 || N == 0) return BL_OK;  // empty output: nothing to read or write
   if (packed == nullptr || gamma == nullptr || x == nullptr || scale == nullptr || y == nullptr ||
       ws == nullptr)
@@ -244,7 +250,7 @@ static int64_t group_total(int64_t ngroups, const int64_t* group_rows) {
 size_t bitlinear_forward_grouped_workspace_bytes(int64_t M, int64_t ngroups, const int64_t* group_rows, int64_t K,
                                                  int fmt, int xdt) {
   const int64_t N = group_total(ngroups, group_rows);
-  if (N < 1 || M < 0 || !nk_ok(N, K) || !fmt_ok(fmt)) return 0;
+  if (N < 1 || !m_ok(M) || !nk_ok(N, K) || !fmt_ok(fmt)) return 0;
   size_t bytes = BL_WS_HEADER_BYTES;
   if (uses_gemm(M, K)) {
     if (xdt != BL_I8) bytes += round256(static_cast<size_t>(M * K));
@@ -270,7 +276,7 @@ bl_status bitlinear_forward_grouped(const uint8_t* packed, int fmt, const float*
   if (!fmt_ok(fmt) || !(float_dt(xdt) || xdt == BL_I8) || !(float_dt(ydt) || ydt == BL_I32))
     return BL_ERR_INVALID_VALUE;
   const int64_t N = group_total(ngroups, group_rows);
-  if (N < 1 || M < 0 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
+  if (N < 1 || !m_ok(M) || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
   if (M == 0) return BL_OK;
   if (packed == nullptr || gammas == nullptr || x == nullptr || scale == nullptr || y == nullptr || ws == nullptr)
     return BL_ERR_INVALID_VALUE;
@@ -330,7 +336,7 @@ bl_status bitlinear_forward_grouped(const uint8_t* packed, int fmt, const float*
 
 // STE backward.
 size_t bitlinear_backward_dx_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt) {
-  if (N < 1 || M < 0 || !nk_ok(N, K) || !fmt_ok(fmt)) return 0;
+  if (N < 1 || !m_ok(M) || !nk_ok(N, K) || !fmt_ok(fmt)) return 0;
   size_t bytes = BL_WS_HEADER_BYTES;
   if (fmt != BL_PACK_I2) bytes += round256(static_cast<size_t>(N * bitlinear_packed_row_bytes(K, BL_PACK_I2)));
   const int64_t mt = M < bl::backward_dx_tokens_per_pass() ? M : bl::backward_dx_tokens_per_pass();
@@ -341,7 +347,7 @@ size_t bitlinear_backward_dx_workspace_bytes(int64_t M, int64_t N, int64_t K, in
 bl_status bitlinear_backward_dx(const uint8_t* packed, int fmt, const float* gamma, int64_t N, int64_t K,
                                 const void* dy, int dydt, int64_t M, float* dx, void* ws, size_t ws_bytes,
                                 void* stream) {
-  if (!fmt_ok(fmt) || !float_dt(dydt) || M < 0 || N < 1 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
+  if (!fmt_ok(fmt) || !float_dt(dydt) || !m_ok(M) || N < 1 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
   if (M == 0) return BL_OK;
   if (packed == nullptr || gamma == nullptr || dy == nullptr || dx == nullptr || ws == nullptr)
     return BL_ERR_INVALID_VALUE;
@@ -365,7 +371,7 @@ bl_status bitlinear_backward_dx(const uint8_t* packed, int fmt, const float* gam
 
 bl_status bitlinear_backward_dw(const void* dy, int dydt, const int8_t* xq, const float* scale, const float* gamma,
                                 int64_t M, int64_t N, int64_t K, float* dw, void* stream) {
-  if (!float_dt(dydt) || M < 0 || N < 1 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
+  if (!float_dt(dydt) || !m_ok(M) || N < 1 || !nk_ok(N, K)) return BL_ERR_INVALID_VALUE;
   if (dw == nullptr || gamma == nullptr || (M > 0 && (dy == nullptr || xq == nullptr || scale == nullptr)))
     return BL_ERR_INVALID_VALUE;
   if (!aligned(dy, 16) || !aligned(xq, 16) || !aligned(dw, 16) || !aligned(scale, 4) || !aligned(gamma, 4))

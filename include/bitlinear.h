@@ -57,8 +57,9 @@
  *     sticky flag in the workspace header; bitlinear_device_status() reports
  *     and clears it.
  *   - Inputs must be finite; NaN or Inf inputs give unspecified codes.
- *   - Limits: 1 <= K <= 2^20; N * K <= 2^32; M, N >= 0 (an empty M or N is a
- *     no-op).
+ *   - Limits: 1 <= K <= 2^20; N * K <= 2^32; 0 <= M, N < 2^31 (an empty M
+ *     or N is a no-op); larger sizes return BL_ERR_INVALID_VALUE (the size
+ *     queries return 0).
  */
 #ifndef BITLINEAR_H
 #define BITLINEAR_H

@@ -159,6 +159,44 @@ def test_host_validation_without_gpu(bl):
     assert L.bitlinear_device_status(null, null) == bl.BL_ERR_INVALID_VALUE
 
 
+def test_size_limits_without_gpu(bl):
+    """Rows and tokens stay below 2^31 (the kernels count them, and the work
+    items of a row, in 32 bits): one past the limit is rejected on the host;
+    at the limit the arguments pass every host check and the call reaches the
+    CUDA runtime, which has no device here (BL_ERR_CUDA)."""
+    L = bl.lib()
+    p = C.c_void_p(1 << 20)
+    null = None
+    top, over = (1 << 31) - 1, 1 << 31
+    big = 1 << 62
+    # N at K = 1, where N K <= 2^32 alone would allow up to 2^32 rows
+    assert L.bitlinear_pack(p, over, 1, 0, p, p, 4096, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_pack(p, top, 1, 0, p, p, 4096, null) == bl.BL_ERR_CUDA
+    assert L.bitlinear_quantize_weights(p, 0, over, 1, 1e-5, 0, p, null, p, p, big, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_quantize_weights(p, 0, top, 1, 1e-5, 0, p, null, p, p, big, null) == bl.BL_ERR_CUDA
+    assert L.bitlinear_binarize_weights(p, 0, over, 1, p, null, p, p, p, big, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_backward_dw(p, 1, p, p, p, 1, over, 1, p, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_backward_dw(p, 1, p, p, p, 1, top, 1, p, null) == bl.BL_ERR_CUDA
+    assert L.bitlinear_forward(p, 0, p, over, 1, p, 1, p, 1, p, 1, p, big, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_forward_workspace_bytes(1, over, 1, 0, 1) == 0
+    assert L.bitlinear_quantize_weights_workspace_bytes(over, 1) == 0
+    # M, tokens
+    assert L.bitlinear_quantize_acts(p, 1, over, 16, p, p, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_quantize_acts(p, 1, top, 16, p, p, null) == bl.BL_ERR_CUDA
+    assert L.bitlinear_layernorm_quantize_acts(p, 1, p, p, 1e-5, over, 16, p, p, p, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_forward(p, 0, p, 64, 16, p, 1, p, over, p, 1, p, big, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_forward(p, 0, p, 64, 16, p, 1, p, top, p, 1, p, big, null) == bl.BL_ERR_CUDA
+    assert L.bitlinear_forward_workspace_bytes(over, 64, 16, 0, 1) == 0
+    assert L.bitlinear_forward_workspace_bytes(top, 64, 16, 0, 1) > top * 16
+    assert L.bitlinear_backward_dx(p, 0, p, 64, 16, p, 1, over, p, p, big, null) == bl.BL_ERR_INVALID_VALUE
+    assert L.bitlinear_backward_dx_workspace_bytes(over, 64, 16, 0) == 0
+    assert L.bitlinear_backward_dw(p, 1, p, p, p, over, 64, 16, p, null) == bl.BL_ERR_INVALID_VALUE
+    # typical shapes pass the host checks too
+    assert L.bitlinear_forward(p, 0, p, 8640, 3200, p, 1, p, 1, p, 1, p, 1 << 30, null) == bl.BL_ERR_CUDA
+    assert L.bitlinear_forward(p, 0, p, 8640, 3200, p, 1, p, 4096, p, 1, p, 1 << 34, null) == bl.BL_ERR_CUDA
+    assert L.bitlinear_backward_dx(p, 0, p, 8640, 3200, p, 1, 1, p, p, 1 << 30, null) == bl.BL_ERR_CUDA
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     from bitlinear_b1_fwd_b200 import binding
     monkeypatch.setattr(binding, "_lib", None)
