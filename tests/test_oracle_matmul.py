@@ -38,6 +38,10 @@ def test_add_sub_skip_restatement(orc):
     assert big.tolist() == [[127 * 28672, 127 * 28672]]
     neg = orc.matmul_i32(-np.ones((1, 28672), np.int8), np.full((1, 28672), 127, np.int8))
     assert neg.tolist() == [[-127 * 28672]]
+    # at the largest K the library takes (2^20) the sum still fits INT32 and is exact
+    K = 1 << 20
+    top = orc.matmul_i32(np.stack([np.ones(K, np.int8), -np.ones(K, np.int8)]), np.full((1, K), 127, np.int8))
+    assert top.tolist() == [[127 * K, -127 * K]] and 127 * K < 2 ** 31
 
 
 def test_parallel_matches_serial(orc):
