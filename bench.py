@@ -129,6 +129,27 @@ def profiled_traffic(kernel: str, workload: str):
     return None
 
 
+def nvml_handle_of(nv, props, device_index: int):
+    """NVML handle of the CUDA device with properties `props`.  NVML numbers
+    every GPU of the machine in PCI order and ignores CUDA_VISIBLE_DEVICES,
+    while CUDA numbers the visible GPUs in its own order, so the device is
+    found by its PCI location; the CUDA index is the fallback."""
+    try:
+        want = (int(props.pci_domain_id), int(props.pci_bus_id), int(props.pci_device_id))
+        count = nv.nvmlDeviceGetCount()
+    except Exception:
+        return nv.nvmlDeviceGetHandleByIndex(device_index)
+    for i in range(count):
+        try:  # a GPU this process may not query is skipped
+            h = nv.nvmlDeviceGetHandleByIndex(i)
+            pi = nv.nvmlDeviceGetPciInfo(h)
+            if (int(pi.domain), int(pi.bus), int(pi.device)) == want:
+                return h
+        except Exception:
+            continue
+    return nv.nvmlDeviceGetHandleByIndex(device_index)
+
+
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML while running (every
     0.2 ms: the timed graphs of short workloads last about a millisecond)."""
@@ -144,9 +165,14 @@ class ClockSampler:
         self.period, self._stop, self._t = period_s, threading.Event(), None
         try:
             import pynvml
+            import torch
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            try:
+                props = torch.cuda.get_device_properties(device_index)
+            except Exception:
+                props = None
+            self.h = nvml_handle_of(pynvml, props, device_index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
         except Exception:
             self.nv = None
