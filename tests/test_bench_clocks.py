@@ -45,3 +45,36 @@ def test_index_is_the_fallback():
     nv = FakeNVML(MACHINE)
     assert bench.nvml_handle_of(nv, None, 3) == ("handle", 3)                  # no CUDA properties
     assert bench.nvml_handle_of(nv, props(1, 0x18, 0), 2) == ("handle", 2)     # no GPU at that location
+
+
+def test_sampler_samples_the_matched_gpu(monkeypatch):
+    """ClockSampler end to end on the fake: the handle, the maximum clock and
+    the samples (with throttle reasons) all come from the GPU at the CUDA
+    device's PCI location."""
+    import sys
+    import time
+    import torch
+
+    class Fake(FakeNVML):
+        NVML_CLOCK_SM = 1
+
+        def nvmlInit(self):
+            pass
+
+        def nvmlDeviceGetMaxClockInfo(self, h, kind):
+            return 1965 if h == ("handle", 5) else 1000
+
+        def nvmlDeviceGetClockInfo(self, h, kind):
+            return 1965 if h == ("handle", 5) else 500
+
+        def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+            return 0x4 if h == ("handle", 5) else 0x40
+
+    monkeypatch.setitem(sys.modules, "pynvml", Fake(MACHINE))
+    monkeypatch.setattr(torch.cuda, "get_device_properties", lambda i: props(0, 0xAB, 0))
+    s = bench.ClockSampler(0)
+    assert s.h == ("handle", 5) and s.max_mhz == 1965
+    with s:
+        time.sleep(0.01)
+    assert s.samples and set(s.samples) == {1965}
+    assert s.reasons == {"sw_power_cap"}
