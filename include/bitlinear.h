@@ -172,8 +172,10 @@ BL_API bl_status bitlinear_absmean_noalloc(const void *W, int wdt, int64_t N, in
                                            void *stream);
 
 /* Ternarize and pack with a gamma that is already on the device (step 2-3 only;
- * for instance a gamma reduced across ranks).  Same arrays as above; `gamma`
- * is an input here. */
+ * for instance a gamma reduced across ranks).  [P3] §3.1 and [P5] "The
+ * Ternary Weight Recipe" (W_q = clamp(round(W / (gamma + eps)), -1, 1));
+ * [P3] §2.3 and §6.3 (formats).  Same arrays as above; `gamma` is an input
+ * here. */
 BL_API bl_status bitlinear_ternarize_pack(const void *W, int wdt, int64_t N, int64_t K,
                                    const float *gamma, float eps, int fmt, uint8_t *packed,
                                    int8_t *codes, void *stream);
